@@ -1,0 +1,191 @@
+/*
+ * spattn.h -- C ABI of the sparse-mask scaled dot-product attention library
+ * (libspattn.so, CUDA, sm_100a).
+ *
+ * The operation. For batch b, head h and query row i, let S_i be the column set
+ * of row i of an n x n attention mask given in CSR form: token i attends to
+ * token j exactly when j is in S_i ("[Proposal] Unified Interface/Implementation
+ * for Sparse Attention", gluon-nlp issue 1407, opening post: a user-defined
+ * CSR/COO mask of shape (n, n)). Then
+ *
+ *     s_ij   = scale * <q_i, k_j> + mask[b,h,i,j] + bias[b,h,i,j]      (j in S_i)
+ *     out_i  = sum_{j in S_i} softmax_j(s_i.) * v_j
+ *     lse_i  = log(sum_{j in S_i} exp(s_ij))                             (natural log)
+ *
+ * The proposal computes this as an SDDMM over the mask's nonzeros, a sparse
+ * row softmax and an SpMM with V. The additive mask and the additive bias
+ * follow "support attentions in AlphaFold2" (flash-attention PR 57, the
+ * attention mask and attention bias shape rules); the scale multiplies the dot
+ * product only. This library fuses the three stages in one pass per row with a
+ * running max and a running sum rescaled by exp(m_old - m_new), dividing by the
+ * sum once at the end ("Implementing and Optimizing the Scaled Dot-Product
+ * Attention on Streaming Dataflow", proposed method), so no nnz-sized score
+ * buffer is ever written.
+ *
+ * A row with no nonzeros, or whose scores are all -inf, gives out = 0 and
+ * lse = -inf.
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer named "device" must point to GPU memory of the current
+ *     device; "host" pointers to CPU memory. The caller owns everything it
+ *     passes in; the library keeps no reference after a call returns, except
+ *     inside a spattn_mask handle, which owns the memory it allocated.
+ *   - Calls are stream-ordered: they enqueue work on `stream` (a cudaStream_t;
+ *     NULL = the legacy default stream) and return without waiting, except
+ *     where a function says it synchronises.
+ *   - Every function returns a spattn_status. On failure nothing has been
+ *     enqueued unless the function says otherwise, and spattn_last_error()
+ *     returns a message for the calling thread.
+ */
+#ifndef SPATTN_H
+#define SPATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SPATTN_OK = 0,
+    SPATTN_ERR_INVALID_ARG = 1, /* null pointer, bad shape, stride or size */
+    SPATTN_ERR_UNSUPPORTED = 2, /* valid request outside what is implemented (dtype, head dim, alignment) */
+    SPATTN_ERR_BAD_CSR = 3,     /* CSR/COO content invalid (see spattn_create_csr_mask) */
+    SPATTN_ERR_CUDA = 4,        /* a CUDA runtime call failed; spattn_last_error() names it */
+    SPATTN_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up */
+    SPATTN_ERR_OOM = 6          /* device memory allocation failed */
+} spattn_status;
+
+typedef enum { SPATTN_BF16 = 0, SPATTN_F32 = 1 } spattn_dtype;
+
+/* A strided 4-D view of device memory. Strides are in elements. A dimension of
+ * size 1 may have any stride (it is read as 0, i.e. broadcast). */
+typedef struct {
+    void* data;        /* device */
+    int32_t dtype;     /* spattn_dtype */
+    int32_t reserved;  /* must be 0 */
+    int64_t shape[4];
+    int64_t stride[4];
+} spattn_tensor;
+
+/* ------------------------------------------------------------------ masks */
+
+/* Mask patterns. The pattern list follows the "Sparse Attention" notes page
+ * (local / sliding window, global tokens, block or strided patterns) and the
+ * gluon-nlp proposal (user-defined CSR/COO masks; a per-token variable window
+ * length in the discussion). Row i of mask m lists, ascending and without
+ * duplicates:
+ *   SLIDING              j with |i - j| <= window
+ *   VARWIN               j with i - w_i <= j <= i + w_i, w_i = half_widths[m*n + i] >= 0
+ *   BLOCK_STRIDED_GLOBAL j in the same block of `block` tokens as i (block > 0), or
+ *                        (j - i) a multiple of `stride` (stride > 0), or
+ *                        i < n_global (global tokens attend to all), or
+ *                        j < n_global (and are attended to by all)
+ *   COO                  the candidate columns of row m*n + i (duplicates merged,
+ *                        any order), plus i itself when add_diagonal != 0
+ *   CSR                  the caller's CSR, which must already be sorted and unique
+ *   DENSE                every j (an all-ones mask)
+ * Columns are clipped to [0, n). */
+typedef enum {
+    SPATTN_MASK_CSR = 0,
+    SPATTN_MASK_SLIDING = 1,
+    SPATTN_MASK_VARWIN = 2,
+    SPATTN_MASK_BLOCK_STRIDED_GLOBAL = 3,
+    SPATTN_MASK_COO = 4,
+    SPATTN_MASK_DENSE = 5
+} spattn_mask_kind;
+
+typedef struct {
+    int32_t kind;         /* spattn_mask_kind */
+    int32_t n;            /* sequence length, >= 1 */
+    int32_t num_masks;    /* masks stacked row-wise: rows m*n .. m*n + n - 1 belong to mask m */
+    int32_t window;       /* SLIDING: half-width, >= 0 */
+    int32_t block;        /* BLOCK_STRIDED_GLOBAL: block size (0 = no block part) */
+    int32_t stride;       /* BLOCK_STRIDED_GLOBAL: stride (0 = no strided part) */
+    int32_t n_global;     /* BLOCK_STRIDED_GLOBAL: number of global tokens (0 = none) */
+    int32_t add_diagonal; /* COO: also include (i, i) */
+    const int32_t* half_widths; /* VARWIN: device, [num_masks * n], each >= 0 */
+    const int32_t* in_row_ptr;  /* CSR, COO: device, [num_masks * n + 1], starts at 0, non-decreasing */
+    const int32_t* in_col_idx;  /* CSR, COO: device, [in_nnz], each in [0, n) */
+    int64_t in_nnz;             /* CSR, COO: in_row_ptr[num_masks * n] */
+} spattn_mask_spec;
+
+/* A built mask: its CSR (row_ptr int32 [num_masks*n + 1], col_idx int32 [nnz]),
+ * plus the schedule the forward pass uses (rows long enough to be split over a
+ * whole thread block). Owns its device memory. */
+typedef struct spattn_mask_s* spattn_mask;
+
+/* Build a CSR mask on the device from a pattern (the proposal's "generate the
+ * corresponding attention mask" step, then the row schedule).
+ * Synchronises `stream` twice (to size col_idx and the schedule). Memory comes
+ * from the library's stream-ordered pool and is released by spattn_destroy_mask.
+ * Errors: INVALID_ARG (bad kind or parameters), BAD_CSR (CSR not sorted/unique,
+ * a column outside [0, n), row_ptr not a valid prefix sum, or a negative
+ * half-width), UNSUPPORTED (more than 2^31 - 1 nonzeros, or a COO row with more
+ * candidates than the builder's limit), OOM, CUDA. On error *out is NULL. */
+int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream, spattn_mask* out);
+
+/* Read a mask's sizes and device CSR pointers (owned by the mask). Any output
+ * pointer may be NULL. n_long: rows handled by the block-per-row kernel. */
+int spattn_mask_info(spattn_mask mask, int32_t* n, int32_t* num_masks, int64_t* nnz,
+                     const int32_t** row_ptr, const int32_t** col_idx, int64_t* n_long);
+
+/* Copy a mask's CSR into caller buffers (device or host memory, any mix):
+ * row_ptr_dst int32 [num_masks * n + 1], col_idx_dst int32 [nnz]; either may be
+ * NULL to skip it. Stream-ordered on `stream`; host destinations should be
+ * pinned for the copy to be asynchronous. */
+int spattn_mask_copy_csr(spattn_mask mask, int32_t* row_ptr_dst, int32_t* col_idx_dst,
+                         void* stream);
+
+/* Release a mask. Stream-ordered on the stream it was created on. NULL is a no-op. */
+int spattn_destroy_mask(spattn_mask mask);
+
+/* --------------------------------------------------------------- forward */
+
+/* Fused masked attention over a raw device CSR.
+ *   q, k, v  [B, H, n, d], dtype bf16 or f32 (all three the same), stride 1 over d,
+ *            d in {32, 64, 128}, base pointers and row strides 16-byte aligned.
+ *   row_ptr  device int32 [num_masks * n + 1]; num_masks is 1 (shared by every b)
+ *            or B (mask b for batch b). Entries are clamped to [0, nnz].
+ *   col_idx  device int32 [nnz]. Columns need not be sorted. A column outside
+ *            [0, n) is skipped and raises the device error flag (read it with
+ *            spattn_device_error). Duplicate columns count once per occurrence.
+ *   add_mask, bias  optional (NULL) 4-D tensors broadcastable to [B, H, n, n]
+ *            (each dimension equal or 1), dtype bf16 or f32; values are added to
+ *            the scaled scores (-inf removes an entry).
+ *   scale    softmax scale applied to <q_i, k_j> only (commonly 1/sqrt(d)).
+ *   out      [B, H, n, d], same dtype as q, stride 1 over d, rounded to nearest even.
+ *   lse      optional device float [B * H * n]; lse[(b*H + h)*n + i].
+ * Uses scratch memory (a list of long rows, O(num_masks * n)) taken from the
+ * library's stream-ordered pool and returned before the call's work completes. */
+int spattn_fwd(const spattn_tensor* q, const spattn_tensor* k, const spattn_tensor* v,
+               const int32_t* row_ptr, const int32_t* col_idx, int32_t num_masks, int64_t nnz,
+               const spattn_tensor* add_mask, const spattn_tensor* bias, float scale,
+               const spattn_tensor* out, float* lse, void* stream);
+
+/* The same operation over a mask built by spattn_create_csr_mask, using its
+ * prebuilt schedule. Allocates nothing. The mask's num_masks must be 1 or B and
+ * its n must match q. */
+int spattn_fwd_mask(const spattn_tensor* q, const spattn_tensor* k, const spattn_tensor* v,
+                    spattn_mask mask, const spattn_tensor* add_mask, const spattn_tensor* bias,
+                    float scale, const spattn_tensor* out, float* lse, void* stream);
+
+/* ------------------------------------------------------------- utilities */
+
+/* Message of the last failed call on this thread ("" if none). Valid until the
+ * thread's next call into the library. */
+const char* spattn_last_error(void);
+
+/* Synchronise `stream`, then read and clear the current device's error flags
+ * raised by kernels (bit 0: a column index outside [0, n) was skipped).
+ * *flags may be NULL. Returns SPATTN_OK, or SPATTN_ERR_BAD_CSR if any flag was set. */
+int spattn_device_error(void* stream, uint32_t* flags);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int spattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPATTN_H */

@@ -1,0 +1,436 @@
+// Fused sparse-mask attention forward on CUDA cores: for each query row, gather
+// the K and V rows named by the row's CSR columns, take the dot products (the
+// SDDMM of the gluon-nlp sparse-attention proposal), keep a running max and a
+// running sum rescaled by exp(m_old - m_new) (the streaming-dataflow SDPA
+// paper's proposed method) and accumulate the weighted V rows (the SpMM), then
+// divide once by the sum. No per-nonzero score is ever stored.
+//
+// Work split. A warp owns one query row. A K/V row of d elements is covered by
+// LPR = d * sizeof(T) / 16 lanes (one 16-byte vector each), so a warp holds
+// G = 32 / LPR groups; group g takes nonzeros p = base + u*G + g (u < U) of each
+// step of STEP = G*U nonzeros and keeps its own running (max, sum, acc); the
+// groups merge with the same rescaling rule at the end of the row. Rows with
+// more than kLongRowThreshold nonzeros go to a second kernel in which eight
+// warps share a row and merge through shared memory.
+//
+// Scores are kept in the base-2 domain: q is pre-multiplied by scale*log2(e)
+// and the additive mask/bias by log2(e), so every exponential is one ex2.
+#include "spattn_internal.cuh"
+
+#include <math.h>
+
+namespace spattn {
+
+__device__ unsigned int g_error_flags = 0;
+
+namespace {
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float lg2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint4 ldg16(const void* p) {
+    return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+template <typename T>
+struct Elem;
+
+template <>
+struct Elem<__nv_bfloat16> {
+    static constexpr int VEC = 8;
+    __device__ __forceinline__ static void unpack(const uint4& r, float* f) {
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            f[2 * t] = __uint_as_float(w[t] << 16);
+            f[2 * t + 1] = __uint_as_float(w[t] & 0xffff0000u);
+        }
+    }
+    __device__ __forceinline__ static uint4 pack(const float* f) {
+        uint32_t w[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * t], f[2 * t + 1]);
+            w[t] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    __device__ __forceinline__ static void store1(void* base, int64_t idx, float x) {
+        reinterpret_cast<__nv_bfloat16*>(base)[idx] = __float2bfloat16_rn(x);
+    }
+};
+
+template <>
+struct Elem<float> {
+    static constexpr int VEC = 4;
+    __device__ __forceinline__ static void unpack(const uint4& r, float* f) {
+        f[0] = __uint_as_float(r.x);
+        f[1] = __uint_as_float(r.y);
+        f[2] = __uint_as_float(r.z);
+        f[3] = __uint_as_float(r.w);
+    }
+    __device__ __forceinline__ static uint4 pack(const float* f) {
+        return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                          __float_as_uint(f[3]));
+    }
+    __device__ __forceinline__ static void store1(void* base, int64_t idx, float x) {
+        reinterpret_cast<float*>(base)[idx] = x;
+    }
+};
+
+template <typename T, int D>
+struct Cfg {
+    static constexpr int VEC = Elem<T>::VEC;
+    static constexpr int LPR = D / VEC;  // lanes per K/V row
+    static constexpr int G = 32 / LPR;   // nonzeros loaded per vector instruction
+    static constexpr int U = (32 / G) < 8 ? (32 / G) : 8;  // nonzeros per group per step
+    static constexpr int STEP = G * U;   // nonzeros per warp step (<= 32)
+    static_assert(D % VEC == 0 && LPR >= 1 && LPR <= 32 && 32 % LPR == 0, "unsupported head dim");
+};
+
+template <int VEC>
+struct State {
+    float m;  // running max (base-2 domain)
+    float l;  // running sum of ex2(s - m)
+    float acc[VEC];
+};
+
+__device__ __forceinline__ float load_addend(const AddendView& a, int64_t off) {
+    if (a.dtype == 0)
+        return __bfloat162float(__ldg(reinterpret_cast<const __nv_bfloat16*>(a.data) + off));
+    return __ldg(reinterpret_cast<const float*>(a.data) + off);
+}
+
+__device__ __forceinline__ void clamp_row(const FwdParams& P, int64_t mrow, int64_t& p0,
+                                          int64_t& p1) {
+    p0 = P.row_ptr[mrow];
+    p1 = P.row_ptr[mrow + 1];
+    p0 = p0 < 0 ? 0 : (p0 > P.nnz ? P.nnz : p0);
+    p1 = p1 < p0 ? p0 : (p1 > P.nnz ? P.nnz : p1);
+}
+
+template <typename T, int D>
+struct RowCtx {
+    const T* kb;   // K of (b, h)
+    const T* vb;   // V of (b, h)
+    int64_t mask_base, bias_base;  // addend offsets of (b, h, i, 0)
+    float qf[Cfg<T, D>::VEC];      // this lane's slice of q_i * scale * log2(e)
+};
+
+template <typename T, int D>
+__device__ __forceinline__ void init_row(const FwdParams& P, int b, int h, int i, int lane,
+                                         RowCtx<T, D>& rc, State<Cfg<T, D>::VEC>& st) {
+    using C = Cfg<T, D>;
+    const int c = lane % C::LPR;
+    const T* q = reinterpret_cast<const T*>(P.q) + b * P.q_sb + h * P.q_sh + i * P.q_sn;
+    rc.kb = reinterpret_cast<const T*>(P.k) + b * P.k_sb + h * P.k_sh;
+    rc.vb = reinterpret_cast<const T*>(P.v) + b * P.v_sb + h * P.v_sh;
+    rc.mask_base = b * P.mask.s0 + h * P.mask.s1 + i * P.mask.s2;
+    rc.bias_base = b * P.bias.s0 + h * P.bias.s1 + i * P.bias.s2;
+    Elem<T>::unpack(ldg16(q + c * C::VEC), rc.qf);
+#pragma unroll
+    for (int e = 0; e < C::VEC; ++e) rc.qf[e] *= P.qk_scale_log2;
+    st.m = -INFINITY;
+    st.l = 0.f;
+#pragma unroll
+    for (int e = 0; e < C::VEC; ++e) st.acc[e] = 0.f;
+}
+
+// Process the steps of STEP nonzeros starting at first, first + stride, ...
+// (below p1) of one row into `st`.
+template <typename T, int D>
+__device__ __forceinline__ void row_steps(const FwdParams& P, const RowCtx<T, D>& rc,
+                                          int64_t first, int64_t p1, int64_t stride, int lane,
+                                          State<Cfg<T, D>::VEC>& st) {
+    using C = Cfg<T, D>;
+    const int g = lane / C::LPR, c = lane % C::LPR;
+    for (int64_t pb = first; pb < p1; pb += stride) {
+        // one coalesced read of this step's columns (and additive terms)
+        int col = -1;
+        float extra = 0.f;
+        const int64_t mp = pb + lane;
+        if (lane < C::STEP && mp < p1) {
+            const int j = __ldg(P.col_idx + mp);
+            if ((unsigned)j < (unsigned)P.n) {
+                col = j;
+                if (P.has_extra) {
+                    float e = 0.f;
+                    if (P.mask.data) e += load_addend(P.mask, rc.mask_base + j * P.mask.s3);
+                    if (P.bias.data) e += load_addend(P.bias, rc.bias_base + j * P.bias.s3);
+                    extra = e * kLog2e;
+                }
+            } else {
+                atomicOr(&g_error_flags, kErrBadColumn);
+            }
+        }
+        int js[C::U];
+        float es[C::U];
+#pragma unroll
+        for (int u = 0; u < C::U; ++u) {
+            js[u] = __shfl_sync(0xffffffffu, col, u * C::G + g);
+            es[u] = __shfl_sync(0xffffffffu, extra, u * C::G + g);
+        }
+        uint4 kr[C::U], vr[C::U];
+#pragma unroll
+        for (int u = 0; u < C::U; ++u) {
+            if (js[u] >= 0) {
+                kr[u] = ldg16(rc.kb + (int64_t)js[u] * P.k_sn + c * C::VEC);
+                vr[u] = ldg16(rc.vb + (int64_t)js[u] * P.v_sn + c * C::VEC);
+            } else {
+                kr[u] = make_uint4(0u, 0u, 0u, 0u);
+                vr[u] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+        float s[C::U];
+#pragma unroll
+        for (int u = 0; u < C::U; ++u) {
+            float kf[C::VEC];
+            Elem<T>::unpack(kr[u], kf);
+            float a = 0.f;
+#pragma unroll
+            for (int e = 0; e < C::VEC; ++e) a = fmaf(rc.qf[e], kf[e], a);
+            s[u] = a;
+        }
+#pragma unroll
+        for (int off = 1; off < C::LPR; off <<= 1) {
+#pragma unroll
+            for (int u = 0; u < C::U; ++u) s[u] += __shfl_xor_sync(0xffffffffu, s[u], off);
+        }
+        float mx = st.m;
+#pragma unroll
+        for (int u = 0; u < C::U; ++u) {
+            s[u] = js[u] >= 0 ? s[u] + es[u] : -INFINITY;
+            mx = fmaxf(mx, s[u]);
+        }
+        const float mu = (mx == -INFINITY) ? 0.f : mx;
+        const float alpha = ex2(st.m - mu);
+        st.l *= alpha;
+#pragma unroll
+        for (int e = 0; e < C::VEC; ++e) st.acc[e] *= alpha;
+#pragma unroll
+        for (int u = 0; u < C::U; ++u) {
+            const float pw = ex2(s[u] - mu);
+            st.l += pw;
+            float vf[C::VEC];
+            Elem<T>::unpack(vr[u], vf);
+#pragma unroll
+            for (int e = 0; e < C::VEC; ++e) st.acc[e] = fmaf(pw, vf[e], st.acc[e]);
+        }
+        st.m = mx;
+    }
+}
+
+// Merge the warp's G group states (same rescaling rule); every group ends
+// holding the merged state.
+template <int VEC, int LPR>
+__device__ __forceinline__ void merge_groups(State<VEC>& st) {
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1) {
+        const float mo = __shfl_xor_sync(0xffffffffu, st.m, off);
+        const float lo = __shfl_xor_sync(0xffffffffu, st.l, off);
+        const float mx = fmaxf(st.m, mo);
+        const float mu = (mx == -INFINITY) ? 0.f : mx;
+        const float a = ex2(st.m - mu), bo = ex2(mo - mu);
+        st.l = st.l * a + lo * bo;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            const float ao = __shfl_xor_sync(0xffffffffu, st.acc[e], off);
+            st.acc[e] = st.acc[e] * a + ao * bo;
+        }
+        st.m = mx;
+    }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) k_fwd_short(const FwdParams P) {
+    using C = Cfg<T, D>;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int blocks_per_bh = (P.n + 7) >> 3;
+    const int bh = blockIdx.x / blocks_per_bh;
+    const int i = (blockIdx.x - bh * blocks_per_bh) * 8 + warp;
+    if (i >= P.n) return;
+    const int b = bh / P.H, h = bh - b * P.H;
+    const int64_t mrow = (int64_t)(P.num_masks == 1 ? 0 : b) * P.n + i;
+    int64_t p0, p1;
+    clamp_row(P, mrow, p0, p1);
+    if (p1 - p0 > kLongRowThreshold) return;  // the long-row kernel owns it
+
+    RowCtx<T, D> rc;
+    State<C::VEC> st;
+    init_row<T, D>(P, b, h, i, lane, rc, st);
+    row_steps<T, D>(P, rc, p0, p1, C::STEP, lane, st);
+    merge_groups<C::VEC, C::LPR>(st);
+
+    if (lane < C::LPR) {
+        const float inv = st.l > 0.f ? 1.f / st.l : 0.f;
+        float o[C::VEC];
+#pragma unroll
+        for (int e = 0; e < C::VEC; ++e) o[e] = st.acc[e] * inv;
+        T* orow = reinterpret_cast<T*>(P.out) + b * P.o_sb + h * P.o_sh + i * P.o_sn;
+        *reinterpret_cast<uint4*>(orow + lane * C::VEC) = Elem<T>::pack(o);
+    }
+    if (lane == 0 && P.lse)
+        P.lse[((int64_t)bh) * P.n + i] = st.l > 0.f ? (st.m + lg2(st.l)) * kLn2 : -INFINITY;
+}
+
+constexpr int kLongWarps = 8;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) k_fwd_long(const FwdParams P) {
+    using C = Cfg<T, D>;
+    __shared__ float sm_m[kLongWarps], sm_l[kLongWarps];
+    __shared__ float sm_acc[kLongWarps][D];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t count = P.long_count_host >= 0 ? P.long_count_host : (int64_t)*P.long_count_dev;
+    const int64_t per_row = P.num_masks == 1 ? (int64_t)P.B * P.H : (int64_t)P.H;
+    const int64_t items = count * per_row;
+    for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+        const int64_t slot = it % count, rep = it / count;
+        const int mrow = P.long_rows[slot];
+        const int i = mrow % P.n;
+        int b, h;
+        if (P.num_masks == 1) {
+            b = (int)(rep / P.H);
+            h = (int)(rep - (int64_t)b * P.H);
+        } else {
+            b = mrow / P.n;
+            h = (int)rep;
+        }
+        int64_t p0, p1;
+        clamp_row(P, mrow, p0, p1);
+
+        RowCtx<T, D> rc;
+        State<C::VEC> st;
+        init_row<T, D>(P, b, h, i, lane, rc, st);
+        row_steps<T, D>(P, rc, p0 + (int64_t)warp * C::STEP, p1, (int64_t)kLongWarps * C::STEP,
+                        lane, st);
+        merge_groups<C::VEC, C::LPR>(st);
+        if (lane == 0) {
+            sm_m[warp] = st.m;
+            sm_l[warp] = st.l;
+        }
+        if (lane < C::LPR) {
+#pragma unroll
+            for (int e = 0; e < C::VEC; ++e) sm_acc[warp][lane * C::VEC + e] = st.acc[e];
+        }
+        __syncthreads();
+        if (threadIdx.x < D) {
+            float mx = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kLongWarps; ++w) mx = fmaxf(mx, sm_m[w]);
+            const float mu = (mx == -INFINITY) ? 0.f : mx;
+            float l = 0.f, a = 0.f;
+#pragma unroll
+            for (int w = 0; w < kLongWarps; ++w) {
+                const float f = ex2(sm_m[w] - mu);
+                l = fmaf(sm_l[w], f, l);
+                a = fmaf(sm_acc[w][threadIdx.x], f, a);
+            }
+            T* orow = reinterpret_cast<T*>(P.out) + b * P.o_sb + h * P.o_sh + i * P.o_sn;
+            Elem<T>::store1(orow, threadIdx.x, l > 0.f ? a / l : 0.f);
+            if (threadIdx.x == 0 && P.lse)
+                P.lse[((int64_t)b * P.H + h) * P.n + i] = l > 0.f ? (mx + lg2(l)) * kLn2 : -INFINITY;
+        }
+        __syncthreads();
+    }
+}
+
+__global__ void k_classify_long(const int32_t* __restrict__ row_ptr, int64_t rows, int64_t nnz,
+                                int32_t* __restrict__ list, int32_t* __restrict__ count) {
+    for (int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; r < rows;
+         r += (int64_t)gridDim.x * blockDim.x) {
+        int64_t p0 = row_ptr[r], p1 = row_ptr[r + 1];
+        p0 = p0 < 0 ? 0 : (p0 > nnz ? nnz : p0);
+        p1 = p1 < p0 ? p0 : (p1 > nnz ? nnz : p1);
+        if (p1 - p0 > kLongRowThreshold) list[atomicAdd(count, 1)] = (int32_t)r;
+    }
+}
+
+template <typename T, int D>
+cudaError_t launch_short_t(const FwdParams& p, cudaStream_t s) {
+    const int64_t blocks = (int64_t)p.B * p.H * ((p.n + 7) / 8);
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    k_fwd_short<T, D><<<(unsigned)blocks, 256, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_long_t(const FwdParams& p, int num_sms, cudaStream_t s) {
+    int64_t grid = (int64_t)num_sms * 4;
+    if (p.long_count_host >= 0) {
+        const int64_t items =
+            p.long_count_host * (p.num_masks == 1 ? (int64_t)p.B * p.H : (int64_t)p.H);
+        if (items == 0) return cudaSuccess;
+        if (items < grid) grid = items;
+    }
+    k_fwd_long<T, D><<<(unsigned)grid, 256, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_short_rows(const FwdParams& p, int dtype, int d, cudaStream_t s) {
+    if (dtype == 0) {
+        switch (d) {
+        case 32: return launch_short_t<__nv_bfloat16, 32>(p, s);
+        case 64: return launch_short_t<__nv_bfloat16, 64>(p, s);
+        case 128: return launch_short_t<__nv_bfloat16, 128>(p, s);
+        }
+    } else {
+        switch (d) {
+        case 32: return launch_short_t<float, 32>(p, s);
+        case 64: return launch_short_t<float, 64>(p, s);
+        case 128: return launch_short_t<float, 128>(p, s);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_fwd_long_rows(const FwdParams& p, int dtype, int d, int num_sms,
+                                 cudaStream_t s) {
+    if (dtype == 0) {
+        switch (d) {
+        case 32: return launch_long_t<__nv_bfloat16, 32>(p, num_sms, s);
+        case 64: return launch_long_t<__nv_bfloat16, 64>(p, num_sms, s);
+        case 128: return launch_long_t<__nv_bfloat16, 128>(p, num_sms, s);
+        }
+    } else {
+        switch (d) {
+        case 32: return launch_long_t<float, 32>(p, num_sms, s);
+        case 64: return launch_long_t<float, 64>(p, num_sms, s);
+        case 128: return launch_long_t<float, 128>(p, num_sms, s);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_classify_long_rows(const int32_t* row_ptr, int64_t rows, int64_t nnz,
+                                      int32_t* list, int32_t* count, cudaStream_t s) {
+    if (rows <= 0) return cudaSuccess;
+    int64_t grid = (rows + 255) / 256;
+    if (grid > 4096) grid = 4096;
+    k_classify_long<<<(unsigned)grid, 256, 0, s>>>(row_ptr, rows, nnz, list, count);
+    return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_device_error(unsigned* flags, cudaStream_t s) {
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return e;
+    unsigned v = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&v, g_error_flags, sizeof v);
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyToSymbol(g_error_flags, &zero, sizeof zero);
+    if (flags) *flags = v;
+    return e;
+}
+
+}  // namespace spattn

@@ -1,0 +1,473 @@
+// Mask builder: an attention-mask pattern -> a sorted, duplicate-free CSR.
+//
+// The gluon-nlp sparse-attention proposal reduces every attention scheme to
+// "generate the corresponding mask" and hand it to one CSR kernel; the pattern
+// list (local / sliding window, global tokens, block or strided) is the one of
+// the "Sparse Attention" notes page, with the per-token variable window of the
+// proposal's discussion, plus user COO candidates and user CSR.
+//
+// Two phases on the device:
+//   phase 1  per-row counts (O(1) for interval rows, an ordered walk for block +
+//            strided + global rows, a sort + merge of duplicates for COO rows,
+//            validation for user CSR), then row_ptr by an exclusive scan;
+//   phase 2  (after the host has read the total and allocated col_idx) the
+//            columns, written in ascending order.
+#include "spattn.h"
+#include "spattn_internal.cuh"
+
+#include <limits.h>
+
+namespace spattn {
+namespace {
+
+constexpr int kScanThreads = 1024;
+constexpr int kScanItems = 4;
+constexpr int kScanTile = kScanThreads * kScanItems;
+constexpr int kCooWarpCap = 1024;   // candidates a warp sorts in shared memory
+constexpr int kCooWarps = 4;        // warps per block in the COO sort kernel
+constexpr int kBitmapMaxBytes = 192 * 1024;
+
+__device__ __forceinline__ void raise(BuildInfo* info, unsigned bit) { atomicOr(&info->err, bit); }
+
+// Interval rows: [lo, hi) for SLIDING / VARWIN / DENSE and the global rows of
+// BLOCK_STRIDED_GLOBAL. Returns false when the row is not an interval.
+__device__ __forceinline__ bool row_interval(const BuildSpec& s, int64_t r, int64_t& lo,
+                                             int64_t& hi, BuildInfo* info) {
+    const int64_t i = r % s.n;
+    switch (s.kind) {
+    case SPATTN_MASK_SLIDING:
+    case SPATTN_MASK_VARWIN: {
+        int64_t w = s.kind == SPATTN_MASK_SLIDING ? s.window : s.half_widths[r];
+        if (w < 0) {
+            if (info) raise(info, kBuildNegativeWidth);
+            lo = hi = 0;
+            return true;
+        }
+        lo = i - w < 0 ? 0 : i - w;
+        hi = i + w + 1 > s.n ? s.n : i + w + 1;
+        return true;
+    }
+    case SPATTN_MASK_DENSE:
+        lo = 0;
+        hi = s.n;
+        return true;
+    case SPATTN_MASK_BLOCK_STRIDED_GLOBAL:
+        if (i < s.n_global) {
+            lo = 0;
+            hi = s.n;
+            return true;
+        }
+        return false;
+    default:
+        return false;
+    }
+}
+
+// Smallest column >= j of a non-global BLOCK_STRIDED_GLOBAL row i, or n.
+__device__ __forceinline__ int64_t bsg_next(const BuildSpec& s, int64_t i, int64_t j) {
+    int64_t c = s.n;
+    if (j < s.n_global) c = j;
+    if (s.block > 0) {
+        const int64_t bs = (i / s.block) * s.block;
+        const int64_t be = bs + s.block < s.n ? bs + s.block : s.n;
+        if (j < be) {
+            const int64_t x = j > bs ? j : bs;
+            if (x < c) c = x;
+        }
+    }
+    if (s.stride > 0) {
+        const int64_t r0 = i % s.stride;
+        const int64_t x = j <= r0 ? r0 : r0 + ((j - r0 + s.stride - 1) / s.stride) * s.stride;
+        if (x < c) c = x;
+    }
+    return c;
+}
+
+__global__ void k_count(BuildSpec s, int32_t* __restrict__ counts, BuildInfo* info) {
+    const int64_t rows = (int64_t)s.num_masks * s.n;
+    for (int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; r < rows;
+         r += (int64_t)gridDim.x * blockDim.x) {
+        int64_t cnt = 0, lo, hi;
+        if (s.kind == SPATTN_MASK_CSR) {
+            const int64_t p0 = s.in_row_ptr[r], p1 = s.in_row_ptr[r + 1];
+            bool ok = p0 >= 0 && p1 >= p0 && p1 <= s.in_nnz;
+            if (r == 0 && p0 != 0) ok = false;
+            if (r == rows - 1 && p1 != s.in_nnz) ok = false;
+            if (!ok) raise(info, kBuildBadRowPtr);
+            cnt = ok ? p1 - p0 : 0;
+        } else if (row_interval(s, r, lo, hi, info)) {
+            cnt = hi - lo;
+        } else {  // non-global row of BLOCK_STRIDED_GLOBAL
+            const int64_t i = r % s.n;
+            for (int64_t j = bsg_next(s, i, 0); j < s.n; j = bsg_next(s, i, j + 1)) ++cnt;
+        }
+        counts[r] = (int32_t)cnt;
+    }
+}
+
+// User CSR: every row strictly increasing with columns in [0, n).
+__global__ void k_check_csr(BuildSpec s, BuildInfo* info) {
+    const int64_t rows = (int64_t)s.num_masks * s.n;
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t r = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+         r += warps) {
+        int64_t p0 = s.in_row_ptr[r], p1 = s.in_row_ptr[r + 1];
+        if (p0 < 0 || p1 < p0 || p1 > s.in_nnz) continue;  // reported by k_count
+        for (int64_t p = p0 + lane; p < p1; p += 32) {
+            const int c = s.in_col_idx[p];
+            if ((unsigned)c >= (unsigned)s.n) raise(info, kBuildBadColumn);
+            if (p > p0 && s.in_col_idx[p - 1] >= c) raise(info, kBuildUnsorted);
+        }
+    }
+}
+
+// COO rows of at most kCooWarpCap candidates (diagonal included): one warp
+// sorts the row in shared memory (bitonic network), drops repeats and writes
+// the result to coo_tmp at in_row_ptr[r] + r. Longer rows are queued.
+__global__ void __launch_bounds__(kCooWarps * 32)
+    k_coo_sort(BuildSpec s, int32_t* __restrict__ counts, int32_t* __restrict__ coo_tmp,
+               int32_t* __restrict__ big_list, int32_t* __restrict__ big_count, BuildInfo* info) {
+    __shared__ int32_t buf[kCooWarps][kCooWarpCap];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int32_t* a = buf[warp];
+    const int64_t rows = (int64_t)s.num_masks * s.n;
+    for (int64_t r = (int64_t)blockIdx.x * kCooWarps + warp; r < rows;
+         r += (int64_t)gridDim.x * kCooWarps) {
+        const int64_t p0 = s.in_row_ptr[r], p1 = s.in_row_ptr[r + 1];
+        bool ok = p0 >= 0 && p1 >= p0 && p1 <= s.in_nnz;
+        if (r == 0 && p0 != 0) ok = false;
+        if (r == rows - 1 && p1 != s.in_nnz) ok = false;
+        if (!ok) {
+            if (lane == 0) {
+                raise(info, kBuildBadRowPtr);
+                counts[r] = 0;
+            }
+            continue;
+        }
+        const int64_t ncand = p1 - p0;
+        const int64_t cnt = ncand + (s.add_diagonal ? 1 : 0);
+        if (cnt > kCooWarpCap) {
+            if (lane == 0) {
+                counts[r] = 0;
+                big_list[atomicAdd(big_count, 1)] = (int32_t)r;
+            }
+            continue;
+        }
+        int P = 32;
+        while (P < cnt) P <<= 1;
+        const int i = (int)(r % s.n);
+        for (int t = lane; t < P; t += 32) {
+            int v = INT_MAX;
+            if (t < ncand) {
+                v = s.in_col_idx[p0 + t];
+                if ((unsigned)v >= (unsigned)s.n) {
+                    raise(info, kBuildBadColumn);
+                    v = INT_MAX;
+                }
+            } else if (t == ncand && s.add_diagonal) {
+                v = i;
+            }
+            a[t] = v;
+        }
+        __syncwarp();
+        for (int k = 2; k <= P; k <<= 1) {
+            for (int j = k >> 1; j > 0; j >>= 1) {
+                for (int t = lane; t < P; t += 32) {
+                    const int u = t ^ j;
+                    if (u > t) {
+                        const int x = a[t], y = a[u];
+                        const bool up = (t & k) == 0;
+                        if ((x > y) == up) {
+                            a[t] = y;
+                            a[u] = x;
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+        }
+        const int64_t base = p0 + r;
+        int written = 0;
+        for (int t0 = 0; t0 < P; t0 += 32) {
+            const int t = t0 + lane;
+            const int v = a[t];
+            const bool keep = v != INT_MAX && (t == 0 || a[t - 1] != v);
+            const unsigned bal = __ballot_sync(0xffffffffu, keep);
+            if (keep) coo_tmp[base + written + __popc(bal & ((1u << lane) - 1u))] = v;
+            written += __popc(bal);
+        }
+        if (lane == 0) counts[r] = written;
+        __syncwarp();
+    }
+}
+
+// Queued long COO rows: one block per row marks the columns in an n-bit map in
+// shared memory and writes the set bits in order.
+__global__ void __launch_bounds__(1024)
+    k_coo_big(BuildSpec s, int32_t* __restrict__ counts, int32_t* __restrict__ coo_tmp,
+              const int32_t* __restrict__ big_list, const int32_t* __restrict__ big_count,
+              BuildInfo* info) {
+    extern __shared__ uint32_t bits[];
+    __shared__ int32_t warp_tot[32];
+    __shared__ int32_t carry;
+    const int words = (s.n + 31) >> 5;
+    const int nb = *big_count;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int q = blockIdx.x; q < nb; q += gridDim.x) {
+        const int64_t r = big_list[q];
+        const int64_t p0 = s.in_row_ptr[r], p1 = s.in_row_ptr[r + 1];
+        for (int w = threadIdx.x; w < words; w += blockDim.x) bits[w] = 0u;
+        if (threadIdx.x == 0) carry = 0;
+        __syncthreads();
+        for (int64_t p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
+            const int c = s.in_col_idx[p];
+            if ((unsigned)c >= (unsigned)s.n) {
+                raise(info, kBuildBadColumn);
+                continue;
+            }
+            atomicOr(&bits[c >> 5], 1u << (c & 31));
+        }
+        if (threadIdx.x == 0 && s.add_diagonal) {
+            const int i = (int)(r % s.n);
+            atomicOr(&bits[i >> 5], 1u << (i & 31));
+        }
+        __syncthreads();
+        const int64_t base = p0 + r;
+        for (int w0 = 0; w0 < words; w0 += blockDim.x) {
+            const int w = w0 + threadIdx.x;
+            const uint32_t m = w < words ? bits[w] : 0u;
+            const int c = __popc(m);
+            int inc = c;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, inc, off);
+                if (lane >= off) inc += y;
+            }
+            if (lane == 31) warp_tot[warp] = inc;
+            __syncthreads();
+            if (warp == 0) {
+                const int nw = blockDim.x >> 5;
+                const int x = lane < nw ? warp_tot[lane] : 0;
+                int xi = x;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, xi, off);
+                    if (lane >= off) xi += y;
+                }
+                if (lane < nw) warp_tot[lane] = xi - x;
+            }
+            __syncthreads();
+            int pos = carry + warp_tot[warp] + inc - c;
+            uint32_t mm = m;
+            while (mm) {
+                const int bit = __ffs(mm) - 1;
+                coo_tmp[base + pos++] = w * 32 + bit;
+                mm &= mm - 1;
+            }
+            __syncthreads();
+            if (threadIdx.x == blockDim.x - 1) carry = pos;
+            __syncthreads();
+        }
+        if (threadIdx.x == 0) counts[r] = carry;
+        __syncthreads();
+    }
+}
+
+__global__ void k_flag_big_rows(const int32_t* big_count, BuildInfo* info) {
+    if (threadIdx.x == 0 && *big_count > 0) raise(info, kBuildRowTooLong);
+}
+
+__device__ __forceinline__ int64_t block_exclusive_scan(int64_t x, int64_t* total) {
+    __shared__ int64_t wsum[32];
+    __shared__ int64_t tot;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int64_t inc = x;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, (long long)inc, off);
+        if (lane >= off) inc += y;
+    }
+    if (lane == 31) wsum[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        const int nw = blockDim.x >> 5;
+        const int64_t w = lane < nw ? wsum[lane] : 0;
+        int64_t wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const long long y = __shfl_up_sync(0xffffffffu, (long long)wi, off);
+            if (lane >= off) wi += y;
+        }
+        if (lane < nw) wsum[lane] = wi - w;
+        if (lane == 31) tot = wi;
+    }
+    __syncthreads();
+    const int64_t res = wsum[warp] + inc - x;
+    *total = tot;
+    __syncthreads();
+    return res;
+}
+
+// Tile t of kScanTile counts: local exclusive prefixes + the tile's total.
+__global__ void __launch_bounds__(kScanThreads)
+    k_scan_tiles(const int32_t* __restrict__ counts, int64_t rows, int64_t* __restrict__ pref,
+                 int64_t* __restrict__ tile_sums) {
+    const int64_t base = (int64_t)blockIdx.x * kScanTile + (int64_t)threadIdx.x * kScanItems;
+    int64_t v[kScanItems], sum = 0;
+#pragma unroll
+    for (int t = 0; t < kScanItems; ++t) {
+        v[t] = base + t < rows ? counts[base + t] : 0;
+        sum += v[t];
+    }
+    int64_t total;
+    int64_t run = block_exclusive_scan(sum, &total);
+#pragma unroll
+    for (int t = 0; t < kScanItems; ++t) {
+        if (base + t < rows) pref[base + t] = run;
+        run += v[t];
+    }
+    if (threadIdx.x == 0) tile_sums[blockIdx.x] = total;
+}
+
+// One block: exclusive scan of the tile totals in place; the grand total -> info.
+__global__ void __launch_bounds__(kScanThreads)
+    k_scan_tile_sums(int64_t* __restrict__ tile_sums, int64_t ntiles, BuildInfo* info) {
+    int64_t carry = 0;
+    for (int64_t t0 = 0; t0 < ntiles; t0 += kScanThreads) {
+        const int64_t t = t0 + threadIdx.x;
+        const int64_t v = t < ntiles ? tile_sums[t] : 0;
+        int64_t total;
+        const int64_t ex = block_exclusive_scan(v, &total);
+        if (t < ntiles) tile_sums[t] = carry + ex;
+        carry += total;
+    }
+    if (threadIdx.x == 0) {
+        info->nnz = carry;
+        if (carry > INT_MAX) atomicOr(&info->err, kBuildTooMany);
+    }
+}
+
+__global__ void k_scan_finalize(const int64_t* __restrict__ pref,
+                                const int64_t* __restrict__ tile_sums, int64_t rows,
+                                const BuildInfo* info, int32_t* __restrict__ row_ptr) {
+    for (int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; r <= rows;
+         r += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t v = r < rows ? pref[r] + tile_sums[r / kScanTile] : info->nnz;
+        row_ptr[r] = v > INT_MAX ? INT_MAX : (int32_t)v;
+    }
+}
+
+// Phase 2, one warp per row: interval rows, COO rows (copied from coo_tmp) and
+// user CSR rows (copied).
+__global__ void k_fill_warp(BuildSpec s, const int32_t* __restrict__ row_ptr,
+                            const int32_t* __restrict__ coo_tmp, int32_t* __restrict__ col_idx) {
+    const int64_t rows = (int64_t)s.num_masks * s.n;
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t r = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+         r += warps) {
+        const int64_t o0 = row_ptr[r], o1 = row_ptr[r + 1];
+        int64_t lo, hi;
+        if (s.kind == SPATTN_MASK_COO) {
+            const int32_t* src = coo_tmp + s.in_row_ptr[r] + r;
+            for (int64_t t = lane; t < o1 - o0; t += 32) col_idx[o0 + t] = src[t];
+        } else if (s.kind == SPATTN_MASK_CSR) {
+            const int32_t* src = s.in_col_idx + s.in_row_ptr[r];
+            for (int64_t t = lane; t < o1 - o0; t += 32) col_idx[o0 + t] = src[t];
+        } else if (row_interval(s, r, lo, hi, nullptr)) {
+            for (int64_t t = lane; t < o1 - o0; t += 32) col_idx[o0 + t] = (int32_t)(lo + t);
+        }
+    }
+}
+
+// Phase 2, one thread per non-global BLOCK_STRIDED_GLOBAL row: ordered walk.
+__global__ void k_fill_bsg(BuildSpec s, const int32_t* __restrict__ row_ptr,
+                           int32_t* __restrict__ col_idx) {
+    const int64_t rows = (int64_t)s.num_masks * s.n;
+    for (int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; r < rows;
+         r += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = r % s.n;
+        if (i < s.n_global) continue;
+        int64_t o = row_ptr[r];
+        const int64_t o1 = row_ptr[r + 1];
+        for (int64_t j = bsg_next(s, i, 0); j < s.n && o < o1; j = bsg_next(s, i, j + 1))
+            col_idx[o++] = (int32_t)j;
+    }
+}
+
+unsigned grid_for(int64_t work, int per_block, int64_t cap = 1 << 16) {
+    int64_t g = (work + per_block - 1) / per_block;
+    if (g < 1) g = 1;
+    if (g > cap) g = cap;
+    return (unsigned)g;
+}
+
+}  // namespace
+
+int64_t scan_tmp_elems(int64_t rows) { return rows + 1 + (rows + kScanTile - 1) / kScanTile + 1; }
+
+cudaError_t build_phase1(const BuildSpec& s, int32_t* row_ptr, int32_t* counts,
+                         int64_t* scan_tmp, int32_t* coo_tmp, BuildInfo* info,
+                         cudaStream_t stream) {
+    const int64_t rows = (int64_t)s.num_masks * s.n;
+    cudaError_t e;
+    if (s.kind == SPATTN_MASK_COO) {
+        // big-row queue lives after the scan area
+        int32_t* big_count = reinterpret_cast<int32_t*>(scan_tmp + scan_tmp_elems(rows));
+        int32_t* big_list = big_count + 4;
+        e = cudaMemsetAsync(big_count, 0, sizeof(int32_t), stream);
+        if (e != cudaSuccess) return e;
+        k_coo_sort<<<grid_for(rows, kCooWarps), kCooWarps * 32, 0, stream>>>(
+            s, counts, coo_tmp, big_list, big_count, info);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (s.in_nnz + (s.add_diagonal ? 1 : 0) > kCooWarpCap) {
+            const int words = (s.n + 31) / 32;
+            const size_t smem = (size_t)words * 4;
+            if (smem <= (size_t)kBitmapMaxBytes) {
+                e = cudaFuncSetAttribute(k_coo_big, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+                if (e != cudaSuccess) return e;
+                k_coo_big<<<grid_for(rows, 1, 512), 1024, smem, stream>>>(s, counts, coo_tmp,
+                                                                         big_list, big_count, info);
+                if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            } else {
+                // the n-bit map does not fit in shared memory: queued rows are an error
+                k_flag_big_rows<<<1, 32, 0, stream>>>(big_count, info);
+                if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            }
+        }
+    } else {
+        k_count<<<grid_for(rows, 256), 256, 0, stream>>>(s, counts, info);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (s.kind == SPATTN_MASK_CSR) {
+            k_check_csr<<<grid_for(rows, 8), 256, 0, stream>>>(s, info);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+    }
+    const int64_t ntiles = (rows + kScanTile - 1) / kScanTile;
+    int64_t* pref = scan_tmp;
+    int64_t* tile_sums = scan_tmp + rows + 1;
+    k_scan_tiles<<<(unsigned)ntiles, kScanThreads, 0, stream>>>(counts, rows, pref, tile_sums);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_scan_tile_sums<<<1, kScanThreads, 0, stream>>>(tile_sums, ntiles, info);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_scan_finalize<<<grid_for(rows + 1, 256), 256, 0, stream>>>(pref, tile_sums, rows, info,
+                                                                 row_ptr);
+    return cudaGetLastError();
+}
+
+cudaError_t build_phase2(const BuildSpec& s, const int32_t* row_ptr, const int32_t* coo_tmp,
+                         int32_t* col_idx, cudaStream_t stream) {
+    const int64_t rows = (int64_t)s.num_masks * s.n;
+    k_fill_warp<<<grid_for(rows, 8), 256, 0, stream>>>(s, row_ptr, coo_tmp, col_idx);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (s.kind == SPATTN_MASK_BLOCK_STRIDED_GLOBAL) {
+        k_fill_bsg<<<grid_for(rows, 128), 128, 0, stream>>>(s, row_ptr, col_idx);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+
+}  // namespace spattn

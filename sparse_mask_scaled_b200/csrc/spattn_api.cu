@@ -1,0 +1,455 @@
+// C ABI of libspattn: argument checks, the stream-ordered memory pool, mask
+// handles and kernel launches. Every numerical step runs in the kernels of
+// fwd_gather.cu and mask_build.cu; this file only validates and schedules.
+//
+// Argument checks run before any CUDA call, so a rejected call touches no
+// device state.
+#include "spattn.h"
+#include "spattn_internal.cuh"
+
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+using namespace spattn;
+
+struct spattn_mask_s {
+    int device;
+    cudaStream_t stream;
+    int32_t n;
+    int32_t num_masks;
+    int64_t nnz;
+    int32_t* row_ptr;
+    int32_t* col_idx;
+    int32_t* long_rows;
+    int64_t n_long;
+};
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+int fail(int status, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+    return status;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    if (e == cudaErrorMemoryAllocation)
+        return fail(SPATTN_ERR_OOM, "%s: %s", what, cudaGetErrorString(e));
+    return fail(SPATTN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define CUDA_TRY(call, what)                      \
+    do {                                          \
+        cudaError_t e_ = (call);                  \
+        if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+    } while (0)
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+cudaMemPool_t g_pool[kMaxDevices];
+int g_num_sms[kMaxDevices];
+
+// The library's stream-ordered pool on `dev` (memory is kept cached between
+// calls rather than returned to the driver).
+cudaError_t device_state(int dev, cudaMemPool_t* pool, int* num_sms) {
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_pool[dev]) {
+        cudaMemPoolProps props;
+        memset(&props, 0, sizeof props);
+        props.allocType = cudaMemAllocationTypePinned;
+        props.handleTypes = cudaMemHandleTypeNone;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t p;
+        cudaError_t e = cudaMemPoolCreate(&p, &props);
+        if (e != cudaSuccess) return e;
+        uint64_t keep = UINT64_MAX;
+        e = cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
+        if (e != cudaSuccess) return e;
+        int sms = 0;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        g_pool[dev] = p;
+        g_num_sms[dev] = sms;
+    }
+    *pool = g_pool[dev];
+    if (num_sms) *num_sms = g_num_sms[dev];
+    return cudaSuccess;
+}
+
+template <typename T>
+cudaError_t pool_alloc(T** ptr, int64_t elems, cudaMemPool_t pool, cudaStream_t s) {
+    const size_t bytes = (size_t)(elems > 0 ? elems : 1) * sizeof(T);
+    return cudaMallocFromPoolAsync(reinterpret_cast<void**>(ptr), bytes, pool, s);
+}
+
+int elem_size(int32_t dtype) { return dtype == SPATTN_BF16 ? 2 : 4; }
+
+bool dtype_ok(int32_t dtype) { return dtype == SPATTN_BF16 || dtype == SPATTN_F32; }
+
+// q, k, v and out: [B, H, n, d] with stride 1 over d and 16-byte vector access.
+int check_qkv(const spattn_tensor* t, const char* name, const int64_t* shape, int32_t dtype) {
+    if (!t) return fail(SPATTN_ERR_INVALID_ARG, "%s is NULL", name);
+    if (t->reserved != 0) return fail(SPATTN_ERR_INVALID_ARG, "%s.reserved must be 0", name);
+    if (t->dtype != dtype)
+        return fail(SPATTN_ERR_INVALID_ARG, "%s dtype %d differs from q's %d", name, t->dtype, dtype);
+    for (int x = 0; x < 4; ++x)
+        if (t->shape[x] != shape[x])
+            return fail(SPATTN_ERR_INVALID_ARG, "%s shape[%d] = %lld, expected %lld", name, x,
+                        (long long)t->shape[x], (long long)shape[x]);
+    if (!t->data) return fail(SPATTN_ERR_INVALID_ARG, "%s.data is NULL", name);
+    if (t->stride[3] != 1) return fail(SPATTN_ERR_UNSUPPORTED, "%s needs stride 1 over d", name);
+    const int es = elem_size(dtype);
+    if (((uintptr_t)t->data) % 16 != 0)
+        return fail(SPATTN_ERR_UNSUPPORTED, "%s.data is not 16-byte aligned", name);
+    for (int x = 0; x < 3; ++x) {
+        if (t->shape[x] > 1 && ((t->stride[x] * es) % 16 != 0))
+            return fail(SPATTN_ERR_UNSUPPORTED, "%s stride[%d] is not a multiple of 16 bytes", name, x);
+        if (t->shape[x] > 1 && t->stride[x] < 0)
+            return fail(SPATTN_ERR_UNSUPPORTED, "%s stride[%d] is negative", name, x);
+    }
+    return SPATTN_OK;
+}
+
+int check_addend(const spattn_tensor* t, const char* name, const int64_t* full, AddendView* view) {
+    memset(view, 0, sizeof *view);
+    if (!t) return SPATTN_OK;
+    if (t->reserved != 0) return fail(SPATTN_ERR_INVALID_ARG, "%s.reserved must be 0", name);
+    if (!dtype_ok(t->dtype)) return fail(SPATTN_ERR_UNSUPPORTED, "%s dtype %d", name, t->dtype);
+    if (!t->data) return fail(SPATTN_ERR_INVALID_ARG, "%s.data is NULL", name);
+    int64_t st[4];
+    for (int x = 0; x < 4; ++x) {
+        if (t->shape[x] != 1 && t->shape[x] != full[x])
+            return fail(SPATTN_ERR_INVALID_ARG,
+                        "%s shape[%d] = %lld does not broadcast to %lld", name, x,
+                        (long long)t->shape[x], (long long)full[x]);
+        st[x] = t->shape[x] == 1 ? 0 : t->stride[x];
+    }
+    if (((uintptr_t)t->data) % elem_size(t->dtype) != 0)
+        return fail(SPATTN_ERR_INVALID_ARG, "%s.data is not element-aligned", name);
+    view->data = t->data;
+    view->dtype = t->dtype == SPATTN_BF16 ? 0 : 1;
+    view->s0 = st[0];
+    view->s1 = st[1];
+    view->s2 = st[2];
+    view->s3 = st[3];
+    return SPATTN_OK;
+}
+
+// Shared argument checks of the two forward entry points. Fills everything in
+// `p` except the CSR and the schedule.
+int check_fwd(const spattn_tensor* q, const spattn_tensor* k, const spattn_tensor* v,
+              const spattn_tensor* add_mask, const spattn_tensor* bias, float scale,
+              const spattn_tensor* out, float* lse, FwdParams* p, int* dtype, int* d) {
+    if (!q) return fail(SPATTN_ERR_INVALID_ARG, "q is NULL");
+    if (!dtype_ok(q->dtype)) return fail(SPATTN_ERR_UNSUPPORTED, "q dtype %d", q->dtype);
+    for (int x = 0; x < 4; ++x)
+        if (q->shape[x] < 0) return fail(SPATTN_ERR_INVALID_ARG, "q shape[%d] < 0", x);
+    const int64_t B = q->shape[0], H = q->shape[1], n = q->shape[2], D = q->shape[3];
+    if (D != 32 && D != 64 && D != 128)
+        return fail(SPATTN_ERR_UNSUPPORTED, "head dim %lld (supported: 32, 64, 128)", (long long)D);
+    if (B > 0x7fffffff || H > 0x7fffffff || n > 0x7ffffffe || B * H > 0x7fffffff)
+        return fail(SPATTN_ERR_UNSUPPORTED, "B, H or n too large");
+    int r;
+    if ((r = check_qkv(q, "q", q->shape, q->dtype))) return r;
+    if ((r = check_qkv(k, "k", q->shape, q->dtype))) return r;
+    if ((r = check_qkv(v, "v", q->shape, q->dtype))) return r;
+    if ((r = check_qkv(out, "out", q->shape, q->dtype))) return r;
+    if (lse && ((uintptr_t)lse) % 4 != 0) return fail(SPATTN_ERR_INVALID_ARG, "lse not aligned");
+    if (!(scale == scale)) return fail(SPATTN_ERR_INVALID_ARG, "scale is NaN");
+    const int64_t full[4] = {B, H, n, n};
+    memset(p, 0, sizeof *p);
+    if ((r = check_addend(add_mask, "add_mask", full, &p->mask))) return r;
+    if ((r = check_addend(bias, "bias", full, &p->bias))) return r;
+    auto bs = [](const spattn_tensor* t, int x) { return t->shape[x] == 1 ? 0 : t->stride[x]; };
+    p->q = q->data;
+    p->k = k->data;
+    p->v = v->data;
+    p->out = out->data;
+    p->lse = lse;
+    p->q_sb = bs(q, 0); p->q_sh = bs(q, 1); p->q_sn = bs(q, 2);
+    p->k_sb = bs(k, 0); p->k_sh = bs(k, 1); p->k_sn = bs(k, 2);
+    p->v_sb = bs(v, 0); p->v_sh = bs(v, 1); p->v_sn = bs(v, 2);
+    p->o_sb = bs(out, 0); p->o_sh = bs(out, 1); p->o_sn = bs(out, 2);
+    p->B = (int)B;
+    p->H = (int)H;
+    p->n = (int)n;
+    p->has_extra = (p->mask.data || p->bias.data) ? 1 : 0;
+    p->qk_scale_log2 = scale * kLog2e;
+    *dtype = q->dtype == SPATTN_BF16 ? 0 : 1;
+    *d = (int)D;
+    return SPATTN_OK;
+}
+
+int launch_fwd(FwdParams& p, int dtype, int d, int num_sms, cudaStream_t s) {
+    cudaError_t e = launch_fwd_long_rows(p, dtype, d, num_sms, s);
+    if (e != cudaSuccess) return cuda_fail(e, "long-row kernel launch");
+    e = launch_fwd_short_rows(p, dtype, d, s);
+    if (e != cudaSuccess) return cuda_fail(e, "row kernel launch");
+    return SPATTN_OK;
+}
+
+int build_status(unsigned err) {
+    if (err & (kBuildTooMany | kBuildRowTooLong)) {
+        return fail(SPATTN_ERR_UNSUPPORTED, "%s",
+                    (err & kBuildTooMany) ? "more than 2^31-1 nonzeros"
+                                          : "a COO row has more than 1024 candidates and n > 1572864");
+    }
+    if (err & kBuildNegativeWidth) return fail(SPATTN_ERR_BAD_CSR, "negative half-width");
+    if (err & kBuildBadRowPtr) return fail(SPATTN_ERR_BAD_CSR, "row_ptr is not a valid prefix sum");
+    if (err & kBuildBadColumn) return fail(SPATTN_ERR_BAD_CSR, "a column index is outside [0, n)");
+    if (err & kBuildUnsorted) return fail(SPATTN_ERR_BAD_CSR, "a CSR row is not strictly increasing");
+    return SPATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* spattn_last_error(void) { return g_msg; }
+
+int spattn_version(void) { return 100; /* 0.1.0 */ }
+
+int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_mask* out) {
+    g_msg[0] = 0;
+    if (!out) return fail(SPATTN_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (!spec) return fail(SPATTN_ERR_INVALID_ARG, "spec is NULL");
+    const spattn_mask_spec& sp = *spec;
+    if (sp.kind < SPATTN_MASK_CSR || sp.kind > SPATTN_MASK_DENSE)
+        return fail(SPATTN_ERR_INVALID_ARG, "unknown mask kind %d", sp.kind);
+    if (sp.n < 1) return fail(SPATTN_ERR_INVALID_ARG, "n must be >= 1");
+    if (sp.num_masks < 1) return fail(SPATTN_ERR_INVALID_ARG, "num_masks must be >= 1");
+    const int64_t rows = (int64_t)sp.n * sp.num_masks;
+    if (rows > 0x7ffffffe) return fail(SPATTN_ERR_UNSUPPORTED, "num_masks * n too large");
+    if (sp.kind == SPATTN_MASK_SLIDING && sp.window < 0)
+        return fail(SPATTN_ERR_INVALID_ARG, "window must be >= 0");
+    if (sp.kind == SPATTN_MASK_VARWIN && !sp.half_widths)
+        return fail(SPATTN_ERR_INVALID_ARG, "half_widths is NULL");
+    if (sp.kind == SPATTN_MASK_BLOCK_STRIDED_GLOBAL &&
+        (sp.block < 0 || sp.stride < 0 || sp.n_global < 0))
+        return fail(SPATTN_ERR_INVALID_ARG, "block, stride and n_global must be >= 0");
+    if (sp.kind == SPATTN_MASK_CSR || sp.kind == SPATTN_MASK_COO) {
+        if (!sp.in_row_ptr) return fail(SPATTN_ERR_INVALID_ARG, "in_row_ptr is NULL");
+        if (sp.in_nnz < 0 || sp.in_nnz > 0x7fffffff)
+            return fail(SPATTN_ERR_INVALID_ARG, "in_nnz out of range");
+        if (sp.in_nnz > 0 && !sp.in_col_idx) return fail(SPATTN_ERR_INVALID_ARG, "in_col_idx is NULL");
+    }
+    cudaStream_t s = (cudaStream_t)stream_v;
+    int dev;
+    CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
+    cudaMemPool_t pool;
+    CUDA_TRY(device_state(dev, &pool, nullptr), "memory pool");
+
+    BuildSpec bs;
+    bs.kind = sp.kind;
+    bs.n = sp.n;
+    bs.num_masks = sp.num_masks;
+    bs.window = sp.window;
+    bs.block = sp.block;
+    bs.stride = sp.stride;
+    bs.n_global = sp.n_global;
+    bs.add_diagonal = sp.add_diagonal ? 1 : 0;
+    bs.half_widths = sp.half_widths;
+    bs.in_row_ptr = sp.in_row_ptr;
+    bs.in_col_idx = sp.in_col_idx;
+    bs.in_nnz = sp.in_nnz;
+
+    int32_t *row_ptr = nullptr, *counts = nullptr, *coo_tmp = nullptr;
+    int64_t* scan_tmp = nullptr;
+    BuildInfo* info = nullptr;
+    const bool coo = sp.kind == SPATTN_MASK_COO;
+    const int64_t scan_elems = scan_tmp_elems(rows) + (coo ? (rows + 6) / 2 + 1 : 0);
+    auto release_tmp = [&]() {
+        if (counts) cudaFreeAsync(counts, s);
+        if (scan_tmp) cudaFreeAsync(scan_tmp, s);
+        if (coo_tmp) cudaFreeAsync(coo_tmp, s);
+        if (info) cudaFreeAsync(info, s);
+        counts = coo_tmp = nullptr;
+        scan_tmp = nullptr;
+        info = nullptr;
+    };
+    cudaError_t e = pool_alloc(&row_ptr, rows + 1, pool, s);
+    if (e == cudaSuccess) e = pool_alloc(&counts, rows, pool, s);
+    if (e == cudaSuccess) e = pool_alloc(&scan_tmp, scan_elems, pool, s);
+    if (e == cudaSuccess && coo) e = pool_alloc(&coo_tmp, sp.in_nnz + rows, pool, s);
+    if (e == cudaSuccess) e = pool_alloc(&info, 1, pool, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(info, 0, sizeof(BuildInfo), s);
+    if (e == cudaSuccess) e = build_phase1(bs, row_ptr, counts, scan_tmp, coo_tmp, info, s);
+    BuildInfo hinfo;
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&hinfo, info, sizeof hinfo, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) {
+        release_tmp();
+        if (row_ptr) cudaFreeAsync(row_ptr, s);
+        return cuda_fail(e, "mask build (phase 1)");
+    }
+    int st = build_status(hinfo.err);
+    if (st != SPATTN_OK) {
+        release_tmp();
+        cudaFreeAsync(row_ptr, s);
+        return st;
+    }
+    spattn_mask m = new spattn_mask_s;
+    memset(m, 0, sizeof *m);
+    m->device = dev;
+    m->stream = s;
+    m->n = sp.n;
+    m->num_masks = sp.num_masks;
+    m->nnz = hinfo.nnz;
+    m->row_ptr = row_ptr;
+    e = pool_alloc(&m->col_idx, hinfo.nnz, pool, s);
+    if (e == cudaSuccess) e = build_phase2(bs, row_ptr, coo_tmp, m->col_idx, s);
+    if (e == cudaSuccess) e = pool_alloc(&m->long_rows, rows, pool, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(&info->n_long, 0, sizeof(int32_t), s);
+    if (e == cudaSuccess)
+        e = launch_classify_long_rows(row_ptr, rows, hinfo.nnz, m->long_rows, &info->n_long, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&hinfo, info, sizeof hinfo, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    release_tmp();
+    if (e != cudaSuccess) {
+        spattn_destroy_mask(m);
+        return cuda_fail(e, "mask build (phase 2)");
+    }
+    m->n_long = hinfo.n_long;
+    *out = m;
+    return SPATTN_OK;
+}
+
+int spattn_mask_info(spattn_mask m, int32_t* n, int32_t* num_masks, int64_t* nnz,
+                     const int32_t** row_ptr, const int32_t** col_idx, int64_t* n_long) {
+    g_msg[0] = 0;
+    if (!m) return fail(SPATTN_ERR_INVALID_ARG, "mask is NULL");
+    if (n) *n = m->n;
+    if (num_masks) *num_masks = m->num_masks;
+    if (nnz) *nnz = m->nnz;
+    if (row_ptr) *row_ptr = m->row_ptr;
+    if (col_idx) *col_idx = m->col_idx;
+    if (n_long) *n_long = m->n_long;
+    return SPATTN_OK;
+}
+
+int spattn_mask_copy_csr(spattn_mask m, int32_t* row_ptr_dst, int32_t* col_idx_dst,
+                         void* stream_v) {
+    g_msg[0] = 0;
+    if (!m) return fail(SPATTN_ERR_INVALID_ARG, "mask is NULL");
+    cudaStream_t s = (cudaStream_t)stream_v;
+    const int64_t rows = (int64_t)m->n * m->num_masks;
+    if (row_ptr_dst)
+        CUDA_TRY(cudaMemcpyAsync(row_ptr_dst, m->row_ptr, (size_t)(rows + 1) * sizeof(int32_t),
+                                 cudaMemcpyDefault, s),
+                 "row_ptr copy");
+    if (col_idx_dst && m->nnz > 0)
+        CUDA_TRY(cudaMemcpyAsync(col_idx_dst, m->col_idx, (size_t)m->nnz * sizeof(int32_t),
+                                 cudaMemcpyDefault, s),
+                 "col_idx copy");
+    return SPATTN_OK;
+}
+
+int spattn_destroy_mask(spattn_mask m) {
+    g_msg[0] = 0;
+    if (!m) return SPATTN_OK;
+    int prev = -1;
+    cudaGetDevice(&prev);
+    if (prev != m->device) cudaSetDevice(m->device);
+    cudaError_t e = cudaSuccess, e2;
+    if (m->row_ptr && (e2 = cudaFreeAsync(m->row_ptr, m->stream)) != cudaSuccess) e = e2;
+    if (m->col_idx && (e2 = cudaFreeAsync(m->col_idx, m->stream)) != cudaSuccess) e = e2;
+    if (m->long_rows && (e2 = cudaFreeAsync(m->long_rows, m->stream)) != cudaSuccess) e = e2;
+    if (prev >= 0 && prev != m->device) cudaSetDevice(prev);
+    delete m;
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync");
+    return SPATTN_OK;
+}
+
+int spattn_fwd(const spattn_tensor* q, const spattn_tensor* k, const spattn_tensor* v,
+               const int32_t* row_ptr, const int32_t* col_idx, int32_t num_masks, int64_t nnz,
+               const spattn_tensor* add_mask, const spattn_tensor* bias, float scale,
+               const spattn_tensor* out, float* lse, void* stream_v) {
+    g_msg[0] = 0;
+    FwdParams p;
+    int dtype, d;
+    int r = check_fwd(q, k, v, add_mask, bias, scale, out, lse, &p, &dtype, &d);
+    if (r) return r;
+    if (num_masks != 1 && num_masks != p.B)
+        return fail(SPATTN_ERR_INVALID_ARG, "num_masks must be 1 or B");
+    if (!row_ptr) return fail(SPATTN_ERR_INVALID_ARG, "row_ptr is NULL");
+    if (nnz < 0) return fail(SPATTN_ERR_INVALID_ARG, "nnz < 0");
+    if (nnz > 0 && !col_idx) return fail(SPATTN_ERR_INVALID_ARG, "col_idx is NULL");
+    if ((int64_t)p.B * p.H * p.n == 0) return SPATTN_OK;
+    cudaStream_t s = (cudaStream_t)stream_v;
+    int dev, sms;
+    CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
+    cudaMemPool_t pool;
+    CUDA_TRY(device_state(dev, &pool, &sms), "memory pool");
+    p.num_masks = num_masks;
+    p.row_ptr = row_ptr;
+    p.col_idx = col_idx;
+    p.nnz = nnz;
+    const int64_t rows = (int64_t)num_masks * p.n;
+    int32_t* scratch = nullptr;  // [0]: long-row count, [1 ..]: long-row list
+    CUDA_TRY(pool_alloc(&scratch, rows + 1, pool, s), "scratch allocation");
+    cudaError_t e = cudaMemsetAsync(scratch, 0, sizeof(int32_t), s);
+    if (e == cudaSuccess) e = launch_classify_long_rows(row_ptr, rows, nnz, scratch + 1, scratch, s);
+    if (e != cudaSuccess) {
+        cudaFreeAsync(scratch, s);
+        return cuda_fail(e, "long-row classification");
+    }
+    p.long_rows = scratch + 1;
+    p.long_count_dev = scratch;
+    p.long_count_host = -1;
+    r = launch_fwd(p, dtype, d, sms, s);
+    cudaError_t ef = cudaFreeAsync(scratch, s);
+    if (r) return r;
+    if (ef != cudaSuccess) return cuda_fail(ef, "cudaFreeAsync");
+    return SPATTN_OK;
+}
+
+int spattn_fwd_mask(const spattn_tensor* q, const spattn_tensor* k, const spattn_tensor* v,
+                    spattn_mask mask, const spattn_tensor* add_mask, const spattn_tensor* bias,
+                    float scale, const spattn_tensor* out, float* lse, void* stream_v) {
+    g_msg[0] = 0;
+    FwdParams p;
+    int dtype, d;
+    int r = check_fwd(q, k, v, add_mask, bias, scale, out, lse, &p, &dtype, &d);
+    if (r) return r;
+    if (!mask) return fail(SPATTN_ERR_INVALID_ARG, "mask is NULL");
+    if (mask->n != p.n) return fail(SPATTN_ERR_INVALID_ARG, "mask n %d != q n %d", mask->n, p.n);
+    if (mask->num_masks != 1 && mask->num_masks != p.B)
+        return fail(SPATTN_ERR_INVALID_ARG, "mask num_masks must be 1 or B");
+    if ((int64_t)p.B * p.H * p.n == 0) return SPATTN_OK;
+    cudaStream_t s = (cudaStream_t)stream_v;
+    int dev, sms;
+    CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
+    if (dev != mask->device) return fail(SPATTN_ERR_INVALID_ARG, "mask lives on another device");
+    cudaMemPool_t pool;
+    CUDA_TRY(device_state(dev, &pool, &sms), "memory pool");
+    p.num_masks = mask->num_masks;
+    p.row_ptr = mask->row_ptr;
+    p.col_idx = mask->col_idx;
+    p.nnz = mask->nnz;
+    p.long_rows = mask->long_rows;
+    p.long_count_dev = nullptr;
+    p.long_count_host = mask->n_long;
+    return launch_fwd(p, dtype, d, sms, s);
+}
+
+int spattn_device_error(void* stream_v, uint32_t* flags) {
+    g_msg[0] = 0;
+    unsigned v = 0;
+    cudaError_t e = read_and_clear_device_error(&v, (cudaStream_t)stream_v);
+    if (flags) *flags = v;
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device error flag");
+    if (v & kErrBadColumn) return fail(SPATTN_ERR_BAD_CSR, "a column index outside [0, n) was skipped");
+    return SPATTN_OK;
+}
+
+}  // extern "C"
