@@ -170,6 +170,30 @@ int spattn_fwd_mask(const spattn_tensor* q, const spattn_tensor* k, const spattn
                     spattn_mask mask, const spattn_tensor* add_mask, const spattn_tensor* bias,
                     float scale, const spattn_tensor* out, float* lse, void* stream);
 
+/* The same operation as spattn_fwd, but the call allocates no device memory.
+ * For callers that cannot call cudaMalloc or take memory from a pool at run
+ * time: for example a host program or plug-in whose memory manager owns the
+ * whole device memory budget and forbids allocations inside its execute step,
+ * or code that must not meet an allocation failure or the synchronisation an
+ * allocation may bring in the middle of its work. The pages describe no such
+ * variant; it has no counterpart there.
+ * The scratch it needs (the list of rows above 1024 nonzeros and its counter)
+ * lives in one fixed array inside the library: SPATTN_NOALLOC_MAX_ROWS + 1
+ * int32 (1 MiB), which every GPU that loads the library holds until the process
+ * exits. num_masks * n must be <= SPATTN_NOALLOC_MAX_ROWS, else the call
+ * returns SPATTN_ERR_UNSUPPORTED without enqueuing anything. The first call on
+ * each device looks up the array's device address (once per device, with that
+ * device current); make that first call before any stream capture. Every call
+ * on a device shares the one array and clears its counter first: calls whose
+ * work can overlap on the GPU (other streams, other host threads) race on it
+ * and must be serialised by the caller. Arguments and errors otherwise as
+ * spattn_fwd. */
+#define SPATTN_NOALLOC_MAX_ROWS 262143
+int spattn_fwd_noalloc(const spattn_tensor* q, const spattn_tensor* k, const spattn_tensor* v,
+                       const int32_t* row_ptr, const int32_t* col_idx, int32_t num_masks,
+                       int64_t nnz, const spattn_tensor* add_mask, const spattn_tensor* bias,
+                       float scale, const spattn_tensor* out, float* lse, void* stream);
+
 /* ------------------------------------------------------------- utilities */
 
 /* Message of the last failed call on this thread ("" if none). Valid until the

@@ -79,6 +79,8 @@ SIGNATURES = {
     "spattn_fwd": (ctypes.c_int, [_TP, _TP, _TP, _P, _P, ctypes.c_int32, ctypes.c_int64, _TP, _TP,
                                   ctypes.c_float, _TP, _P, _P]),
     "spattn_fwd_mask": (ctypes.c_int, [_TP, _TP, _TP, _P, _TP, _TP, ctypes.c_float, _TP, _P, _P]),
+    "spattn_fwd_noalloc": (ctypes.c_int, [_TP, _TP, _TP, _P, _P, ctypes.c_int32, ctypes.c_int64, _TP,
+                                          _TP, ctypes.c_float, _TP, _P, _P]),
     "spattn_last_error": (ctypes.c_char_p, []),
     "spattn_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "spattn_version": (ctypes.c_int, []),
@@ -232,6 +234,29 @@ def spattn_fwd_mask(q, k, v, mask: Mask, add_mask=None, bias=None, scale: Option
                                ctypes.byref(db) if db is not None else None, float(scale),
                                ctypes.byref(do), _ptr(lse), _stream(stream)))
     return out, lse
+
+
+def spattn_fwd_noalloc(q, k, v, row_ptr, col_idx, num_masks: int = 1, add_mask=None, bias=None,
+                       scale: Optional[float] = None, out=None, lse=None, stream=None):
+    """spattn_fwd without any device allocation inside the call: its scratch is
+    a fixed array in the library (num_masks * n <= NOALLOC_MAX_ROWS). For
+    callers that cannot allocate device memory while they run. ``out`` and
+    ``lse`` must be passed in (this wrapper allocates nothing either)."""
+    if out is None or lse is None:
+        raise ValueError("spattn_fwd_noalloc needs caller-provided out and lse")
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
+    dq, dk, dv, do = tensor_desc(q), tensor_desc(k), tensor_desc(v), tensor_desc(out)
+    dm = tensor_desc(add_mask) if add_mask is not None else None
+    db = tensor_desc(bias) if bias is not None else None
+    _check(LIB.spattn_fwd_noalloc(ctypes.byref(dq), ctypes.byref(dk), ctypes.byref(dv),
+                                  _ptr(row_ptr), _ptr(col_idx), int(num_masks), int(col_idx.numel()),
+                                  ctypes.byref(dm) if dm is not None else None,
+                                  ctypes.byref(db) if db is not None else None, float(scale),
+                                  ctypes.byref(do), _ptr(lse), _stream(stream)))
+    return out, lse
+
+
+NOALLOC_MAX_ROWS = 262143
 
 
 def spattn_device_error(stream=None) -> int:

@@ -442,6 +442,74 @@ int spattn_fwd_mask(const spattn_tensor* q, const spattn_tensor* k, const spattn
     return launch_fwd(p, dtype, d, sms, s);
 }
 
+// ---- allocation-free forward: its scratch is this fixed array, part of the
+// library image on every device that loads it.
+static __device__ __align__(256) int32_t g_noalloc_scratch[SPATTN_NOALLOC_MAX_ROWS + 1];
+
+static std::mutex g_noalloc_mu;
+static int32_t* g_noalloc_ptr[kMaxDevices];
+static int g_noalloc_sms[kMaxDevices];
+
+// Device address of the scratch array and the SM count, looked up once per
+// device with that device current. In host code the array's name is only a
+// host-side stand-in, so the kernels are always given the looked-up address.
+static int noalloc_setup(int dev, int32_t** ptr, int* sms) {
+    if (dev < 0 || dev >= kMaxDevices) return fail(SPATTN_ERR_CUDA, "device %d out of range", dev);
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        int32_t* p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+        int n_sms = 0;
+        e = cudaDeviceGetAttribute(&n_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        g_noalloc_sms[dev] = n_sms;
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    *sms = g_noalloc_sms[dev];
+    return SPATTN_OK;
+}
+
+int spattn_fwd_noalloc(const spattn_tensor* q, const spattn_tensor* k, const spattn_tensor* v,
+                       const int32_t* row_ptr, const int32_t* col_idx, int32_t num_masks,
+                       int64_t nnz, const spattn_tensor* add_mask, const spattn_tensor* bias,
+                       float scale, const spattn_tensor* out, float* lse, void* stream_v) {
+    g_msg[0] = 0;
+    FwdParams p;
+    int dtype, d;
+    int r = check_fwd(q, k, v, add_mask, bias, scale, out, lse, &p, &dtype, &d);
+    if (r) return r;
+    if (num_masks != 1 && num_masks != p.B)
+        return fail(SPATTN_ERR_INVALID_ARG, "num_masks must be 1 or B");
+    if (!row_ptr) return fail(SPATTN_ERR_INVALID_ARG, "row_ptr is NULL");
+    if (nnz < 0) return fail(SPATTN_ERR_INVALID_ARG, "nnz < 0");
+    if (nnz > 0 && !col_idx) return fail(SPATTN_ERR_INVALID_ARG, "col_idx is NULL");
+    const int64_t rows = (int64_t)num_masks * p.n;
+    if (rows > SPATTN_NOALLOC_MAX_ROWS)
+        return fail(SPATTN_ERR_UNSUPPORTED,
+                    "spattn_fwd_noalloc: num_masks * n = %lld exceeds its fixed scratch of %d rows",
+                    (long long)rows, SPATTN_NOALLOC_MAX_ROWS);
+    if ((int64_t)p.B * p.H * p.n == 0) return SPATTN_OK;
+    cudaStream_t s = (cudaStream_t)stream_v;
+    int dev, sms;
+    CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
+    int32_t* scratch = nullptr;  // [0]: long-row count, [1 ..]: long-row list
+    if ((r = noalloc_setup(dev, &scratch, &sms))) return r;
+    p.num_masks = num_masks;
+    p.row_ptr = row_ptr;
+    p.col_idx = col_idx;
+    p.nnz = nnz;
+    // the array keeps the previous call's contents: the counter must restart at 0
+    CUDA_TRY(cudaMemsetAsync(scratch, 0, sizeof(int32_t), s), "clearing the no-alloc counter");
+    CUDA_TRY(launch_classify_long_rows(row_ptr, rows, nnz, scratch + 1, scratch, s),
+             "long-row classification");
+    p.long_rows = scratch + 1;
+    p.long_count_dev = scratch;
+    p.long_count_host = -1;
+    return launch_fwd(p, dtype, d, sms, s);
+}
+
 int spattn_device_error(void* stream_v, uint32_t* flags) {
     g_msg[0] = 0;
     unsigned v = 0;
