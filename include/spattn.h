@@ -108,11 +108,19 @@ typedef struct {
     const int32_t* in_row_ptr;  /* CSR, COO: device, [num_masks * n + 1], starts at 0, non-decreasing */
     const int32_t* in_col_idx;  /* CSR, COO: device, [in_nnz], each in [0, n) */
     int64_t in_nnz;             /* CSR, COO: in_row_ptr[num_masks * n] */
+    int32_t tile_min_nnz;       /* tensor-core tiles: a 128 x 128 tile with at least this many
+                                   nonzeros is computed on tensor cores (bf16 inputs);
+                                   0 = default (256), < 0 = never */
+    int32_t reserved;           /* must be 0 */
 } spattn_mask_spec;
 
 /* A built mask: its CSR (row_ptr int32 [num_masks*n + 1], col_idx int32 [nnz]),
- * plus the schedule the forward pass uses (rows long enough to be split over a
- * whole thread block). Owns its device memory. */
+ * plus the schedule the forward pass uses: rows long enough to be split over a
+ * whole thread block, and the tile plan -- the 128 x 128 tiles (128 query rows
+ * by 128 keys) that hold at least tile_min_nnz nonzeros, each with a per-row
+ * bit mask, and the residual CSR of the entries outside those tiles. (Blocks
+ * are cheaper than single entries: the block-sparse remark of the gluon-nlp
+ * discussion, applied tile by tile to any CSR.) Owns its device memory. */
 typedef struct spattn_mask_s* spattn_mask;
 
 /* Build a CSR mask on the device from a pattern (the proposal's "generate the
@@ -136,6 +144,24 @@ int spattn_mask_info(spattn_mask mask, int32_t* n, int32_t* num_masks, int64_t* 
  * pinned for the copy to be asynchronous. */
 int spattn_mask_copy_csr(spattn_mask mask, int32_t* row_ptr_dst, int32_t* col_idx_dst,
                          void* stream);
+
+/* The tile plan's sizes: tensor-core tiles, residual nonzeros (the entries the
+ * gather kernel processes on bf16 inputs) and rows with entries on both paths.
+ * Any output pointer may be NULL. */
+int spattn_mask_plan_info(spattn_mask mask, int64_t* n_tiles, int64_t* residual_nnz,
+                          int64_t* n_mixed_rows);
+
+/* Copy the tile plan into caller buffers (device or host, any may be NULL):
+ * block_tile_off int32 [num_masks * ceil(n/128) + 1] (tiles of query block x are
+ * tile ids block_tile_off[x] .. block_tile_off[x+1]-1), tile_info int32 [n_tiles]
+ * (key tile index, bit 31 set when all 128 x 128 entries are present),
+ * tile_bits uint32 [n_tiles * 128 * 4] (row r of a tile: 4 words, bit c of word
+ * c/32 = column c), residual row_ptr int32 [num_masks * n + 1] and col_idx
+ * int32 [residual_nnz]. Returns SPATTN_ERR_INVALID_ARG when the mask has no
+ * tile plan. Stream-ordered on `stream`. */
+int spattn_mask_copy_plan(spattn_mask mask, int32_t* block_tile_off, int32_t* tile_info,
+                          uint32_t* tile_bits, int32_t* res_row_ptr, int32_t* res_col_idx,
+                          void* stream);
 
 /* Release a mask. Stream-ordered on the stream it was created on. NULL is a no-op. */
 int spattn_destroy_mask(spattn_mask mask);
@@ -164,8 +190,15 @@ int spattn_fwd(const spattn_tensor* q, const spattn_tensor* k, const spattn_tens
                const spattn_tensor* out, float* lse, void* stream);
 
 /* The same operation over a mask built by spattn_create_csr_mask, using its
- * prebuilt schedule. Allocates nothing. The mask's num_masks must be 1 or B and
- * its n must match q. */
+ * prebuilt schedule. The mask's num_masks must be 1 or B and its n must match q.
+ * With bf16 inputs and a tile plan, the plan's tiles run on tensor cores
+ * (tcgen05) and the residual entries on the gather kernel; rows with entries
+ * on both paths are merged with the running max/sum rule. Those rows need a
+ * workspace of B*H*n*(d+2) floats, taken from the library's stream-ordered
+ * pool for the duration of the call (only when the plan has such rows).
+ * fp32 inputs use the gather kernel for every entry.
+ * A bounded wait in the tensor-core kernel that expires raises device error
+ * flag bit 1 (see spattn_device_error). */
 int spattn_fwd_mask(const spattn_tensor* q, const spattn_tensor* k, const spattn_tensor* v,
                     spattn_mask mask, const spattn_tensor* add_mask, const spattn_tensor* bias,
                     float scale, const spattn_tensor* out, float* lse, void* stream);
@@ -201,8 +234,10 @@ int spattn_fwd_noalloc(const spattn_tensor* q, const spattn_tensor* k, const spa
 const char* spattn_last_error(void);
 
 /* Synchronise `stream`, then read and clear the current device's error flags
- * raised by kernels (bit 0: a column index outside [0, n) was skipped).
- * *flags may be NULL. Returns SPATTN_OK, or SPATTN_ERR_BAD_CSR if any flag was set. */
+ * raised by kernels (bit 0: a column index outside [0, n) was skipped; bit 1:
+ * a bounded wait in the tensor-core kernel expired and its rows are invalid).
+ * *flags may be NULL. Returns SPATTN_OK, SPATTN_ERR_TIMEOUT if bit 1 was set,
+ * else SPATTN_ERR_BAD_CSR if bit 0 was set. */
 int spattn_device_error(void* stream, uint32_t* flags);
 
 /* Library version: major * 10000 + minor * 100 + patch. */

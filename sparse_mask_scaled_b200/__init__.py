@@ -61,7 +61,8 @@ class spattn_mask_spec(ctypes.Structure):
                 ("window", ctypes.c_int32), ("block", ctypes.c_int32), ("stride", ctypes.c_int32),
                 ("n_global", ctypes.c_int32), ("add_diagonal", ctypes.c_int32),
                 ("half_widths", ctypes.c_void_p), ("in_row_ptr", ctypes.c_void_p),
-                ("in_col_idx", ctypes.c_void_p), ("in_nnz", ctypes.c_int64)]
+                ("in_col_idx", ctypes.c_void_p), ("in_nnz", ctypes.c_int64),
+                ("tile_min_nnz", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p
@@ -75,6 +76,10 @@ SIGNATURES = {
                                         ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(_P),
                                         ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_int64)]),
     "spattn_mask_copy_csr": (ctypes.c_int, [_P, _P, _P, _P]),
+    "spattn_mask_plan_info": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int64),
+                                             ctypes.POINTER(ctypes.c_int64),
+                                             ctypes.POINTER(ctypes.c_int64)]),
+    "spattn_mask_copy_plan": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P]),
     "spattn_destroy_mask": (ctypes.c_int, [_P]),
     "spattn_fwd": (ctypes.c_int, [_TP, _TP, _TP, _P, _P, ctypes.c_int32, ctypes.c_int64, _TP, _TP,
                                   ctypes.c_float, _TP, _P, _P]),
@@ -146,6 +151,9 @@ class Mask:
         _check(LIB.spattn_mask_info(handle, ctypes.byref(n), ctypes.byref(nm), ctypes.byref(nnz),
                                     ctypes.byref(rp), ctypes.byref(ci), ctypes.byref(nl)))
         self.n, self.num_masks, self.nnz, self.n_long = n.value, nm.value, nnz.value, nl.value
+        nt, rn, nmix = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+        _check(LIB.spattn_mask_plan_info(handle, ctypes.byref(nt), ctypes.byref(rn), ctypes.byref(nmix)))
+        self.n_tiles, self.residual_nnz, self.n_mixed_rows = nt.value, rn.value, nmix.value
 
     def csr(self, stream=None):
         """Copies of (row_ptr, col_idx) as int32 torch tensors on the current device."""
@@ -154,6 +162,22 @@ class Mask:
         ci = torch.empty(max(1, self.nnz), dtype=torch.int32, device="cuda")
         _check(LIB.spattn_mask_copy_csr(self.handle, rp.data_ptr(), ci.data_ptr(), _stream(stream)))
         return rp, ci[: self.nnz]
+
+    def plan(self, stream=None):
+        """Copies of the tile plan (block_tile_off, tile_info, tile_bits,
+        residual row_ptr, residual col_idx) as int32 CUDA tensors, or None."""
+        import torch
+        if self.n_tiles == 0:
+            return None
+        nqb = (self.n + 127) // 128
+        bto = torch.empty(self.num_masks * nqb + 1, dtype=torch.int32, device="cuda")
+        info = torch.empty(max(1, self.n_tiles), dtype=torch.int32, device="cuda")
+        bits = torch.empty(max(1, self.n_tiles * 128 * 4), dtype=torch.int32, device="cuda")
+        rrp = torch.empty(self.num_masks * self.n + 1, dtype=torch.int32, device="cuda")
+        rci = torch.empty(max(1, self.residual_nnz), dtype=torch.int32, device="cuda")
+        _check(LIB.spattn_mask_copy_plan(self.handle, bto.data_ptr(), info.data_ptr(), bits.data_ptr(),
+                                         rrp.data_ptr(), rci.data_ptr(), _stream(stream)))
+        return bto, info[: self.n_tiles], bits[: self.n_tiles * 512], rrp, rci[: self.residual_nnz]
 
     def close(self):
         if self.handle:
@@ -176,7 +200,7 @@ class Mask:
 def spattn_create_csr_mask(kind, n: int, num_masks: int = 1, *, window: int = 0, block: int = 0,
                            stride: int = 0, n_global: int = 0, add_diagonal: bool = False,
                            half_widths=None, in_row_ptr=None, in_col_idx=None,
-                           stream=None) -> Mask:
+                           tile_min_nnz: int = 0, stream=None) -> Mask:
     """Build a CSR mask on the device. ``kind``: a name of MASK_KINDS or its code.
     Array arguments are int32 CUDA tensors."""
     spec = spattn_mask_spec()
@@ -188,6 +212,8 @@ def spattn_create_csr_mask(kind, n: int, num_masks: int = 1, *, window: int = 0,
     spec.in_row_ptr = _ptr(in_row_ptr)
     spec.in_col_idx = _ptr(in_col_idx)
     spec.in_nnz = 0 if in_col_idx is None else int(in_col_idx.numel())
+    spec.tile_min_nnz = int(tile_min_nnz)
+    spec.reserved = 0
     h = _P()
     _check(LIB.spattn_create_csr_mask(ctypes.byref(spec), _stream(stream), ctypes.byref(h)))
     return Mask(h.value)

@@ -20,6 +20,24 @@ LIB = os.path.join(PKG, "libspattn.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
+def cutlass_include() -> str:
+    """CuTe/CUTLASS headers (used only for the tcgen05 descriptor unions)."""
+    cands = [os.environ.get("CUTLASS_INCLUDE")]
+    try:
+        import importlib.util
+        spec = importlib.util.find_spec("flashinfer")
+        if spec and spec.submodule_search_locations:
+            cands.append(os.path.join(list(spec.submodule_search_locations)[0], "data", "cutlass", "include"))
+    except Exception:
+        pass
+    cands.append(os.path.join(sys.prefix, "lib", f"python{sys.version_info.major}.{sys.version_info.minor}",
+                              "site-packages", "flashinfer", "data", "cutlass", "include"))
+    for c in cands:
+        if c and os.path.exists(os.path.join(c, "cute", "arch", "mma_sm100_desc.hpp")):
+            return c
+    raise RuntimeError("CuTe/CUTLASS headers not found (set CUTLASS_INCLUDE)")
+
+
 def _nvcc() -> str:
     for cand in (os.environ.get("NVCC"), shutil.which("nvcc"), "/usr/local/cuda/bin/nvcc"):
         if cand and os.path.exists(cand):
@@ -49,7 +67,7 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     objdir = os.path.join(PKG, "_build")
     os.makedirs(objdir, exist_ok=True)
     common = [nvcc, "-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC",
-              "-I", INCLUDE, "-I", CSRC, "--expt-relaxed-constexpr", *extra]
+              "-I", INCLUDE, "-I", CSRC, "-I", cutlass_include(), "--expt-relaxed-constexpr", *extra]
     objs = []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")

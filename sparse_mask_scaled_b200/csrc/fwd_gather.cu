@@ -250,6 +250,13 @@ __device__ __forceinline__ void merge_groups(State<VEC>& st) {
     }
 }
 
+template <int VEC>
+__device__ __forceinline__ void write_partial(float* dst, const float (&acc)[VEC]) {
+#pragma unroll
+    for (int e = 0; e < VEC; e += 4)
+        *reinterpret_cast<float4*>(dst + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(256) k_fwd_short(const FwdParams P) {
     using C = Cfg<T, D>;
@@ -270,6 +277,22 @@ __global__ void __launch_bounds__(256) k_fwd_short(const FwdParams P) {
     row_steps<T, D>(P, rc, p0, p1, C::STEP, lane, st);
     merge_groups<C::VEC, C::LPR>(st);
 
+    if (P.qb_tile_off) {
+        const int64_t blk = (int64_t)(P.num_masks == 1 ? 0 : b) * P.nqb + (i >> 7);
+        if (P.qb_tile_off[blk + 1] > P.qb_tile_off[blk]) {
+            // the tensor-core kernel finishes this row; hand over the partial state
+            if (p1 > p0) {
+                const int64_t wrow = (int64_t)bh * P.n + i;
+                if (lane < C::LPR)
+                    write_partial<C::VEC>(P.ws_acc + wrow * D + lane * C::VEC, st.acc);
+                if (lane == 0) {
+                    P.ws_ml[wrow * 2] = st.m;
+                    P.ws_ml[wrow * 2 + 1] = st.l;
+                }
+            }
+            return;
+        }
+    }
     if (lane < C::LPR) {
         const float inv = st.l > 0.f ? 1.f / st.l : 0.f;
         float o[C::VEC];
@@ -335,10 +358,24 @@ __global__ void __launch_bounds__(256) k_fwd_long(const FwdParams P) {
                 l = fmaf(sm_l[w], f, l);
                 a = fmaf(sm_acc[w][threadIdx.x], f, a);
             }
-            T* orow = reinterpret_cast<T*>(P.out) + b * P.o_sb + h * P.o_sh + i * P.o_sn;
-            Elem<T>::store1(orow, threadIdx.x, l > 0.f ? a / l : 0.f);
-            if (threadIdx.x == 0 && P.lse)
-                P.lse[((int64_t)b * P.H + h) * P.n + i] = l > 0.f ? (mx + lg2(l)) * kLn2 : -INFINITY;
+            bool partial = false;
+            if (P.qb_tile_off) {
+                const int64_t blk = (int64_t)(P.num_masks == 1 ? 0 : b) * P.nqb + (i >> 7);
+                partial = P.qb_tile_off[blk + 1] > P.qb_tile_off[blk];
+            }
+            const int64_t wrow = ((int64_t)b * P.H + h) * P.n + i;
+            if (partial) {
+                P.ws_acc[wrow * D + threadIdx.x] = a;
+                if (threadIdx.x == 0) {
+                    P.ws_ml[wrow * 2] = mx;
+                    P.ws_ml[wrow * 2 + 1] = l;
+                }
+            } else {
+                T* orow = reinterpret_cast<T*>(P.out) + b * P.o_sb + h * P.o_sh + i * P.o_sn;
+                Elem<T>::store1(orow, threadIdx.x, l > 0.f ? a / l : 0.f);
+                if (threadIdx.x == 0 && P.lse)
+                    P.lse[wrow] = l > 0.f ? (mx + lg2(l)) * kLn2 : -INFINITY;
+            }
         }
         __syncthreads();
     }
@@ -420,6 +457,10 @@ cudaError_t launch_classify_long_rows(const int32_t* row_ptr, int64_t rows, int6
     if (grid > 4096) grid = 4096;
     k_classify_long<<<(unsigned)grid, 256, 0, s>>>(row_ptr, rows, nnz, list, count);
     return cudaGetLastError();
+}
+
+cudaError_t error_flag_address(unsigned** p) {
+    return cudaGetSymbolAddress(reinterpret_cast<void**>(p), g_error_flags);
 }
 
 cudaError_t read_and_clear_device_error(unsigned* flags, cudaStream_t s) {

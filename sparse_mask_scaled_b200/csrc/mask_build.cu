@@ -330,9 +330,11 @@ __global__ void __launch_bounds__(kScanThreads)
     if (threadIdx.x == 0) tile_sums[blockIdx.x] = total;
 }
 
-// One block: exclusive scan of the tile totals in place; the grand total -> info.
+// One block: exclusive scan of the tile totals in place; the grand total -> *total
+// (and the kBuildTooMany bit of *err when it does not fit int32).
 __global__ void __launch_bounds__(kScanThreads)
-    k_scan_tile_sums(int64_t* __restrict__ tile_sums, int64_t ntiles, BuildInfo* info) {
+    k_scan_tile_sums(int64_t* __restrict__ tile_sums, int64_t ntiles, int64_t* total_out,
+                     unsigned* err) {
     int64_t carry = 0;
     for (int64_t t0 = 0; t0 < ntiles; t0 += kScanThreads) {
         const int64_t t = t0 + threadIdx.x;
@@ -343,17 +345,17 @@ __global__ void __launch_bounds__(kScanThreads)
         carry += total;
     }
     if (threadIdx.x == 0) {
-        info->nnz = carry;
-        if (carry > INT_MAX) atomicOr(&info->err, kBuildTooMany);
+        *total_out = carry;
+        if (carry > INT_MAX) atomicOr(err, kBuildTooMany);
     }
 }
 
 __global__ void k_scan_finalize(const int64_t* __restrict__ pref,
                                 const int64_t* __restrict__ tile_sums, int64_t rows,
-                                const BuildInfo* info, int32_t* __restrict__ row_ptr) {
+                                const int64_t* total, int32_t* __restrict__ row_ptr) {
     for (int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; r <= rows;
          r += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t v = r < rows ? pref[r] + tile_sums[r / kScanTile] : info->nnz;
+        const int64_t v = r < rows ? pref[r] + tile_sums[r / kScanTile] : *total;
         row_ptr[r] = v > INT_MAX ? INT_MAX : (int32_t)v;
     }
 }
@@ -445,15 +447,20 @@ cudaError_t build_phase1(const BuildSpec& s, int32_t* row_ptr, int32_t* counts,
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
     }
+    return scan_counts(counts, rows, row_ptr, scan_tmp, &info->nnz, &info->err, stream);
+}
+
+cudaError_t scan_counts(const int32_t* counts, int64_t rows, int32_t* out, int64_t* scan_tmp,
+                        int64_t* total, unsigned* err, cudaStream_t stream) {
     const int64_t ntiles = (rows + kScanTile - 1) / kScanTile;
     int64_t* pref = scan_tmp;
     int64_t* tile_sums = scan_tmp + rows + 1;
+    cudaError_t e;
     k_scan_tiles<<<(unsigned)ntiles, kScanThreads, 0, stream>>>(counts, rows, pref, tile_sums);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_scan_tile_sums<<<1, kScanThreads, 0, stream>>>(tile_sums, ntiles, info);
+    k_scan_tile_sums<<<1, kScanThreads, 0, stream>>>(tile_sums, ntiles, total, err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_scan_finalize<<<grid_for(rows + 1, 256), 256, 0, stream>>>(pref, tile_sums, rows, info,
-                                                                 row_ptr);
+    k_scan_finalize<<<grid_for(rows + 1, 256), 256, 0, stream>>>(pref, tile_sums, rows, total, out);
     return cudaGetLastError();
 }
 

@@ -1,0 +1,188 @@
+// Tile plan of a built mask: which parts of the CSR go to the tensor-core
+// kernel and which stay with the gather kernel.
+//
+// The n x n mask is cut into 128 x 128 tiles (128 query rows by 128 keys).
+// A tile holding at least `tile_min_nnz` nonzeros becomes a tensor-core tile:
+// the kernel computes all 128 x 128 scores with tcgen05 MMAs and a per-row
+// 128-bit mask drops the entries the CSR does not list (the block-sparse idea
+// of the gluon-nlp discussion -- whole blocks are cheaper than single
+// entries -- applied per tile of an arbitrary CSR). The remaining nonzeros form
+// the residual CSR, which the gather kernel processes. Rows that have entries
+// in both are merged with the streaming-softmax rescaling rule.
+#include "spattn_internal.cuh"
+
+namespace spattn {
+namespace {
+
+// One warp per mask row: count the row's nonzeros per key tile (columns are
+// sorted, so a tile's entries form one run per 32-entry chunk).
+__global__ void k_tile_count(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
+                             int n, int64_t rows, int nqb, int nkt, int32_t* __restrict__ cnt) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t r = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+         r += warps) {
+        const int64_t m = r / n, i = r - m * n;
+        const int64_t base = (m * nqb + (i >> 7)) * nkt;
+        const int64_t p0 = row_ptr[r], p1 = row_ptr[r + 1];
+        for (int64_t c0 = p0; c0 < p1; c0 += 32) {
+            const int64_t p = c0 + lane;
+            const bool valid = p < p1;
+            const int kt = valid ? (col_idx[p] >> 7) : -1;
+            const int prev = __shfl_up_sync(0xffffffffu, kt, 1);
+            const bool head = valid && (lane == 0 || prev != kt);
+            const unsigned heads = __ballot_sync(0xffffffffu, head);
+            if (head) {
+                const unsigned above = lane == 31 ? 0u : (heads & (0xffffffffu << (lane + 1)));
+                const int nvalid = (int)((p1 - c0) < 32 ? (p1 - c0) : 32);
+                const int nxt = above ? __ffs(above) - 1 : nvalid;
+                atomicAdd(&cnt[base + kt], nxt - lane);
+            }
+        }
+    }
+}
+
+// One thread per (mask, query block): how many of its key tiles are selected.
+__global__ void k_tile_select(const int32_t* __restrict__ cnt, int64_t nblocks, int nkt,
+                              int min_nnz, int32_t* __restrict__ block_ntiles,
+                              int32_t* __restrict__ n_tc_blocks) {
+    for (int64_t x = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; x < nblocks;
+         x += (int64_t)gridDim.x * blockDim.x) {
+        int c = 0;
+        for (int kt = 0; kt < nkt; ++kt) c += cnt[x * nkt + kt] >= min_nnz;
+        block_ntiles[x] = c;
+        if (c > 0) atomicAdd(n_tc_blocks, 1);
+    }
+}
+
+// Number the selected tiles (block-major, key tiles ascending) and turn the
+// count array into a map (tile id, or -1).
+__global__ void k_tile_assign(int32_t* __restrict__ cnt_map, int64_t nblocks, int nkt, int min_nnz,
+                              const int32_t* __restrict__ block_tile_off,
+                              int32_t* __restrict__ tile_info) {
+    for (int64_t x = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; x < nblocks;
+         x += (int64_t)gridDim.x * blockDim.x) {
+        int idx = block_tile_off[x];
+        for (int kt = 0; kt < nkt; ++kt) {
+            const int c = cnt_map[x * nkt + kt];
+            if (c >= min_nnz) {
+                tile_info[idx] = kt | (c == kTileM * kTileN ? (int)kTileDenseBit : 0);
+                cnt_map[x * nkt + kt] = idx++;
+            } else {
+                cnt_map[x * nkt + kt] = -1;
+            }
+        }
+    }
+}
+
+// One warp per row: set the bits of entries in selected tiles, count the rest.
+__global__ void k_tile_bits(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
+                            int n, int64_t rows, int nqb, int nkt, const int32_t* __restrict__ map,
+                            uint32_t* __restrict__ bits, int32_t* __restrict__ res_cnt) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t r = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+         r += warps) {
+        const int64_t m = r / n, i = r - m * n;
+        const int64_t base = (m * nqb + (i >> 7)) * nkt;
+        const int row_in_tile = (int)(i & 127);
+        int res = 0;
+        for (int64_t p = row_ptr[r] + lane; p < row_ptr[r + 1]; p += 32) {
+            const int j = col_idx[p];
+            const int id = map[base + (j >> 7)];
+            if (id >= 0) {
+                const int c = j & 127;
+                atomicOr(&bits[((int64_t)id * kTileM + row_in_tile) * 4 + (c >> 5)], 1u << (c & 31));
+            } else {
+                ++res;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) res += __shfl_xor_sync(0xffffffffu, res, off);
+        if (lane == 0) res_cnt[r] = res;
+    }
+}
+
+// One warp per row: copy the residual entries (ascending) and count the rows
+// that mix tensor-core tiles and residual entries.
+__global__ void k_residual_fill(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
+                                int n, int64_t rows, int nqb, int nkt, const int32_t* __restrict__ map,
+                                const int32_t* __restrict__ block_tile_off,
+                                const int32_t* __restrict__ res_row_ptr, int32_t* __restrict__ res_col,
+                                int32_t* __restrict__ n_mixed) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t r = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+         r += warps) {
+        const int64_t m = r / n, i = r - m * n;
+        const int64_t blk = m * nqb + (i >> 7);
+        const int64_t base = blk * nkt;
+        int64_t o = res_row_ptr[r];
+        const int64_t p1 = row_ptr[r + 1];
+        for (int64_t c0 = row_ptr[r]; c0 < p1; c0 += 32) {
+            const int64_t p = c0 + lane;
+            int j = -1;
+            bool keep = false;
+            if (p < p1) {
+                j = col_idx[p];
+                keep = map[base + (j >> 7)] < 0;
+            }
+            const unsigned bal = __ballot_sync(0xffffffffu, keep);
+            if (keep) res_col[o + __popc(bal & ((1u << lane) - 1u))] = j;
+            o += __popc(bal);
+        }
+        if (lane == 0 && block_tile_off[blk + 1] > block_tile_off[blk] &&
+            res_row_ptr[r + 1] > res_row_ptr[r])
+            atomicAdd(n_mixed, 1);
+    }
+}
+
+unsigned grid_for(int64_t work, int per_block, int64_t cap = 1 << 16) {
+    int64_t g = (work + per_block - 1) / per_block;
+    if (g < 1) g = 1;
+    if (g > cap) g = cap;
+    return (unsigned)g;
+}
+
+}  // namespace
+
+int64_t plan_tile_capacity(int64_t nblocks, int nkt, int64_t nnz, int min_nnz) {
+    const int64_t by_grid = nblocks * nkt;
+    const int64_t by_nnz = nnz / (min_nnz > 0 ? min_nnz : 1) + 1;
+    return by_grid < by_nnz ? by_grid : by_nnz;
+}
+
+cudaError_t build_plan(const int32_t* row_ptr, const int32_t* col_idx, int n, int num_masks,
+                       int64_t nnz, int min_nnz, const PlanBuffers& b, PlanCounters* counters,
+                       cudaStream_t s) {
+    const int64_t rows = (int64_t)num_masks * n;
+    const int nqb = (n + kTileM - 1) / kTileM, nkt = (n + kTileN - 1) / kTileN;
+    const int64_t nblocks = (int64_t)num_masks * nqb;
+    cudaError_t e;
+    if ((e = cudaMemsetAsync(b.cnt_map, 0, sizeof(int32_t) * nblocks * nkt, s)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(b.tile_bits, 0, sizeof(uint32_t) * b.tile_cap * kTileM * 4, s)) != cudaSuccess)
+        return e;
+    k_tile_count<<<grid_for(rows, 8), 256, 0, s>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_tile_select<<<grid_for(nblocks, 128), 128, 0, s>>>(b.cnt_map, nblocks, nkt, min_nnz, b.block_ntiles,
+                                                        &counters->n_tc_blocks);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = scan_counts(b.block_ntiles, nblocks, b.block_tile_off, b.scan_tmp, &counters->n_tiles,
+                    &counters->err, s);
+    if (e != cudaSuccess) return e;
+    k_tile_assign<<<grid_for(nblocks, 128), 128, 0, s>>>(b.cnt_map, nblocks, nkt, min_nnz,
+                                                        b.block_tile_off, b.tile_info);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_tile_bits<<<grid_for(rows, 8), 256, 0, s>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map,
+                                                 b.tile_bits, b.res_cnt);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = scan_counts(b.res_cnt, rows, b.res_row_ptr, b.scan_tmp, &counters->res_nnz, &counters->err, s);
+    if (e != cudaSuccess) return e;
+    k_residual_fill<<<grid_for(rows, 8), 256, 0, s>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map,
+                                                     b.block_tile_off, b.res_row_ptr, b.res_col_idx,
+                                                     &counters->n_mixed);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return launch_classify_long_rows(b.res_row_ptr, rows, nnz, b.res_long, &counters->res_n_long, s);
+}
+
+}  // namespace spattn

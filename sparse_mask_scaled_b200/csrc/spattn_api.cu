@@ -25,6 +25,16 @@ struct spattn_mask_s {
     int32_t* col_idx;
     int32_t* long_rows;
     int64_t n_long;
+    // tile plan (tensor-core tiles + residual CSR); has_plan = false when no tile qualifies
+    bool has_plan;
+    int32_t nqb;
+    int64_t n_tiles, res_nnz, n_mixed, n_tc_blocks, res_n_long;
+    int32_t* block_tile_off;
+    int32_t* tile_info;
+    uint32_t* tile_bits;
+    int32_t* res_row_ptr;
+    int32_t* res_col_idx;
+    int32_t* res_long;
 };
 
 namespace {
@@ -197,6 +207,19 @@ int launch_fwd(FwdParams& p, int dtype, int d, int num_sms, cudaStream_t s) {
     return SPATTN_OK;
 }
 
+void free_plan(spattn_mask m) {
+    int32_t** ptrs[] = {&m->block_tile_off, &m->tile_info, &m->res_row_ptr, &m->res_col_idx, &m->res_long};
+    for (int32_t** p : ptrs) {
+        if (*p) cudaFreeAsync(*p, m->stream);
+        *p = nullptr;
+    }
+    if (m->tile_bits) cudaFreeAsync(m->tile_bits, m->stream);
+    m->tile_bits = nullptr;
+    m->has_plan = false;
+}
+
+unsigned* g_err_ptr[kMaxDevices];
+
 int build_status(unsigned err) {
     if (err & (kBuildTooMany | kBuildRowTooLong)) {
         return fail(SPATTN_ERR_UNSUPPORTED, "%s",
@@ -237,6 +260,7 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
     if (sp.kind == SPATTN_MASK_BLOCK_STRIDED_GLOBAL &&
         (sp.block < 0 || sp.stride < 0 || sp.n_global < 0))
         return fail(SPATTN_ERR_INVALID_ARG, "block, stride and n_global must be >= 0");
+    if (sp.reserved != 0) return fail(SPATTN_ERR_INVALID_ARG, "spec.reserved must be 0");
     if (sp.kind == SPATTN_MASK_CSR || sp.kind == SPATTN_MASK_COO) {
         if (!sp.in_row_ptr) return fail(SPATTN_ERR_INVALID_ARG, "in_row_ptr is NULL");
         if (sp.in_nnz < 0 || sp.in_nnz > 0x7fffffff)
@@ -312,15 +336,102 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
     if (e == cudaSuccess) e = cudaMemsetAsync(&info->n_long, 0, sizeof(int32_t), s);
     if (e == cudaSuccess)
         e = launch_classify_long_rows(row_ptr, rows, hinfo.nnz, m->long_rows, &info->n_long, s);
+
+    // tile plan: tensor-core tiles, their bit masks and the residual CSR
+    const int min_nnz = sp.tile_min_nnz == 0 ? kTileMinNnzDefault : sp.tile_min_nnz;
+    const int nqb = (sp.n + kTileM - 1) / kTileM, nkt = (sp.n + kTileN - 1) / kTileN;
+    const int64_t nblocks = (int64_t)sp.num_masks * nqb;
+    const bool plan = sp.tile_min_nnz >= 0 && hinfo.nnz > 0 && nblocks * nkt <= kPlanMaxTileGrid;
+    PlanBuffers pb;
+    memset(&pb, 0, sizeof pb);
+    PlanCounters* pc = nullptr;
+    PlanCounters hpc;
+    memset(&hpc, 0, sizeof hpc);
+    if (plan && e == cudaSuccess) {
+        m->nqb = nqb;
+        pb.tile_cap = plan_tile_capacity(nblocks, nkt, hinfo.nnz, min_nnz);
+        const int64_t scan_rows = rows > nblocks ? rows : nblocks;
+        if (e == cudaSuccess) e = pool_alloc(&pc, 1, pool, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(pc, 0, sizeof(PlanCounters), s);
+        if (e == cudaSuccess) e = pool_alloc(&pb.cnt_map, nblocks * nkt, pool, s);
+        if (e == cudaSuccess) e = pool_alloc(&pb.block_ntiles, nblocks, pool, s);
+        if (e == cudaSuccess) e = pool_alloc(&pb.scan_tmp, scan_tmp_elems(scan_rows), pool, s);
+        if (e == cudaSuccess) e = pool_alloc(&pb.res_cnt, rows, pool, s);
+        if (e == cudaSuccess) e = pool_alloc(&m->block_tile_off, nblocks + 1, pool, s);
+        if (e == cudaSuccess) e = pool_alloc(&m->tile_info, pb.tile_cap, pool, s);
+        if (e == cudaSuccess) e = pool_alloc(&m->tile_bits, pb.tile_cap * kTileM * 4, pool, s);
+        if (e == cudaSuccess) e = pool_alloc(&m->res_row_ptr, rows + 1, pool, s);
+        if (e == cudaSuccess) e = pool_alloc(&m->res_col_idx, hinfo.nnz, pool, s);
+        if (e == cudaSuccess) e = pool_alloc(&m->res_long, rows, pool, s);
+        pb.block_tile_off = m->block_tile_off;
+        pb.tile_info = m->tile_info;
+        pb.tile_bits = m->tile_bits;
+        pb.res_row_ptr = m->res_row_ptr;
+        pb.res_col_idx = m->res_col_idx;
+        pb.res_long = m->res_long;
+        if (e == cudaSuccess)
+            e = build_plan(row_ptr, m->col_idx, sp.n, sp.num_masks, hinfo.nnz, min_nnz, pb, pc, s);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(&hpc, pc, sizeof hpc, cudaMemcpyDeviceToHost, s);
+    }
     if (e == cudaSuccess) e = cudaMemcpyAsync(&hinfo, info, sizeof hinfo, cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     release_tmp();
+    if (pc) cudaFreeAsync(pc, s);
+    if (pb.cnt_map) cudaFreeAsync(pb.cnt_map, s);
+    if (pb.block_ntiles) cudaFreeAsync(pb.block_ntiles, s);
+    if (pb.scan_tmp) cudaFreeAsync(pb.scan_tmp, s);
+    if (pb.res_cnt) cudaFreeAsync(pb.res_cnt, s);
     if (e != cudaSuccess) {
         spattn_destroy_mask(m);
         return cuda_fail(e, "mask build (phase 2)");
     }
     m->n_long = hinfo.n_long;
+    if (plan) {
+        m->n_tiles = hpc.n_tiles;
+        m->res_nnz = hpc.res_nnz;
+        m->n_mixed = hpc.n_mixed;
+        m->n_tc_blocks = hpc.n_tc_blocks;
+        m->res_n_long = hpc.res_n_long;
+        m->has_plan = hpc.n_tiles > 0;
+        if (!m->has_plan) free_plan(m);
+    }
     *out = m;
+    return SPATTN_OK;
+}
+
+int spattn_mask_copy_plan(spattn_mask m, int32_t* block_tile_off, int32_t* tile_info,
+                          uint32_t* tile_bits, int32_t* res_row_ptr, int32_t* res_col_idx,
+                          void* stream_v) {
+    g_msg[0] = 0;
+    if (!m) return fail(SPATTN_ERR_INVALID_ARG, "mask is NULL");
+    if (!m->has_plan) return fail(SPATTN_ERR_INVALID_ARG, "the mask has no tile plan");
+    cudaStream_t s = (cudaStream_t)stream_v;
+    const int64_t rows = (int64_t)m->n * m->num_masks;
+    const int64_t nblocks = (int64_t)m->num_masks * m->nqb;
+    struct Item {
+        void* dst;
+        const void* src;
+        size_t bytes;
+    } items[] = {
+        {block_tile_off, m->block_tile_off, (size_t)(nblocks + 1) * 4},
+        {tile_info, m->tile_info, (size_t)m->n_tiles * 4},
+        {tile_bits, m->tile_bits, (size_t)m->n_tiles * kTileM * 4 * 4},
+        {res_row_ptr, m->res_row_ptr, (size_t)(rows + 1) * 4},
+        {res_col_idx, m->res_col_idx, (size_t)m->res_nnz * 4},
+    };
+    for (const Item& it : items)
+        if (it.dst && it.bytes)
+            CUDA_TRY(cudaMemcpyAsync(it.dst, it.src, it.bytes, cudaMemcpyDefault, s), "plan copy");
+    return SPATTN_OK;
+}
+
+int spattn_mask_plan_info(spattn_mask m, int64_t* n_tiles, int64_t* residual_nnz,
+                          int64_t* n_mixed_rows) {
+    g_msg[0] = 0;
+    if (!m) return fail(SPATTN_ERR_INVALID_ARG, "mask is NULL");
+    if (n_tiles) *n_tiles = m->has_plan ? m->n_tiles : 0;
+    if (residual_nnz) *residual_nnz = m->has_plan ? m->res_nnz : m->nnz;
+    if (n_mixed_rows) *n_mixed_rows = m->has_plan ? m->n_mixed : 0;
     return SPATTN_OK;
 }
 
@@ -364,6 +475,7 @@ int spattn_destroy_mask(spattn_mask m) {
     if (m->row_ptr && (e2 = cudaFreeAsync(m->row_ptr, m->stream)) != cudaSuccess) e = e2;
     if (m->col_idx && (e2 = cudaFreeAsync(m->col_idx, m->stream)) != cudaSuccess) e = e2;
     if (m->long_rows && (e2 = cudaFreeAsync(m->long_rows, m->stream)) != cudaSuccess) e = e2;
+    free_plan(m);
     if (prev >= 0 && prev != m->device) cudaSetDevice(prev);
     delete m;
     if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync");
@@ -433,13 +545,72 @@ int spattn_fwd_mask(const spattn_tensor* q, const spattn_tensor* k, const spattn
     cudaMemPool_t pool;
     CUDA_TRY(device_state(dev, &pool, &sms), "memory pool");
     p.num_masks = mask->num_masks;
-    p.row_ptr = mask->row_ptr;
-    p.col_idx = mask->col_idx;
-    p.nnz = mask->nnz;
-    p.long_rows = mask->long_rows;
     p.long_count_dev = nullptr;
-    p.long_count_host = mask->n_long;
-    return launch_fwd(p, dtype, d, sms, s);
+    if (!(mask->has_plan && dtype == 0)) {  // every entry on the gather kernel
+        p.row_ptr = mask->row_ptr;
+        p.col_idx = mask->col_idx;
+        p.nnz = mask->nnz;
+        p.long_rows = mask->long_rows;
+        p.long_count_host = mask->n_long;
+        return launch_fwd(p, dtype, d, sms, s);
+    }
+    // tile plan: residual entries on the gather kernel, tiles on tensor cores
+    p.row_ptr = mask->res_row_ptr;
+    p.col_idx = mask->res_col_idx;
+    p.nnz = mask->res_nnz;
+    p.long_rows = mask->res_long;
+    p.long_count_host = mask->res_n_long;
+    p.qb_tile_off = mask->block_tile_off;
+    p.nqb = mask->nqb;
+    float* ws = nullptr;
+    const int64_t rows_all = (int64_t)p.B * p.H * p.n;
+    if (mask->n_mixed > 0) {
+        CUDA_TRY(pool_alloc(&ws, rows_all * (d + 2), pool, s), "partial-state workspace");
+        p.ws_ml = ws;
+        p.ws_acc = ws + rows_all * 2;
+    }
+    const int64_t nblocks = (int64_t)mask->num_masks * mask->nqb;
+    if (mask->res_nnz > 0 || mask->n_tc_blocks < nblocks) {
+        r = launch_fwd(p, dtype, d, sms, s);
+        if (r) {
+            if (ws) cudaFreeAsync(ws, s);
+            return r;
+        }
+    }
+    if (!g_err_ptr[dev]) {
+        unsigned* ep = nullptr;
+        CUDA_TRY(error_flag_address(&ep), "error flag address");
+        g_err_ptr[dev] = ep;
+    }
+    TcParams tp;
+    memset(&tp, 0, sizeof tp);
+    tp.B = p.B;
+    tp.H = p.H;
+    tp.n = p.n;
+    tp.num_masks = mask->num_masks;
+    tp.nqb = mask->nqb;
+    tp.block_tile_off = mask->block_tile_off;
+    tp.tile_info = mask->tile_info;
+    tp.tile_bits = mask->tile_bits;
+    tp.res_row_ptr = mask->res_row_ptr;
+    tp.ws_ml = p.ws_ml;
+    tp.ws_acc = p.ws_acc;
+    tp.out = p.out;
+    tp.o_sb = p.o_sb;
+    tp.o_sh = p.o_sh;
+    tp.o_sn = p.o_sn;
+    tp.lse = p.lse;
+    tp.mask = p.mask;
+    tp.bias = p.bias;
+    tp.has_extra = p.has_extra;
+    tp.qk_scale_log2 = p.qk_scale_log2;
+    tp.err = g_err_ptr[dev];
+    const TcOperand oq{p.q, p.q_sn, p.q_sh, p.q_sb}, ok{p.k, p.k_sn, p.k_sh, p.k_sb},
+        ov{p.v, p.v_sn, p.v_sh, p.v_sb};
+    cudaError_t e = launch_fwd_tc(oq, ok, ov, d, tp, s);
+    if (ws) cudaFreeAsync(ws, s);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core kernel launch");
+    return SPATTN_OK;
 }
 
 // ---- allocation-free forward: its scratch is this fixed array, part of the
@@ -516,6 +687,7 @@ int spattn_device_error(void* stream_v, uint32_t* flags) {
     cudaError_t e = read_and_clear_device_error(&v, (cudaStream_t)stream_v);
     if (flags) *flags = v;
     if (e != cudaSuccess) return cuda_fail(e, "reading the device error flag");
+    if (v & kErrTimeout) return fail(SPATTN_ERR_TIMEOUT, "a bounded wait in the tensor-core kernel expired");
     if (v & kErrBadColumn) return fail(SPATTN_ERR_BAD_CSR, "a column index outside [0, n) was skipped");
     return SPATTN_OK;
 }

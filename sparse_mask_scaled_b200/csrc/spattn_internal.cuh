@@ -12,6 +12,15 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 // device error flag bits (read by spattn_device_error)
 constexpr unsigned kErrBadColumn = 1u;
+constexpr unsigned kErrTimeout = 2u;  // a bounded wait of the tensor-core kernel expired
+
+// Tensor-core tiling: 128 query rows by 128 keys.
+constexpr int kTileM = 128;
+constexpr int kTileN = 128;
+constexpr unsigned kTileDenseBit = 0x80000000u;  // tile_info flag: all 128 x 128 entries present
+constexpr int kTileMinNnzDefault = 256;
+// Tile planning is skipped when num_masks * (n/128)^2 exceeds this (count array size).
+constexpr int64_t kPlanMaxTileGrid = int64_t(1) << 26;
 
 // Rows with more nonzeros than this are processed by a whole thread block
 // (eight warps) instead of one warp.
@@ -46,7 +55,66 @@ struct FwdParams {
     const int32_t* long_rows;
     const int32_t* long_count_dev;  // device count (used when long_count_host < 0)
     int64_t long_count_host;        // host count, or -1
+    // With a tensor-core plan: rows of query blocks that have tensor-core tiles
+    // write their partial state (m in base 2, l, unnormalised acc) to ws_ml /
+    // ws_acc instead of the output (only when they have gathered entries).
+    const int32_t* qb_tile_off;  // [num_masks * nqb + 1] or nullptr
+    int nqb;
+    float* ws_ml;   // [B*H*n*2]
+    float* ws_acc;  // [B*H*n*d]
 };
+
+// Tensor-core kernel (fwd_tc.cu).
+struct TcOperand {
+    const void* data;  // bf16 [B, H, n, d], stride 1 over d
+    int64_t s_n, s_h, s_b;
+};
+struct TcParams {
+    int B, H, n, num_masks, nqb;
+    const int32_t* block_tile_off;  // [num_masks * nqb + 1]
+    const int32_t* tile_info;       // key tile | kTileDenseBit
+    const uint32_t* tile_bits;      // [tiles][128 rows][4 words]
+    const int32_t* res_row_ptr;     // residual CSR (a row with entries has a partial)
+    const float* ws_ml;             // partials from the gather kernel, or nullptr
+    const float* ws_acc;
+    void* out;
+    int64_t o_sb, o_sh, o_sn;
+    float* lse;
+    AddendView mask, bias;
+    int has_extra;
+    float qk_scale_log2;
+    unsigned* err;
+};
+cudaError_t launch_fwd_tc(const TcOperand& q, const TcOperand& k, const TcOperand& v, int d,
+                          const TcParams& p, cudaStream_t stream);
+cudaError_t error_flag_address(unsigned** p);
+
+// Tile plan (plan.cu).
+struct PlanBuffers {
+    int32_t* cnt_map;         // [nblocks * nkt] (temporary)
+    int32_t* block_ntiles;    // [nblocks] (temporary)
+    int32_t* block_tile_off;  // [nblocks + 1]
+    int64_t* scan_tmp;        // [scan_tmp_elems(max(rows, nblocks))] (temporary)
+    int32_t* tile_info;       // [tile_cap]
+    uint32_t* tile_bits;      // [tile_cap * 128 * 4]
+    int64_t tile_cap;
+    int32_t* res_cnt;         // [rows] (temporary)
+    int32_t* res_row_ptr;     // [rows + 1]
+    int32_t* res_col_idx;     // [nnz]
+    int32_t* res_long;        // [rows]
+};
+struct PlanCounters {  // device-side results
+    int64_t n_tiles;
+    int64_t res_nnz;
+    int32_t n_mixed;      // rows with entries on both paths
+    int32_t res_n_long;   // long rows of the residual CSR
+    int32_t n_tc_blocks;  // query blocks with at least one tile
+    unsigned err;
+};
+int64_t plan_tile_capacity(int64_t nblocks, int nkt, int64_t nnz, int min_nnz);
+cudaError_t build_plan(const int32_t* row_ptr, const int32_t* col_idx, int n, int num_masks,
+                       int64_t nnz, int min_nnz, const PlanBuffers& b, PlanCounters* counters,
+                       cudaStream_t s);
 
 // ---------------------------------------------------------------- launchers
 // All launchers enqueue on `stream` and return the cudaGetLastError() result.
@@ -99,6 +167,11 @@ cudaError_t build_phase1(const BuildSpec& s, int32_t* row_ptr, int32_t* counts,
                          int64_t* scan_tmp, int32_t* coo_tmp, BuildInfo* info,
                          cudaStream_t stream);
 int64_t scan_tmp_elems(int64_t rows);
+// Exclusive scan of int32 counts [rows] into out int32 [rows + 1]; the total goes
+// to *total (device) and overflow past INT32_MAX sets kBuildTooMany in *err.
+// scan_tmp: int64 [scan_tmp_elems(rows)].
+cudaError_t scan_counts(const int32_t* counts, int64_t rows, int32_t* out, int64_t* scan_tmp,
+                        int64_t* total, unsigned* err, cudaStream_t stream);
 // Phase 2: write col_idx from the pattern (or copy it from coo_tmp / in_col_idx).
 cudaError_t build_phase2(const BuildSpec& s, const int32_t* row_ptr, const int32_t* coo_tmp,
                          int32_t* col_idx, cudaStream_t stream);

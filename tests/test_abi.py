@@ -39,7 +39,8 @@ def test_python_binding_covers_every_symbol():
     names = _declared_functions()
     assert set(names) == set(sp.SIGNATURES)
     for n in names:
-        if n in ("spattn_mask_info", "spattn_mask_copy_csr", "spattn_destroy_mask"):
+        if n in ("spattn_mask_info", "spattn_mask_copy_csr", "spattn_destroy_mask",
+                 "spattn_mask_plan_info", "spattn_mask_copy_plan"):
             continue        # reached through sp.Mask
         assert callable(getattr(sp, n)), n
 
@@ -48,9 +49,10 @@ def test_struct_layouts_match_the_header():
     # spattn_tensor: pointer, 2 x int32, 4 x int64, 4 x int64
     assert ctypes.sizeof(sp.spattn_tensor) == 8 + 8 + 32 + 32
     assert sp.spattn_tensor.shape.offset == 16
-    # spattn_mask_spec: 8 x int32, 3 pointers, int64
-    assert ctypes.sizeof(sp.spattn_mask_spec) == 32 + 24 + 8
+    # spattn_mask_spec: 8 x int32, 3 pointers, int64, 2 x int32
+    assert ctypes.sizeof(sp.spattn_mask_spec) == 32 + 24 + 8 + 8
     assert sp.spattn_mask_spec.half_widths.offset == 32
+    assert sp.spattn_mask_spec.tile_min_nnz.offset == 64
 
 
 def test_version():
