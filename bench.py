@@ -277,6 +277,8 @@ def bench_ours(args, rank, world, torch, sp):
     with g.create() as m0:
         nnz_masks = m0.nnz
         n_long = m0.n_long
+        plan = {"tensor_core_tiles": m0.n_tiles, "residual_nnz": m0.residual_nnz,
+                "mixed_rows": m0.n_mixed_rows}
     # nnz summed over (b, h): every head shares its batch element's mask
     if wl.mask.num_masks == 1:
         nnz_total = nnz_masks * wl.B * wl.H
@@ -353,7 +355,8 @@ def bench_ours(args, rank, world, torch, sp):
                    "nnz_total": nnz_total, "flop_per_step": flops,
                    "l2": "flushed before every timed step (256 MiB write)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "step": "device mask build (pattern -> CSR -> row schedule) + fused forward"},
+                   "step": "device mask build (pattern -> CSR -> row schedule + tile plan) + fused forward",
+                   "plan_per_mask_set": plan},
         "fwd": {"ms": round(t_fwd, 4), "tflops": round(flops / (t_fwd * 1e-3) / 1e12, 3),
                 "effective_gbs": round(achieved, 1)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
@@ -450,8 +453,9 @@ def other_workloads(torch, sp, skip):
                 torch.cuda.synchronize()
                 build_ms = (time.perf_counter() - tb) * 1e3
                 m2.close()
+                plan = {"tiles": m.n_tiles, "residual_nnz": m.residual_nnz, "mixed_rows": m.n_mixed_rows}
             alg, _ = algorithmic_bytes(wl, nnz_total)
-            res[wl.name] = {"fwd_ms": round(t, 4), "tflops": round(4.0 * nnz_total * wl.d / (t * 1e-3) / 1e12, 3),
+            res[wl.name] = {"plan": plan, "fwd_ms": round(t, 4), "tflops": round(4.0 * nnz_total * wl.d / (t * 1e-3) / 1e12, 3),
                             "effective_gbs": round(alg / (t * 1e-3) / 1e9, 1),
                             "frac_hbm": round(alg / (t * 1e-3) / 1e9 / hbm_peak, 4),
                             "nnz_total": nnz_total, "mask_build_wall_ms": round(build_ms, 3)}

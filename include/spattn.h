@@ -110,7 +110,7 @@ typedef struct {
     int64_t in_nnz;             /* CSR, COO: in_row_ptr[num_masks * n] */
     int32_t tile_min_nnz;       /* tensor-core tiles: a 128 x 128 tile with at least this many
                                    nonzeros is computed on tensor cores (bf16 inputs);
-                                   0 = default (256), < 0 = never */
+                                   0 = default (512), < 0 = never */
     int32_t reserved;           /* must be 0 */
 } spattn_mask_spec;
 
@@ -156,7 +156,7 @@ int spattn_mask_plan_info(spattn_mask mask, int64_t* n_tiles, int64_t* residual_
  * tile ids block_tile_off[x] .. block_tile_off[x+1]-1), tile_info int32 [n_tiles]
  * (key tile index, bit 31 set when all 128 x 128 entries are present),
  * tile_bits uint32 [n_tiles * 128 * 4] (row r of a tile: 4 words, bit c of word
- * c/32 = column c), residual row_ptr int32 [num_masks * n + 1] and col_idx
+ * c/32 = column c; left zero for dense tiles, whose entries are all present), residual row_ptr int32 [num_masks * n + 1] and col_idx
  * int32 [residual_nnz]. Returns SPATTN_ERR_INVALID_ARG when the mask has no
  * tile plan. Stream-ordered on `stream`. */
 int spattn_mask_copy_plan(spattn_mask mask, int32_t* block_tile_off, int32_t* tile_info,

@@ -45,6 +45,39 @@ __device__ __forceinline__ float lg2(float x) {
     return y;
 }
 
+// Two fp32 lanes per instruction (fma.rn.f32x2 / add.f32x2 / mul.f32x2).
+__device__ __forceinline__ uint64_t pack2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t r, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// (x0, x1) = (s0, s1) * c2 + (x0, x1), s given as raw fp32 bits
+__device__ __forceinline__ void fma2_inplace(float& x0, float& x1, uint32_t s0, uint32_t s1, uint64_t c2) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(d)
+        : "l"(pack2(__uint_as_float(s0), __uint_as_float(s1))), "l"(c2), "l"(pack2(x0, x1)));
+    unpack2(d, x0, x1);
+}
+__device__ __forceinline__ void mul2(float& x0, float& x1, uint32_t s0, uint32_t s1, uint64_t c2) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pack2(__uint_as_float(s0), __uint_as_float(s1))), "l"(c2));
+    unpack2(d, x0, x1);
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // Makes every use of r[] depend on the TMEM load having completed.
 __device__ __forceinline__ void tmem_wait_ld_dep(uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;"
@@ -77,19 +110,20 @@ struct TcCfg {
     static constexpr int OFF_BAR = OFF_P + P_BYTES;  // 5 mbarriers + tmem slot + abort flag
     // At least 100 KB so that no more than two CTAs (2 x 256 TMEM columns) share
     // an SM and tcgen05.alloc never has to wait; d = 64 fits two CTAs per SM.
-    static constexpr int SMEM_BYTES = OFF_BAR + 64 > 100 * 1024 ? OFF_BAR + 64 : 100 * 1024;
+    static constexpr int SMEM_BYTES = OFF_BAR + 128 > 100 * 1024 ? OFF_BAR + 128 : 100 * 1024;
     static_assert(D == 32 || D == 64 || D == 128, "head dim");
 };
 
-// Adds log2(e) * addend[b, h, i, jj0 + j] to x[j] for j < ncols.
-__device__ __forceinline__ void add_addend_row(const AddendView& a, int64_t rowbase, int jj0,
-                                               int ncols, float (&x)[128]) {
-    const int64_t off0 = rowbase + (int64_t)jj0 * a.s3;
-    if (a.dtype == 0 && a.s3 == 1 && ncols == 128 &&
+// Adds log2(e) * addend[b, h, i, c0 + j] to x[j] for j < ncols (an N-column run).
+template <int N>
+__device__ __forceinline__ void add_addend_run(const AddendView& a, int64_t rowbase, int c0, int ncols,
+                                               float (&x)[N]) {
+    const int64_t off0 = rowbase + (int64_t)c0 * a.s3;
+    if (a.dtype == 0 && a.s3 == 1 && ncols == N &&
         ((reinterpret_cast<uintptr_t>(a.data) + (uintptr_t)off0 * 2) & 15) == 0) {
         const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.data) + off0);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
+        for (int c = 0; c < N / 8; ++c) {
             const uint4 w = __ldg(p + c);
             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -101,7 +135,7 @@ __device__ __forceinline__ void add_addend_row(const AddendView& a, int64_t rowb
         return;
     }
 #pragma unroll
-    for (int j = 0; j < 128; ++j) {
+    for (int j = 0; j < N; ++j) {
         if (j < ncols) {
             const int64_t off = off0 + (int64_t)j * a.s3;
             const float v = a.dtype == 0
@@ -228,58 +262,85 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t bias_rowbase = (int64_t)b * P.bias.s0 + (int64_t)h * P.bias.s1 + (int64_t)i * P.bias.s2;
     float m_ref = -INFINITY, l = 0.f;
 
+    // tile u's info and row bits are loaded one tile ahead
+    int next_info = P.tile_info[t_begin];
+    uint4 next_bits = make_uint4(0u, 0u, 0u, 0u);
+    if (next_info >= 0 && row_ok)
+        next_bits = __ldg(reinterpret_cast<const uint4*>(P.tile_bits) + ((int64_t)t_begin * 128 + row));
+    const uint64_t c2 = pack2(P.qk_scale_log2, P.qk_scale_log2);
+
     for (int u = 0; u < T; ++u) {
-        const int info = P.tile_info[t_begin + u];
+        const int info = next_info;
+        const uint4 wbits = next_bits;
+        if (u + 1 < T) {
+            next_info = P.tile_info[t_begin + u + 1];
+            if (next_info >= 0 && row_ok)
+                next_bits = __ldg(reinterpret_cast<const uint4*>(P.tile_bits) +
+                                  ((int64_t)(t_begin + u + 1) * 128 + row));
+        }
         const int kt = info & 0x7fffffff;
-        const bool dense = info < 0;
-        uint32_t bits[4] = {0u, 0u, 0u, 0u};
-        if (dense) {
-            bits[0] = bits[1] = bits[2] = bits[3] = 0xffffffffu;
-        } else if (row_ok) {
-            const uint4 w = __ldg(reinterpret_cast<const uint4*>(P.tile_bits) + ((int64_t)(t_begin + u) * 128 + row));
-            bits[0] = w.x;
-            bits[1] = w.y;
-            bits[2] = w.z;
-            bits[3] = w.w;
-        }
-        float x[128];
-#pragma unroll
-        for (int j = 0; j < 128; ++j) x[j] = 0.f;
+        const bool dense = info < 0;  // the same for the whole CTA
+        const bool extra = P.has_extra && row_ok;
         const int jj0 = kt * 128;
-        const int ncols = P.n - jj0 < 128 ? P.n - jj0 : 128;
-        if (P.has_extra && row_ok) {
-            if (P.mask.data) add_addend_row(P.mask, mask_rowbase, jj0, ncols, x);
-            if (P.bias.data) add_addend_row(P.bias, bias_rowbase, jj0, ncols, x);
-        }
+        const uint32_t bw[4] = {wbits.x, wbits.y, wbits.z, wbits.w};
 
         wait(barS, (uint32_t)(u & 1));
         tc_fence_after();
         __syncwarp();
-        {
-            uint32_t r0[32], r1[32], r2[32], r3[32];
-            tmem_ld32(tS + lane_base + 0, r0);
-            tmem_ld32(tS + lane_base + 32, r1);
-            tmem_ld32(tS + lane_base + 64, r2);
-            tmem_ld32(tS + lane_base + 96, r3);
+        // pass 1, 64 columns at a time: x = scale*log2(e)*S (+ log2(e)*(mask + bias)),
+        // entries the CSR does not list -> -inf, row max; x goes back into TMEM
+        float ma = -INFINITY, mb = -INFINITY, mc = -INFINITY, md = -INFINITY;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float xh[64];
+            if (extra) {
+#pragma unroll
+                for (int j = 0; j < 64; ++j) xh[j] = 0.f;
+                const int c0 = jj0 + half * 64;
+                const int ncols = P.n - c0 < 64 ? P.n - c0 : 64;
+                if (P.mask.data) add_addend_run<64>(P.mask, mask_rowbase, c0, ncols, xh);
+                if (P.bias.data) add_addend_run<64>(P.bias, bias_rowbase, c0, ncols, xh);
+            }
+            uint32_t r0[32], r1[32];
+            tmem_ld32(tS + lane_base + half * 64, r0);
+            tmem_ld32(tS + lane_base + half * 64 + 32, r1);
             tmem_wait_ld_dep(r0);
             tmem_wait_ld_dep(r1);
-            tmem_wait_ld_dep(r2);
-            tmem_wait_ld_dep(r3);
+            if (extra) {
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    fma2_inplace(xh[2 * k], xh[2 * k + 1], r0[2 * k], r0[2 * k + 1], c2);
+                    fma2_inplace(xh[32 + 2 * k], xh[33 + 2 * k], r1[2 * k], r1[2 * k + 1], c2);
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    mul2(xh[2 * k], xh[2 * k + 1], r0[2 * k], r0[2 * k + 1], c2);
+                    mul2(xh[32 + 2 * k], xh[33 + 2 * k], r1[2 * k], r1[2 * k + 1], c2);
+                }
+            }
+            if (!dense) {
+#pragma unroll
+                for (int j = 0; j < 64; ++j)
+                    xh[j] = ((bw[half * 2 + (j >> 5)] >> (j & 31)) & 1u) ? xh[j] : -INFINITY;
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                ma = fmax3(ma, xh[8 * k + 0], xh[8 * k + 1]);
+                mb = fmax3(mb, xh[8 * k + 2], xh[8 * k + 3]);
+                mc = fmax3(mc, xh[8 * k + 4], xh[8 * k + 5]);
+                md = fmax3(md, xh[8 * k + 6], xh[8 * k + 7]);
+            }
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                x[j] = fmaf(__uint_as_float(r0[j]), P.qk_scale_log2, x[j]);
-                x[32 + j] = fmaf(__uint_as_float(r1[j]), P.qk_scale_log2, x[32 + j]);
-                x[64 + j] = fmaf(__uint_as_float(r2[j]), P.qk_scale_log2, x[64 + j]);
-                x[96 + j] = fmaf(__uint_as_float(r3[j]), P.qk_scale_log2, x[96 + j]);
+                r0[j] = __float_as_uint(xh[j]);
+                r1[j] = __float_as_uint(xh[32 + j]);
             }
+            tmem_st32(tS + lane_base + half * 64, r0);
+            tmem_st32(tS + lane_base + half * 64 + 32, r1);
         }
-        float mx = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < 128; ++j) {
-            const bool on = (bits[j >> 5] >> (j & 31)) & 1u;
-            x[j] = on ? x[j] : -INFINITY;
-            mx = fmaxf(mx, x[j]);
-        }
+        tmem_wait_st();
+        const float mx = fmax3(ma, mb, fmaxf(mc, md));
         const bool need = mx > m_ref + kRescaleThreshold;
         float alpha = 1.f;
         if (need) {
@@ -288,47 +349,67 @@ __global__ void __launch_bounds__(kThreads, 1)
             l *= alpha;
         }
         const float mu = m_ref == -INFINITY ? 0.f : m_ref;
-        uint32_t pk[64];
-        float lsum = 0.f;
-#pragma unroll
-        for (int k = 0; k < 64; ++k) {
-            const float p0 = ex2(x[2 * k] - mu), p1 = ex2(x[2 * k + 1] - mu);
-            lsum += p0 + p1;
-            __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
-            pk[k] = *reinterpret_cast<uint32_t*>(&hv);
-        }
-        l += lsum;
+        const uint64_t nmu2 = pack2(-mu, -mu);
+        uint64_t sa = pack2(0.f, 0.f), sb = sa;  // two running pair sums
 
-        // P V of the previous tile must be done before sP is overwritten and O rescaled
-        if (u > 0) {
-            wait(barO, (uint32_t)((u - 1) & 1));
-            tc_fence_after();
-            if (tid == 0 && u + 1 < T && !*abort_flag) issue_kv(u + 1);  // its buffer is free now
-            __syncwarp();
-            if (__any_sync(0xffffffffu, need)) {
-#pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t ro[32];
-                    tmem_ld32(tO + lane_base + c * 32, ro);
-                    tmem_wait_ld_dep(ro);
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) ro[j] = __float_as_uint(__uint_as_float(ro[j]) * alpha);
-                    tmem_st32(tO + lane_base + c * 32, ro);
-                }
-                tmem_wait_st();
-            }
-        }
-        // P (bf16) into the K-major, 128-byte-swizzled A operand layout
+        // pass 2, per 64-key chunk: p = exp2(x - m), row sum, P (bf16) into the K-major,
+        // 128-byte-swizzled A operand layout of the P V MMA (chunk kc = keys 64kc ..)
 #pragma unroll
         for (int kc = 0; kc < 2; ++kc) {
+            uint32_t r0[32], r1[32];
+            tmem_ld32(tS + lane_base + kc * 64, r0);
+            tmem_ld32(tS + lane_base + kc * 64 + 32, r1);
+            tmem_wait_ld_dep(r0);
+            tmem_wait_ld_dep(r1);
+            uint32_t pk[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                const uint32_t w0 = k < 16 ? r0[2 * k] : r1[2 * k - 32];
+                const uint32_t w1 = k < 16 ? r0[2 * k + 1] : r1[2 * k - 31];
+                float p0, p1;
+                unpack2(add2(pack2(__uint_as_float(w0), __uint_as_float(w1)), nmu2), p0, p1);
+                p0 = ex2(p0);
+                p1 = ex2(p1);
+                if (k & 1)
+                    sb = add2(sb, pack2(p0, p1));
+                else
+                    sa = add2(sa, pack2(p0, p1));
+                __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
+                pk[k] = *reinterpret_cast<uint32_t*>(&hv);
+            }
+            if (kc == 0 && u > 0) {
+                // P V of the previous tile reads sP: it must be done before sP is overwritten
+
+                wait(barO, (uint32_t)((u - 1) & 1));
+                tc_fence_after();
+                if (tid == 0 && u + 1 < T && !*abort_flag) issue_kv(u + 1);  // its buffer is free now
+                __syncwarp();
+                if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t ro[32];
+                        tmem_ld32(tO + lane_base + c * 32, ro);
+                        tmem_wait_ld_dep(ro);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) ro[j] = __float_as_uint(__uint_as_float(ro[j]) * alpha);
+                        tmem_st32(tO + lane_base + c * 32, ro);
+                    }
+                    tmem_wait_st();
+                }
+            }
 #pragma unroll
             for (int piece = 0; piece < 8; ++piece) {
-                const int k = kc * 32 + piece * 4;
                 const uint32_t addr = sP + (uint32_t)(kc * 16384 + row * 128 + ((piece ^ (row & 7)) << 4));
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[k]),
-                             "r"(pk[k + 1]), "r"(pk[k + 2]), "r"(pk[k + 3])
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[piece * 4]),
+                             "r"(pk[piece * 4 + 1]), "r"(pk[piece * 4 + 2]), "r"(pk[piece * 4 + 3])
                              : "memory");
             }
+        }
+        {
+            float s0, s1, s2, s3;
+            unpack2(sa, s0, s1);
+            unpack2(sb, s2, s3);
+            l += (s0 + s1) + (s2 + s3);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -415,6 +496,392 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ----------------------------------------------------------------------------
+// Pipelined variant for d <= 64, two threads per query row (8 warps per CTA).
+// O accumulates in registers (each thread owns d/2 of its row's columns),
+// which frees TMEM for two S buffers (2 x 128 columns, two CTAs per SM). Thread
+// (half, row) handles keys 64*half .. 64*half + 63 of each tile. P V(u) is
+// written into S(u)'s buffer once softmax(u) has finished with it, and S(u+1)
+// is issued in the middle of softmax(u), so the tensor core computes the next
+// tile's scores while the threads exponentiate the current one:
+//   softmax(u): wait S(u) | pass 1 (scale, mask, partial max; x back to TMEM) |
+//               wait P V(u-1), add it to O | partial max out | sync ->
+//               issue S(u+1) | row max | pass 2 (exp2, sum, P to smem) |
+//               sync -> issue P V(u), K(u+2)
+// The partial maxima travel through the P buffer: thread (h, r) leaves its
+// value in row r of P chunk 1-h, which only its partner (1-h, r) reads and
+// later overwrites with its own P.
+constexpr int kPipeThreads = 256;
+
+template <int D, bool EXTRA>
+__global__ void __launch_bounds__(kPipeThreads, 2)
+    k_fwd_tc_pipe(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const TcParams P) {
+    using C = TcCfg<D>;
+    static_assert(D <= 64, "O is kept in registers");
+    constexpr int DH = D / 2;  // O columns per thread
+    extern __shared__ __align__(1024) uint8_t smem[];
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int half = warp >> 2;       // key half of each tile (and O column half)
+    const int row = tid & 127;        // query row in the block == TMEM lane
+    const int bh = blockIdx.x / P.nqb, qb = blockIdx.x - bh * P.nqb;
+    const int b = bh / P.H, h = bh - b * P.H;
+    const int mk = P.num_masks == 1 ? 0 : b;
+    const int64_t blk = (int64_t)mk * P.nqb + qb;
+    const int t_begin = P.block_tile_off[blk];
+    const int T = P.block_tile_off[blk + 1] - t_begin;
+    if (T <= 0) return;
+    if (smem_u32(smem) & 1023u) {
+        if (tid == 0) atomicOr(P.err, kErrTimeout);
+        return;
+    }
+
+    const uint32_t sQ = smem_u32(smem + C::OFF_Q);
+    const uint32_t sK0 = smem_u32(smem + C::OFF_K), sV0 = smem_u32(smem + C::OFF_V);
+    const uint32_t sP = smem_u32(smem + C::OFF_P);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    // barriers: Q, K[2], V[2], S[2], O
+    const uint32_t barQ = smem_u32(bars + 0), barK0 = smem_u32(bars + 1), barV0 = smem_u32(bars + 3),
+                   barS0 = smem_u32(bars + 5), barO = smem_u32(bars + 7);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    // partner exchange slot: row `row` of P chunk (1 - half), first 16 bytes (swizzled)
+    const uint32_t my_slot = sP + (uint32_t)((half ^ 1) * 16384 + row * 128 + ((0 ^ (row & 7)) << 4));
+    const uint32_t partner_slot = sP + (uint32_t)(half * 16384 + row * 128 + ((0 ^ (row & 7)) << 4));
+
+    if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    if (tid == 0) {
+        for (int x = 0; x < 8; ++x) mbar_init(smem_u32(bars + x), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+
+    // thread 0: issued operations per barrier (scalars: no dynamically indexed arrays)
+    int n_k0 = 0, n_k1 = 0, n_v0 = 0, n_v1 = 0, n_s0 = 0, n_s1 = 0, n_pv = 0;
+
+    auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+        if (*abort_flag) return false;
+        if (mbar_wait_bounded(bar, parity, kWaitCycles)) return true;
+        *abort_flag = 1;
+        return false;
+    };
+    auto tile_kt = [&](int u) { return P.tile_info[t_begin + u] & 0x7fffffff; };
+    auto issue_k = [&](int u) {
+        const uint32_t bar = barK0 + 8u * (u & 1);
+        mbar_expect_tx(bar, (uint32_t)C::TILE_BYTES);
+        tma_load_4d(sK0 + (uint32_t)((u & 1) * C::TILE_BYTES), &tmK, bar, 0, tile_kt(u) * 128, h, b);
+        if (u & 1) ++n_k1; else ++n_k0;
+    };
+    auto issue_v = [&](int u) {
+        const uint32_t bar = barV0 + 8u * (u & 1);
+        mbar_expect_tx(bar, (uint32_t)C::TILE_BYTES);
+        tma_load_4d(sV0 + (uint32_t)((u & 1) * C::TILE_BYTES), &tmV, bar, 0, tile_kt(u) * 128, h, b);
+        if (u & 1) ++n_v1; else ++n_v0;
+    };
+    const uint32_t idS = idesc_bf16_f32(128, 128, false);
+    const uint32_t idO = idesc_bf16_f32(128, D, true);
+    auto issue_S = [&](int u) {  // S(u) into TMEM buffer u & 1
+        const uint32_t sK = sK0 + (uint32_t)((u & 1) * C::TILE_BYTES);
+        const uint32_t dst = tmem + 128u * (u & 1);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            const uint64_t da = smem_desc(sQ + ks * 32, 16, C::SBO, C::LAYOUT);
+            const uint64_t db = smem_desc(sK + ks * 32, 16, C::SBO, C::LAYOUT);
+            mma_bf16_ss(dst, da, db, idS, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(barS0 + 8u * (u & 1));
+        if (u & 1) ++n_s1; else ++n_s0;
+    };
+    auto issue_PV = [&](int u) {  // P V(u) into columns [0, D) of TMEM buffer u & 1
+        const uint32_t sV = sV0 + (uint32_t)((u & 1) * C::TILE_BYTES);
+        const uint32_t dst = tmem + 128u * (u & 1);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t da = smem_desc(sP + (uint32_t)((ks >> 2) * 16384 + (ks & 3) * 32), 16, 1024,
+                                          cute::UMMA::LayoutType::SWIZZLE_128B);
+            const uint64_t db = smem_desc(sV + (uint32_t)(ks * 16 * C::ROW_BYTES), C::CHUNK_BYTES, C::SBO,
+                                          C::LAYOUT);
+            mma_bf16_ss(dst, da, db, idO, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(barO);
+        ++n_pv;
+    };
+
+    if (tid == 0) {
+        mbar_expect_tx(barQ, (uint32_t)C::TILE_BYTES);
+        tma_load_4d(sQ, &tmQ, barQ, 0, qb * 128, h, b);
+        issue_k(0);
+        issue_v(0);
+        if (T > 1) {
+            issue_k(1);
+            issue_v(1);
+        }
+        if (wait(barQ, 0) && wait(barK0, 0)) {
+            tc_fence_after();
+            issue_S(0);
+        }
+    }
+
+    const int i = qb * 128 + row;
+    const bool row_ok = i < P.n;
+    const int64_t mask_rowbase = (int64_t)b * P.mask.s0 + (int64_t)h * P.mask.s1 + (int64_t)i * P.mask.s2;
+    const int64_t bias_rowbase = (int64_t)b * P.bias.s0 + (int64_t)h * P.bias.s1 + (int64_t)i * P.bias.s2;
+    float m_ref = -INFINITY, l = 0.f;  // l: this thread's half of the row sum
+    float mu_o = 0.f, mu_prev = 0.f;   // reference of O's contents / of the last P
+    float o[DH];
+#pragma unroll
+    for (int e = 0; e < DH; ++e) o[e] = 0.f;
+
+    // adds this thread's columns of P V(u) (TMEM buffer u & 1) to O, rescaled to P(u)'s reference
+    auto accumulate_pv = [&](int u) {
+        const float f = ex2(mu_o - mu_prev);
+        const uint32_t src = tmem + 128u * (u & 1) + lane_base + half * DH;
+        if constexpr (DH == 32) {
+            uint32_t r[32];
+            tmem_ld32(src, r);
+            tmem_wait_ld_dep(r);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = fmaf(o[j], f, __uint_as_float(r[j]));
+        } else {
+            uint32_t r[16];
+            tmem_ld16(src, r);
+            asm volatile("tcgen05.wait::ld.sync.aligned;"
+                         : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                           "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                           "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                         :
+                         : "memory");
+#pragma unroll
+            for (int j = 0; j < 16; ++j) o[j] = fmaf(o[j], f, __uint_as_float(r[j]));
+        }
+        mu_o = mu_prev;
+    };
+
+    int next_info = P.tile_info[t_begin];
+    uint2 next_bits = make_uint2(0u, 0u);
+    if (next_info >= 0 && row_ok)
+        next_bits = __ldg(reinterpret_cast<const uint2*>(P.tile_bits) + ((int64_t)t_begin * 128 + row) * 2 + half);
+    const uint64_t c2 = pack2(P.qk_scale_log2, P.qk_scale_log2);
+
+    for (int u = 0; u < T; ++u) {
+        const int info = next_info;
+        const uint2 wbits = next_bits;
+        if (u + 1 < T) {
+            next_info = P.tile_info[t_begin + u + 1];
+            if (next_info >= 0 && row_ok)
+                next_bits = __ldg(reinterpret_cast<const uint2*>(P.tile_bits) +
+                                  ((int64_t)(t_begin + u + 1) * 128 + row) * 2 + half);
+        }
+        const int kt = info & 0x7fffffff;
+        const bool dense = info < 0;
+        const bool extra = EXTRA && row_ok;
+        const uint32_t bw[2] = {wbits.x, wbits.y};
+        const uint32_t tS = tmem + 128u * (u & 1) + lane_base + half * 64;
+
+        wait(barS0 + 8u * (u & 1), (uint32_t)((u >> 1) & 1));
+        tc_fence_after();
+        __syncwarp();
+        // pass 1: x = scale*log2(e)*S (+ log2(e)*(mask + bias)), unlisted entries -inf,
+        // partial max; x goes back into TMEM
+        float ma = -INFINITY, mb = -INFINITY, mc = -INFINITY, md = -INFINITY;
+#pragma unroll
+        for (int qtr = 0; qtr < 2; ++qtr) {  // 32 columns at a time
+            float xq[32];
+            if (extra) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) xq[j] = 0.f;
+                const int c0 = kt * 128 + half * 64 + qtr * 32;
+                const int ncols = P.n - c0 < 32 ? P.n - c0 : 32;
+                if (P.mask.data) add_addend_run<32>(P.mask, mask_rowbase, c0, ncols, xq);
+                if (P.bias.data) add_addend_run<32>(P.bias, bias_rowbase, c0, ncols, xq);
+            }
+            uint32_t r0[32];
+            tmem_ld32(tS + qtr * 32, r0);
+            tmem_wait_ld_dep(r0);
+            if (extra) {
+#pragma unroll
+                for (int k = 0; k < 16; ++k) fma2_inplace(xq[2 * k], xq[2 * k + 1], r0[2 * k], r0[2 * k + 1], c2);
+            } else {
+#pragma unroll
+                for (int k = 0; k < 16; ++k) mul2(xq[2 * k], xq[2 * k + 1], r0[2 * k], r0[2 * k + 1], c2);
+            }
+            if (!dense) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) xq[j] = ((bw[qtr] >> j) & 1u) ? xq[j] : -INFINITY;
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                ma = fmax3(ma, xq[8 * k + 0], xq[8 * k + 1]);
+                mb = fmax3(mb, xq[8 * k + 2], xq[8 * k + 3]);
+                mc = fmax3(mc, xq[8 * k + 4], xq[8 * k + 5]);
+                md = fmax3(md, xq[8 * k + 6], xq[8 * k + 7]);
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) r0[j] = __float_as_uint(xq[j]);
+            tmem_st32(tS + qtr * 32, r0);
+        }
+        tmem_wait_st();
+        const float my_max = fmax3(ma, mb, fmaxf(mc, md));
+
+        if (u > 0) {  // P V(u-1) is in the other buffer; V(u-1)'s buffer is free after it
+            wait(barO, (uint32_t)((u - 1) & 1));
+            tc_fence_after();
+            if (tid == 0 && u + 1 < T && !*abort_flag) issue_v(u + 1);
+            __syncwarp();
+            accumulate_pv(u - 1);
+        }
+        // sP is free (P V(u-1) done): leave the partial max for the partner
+        asm volatile("st.shared.f32 [%0], %1;" ::"r"(my_slot), "f"(my_max) : "memory");
+        // mid-tile: the other TMEM buffer is free -> S(u+1) runs while this tile exponentiates
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && u + 1 < T && !*abort_flag) {
+            tc_fence_after();
+            if (wait(barK0 + 8u * ((u + 1) & 1), (uint32_t)(((u + 1) >> 1) & 1))) {
+                tc_fence_after();
+                issue_S(u + 1);
+            }
+        }
+        __syncwarp();
+        float other_max;
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(other_max) : "r"(partner_slot) : "memory");
+        const float mx = fmaxf(my_max, other_max);
+        if (mx > m_ref + kRescaleThreshold) {
+            l *= ex2(m_ref - mx);
+            m_ref = mx;
+        }
+        const float mu = m_ref == -INFINITY ? 0.f : m_ref;
+
+        // pass 2: p = exp2(x - mu), partial sum, P (bf16) into chunk `half` of the K-major,
+        // 128-byte-swizzled A operand layout
+        const uint64_t nmu2 = pack2(-mu, -mu);
+        uint64_t sa = pack2(0.f, 0.f), sb = sa;
+#pragma unroll
+        for (int qtr = 0; qtr < 2; ++qtr) {
+            uint32_t r0[32];
+            tmem_ld32(tS + qtr * 32, r0);
+            tmem_wait_ld_dep(r0);
+            uint32_t pk[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                float p0, p1;
+                unpack2(add2(pack2(__uint_as_float(r0[2 * k]), __uint_as_float(r0[2 * k + 1])), nmu2), p0, p1);
+                p0 = ex2(p0);
+                p1 = ex2(p1);
+                if (k & 1)
+                    sb = add2(sb, pack2(p0, p1));
+                else
+                    sa = add2(sa, pack2(p0, p1));
+                __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
+                pk[k] = *reinterpret_cast<uint32_t*>(&hv);
+            }
+#pragma unroll
+            for (int pc = 0; pc < 4; ++pc) {
+                const int piece = qtr * 4 + pc;
+                const uint32_t addr = sP + (uint32_t)(half * 16384 + row * 128 + ((piece ^ (row & 7)) << 4));
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[pc * 4]),
+                             "r"(pk[pc * 4 + 1]), "r"(pk[pc * 4 + 2]), "r"(pk[pc * 4 + 3])
+                             : "memory");
+            }
+        }
+        {
+            float s0, s1, s2, s3;
+            unpack2(sa, s0, s1);
+            unpack2(sb, s2, s3);
+            l += (s0 + s1) + (s2 + s3);
+        }
+        mu_prev = mu;
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && !*abort_flag) {
+            tc_fence_after();
+            if (u + 2 < T) issue_k(u + 2);  // S(u) consumed K(u) long ago
+            if (wait(barV0 + 8u * (u & 1), (uint32_t)((u >> 1) & 1))) {
+                tc_fence_after();
+                issue_PV(u);
+            }
+        }
+    }
+
+    // ------------------------------------------------------------ epilogue
+    wait(barO, (uint32_t)((T - 1) & 1));
+    tc_fence_after();
+    __syncwarp();
+    accumulate_pv(T - 1);
+    // combine the two halves of the row sum (sP is free: the last P V is done)
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(my_slot), "f"(l) : "memory");
+    __syncthreads();
+    float l_other;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(l_other) : "r"(partner_slot) : "memory");
+    const float l_row = l + l_other;
+    if (row_ok && !*abort_flag) {
+        float M = m_ref, L = l_row, fa;
+        const int64_t mrow = (int64_t)mk * P.n + i;
+        const int64_t wrow = (int64_t)bh * P.n + i;
+        const bool mixed = P.ws_ml && P.res_row_ptr[mrow + 1] > P.res_row_ptr[mrow];
+        float fg = 0.f;
+        if (mixed) {
+            const float mg = P.ws_ml[wrow * 2], lg = P.ws_ml[wrow * 2 + 1];
+            M = fmaxf(m_ref, mg);
+            const float Mu = M == -INFINITY ? 0.f : M;
+            fa = ex2(mu_o - Mu);
+            fg = ex2(mg - Mu);
+            L = l_row * ex2(m_ref - Mu) + lg * fg;
+        } else {
+            fa = ex2(mu_o - (m_ref == -INFINITY ? 0.f : m_ref));
+        }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(P.out) + (int64_t)b * P.o_sb +
+                              (int64_t)h * P.o_sh + (int64_t)i * P.o_sn + half * DH;
+        const float* acc = mixed ? P.ws_acc + wrow * D + half * DH : nullptr;
+#pragma unroll
+        for (int e8 = 0; e8 < DH / 8; ++e8) {
+            float v[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                float val = o[e8 * 8 + t] * fa;
+                if (mixed) val = fmaf(acc[e8 * 8 + t], fg, val);
+                v[t] = val * inv;
+            }
+            uint32_t w[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                __nv_bfloat162 hv = __floats2bfloat162_rn(v[2 * t], v[2 * t + 1]);
+                w[t] = *reinterpret_cast<uint32_t*>(&hv);
+            }
+            *reinterpret_cast<uint4*>(orow + e8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        if (P.lse && half == 0) P.lse[wrow] = L > 0.f ? (M + lg2(L)) * kLn2 : -INFINITY;
+    }
+
+    // ------------------------------------------------------------ teardown
+    if (tid == 0 && *abort_flag) {
+        const long long lim = kWaitCycles / 16;
+        const int cnt[6] = {n_k0, n_k1, n_v0, n_v1, n_s0, n_s1};
+        const uint32_t bar6[6] = {barK0, barK0 + 8u, barV0, barV0 + 8u, barS0, barS0 + 8u};
+        for (int x = 0; x < 6; ++x)
+            if (cnt[x]) mbar_wait_bounded(bar6[x], (uint32_t)((cnt[x] - 1) & 1), lim);
+        if (n_pv) mbar_wait_bounded(barO, (uint32_t)((n_pv - 1) & 1), lim);
+        atomicOr(P.err, kErrTimeout);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
@@ -459,8 +926,17 @@ cudaError_t launch_tc_t(const TcOperand& q, const TcOperand& k, const TcOperand&
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, []() {
-        attr_err = cudaFuncSetAttribute(k_fwd_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        C::SMEM_BYTES);
+        constexpr int DP = D <= 64 ? D : 64;
+        if (D <= 64) {
+            attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_pipe<DP, false>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+            if (attr_err == cudaSuccess)
+                attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_pipe<DP, true>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        } else {
+            attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc<D>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        }
     });
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap mq, mk, mv;
@@ -470,7 +946,13 @@ cudaError_t launch_tc_t(const TcOperand& q, const TcOperand& k, const TcOperand&
     if ((e = make_map(&mv, v, p.B, p.H, p.n, D, C::CHUNK_ELEMS)) != cudaSuccess) return e;
     const int64_t grid = (int64_t)p.B * p.H * p.nqb;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    k_fwd_tc<D><<<(unsigned)grid, kThreads, C::SMEM_BYTES, s>>>(mq, mk, mv, p);
+    constexpr int DP = D <= 64 ? D : 64;
+    if (D <= 64 && p.has_extra)
+        k_fwd_tc_pipe<DP, true><<<(unsigned)grid, kPipeThreads, C::SMEM_BYTES, s>>>(mq, mk, mv, p);
+    else if (D <= 64)
+        k_fwd_tc_pipe<DP, false><<<(unsigned)grid, kPipeThreads, C::SMEM_BYTES, s>>>(mq, mk, mv, p);
+    else
+        k_fwd_tc<D><<<(unsigned)grid, kThreads, C::SMEM_BYTES, s>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }
 

@@ -83,7 +83,8 @@ __device__ __forceinline__ int64_t bsg_next(const BuildSpec& s, int64_t i, int64
     return c;
 }
 
-__global__ void k_count(BuildSpec s, int32_t* __restrict__ counts, BuildInfo* info) {
+__global__ void k_count(BuildSpec s, int32_t* __restrict__ counts, BuildInfo* info,
+                        int32_t* __restrict__ long_rows) {
     const int64_t rows = (int64_t)s.num_masks * s.n;
     for (int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; r < rows;
          r += (int64_t)gridDim.x * blockDim.x) {
@@ -102,7 +103,16 @@ __global__ void k_count(BuildSpec s, int32_t* __restrict__ counts, BuildInfo* in
             for (int64_t j = bsg_next(s, i, 0); j < s.n; j = bsg_next(s, i, j + 1)) ++cnt;
         }
         counts[r] = (int32_t)cnt;
+        if (cnt > kLongRowThreshold && long_rows) long_rows[atomicAdd(&info->n_long, 1)] = (int32_t)r;
     }
+}
+
+// Rows longer than kLongRowThreshold, from per-row counts (COO kind).
+__global__ void k_classify_counts(const int32_t* __restrict__ counts, int64_t rows,
+                                  int32_t* __restrict__ long_rows, BuildInfo* info) {
+    for (int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; r < rows;
+         r += (int64_t)gridDim.x * blockDim.x)
+        if (counts[r] > kLongRowThreshold) long_rows[atomicAdd(&info->n_long, 1)] = (int32_t)r;
 }
 
 // User CSR: every row strictly increasing with columns in [0, n).
@@ -309,6 +319,37 @@ __device__ __forceinline__ int64_t block_exclusive_scan(int64_t x, int64_t* tota
     return res;
 }
 
+// Arrays up to kScanSmallMax: a single block scans tile after tile.
+constexpr int64_t kScanSmallMax = 16 * kScanTile;
+
+__global__ void __launch_bounds__(kScanThreads)
+    k_scan_small(const int32_t* __restrict__ counts, int64_t rows, int32_t* __restrict__ out,
+                 int64_t* total_out, unsigned* err) {
+    int64_t carry = 0;
+    for (int64_t t0 = 0; t0 < rows; t0 += kScanTile) {
+        const int64_t base = t0 + (int64_t)threadIdx.x * kScanItems;
+        int64_t v[kScanItems], sum = 0;
+#pragma unroll
+        for (int t = 0; t < kScanItems; ++t) {
+            v[t] = base + t < rows ? counts[base + t] : 0;
+            sum += v[t];
+        }
+        int64_t total;
+        int64_t run = carry + block_exclusive_scan(sum, &total);
+#pragma unroll
+        for (int t = 0; t < kScanItems; ++t) {
+            if (base + t < rows) out[base + t] = run > INT_MAX ? INT_MAX : (int32_t)run;
+            run += v[t];
+        }
+        carry += total;
+    }
+    if (threadIdx.x == 0) {
+        out[rows] = carry > INT_MAX ? INT_MAX : (int32_t)carry;
+        *total_out = carry;
+        if (carry > INT_MAX) atomicOr(err, kBuildTooMany);
+    }
+}
+
 // Tile t of kScanTile counts: local exclusive prefixes + the tile's total.
 __global__ void __launch_bounds__(kScanThreads)
     k_scan_tiles(const int32_t* __restrict__ counts, int64_t rows, int64_t* __restrict__ pref,
@@ -411,7 +452,7 @@ int64_t scan_tmp_elems(int64_t rows) { return rows + 1 + (rows + kScanTile - 1) 
 
 cudaError_t build_phase1(const BuildSpec& s, int32_t* row_ptr, int32_t* counts,
                          int64_t* scan_tmp, int32_t* coo_tmp, BuildInfo* info,
-                         cudaStream_t stream) {
+                         int32_t* long_rows, cudaStream_t stream) {
     const int64_t rows = (int64_t)s.num_masks * s.n;
     cudaError_t e;
     if (s.kind == SPATTN_MASK_COO) {
@@ -440,18 +481,26 @@ cudaError_t build_phase1(const BuildSpec& s, int32_t* row_ptr, int32_t* counts,
             }
         }
     } else {
-        k_count<<<grid_for(rows, 256), 256, 0, stream>>>(s, counts, info);
+        k_count<<<grid_for(rows, 256), 256, 0, stream>>>(s, counts, info, long_rows);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         if (s.kind == SPATTN_MASK_CSR) {
             k_check_csr<<<grid_for(rows, 8), 256, 0, stream>>>(s, info);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
     }
+    if (s.kind == SPATTN_MASK_COO) {
+        k_classify_counts<<<grid_for(rows, 256), 256, 0, stream>>>(counts, rows, long_rows, info);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     return scan_counts(counts, rows, row_ptr, scan_tmp, &info->nnz, &info->err, stream);
 }
 
 cudaError_t scan_counts(const int32_t* counts, int64_t rows, int32_t* out, int64_t* scan_tmp,
                         int64_t* total, unsigned* err, cudaStream_t stream) {
+    if (rows <= kScanSmallMax) {  // one block walks the tiles with a running carry
+        k_scan_small<<<1, kScanThreads, 0, stream>>>(counts, rows, out, total, err);
+        return cudaGetLastError();
+    }
     const int64_t ntiles = (rows + kScanTile - 1) / kScanTile;
     int64_t* pref = scan_tmp;
     int64_t* tile_sums = scan_tmp + rows + 1;

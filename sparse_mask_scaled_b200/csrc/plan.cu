@@ -56,29 +56,42 @@ __global__ void k_tile_select(const int32_t* __restrict__ cnt, int64_t nblocks, 
 }
 
 // Number the selected tiles (block-major, key tiles ascending) and turn the
-// count array into a map (tile id, or -1).
+// count array into a map (tile id, or -1). One warp per query block.
 __global__ void k_tile_assign(int32_t* __restrict__ cnt_map, int64_t nblocks, int nkt, int min_nnz,
                               const int32_t* __restrict__ block_tile_off,
                               int32_t* __restrict__ tile_info) {
-    for (int64_t x = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; x < nblocks;
-         x += (int64_t)gridDim.x * blockDim.x) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t x = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5); x < nblocks;
+         x += warps) {
         int idx = block_tile_off[x];
-        for (int kt = 0; kt < nkt; ++kt) {
-            const int c = cnt_map[x * nkt + kt];
-            if (c >= min_nnz) {
-                tile_info[idx] = kt | (c == kTileM * kTileN ? (int)kTileDenseBit : 0);
-                cnt_map[x * nkt + kt] = idx++;
-            } else {
-                cnt_map[x * nkt + kt] = -1;
+        for (int k0 = 0; k0 < nkt; k0 += 32) {
+            const int kt = k0 + lane;
+            const int c = kt < nkt ? cnt_map[x * nkt + kt] : 0;
+            const bool sel = kt < nkt && c >= min_nnz;
+            const unsigned bal = __ballot_sync(0xffffffffu, sel);
+            if (kt < nkt) {
+                if (sel) {
+                    const int id = idx + __popc(bal & ((1u << lane) - 1u));
+                    tile_info[id] = kt | (c == kTileM * kTileN ? (int)kTileDenseBit : 0);
+                    cnt_map[x * nkt + kt] = id;
+                } else {
+                    cnt_map[x * nkt + kt] = -1;
+                }
             }
+            idx += __popc(bal);
         }
     }
 }
 
-// One warp per row: set the bits of entries in selected tiles, count the rest.
+// One warp per row: set the bits of entries in selected (not dense) tiles, one
+// atomic per 32-bit word (columns are sorted, so a word's entries are adjacent
+// lanes), count the rest and list rows whose residual is long.
 __global__ void k_tile_bits(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
                             int n, int64_t rows, int nqb, int nkt, const int32_t* __restrict__ map,
-                            uint32_t* __restrict__ bits, int32_t* __restrict__ res_cnt) {
+                            const int32_t* __restrict__ tile_info, uint32_t* __restrict__ bits,
+                            int32_t* __restrict__ res_cnt, int32_t* __restrict__ res_long,
+                            int32_t* __restrict__ res_n_long) {
     const int lane = threadIdx.x & 31;
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
     for (int64_t r = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
@@ -87,19 +100,34 @@ __global__ void k_tile_bits(const int32_t* __restrict__ row_ptr, const int32_t* 
         const int64_t base = (m * nqb + (i >> 7)) * nkt;
         const int row_in_tile = (int)(i & 127);
         int res = 0;
-        for (int64_t p = row_ptr[r] + lane; p < row_ptr[r + 1]; p += 32) {
-            const int j = col_idx[p];
-            const int id = map[base + (j >> 7)];
-            if (id >= 0) {
-                const int c = j & 127;
-                atomicOr(&bits[((int64_t)id * kTileM + row_in_tile) * 4 + (c >> 5)], 1u << (c & 31));
-            } else {
-                ++res;
+        const int64_t p1 = row_ptr[r + 1];
+        for (int64_t c0 = row_ptr[r]; c0 < p1; c0 += 32) {
+            const int64_t p = c0 + lane;
+            int key = -1;
+            uint32_t bit = 0u;
+            bool residual = false;
+            if (p < p1) {
+                const int j = col_idx[p];
+                const int id = map[base + (j >> 7)];
+                if (id >= 0) {
+                    if (tile_info[id] >= 0) {  // dense tiles need no bits
+                        key = id * 4 + ((j & 127) >> 5);
+                        bit = 1u << (j & 31);
+                    }
+                } else {
+                    residual = true;
+                }
             }
+            res += __popc(__ballot_sync(0xffffffffu, residual));
+            const unsigned grp = __match_any_sync(0xffffffffu, key);
+            const uint32_t word = __reduce_or_sync(grp, bit);
+            if (key >= 0 && lane == __ffs(grp) - 1)
+                atomicOr(&bits[((int64_t)(key >> 2) * kTileM + row_in_tile) * 4 + (key & 3)], word);
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) res += __shfl_xor_sync(0xffffffffu, res, off);
-        if (lane == 0) res_cnt[r] = res;
+        if (lane == 0) {
+            res_cnt[r] = res;
+            if (res > kLongRowThreshold) res_long[atomicAdd(res_n_long, 1)] = (int32_t)r;
+        }
     }
 }
 
@@ -118,6 +146,7 @@ __global__ void k_residual_fill(const int32_t* __restrict__ row_ptr, const int32
         const int64_t blk = m * nqb + (i >> 7);
         const int64_t base = blk * nkt;
         int64_t o = res_row_ptr[r];
+        if (res_row_ptr[r + 1] == o) continue;  // nothing left for the gather kernel
         const int64_t p1 = row_ptr[r + 1];
         for (int64_t c0 = row_ptr[r]; c0 < p1; c0 += 32) {
             const int64_t p = c0 + lane;
@@ -131,9 +160,7 @@ __global__ void k_residual_fill(const int32_t* __restrict__ row_ptr, const int32
             if (keep) res_col[o + __popc(bal & ((1u << lane) - 1u))] = j;
             o += __popc(bal);
         }
-        if (lane == 0 && block_tile_off[blk + 1] > block_tile_off[blk] &&
-            res_row_ptr[r + 1] > res_row_ptr[r])
-            atomicAdd(n_mixed, 1);
+        if (lane == 0 && block_tile_off[blk + 1] > block_tile_off[blk]) atomicAdd(n_mixed, 1);
     }
 }
 
@@ -170,19 +197,19 @@ cudaError_t build_plan(const int32_t* row_ptr, const int32_t* col_idx, int n, in
     e = scan_counts(b.block_ntiles, nblocks, b.block_tile_off, b.scan_tmp, &counters->n_tiles,
                     &counters->err, s);
     if (e != cudaSuccess) return e;
-    k_tile_assign<<<grid_for(nblocks, 128), 128, 0, s>>>(b.cnt_map, nblocks, nkt, min_nnz,
-                                                        b.block_tile_off, b.tile_info);
+    k_tile_assign<<<grid_for(nblocks, 8), 256, 0, s>>>(b.cnt_map, nblocks, nkt, min_nnz,
+                                                      b.block_tile_off, b.tile_info);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k_tile_bits<<<grid_for(rows, 8), 256, 0, s>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map,
-                                                 b.tile_bits, b.res_cnt);
+                                                 b.tile_info, b.tile_bits, b.res_cnt, b.res_long,
+                                                 &counters->res_n_long);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     e = scan_counts(b.res_cnt, rows, b.res_row_ptr, b.scan_tmp, &counters->res_nnz, &counters->err, s);
     if (e != cudaSuccess) return e;
     k_residual_fill<<<grid_for(rows, 8), 256, 0, s>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map,
                                                      b.block_tile_off, b.res_row_ptr, b.res_col_idx,
                                                      &counters->n_mixed);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    return launch_classify_long_rows(b.res_row_ptr, rows, nnz, b.res_long, &counters->res_n_long, s);
+    return cudaGetLastError();
 }
 
 }  // namespace spattn

@@ -35,6 +35,10 @@ struct spattn_mask_s {
     int32_t* res_row_ptr;
     int32_t* res_col_idx;
     int32_t* res_long;
+    // owned pool blocks the arrays above are carved from
+    void* block_csr;   // row_ptr, long_rows
+    void* block_col;   // col_idx
+    void* block_plan;  // block_tile_off, tile_info, tile_bits, res_row_ptr, res_col_idx, res_long
 };
 
 namespace {
@@ -208,15 +212,28 @@ int launch_fwd(FwdParams& p, int dtype, int d, int num_sms, cudaStream_t s) {
 }
 
 void free_plan(spattn_mask m) {
-    int32_t** ptrs[] = {&m->block_tile_off, &m->tile_info, &m->res_row_ptr, &m->res_col_idx, &m->res_long};
-    for (int32_t** p : ptrs) {
-        if (*p) cudaFreeAsync(*p, m->stream);
-        *p = nullptr;
-    }
-    if (m->tile_bits) cudaFreeAsync(m->tile_bits, m->stream);
+    if (m->block_plan) cudaFreeAsync(m->block_plan, m->stream);
+    m->block_plan = nullptr;
+    m->block_tile_off = m->tile_info = m->res_row_ptr = m->res_col_idx = m->res_long = nullptr;
     m->tile_bits = nullptr;
     m->has_plan = false;
 }
+
+// Lays out arrays in one pool allocation (each start 256-byte aligned).
+struct Carve {
+    size_t off[16];
+    size_t total = 0;
+    int n = 0;
+    int add(size_t bytes) {
+        off[n] = total;
+        total += (bytes + 255) & ~size_t(255);
+        return n++;
+    }
+    template <typename T>
+    T* at(void* base, int k) const {
+        return reinterpret_cast<T*>(static_cast<char*>(base) + off[k]);
+    }
+};
 
 unsigned* g_err_ptr[kMaxDevices];
 
@@ -287,40 +304,37 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
     bs.in_col_idx = sp.in_col_idx;
     bs.in_nnz = sp.in_nnz;
 
-    int32_t *row_ptr = nullptr, *counts = nullptr, *coo_tmp = nullptr;
-    int64_t* scan_tmp = nullptr;
-    BuildInfo* info = nullptr;
     const bool coo = sp.kind == SPATTN_MASK_COO;
-    const int64_t scan_elems = scan_tmp_elems(rows) + (coo ? (rows + 6) / 2 + 1 : 0);
-    auto release_tmp = [&]() {
-        if (counts) cudaFreeAsync(counts, s);
-        if (scan_tmp) cudaFreeAsync(scan_tmp, s);
-        if (coo_tmp) cudaFreeAsync(coo_tmp, s);
-        if (info) cudaFreeAsync(info, s);
-        counts = coo_tmp = nullptr;
-        scan_tmp = nullptr;
-        info = nullptr;
-    };
-    cudaError_t e = pool_alloc(&row_ptr, rows + 1, pool, s);
-    if (e == cudaSuccess) e = pool_alloc(&counts, rows, pool, s);
-    if (e == cudaSuccess) e = pool_alloc(&scan_tmp, scan_elems, pool, s);
-    if (e == cudaSuccess && coo) e = pool_alloc(&coo_tmp, sp.in_nnz + rows, pool, s);
-    if (e == cudaSuccess) e = pool_alloc(&info, 1, pool, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(info, 0, sizeof(BuildInfo), s);
-    if (e == cudaSuccess) e = build_phase1(bs, row_ptr, counts, scan_tmp, coo_tmp, info, s);
+    // phase 1 memory: the mask's row_ptr + long-row list, and temporaries
+    Carve ca;
+    const int k_rp = ca.add((rows + 1) * 4), k_long = ca.add(rows * 4);
+    Carve ct;
+    const int k_info = ct.add(sizeof(BuildInfo)), k_cnt = ct.add(rows * 4);
+    const int k_scan = ct.add((scan_tmp_elems(rows) + (coo ? (rows + 6) / 2 + 1 : 0)) * 8);
+    const int k_coo = ct.add(coo ? (sp.in_nnz + rows) * 4 : 0);
+    void *blk_a = nullptr, *blk_t = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync(&blk_a, ca.total, pool, s);
+    if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&blk_t, ct.total, pool, s);
+    if (e != cudaSuccess) {
+        if (blk_a) cudaFreeAsync(blk_a, s);
+        return cuda_fail(e, "mask allocation");
+    }
+    int32_t* row_ptr = ca.at<int32_t>(blk_a, k_rp);
+    int32_t* long_rows = ca.at<int32_t>(blk_a, k_long);
+    BuildInfo* info = ct.at<BuildInfo>(blk_t, k_info);
+    int32_t* counts = ct.at<int32_t>(blk_t, k_cnt);
+    int64_t* scan_tmp = ct.at<int64_t>(blk_t, k_scan);
+    int32_t* coo_tmp = coo ? ct.at<int32_t>(blk_t, k_coo) : nullptr;
+    e = cudaMemsetAsync(info, 0, sizeof(BuildInfo), s);
+    if (e == cudaSuccess) e = build_phase1(bs, row_ptr, counts, scan_tmp, coo_tmp, info, long_rows, s);
     BuildInfo hinfo;
     if (e == cudaSuccess) e = cudaMemcpyAsync(&hinfo, info, sizeof hinfo, cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-    if (e != cudaSuccess) {
-        release_tmp();
-        if (row_ptr) cudaFreeAsync(row_ptr, s);
-        return cuda_fail(e, "mask build (phase 1)");
-    }
-    int st = build_status(hinfo.err);
-    if (st != SPATTN_OK) {
-        release_tmp();
-        cudaFreeAsync(row_ptr, s);
-        return st;
+    int st = e == cudaSuccess ? build_status(hinfo.err) : SPATTN_OK;
+    if (e != cudaSuccess || st != SPATTN_OK) {
+        cudaFreeAsync(blk_t, s);
+        cudaFreeAsync(blk_a, s);
+        return e != cudaSuccess ? cuda_fail(e, "mask build (phase 1)") : st;
     }
     spattn_mask m = new spattn_mask_s;
     memset(m, 0, sizeof *m);
@@ -329,63 +343,65 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
     m->n = sp.n;
     m->num_masks = sp.num_masks;
     m->nnz = hinfo.nnz;
+    m->n_long = hinfo.n_long;
     m->row_ptr = row_ptr;
-    e = pool_alloc(&m->col_idx, hinfo.nnz, pool, s);
-    if (e == cudaSuccess) e = build_phase2(bs, row_ptr, coo_tmp, m->col_idx, s);
-    if (e == cudaSuccess) e = pool_alloc(&m->long_rows, rows, pool, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(&info->n_long, 0, sizeof(int32_t), s);
-    if (e == cudaSuccess)
-        e = launch_classify_long_rows(row_ptr, rows, hinfo.nnz, m->long_rows, &info->n_long, s);
+    m->long_rows = long_rows;
+    m->block_csr = blk_a;
 
-    // tile plan: tensor-core tiles, their bit masks and the residual CSR
+    // phase 2 memory: col_idx, the tile plan, and the plan's temporaries
     const int min_nnz = sp.tile_min_nnz == 0 ? kTileMinNnzDefault : sp.tile_min_nnz;
     const int nqb = (sp.n + kTileM - 1) / kTileM, nkt = (sp.n + kTileN - 1) / kTileN;
     const int64_t nblocks = (int64_t)sp.num_masks * nqb;
     const bool plan = sp.tile_min_nnz >= 0 && hinfo.nnz > 0 && nblocks * nkt <= kPlanMaxTileGrid;
     PlanBuffers pb;
     memset(&pb, 0, sizeof pb);
-    PlanCounters* pc = nullptr;
     PlanCounters hpc;
     memset(&hpc, 0, sizeof hpc);
+    void* blk_t2 = nullptr;
+    e = cudaMallocFromPoolAsync(&m->block_col, (size_t)(hinfo.nnz > 0 ? hinfo.nnz : 1) * 4, pool, s);
+    if (e == cudaSuccess) {
+        m->col_idx = static_cast<int32_t*>(m->block_col);
+        e = build_phase2(bs, row_ptr, coo_tmp, m->col_idx, s);
+    }
     if (plan && e == cudaSuccess) {
         m->nqb = nqb;
         pb.tile_cap = plan_tile_capacity(nblocks, nkt, hinfo.nnz, min_nnz);
+        Carve cp;
+        const int k_bto = cp.add((nblocks + 1) * 4), k_ti = cp.add(pb.tile_cap * 4),
+                  k_tb = cp.add(pb.tile_cap * kTileM * 16), k_rrp = cp.add((rows + 1) * 4),
+                  k_rci = cp.add(hinfo.nnz * 4), k_rl = cp.add(rows * 4);
+        Carve c2;
         const int64_t scan_rows = rows > nblocks ? rows : nblocks;
-        if (e == cudaSuccess) e = pool_alloc(&pc, 1, pool, s);
-        if (e == cudaSuccess) e = cudaMemsetAsync(pc, 0, sizeof(PlanCounters), s);
-        if (e == cudaSuccess) e = pool_alloc(&pb.cnt_map, nblocks * nkt, pool, s);
-        if (e == cudaSuccess) e = pool_alloc(&pb.block_ntiles, nblocks, pool, s);
-        if (e == cudaSuccess) e = pool_alloc(&pb.scan_tmp, scan_tmp_elems(scan_rows), pool, s);
-        if (e == cudaSuccess) e = pool_alloc(&pb.res_cnt, rows, pool, s);
-        if (e == cudaSuccess) e = pool_alloc(&m->block_tile_off, nblocks + 1, pool, s);
-        if (e == cudaSuccess) e = pool_alloc(&m->tile_info, pb.tile_cap, pool, s);
-        if (e == cudaSuccess) e = pool_alloc(&m->tile_bits, pb.tile_cap * kTileM * 4, pool, s);
-        if (e == cudaSuccess) e = pool_alloc(&m->res_row_ptr, rows + 1, pool, s);
-        if (e == cudaSuccess) e = pool_alloc(&m->res_col_idx, hinfo.nnz, pool, s);
-        if (e == cudaSuccess) e = pool_alloc(&m->res_long, rows, pool, s);
-        pb.block_tile_off = m->block_tile_off;
-        pb.tile_info = m->tile_info;
-        pb.tile_bits = m->tile_bits;
-        pb.res_row_ptr = m->res_row_ptr;
-        pb.res_col_idx = m->res_col_idx;
-        pb.res_long = m->res_long;
-        if (e == cudaSuccess)
-            e = build_plan(row_ptr, m->col_idx, sp.n, sp.num_masks, hinfo.nnz, min_nnz, pb, pc, s);
-        if (e == cudaSuccess) e = cudaMemcpyAsync(&hpc, pc, sizeof hpc, cudaMemcpyDeviceToHost, s);
+        const int k_pc = c2.add(sizeof(PlanCounters)), k_cm = c2.add(nblocks * nkt * 4),
+                  k_bn = c2.add(nblocks * 4), k_st = c2.add(scan_tmp_elems(scan_rows) * 8),
+                  k_rc = c2.add(rows * 4);
+        e = cudaMallocFromPoolAsync(&m->block_plan, cp.total, pool, s);
+        if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&blk_t2, c2.total, pool, s);
+        if (e == cudaSuccess) {
+            m->block_tile_off = pb.block_tile_off = cp.at<int32_t>(m->block_plan, k_bto);
+            m->tile_info = pb.tile_info = cp.at<int32_t>(m->block_plan, k_ti);
+            m->tile_bits = pb.tile_bits = cp.at<uint32_t>(m->block_plan, k_tb);
+            m->res_row_ptr = pb.res_row_ptr = cp.at<int32_t>(m->block_plan, k_rrp);
+            m->res_col_idx = pb.res_col_idx = cp.at<int32_t>(m->block_plan, k_rci);
+            m->res_long = pb.res_long = cp.at<int32_t>(m->block_plan, k_rl);
+            PlanCounters* pc = c2.at<PlanCounters>(blk_t2, k_pc);
+            pb.cnt_map = c2.at<int32_t>(blk_t2, k_cm);
+            pb.block_ntiles = c2.at<int32_t>(blk_t2, k_bn);
+            pb.scan_tmp = c2.at<int64_t>(blk_t2, k_st);
+            pb.res_cnt = c2.at<int32_t>(blk_t2, k_rc);
+            e = cudaMemsetAsync(pc, 0, sizeof(PlanCounters), s);
+            if (e == cudaSuccess)
+                e = build_plan(row_ptr, m->col_idx, sp.n, sp.num_masks, hinfo.nnz, min_nnz, pb, pc, s);
+            if (e == cudaSuccess) e = cudaMemcpyAsync(&hpc, pc, sizeof hpc, cudaMemcpyDeviceToHost, s);
+            if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        }
     }
-    if (e == cudaSuccess) e = cudaMemcpyAsync(&hinfo, info, sizeof hinfo, cudaMemcpyDeviceToHost, s);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-    release_tmp();
-    if (pc) cudaFreeAsync(pc, s);
-    if (pb.cnt_map) cudaFreeAsync(pb.cnt_map, s);
-    if (pb.block_ntiles) cudaFreeAsync(pb.block_ntiles, s);
-    if (pb.scan_tmp) cudaFreeAsync(pb.scan_tmp, s);
-    if (pb.res_cnt) cudaFreeAsync(pb.res_cnt, s);
+    cudaFreeAsync(blk_t, s);
+    if (blk_t2) cudaFreeAsync(blk_t2, s);
     if (e != cudaSuccess) {
         spattn_destroy_mask(m);
         return cuda_fail(e, "mask build (phase 2)");
     }
-    m->n_long = hinfo.n_long;
     if (plan) {
         m->n_tiles = hpc.n_tiles;
         m->res_nnz = hpc.res_nnz;
@@ -472,9 +488,8 @@ int spattn_destroy_mask(spattn_mask m) {
     cudaGetDevice(&prev);
     if (prev != m->device) cudaSetDevice(m->device);
     cudaError_t e = cudaSuccess, e2;
-    if (m->row_ptr && (e2 = cudaFreeAsync(m->row_ptr, m->stream)) != cudaSuccess) e = e2;
-    if (m->col_idx && (e2 = cudaFreeAsync(m->col_idx, m->stream)) != cudaSuccess) e = e2;
-    if (m->long_rows && (e2 = cudaFreeAsync(m->long_rows, m->stream)) != cudaSuccess) e = e2;
+    if (m->block_csr && (e2 = cudaFreeAsync(m->block_csr, m->stream)) != cudaSuccess) e = e2;
+    if (m->block_col && (e2 = cudaFreeAsync(m->block_col, m->stream)) != cudaSuccess) e = e2;
     free_plan(m);
     if (prev >= 0 && prev != m->device) cudaSetDevice(prev);
     delete m;

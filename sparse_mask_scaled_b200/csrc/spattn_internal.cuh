@@ -18,7 +18,7 @@ constexpr unsigned kErrTimeout = 2u;  // a bounded wait of the tensor-core kerne
 constexpr int kTileM = 128;
 constexpr int kTileN = 128;
 constexpr unsigned kTileDenseBit = 0x80000000u;  // tile_info flag: all 128 x 128 entries present
-constexpr int kTileMinNnzDefault = 256;
+constexpr int kTileMinNnzDefault = 512;
 // Tile planning is skipped when num_masks * (n/128)^2 exceeds this (count array size).
 constexpr int64_t kPlanMaxTileGrid = int64_t(1) << 26;
 
@@ -163,9 +163,11 @@ enum BuildErr : unsigned {
 // `scan_tmp` int64 [scan_tmp_elems(rows)] followed, for COO, by int32
 // [rows + 4] (the queue of long COO rows); coo_tmp int32 [in_nnz + rows]
 // (COO only). info->err must start at 0.
+// Also lists rows with more than kLongRowThreshold entries in long_rows [rows],
+// counted in info->n_long.
 cudaError_t build_phase1(const BuildSpec& s, int32_t* row_ptr, int32_t* counts,
                          int64_t* scan_tmp, int32_t* coo_tmp, BuildInfo* info,
-                         cudaStream_t stream);
+                         int32_t* long_rows, cudaStream_t stream);
 int64_t scan_tmp_elems(int64_t rows);
 // Exclusive scan of int32 counts [rows] into out int32 [rows + 1]; the total goes
 // to *total (device) and overflow past INT32_MAX sets kBuildTooMany in *err.

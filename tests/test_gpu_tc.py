@@ -56,6 +56,10 @@ def _check_plan(mask, rp, ci, n, nm, thr):
             dense = info[t] < 0
             assert dense == (cnt[x, kt] == 128 * 128)
             w = bits[t * 512:(t + 1) * 512].view(np.uint32).reshape(128, 4)
+            if dense:      # all entries present; bits are not stored
+                assert not w.any()
+                covered.update((m * n + qb * 128 + rr, kt * 128 + c) for rr in range(128) for c in range(128))
+                continue
             for rr in range(128):
                 i = qb * 128 + rr
                 word = w[rr]
@@ -89,7 +93,7 @@ def test_plan_partitions_the_csr(cfg, kw, thr):
     rp, ci = oracle.mask_from_params(wl.mask)
     mp = wl.mask
     with build_mask(mp) if thr == 0 else _mask_with_thr(mp, thr) as m:
-        _check_plan(m, rp, ci, mp.n, mp.num_masks, 256 if thr == 0 else thr)
+        _check_plan(m, rp, ci, mp.n, mp.num_masks, 512 if thr == 0 else thr)
 
 
 def _mask_with_thr(mp, thr):
