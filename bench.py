@@ -86,7 +86,7 @@ def algorithmic_bytes(wl, nnz_total):
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples every 200 ms while the timed region runs."""
+    """nvidia-smi samples every 20 ms while the timed region runs."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -101,7 +101,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", self.device_id],
+                 "-lms", "20", "-i", self.device_id],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -144,12 +144,13 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- traffic
-def committed_traffic(kernel_file: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary for this workload,
-    or None when the kernel source changed since the capture (hash mismatch)."""
-    path = os.path.join(ROOT, "profiles", f"gather_fwd_{workload}.md")
+def committed_traffic(kernel_src: str, prefix: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this kernel and
+    workload, or None when the kernel source changed since the capture."""
+    path = os.path.join(ROOT, "profiles", f"{prefix}_{workload}.md")
     if not os.path.exists(path):
         return None
+    kernel_file = os.path.join(ROOT, "sparse_mask_scaled_b200", "csrc", kernel_src)
     want = hashlib.sha256(open(kernel_file, "rb").read()).hexdigest()[:16]
     vals = {}
     for ln in open(path):
@@ -251,6 +252,48 @@ class GpuWorkload:
                                        lse=self.lse if lse is None else lse)
 
 
+MUFU_EX2_PER_CLK_PER_SM = 16   # B200 special-function unit: 4 per SM sub-partition
+
+
+def forward_roofline(wl, plan, nnz_total, flops, alg_bytes, per_nnz, t_fwd_ms, hbm_peak, tc_peak, peak_src):
+    """Roofline of the forward's dominant kernel. With a tensor-core plan that
+    kernel is the tcgen05 tile kernel: bound 'tensor', achieved = the metric's
+    algorithmic FLOPs (4 * nnz * d) over the forward time against the measured
+    dense bf16 peak; the MMA FLOPs actually executed (whole 128 x 128 tiles) and
+    the exp2 rate against the special-function-unit peak are reported beside it.
+    Without tiles the gather kernel dominates: bound 'hbm', achieved = the
+    method's bytes (K and V row + column index per nonzero, q/out/lse/row pointer
+    per row) over the forward time against the measured copy bandwidth."""
+    rep = wl.B * wl.H if wl.mask.num_masks == 1 else wl.H
+    dt = "bf16" if wl.dtype == workloads.BF16 else "f32"
+    extra = wl.add_mask is not None or wl.bias is not None
+    t = t_fwd_ms * 1e-3
+    src_peak = "measured MEASURED_PEAKS.json" if peak_src == "measured" else "fallback"
+    if plan["tensor_core_tiles"] > 0 and wl.dtype == workloads.BF16:
+        kname = f"k_fwd_tc_pipe<{wl.d},{int(extra)}>" if wl.d <= 64 else f"k_fwd_tc<{wl.d}>"
+        tiles = plan["tensor_core_tiles"] * rep
+        mma_flops = tiles * 2 * (2 * 128 * 128 * wl.d)
+        ex2 = tiles * 128 * 128
+        sms, clk = 148, 1.965e9
+        achieved = flops / t / 1e12
+        return {"bound": "tensor", "achieved": round(achieved, 2), "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": round(achieved / tc_peak, 4),
+                "traffic": committed_traffic("fwd_tc.cu", "tc_fwd", wl.name),
+                "kernel": kname, "algorithmic_flop_per_launch": flops,
+                "mma_flop_executed_per_launch": mma_flops,
+                "mma_tflops_executed": round(mma_flops / t / 1e12, 2),
+                "ex2_per_launch": ex2,
+                "ex2_frac_of_sfu_peak": round(ex2 / t / (sms * MUFU_EX2_PER_CLK_PER_SM * clk), 4),
+                "effective_gbs": round(alg_bytes / t / 1e9, 1),
+                "peak_source": f"bf16_tflops ({src_peak}, burst: the kernel runs for well under a second)"}
+    achieved = alg_bytes / t / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+            "frac": round(achieved / hbm_peak, 4),
+            "traffic": committed_traffic("fwd_gather.cu", "gather_fwd", wl.name),
+            "kernel": f"k_fwd_short<{dt},{wl.d}>", "algorithmic_bytes_per_launch": alg_bytes,
+            "bytes_per_nnz": per_nnz, "peak_source": f"hbm_gbs ({src_peak})"}
+
+
 def kernel_launches_per_step(wl, n_long):
     """Kernels of this library launched by one step (mask build + forward)."""
     kind = wl.mask.kind
@@ -266,9 +309,28 @@ def kernel_launches_per_step(wl, n_long):
     return build + fwd, fwd
 
 
+def replica_seed(config: int, rank: int) -> int:
+    """Each rank runs its own replica of the workload (rank 0: the standard seed)."""
+    return 1000 + config + 7919 * rank
+
+
+def max_over_ranks(values, torch, device, world: int):
+    """Element-wise maximum of per-rank timings (the slowest rank sets the time)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_value(world: int, flop_per_step: float, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: the work of all ranks over the slowest rank's step time."""
+    return world * flop_per_step / (ms_per_step * 1e-3) / 1e12
+
+
 def bench_ours(args, rank, world, torch, sp):
     dev = torch.cuda.current_device()
-    wl = workloads.make(args.config, seed=(1000 + args.config) if rank == 0 else 1000 + args.config + 7919 * rank)
+    wl = workloads.make(args.config, seed=replica_seed(args.config, rank))
     g = GpuWorkload(wl, torch, sp)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
@@ -327,23 +389,18 @@ def bench_ours(args, rank, world, torch, sp):
     # ---- end to end: pinned host inputs -> device -> step -> host result
     e2e = e2e_measure(args, g, torch, stream, flush, flops)
 
-    t_max = t_total
-    if world > 1:
-        tt = torch.tensor([t_total, e2e["ms_per_step"]], dtype=torch.float64, device="cuda")
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        t_max, e2e_max = float(tt[0]), float(tt[1])
-        e2e["ms_per_step"] = e2e_max
+    t_max, e2e["ms_per_step"] = max_over_ranks([t_total, e2e["ms_per_step"]], torch, "cuda", world)
     ms_per_step = t_max / args.steps
-    value = world * flops / (ms_per_step * 1e-3) / 1e12
-    e2e_value = world * flops / (e2e["ms_per_step"] * 1e-3) / 1e12
+    value = job_value(world, flops, ms_per_step)
+    e2e_value = job_value(world, flops, e2e["ms_per_step"])
 
     alg_bytes, per_nnz = algorithmic_bytes(wl, nnz_total)
     hbm_peak, tc_peak, peak_src = measured_peaks()
-    achieved = alg_bytes / (t_fwd * 1e-3) / 1e9
-    kfile = os.path.join(ROOT, "sparse_mask_scaled_b200", "csrc", "fwd_gather.cu")
-    traffic = committed_traffic(kfile, wl.name)
+    eff_gbs = alg_bytes / (t_fwd * 1e-3) / 1e9
     launches, fwd_launches = kernel_launches_per_step(wl, n_long)
     clocks = clk.summary()
+    roofline = forward_roofline(wl, plan, nnz_total, flops, alg_bytes, per_nnz, t_fwd, hbm_peak, tc_peak,
+                                peak_src)
 
     result = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
@@ -358,12 +415,8 @@ def bench_ours(args, rank, world, torch, sp):
                    "step": "device mask build (pattern -> CSR -> row schedule + tile plan) + fused forward",
                    "plan_per_mask_set": plan},
         "fwd": {"ms": round(t_fwd, 4), "tflops": round(flops / (t_fwd * 1e-3) / 1e12, 3),
-                "effective_gbs": round(achieved, 1)},
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                     "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
-                     "kernel": f"k_fwd_short<{'bf16' if wl.dtype == workloads.BF16 else 'f32'},{wl.d}>",
-                     "algorithmic_bytes_per_launch": alg_bytes, "bytes_per_nnz": per_nnz,
-                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback 6.65 TB/s"},
+                "effective_gbs": round(eff_gbs, 1)},
+        "roofline": roofline,
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": round(e2e["ms_per_step"], 4)},
         "gpu_launches": launches * args.steps,

@@ -164,6 +164,125 @@ __global__ void k_residual_fill(const int32_t* __restrict__ row_ptr, const int32
     }
 }
 
+// ---------------------------------------------------------------------------
+// Interval rows (sliding window, variable window, dense): each row's columns are
+// one run [lo, hi), read from the row's first and last CSR entry. Counts, bits
+// and residual runs follow from the run's overlap with each tile, without
+// reading the rest of col_idx.
+
+__device__ __forceinline__ void row_run(const int32_t* __restrict__ row_ptr,
+                                        const int32_t* __restrict__ col_idx, int64_t r, int& lo,
+                                        int& hi) {
+    const int64_t p0 = row_ptr[r], p1 = row_ptr[r + 1];
+    if (p1 > p0) {
+        lo = col_idx[p0];
+        hi = col_idx[p1 - 1] + 1;
+    } else {
+        lo = hi = 0;
+    }
+}
+
+__device__ __forceinline__ int overlap(int lo, int hi, int c0, int c1) {
+    const int a = lo > c0 ? lo : c0, z = hi < c1 ? hi : c1;
+    return z > a ? z - a : 0;
+}
+
+// One warp per 32 rows of a query block: per-tile counts, one atomic per tile.
+__global__ void k_itv_count(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
+                            int n, int64_t nblocks, int nqb, int nkt, int32_t* __restrict__ cnt) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = nblocks * 4;
+    for (int64_t w = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5); w < nwarps;
+         w += (int64_t)gridDim.x * (blockDim.x >> 5)) {
+        const int64_t blk = w >> 2;
+        const int64_t m = blk / nqb;
+        const int i = (int)(blk - m * nqb) * kTileM + (int)(w & 3) * 32 + lane;
+        int lo = 0, hi = 0;
+        if (i < n) row_run(row_ptr, col_idx, m * n + i, lo, hi);
+        const bool any = hi > lo;
+        int k0 = any ? lo >> 7 : 0x7fffffff, k1 = any ? (hi - 1) >> 7 : -1;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            k0 = min(k0, __shfl_xor_sync(0xffffffffu, k0, off));
+            k1 = max(k1, __shfl_xor_sync(0xffffffffu, k1, off));
+        }
+        for (int kt = k0; kt <= k1; ++kt) {
+            int c = overlap(lo, hi, kt * kTileN, kt * kTileN + kTileN);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+            if (lane == 0 && c) atomicAdd(&cnt[blk * nkt + kt], c);
+        }
+    }
+}
+
+// One thread per row slot of every query block: the row's bits in each
+// selected (not dense) tile of its block -- zero words included, so the bit
+// array needs no clearing -- and its residual count.
+__global__ void k_itv_bits(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
+                           int n, int64_t nblocks, int nqb, const int32_t* __restrict__ block_tile_off,
+                           const int32_t* __restrict__ tile_info, uint32_t* __restrict__ bits,
+                           int32_t* __restrict__ res_cnt, int32_t* __restrict__ res_long,
+                           int32_t* __restrict__ res_n_long) {
+    for (int64_t x = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; x < nblocks * kTileM;
+         x += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t blk = x / kTileM;
+        const int row = (int)(x - blk * kTileM);
+        const int64_t m = blk / nqb;
+        const int i = (int)(blk - m * nqb) * kTileM + row;
+        int lo = 0, hi = 0;
+        if (i < n) row_run(row_ptr, col_idx, m * n + i, lo, hi);
+        int in_tiles = 0;
+        for (int t = block_tile_off[blk]; t < block_tile_off[blk + 1]; ++t) {
+            const int info = tile_info[t];
+            const int c0 = (info & 0x7fffffff) * kTileN;
+            in_tiles += overlap(lo, hi, c0, c0 + kTileN);
+            uint4* dst = reinterpret_cast<uint4*>(bits + ((int64_t)t * kTileM + row) * 4);
+            if (info < 0) {  // dense: the kernel reads no bits; store zero words
+                *dst = make_uint4(0u, 0u, 0u, 0u);
+                continue;
+            }
+            uint32_t w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int a = c0 + 32 * q;
+                const int lo2 = lo > a ? lo : a, hi2 = hi < a + 32 ? hi : a + 32;
+                const int len = hi2 - lo2;
+                w[q] = len <= 0 ? 0u : (len == 32 ? 0xffffffffu : (((1u << len) - 1u) << (lo2 - a)));
+            }
+            *dst = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        if (i < n) {
+            const int res = (hi - lo) - in_tiles;
+            res_cnt[m * n + i] = res;
+            if (res > kLongRowThreshold) res_long[atomicAdd(res_n_long, 1)] = (int32_t)(m * n + i);
+        }
+    }
+}
+
+// One thread per row: the residual runs (parts of [lo, hi) in unselected tiles).
+__global__ void k_itv_residual(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
+                               int n, int64_t rows, int nqb, int nkt, const int32_t* __restrict__ map,
+                               const int32_t* __restrict__ block_tile_off,
+                               const int32_t* __restrict__ res_row_ptr, int32_t* __restrict__ res_col,
+                               int32_t* __restrict__ n_mixed) {
+    for (int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; r < rows;
+         r += (int64_t)gridDim.x * blockDim.x) {
+        int64_t o = res_row_ptr[r];
+        if (res_row_ptr[r + 1] == o) continue;
+        const int64_t m = r / n, i = r - m * n;
+        const int64_t blk = m * nqb + (i >> 7);
+        int lo, hi;
+        row_run(row_ptr, col_idx, r, lo, hi);
+        for (int kt = lo >> 7; kt <= (hi - 1) >> 7; ++kt) {
+            if (map[blk * nkt + kt] >= 0) continue;
+            const int a = lo > kt * kTileN ? lo : kt * kTileN;
+            const int z = hi < kt * kTileN + kTileN ? hi : kt * kTileN + kTileN;
+            for (int j = a; j < z; ++j) res_col[o++] = j;
+        }
+        if (block_tile_off[blk + 1] > block_tile_off[blk]) atomicAdd(n_mixed, 1);
+    }
+}
+
 unsigned grid_for(int64_t work, int per_block, int64_t cap = 1 << 16) {
     int64_t g = (work + per_block - 1) / per_block;
     if (g < 1) g = 1;
@@ -180,16 +299,22 @@ int64_t plan_tile_capacity(int64_t nblocks, int nkt, int64_t nnz, int min_nnz) {
 }
 
 cudaError_t build_plan(const int32_t* row_ptr, const int32_t* col_idx, int n, int num_masks,
-                       int64_t nnz, int min_nnz, const PlanBuffers& b, PlanCounters* counters,
-                       cudaStream_t s) {
+                       int64_t nnz, int min_nnz, bool intervals, const PlanBuffers& b,
+                       PlanCounters* counters, cudaStream_t s) {
     const int64_t rows = (int64_t)num_masks * n;
     const int nqb = (n + kTileM - 1) / kTileM, nkt = (n + kTileN - 1) / kTileN;
     const int64_t nblocks = (int64_t)num_masks * nqb;
     cudaError_t e;
     if ((e = cudaMemsetAsync(b.cnt_map, 0, sizeof(int32_t) * nblocks * nkt, s)) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(b.tile_bits, 0, sizeof(uint32_t) * b.tile_cap * kTileM * 4, s)) != cudaSuccess)
-        return e;
-    k_tile_count<<<grid_for(rows, 8), 256, 0, s>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map);
+    if (intervals) {
+        k_itv_count<<<grid_for(nblocks * 4, 8), 256, 0, s>>>(row_ptr, col_idx, n, nblocks, nqb, nkt,
+                                                            b.cnt_map);
+    } else {
+        if ((e = cudaMemsetAsync(b.tile_bits, 0, sizeof(uint32_t) * b.tile_cap * kTileM * 4, s)) !=
+            cudaSuccess)
+            return e;
+        k_tile_count<<<grid_for(rows, 8), 256, 0, s>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k_tile_select<<<grid_for(nblocks, 128), 128, 0, s>>>(b.cnt_map, nblocks, nkt, min_nnz, b.block_ntiles,
                                                         &counters->n_tc_blocks);
@@ -200,15 +325,25 @@ cudaError_t build_plan(const int32_t* row_ptr, const int32_t* col_idx, int n, in
     k_tile_assign<<<grid_for(nblocks, 8), 256, 0, s>>>(b.cnt_map, nblocks, nkt, min_nnz,
                                                       b.block_tile_off, b.tile_info);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_tile_bits<<<grid_for(rows, 8), 256, 0, s>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map,
-                                                 b.tile_info, b.tile_bits, b.res_cnt, b.res_long,
-                                                 &counters->res_n_long);
+    if (intervals)
+        k_itv_bits<<<grid_for(nblocks * kTileM, 256), 256, 0, s>>>(
+            row_ptr, col_idx, n, nblocks, nqb, b.block_tile_off, b.tile_info, b.tile_bits, b.res_cnt,
+            b.res_long, &counters->res_n_long);
+    else
+        k_tile_bits<<<grid_for(rows, 8), 256, 0, s>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map,
+                                                     b.tile_info, b.tile_bits, b.res_cnt, b.res_long,
+                                                     &counters->res_n_long);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     e = scan_counts(b.res_cnt, rows, b.res_row_ptr, b.scan_tmp, &counters->res_nnz, &counters->err, s);
     if (e != cudaSuccess) return e;
-    k_residual_fill<<<grid_for(rows, 8), 256, 0, s>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map,
-                                                     b.block_tile_off, b.res_row_ptr, b.res_col_idx,
-                                                     &counters->n_mixed);
+    if (intervals)
+        k_itv_residual<<<grid_for(rows, 256), 256, 0, s>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map,
+                                                          b.block_tile_off, b.res_row_ptr, b.res_col_idx,
+                                                          &counters->n_mixed);
+    else
+        k_residual_fill<<<grid_for(rows, 8), 256, 0, s>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map,
+                                                         b.block_tile_off, b.res_row_ptr, b.res_col_idx,
+                                                         &counters->n_mixed);
     return cudaGetLastError();
 }
 

@@ -391,7 +391,10 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
             pb.res_cnt = c2.at<int32_t>(blk_t2, k_rc);
             e = cudaMemsetAsync(pc, 0, sizeof(PlanCounters), s);
             if (e == cudaSuccess)
-                e = build_plan(row_ptr, m->col_idx, sp.n, sp.num_masks, hinfo.nnz, min_nnz, pb, pc, s);
+                e = build_plan(row_ptr, m->col_idx, sp.n, sp.num_masks, hinfo.nnz, min_nnz,
+                               sp.kind == SPATTN_MASK_SLIDING || sp.kind == SPATTN_MASK_VARWIN ||
+                                   sp.kind == SPATTN_MASK_DENSE,
+                               pb, pc, s);
             if (e == cudaSuccess) e = cudaMemcpyAsync(&hpc, pc, sizeof hpc, cudaMemcpyDeviceToHost, s);
             if (e == cudaSuccess) e = cudaStreamSynchronize(s);
         }

@@ -112,9 +112,11 @@ struct PlanCounters {  // device-side results
     unsigned err;
 };
 int64_t plan_tile_capacity(int64_t nblocks, int nkt, int64_t nnz, int min_nnz);
+// intervals: every row's columns form one contiguous run (sliding window,
+// variable window, dense), which lets the plan skip reading col_idx.
 cudaError_t build_plan(const int32_t* row_ptr, const int32_t* col_idx, int n, int num_masks,
-                       int64_t nnz, int min_nnz, const PlanBuffers& b, PlanCounters* counters,
-                       cudaStream_t s);
+                       int64_t nnz, int min_nnz, bool intervals, const PlanBuffers& b,
+                       PlanCounters* counters, cudaStream_t s);
 
 // ---------------------------------------------------------------- launchers
 // All launchers enqueue on `stream` and return the cudaGetLastError() result.

@@ -87,6 +87,8 @@ def _check_plan(mask, rp, ci, n, nm, thr):
     (3, dict(B=1, H=1, n=1000), 0),         # block + strided + global
     (4, dict(B=2, H=1, n=256), 0),          # dense
     (2, dict(B=2, H=1, n=1000), 600),       # random: some tiles selected, rest residual
+    (1, dict(B=2, H=1, n=900), 9000),       # variable window (interval plan): window edges residual
+    (0, dict(B=1, H=1, n=333), 2000),       # sliding window (interval plan), ragged n
 ])
 def test_plan_partitions_the_csr(cfg, kw, thr):
     wl = workloads.make(cfg, **kw)
@@ -211,4 +213,22 @@ def test_evoformer_workload_on_tensor_cores():
         torch.cuda.synchronize()
     assert_close(to_f64(out).reshape(-1, wl.d), to_f64(lse), out_ref.reshape(-1, wl.d),
                  lse_ref.reshape(-1), wl.dtype, "evoformer")
+    assert sp.spattn_device_error() == 0
+
+
+@pytest.mark.parametrize("thr", [0, 9000, 12000])
+def test_variable_window_interval_plan_forward(thr):
+    """Variable window masks use the interval plan; high thresholds leave the
+    window edges to the gather kernel, so rows mix both paths."""
+    wl = workloads.make(1, B=2, H=3, n=1100)
+    q, k, v, _, _ = device_inputs(wl)
+    rp, ci = oracle.mask_from_params(wl.mask)
+    out_ref, lse_ref = oracle.masked_sdpa(wl.q.raw, wl.k.raw, wl.v.raw, rp, ci, wl.mask.num_masks, wl.scale)
+    with _mask_with_thr(wl.mask, thr) as m:
+        if thr == 9000:
+            assert m.n_tiles > 0 and m.n_mixed_rows > 0
+        out, lse = sp.spattn_fwd_mask(q, k, v, m, scale=wl.scale)
+        torch.cuda.synchronize()
+    assert_close(to_f64(out).reshape(-1, wl.d), to_f64(lse), out_ref.reshape(-1, wl.d),
+                 lse_ref.reshape(-1), wl.dtype, f"varwin thr={thr}")
     assert sp.spattn_device_error() == 0
