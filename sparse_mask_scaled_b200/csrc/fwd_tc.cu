@@ -78,6 +78,15 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
+__device__ __forceinline__ void tmem_wait_ld_dep16(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+}
+
 // Makes every use of r[] depend on the TMEM load having completed.
 __device__ __forceinline__ void tmem_wait_ld_dep(uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;"
@@ -497,20 +506,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ----------------------------------------------------------------------------
-// Pipelined variant for d <= 64, two threads per query row (8 warps per CTA).
-// O accumulates in registers (each thread owns d/2 of its row's columns),
-// which frees TMEM for two S buffers (2 x 128 columns, two CTAs per SM). Thread
-// (half, row) handles keys 64*half .. 64*half + 63 of each tile. P V(u) is
-// written into S(u)'s buffer once softmax(u) has finished with it, and S(u+1)
-// is issued in the middle of softmax(u), so the tensor core computes the next
-// tile's scores while the threads exponentiate the current one:
-//   softmax(u): wait S(u) | pass 1 (scale, mask, partial max; x back to TMEM) |
-//               wait P V(u-1), add it to O | partial max out | sync ->
-//               issue S(u+1) | row max | pass 2 (exp2, sum, P to smem) |
-//               sync -> issue P V(u), K(u+2)
-// The partial maxima travel through the P buffer: thread (h, r) leaves its
-// value in row r of P chunk 1-h, which only its partner (1-h, r) reads and
-// later overwrites with its own P.
+// Main variant for d <= 64: two threads per query row (8 warps per CTA, two CTAs
+// per SM). Thread (half, row) handles keys 64*half .. 64*half + 63 of each tile
+// and O columns half*d/2 .. of its row. Per tile:
+//   wait S(u) | load its 64 scores into registers (one TMEM round trip) | scale,
+//   add mask/bias, drop unlisted entries, partial max | wait P V(u-1) |
+//   partial max to the partner (through the P buffer) | sync -> issue S(u+1)
+//   (the S columns are free: the scores are in registers) | row max; if it grew
+//   by more than 2^8, rescale O in TMEM | exp2, partial sum, P to smem | sync ->
+//   issue P V(u) accumulating into O in TMEM, and K(u+2)
+// O stays in TMEM (M = 128, N = d accumulator) for the whole block, so no tile
+// needs to read it back.
 constexpr int kPipeThreads = 256;
 
 template <int D, bool EXTRA>
@@ -518,13 +524,13 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
     k_fwd_tc_pipe(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const TcParams P) {
     using C = TcCfg<D>;
-    static_assert(D <= 64, "O is kept in registers");
+    static_assert(D <= 64, "two threads per row split d/2 O columns each");
     constexpr int DH = D / 2;  // O columns per thread
     extern __shared__ __align__(1024) uint8_t smem[];
 
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int half = warp >> 2;       // key half of each tile (and O column half)
-    const int row = tid & 127;        // query row in the block == TMEM lane
+    const int half = warp >> 2;  // key half of each tile (and O column half)
+    const int row = tid & 127;   // query row in the block == TMEM lane
     const int bh = blockIdx.x / P.nqb, qb = blockIdx.x - bh * P.nqb;
     const int b = bh / P.H, h = bh - b * P.H;
     const int mk = P.num_masks == 1 ? 0 : b;
@@ -541,18 +547,19 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
     const uint32_t sK0 = smem_u32(smem + C::OFF_K), sV0 = smem_u32(smem + C::OFF_V);
     const uint32_t sP = smem_u32(smem + C::OFF_P);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-    // barriers: Q, K[2], V[2], S[2], O
+    // barriers: Q, K[2], V[2], S, O
     const uint32_t barQ = smem_u32(bars + 0), barK0 = smem_u32(bars + 1), barV0 = smem_u32(bars + 3),
-                   barS0 = smem_u32(bars + 5), barO = smem_u32(bars + 7);
+                   barS = smem_u32(bars + 5), barO = smem_u32(bars + 6);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    // partner exchange slot: row `row` of P chunk (1 - half), first 16 bytes (swizzled)
+    // partner exchange slot: row `row` of P chunk (1 - half), first 16 bytes (swizzled);
+    // only the partner reads it, and the partner overwrites it with its own P later
     const uint32_t my_slot = sP + (uint32_t)((half ^ 1) * 16384 + row * 128 + ((0 ^ (row & 7)) << 4));
     const uint32_t partner_slot = sP + (uint32_t)(half * 16384 + row * 128 + ((0 ^ (row & 7)) << 4));
 
     if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     if (tid == 0) {
-        for (int x = 0; x < 8; ++x) mbar_init(smem_u32(bars + x), 1);
+        for (int x = 0; x < 7; ++x) mbar_init(smem_u32(bars + x), 1);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&tmQ);
@@ -563,10 +570,11 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const uint32_t tS = tmem, tO = tmem + 128;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
 
     // thread 0: issued operations per barrier (scalars: no dynamically indexed arrays)
-    int n_k0 = 0, n_k1 = 0, n_v0 = 0, n_v1 = 0, n_s0 = 0, n_s1 = 0, n_pv = 0;
+    int n_k0 = 0, n_k1 = 0, n_v0 = 0, n_v1 = 0, n_s = 0, n_pv = 0;
 
     auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
         if (*abort_flag) return false;
@@ -589,28 +597,26 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
     };
     const uint32_t idS = idesc_bf16_f32(128, 128, false);
     const uint32_t idO = idesc_bf16_f32(128, D, true);
-    auto issue_S = [&](int u) {  // S(u) into TMEM buffer u & 1
+    auto issue_S = [&](int u) {
         const uint32_t sK = sK0 + (uint32_t)((u & 1) * C::TILE_BYTES);
-        const uint32_t dst = tmem + 128u * (u & 1);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
             const uint64_t da = smem_desc(sQ + ks * 32, 16, C::SBO, C::LAYOUT);
             const uint64_t db = smem_desc(sK + ks * 32, 16, C::SBO, C::LAYOUT);
-            mma_bf16_ss(dst, da, db, idS, ks > 0 ? 1u : 0u);
+            mma_bf16_ss(tS, da, db, idS, ks > 0 ? 1u : 0u);
         }
-        mma_commit(barS0 + 8u * (u & 1));
-        if (u & 1) ++n_s1; else ++n_s0;
+        mma_commit(barS);
+        ++n_s;
     };
-    auto issue_PV = [&](int u) {  // P V(u) into columns [0, D) of TMEM buffer u & 1
+    auto issue_PV = [&](int u) {
         const uint32_t sV = sV0 + (uint32_t)((u & 1) * C::TILE_BYTES);
-        const uint32_t dst = tmem + 128u * (u & 1);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
             const uint64_t da = smem_desc(sP + (uint32_t)((ks >> 2) * 16384 + (ks & 3) * 32), 16, 1024,
                                           cute::UMMA::LayoutType::SWIZZLE_128B);
             const uint64_t db = smem_desc(sV + (uint32_t)(ks * 16 * C::ROW_BYTES), C::CHUNK_BYTES, C::SBO,
                                           C::LAYOUT);
-            mma_bf16_ss(dst, da, db, idO, ks > 0 ? 1u : 0u);
+            mma_bf16_ss(tO, da, db, idO, (u > 0 || ks > 0) ? 1u : 0u);
         }
         mma_commit(barO);
         ++n_pv;
@@ -636,35 +642,6 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
     const int64_t mask_rowbase = (int64_t)b * P.mask.s0 + (int64_t)h * P.mask.s1 + (int64_t)i * P.mask.s2;
     const int64_t bias_rowbase = (int64_t)b * P.bias.s0 + (int64_t)h * P.bias.s1 + (int64_t)i * P.bias.s2;
     float m_ref = -INFINITY, l = 0.f;  // l: this thread's half of the row sum
-    float mu_o = 0.f, mu_prev = 0.f;   // reference of O's contents / of the last P
-    float o[DH];
-#pragma unroll
-    for (int e = 0; e < DH; ++e) o[e] = 0.f;
-
-    // adds this thread's columns of P V(u) (TMEM buffer u & 1) to O, rescaled to P(u)'s reference
-    auto accumulate_pv = [&](int u) {
-        const float f = ex2(mu_o - mu_prev);
-        const uint32_t src = tmem + 128u * (u & 1) + lane_base + half * DH;
-        if constexpr (DH == 32) {
-            uint32_t r[32];
-            tmem_ld32(src, r);
-            tmem_wait_ld_dep(r);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = fmaf(o[j], f, __uint_as_float(r[j]));
-        } else {
-            uint32_t r[16];
-            tmem_ld16(src, r);
-            asm volatile("tcgen05.wait::ld.sync.aligned;"
-                         : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
-                           "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
-                           "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
-                         :
-                         : "memory");
-#pragma unroll
-            for (int j = 0; j < 16; ++j) o[j] = fmaf(o[j], f, __uint_as_float(r[j]));
-        }
-        mu_o = mu_prev;
-    };
 
     int next_info = P.tile_info[t_begin];
     uint2 next_bits = make_uint2(0u, 0u);
@@ -684,64 +661,55 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
         const int kt = info & 0x7fffffff;
         const bool dense = info < 0;
         const bool extra = EXTRA && row_ok;
-        const uint32_t bw[2] = {wbits.x, wbits.y};
-        const uint32_t tS = tmem + 128u * (u & 1) + lane_base + half * 64;
 
-        wait(barS0 + 8u * (u & 1), (uint32_t)((u >> 1) & 1));
+        float x[64];
+
+        wait(barS, (uint32_t)(u & 1));
         tc_fence_after();
+        if (tid == 0 && u + 2 < T && !*abort_flag) issue_k(u + 2);  // S(u) consumed K(u)
         __syncwarp();
-        // pass 1: x = scale*log2(e)*S (+ log2(e)*(mask + bias)), unlisted entries -inf,
-        // partial max; x goes back into TMEM
+        {
+            uint32_t r0[32], r1[32];
+            tmem_ld32(tS + lane_base + half * 64, r0);
+            tmem_ld32(tS + lane_base + half * 64 + 32, r1);
+            tmem_wait_ld_dep(r0);
+            tmem_wait_ld_dep(r1);
+            // x = scale*log2(e)*S, two lanes per instruction
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                mul2(x[2 * k], x[2 * k + 1], r0[2 * k], r0[2 * k + 1], c2);
+                mul2(x[32 + 2 * k], x[33 + 2 * k], r1[2 * k], r1[2 * k + 1], c2);
+            }
+        }
+        if (extra) {  // + log2(e) * (mask + bias)
+            const int c0 = kt * 128 + half * 64;
+            const int ncols = P.n - c0 < 64 ? P.n - c0 : 64;
+            if (P.mask.data) add_addend_run<64>(P.mask, mask_rowbase, c0, ncols, x);
+            if (P.bias.data) add_addend_run<64>(P.bias, bias_rowbase, c0, ncols, x);
+        }
+        if (!dense) {  // entries the CSR does not list
+            const uint32_t bw[2] = {wbits.x, wbits.y};
+#pragma unroll
+            for (int j = 0; j < 64; ++j) x[j] = ((bw[j >> 5] >> (j & 31)) & 1u) ? x[j] : -INFINITY;
+        }
         float ma = -INFINITY, mb = -INFINITY, mc = -INFINITY, md = -INFINITY;
 #pragma unroll
-        for (int qtr = 0; qtr < 2; ++qtr) {  // 32 columns at a time
-            float xq[32];
-            if (extra) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) xq[j] = 0.f;
-                const int c0 = kt * 128 + half * 64 + qtr * 32;
-                const int ncols = P.n - c0 < 32 ? P.n - c0 : 32;
-                if (P.mask.data) add_addend_run<32>(P.mask, mask_rowbase, c0, ncols, xq);
-                if (P.bias.data) add_addend_run<32>(P.bias, bias_rowbase, c0, ncols, xq);
-            }
-            uint32_t r0[32];
-            tmem_ld32(tS + qtr * 32, r0);
-            tmem_wait_ld_dep(r0);
-            if (extra) {
-#pragma unroll
-                for (int k = 0; k < 16; ++k) fma2_inplace(xq[2 * k], xq[2 * k + 1], r0[2 * k], r0[2 * k + 1], c2);
-            } else {
-#pragma unroll
-                for (int k = 0; k < 16; ++k) mul2(xq[2 * k], xq[2 * k + 1], r0[2 * k], r0[2 * k + 1], c2);
-            }
-            if (!dense) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) xq[j] = ((bw[qtr] >> j) & 1u) ? xq[j] : -INFINITY;
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                ma = fmax3(ma, xq[8 * k + 0], xq[8 * k + 1]);
-                mb = fmax3(mb, xq[8 * k + 2], xq[8 * k + 3]);
-                mc = fmax3(mc, xq[8 * k + 4], xq[8 * k + 5]);
-                md = fmax3(md, xq[8 * k + 6], xq[8 * k + 7]);
-            }
-#pragma unroll
-            for (int j = 0; j < 32; ++j) r0[j] = __float_as_uint(xq[j]);
-            tmem_st32(tS + qtr * 32, r0);
+        for (int k = 0; k < 8; ++k) {
+            ma = fmax3(ma, x[8 * k + 0], x[8 * k + 1]);
+            mb = fmax3(mb, x[8 * k + 2], x[8 * k + 3]);
+            mc = fmax3(mc, x[8 * k + 4], x[8 * k + 5]);
+            md = fmax3(md, x[8 * k + 6], x[8 * k + 7]);
         }
-        tmem_wait_st();
         const float my_max = fmax3(ma, mb, fmaxf(mc, md));
 
-        if (u > 0) {  // P V(u-1) is in the other buffer; V(u-1)'s buffer is free after it
+        if (u > 0) {  // P V(u-1) must be done: it reads sP and accumulates into O
             wait(barO, (uint32_t)((u - 1) & 1));
             tc_fence_after();
-            if (tid == 0 && u + 1 < T && !*abort_flag) issue_v(u + 1);
+            if (tid == 0 && u + 1 < T && !*abort_flag) issue_v(u + 1);  // V(u-1)'s buffer is free
             __syncwarp();
-            accumulate_pv(u - 1);
         }
-        // sP is free (P V(u-1) done): leave the partial max for the partner
         asm volatile("st.shared.f32 [%0], %1;" ::"r"(my_slot), "f"(my_max) : "memory");
-        // mid-tile: the other TMEM buffer is free -> S(u+1) runs while this tile exponentiates
+        // the S columns are free (scores are in registers): S(u+1) runs during exp2
         tc_fence_before();
         __syncthreads();
         if (tid == 0 && u + 1 < T && !*abort_flag) {
@@ -755,26 +723,45 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
         float other_max;
         asm volatile("ld.shared.f32 %0, [%1];" : "=f"(other_max) : "r"(partner_slot) : "memory");
         const float mx = fmaxf(my_max, other_max);
-        if (mx > m_ref + kRescaleThreshold) {
-            l *= ex2(m_ref - mx);
+        const bool need = mx > m_ref + kRescaleThreshold;
+        float alpha = 1.f;
+        if (need) {
+            alpha = ex2(m_ref - mx);
             m_ref = mx;
+            l *= alpha;
+        }
+        if (u > 0 && __any_sync(0xffffffffu, need)) {  // O holds P V(0..u-1): bring it to the new max
+            const uint32_t src = tO + lane_base + half * DH;
+            if constexpr (DH == 32) {
+                uint32_t ro[32];
+                tmem_ld32(src, ro);
+                tmem_wait_ld_dep(ro);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) ro[j] = __float_as_uint(__uint_as_float(ro[j]) * alpha);
+                tmem_st32(src, ro);
+            } else {
+                uint32_t ro[16];
+                tmem_ld16(src, ro);
+                tmem_wait_ld_dep16(ro);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) ro[j] = __float_as_uint(__uint_as_float(ro[j]) * alpha);
+                tmem_st16(src, ro);
+            }
+            tmem_wait_st();
         }
         const float mu = m_ref == -INFINITY ? 0.f : m_ref;
-
-        // pass 2: p = exp2(x - mu), partial sum, P (bf16) into chunk `half` of the K-major,
+        // p = exp2(x - mu), partial sum, P (bf16) into chunk `half` of the K-major,
         // 128-byte-swizzled A operand layout
         const uint64_t nmu2 = pack2(-mu, -mu);
         uint64_t sa = pack2(0.f, 0.f), sb = sa;
 #pragma unroll
-        for (int qtr = 0; qtr < 2; ++qtr) {
-            uint32_t r0[32];
-            tmem_ld32(tS + qtr * 32, r0);
-            tmem_wait_ld_dep(r0);
-            uint32_t pk[16];
+        for (int piece = 0; piece < 8; ++piece) {
+            uint32_t pk[4];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
+            for (int t = 0; t < 4; ++t) {
+                const int k = piece * 4 + t;
                 float p0, p1;
-                unpack2(add2(pack2(__uint_as_float(r0[2 * k]), __uint_as_float(r0[2 * k + 1])), nmu2), p0, p1);
+                unpack2(add2(pack2(x[2 * k], x[2 * k + 1]), nmu2), p0, p1);
                 p0 = ex2(p0);
                 p1 = ex2(p1);
                 if (k & 1)
@@ -782,16 +769,12 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
                 else
                     sa = add2(sa, pack2(p0, p1));
                 __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
-                pk[k] = *reinterpret_cast<uint32_t*>(&hv);
+                pk[t] = *reinterpret_cast<uint32_t*>(&hv);
             }
-#pragma unroll
-            for (int pc = 0; pc < 4; ++pc) {
-                const int piece = qtr * 4 + pc;
-                const uint32_t addr = sP + (uint32_t)(half * 16384 + row * 128 + ((piece ^ (row & 7)) << 4));
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[pc * 4]),
-                             "r"(pk[pc * 4 + 1]), "r"(pk[pc * 4 + 2]), "r"(pk[pc * 4 + 3])
-                             : "memory");
-            }
+            const uint32_t addr = sP + (uint32_t)(half * 16384 + row * 128 + ((piece ^ (row & 7)) << 4));
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[0]), "r"(pk[1]),
+                         "r"(pk[2]), "r"(pk[3])
+                         : "memory");
         }
         {
             float s0, s1, s2, s3;
@@ -799,13 +782,11 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
             unpack2(sb, s2, s3);
             l += (s0 + s1) + (s2 + s3);
         }
-        mu_prev = mu;
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         if (tid == 0 && !*abort_flag) {
             tc_fence_after();
-            if (u + 2 < T) issue_k(u + 2);  // S(u) consumed K(u) long ago
             if (wait(barV0 + 8u * (u & 1), (uint32_t)((u >> 1) & 1))) {
                 tc_fence_after();
                 issue_PV(u);
@@ -817,7 +798,23 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
     wait(barO, (uint32_t)((T - 1) & 1));
     tc_fence_after();
     __syncwarp();
-    accumulate_pv(T - 1);
+    float o[DH];
+    {
+        const uint32_t src = tO + lane_base + half * DH;
+        if constexpr (DH == 32) {
+            uint32_t ro[32];
+            tmem_ld32(src, ro);
+            tmem_wait_ld_dep(ro);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __uint_as_float(ro[j]);
+        } else {
+            uint32_t ro[16];
+            tmem_ld16(src, ro);
+            tmem_wait_ld_dep16(ro);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) o[j] = __uint_as_float(ro[j]);
+        }
+    }
     // combine the two halves of the row sum (sP is free: the last P V is done)
     asm volatile("st.shared.f32 [%0], %1;" ::"r"(my_slot), "f"(l) : "memory");
     __syncthreads();
@@ -825,7 +822,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
     asm volatile("ld.shared.f32 %0, [%1];" : "=f"(l_other) : "r"(partner_slot) : "memory");
     const float l_row = l + l_other;
     if (row_ok && !*abort_flag) {
-        float M = m_ref, L = l_row, fa;
+        float M = m_ref, L = l_row, fa = 1.f;
         const int64_t mrow = (int64_t)mk * P.n + i;
         const int64_t wrow = (int64_t)bh * P.n + i;
         const bool mixed = P.ws_ml && P.res_row_ptr[mrow + 1] > P.res_row_ptr[mrow];
@@ -834,11 +831,9 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
             const float mg = P.ws_ml[wrow * 2], lg = P.ws_ml[wrow * 2 + 1];
             M = fmaxf(m_ref, mg);
             const float Mu = M == -INFINITY ? 0.f : M;
-            fa = ex2(mu_o - Mu);
+            fa = ex2(m_ref - Mu);
             fg = ex2(mg - Mu);
-            L = l_row * ex2(m_ref - Mu) + lg * fg;
-        } else {
-            fa = ex2(mu_o - (m_ref == -INFINITY ? 0.f : m_ref));
+            L = l_row * fa + lg * fg;
         }
         const float inv = L > 0.f ? 1.f / L : 0.f;
         __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(P.out) + (int64_t)b * P.o_sb +
@@ -867,10 +862,11 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
     // ------------------------------------------------------------ teardown
     if (tid == 0 && *abort_flag) {
         const long long lim = kWaitCycles / 16;
-        const int cnt[6] = {n_k0, n_k1, n_v0, n_v1, n_s0, n_s1};
-        const uint32_t bar6[6] = {barK0, barK0 + 8u, barV0, barV0 + 8u, barS0, barS0 + 8u};
-        for (int x = 0; x < 6; ++x)
-            if (cnt[x]) mbar_wait_bounded(bar6[x], (uint32_t)((cnt[x] - 1) & 1), lim);
+        const int cnt[4] = {n_k0, n_k1, n_v0, n_v1};
+        const uint32_t bar4[4] = {barK0, barK0 + 8u, barV0, barV0 + 8u};
+        for (int x = 0; x < 4; ++x)
+            if (cnt[x]) mbar_wait_bounded(bar4[x], (uint32_t)((cnt[x] - 1) & 1), lim);
+        if (n_s) mbar_wait_bounded(barS, (uint32_t)((n_s - 1) & 1), lim);
         if (n_pv) mbar_wait_bounded(barO, (uint32_t)((n_pv - 1) & 1), lim);
         atomicOr(P.err, kErrTimeout);
     }

@@ -319,25 +319,41 @@ __device__ __forceinline__ int64_t block_exclusive_scan(int64_t x, int64_t* tota
     return res;
 }
 
-// Arrays up to kScanSmallMax: a single block scans tile after tile.
-constexpr int64_t kScanSmallMax = 16 * kScanTile;
+// Arrays up to kScanSmallMax: a single block scans them, 16 consecutive
+// counts per thread per pass (one pass up to 16,384 counts), carrying the
+// running total from pass to pass.
+constexpr int kSmallItems = 16;
+constexpr int64_t kScanSmallTile = (int64_t)kScanThreads * kSmallItems;
+constexpr int64_t kScanSmallMax = 4 * kScanSmallTile;
 
 __global__ void __launch_bounds__(kScanThreads)
     k_scan_small(const int32_t* __restrict__ counts, int64_t rows, int32_t* __restrict__ out,
                  int64_t* total_out, unsigned* err) {
     int64_t carry = 0;
-    for (int64_t t0 = 0; t0 < rows; t0 += kScanTile) {
-        const int64_t base = t0 + (int64_t)threadIdx.x * kScanItems;
-        int64_t v[kScanItems], sum = 0;
+    for (int64_t t0 = 0; t0 < rows; t0 += kScanSmallTile) {
+        const int64_t base = t0 + (int64_t)threadIdx.x * kSmallItems;
+        int32_t v[kSmallItems];
+        int64_t sum = 0;
+        if (base + kSmallItems <= rows && (base & 3) == 0) {
+            const int4* p = reinterpret_cast<const int4*>(counts + base);
 #pragma unroll
-        for (int t = 0; t < kScanItems; ++t) {
-            v[t] = base + t < rows ? counts[base + t] : 0;
-            sum += v[t];
+            for (int t = 0; t < kSmallItems / 4; ++t) {
+                const int4 w = __ldg(p + t);
+                v[4 * t] = w.x;
+                v[4 * t + 1] = w.y;
+                v[4 * t + 2] = w.z;
+                v[4 * t + 3] = w.w;
+            }
+        } else {
+#pragma unroll
+            for (int t = 0; t < kSmallItems; ++t) v[t] = base + t < rows ? counts[base + t] : 0;
         }
+#pragma unroll
+        for (int t = 0; t < kSmallItems; ++t) sum += v[t];
         int64_t total;
         int64_t run = carry + block_exclusive_scan(sum, &total);
 #pragma unroll
-        for (int t = 0; t < kScanItems; ++t) {
+        for (int t = 0; t < kSmallItems; ++t) {
             if (base + t < rows) out[base + t] = run > INT_MAX ? INT_MAX : (int32_t)run;
             run += v[t];
         }

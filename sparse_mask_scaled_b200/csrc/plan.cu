@@ -283,6 +283,93 @@ __global__ void k_itv_residual(const int32_t* __restrict__ row_ptr, const int32_
     }
 }
 
+// One block: select the tiles of every query block, number them (block-major,
+// key tiles ascending), write block_tile_off and the tile map -- the work of
+// k_tile_select + scan + k_tile_assign in one launch, for block grids up to
+// kFusedSelectMax query blocks.
+constexpr int kFusedSelectMax = 1 << 16;
+
+__global__ void __launch_bounds__(1024)
+    k_tile_select_fused(int32_t* __restrict__ cnt_map, int nblocks, int nkt, int min_nnz,
+                        int32_t* __restrict__ block_tile_off, int32_t* __restrict__ tile_info,
+                        PlanCounters* counters) {
+    __shared__ int32_t wsum[32];
+    __shared__ int32_t carry_s;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) carry_s = 0;
+    __syncthreads();
+    int tc_blocks = 0;
+    // pass 1: per-block selected counts, scanned into block_tile_off
+    for (int x0 = 0; x0 < nblocks; x0 += 1024) {
+        const int x = x0 + threadIdx.x;
+        int c = 0;
+        if (x < nblocks)
+            for (int kt = 0; kt < nkt; ++kt) c += cnt_map[(int64_t)x * nkt + kt] >= min_nnz;
+        tc_blocks += c > 0;
+        int inc = c;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, inc, off);
+            if (lane >= off) inc += y;
+        }
+        if (lane == 31) wsum[warp] = inc;
+        __syncthreads();
+        if (warp == 0) {
+            const int w = wsum[lane];
+            int wi = w;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, wi, off);
+                if (lane >= off) wi += y;
+            }
+            wsum[lane] = wi - w;
+        }
+        __syncthreads();
+        const int carry = carry_s;
+        if (x < nblocks) block_tile_off[x] = carry + wsum[warp] + inc - c;
+        __syncthreads();
+        if (threadIdx.x == 1023) carry_s = carry + wsum[warp] + inc;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        block_tile_off[nblocks] = carry_s;
+        counters->n_tiles = carry_s;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) tc_blocks += __shfl_xor_sync(0xffffffffu, tc_blocks, off);
+    if (lane == 0 && tc_blocks) atomicAdd(&counters->n_tc_blocks, tc_blocks);
+    __syncthreads();
+    // pass 2: one warp per block numbers its selected tiles
+    for (int x = warp; x < nblocks; x += 32) {
+        int idx = block_tile_off[x];
+        for (int k0 = 0; k0 < nkt; k0 += 32) {
+            const int kt = k0 + lane;
+            const int c = kt < nkt ? cnt_map[(int64_t)x * nkt + kt] : 0;
+            const bool sel = kt < nkt && c >= min_nnz;
+            const unsigned bal = __ballot_sync(0xffffffffu, sel);
+            if (kt < nkt) {
+                if (sel) {
+                    const int id = idx + __popc(bal & ((1u << lane) - 1u));
+                    tile_info[id] = kt | (c == kTileM * kTileN ? (int)kTileDenseBit : 0);
+                    cnt_map[(int64_t)x * nkt + kt] = id;
+                } else {
+                    cnt_map[(int64_t)x * nkt + kt] = -1;
+                }
+            }
+            idx += __popc(bal);
+        }
+    }
+}
+
+// Clears the tile count array and the plan counters.
+__global__ void k_plan_zero(int32_t* __restrict__ cnt, int64_t n_cnt, PlanCounters* counters) {
+    for (int64_t x = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; x < n_cnt;
+         x += (int64_t)gridDim.x * blockDim.x)
+        cnt[x] = 0;
+    if (blockIdx.x == 0 && threadIdx.x < sizeof(PlanCounters) / 4)
+        reinterpret_cast<uint32_t*>(counters)[threadIdx.x] = 0u;
+}
+
 unsigned grid_for(int64_t work, int per_block, int64_t cap = 1 << 16) {
     int64_t g = (work + per_block - 1) / per_block;
     if (g < 1) g = 1;
@@ -305,7 +392,8 @@ cudaError_t build_plan(const int32_t* row_ptr, const int32_t* col_idx, int n, in
     const int nqb = (n + kTileM - 1) / kTileM, nkt = (n + kTileN - 1) / kTileN;
     const int64_t nblocks = (int64_t)num_masks * nqb;
     cudaError_t e;
-    if ((e = cudaMemsetAsync(b.cnt_map, 0, sizeof(int32_t) * nblocks * nkt, s)) != cudaSuccess) return e;
+    k_plan_zero<<<grid_for(nblocks * nkt, 256, 1024), 256, 0, s>>>(b.cnt_map, nblocks * nkt, counters);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (intervals) {
         k_itv_count<<<grid_for(nblocks * 4, 8), 256, 0, s>>>(row_ptr, col_idx, n, nblocks, nqb, nkt,
                                                             b.cnt_map);
@@ -316,14 +404,19 @@ cudaError_t build_plan(const int32_t* row_ptr, const int32_t* col_idx, int n, in
         k_tile_count<<<grid_for(rows, 8), 256, 0, s>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_tile_select<<<grid_for(nblocks, 128), 128, 0, s>>>(b.cnt_map, nblocks, nkt, min_nnz, b.block_ntiles,
-                                                        &counters->n_tc_blocks);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    e = scan_counts(b.block_ntiles, nblocks, b.block_tile_off, b.scan_tmp, &counters->n_tiles,
-                    &counters->err, s);
-    if (e != cudaSuccess) return e;
-    k_tile_assign<<<grid_for(nblocks, 8), 256, 0, s>>>(b.cnt_map, nblocks, nkt, min_nnz,
-                                                      b.block_tile_off, b.tile_info);
+    if (nblocks <= kFusedSelectMax) {
+        k_tile_select_fused<<<1, 1024, 0, s>>>(b.cnt_map, (int)nblocks, nkt, min_nnz, b.block_tile_off,
+                                               b.tile_info, counters);
+    } else {
+        k_tile_select<<<grid_for(nblocks, 128), 128, 0, s>>>(b.cnt_map, nblocks, nkt, min_nnz,
+                                                            b.block_ntiles, &counters->n_tc_blocks);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = scan_counts(b.block_ntiles, nblocks, b.block_tile_off, b.scan_tmp, &counters->n_tiles,
+                        &counters->err, s);
+        if (e != cudaSuccess) return e;
+        k_tile_assign<<<grid_for(nblocks, 8), 256, 0, s>>>(b.cnt_map, nblocks, nkt, min_nnz,
+                                                          b.block_tile_off, b.tile_info);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (intervals)
         k_itv_bits<<<grid_for(nblocks * kTileM, 256), 256, 0, s>>>(

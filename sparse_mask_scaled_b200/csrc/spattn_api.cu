@@ -389,9 +389,7 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
             pb.block_ntiles = c2.at<int32_t>(blk_t2, k_bn);
             pb.scan_tmp = c2.at<int64_t>(blk_t2, k_st);
             pb.res_cnt = c2.at<int32_t>(blk_t2, k_rc);
-            e = cudaMemsetAsync(pc, 0, sizeof(PlanCounters), s);
-            if (e == cudaSuccess)
-                e = build_plan(row_ptr, m->col_idx, sp.n, sp.num_masks, hinfo.nnz, min_nnz,
+            e = build_plan(row_ptr, m->col_idx, sp.n, sp.num_masks, hinfo.nnz, min_nnz,
                                sp.kind == SPATTN_MASK_SLIDING || sp.kind == SPATTN_MASK_VARWIN ||
                                    sp.kind == SPATTN_MASK_DENSE,
                                pb, pc, s);
