@@ -294,21 +294,6 @@ def forward_roofline(wl, plan, nnz_total, flops, alg_bytes, per_nnz, t_fwd_ms, h
             "bytes_per_nnz": per_nnz, "peak_source": f"hbm_gbs ({src_peak})"}
 
 
-def kernel_launches_per_step(wl, n_long):
-    """Kernels of this library launched by one step (mask build + forward)."""
-    kind = wl.mask.kind
-    build = {"sliding": 1, "varwin": 1, "dense": 1, "bsg": 1, "coo": 1}[kind]   # counts / sort
-    if kind == "coo" and int(wl.mask.cand_row_ptr[-1]) + 1 > 1024:
-        build += 1                                                            # long COO rows
-    build += 3                      # scan: tiles, tile sums, finalize
-    build += 1                      # fill
-    if kind == "bsg":
-        build += 1                  # ordered walk of non-global rows
-    build += 1                      # long-row classification
-    fwd = 1 + (1 if n_long > 0 else 0)
-    return build + fwd, fwd
-
-
 def replica_seed(config: int, rank: int) -> int:
     """Each rank runs its own replica of the workload (rank 0: the standard seed)."""
     return 1000 + config + 7919 * rank
@@ -338,7 +323,6 @@ def bench_ours(args, rank, world, torch, sp):
     # mask statistics (same for every step)
     with g.create() as m0:
         nnz_masks = m0.nnz
-        n_long = m0.n_long
         plan = {"tensor_core_tiles": m0.n_tiles, "residual_nnz": m0.residual_nnz,
                 "mixed_rows": m0.n_mixed_rows}
     # nnz summed over (b, h): every head shares its batch element's mask
@@ -367,6 +351,7 @@ def bench_ours(args, rank, world, torch, sp):
     torch.cuda.synchronize()
     starts, ends, fwd_evs = [], [], []
     smi_id = _smi_id(torch, dev)
+    launches0 = sp.spattn_launch_count()
     with ClockSampler(smi_id) as clk:
         for _ in range(args.steps):
             flush.zero_()                      # evict L2 between steps (outside the events)
@@ -378,6 +363,7 @@ def bench_ours(args, rank, world, torch, sp):
             starts.append(s)
             ends.append(e)
         torch.cuda.synchronize()
+    launches = sp.spattn_launch_count() - launches0    # kernels the library enqueued while timed
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -397,7 +383,6 @@ def bench_ours(args, rank, world, torch, sp):
     alg_bytes, per_nnz = algorithmic_bytes(wl, nnz_total)
     hbm_peak, tc_peak, peak_src = measured_peaks()
     eff_gbs = alg_bytes / (t_fwd * 1e-3) / 1e9
-    launches, fwd_launches = kernel_launches_per_step(wl, n_long)
     clocks = clk.summary()
     roofline = forward_roofline(wl, plan, nnz_total, flops, alg_bytes, per_nnz, t_fwd, hbm_peak, tc_peak,
                                 peak_src)
@@ -419,7 +404,7 @@ def bench_ours(args, rank, world, torch, sp):
         "roofline": roofline,
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": round(e2e["ms_per_step"], 4)},
-        "gpu_launches": launches * args.steps,
+        "gpu_launches": launches,
         "clocks": clocks,
     }
     return result, wl

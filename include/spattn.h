@@ -243,6 +243,11 @@ int spattn_device_error(void* stream, uint32_t* flags);
 /* Library version: major * 10000 + minor * 100 + patch. */
 int spattn_version(void);
 
+/* Number of kernels this library has enqueued since it was loaded, over all
+ * threads and devices (a diagnostic with no counterpart in the method: it lets
+ * a caller count the launches a sequence of calls costs). Never fails. */
+uint64_t spattn_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

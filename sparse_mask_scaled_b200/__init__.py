@@ -5,7 +5,7 @@ This module only marshals arguments: torch tensors become ``spattn_tensor``
 descriptors (pointer, dtype, shape, strides) and Python numbers become C
 integers/floats. Every step of the computation runs in libspattn's CUDA kernels;
 there is no fallback. Importing the module fails if ``libspattn.so`` has not been
-built (``python -m sparse_mask_scaled_b200._build``).
+built (``python sparse_mask_scaled_b200/_build.py``).
 
 PyTorch provides device memory and streams only.
 """
@@ -89,15 +89,19 @@ SIGNATURES = {
     "spattn_last_error": (ctypes.c_char_p, []),
     "spattn_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "spattn_version": (ctypes.c_int, []),
+    "spattn_launch_count": (ctypes.c_uint64, []),
 }
 
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m sparse_mask_scaled_b200._build`"
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python sparse_mask_scaled_b200/_build.py`"
                           " (the CUDA library is required; there is no fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in SIGNATURES.items():
+        if not hasattr(lib, name):
+            raise ImportError(f"{LIB_PATH} does not export {name}: it is older than the sources,"
+                              " rebuild it with `python sparse_mask_scaled_b200/_build.py`")
         fn = getattr(lib, name)
         fn.restype = res
         fn.argtypes = args
@@ -300,3 +304,8 @@ def spattn_last_error() -> str:
 
 def spattn_version() -> int:
     return LIB.spattn_version()
+
+
+def spattn_launch_count() -> int:
+    """Kernels the library has enqueued since it was loaded (all threads, devices)."""
+    return int(LIB.spattn_launch_count())

@@ -396,7 +396,7 @@ template <typename T, int D>
 cudaError_t launch_short_t(const FwdParams& p, cudaStream_t s) {
     const int64_t blocks = (int64_t)p.B * p.H * ((p.n + 7) / 8);
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    k_fwd_short<T, D><<<(unsigned)blocks, 256, 0, s>>>(p);
+    k_fwd_short<T, D><<<(unsigned)blocks, 256, 0, counted(s)>>>(p);
     return cudaGetLastError();
 }
 
@@ -409,7 +409,7 @@ cudaError_t launch_long_t(const FwdParams& p, int num_sms, cudaStream_t s) {
         if (items == 0) return cudaSuccess;
         if (items < grid) grid = items;
     }
-    k_fwd_long<T, D><<<(unsigned)grid, 256, 0, s>>>(p);
+    k_fwd_long<T, D><<<(unsigned)grid, 256, 0, counted(s)>>>(p);
     return cudaGetLastError();
 }
 
@@ -455,7 +455,7 @@ cudaError_t launch_classify_long_rows(const int32_t* row_ptr, int64_t rows, int6
     if (rows <= 0) return cudaSuccess;
     int64_t grid = (rows + 255) / 256;
     if (grid > 4096) grid = 4096;
-    k_classify_long<<<(unsigned)grid, 256, 0, s>>>(row_ptr, rows, nnz, list, count);
+    k_classify_long<<<(unsigned)grid, 256, 0, counted(s)>>>(row_ptr, rows, nnz, list, count);
     return cudaGetLastError();
 }
 

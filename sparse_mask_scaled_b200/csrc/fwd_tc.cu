@@ -944,11 +944,11 @@ cudaError_t launch_tc_t(const TcOperand& q, const TcOperand& k, const TcOperand&
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     constexpr int DP = D <= 64 ? D : 64;
     if (D <= 64 && p.has_extra)
-        k_fwd_tc_pipe<DP, true><<<(unsigned)grid, kPipeThreads, C::SMEM_BYTES, s>>>(mq, mk, mv, p);
+        k_fwd_tc_pipe<DP, true><<<(unsigned)grid, kPipeThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, p);
     else if (D <= 64)
-        k_fwd_tc_pipe<DP, false><<<(unsigned)grid, kPipeThreads, C::SMEM_BYTES, s>>>(mq, mk, mv, p);
+        k_fwd_tc_pipe<DP, false><<<(unsigned)grid, kPipeThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, p);
     else
-        k_fwd_tc<D><<<(unsigned)grid, kThreads, C::SMEM_BYTES, s>>>(mq, mk, mv, p);
+        k_fwd_tc<D><<<(unsigned)grid, kThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }
 

@@ -319,50 +319,140 @@ __device__ __forceinline__ int64_t block_exclusive_scan(int64_t x, int64_t* tota
     return res;
 }
 
-// Arrays up to kScanSmallMax: a single block scans them, 16 consecutive
-// counts per thread per pass (one pass up to 16,384 counts), carrying the
-// running total from pass to pass.
-constexpr int kSmallItems = 16;
-constexpr int64_t kScanSmallTile = (int64_t)kScanThreads * kSmallItems;
-constexpr int64_t kScanSmallMax = 4 * kScanSmallTile;
+// Arrays up to kScanSmallMax: a single block scans them in passes of
+// kPassRows values, carrying the running total from pass to pass. Values go
+// through shared memory so that global loads and stores are coalesced (value
+// t0 + j * 1024 + tid by thread tid), while the scan itself takes kPassItems
+// consecutive values per thread (one pad word per 32 keeps those reads free of
+// bank conflicts).
+constexpr int kPassItems = 8;
+constexpr int kPassRows = kScanThreads * kPassItems;
+constexpr int64_t kScanSmallMax = 8 * (int64_t)kPassRows;
+
+__device__ __forceinline__ int pad32(int i) { return i + (i >> 5); }
+
+// out[r] = sum of get(0 .. r-1) for r < rows, clamped to INT_MAX; returns the
+// total. With kLong, rows whose value exceeds kLongRowThreshold are listed in
+// row order in long_rows and counted in *n_long.
+template <bool kLong, class Get>
+__device__ __forceinline__ int64_t block_scan_rows(int64_t rows, Get get, int32_t* __restrict__ out,
+                                                   int32_t* __restrict__ long_rows, int64_t* n_long) {
+    __shared__ int32_t sv[kPassRows + kPassRows / 32];
+    const int tid = threadIdx.x;
+    int64_t carry = 0, long_carry = 0;
+    for (int64_t t0 = 0; t0 < rows; t0 += kPassRows) {
+        int32_t g[kPassItems];
+#pragma unroll
+        for (int j = 0; j < kPassItems; ++j) {
+            const int64_t r = t0 + j * kScanThreads + tid;
+            g[j] = r < rows ? get(r) : 0;
+        }
+#pragma unroll
+        for (int j = 0; j < kPassItems; ++j) sv[pad32(j * kScanThreads + tid)] = g[j];
+        __syncthreads();
+        int32_t v[kPassItems];
+        int64_t sum = 0, nl = 0;
+#pragma unroll
+        for (int t = 0; t < kPassItems; ++t) {
+            v[t] = sv[pad32(tid * kPassItems + t)];
+            sum += v[t];
+            nl += v[t] > kLongRowThreshold;
+        }
+        int64_t tot, ltot = 0, lrun = 0;
+        int64_t run = carry + block_exclusive_scan(sum, &tot);  // ends with a barrier
+        if (kLong) lrun = long_carry + block_exclusive_scan(nl, &ltot);
+#pragma unroll
+        for (int t = 0; t < kPassItems; ++t) {
+            sv[pad32(tid * kPassItems + t)] = run > INT_MAX ? INT_MAX : (int32_t)run;
+            if (kLong && v[t] > kLongRowThreshold) long_rows[lrun++] = (int32_t)(t0 + tid * kPassItems + t);
+            run += v[t];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < kPassItems; ++j) {
+            const int64_t r = t0 + j * kScanThreads + tid;
+            if (r < rows) out[r] = sv[pad32(j * kScanThreads + tid)];
+        }
+        carry += tot;
+        long_carry += ltot;
+        __syncthreads();  // the next pass refills sv
+    }
+    if (kLong) *n_long = long_carry;
+    return carry;
+}
 
 __global__ void __launch_bounds__(kScanThreads)
     k_scan_small(const int32_t* __restrict__ counts, int64_t rows, int32_t* __restrict__ out,
                  int64_t* total_out, unsigned* err) {
-    int64_t carry = 0;
-    for (int64_t t0 = 0; t0 < rows; t0 += kScanSmallTile) {
-        const int64_t base = t0 + (int64_t)threadIdx.x * kSmallItems;
-        int32_t v[kSmallItems];
-        int64_t sum = 0;
-        if (base + kSmallItems <= rows && (base & 3) == 0) {
-            const int4* p = reinterpret_cast<const int4*>(counts + base);
-#pragma unroll
-            for (int t = 0; t < kSmallItems / 4; ++t) {
-                const int4 w = __ldg(p + t);
-                v[4 * t] = w.x;
-                v[4 * t + 1] = w.y;
-                v[4 * t + 2] = w.z;
-                v[4 * t + 3] = w.w;
-            }
-        } else {
-#pragma unroll
-            for (int t = 0; t < kSmallItems; ++t) v[t] = base + t < rows ? counts[base + t] : 0;
-        }
-#pragma unroll
-        for (int t = 0; t < kSmallItems; ++t) sum += v[t];
-        int64_t total;
-        int64_t run = carry + block_exclusive_scan(sum, &total);
-#pragma unroll
-        for (int t = 0; t < kSmallItems; ++t) {
-            if (base + t < rows) out[base + t] = run > INT_MAX ? INT_MAX : (int32_t)run;
-            run += v[t];
-        }
-        carry += total;
-    }
+    const int64_t carry =
+        block_scan_rows<false>(rows, [&](int64_t r) { return counts[r]; }, out, nullptr, nullptr);
     if (threadIdx.x == 0) {
         out[rows] = carry > INT_MAX ? INT_MAX : (int32_t)carry;
         *total_out = carry;
         if (carry > INT_MAX) atomicOr(err, kBuildTooMany);
+    }
+}
+
+// Entries of row r for one mask kind (not COO); bad user row pointers and
+// negative half-widths count 0 and set their bit in err.
+template <int K>
+__device__ __forceinline__ int32_t row_count(const BuildSpec& s, int64_t r, int64_t rows, unsigned& err) {
+    if (K == SPATTN_MASK_CSR) {
+        const int64_t p0 = s.in_row_ptr[r], p1 = s.in_row_ptr[r + 1];
+        bool ok = p0 >= 0 && p1 >= p0 && p1 <= s.in_nnz;
+        if (r == 0 && p0 != 0) ok = false;
+        if (r == rows - 1 && p1 != s.in_nnz) ok = false;
+        if (!ok) err |= kBuildBadRowPtr;
+        return ok ? (int32_t)(p1 - p0) : 0;
+    } else if (K == SPATTN_MASK_DENSE) {
+        return s.n;
+    } else if (K == SPATTN_MASK_SLIDING || K == SPATTN_MASK_VARWIN) {
+        const int64_t i = r % s.n;
+        const int64_t w = K == SPATTN_MASK_SLIDING ? s.window : s.half_widths[r];
+        if (w < 0) {
+            err |= kBuildNegativeWidth;
+            return 0;
+        }
+        const int64_t lo = i - w < 0 ? 0 : i - w;
+        const int64_t hi = i + w + 1 > s.n ? s.n : i + w + 1;
+        return (int32_t)(hi - lo);
+    } else {  // BLOCK_STRIDED_GLOBAL: global rows are full, the others walk their columns
+        const int64_t i = r % s.n;
+        if (i < s.n_global) return s.n;
+        int32_t cnt = 0;
+        for (int64_t j = bsg_next(s, i, 0); j < s.n; j = bsg_next(s, i, j + 1)) ++cnt;
+        return cnt;
+    }
+}
+
+// Phase 1 in one launch for masks of at most kSingleMax rows (every kind but
+// COO): per-row counts, their exclusive scan into row_ptr, the list of rows
+// longer than kLongRowThreshold (in row order) and the info block -- written,
+// not accumulated, so it needs no clearing -- and, optionally, the clearing of
+// zero_words int32 words at zero_buf (the tile plan's counters and counts).
+constexpr int64_t kSingleMax = kScanSmallMax;
+
+template <int K>
+__global__ void __launch_bounds__(kScanThreads)
+    k_count_scan_single(BuildSpec s, int32_t* __restrict__ row_ptr, int32_t* __restrict__ long_rows,
+                        BuildInfo* info, int32_t* __restrict__ zero_buf, int64_t zero_words) {
+    __shared__ unsigned err_s;
+    if (threadIdx.x == 0) err_s = 0u;
+    for (int64_t x = threadIdx.x; x < zero_words; x += blockDim.x) zero_buf[x] = 0;
+    const int64_t rows = (int64_t)s.num_masks * s.n;
+    unsigned err = 0u;
+    int64_t n_long = 0;
+    const int64_t total = block_scan_rows<true>(
+        rows, [&](int64_t r) { return row_count<K>(s, r, rows, err); }, row_ptr, long_rows, &n_long);
+    if (err) atomicOr(&err_s, err);  // err_s was set before the scan's barriers
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        row_ptr[rows] = total > INT_MAX ? INT_MAX : (int32_t)total;
+        info->nnz = total;
+        info->n_long = (int32_t)n_long;
+        info->err = err_s | (total > INT_MAX ? (unsigned)kBuildTooMany : 0u);
+        info->pad = 0u;
+        info->pad2 = 0;
     }
 }
 
@@ -420,7 +510,8 @@ __global__ void k_scan_finalize(const int64_t* __restrict__ pref,
 // Phase 2, one warp per row: interval rows, COO rows (copied from coo_tmp) and
 // user CSR rows (copied).
 __global__ void k_fill_warp(BuildSpec s, const int32_t* __restrict__ row_ptr,
-                            const int32_t* __restrict__ coo_tmp, int32_t* __restrict__ col_idx) {
+                            const int32_t* __restrict__ coo_tmp, int32_t* __restrict__ col_idx,
+                            int32_t* __restrict__ tile_cnt, int nqb, int nkt) {
     const int64_t rows = (int64_t)s.num_masks * s.n;
     const int lane = threadIdx.x & 31;
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -436,6 +527,15 @@ __global__ void k_fill_warp(BuildSpec s, const int32_t* __restrict__ row_ptr,
             for (int64_t t = lane; t < o1 - o0; t += 32) col_idx[o0 + t] = src[t];
         } else if (row_interval(s, r, lo, hi, nullptr)) {
             for (int64_t t = lane; t < o1 - o0; t += 32) col_idx[o0 + t] = (int32_t)(lo + t);
+            if (tile_cnt && hi > lo) {  // the row's share of each 128 x 128 tile it touches
+                const int64_t m = r / s.n, i = r - m * s.n;
+                const int64_t base = (m * nqb + (i >> 7)) * nkt;
+                for (int64_t kt = (lo >> 7) + lane; kt <= (hi - 1) >> 7; kt += 32) {
+                    const int64_t a = lo > kt * 128 ? lo : kt * 128;
+                    const int64_t z = hi < kt * 128 + 128 ? hi : kt * 128 + 128;
+                    atomicAdd(&tile_cnt[base + kt], (int)(z - a));
+                }
+            }
         }
     }
 }
@@ -468,16 +568,55 @@ int64_t scan_tmp_elems(int64_t rows) { return rows + 1 + (rows + kScanTile - 1) 
 
 cudaError_t build_phase1(const BuildSpec& s, int32_t* row_ptr, int32_t* counts,
                          int64_t* scan_tmp, int32_t* coo_tmp, BuildInfo* info,
-                         int32_t* long_rows, cudaStream_t stream) {
+                         int32_t* long_rows, int32_t* zero_buf, int64_t zero_words,
+                         bool* zeroed, cudaStream_t stream) {
     const int64_t rows = (int64_t)s.num_masks * s.n;
     cudaError_t e;
+    *zeroed = false;
+    // block + strided + global rows walk their columns to count them: one
+    // block only takes the small ones
+    const bool single = s.kind == SPATTN_MASK_BLOCK_STRIDED_GLOBAL ? rows <= kPassRows / 2
+                                                                  : s.kind != SPATTN_MASK_COO && rows <= kSingleMax;
+    if (single) {
+        const int64_t zw = zero_buf ? zero_words : 0;
+        switch (s.kind) {
+        case SPATTN_MASK_CSR:
+            k_count_scan_single<SPATTN_MASK_CSR><<<1, kScanThreads, 0, counted(stream)>>>(
+                s, row_ptr, long_rows, info, zero_buf, zw);
+            break;
+        case SPATTN_MASK_SLIDING:
+            k_count_scan_single<SPATTN_MASK_SLIDING><<<1, kScanThreads, 0, counted(stream)>>>(
+                s, row_ptr, long_rows, info, zero_buf, zw);
+            break;
+        case SPATTN_MASK_VARWIN:
+            k_count_scan_single<SPATTN_MASK_VARWIN><<<1, kScanThreads, 0, counted(stream)>>>(
+                s, row_ptr, long_rows, info, zero_buf, zw);
+            break;
+        case SPATTN_MASK_DENSE:
+            k_count_scan_single<SPATTN_MASK_DENSE><<<1, kScanThreads, 0, counted(stream)>>>(
+                s, row_ptr, long_rows, info, zero_buf, zw);
+            break;
+        default:
+            k_count_scan_single<SPATTN_MASK_BLOCK_STRIDED_GLOBAL><<<1, kScanThreads, 0, counted(stream)>>>(
+                s, row_ptr, long_rows, info, zero_buf, zw);
+            break;
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        *zeroed = zero_buf != nullptr;
+        if (s.kind == SPATTN_MASK_CSR) {
+            k_check_csr<<<grid_for(rows, 8), 256, 0, counted(stream)>>>(s, info);
+            e = cudaGetLastError();
+        }
+        return e;
+    }
+    if ((e = cudaMemsetAsync(info, 0, sizeof(BuildInfo), stream)) != cudaSuccess) return e;
     if (s.kind == SPATTN_MASK_COO) {
         // big-row queue lives after the scan area
         int32_t* big_count = reinterpret_cast<int32_t*>(scan_tmp + scan_tmp_elems(rows));
         int32_t* big_list = big_count + 4;
         e = cudaMemsetAsync(big_count, 0, sizeof(int32_t), stream);
         if (e != cudaSuccess) return e;
-        k_coo_sort<<<grid_for(rows, kCooWarps), kCooWarps * 32, 0, stream>>>(
+        k_coo_sort<<<grid_for(rows, kCooWarps), kCooWarps * 32, 0, counted(stream)>>>(
             s, counts, coo_tmp, big_list, big_count, info);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         if (s.in_nnz + (s.add_diagonal ? 1 : 0) > kCooWarpCap) {
@@ -487,25 +626,25 @@ cudaError_t build_phase1(const BuildSpec& s, int32_t* row_ptr, int32_t* counts,
                 e = cudaFuncSetAttribute(k_coo_big, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
                 if (e != cudaSuccess) return e;
-                k_coo_big<<<grid_for(rows, 1, 512), 1024, smem, stream>>>(s, counts, coo_tmp,
+                k_coo_big<<<grid_for(rows, 1, 512), 1024, smem, counted(stream)>>>(s, counts, coo_tmp,
                                                                          big_list, big_count, info);
                 if ((e = cudaGetLastError()) != cudaSuccess) return e;
             } else {
                 // the n-bit map does not fit in shared memory: queued rows are an error
-                k_flag_big_rows<<<1, 32, 0, stream>>>(big_count, info);
+                k_flag_big_rows<<<1, 32, 0, counted(stream)>>>(big_count, info);
                 if ((e = cudaGetLastError()) != cudaSuccess) return e;
             }
         }
     } else {
-        k_count<<<grid_for(rows, 256), 256, 0, stream>>>(s, counts, info, long_rows);
+        k_count<<<grid_for(rows, 256), 256, 0, counted(stream)>>>(s, counts, info, long_rows);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         if (s.kind == SPATTN_MASK_CSR) {
-            k_check_csr<<<grid_for(rows, 8), 256, 0, stream>>>(s, info);
+            k_check_csr<<<grid_for(rows, 8), 256, 0, counted(stream)>>>(s, info);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
     }
     if (s.kind == SPATTN_MASK_COO) {
-        k_classify_counts<<<grid_for(rows, 256), 256, 0, stream>>>(counts, rows, long_rows, info);
+        k_classify_counts<<<grid_for(rows, 256), 256, 0, counted(stream)>>>(counts, rows, long_rows, info);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return scan_counts(counts, rows, row_ptr, scan_tmp, &info->nnz, &info->err, stream);
@@ -514,29 +653,30 @@ cudaError_t build_phase1(const BuildSpec& s, int32_t* row_ptr, int32_t* counts,
 cudaError_t scan_counts(const int32_t* counts, int64_t rows, int32_t* out, int64_t* scan_tmp,
                         int64_t* total, unsigned* err, cudaStream_t stream) {
     if (rows <= kScanSmallMax) {  // one block walks the tiles with a running carry
-        k_scan_small<<<1, kScanThreads, 0, stream>>>(counts, rows, out, total, err);
+        k_scan_small<<<1, kScanThreads, 0, counted(stream)>>>(counts, rows, out, total, err);
         return cudaGetLastError();
     }
     const int64_t ntiles = (rows + kScanTile - 1) / kScanTile;
     int64_t* pref = scan_tmp;
     int64_t* tile_sums = scan_tmp + rows + 1;
     cudaError_t e;
-    k_scan_tiles<<<(unsigned)ntiles, kScanThreads, 0, stream>>>(counts, rows, pref, tile_sums);
+    k_scan_tiles<<<(unsigned)ntiles, kScanThreads, 0, counted(stream)>>>(counts, rows, pref, tile_sums);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_scan_tile_sums<<<1, kScanThreads, 0, stream>>>(tile_sums, ntiles, total, err);
+    k_scan_tile_sums<<<1, kScanThreads, 0, counted(stream)>>>(tile_sums, ntiles, total, err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_scan_finalize<<<grid_for(rows + 1, 256), 256, 0, stream>>>(pref, tile_sums, rows, total, out);
+    k_scan_finalize<<<grid_for(rows + 1, 256), 256, 0, counted(stream)>>>(pref, tile_sums, rows, total, out);
     return cudaGetLastError();
 }
 
 cudaError_t build_phase2(const BuildSpec& s, const int32_t* row_ptr, const int32_t* coo_tmp,
-                         int32_t* col_idx, cudaStream_t stream) {
+                         int32_t* col_idx, int32_t* tile_cnt, cudaStream_t stream) {
     const int64_t rows = (int64_t)s.num_masks * s.n;
-    k_fill_warp<<<grid_for(rows, 8), 256, 0, stream>>>(s, row_ptr, coo_tmp, col_idx);
+    const int nqb = (s.n + kTileM - 1) / kTileM, nkt = (s.n + kTileN - 1) / kTileN;
+    k_fill_warp<<<grid_for(rows, 8), 256, 0, counted(stream)>>>(s, row_ptr, coo_tmp, col_idx, tile_cnt, nqb, nkt);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (s.kind == SPATTN_MASK_BLOCK_STRIDED_GLOBAL) {
-        k_fill_bsg<<<grid_for(rows, 128), 128, 0, stream>>>(s, row_ptr, col_idx);
+        k_fill_bsg<<<grid_for(rows, 128), 128, 0, counted(stream)>>>(s, row_ptr, col_idx);
         e = cudaGetLastError();
     }
     return e;

@@ -303,8 +303,18 @@ __global__ void __launch_bounds__(1024)
     for (int x0 = 0; x0 < nblocks; x0 += 1024) {
         const int x = x0 + threadIdx.x;
         int c = 0;
-        if (x < nblocks)
-            for (int kt = 0; kt < nkt; ++kt) c += cnt_map[(int64_t)x * nkt + kt] >= min_nnz;
+        if (x < nblocks) {  // eight independent loads in flight per step
+            const int32_t* row = cnt_map + (int64_t)x * nkt;
+            int kt = 0;
+            for (; kt + 8 <= nkt; kt += 8) {
+                int32_t v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v[u] = row[kt + u];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) c += v[u] >= min_nnz;
+            }
+            for (; kt < nkt; ++kt) c += row[kt] >= min_nnz;
+        }
         tc_blocks += c > 0;
         int inc = c;
 #pragma unroll
@@ -386,55 +396,58 @@ int64_t plan_tile_capacity(int64_t nblocks, int nkt, int64_t nnz, int min_nnz) {
 }
 
 cudaError_t build_plan(const int32_t* row_ptr, const int32_t* col_idx, int n, int num_masks,
-                       int64_t nnz, int min_nnz, bool intervals, const PlanBuffers& b,
-                       PlanCounters* counters, cudaStream_t s) {
+                       int64_t nnz, int min_nnz, bool intervals, bool zeroed, bool precounted,
+                       const PlanBuffers& b, PlanCounters* counters, cudaStream_t s) {
     const int64_t rows = (int64_t)num_masks * n;
     const int nqb = (n + kTileM - 1) / kTileM, nkt = (n + kTileN - 1) / kTileN;
     const int64_t nblocks = (int64_t)num_masks * nqb;
     cudaError_t e;
-    k_plan_zero<<<grid_for(nblocks * nkt, 256, 1024), 256, 0, s>>>(b.cnt_map, nblocks * nkt, counters);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (!zeroed) {
+        k_plan_zero<<<grid_for(nblocks * nkt, 256, 1024), 256, 0, counted(s)>>>(b.cnt_map, nblocks * nkt, counters);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     if (intervals) {
-        k_itv_count<<<grid_for(nblocks * 4, 8), 256, 0, s>>>(row_ptr, col_idx, n, nblocks, nqb, nkt,
-                                                            b.cnt_map);
+        if (!precounted)
+            k_itv_count<<<grid_for(nblocks * 4, 8), 256, 0, counted(s)>>>(row_ptr, col_idx, n, nblocks, nqb, nkt,
+                                                                b.cnt_map);
     } else {
         if ((e = cudaMemsetAsync(b.tile_bits, 0, sizeof(uint32_t) * b.tile_cap * kTileM * 4, s)) !=
             cudaSuccess)
             return e;
-        k_tile_count<<<grid_for(rows, 8), 256, 0, s>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map);
+        k_tile_count<<<grid_for(rows, 8), 256, 0, counted(s)>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (nblocks <= kFusedSelectMax) {
-        k_tile_select_fused<<<1, 1024, 0, s>>>(b.cnt_map, (int)nblocks, nkt, min_nnz, b.block_tile_off,
+        k_tile_select_fused<<<1, 1024, 0, counted(s)>>>(b.cnt_map, (int)nblocks, nkt, min_nnz, b.block_tile_off,
                                                b.tile_info, counters);
     } else {
-        k_tile_select<<<grid_for(nblocks, 128), 128, 0, s>>>(b.cnt_map, nblocks, nkt, min_nnz,
+        k_tile_select<<<grid_for(nblocks, 128), 128, 0, counted(s)>>>(b.cnt_map, nblocks, nkt, min_nnz,
                                                             b.block_ntiles, &counters->n_tc_blocks);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         e = scan_counts(b.block_ntiles, nblocks, b.block_tile_off, b.scan_tmp, &counters->n_tiles,
                         &counters->err, s);
         if (e != cudaSuccess) return e;
-        k_tile_assign<<<grid_for(nblocks, 8), 256, 0, s>>>(b.cnt_map, nblocks, nkt, min_nnz,
+        k_tile_assign<<<grid_for(nblocks, 8), 256, 0, counted(s)>>>(b.cnt_map, nblocks, nkt, min_nnz,
                                                           b.block_tile_off, b.tile_info);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (intervals)
-        k_itv_bits<<<grid_for(nblocks * kTileM, 256), 256, 0, s>>>(
+        k_itv_bits<<<grid_for(nblocks * kTileM, 256), 256, 0, counted(s)>>>(
             row_ptr, col_idx, n, nblocks, nqb, b.block_tile_off, b.tile_info, b.tile_bits, b.res_cnt,
             b.res_long, &counters->res_n_long);
     else
-        k_tile_bits<<<grid_for(rows, 8), 256, 0, s>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map,
+        k_tile_bits<<<grid_for(rows, 8), 256, 0, counted(s)>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map,
                                                      b.tile_info, b.tile_bits, b.res_cnt, b.res_long,
                                                      &counters->res_n_long);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     e = scan_counts(b.res_cnt, rows, b.res_row_ptr, b.scan_tmp, &counters->res_nnz, &counters->err, s);
     if (e != cudaSuccess) return e;
     if (intervals)
-        k_itv_residual<<<grid_for(rows, 256), 256, 0, s>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map,
+        k_itv_residual<<<grid_for(rows, 256), 256, 0, counted(s)>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map,
                                                           b.block_tile_off, b.res_row_ptr, b.res_col_idx,
                                                           &counters->n_mixed);
     else
-        k_residual_fill<<<grid_for(rows, 8), 256, 0, s>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map,
+        k_residual_fill<<<grid_for(rows, 8), 256, 0, counted(s)>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map,
                                                          b.block_tile_off, b.res_row_ptr, b.res_col_idx,
                                                          &counters->n_mixed);
     return cudaGetLastError();

@@ -1,6 +1,7 @@
 // C ABI of libspattn: argument checks, the stream-ordered memory pool, mask
 // handles and kernel launches. Every numerical step runs in the kernels of
-// fwd_gather.cu and mask_build.cu; this file only validates and schedules.
+// fwd_gather.cu, fwd_tc.cu, mask_build.cu and plan.cu; this file only validates
+// and schedules.
 //
 // Argument checks run before any CUDA call, so a rejected call touches no
 // device state.
@@ -11,9 +12,20 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 using namespace spattn;
+
+namespace spattn {
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}  // namespace
+cudaStream_t counted(cudaStream_t s) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return s;
+}
+}  // namespace spattn
 
 struct spattn_mask_s {
     int device;
@@ -237,6 +249,7 @@ struct Carve {
 
 unsigned* g_err_ptr[kMaxDevices];
 
+
 int build_status(unsigned err) {
     if (err & (kBuildTooMany | kBuildRowTooLong)) {
         return fail(SPATTN_ERR_UNSUPPORTED, "%s",
@@ -257,6 +270,8 @@ extern "C" {
 const char* spattn_last_error(void) { return g_msg; }
 
 int spattn_version(void) { return 100; /* 0.1.0 */ }
+
+uint64_t spattn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_mask* out) {
     g_msg[0] = 0;
@@ -305,13 +320,28 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
     bs.in_nnz = sp.in_nnz;
 
     const bool coo = sp.kind == SPATTN_MASK_COO;
-    // phase 1 memory: the mask's row_ptr + long-row list, and temporaries
+    const bool intervals = sp.kind == SPATTN_MASK_SLIDING || sp.kind == SPATTN_MASK_VARWIN ||
+                           sp.kind == SPATTN_MASK_DENSE;
+    const int min_nnz = sp.tile_min_nnz == 0 ? kTileMinNnzDefault : sp.tile_min_nnz;
+    const int nqb = (sp.n + kTileM - 1) / kTileM, nkt = (sp.n + kTileN - 1) / kTileN;
+    const int64_t nblocks = (int64_t)sp.num_masks * nqb;
+    const bool plan_possible = sp.tile_min_nnz >= 0 && nblocks * nkt <= kPlanMaxTileGrid;
+    // phase 1 memory: the mask's row_ptr + long-row list, and temporaries --
+    // those of the build and, as their sizes do not depend on nnz, the tile
+    // plan's (counters first, then the per-tile counts, so one run of words
+    // clears both)
     Carve ca;
     const int k_rp = ca.add((rows + 1) * 4), k_long = ca.add(rows * 4);
     Carve ct;
     const int k_info = ct.add(sizeof(BuildInfo)), k_cnt = ct.add(rows * 4);
     const int k_scan = ct.add((scan_tmp_elems(rows) + (coo ? (rows + 6) / 2 + 1 : 0)) * 8);
     const int k_coo = ct.add(coo ? (sp.in_nnz + rows) * 4 : 0);
+    const int64_t scan_rows = rows > nblocks ? rows : nblocks;
+    const int64_t cnt_words = plan_possible ? nblocks * nkt : 0;
+    const int k_pc = ct.add(plan_possible ? sizeof(PlanCounters) : 0),
+              k_cm = ct.add(cnt_words * 4), k_bn = ct.add(plan_possible ? nblocks * 4 : 0),
+              k_st = ct.add(plan_possible ? scan_tmp_elems(scan_rows) * 8 : 0),
+              k_rc = ct.add(plan_possible ? rows * 4 : 0);
     void *blk_a = nullptr, *blk_t = nullptr;
     cudaError_t e = cudaMallocFromPoolAsync(&blk_a, ca.total, pool, s);
     if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&blk_t, ct.total, pool, s);
@@ -325,8 +355,12 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
     int32_t* counts = ct.at<int32_t>(blk_t, k_cnt);
     int64_t* scan_tmp = ct.at<int64_t>(blk_t, k_scan);
     int32_t* coo_tmp = coo ? ct.at<int32_t>(blk_t, k_coo) : nullptr;
-    e = cudaMemsetAsync(info, 0, sizeof(BuildInfo), s);
-    if (e == cudaSuccess) e = build_phase1(bs, row_ptr, counts, scan_tmp, coo_tmp, info, long_rows, s);
+    // words from the counters to the end of the count array
+    const int64_t zero_words = plan_possible ? (int64_t)(ct.off[k_cm] - ct.off[k_pc]) / 4 + cnt_words : 0;
+    bool zeroed = false;
+    e = build_phase1(bs, row_ptr, counts, scan_tmp, coo_tmp, info, long_rows,
+                     zero_words > 0 && zero_words <= kPlanZeroInline ? ct.at<int32_t>(blk_t, k_pc) : nullptr,
+                     zero_words, &zeroed, s);
     BuildInfo hinfo;
     if (e == cudaSuccess) e = cudaMemcpyAsync(&hinfo, info, sizeof hinfo, cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
@@ -348,20 +382,19 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
     m->long_rows = long_rows;
     m->block_csr = blk_a;
 
-    // phase 2 memory: col_idx, the tile plan, and the plan's temporaries
-    const int min_nnz = sp.tile_min_nnz == 0 ? kTileMinNnzDefault : sp.tile_min_nnz;
-    const int nqb = (sp.n + kTileM - 1) / kTileM, nkt = (sp.n + kTileN - 1) / kTileN;
-    const int64_t nblocks = (int64_t)sp.num_masks * nqb;
-    const bool plan = sp.tile_min_nnz >= 0 && hinfo.nnz > 0 && nblocks * nkt <= kPlanMaxTileGrid;
+    // phase 2 memory: col_idx and the tile plan
+    const bool plan = plan_possible && hinfo.nnz > 0;
+    // interval rows hand their per-tile counts to the plan while writing columns
+    const bool precounted = plan && intervals && zeroed;
     PlanBuffers pb;
     memset(&pb, 0, sizeof pb);
     PlanCounters hpc;
     memset(&hpc, 0, sizeof hpc);
-    void* blk_t2 = nullptr;
     e = cudaMallocFromPoolAsync(&m->block_col, (size_t)(hinfo.nnz > 0 ? hinfo.nnz : 1) * 4, pool, s);
     if (e == cudaSuccess) {
         m->col_idx = static_cast<int32_t*>(m->block_col);
-        e = build_phase2(bs, row_ptr, coo_tmp, m->col_idx, s);
+        e = build_phase2(bs, row_ptr, coo_tmp, m->col_idx,
+                         precounted ? ct.at<int32_t>(blk_t, k_cm) : nullptr, s);
     }
     if (plan && e == cudaSuccess) {
         m->nqb = nqb;
@@ -370,13 +403,7 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
         const int k_bto = cp.add((nblocks + 1) * 4), k_ti = cp.add(pb.tile_cap * 4),
                   k_tb = cp.add(pb.tile_cap * kTileM * 16), k_rrp = cp.add((rows + 1) * 4),
                   k_rci = cp.add(hinfo.nnz * 4), k_rl = cp.add(rows * 4);
-        Carve c2;
-        const int64_t scan_rows = rows > nblocks ? rows : nblocks;
-        const int k_pc = c2.add(sizeof(PlanCounters)), k_cm = c2.add(nblocks * nkt * 4),
-                  k_bn = c2.add(nblocks * 4), k_st = c2.add(scan_tmp_elems(scan_rows) * 8),
-                  k_rc = c2.add(rows * 4);
         e = cudaMallocFromPoolAsync(&m->block_plan, cp.total, pool, s);
-        if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&blk_t2, c2.total, pool, s);
         if (e == cudaSuccess) {
             m->block_tile_off = pb.block_tile_off = cp.at<int32_t>(m->block_plan, k_bto);
             m->tile_info = pb.tile_info = cp.at<int32_t>(m->block_plan, k_ti);
@@ -384,21 +411,18 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
             m->res_row_ptr = pb.res_row_ptr = cp.at<int32_t>(m->block_plan, k_rrp);
             m->res_col_idx = pb.res_col_idx = cp.at<int32_t>(m->block_plan, k_rci);
             m->res_long = pb.res_long = cp.at<int32_t>(m->block_plan, k_rl);
-            PlanCounters* pc = c2.at<PlanCounters>(blk_t2, k_pc);
-            pb.cnt_map = c2.at<int32_t>(blk_t2, k_cm);
-            pb.block_ntiles = c2.at<int32_t>(blk_t2, k_bn);
-            pb.scan_tmp = c2.at<int64_t>(blk_t2, k_st);
-            pb.res_cnt = c2.at<int32_t>(blk_t2, k_rc);
-            e = build_plan(row_ptr, m->col_idx, sp.n, sp.num_masks, hinfo.nnz, min_nnz,
-                               sp.kind == SPATTN_MASK_SLIDING || sp.kind == SPATTN_MASK_VARWIN ||
-                                   sp.kind == SPATTN_MASK_DENSE,
-                               pb, pc, s);
+            PlanCounters* pc = ct.at<PlanCounters>(blk_t, k_pc);
+            pb.cnt_map = ct.at<int32_t>(blk_t, k_cm);
+            pb.block_ntiles = ct.at<int32_t>(blk_t, k_bn);
+            pb.scan_tmp = ct.at<int64_t>(blk_t, k_st);
+            pb.res_cnt = ct.at<int32_t>(blk_t, k_rc);
+            e = build_plan(row_ptr, m->col_idx, sp.n, sp.num_masks, hinfo.nnz, min_nnz, intervals,
+                           zeroed, precounted, pb, pc, s);
             if (e == cudaSuccess) e = cudaMemcpyAsync(&hpc, pc, sizeof hpc, cudaMemcpyDeviceToHost, s);
             if (e == cudaSuccess) e = cudaStreamSynchronize(s);
         }
     }
     cudaFreeAsync(blk_t, s);
-    if (blk_t2) cudaFreeAsync(blk_t2, s);
     if (e != cudaSuccess) {
         spattn_destroy_mask(m);
         return cuda_fail(e, "mask build (phase 2)");

@@ -20,6 +20,7 @@ constexpr int kTileN = 128;
 constexpr unsigned kTileDenseBit = 0x80000000u;  // tile_info flag: all 128 x 128 entries present
 constexpr int kTileMinNnzDefault = 512;
 // Tile planning is skipped when num_masks * (n/128)^2 exceeds this (count array size).
+constexpr int64_t kPlanZeroInline = 1 << 18;  // words the single-launch build clears
 constexpr int64_t kPlanMaxTileGrid = int64_t(1) << 26;
 
 // Rows with more nonzeros than this are processed by a whole thread block
@@ -88,6 +89,9 @@ struct TcParams {
 cudaError_t launch_fwd_tc(const TcOperand& q, const TcOperand& k, const TcOperand& v, int d,
                           const TcParams& p, cudaStream_t stream);
 cudaError_t error_flag_address(unsigned** p);
+// Every kernel launch of the library passes its stream through counted(),
+// which adds one to the count spattn_launch_count() reports.
+cudaStream_t counted(cudaStream_t s);
 
 // Tile plan (plan.cu).
 struct PlanBuffers {
@@ -114,9 +118,11 @@ struct PlanCounters {  // device-side results
 int64_t plan_tile_capacity(int64_t nblocks, int nkt, int64_t nnz, int min_nnz);
 // intervals: every row's columns form one contiguous run (sliding window,
 // variable window, dense), which lets the plan skip reading col_idx.
+// zeroed: the count array and the counters are already clear; precounted: the count
+// array already holds the per-tile counts (interval rows, from build_phase2).
 cudaError_t build_plan(const int32_t* row_ptr, const int32_t* col_idx, int n, int num_masks,
-                       int64_t nnz, int min_nnz, bool intervals, const PlanBuffers& b,
-                       PlanCounters* counters, cudaStream_t s);
+                       int64_t nnz, int min_nnz, bool intervals, bool zeroed, bool precounted,
+                       const PlanBuffers& b, PlanCounters* counters, cudaStream_t s);
 
 // ---------------------------------------------------------------- launchers
 // All launchers enqueue on `stream` and return the cudaGetLastError() result.
@@ -164,12 +170,15 @@ enum BuildErr : unsigned {
 // Writes info->err and info->nnz. Scratch: `counts` int32 [rows];
 // `scan_tmp` int64 [scan_tmp_elems(rows)] followed, for COO, by int32
 // [rows + 4] (the queue of long COO rows); coo_tmp int32 [in_nnz + rows]
-// (COO only). info->err must start at 0.
+// (COO only).
 // Also lists rows with more than kLongRowThreshold entries in long_rows [rows],
-// counted in info->n_long.
+// counted in info->n_long. Writes (or clears, then accumulates) *info. When
+// the single-launch path is taken and zero_buf is given, also clears
+// zero_words int32 words there and sets *zeroed.
 cudaError_t build_phase1(const BuildSpec& s, int32_t* row_ptr, int32_t* counts,
                          int64_t* scan_tmp, int32_t* coo_tmp, BuildInfo* info,
-                         int32_t* long_rows, cudaStream_t stream);
+                         int32_t* long_rows, int32_t* zero_buf, int64_t zero_words, bool* zeroed,
+                         cudaStream_t stream);
 int64_t scan_tmp_elems(int64_t rows);
 // Exclusive scan of int32 counts [rows] into out int32 [rows + 1]; the total goes
 // to *total (device) and overflow past INT32_MAX sets kBuildTooMany in *err.
@@ -177,7 +186,9 @@ int64_t scan_tmp_elems(int64_t rows);
 cudaError_t scan_counts(const int32_t* counts, int64_t rows, int32_t* out, int64_t* scan_tmp,
                         int64_t* total, unsigned* err, cudaStream_t stream);
 // Phase 2: write col_idx from the pattern (or copy it from coo_tmp / in_col_idx).
+// With tile_cnt (cleared, [num_masks * nqb * nkt]), interval rows also add their
+// per-tile counts for the tile plan.
 cudaError_t build_phase2(const BuildSpec& s, const int32_t* row_ptr, const int32_t* coo_tmp,
-                         int32_t* col_idx, cudaStream_t stream);
+                         int32_t* col_idx, int32_t* tile_cnt, cudaStream_t stream);
 
 }  // namespace spattn

@@ -181,3 +181,11 @@ def test_mask_spec_validation(kw, frag):
 def test_null_mask_handle():
     assert sp.LIB.spattn_destroy_mask(None) == sp.SPATTN_OK
     assert sp.LIB.spattn_mask_info(None, None, None, None, None, None, None) == sp.SPATTN_ERR_INVALID_ARG
+
+
+def test_rejected_calls_launch_nothing():
+    before = sp.spattn_launch_count()
+    _fwd(_desc((2, 3, 16, 48)))
+    _create(kind=9)
+    _fwd(_desc(S), num_masks=3)
+    assert sp.spattn_launch_count() == before

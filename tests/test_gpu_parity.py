@@ -312,3 +312,33 @@ def test_builder_parameter_corners(kind, kw):
     with build_mask(mp) as m:
         rp, ci = _gpu_csr(m)
     assert np.array_equal(rp, rp_ref) and np.array_equal(ci, ci_ref)
+
+
+@pytest.mark.parametrize("n,nm", [(16, 1), (32768, 2), (35000, 2)])
+def test_user_csr_both_build_paths(n, nm):
+    """User CSR through both phase-1 paths (one launch up to 65,536 rows, the
+    multi-launch scan above): the copy is exact, long rows are listed, and a
+    broken row_ptr or an unsorted row is still rejected."""
+    rng = np.random.default_rng(n)
+    lens = rng.integers(0, 12, size=nm * n)
+    lens[:: max(1, (nm * n) // 3)] = min(n, 1100)            # a few long rows
+    rows = [np.sort(rng.choice(n, size=int(c), replace=False)) for c in lens]
+    rp = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    ci = np.concatenate(rows).astype(np.int32)
+    drp, dci = torch.from_numpy(rp).cuda(), torch.from_numpy(ci).cuda()
+    with sp.spattn_create_csr_mask("csr", n, nm, in_row_ptr=drp, in_col_idx=dci) as m:
+        r2, c2 = m.csr()
+        assert m.nnz == int(rp[-1])
+        assert m.n_long == int(np.sum(lens > 1024))
+        assert torch.equal(r2, drp) and torch.equal(c2, dci)
+    bad = rp.copy()
+    bad[nm * n // 2] = bad[nm * n // 2 + 1] + 1                 # decreasing row_ptr
+    with pytest.raises(sp.SpattnError) as e:
+        sp.spattn_create_csr_mask("csr", n, nm, in_row_ptr=torch.from_numpy(bad).cuda(), in_col_idx=dci)
+    assert e.value.status == sp.SPATTN_ERR_BAD_CSR
+    j = int(np.argmax(lens >= 2))
+    uns = ci.copy()
+    uns[rp[j]], uns[rp[j] + 1] = uns[rp[j] + 1], uns[rp[j]]     # swap two columns of a row
+    with pytest.raises(sp.SpattnError) as e:
+        sp.spattn_create_csr_mask("csr", n, nm, in_row_ptr=drp, in_col_idx=torch.from_numpy(uns).cuda())
+    assert e.value.status == sp.SPATTN_ERR_BAD_CSR

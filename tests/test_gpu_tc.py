@@ -232,3 +232,81 @@ def test_variable_window_interval_plan_forward(thr):
     assert_close(to_f64(out).reshape(-1, wl.d), to_f64(lse), out_ref.reshape(-1, wl.d),
                  lse_ref.reshape(-1), wl.dtype, f"varwin thr={thr}")
     assert sp.spattn_device_error() == 0
+
+
+def _check_interval_plan(mask, rp, ci, n, nm, thr):
+    """Vectorised plan check for masks whose rows are single runs [lo, hi):
+    selected tiles, dense flags, every bit of every stored tile, and the
+    residual CSR (the run minus the selected tiles, ascending)."""
+    rows = nm * n
+    ln = np.diff(rp)
+    lo = np.where(ln > 0, ci[np.minimum(rp[:-1], max(ci.size - 1, 0))], 0).astype(np.int64)
+    hi = lo + ln
+    assert np.array_equal(ci, np.concatenate([np.arange(a, b) for a, b in zip(lo, hi)]))
+    nqb = (n + 127) // 128
+    r = np.arange(rows)
+    blk = (r // n) * nqb + (r % n) // 128
+    span = int(ln.max()) // 128 + 2
+    cnt = np.zeros((nm * nqb, nqb), np.int64)
+    parts = []
+    for j in range(span):
+        kt = lo // 128 + j
+        ov = np.minimum(hi, kt * 128 + 128) - np.maximum(lo, kt * 128)
+        ok = (ov > 0) & (kt < nqb)
+        np.add.at(cnt, (blk[ok], kt[ok]), ov[ok])
+        parts.append((kt, np.where(ok, ov, 0)))
+    sel = cnt >= thr
+    plan = mask.plan()
+    assert mask.n_tiles == int(sel.sum())
+    bto, info, bits, rrp, rci = (x.cpu().numpy() for x in plan)
+    assert np.array_equal(np.diff(bto), sel.sum(axis=1))
+    tb, tk = np.nonzero(sel)                      # tiles in (block, key tile) order
+    assert np.array_equal(info & 0x7fffffff, tk)
+    dense = info < 0
+    assert np.array_equal(dense, cnt[tb, tk] == 128 * 128)
+    # bits: row rr of tile t holds [lo, hi) clipped to the tile
+    got = np.unpackbits(bits.view(np.uint8).reshape(-1, 128, 16), axis=2, bitorder="little").astype(bool)
+    qrow = (tb % nqb)[:, None] * 128 + np.arange(128)[None, :]            # [T, 128]
+    valid = qrow < n
+    grow = np.where(valid, (tb // nqb)[:, None] * n + qrow, 0)
+    a = np.clip(lo[grow] - tk[:, None] * 128, 0, 128)
+    b = np.clip(hi[grow] - tk[:, None] * 128, 0, 128)
+    c = np.arange(128)[None, None, :]
+    want = (c >= a[:, :, None]) & (c < b[:, :, None]) & valid[:, :, None] & ~dense[:, None, None]
+    assert np.array_equal(got, want)
+    # residual: what the selected tiles leave of each run
+    res = ln.copy()
+    for kt, ov in parts:
+        res -= np.where(sel[blk, np.minimum(kt, nqb - 1)], ov, 0)
+    assert np.array_equal(np.diff(rrp), res)
+    assert mask.residual_nnz == int(res.sum())
+    rrow = np.repeat(r, res)
+    assert np.all((rci >= lo[rrow]) & (rci < hi[rrow]))
+    assert not sel[blk[rrow], rci // 128].any()
+    same = rrow[1:] == rrow[:-1]
+    assert np.all(np.diff(rci)[same] > 0)
+
+
+@pytest.mark.parametrize("n,thr", [(32000, 9000), (33000, 9000), (33000, 0)])
+def test_interval_plan_both_build_paths(n, thr):
+    """Two masks of n rows each: up to 65,536 rows the mask build runs as one
+    launch that also clears the plan's counts, and the column fill counts the
+    tiles; above it the plan clears and counts by itself. Both must give the
+    same plan and forward."""
+    wl = workloads.make(1, B=2, H=1, n=n)
+    rp, ci = oracle.mask_from_params(wl.mask)
+    with _mask_with_thr(wl.mask, thr) as m:
+        grp, gci = m.csr()
+        assert np.array_equal(grp.cpu().numpy(), rp) and np.array_equal(gci.cpu().numpy(), ci)
+        _check_interval_plan(m, rp, ci, n, wl.mask.num_masks, 512 if thr == 0 else thr)
+        q, k, v, _, _ = device_inputs(wl)
+        out, lse = sp.spattn_fwd_mask(q, k, v, m, scale=wl.scale)
+        torch.cuda.synchronize()
+    rng = np.random.default_rng(n)
+    rows = np.unique(np.concatenate([rng.integers(0, 2 * n, 400), [0, n - 1, n, 2 * n - 1]]))
+    out_ref, lse_ref = oracle.masked_sdpa(wl.q.raw, wl.k.raw, wl.v.raw, rp, ci, wl.mask.num_masks,
+                                          wl.scale, rows=rows)
+    idx = torch.from_numpy(rows).cuda()
+    assert_close(to_f64(out.reshape(-1, wl.d)[idx]), to_f64(lse[idx]), out_ref, lse_ref, wl.dtype,
+                 f"varwin n={n} thr={thr}")
+    assert sp.spattn_device_error() == 0
