@@ -242,7 +242,7 @@ class GpuWorkload:
             n_global=mp.n_global, add_diagonal=mp.add_diagonal,
             half_widths=self.hw if hw is None else hw,
             in_row_ptr=self.crp if crp is None else crp,
-            in_col_idx=self.ccols if ccols is None else ccols)
+            in_col_idx=self.ccols if ccols is None else ccols, asynchronous=True)
 
     def fwd(self, m, q=None, k=None, v=None, out=None, lse=None):
         return self.sp.spattn_fwd_mask(self.q if q is None else q, self.k if k is None else k,

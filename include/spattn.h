@@ -111,8 +111,13 @@ typedef struct {
     int32_t tile_min_nnz;       /* tensor-core tiles: a 128 x 128 tile with at least this many
                                    nonzeros is computed on tensor cores (bf16 inputs);
                                    0 = default (512), < 0 = never */
-    int32_t reserved;           /* must be 0 */
+    uint32_t flags;             /* SPATTN_MASK_* flags below, or 0 */
 } spattn_mask_spec;
+
+/* spec.flags: SLIDING, VARWIN and DENSE masks are built without waiting for
+ * the device (no host synchronisation; see spattn_create_csr_mask). Other
+ * kinds ignore it. */
+#define SPATTN_MASK_ASYNC 1u
 
 /* A built mask: its CSR (row_ptr int32 [num_masks*n + 1], col_idx int32 [nnz]),
  * plus the schedule the forward pass uses: rows long enough to be split over a
@@ -120,34 +125,54 @@ typedef struct {
  * by 128 keys) that hold at least tile_min_nnz nonzeros, each with a per-row
  * bit mask, and the residual CSR of the entries outside those tiles. (Blocks
  * are cheaper than single entries: the block-sparse remark of the gluon-nlp
- * discussion, applied tile by tile to any CSR.) Owns its device memory. */
+ * discussion, applied tile by tile to any CSR.) Owns its device memory.
+ *
+ * Interval masks. Every row of a SLIDING, VARWIN or DENSE mask is one run of
+ * columns [lo, hi), so such a mask (up to 1,048,576 keys and 65,536 query
+ * blocks of 128 rows) keeps the runs and its tile selection instead: the
+ * forward pass derives columns and tile bits from the runs, and the CSR, the
+ * tile bits and the residual CSR are written only when a call below asks for
+ * them (that call synchronises the mask's stream once, and the arrays are then
+ * kept until the mask is destroyed). */
 typedef struct spattn_mask_s* spattn_mask;
 
 /* Build a CSR mask on the device from a pattern (the proposal's "generate the
  * corresponding attention mask" step, then the row schedule).
- * Synchronises `stream` twice (to size col_idx and the schedule). Memory comes
- * from the library's stream-ordered pool and is released by spattn_destroy_mask.
- * Errors: INVALID_ARG (bad kind or parameters), BAD_CSR (CSR not sorted/unique,
- * a column outside [0, n), row_ptr not a valid prefix sum, or a negative
- * half-width), UNSUPPORTED (more than 2^31 - 1 nonzeros, or a COO row with more
- * candidates than the builder's limit), OOM, CUDA. On error *out is NULL. */
+ * Synchronises `stream` (twice for CSR, COO and BLOCK_STRIDED_GLOBAL masks, to
+ * size col_idx and the schedule; once for interval masks, to check the
+ * half-widths; not at all for interval masks with SPATTN_MASK_ASYNC). With
+ * SPATTN_MASK_ASYNC the call only enqueues the build: a negative half-width is
+ * then not reported here -- its row is left empty and the device error flag
+ * bit 0 is raised (see spattn_device_error) -- and the size queries below wait
+ * for the build. Memory comes from the library's stream-ordered pool and is
+ * released by spattn_destroy_mask.
+ * Errors: INVALID_ARG (bad kind, parameters or flags), BAD_CSR (CSR not
+ * sorted/unique, a column outside [0, n), row_ptr not a valid prefix sum, or a
+ * negative half-width), UNSUPPORTED (more than 2^31 - 1 nonzeros, or a COO row
+ * with more candidates than the builder's limit), OOM, CUDA. On error *out is
+ * NULL. */
 int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream, spattn_mask* out);
 
 /* Read a mask's sizes and device CSR pointers (owned by the mask). Any output
- * pointer may be NULL. n_long: rows handled by the block-per-row kernel. */
+ * pointer may be NULL. n_long: rows with more than 1024 nonzeros (handled by
+ * a whole thread block). nnz and n_long wait for an asynchronous build; asking
+ * for row_ptr or col_idx of an interval mask writes its CSR first (synchronises;
+ * UNSUPPORTED above 2^31 - 1 nonzeros). */
 int spattn_mask_info(spattn_mask mask, int32_t* n, int32_t* num_masks, int64_t* nnz,
                      const int32_t** row_ptr, const int32_t** col_idx, int64_t* n_long);
 
 /* Copy a mask's CSR into caller buffers (device or host memory, any mix):
  * row_ptr_dst int32 [num_masks * n + 1], col_idx_dst int32 [nnz]; either may be
  * NULL to skip it. Stream-ordered on `stream`; host destinations should be
- * pinned for the copy to be asynchronous. */
+ * pinned for the copy to be asynchronous. Interval masks write their CSR first
+ * (as spattn_mask_info). */
 int spattn_mask_copy_csr(spattn_mask mask, int32_t* row_ptr_dst, int32_t* col_idx_dst,
                          void* stream);
 
 /* The tile plan's sizes: tensor-core tiles, residual nonzeros (the entries the
  * gather kernel processes on bf16 inputs) and rows with entries on both paths.
- * Any output pointer may be NULL. */
+ * Any output pointer may be NULL. Waits for an asynchronous build; n_mixed_rows
+ * of an interval mask writes its explicit plan first (synchronises). */
 int spattn_mask_plan_info(spattn_mask mask, int64_t* n_tiles, int64_t* residual_nnz,
                           int64_t* n_mixed_rows);
 
@@ -158,7 +183,8 @@ int spattn_mask_plan_info(spattn_mask mask, int64_t* n_tiles, int64_t* residual_
  * tile_bits uint32 [n_tiles * 128 * 4] (row r of a tile: 4 words, bit c of word
  * c/32 = column c; left zero for dense tiles, whose entries are all present), residual row_ptr int32 [num_masks * n + 1] and col_idx
  * int32 [residual_nnz]. Returns SPATTN_ERR_INVALID_ARG when the mask has no
- * tile plan. Stream-ordered on `stream`. */
+ * tile plan. Stream-ordered on `stream`; interval masks write these arrays
+ * first (synchronises). */
 int spattn_mask_copy_plan(spattn_mask mask, int32_t* block_tile_off, int32_t* tile_info,
                           uint32_t* tile_bits, int32_t* res_row_ptr, int32_t* res_col_idx,
                           void* stream);
@@ -195,7 +221,9 @@ int spattn_fwd(const spattn_tensor* q, const spattn_tensor* k, const spattn_tens
  * (tcgen05) and the residual entries on the gather kernel; rows with entries
  * on both paths are merged with the running max/sum rule. Those rows need a
  * workspace of B*H*n*(d+2) floats, taken from the library's stream-ordered
- * pool for the duration of the call (only when the plan has such rows).
+ * pool for the duration of the call (only when the plan may have such rows:
+ * for an interval mask whose build has not completed when the call is made,
+ * whenever its parameters do not rule them out). Never synchronises.
  * fp32 inputs use the gather kernel for every entry.
  * A bounded wait in the tensor-core kernel that expires raises device error
  * flag bit 1 (see spattn_device_error). */
@@ -234,7 +262,8 @@ int spattn_fwd_noalloc(const spattn_tensor* q, const spattn_tensor* k, const spa
 const char* spattn_last_error(void);
 
 /* Synchronise `stream`, then read and clear the current device's error flags
- * raised by kernels (bit 0: a column index outside [0, n) was skipped; bit 1:
+ * raised by kernels (bit 0: a column index outside [0, n) was skipped, or an
+ * asynchronous interval-mask build met a negative half-width; bit 1:
  * a bounded wait in the tensor-core kernel expired and its rows are invalid).
  * *flags may be NULL. Returns SPATTN_OK, SPATTN_ERR_TIMEOUT if bit 1 was set,
  * else SPATTN_ERR_BAD_CSR if bit 0 was set. */

@@ -56,13 +56,16 @@ class spattn_tensor(ctypes.Structure):
                 ("stride", ctypes.c_int64 * 4)]
 
 
+SPATTN_MASK_ASYNC = 1
+
+
 class spattn_mask_spec(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("n", ctypes.c_int32), ("num_masks", ctypes.c_int32),
                 ("window", ctypes.c_int32), ("block", ctypes.c_int32), ("stride", ctypes.c_int32),
                 ("n_global", ctypes.c_int32), ("add_diagonal", ctypes.c_int32),
                 ("half_widths", ctypes.c_void_p), ("in_row_ptr", ctypes.c_void_p),
                 ("in_col_idx", ctypes.c_void_p), ("in_nnz", ctypes.c_int64),
-                ("tile_min_nnz", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("tile_min_nnz", ctypes.c_int32), ("flags", ctypes.c_uint32)]
 
 
 _P = ctypes.c_void_p
@@ -146,18 +149,57 @@ def _ptr(t) -> Optional[int]:
 
 
 class Mask:
-    """A mask built on the device by ``spattn_create_csr_mask`` (owns its memory)."""
+    """A mask built on the device by ``spattn_create_csr_mask`` (owns its memory).
 
-    def __init__(self, handle: int):
+    Sizes are read from the library on first use: for an asynchronous build that
+    waits for it, and ``n_mixed_rows`` of an interval mask writes its explicit
+    plan first."""
+
+    def __init__(self, handle: int, n: int, num_masks: int):
         self.handle = handle
-        n, nm, nnz, nl = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int64(), ctypes.c_int64()
-        rp, ci = _P(), _P()
-        _check(LIB.spattn_mask_info(handle, ctypes.byref(n), ctypes.byref(nm), ctypes.byref(nnz),
-                                    ctypes.byref(rp), ctypes.byref(ci), ctypes.byref(nl)))
-        self.n, self.num_masks, self.nnz, self.n_long = n.value, nm.value, nnz.value, nl.value
-        nt, rn, nmix = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
-        _check(LIB.spattn_mask_plan_info(handle, ctypes.byref(nt), ctypes.byref(rn), ctypes.byref(nmix)))
-        self.n_tiles, self.residual_nnz, self.n_mixed_rows = nt.value, rn.value, nmix.value
+        self.n, self.num_masks = n, num_masks
+        self._sizes = None
+        self._plan_sizes = None
+        self._mixed = None
+
+    def _info(self):
+        if self._sizes is None:
+            nnz, nl = ctypes.c_int64(), ctypes.c_int64()
+            _check(LIB.spattn_mask_info(self.handle, None, None, ctypes.byref(nnz), None, None,
+                                        ctypes.byref(nl)))
+            self._sizes = (nnz.value, nl.value)
+        return self._sizes
+
+    def _plan_info(self):
+        if self._plan_sizes is None:
+            nt, rn = ctypes.c_int64(), ctypes.c_int64()
+            _check(LIB.spattn_mask_plan_info(self.handle, ctypes.byref(nt), ctypes.byref(rn), None))
+            self._plan_sizes = (nt.value, rn.value)
+        return self._plan_sizes
+
+    @property
+    def nnz(self) -> int:
+        return self._info()[0]
+
+    @property
+    def n_long(self) -> int:
+        return self._info()[1]
+
+    @property
+    def n_tiles(self) -> int:
+        return self._plan_info()[0]
+
+    @property
+    def residual_nnz(self) -> int:
+        return self._plan_info()[1]
+
+    @property
+    def n_mixed_rows(self) -> int:
+        if self._mixed is None:
+            nm = ctypes.c_int64()
+            _check(LIB.spattn_mask_plan_info(self.handle, None, None, ctypes.byref(nm)))
+            self._mixed = nm.value
+        return self._mixed
 
     def csr(self, stream=None):
         """Copies of (row_ptr, col_idx) as int32 torch tensors on the current device."""
@@ -204,9 +246,11 @@ class Mask:
 def spattn_create_csr_mask(kind, n: int, num_masks: int = 1, *, window: int = 0, block: int = 0,
                            stride: int = 0, n_global: int = 0, add_diagonal: bool = False,
                            half_widths=None, in_row_ptr=None, in_col_idx=None,
-                           tile_min_nnz: int = 0, stream=None) -> Mask:
+                           tile_min_nnz: int = 0, asynchronous: bool = False,
+                           stream=None) -> Mask:
     """Build a CSR mask on the device. ``kind``: a name of MASK_KINDS or its code.
-    Array arguments are int32 CUDA tensors."""
+    Array arguments are int32 CUDA tensors. ``asynchronous``: SPATTN_MASK_ASYNC
+    (interval masks are built without a host synchronisation)."""
     spec = spattn_mask_spec()
     spec.kind = MASK_KINDS[kind] if isinstance(kind, str) else int(kind)
     spec.n, spec.num_masks = n, num_masks
@@ -217,10 +261,10 @@ def spattn_create_csr_mask(kind, n: int, num_masks: int = 1, *, window: int = 0,
     spec.in_col_idx = _ptr(in_col_idx)
     spec.in_nnz = 0 if in_col_idx is None else int(in_col_idx.numel())
     spec.tile_min_nnz = int(tile_min_nnz)
-    spec.reserved = 0
+    spec.flags = SPATTN_MASK_ASYNC if asynchronous else 0
     h = _P()
     _check(LIB.spattn_create_csr_mask(ctypes.byref(spec), _stream(stream), ctypes.byref(h)))
-    return Mask(h.value)
+    return Mask(h.value, n, num_masks)
 
 
 def _outputs(q, out, lse, want_lse):

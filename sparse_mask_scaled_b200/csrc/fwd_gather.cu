@@ -146,8 +146,9 @@ __device__ __forceinline__ void init_row(const FwdParams& P, int b, int h, int i
 }
 
 // Process the steps of STEP nonzeros starting at first, first + stride, ...
-// (below p1) of one row into `st`.
-template <typename T, int D>
+// (below p1) of one row into `st`. kRun: the positions are the columns
+// themselves (a run of an interval row), else indices into col_idx.
+template <typename T, int D, bool kRun = false>
 __device__ __forceinline__ void row_steps(const FwdParams& P, const RowCtx<T, D>& rc,
                                           int64_t first, int64_t p1, int64_t stride, int lane,
                                           State<Cfg<T, D>::VEC>& st) {
@@ -159,7 +160,7 @@ __device__ __forceinline__ void row_steps(const FwdParams& P, const RowCtx<T, D>
         float extra = 0.f;
         const int64_t mp = pb + lane;
         if (lane < C::STEP && mp < p1) {
-            const int j = __ldg(P.col_idx + mp);
+            const int j = kRun ? (int)mp : __ldg(P.col_idx + mp);
             if ((unsigned)j < (unsigned)P.n) {
                 col = j;
                 if (P.has_extra) {
@@ -305,6 +306,161 @@ __global__ void __launch_bounds__(256) k_fwd_short(const FwdParams P) {
         P.lse[((int64_t)bh) * P.n + i] = st.l > 0.f ? (st.m + lg2(st.l)) * kLn2 : -INFINITY;
 }
 
+// The warp-uniform runs of an interval row [lo, hi) that lie in unselected key
+// tiles (tm[kt] < 0), merged across neighbouring tiles up to 32 tiles at a
+// time; the whole run when tm is null. fn(a, z) is called by every lane.
+template <class F>
+__device__ __forceinline__ void for_each_run(const int32_t* __restrict__ tm, int lo, int hi, int lane,
+                                             F&& fn) {
+    if (hi <= lo) return;
+    if (!tm) {
+        fn(lo, hi);
+        return;
+    }
+    const int k0 = lo >> 7, k1 = (hi - 1) >> 7;
+    for (int c0 = k0; c0 <= k1; c0 += 32) {
+        const int kt = c0 + lane;
+        unsigned bits = __ballot_sync(0xffffffffu, kt <= k1 && __ldg(tm + kt) < 0);
+        while (bits) {
+            const int s = __ffs(bits) - 1;
+            const unsigned inv = ~(bits >> s);
+            const int len = inv ? __ffs(inv) - 1 : 32 - s;
+            const int ta = c0 + s, tz = ta + len;
+            fn(lo > ta * kTileN ? lo : ta * kTileN, hi < tz * kTileN ? hi : tz * kTileN);
+            bits = s + len >= 32 ? 0u : (bits & (0xffffffffu << (s + len)));
+        }
+    }
+}
+
+// Final output of a row (out = acc / l, lse), or its partial state for the
+// tensor-core kernel. Lanes < LPR hold the row's acc slices.
+template <typename T, int D>
+__device__ __forceinline__ void finish_row(const FwdParams& P, int b, int h, int i, int lane,
+                                           const State<Cfg<T, D>::VEC>& st, bool partial) {
+    using C = Cfg<T, D>;
+    const int64_t wrow = ((int64_t)b * P.H + h) * P.n + i;
+    if (partial) {
+        if (lane < C::LPR) write_partial<C::VEC>(P.ws_acc + wrow * D + lane * C::VEC, st.acc);
+        if (lane == 0) {
+            P.ws_ml[wrow * 2] = st.m;
+            P.ws_ml[wrow * 2 + 1] = st.l;
+        }
+        return;
+    }
+    if (lane < C::LPR) {
+        const float inv = st.l > 0.f ? 1.f / st.l : 0.f;
+        float o[C::VEC];
+#pragma unroll
+        for (int e = 0; e < C::VEC; ++e) o[e] = st.acc[e] * inv;
+        T* orow = reinterpret_cast<T*>(P.out) + b * P.o_sb + h * P.o_sh + i * P.o_sn;
+        *reinterpret_cast<uint4*>(orow + lane * C::VEC) = Elem<T>::pack(o);
+    }
+    if (lane == 0 && P.lse) P.lse[wrow] = st.l > 0.f ? (st.m + lg2(st.l)) * kLn2 : -INFINITY;
+}
+
+// Eight rows i0 .. i0 + 7 of (b, h) (see k_fwd_itv).
+template <typename T, int D>
+__device__ __forceinline__ void itv_rows8(const FwdParams& P, int b, int h, int mk, int i0,
+                                          const int32_t* __restrict__ tm, bool partial) {
+    using C = Cfg<T, D>;
+    __shared__ float sm_m[8], sm_l[8];
+    __shared__ float sm_acc[8][D];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int i = i0 + warp;
+    int lo = 0, hi = 0;
+    if (i < P.n) {
+        const int2 v = P.itv_lohi[(int64_t)mk * P.n + i];
+        lo = v.x;
+        hi = v.y;
+    }
+    int len = 0;
+    for_each_run(tm, lo, hi, lane, [&](int a, int z) { len += z - a; });
+    if (!__syncthreads_or(len > kLongRowThreshold)) {
+        if (i >= P.n) return;  // the caller's loop ends with this group
+        RowCtx<T, D> rc;
+        State<C::VEC> st;
+        init_row<T, D>(P, b, h, i, lane, rc, st);
+        for_each_run(tm, lo, hi, lane,
+                     [&](int a, int z) { row_steps<T, D, true>(P, rc, a, z, C::STEP, lane, st); });
+        merge_groups<C::VEC, C::LPR>(st);
+        finish_row<T, D>(P, b, h, i, lane, st, partial);
+        return;
+    }
+    for (int rr = 0; rr < 8 && i0 + rr < P.n; ++rr) {
+        const int ii = i0 + rr;
+        const int2 v = P.itv_lohi[(int64_t)mk * P.n + ii];
+        RowCtx<T, D> rc;
+        State<C::VEC> st;
+        init_row<T, D>(P, b, h, ii, lane, rc, st);
+        for_each_run(tm, v.x, v.y, lane, [&](int a, int z) {
+            row_steps<T, D, true>(P, rc, a + warp * C::STEP, z, 8 * C::STEP, lane, st);
+        });
+        merge_groups<C::VEC, C::LPR>(st);
+        if (lane == 0) {
+            sm_m[warp] = st.m;
+            sm_l[warp] = st.l;
+        }
+        if (lane < C::LPR) {
+#pragma unroll
+            for (int e = 0; e < C::VEC; ++e) sm_acc[warp][lane * C::VEC + e] = st.acc[e];
+        }
+        __syncthreads();
+        if (warp == 0) {  // merge the eight warps' states; lanes < LPR own acc slices
+            float mx = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) mx = fmaxf(mx, sm_m[w]);
+            const float mu = (mx == -INFINITY) ? 0.f : mx;
+            State<C::VEC> t;
+            t.m = mx;
+            t.l = 0.f;
+#pragma unroll
+            for (int e = 0; e < C::VEC; ++e) t.acc[e] = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                const float f = ex2(sm_m[w] - mu);
+                t.l = fmaf(sm_l[w], f, t.l);
+                if (lane < C::LPR) {
+#pragma unroll
+                    for (int e = 0; e < C::VEC; ++e) t.acc[e] = fmaf(sm_acc[w][lane * C::VEC + e], f, t.acc[e]);
+                }
+            }
+            finish_row<T, D>(P, b, h, ii, lane, t, partial);
+        }
+        __syncthreads();
+    }
+}
+
+// Interval masks. A block takes 128 / itv_slices rows of one 128-row query
+// block of one (b, h), eight at a time: eight warps, one row each; when any of
+// the eight has more than kLongRowThreshold entries to gather, the warps take
+// those rows one after the other together instead (merging through shared
+// memory). In a query block with tensor-core tiles every row hands over its
+// partial state (l = 0 when it gathered nothing), and query blocks without
+// entries outside their tiles return at once.
+template <typename T, int D>
+__global__ void __launch_bounds__(256, 2) k_fwd_itv(const FwdParams P) {
+    const int slices = P.itv_slices, rows_per = kTileM / slices;
+    const int per_bh = P.nqb * slices;
+    const int bh = blockIdx.x / per_bh;
+    const int rem = blockIdx.x - bh * per_bh;
+    const int qb = rem / slices;
+    const int b = bh / P.H, h = bh - b * P.H;
+    const int mk = P.num_masks == 1 ? 0 : b;
+    const int64_t blk = (int64_t)mk * P.nqb + qb;
+    const int32_t* tm = nullptr;
+    bool partial = false;
+    if (P.tmap) {
+        tm = P.tmap + blk * P.nkt;
+        if (P.qb_tile_off[blk + 1] > P.qb_tile_off[blk]) {
+            if (!P.blk_res[blk]) return;  // the tensor-core kernel does every row alone
+            partial = true;
+        }
+    }
+    const int r0 = qb * kTileM + (rem - qb * slices) * rows_per;
+    const int r1 = min(r0 + rows_per, P.n);
+    for (int i0 = r0; i0 < r1; i0 += 8) itv_rows8<T, D>(P, b, h, mk, i0, tm, partial);
+}
+
 constexpr int kLongWarps = 8;
 
 template <typename T, int D>
@@ -401,6 +557,16 @@ cudaError_t launch_short_t(const FwdParams& p, cudaStream_t s) {
 }
 
 template <typename T, int D>
+cudaError_t launch_itv_t(const FwdParams& p, cudaStream_t s) {
+    if (p.itv_slices < 1 || p.itv_slices > 16 || (p.itv_slices & (p.itv_slices - 1)))
+        return cudaErrorInvalidValue;
+    const int64_t blocks = (int64_t)p.B * p.H * p.nqb * p.itv_slices;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    k_fwd_itv<T, D><<<(unsigned)blocks, 256, 0, counted(s)>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
 cudaError_t launch_long_t(const FwdParams& p, int num_sms, cudaStream_t s) {
     int64_t grid = (int64_t)num_sms * 4;
     if (p.long_count_host >= 0) {
@@ -427,6 +593,23 @@ cudaError_t launch_fwd_short_rows(const FwdParams& p, int dtype, int d, cudaStre
         case 32: return launch_short_t<float, 32>(p, s);
         case 64: return launch_short_t<float, 64>(p, s);
         case 128: return launch_short_t<float, 128>(p, s);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_fwd_itv(const FwdParams& p, int dtype, int d, cudaStream_t s) {
+    if (dtype == 0) {
+        switch (d) {
+        case 32: return launch_itv_t<__nv_bfloat16, 32>(p, s);
+        case 64: return launch_itv_t<__nv_bfloat16, 64>(p, s);
+        case 128: return launch_itv_t<__nv_bfloat16, 128>(p, s);
+        }
+    } else {
+        switch (d) {
+        case 32: return launch_itv_t<float, 32>(p, s);
+        case 64: return launch_itv_t<float, 64>(p, s);
+        case 128: return launch_itv_t<float, 128>(p, s);
         }
     }
     return cudaErrorInvalidValue;

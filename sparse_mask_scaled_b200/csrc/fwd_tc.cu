@@ -155,6 +155,45 @@ __device__ __forceinline__ void add_addend_run(const AddendView& a, int64_t rowb
     }
 }
 
+// Bits of the columns [c0, c0 + 32) that lie in the run [lo, hi).
+__device__ __forceinline__ uint32_t run_word(int lo, int hi, int c0) {
+    int a = lo - c0, z = hi - c0;
+    a = a < 0 ? 0 : (a > 32 ? 32 : a);
+    z = z < 0 ? 0 : (z > 32 ? 32 : z);
+    if (z <= a) return 0u;
+    const uint32_t top = z == 32 ? 0xffffffffu : ((1u << z) - 1u);
+    return top & ~((1u << a) - 1u);  // a < 32 here
+}
+
+// Row `row` of tile t (key tile in `info`): its 128 mask bits, from the tile's
+// stored bits or, for interval masks, from the row's run [lo, hi).
+__device__ __forceinline__ uint4 tile_row_bits4(const TcParams& P, int t, int info, int row, int lo, int hi) {
+    if (P.itv_lohi) {
+        const int c0 = (info & 0x7fffffff) * kTileN;
+        return make_uint4(run_word(lo, hi, c0), run_word(lo, hi, c0 + 32), run_word(lo, hi, c0 + 64),
+                          run_word(lo, hi, c0 + 96));
+    }
+    return __ldg(reinterpret_cast<const uint4*>(P.tile_bits) + ((int64_t)t * 128 + row));
+}
+
+// The same for key half `half` (64 columns).
+__device__ __forceinline__ uint2 tile_row_bits2(const TcParams& P, int t, int info, int row, int half, int lo,
+                                                int hi) {
+    if (P.itv_lohi) {
+        const int c0 = (info & 0x7fffffff) * kTileN + half * 64;
+        return make_uint2(run_word(lo, hi, c0), run_word(lo, hi, c0 + 32));
+    }
+    return __ldg(reinterpret_cast<const uint2*>(P.tile_bits) + ((int64_t)t * 128 + row) * 2 + half);
+}
+
+// Whether row (mrow of the mask, wrow of the output) has a partial state from
+// the gather kernel to merge.
+__device__ __forceinline__ bool has_partial(const TcParams& P, int64_t blk, int64_t mrow, int64_t wrow) {
+    if (!P.ws_ml) return false;
+    if (P.blk_res) return P.blk_res[blk] && P.ws_ml[wrow * 2 + 1] > 0.f;
+    return P.res_row_ptr[mrow + 1] > P.res_row_ptr[mrow];
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     k_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -270,12 +309,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t mask_rowbase = (int64_t)b * P.mask.s0 + (int64_t)h * P.mask.s1 + (int64_t)i * P.mask.s2;
     const int64_t bias_rowbase = (int64_t)b * P.bias.s0 + (int64_t)h * P.bias.s1 + (int64_t)i * P.bias.s2;
     float m_ref = -INFINITY, l = 0.f;
+    int rlo = 0, rhi = 0;  // interval masks: the row's run
+    if (P.itv_lohi && row_ok) {
+        const int2 v = P.itv_lohi[(int64_t)mk * P.n + i];
+        rlo = v.x;
+        rhi = v.y;
+    }
 
     // tile u's info and row bits are loaded one tile ahead
     int next_info = P.tile_info[t_begin];
     uint4 next_bits = make_uint4(0u, 0u, 0u, 0u);
-    if (next_info >= 0 && row_ok)
-        next_bits = __ldg(reinterpret_cast<const uint4*>(P.tile_bits) + ((int64_t)t_begin * 128 + row));
+    if (next_info >= 0 && row_ok && !P.itv_lohi) next_bits = tile_row_bits4(P, t_begin, next_info, row, rlo, rhi);
     const uint64_t c2 = pack2(P.qk_scale_log2, P.qk_scale_log2);
 
     for (int u = 0; u < T; ++u) {
@@ -283,15 +327,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint4 wbits = next_bits;
         if (u + 1 < T) {
             next_info = P.tile_info[t_begin + u + 1];
-            if (next_info >= 0 && row_ok)
-                next_bits = __ldg(reinterpret_cast<const uint4*>(P.tile_bits) +
-                                  ((int64_t)(t_begin + u + 1) * 128 + row));
+            if (next_info >= 0 && row_ok && !P.itv_lohi)
+                next_bits = tile_row_bits4(P, t_begin + u + 1, next_info, row, rlo, rhi);
         }
         const int kt = info & 0x7fffffff;
         const bool dense = info < 0;  // the same for the whole CTA
         const bool extra = P.has_extra && row_ok;
         const int jj0 = kt * 128;
-        const uint32_t bw[4] = {wbits.x, wbits.y, wbits.z, wbits.w};
+        const uint4 wb = P.itv_lohi && row_ok && !dense ? tile_row_bits4(P, 0, info, row, rlo, rhi) : wbits;
+        const uint32_t bw[4] = {wb.x, wb.y, wb.z, wb.w};
 
         wait(barS, (uint32_t)(u & 1));
         tc_fence_after();
@@ -450,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float M = m_ref, L = l, fa = 1.f;
         const int64_t mrow = (int64_t)mk * P.n + i;
         const int64_t wrow = (int64_t)bh * P.n + i;
-        const bool mixed = P.ws_ml && P.res_row_ptr[mrow + 1] > P.res_row_ptr[mrow];
+        const bool mixed = has_partial(P, blk, mrow, wrow);
         float mg = -INFINITY, lg = 0.f, fg = 0.f;
         if (mixed) {
             mg = P.ws_ml[wrow * 2];
@@ -642,11 +686,17 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
     const int64_t mask_rowbase = (int64_t)b * P.mask.s0 + (int64_t)h * P.mask.s1 + (int64_t)i * P.mask.s2;
     const int64_t bias_rowbase = (int64_t)b * P.bias.s0 + (int64_t)h * P.bias.s1 + (int64_t)i * P.bias.s2;
     float m_ref = -INFINITY, l = 0.f;  // l: this thread's half of the row sum
+    int rlo = 0, rhi = 0;  // interval masks: the row's run
+    if (P.itv_lohi && row_ok) {
+        const int2 v = P.itv_lohi[(int64_t)mk * P.n + i];
+        rlo = v.x;
+        rhi = v.y;
+    }
 
     int next_info = P.tile_info[t_begin];
-    uint2 next_bits = make_uint2(0u, 0u);
-    if (next_info >= 0 && row_ok)
-        next_bits = __ldg(reinterpret_cast<const uint2*>(P.tile_bits) + ((int64_t)t_begin * 128 + row) * 2 + half);
+    uint2 next_bits = make_uint2(0u, 0u);  // stored bits, loaded one tile ahead
+    if (next_info >= 0 && row_ok && !P.itv_lohi)
+        next_bits = tile_row_bits2(P, t_begin, next_info, row, half, rlo, rhi);
     const uint64_t c2 = pack2(P.qk_scale_log2, P.qk_scale_log2);
 
     for (int u = 0; u < T; ++u) {
@@ -654,9 +704,8 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
         const uint2 wbits = next_bits;
         if (u + 1 < T) {
             next_info = P.tile_info[t_begin + u + 1];
-            if (next_info >= 0 && row_ok)
-                next_bits = __ldg(reinterpret_cast<const uint2*>(P.tile_bits) +
-                                  ((int64_t)(t_begin + u + 1) * 128 + row) * 2 + half);
+            if (next_info >= 0 && row_ok && !P.itv_lohi)
+                next_bits = tile_row_bits2(P, t_begin + u + 1, next_info, row, half, rlo, rhi);
         }
         const int kt = info & 0x7fffffff;
         const bool dense = info < 0;
@@ -688,7 +737,8 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
             if (P.bias.data) add_addend_run<64>(P.bias, bias_rowbase, c0, ncols, x);
         }
         if (!dense) {  // entries the CSR does not list
-            const uint32_t bw[2] = {wbits.x, wbits.y};
+            const uint2 wb = P.itv_lohi ? tile_row_bits2(P, 0, info, row, half, rlo, rhi) : wbits;
+            const uint32_t bw[2] = {wb.x, wb.y};
 #pragma unroll
             for (int j = 0; j < 64; ++j) x[j] = ((bw[j >> 5] >> (j & 31)) & 1u) ? x[j] : -INFINITY;
         }
@@ -825,7 +875,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
         float M = m_ref, L = l_row, fa = 1.f;
         const int64_t mrow = (int64_t)mk * P.n + i;
         const int64_t wrow = (int64_t)bh * P.n + i;
-        const bool mixed = P.ws_ml && P.res_row_ptr[mrow + 1] > P.res_row_ptr[mrow];
+        const bool mixed = has_partial(P, blk, mrow, wrow);
         float fg = 0.f;
         if (mixed) {
             const float mg = P.ws_ml[wrow * 2], lg = P.ws_ml[wrow * 2 + 1];

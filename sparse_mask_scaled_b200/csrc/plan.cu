@@ -9,6 +9,7 @@
 // entries -- applied per tile of an arbitrary CSR). The remaining nonzeros form
 // the residual CSR, which the gather kernel processes. Rows that have entries
 // in both are merged with the streaming-softmax rescaling rule.
+#include "spattn.h"
 #include "spattn_internal.cuh"
 
 namespace spattn {
@@ -170,9 +171,17 @@ __global__ void k_residual_fill(const int32_t* __restrict__ row_ptr, const int32
 // and residual runs follow from the run's overlap with each tile, without
 // reading the rest of col_idx.
 
+// The run [lo, hi) of an interval row: from the mask's runs when given, else
+// from its first and last CSR column.
 __device__ __forceinline__ void row_run(const int32_t* __restrict__ row_ptr,
-                                        const int32_t* __restrict__ col_idx, int64_t r, int& lo,
-                                        int& hi) {
+                                        const int32_t* __restrict__ col_idx,
+                                        const int2* __restrict__ lohi, int64_t r, int& lo, int& hi) {
+    if (lohi) {
+        const int2 v = lohi[r];
+        lo = v.x;
+        hi = v.y;
+        return;
+    }
     const int64_t p0 = row_ptr[r], p1 = row_ptr[r + 1];
     if (p1 > p0) {
         lo = col_idx[p0];
@@ -189,7 +198,7 @@ __device__ __forceinline__ int overlap(int lo, int hi, int c0, int c1) {
 
 // One warp per 32 rows of a query block: per-tile counts, one atomic per tile.
 __global__ void k_itv_count(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
-                            int n, int64_t nblocks, int nqb, int nkt, int32_t* __restrict__ cnt) {
+                            const int2* __restrict__ lohi, int n, int64_t nblocks, int nqb, int nkt, int32_t* __restrict__ cnt) {
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = nblocks * 4;
     for (int64_t w = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5); w < nwarps;
@@ -198,7 +207,7 @@ __global__ void k_itv_count(const int32_t* __restrict__ row_ptr, const int32_t* 
         const int64_t m = blk / nqb;
         const int i = (int)(blk - m * nqb) * kTileM + (int)(w & 3) * 32 + lane;
         int lo = 0, hi = 0;
-        if (i < n) row_run(row_ptr, col_idx, m * n + i, lo, hi);
+        if (i < n) row_run(row_ptr, col_idx, lohi, m * n + i, lo, hi);
         const bool any = hi > lo;
         int k0 = any ? lo >> 7 : 0x7fffffff, k1 = any ? (hi - 1) >> 7 : -1;
 #pragma unroll
@@ -219,7 +228,7 @@ __global__ void k_itv_count(const int32_t* __restrict__ row_ptr, const int32_t* 
 // selected (not dense) tile of its block -- zero words included, so the bit
 // array needs no clearing -- and its residual count.
 __global__ void k_itv_bits(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
-                           int n, int64_t nblocks, int nqb, const int32_t* __restrict__ block_tile_off,
+                           const int2* __restrict__ lohi, int n, int64_t nblocks, int nqb, const int32_t* __restrict__ block_tile_off,
                            const int32_t* __restrict__ tile_info, uint32_t* __restrict__ bits,
                            int32_t* __restrict__ res_cnt, int32_t* __restrict__ res_long,
                            int32_t* __restrict__ res_n_long) {
@@ -230,7 +239,7 @@ __global__ void k_itv_bits(const int32_t* __restrict__ row_ptr, const int32_t* _
         const int64_t m = blk / nqb;
         const int i = (int)(blk - m * nqb) * kTileM + row;
         int lo = 0, hi = 0;
-        if (i < n) row_run(row_ptr, col_idx, m * n + i, lo, hi);
+        if (i < n) row_run(row_ptr, col_idx, lohi, m * n + i, lo, hi);
         int in_tiles = 0;
         for (int t = block_tile_off[blk]; t < block_tile_off[blk + 1]; ++t) {
             const int info = tile_info[t];
@@ -261,7 +270,7 @@ __global__ void k_itv_bits(const int32_t* __restrict__ row_ptr, const int32_t* _
 
 // One thread per row: the residual runs (parts of [lo, hi) in unselected tiles).
 __global__ void k_itv_residual(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
-                               int n, int64_t rows, int nqb, int nkt, const int32_t* __restrict__ map,
+                               const int2* __restrict__ lohi, int n, int64_t rows, int nqb, int nkt, const int32_t* __restrict__ map,
                                const int32_t* __restrict__ block_tile_off,
                                const int32_t* __restrict__ res_row_ptr, int32_t* __restrict__ res_col,
                                int32_t* __restrict__ n_mixed) {
@@ -272,7 +281,7 @@ __global__ void k_itv_residual(const int32_t* __restrict__ row_ptr, const int32_
         const int64_t m = r / n, i = r - m * n;
         const int64_t blk = m * nqb + (i >> 7);
         int lo, hi;
-        row_run(row_ptr, col_idx, r, lo, hi);
+        row_run(row_ptr, col_idx, lohi, r, lo, hi);
         for (int kt = lo >> 7; kt <= (hi - 1) >> 7; ++kt) {
             if (map[blk * nkt + kt] >= 0) continue;
             const int a = lo > kt * kTileN ? lo : kt * kTileN;
@@ -380,6 +389,207 @@ __global__ void k_plan_zero(int32_t* __restrict__ cnt, int64_t n_cnt, PlanCounte
         reinterpret_cast<uint32_t*>(counters)[threadIdx.x] = 0u;
 }
 
+// ------------------------------------------------- implicit interval masks
+// Step 1, one CTA of 128 threads per query block (128 rows of one mask): each
+// row's run [lo, hi) from the pattern, the block's entry count per key tile
+// (all nkt of them, zeros included, so nothing needs clearing first) and, per
+// block, the rows above kLongRowThreshold entries and the rows with a negative
+// half-width (which are left empty).
+__global__ void __launch_bounds__(kTileM)
+    k_itv_rows(ItvSpec s, int2* __restrict__ lohi, int32_t* __restrict__ cnt, int2* __restrict__ bstat) {
+    extern __shared__ int32_t cs[];  // [nkt]
+    const int64_t blk = blockIdx.x;
+    const int64_t m = blk / s.nqb;
+    const int qb = (int)(blk - m * s.nqb);
+    for (int kt = threadIdx.x; kt < s.nkt; kt += kTileM) cs[kt] = 0;
+    __syncthreads();
+    const int i = qb * kTileM + threadIdx.x;
+    int lo = 0, hi = 0;
+    bool bad = false;
+    if (i < s.n) {
+        const int64_t r = m * s.n + i;
+        if (s.kind == SPATTN_MASK_DENSE) {
+            hi = s.n;
+        } else {
+            const int64_t w = s.kind == SPATTN_MASK_SLIDING ? (int64_t)s.window : (int64_t)s.half_widths[r];
+            if (w < 0) {
+                bad = true;
+            } else {
+                lo = (int)(i - w < 0 ? 0 : i - w);
+                hi = (int)(i + w + 1 > s.n ? s.n : i + w + 1);
+            }
+        }
+        lohi[r] = make_int2(lo, hi);
+    }
+    const int lane = threadIdx.x & 31;
+    const bool any = hi > lo;
+    int k0 = any ? lo >> 7 : 0x7fffffff, k1 = any ? (hi - 1) >> 7 : -1;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        k0 = min(k0, __shfl_xor_sync(0xffffffffu, k0, off));
+        k1 = max(k1, __shfl_xor_sync(0xffffffffu, k1, off));
+    }
+    for (int kt = k0; kt <= k1; ++kt) {  // one shared atomic per tile and warp
+        int c = overlap(lo, hi, kt * kTileN, kt * kTileN + kTileN);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+        if (lane == 0 && c) atomicAdd(&cs[kt], c);
+    }
+    const int n_long = __syncthreads_count(hi - lo > kLongRowThreshold);
+    const int n_bad = __syncthreads_count(bad);
+    for (int kt = threadIdx.x; kt < s.nkt; kt += kTileM) cnt[blk * s.nkt + kt] = cs[kt];
+    if (threadIdx.x == 0) bstat[blk] = make_int2(n_long, n_bad);
+    if (bad && s.err_flags) atomicOr(s.err_flags, kErrBadColumn);
+}
+
+// Step 2, one thread block: the selection of k_tile_select_fused (tiles with at
+// least min_nnz entries, numbered block-major; the count array becomes the
+// tile map), plus, per query block, whether it keeps entries outside its
+// selected tiles (blk_res), and the mask's totals -- written, not accumulated.
+__global__ void __launch_bounds__(1024)
+    k_itv_select(int32_t* __restrict__ cnt_map, int nblocks, int nkt, int min_nnz,
+                 const int2* __restrict__ bstat, int32_t* __restrict__ block_tile_off,
+                 int32_t* __restrict__ tile_info, int32_t* __restrict__ blk_res, ItvCounters* out) {
+    __shared__ int32_t wsum[32];
+    __shared__ int32_t carry_s;
+    __shared__ unsigned long long s_nnz, s_res;
+    __shared__ int s_long, s_bad, s_tcb;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) {
+        carry_s = 0;
+        s_nnz = s_res = 0ull;
+        s_long = s_bad = s_tcb = 0;
+    }
+    __syncthreads();
+    unsigned long long nnz = 0, res = 0;
+    int nlong = 0, nbad = 0, tcb = 0;
+    for (int x0 = 0; x0 < nblocks; x0 += 1024) {
+        const int x = x0 + threadIdx.x;
+        int c = 0;
+        if (x < nblocks) {
+            const int32_t* row = cnt_map + (int64_t)x * nkt;
+            int64_t bn = 0, br = 0;
+            int kt = 0;
+            for (; kt + 8 <= nkt; kt += 8) {  // eight independent loads in flight
+                int32_t v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v[u] = row[kt + u];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const bool sel = min_nnz > 0 && v[u] >= min_nnz;
+                    c += sel;
+                    bn += v[u];
+                    br += sel ? 0 : v[u];
+                }
+            }
+            for (; kt < nkt; ++kt) {
+                const int32_t v = row[kt];
+                const bool sel = min_nnz > 0 && v >= min_nnz;
+                c += sel;
+                bn += v;
+                br += sel ? 0 : v;
+            }
+            blk_res[x] = br > 0;
+            nnz += bn;
+            res += br;
+            tcb += c > 0;
+            const int2 st = bstat[x];
+            nlong += st.x;
+            nbad += st.y;
+        }
+        int inc = c;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, inc, off);
+            if (lane >= off) inc += y;
+        }
+        if (lane == 31) wsum[warp] = inc;
+        __syncthreads();
+        if (warp == 0) {
+            const int w = wsum[lane];
+            int wi = w;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, wi, off);
+                if (lane >= off) wi += y;
+            }
+            wsum[lane] = wi - w;
+        }
+        __syncthreads();
+        const int carry = carry_s;
+        if (x < nblocks) block_tile_off[x] = carry + wsum[warp] + inc - c;
+        __syncthreads();
+        if (threadIdx.x == 1023) carry_s = carry + wsum[warp] + inc;
+        __syncthreads();
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        nnz += __shfl_xor_sync(0xffffffffu, nnz, off);
+        res += __shfl_xor_sync(0xffffffffu, res, off);
+        nlong += __shfl_xor_sync(0xffffffffu, nlong, off);
+        nbad += __shfl_xor_sync(0xffffffffu, nbad, off);
+        tcb += __shfl_xor_sync(0xffffffffu, tcb, off);
+    }
+    if (lane == 0) {
+        atomicAdd(&s_nnz, nnz);
+        atomicAdd(&s_res, res);
+        atomicAdd(&s_long, nlong);
+        atomicAdd(&s_bad, nbad);
+        atomicAdd(&s_tcb, tcb);
+    }
+    // one warp per query block numbers its selected tiles
+    for (int x = warp; x < nblocks; x += 32) {
+        int idx = block_tile_off[x];
+        for (int k0 = 0; k0 < nkt; k0 += 32) {
+            const int kt = k0 + lane;
+            const int c = kt < nkt ? cnt_map[(int64_t)x * nkt + kt] : 0;
+            const bool sel = kt < nkt && min_nnz > 0 && c >= min_nnz;
+            const unsigned bal = __ballot_sync(0xffffffffu, sel);
+            if (kt < nkt) {
+                if (sel) {
+                    const int id = idx + __popc(bal & ((1u << lane) - 1u));
+                    tile_info[id] = kt | (c == kTileM * kTileN ? (int)kTileDenseBit : 0);
+                    cnt_map[(int64_t)x * nkt + kt] = id;
+                } else {
+                    cnt_map[(int64_t)x * nkt + kt] = -1;
+                }
+            }
+            idx += __popc(bal);
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        block_tile_off[nblocks] = carry_s;
+        out->nnz = (int64_t)s_nnz;
+        out->n_tiles = carry_s;
+        out->res_nnz = (int64_t)s_res;
+        out->n_long = s_long;
+        out->n_tc_blocks = s_tcb;
+        out->err = s_bad ? (unsigned)kBuildNegativeWidth : 0u;
+        out->pad = 0;
+    }
+}
+
+__global__ void k_lohi_counts(const int2* __restrict__ lohi, int64_t rows, int32_t* __restrict__ counts) {
+    for (int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; r < rows;
+         r += (int64_t)gridDim.x * blockDim.x) {
+        const int2 v = lohi[r];
+        counts[r] = v.y > v.x ? v.y - v.x : 0;
+    }
+}
+
+// One warp per row: columns lo, lo + 1, ..., hi - 1.
+__global__ void k_lohi_fill(const int2* __restrict__ lohi, int64_t rows, const int32_t* __restrict__ row_ptr,
+                            int32_t* __restrict__ col_idx) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t r = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+        const int2 v = lohi[r];
+        const int64_t o = row_ptr[r];
+        for (int t = lane; t < v.y - v.x; t += 32) col_idx[o + t] = v.x + t;
+    }
+}
+
 unsigned grid_for(int64_t work, int per_block, int64_t cap = 1 << 16) {
     int64_t g = (work + per_block - 1) / per_block;
     if (g < 1) g = 1;
@@ -408,7 +618,7 @@ cudaError_t build_plan(const int32_t* row_ptr, const int32_t* col_idx, int n, in
     }
     if (intervals) {
         if (!precounted)
-            k_itv_count<<<grid_for(nblocks * 4, 8), 256, 0, counted(s)>>>(row_ptr, col_idx, n, nblocks, nqb, nkt,
+            k_itv_count<<<grid_for(nblocks * 4, 8), 256, 0, counted(s)>>>(row_ptr, col_idx, nullptr, n, nblocks, nqb, nkt,
                                                                 b.cnt_map);
     } else {
         if ((e = cudaMemsetAsync(b.tile_bits, 0, sizeof(uint32_t) * b.tile_cap * kTileM * 4, s)) !=
@@ -433,7 +643,7 @@ cudaError_t build_plan(const int32_t* row_ptr, const int32_t* col_idx, int n, in
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (intervals)
         k_itv_bits<<<grid_for(nblocks * kTileM, 256), 256, 0, counted(s)>>>(
-            row_ptr, col_idx, n, nblocks, nqb, b.block_tile_off, b.tile_info, b.tile_bits, b.res_cnt,
+            row_ptr, col_idx, nullptr, n, nblocks, nqb, b.block_tile_off, b.tile_info, b.tile_bits, b.res_cnt,
             b.res_long, &counters->res_n_long);
     else
         k_tile_bits<<<grid_for(rows, 8), 256, 0, counted(s)>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map,
@@ -443,13 +653,59 @@ cudaError_t build_plan(const int32_t* row_ptr, const int32_t* col_idx, int n, in
     e = scan_counts(b.res_cnt, rows, b.res_row_ptr, b.scan_tmp, &counters->res_nnz, &counters->err, s);
     if (e != cudaSuccess) return e;
     if (intervals)
-        k_itv_residual<<<grid_for(rows, 256), 256, 0, counted(s)>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map,
+        k_itv_residual<<<grid_for(rows, 256), 256, 0, counted(s)>>>(row_ptr, col_idx, nullptr, n, rows, nqb, nkt, b.cnt_map,
                                                           b.block_tile_off, b.res_row_ptr, b.res_col_idx,
                                                           &counters->n_mixed);
     else
         k_residual_fill<<<grid_for(rows, 8), 256, 0, counted(s)>>>(row_ptr, col_idx, n, rows, nqb, nkt, b.cnt_map,
                                                          b.block_tile_off, b.res_row_ptr, b.res_col_idx,
                                                          &counters->n_mixed);
+    return cudaGetLastError();
+}
+
+
+cudaError_t itv_build(const ItvSpec& s, int2* lohi, int32_t* cnt, int2* bstat, int32_t* block_tile_off,
+                      int32_t* tile_info, int32_t* blk_res, int min_nnz, ItvCounters* counters,
+                      cudaStream_t stream) {
+    const int64_t nblocks = (int64_t)s.num_masks * s.nqb;
+    if (s.nkt > kItvMaxKeyTiles || nblocks > kItvMaxBlocks) return cudaErrorInvalidValue;
+    k_itv_rows<<<(unsigned)nblocks, kTileM, (size_t)s.nkt * 4, counted(stream)>>>(s, lohi, cnt, bstat);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    k_itv_select<<<1, 1024, 0, counted(stream)>>>(cnt, (int)nblocks, s.nkt, min_nnz, bstat, block_tile_off,
+                                                  tile_info, blk_res, counters);
+    return cudaGetLastError();
+}
+
+cudaError_t itv_write_csr(const int2* lohi, int64_t rows, int32_t* counts, int32_t* row_ptr,
+                          int32_t* col_idx, int64_t* scan_tmp, int64_t* total, unsigned* err,
+                          cudaStream_t stream) {
+    k_lohi_counts<<<grid_for(rows, 256), 256, 0, counted(stream)>>>(lohi, rows, counts);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if ((e = scan_counts(counts, rows, row_ptr, scan_tmp, total, err, stream)) != cudaSuccess) return e;
+    if (col_idx) {
+        k_lohi_fill<<<grid_for(rows, 8), 256, 0, counted(stream)>>>(lohi, rows, row_ptr, col_idx);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+
+cudaError_t itv_write_plan(const int2* lohi, int n, int num_masks, const PlanBuffers& b,
+                           PlanCounters* counters, cudaStream_t s) {
+    const int64_t rows = (int64_t)num_masks * n;
+    const int nqb = (n + kTileM - 1) / kTileM, nkt = (n + kTileN - 1) / kTileN;
+    const int64_t nblocks = (int64_t)num_masks * nqb;
+    k_itv_bits<<<grid_for(nblocks * kTileM, 256), 256, 0, counted(s)>>>(
+        nullptr, nullptr, lohi, n, nblocks, nqb, b.block_tile_off, b.tile_info, b.tile_bits, b.res_cnt,
+        b.res_long, &counters->res_n_long);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = scan_counts(b.res_cnt, rows, b.res_row_ptr, b.scan_tmp, &counters->res_nnz, &counters->err, s);
+    if (e != cudaSuccess) return e;
+    k_itv_residual<<<grid_for(rows, 256), 256, 0, counted(s)>>>(nullptr, nullptr, lohi, n, rows, nqb, nkt,
+                                                               b.cnt_map, b.block_tile_off, b.res_row_ptr,
+                                                               b.res_col_idx, &counters->n_mixed);
     return cudaGetLastError();
 }
 

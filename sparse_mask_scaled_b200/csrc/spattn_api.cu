@@ -12,8 +12,10 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 using namespace spattn;
 
@@ -51,6 +53,24 @@ struct spattn_mask_s {
     void* block_csr;   // row_ptr, long_rows
     void* block_col;   // col_idx
     void* block_plan;  // block_tile_off, tile_info, tile_bits, res_row_ptr, res_col_idx, res_long
+    // Implicit interval masks (SLIDING, VARWIN, DENSE): per-row runs and the
+    // tile map are what the forward pass reads; row_ptr / col_idx and the
+    // explicit plan arrays above are written only when asked for.
+    bool implicit;
+    int kind;
+    int32_t window;
+    int min_nnz;         // selection threshold, 0 = no tile plan
+    int32_t nkt;
+    int2* lohi;          // [rows]
+    int32_t* tmap;       // [nblocks * nkt]: tile id or -1
+    int32_t* blk_res;    // [nblocks]
+    void* block_itv;     // lohi, tmap, block_tile_off, tile_info, blk_res
+    ItvCounters* cnt_host;  // mapped host memory the build writes its totals to
+    ItvCounters* cnt_dev;   // the same memory as the device addresses it
+    cudaEvent_t built;      // recorded after the build
+    bool counters_valid;    // cnt_host has been read into the fields above
+    bool plan_written;      // the explicit plan arrays exist
+    bool host_no_residual;  // known from the parameters: every entry lies in a selected tile
 };
 
 namespace {
@@ -115,6 +135,57 @@ template <typename T>
 cudaError_t pool_alloc(T** ptr, int64_t elems, cudaMemPool_t pool, cudaStream_t s) {
     const size_t bytes = (size_t)(elems > 0 ? elems : 1) * sizeof(T);
     return cudaMallocFromPoolAsync(reinterpret_cast<void**>(ptr), bytes, pool, s);
+}
+
+// Mapped host slots for the totals of an interval-mask build, each with an
+// event, recycled once the build that last wrote the slot has completed (a
+// destroyed mask's build may still be running).
+struct HostSlot {
+    ItvCounters* host;
+    ItvCounters* dev;
+    cudaEvent_t ev;
+};
+std::mutex g_slot_mu;
+std::vector<HostSlot> g_slot_free[kMaxDevices], g_slot_pending[kMaxDevices];
+constexpr int kSlotChunk = 64;
+
+cudaError_t get_slot(int dev, HostSlot* out) {
+    std::lock_guard<std::mutex> lk(g_slot_mu);
+    std::vector<HostSlot>& pend = g_slot_pending[dev];
+    std::vector<HostSlot>& fr = g_slot_free[dev];
+    for (size_t x = 0; x < pend.size();) {
+        if (cudaEventQuery(pend[x].ev) == cudaSuccess) {
+            fr.push_back(pend[x]);
+            pend[x] = pend.back();
+            pend.pop_back();
+        } else {
+            ++x;
+        }
+    }
+    (void)cudaGetLastError();  // a not-ready query is not an error of the next call
+    if (fr.empty()) {
+        void* h = nullptr;
+        cudaError_t e = cudaHostAlloc(&h, sizeof(ItvCounters) * kSlotChunk,
+                                      cudaHostAllocMapped | cudaHostAllocPortable);
+        if (e != cudaSuccess) return e;
+        void* d = nullptr;
+        if ((e = cudaHostGetDevicePointer(&d, h, 0)) != cudaSuccess) return e;
+        for (int x = 0; x < kSlotChunk; ++x) {
+            HostSlot sl;
+            sl.host = static_cast<ItvCounters*>(h) + x;
+            sl.dev = static_cast<ItvCounters*>(d) + x;
+            if ((e = cudaEventCreateWithFlags(&sl.ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+            fr.push_back(sl);
+        }
+    }
+    *out = fr.back();
+    fr.pop_back();
+    return cudaSuccess;
+}
+
+void put_slot(int dev, const HostSlot& sl) {
+    std::lock_guard<std::mutex> lk(g_slot_mu);
+    g_slot_pending[dev].push_back(sl);
 }
 
 int elem_size(int32_t dtype) { return dtype == SPATTN_BF16 ? 2 : 4; }
@@ -263,6 +334,343 @@ int build_status(unsigned err) {
     return SPATTN_OK;
 }
 
+// Device address of the device error flags, looked up once per device.
+int err_flags_ptr(int dev, unsigned** out) {
+    if (!g_err_ptr[dev]) {
+        unsigned* ep = nullptr;
+        CUDA_TRY(error_flag_address(&ep), "error flag address");
+        g_err_ptr[dev] = ep;
+    }
+    *out = g_err_ptr[dev];
+    return SPATTN_OK;
+}
+
+// ---------------------------------------------------------- interval masks
+
+bool implicit_kind(int kind) {
+    return kind == SPATTN_MASK_SLIDING || kind == SPATTN_MASK_VARWIN || kind == SPATTN_MASK_DENSE;
+}
+
+// Whether every entry of a SLIDING or DENSE mask lies in a tile of at least
+// min_nnz entries -- then the forward pass needs no gather kernel. Exact (the
+// build's tile counts, from the parameters); false when unknown or when
+// telling would cost more than a few million steps.
+bool interval_all_in_tiles(int kind, int64_t n, int64_t w, int min_nnz) {
+    if (min_nnz <= 0) return false;
+    const int64_t nqb = (n + kTileM - 1) / kTileM;
+    if (kind == SPATTN_MASK_DENSE) {
+        const int64_t last = n - kTileM * (nqb - 1);  // rows and keys of the ragged last tiles
+        return last * last >= min_nnz;
+    }
+    if (kind != SPATTN_MASK_SLIDING) return false;
+    const int64_t nkt = (n + kTileN - 1) / kTileN;
+    const int64_t span = std::min<int64_t>(nkt, (2 * w) / kTileN + 3);
+    if (nqb * span * kTileM > (int64_t(1) << 22)) return false;
+    for (int64_t qb = 0; qb < nqb; ++qb) {
+        const int64_t i0 = qb * kTileM, i1 = std::min<int64_t>(n, i0 + kTileM);
+        const int64_t lo_min = std::max<int64_t>(0, i0 - w), hi_max = std::min<int64_t>(n, i1 + w);
+        for (int64_t kt = lo_min / kTileN; kt <= (hi_max - 1) / kTileN; ++kt) {
+            int64_t c = 0;
+            for (int64_t i = i0; i < i1; ++i) {
+                const int64_t lo = std::max<int64_t>(0, i - w), hi = std::min<int64_t>(n, i + w + 1);
+                c += std::max<int64_t>(0, std::min<int64_t>(hi, kt * kTileN + kTileN) -
+                                              std::max<int64_t>(lo, kt * kTileN));
+            }
+            if (c > 0 && c < min_nnz) return false;
+        }
+    }
+    return true;
+}
+
+// The build's totals into the mask's fields. wait: block until the build has
+// run; else only read them if it already has (*ready tells which).
+int read_counters(spattn_mask m, bool wait, bool* ready = nullptr) {
+    if (ready) *ready = true;
+    if (!m->implicit || m->counters_valid) return SPATTN_OK;
+    if (wait) {
+        CUDA_TRY(cudaEventSynchronize(m->built), "waiting for the mask build");
+    } else {
+        const cudaError_t q = cudaEventQuery(m->built);
+        if (q == cudaErrorNotReady) {
+            (void)cudaGetLastError();
+            if (ready) *ready = false;
+            return SPATTN_OK;
+        }
+        if (q != cudaSuccess) return cuda_fail(q, "mask build");
+    }
+    const volatile ItvCounters* c = m->cnt_host;
+    m->nnz = c->nnz;
+    m->n_long = c->n_long;
+    m->n_tiles = c->n_tiles;
+    m->res_nnz = c->res_nnz;
+    m->n_tc_blocks = c->n_tc_blocks;
+    m->counters_valid = true;
+    return SPATTN_OK;
+}
+
+int create_implicit(const spattn_mask_spec& sp, cudaStream_t s, int dev, cudaMemPool_t pool,
+                    spattn_mask* out) {
+    const bool async = (sp.flags & SPATTN_MASK_ASYNC) != 0;
+    const int64_t rows = (int64_t)sp.n * sp.num_masks;
+    const int nqb = (sp.n + kTileM - 1) / kTileM, nkt = (sp.n + kTileN - 1) / kTileN;
+    const int64_t nblocks = (int64_t)sp.num_masks * nqb;
+    const int min_nnz =
+        sp.tile_min_nnz < 0 ? 0 : (sp.tile_min_nnz == 0 ? kTileMinNnzDefault : sp.tile_min_nnz);
+    unsigned* ef = nullptr;
+    if (async) {
+        const int r = err_flags_ptr(dev, &ef);
+        if (r) return r;
+    }
+    Carve c;
+    const int k_lh = c.add(rows * 8), k_tm = c.add(nblocks * nkt * 4), k_bs = c.add(nblocks * 8),
+              k_bto = c.add((nblocks + 1) * 4), k_ti = c.add(nblocks * nkt * 4), k_br = c.add(nblocks * 4);
+    void* blk = nullptr;
+    CUDA_TRY(cudaMallocFromPoolAsync(&blk, c.total, pool, s), "mask allocation");
+    HostSlot sl;
+    cudaError_t e = get_slot(dev, &sl);
+    if (e != cudaSuccess) {
+        cudaFreeAsync(blk, s);
+        return cuda_fail(e, "mapped host memory for the mask totals");
+    }
+    ItvSpec is;
+    is.kind = sp.kind;
+    is.n = sp.n;
+    is.num_masks = sp.num_masks;
+    is.window = sp.window;
+    is.half_widths = sp.half_widths;
+    is.nqb = nqb;
+    is.nkt = nkt;
+    is.err_flags = ef;
+    e = itv_build(is, c.at<int2>(blk, k_lh), c.at<int32_t>(blk, k_tm), c.at<int2>(blk, k_bs),
+                  c.at<int32_t>(blk, k_bto), c.at<int32_t>(blk, k_ti), c.at<int32_t>(blk, k_br), min_nnz,
+                  sl.dev, s);
+    if (e == cudaSuccess) e = cudaEventRecord(sl.ev, s);
+    if (e != cudaSuccess) {
+        cudaFreeAsync(blk, s);
+        put_slot(dev, sl);
+        return cuda_fail(e, "interval mask build");
+    }
+    spattn_mask m = new spattn_mask_s;
+    memset(m, 0, sizeof *m);
+    m->device = dev;
+    m->stream = s;
+    m->n = sp.n;
+    m->num_masks = sp.num_masks;
+    m->implicit = true;
+    m->kind = sp.kind;
+    m->window = sp.window;
+    m->min_nnz = min_nnz;
+    m->nqb = nqb;
+    m->nkt = nkt;
+    m->lohi = c.at<int2>(blk, k_lh);
+    m->tmap = c.at<int32_t>(blk, k_tm);
+    m->block_tile_off = c.at<int32_t>(blk, k_bto);
+    m->tile_info = c.at<int32_t>(blk, k_ti);
+    m->blk_res = c.at<int32_t>(blk, k_br);
+    m->block_itv = blk;
+    m->cnt_host = sl.host;
+    m->cnt_dev = sl.dev;
+    m->built = sl.ev;
+    m->has_plan = min_nnz > 0;
+    m->host_no_residual = interval_all_in_tiles(sp.kind, sp.n, sp.window, min_nnz);
+    if (!async) {
+        int r = read_counters(m, true);
+        const unsigned err = static_cast<const volatile ItvCounters*>(m->cnt_host)->err;
+        if (r == SPATTN_OK && err) r = build_status(err);
+        if (r != SPATTN_OK) {
+            spattn_destroy_mask(m);
+            return r;
+        }
+    }
+    *out = m;
+    return SPATTN_OK;
+}
+
+// row_ptr and col_idx of an interval mask, written on first request.
+int write_csr(spattn_mask m) {
+    if (!m->implicit || m->row_ptr) return SPATTN_OK;
+    int r = read_counters(m, true);
+    if (r) return r;
+    if (m->nnz > 0x7fffffffLL)
+        return fail(SPATTN_ERR_UNSUPPORTED, "the mask has more than 2^31 - 1 nonzeros for a CSR");
+    const int64_t rows = (int64_t)m->n * m->num_masks;
+    cudaMemPool_t pool;
+    CUDA_TRY(device_state(m->device, &pool, nullptr), "memory pool");
+    cudaStream_t s = m->stream;
+    Carve ct;
+    const int k_cnt = ct.add(rows * 4), k_scan = ct.add(scan_tmp_elems(rows) * 8), k_tot = ct.add(16);
+    void *a = nullptr, *t = nullptr, *col = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync(&a, (size_t)(rows + 1) * 4, pool, s);
+    if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&t, ct.total, pool, s);
+    if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&col, (size_t)(m->nnz > 0 ? m->nnz : 1) * 4, pool, s);
+    if (e == cudaSuccess) {
+        int64_t* tot = ct.at<int64_t>(t, k_tot);
+        e = itv_write_csr(m->lohi, rows, ct.at<int32_t>(t, k_cnt), static_cast<int32_t*>(a),
+                          static_cast<int32_t*>(col), ct.at<int64_t>(t, k_scan), tot,
+                          reinterpret_cast<unsigned*>(tot + 1), s);
+    }
+    if (t) cudaFreeAsync(t, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) {
+        if (a) cudaFreeAsync(a, s);
+        if (col) cudaFreeAsync(col, s);
+        return cuda_fail(e, "writing the mask's CSR");
+    }
+    m->block_csr = a;
+    m->block_col = col;
+    m->row_ptr = static_cast<int32_t*>(a);
+    m->col_idx = static_cast<int32_t*>(col);
+    return SPATTN_OK;
+}
+
+// The explicit plan arrays of an interval mask (tile bits, residual CSR) and
+// its mixed-row count, written on first request.
+int write_plan(spattn_mask m) {
+    if (!m->implicit || m->plan_written) return SPATTN_OK;
+    int r = read_counters(m, true);
+    if (r) return r;
+    if (m->n_tiles == 0) {
+        m->plan_written = true;
+        return SPATTN_OK;
+    }
+    const int64_t rows = (int64_t)m->n * m->num_masks;
+    cudaMemPool_t pool;
+    CUDA_TRY(device_state(m->device, &pool, nullptr), "memory pool");
+    cudaStream_t s = m->stream;
+    Carve cp;
+    const int k_tb = cp.add(m->n_tiles * kTileM * 16), k_rrp = cp.add((rows + 1) * 4),
+              k_rci = cp.add(m->res_nnz * 4), k_rl = cp.add(rows * 4);
+    Carve ct;
+    const int k_pc = ct.add(sizeof(PlanCounters)), k_rc = ct.add(rows * 4),
+              k_st = ct.add(scan_tmp_elems(rows) * 8);
+    void *a = nullptr, *t = nullptr;
+    PlanCounters hpc;
+    cudaError_t e = cudaMallocFromPoolAsync(&a, cp.total, pool, s);
+    if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&t, ct.total, pool, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ct.at<PlanCounters>(t, k_pc), 0, sizeof(PlanCounters), s);
+    if (e == cudaSuccess) {
+        PlanBuffers pb;
+        memset(&pb, 0, sizeof pb);
+        pb.cnt_map = m->tmap;
+        pb.block_tile_off = m->block_tile_off;
+        pb.tile_info = m->tile_info;
+        pb.tile_cap = m->n_tiles;
+        pb.tile_bits = cp.at<uint32_t>(a, k_tb);
+        pb.res_row_ptr = cp.at<int32_t>(a, k_rrp);
+        pb.res_col_idx = cp.at<int32_t>(a, k_rci);
+        pb.res_long = cp.at<int32_t>(a, k_rl);
+        pb.res_cnt = ct.at<int32_t>(t, k_rc);
+        pb.scan_tmp = ct.at<int64_t>(t, k_st);
+        e = itv_write_plan(m->lohi, m->n, m->num_masks, pb, ct.at<PlanCounters>(t, k_pc), s);
+    }
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(&hpc, ct.at<PlanCounters>(t, k_pc), sizeof hpc, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (t) cudaFreeAsync(t, s);
+    if (e != cudaSuccess) {
+        if (a) cudaFreeAsync(a, s);
+        return cuda_fail(e, "writing the mask's tile plan");
+    }
+    m->block_plan = a;
+    m->tile_bits = cp.at<uint32_t>(a, k_tb);
+    m->res_row_ptr = cp.at<int32_t>(a, k_rrp);
+    m->res_col_idx = cp.at<int32_t>(a, k_rci);
+    m->res_long = cp.at<int32_t>(a, k_rl);
+    m->n_mixed = hpc.n_mixed;
+    m->res_n_long = hpc.res_n_long;
+    m->plan_written = true;
+    return SPATTN_OK;
+}
+
+
+// The tensor-core kernel over the mask's tiles; blk_res: interval masks whose
+// gather kernel ran (its partial states are in p.ws_ml / p.ws_acc).
+int launch_tc(const FwdParams& p, int d, spattn_mask m, int dev, const int32_t* blk_res,
+              cudaStream_t s) {
+    unsigned* ef = nullptr;
+    int r = err_flags_ptr(dev, &ef);
+    if (r) return r;
+    TcParams tp;
+    memset(&tp, 0, sizeof tp);
+    tp.B = p.B;
+    tp.H = p.H;
+    tp.n = p.n;
+    tp.num_masks = m->num_masks;
+    tp.nqb = m->nqb;
+    tp.block_tile_off = m->block_tile_off;
+    tp.tile_info = m->tile_info;
+    if (m->implicit) {
+        tp.itv_lohi = m->lohi;
+        tp.blk_res = blk_res;
+    } else {
+        tp.tile_bits = m->tile_bits;
+        tp.res_row_ptr = m->res_row_ptr;
+    }
+    tp.ws_ml = p.ws_ml;
+    tp.ws_acc = p.ws_acc;
+    tp.out = p.out;
+    tp.o_sb = p.o_sb;
+    tp.o_sh = p.o_sh;
+    tp.o_sn = p.o_sn;
+    tp.lse = p.lse;
+    tp.mask = p.mask;
+    tp.bias = p.bias;
+    tp.has_extra = p.has_extra;
+    tp.qk_scale_log2 = p.qk_scale_log2;
+    tp.err = ef;
+    const TcOperand oq{p.q, p.q_sn, p.q_sh, p.q_sb}, ok{p.k, p.k_sn, p.k_sh, p.k_sb},
+        ov{p.v, p.v_sn, p.v_sh, p.v_sb};
+    const cudaError_t e = launch_fwd_tc(oq, ok, ov, d, tp, s);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core kernel launch");
+    return SPATTN_OK;
+}
+
+// Forward over an interval mask. Without tensor-core tiles (fp32, no plan, or
+// none selected) the interval gather kernel does every entry. With tiles it
+// runs first only when entries outside the tiles may exist -- known exactly
+// once the build's totals are in (it does not wait for them) or, before that,
+// from the pattern's parameters -- and hands partial states to the
+// tensor-core kernel.
+int fwd_interval(FwdParams& p, int dtype, int d, spattn_mask m, cudaStream_t s, cudaMemPool_t pool,
+                 int dev, int num_sms) {
+    p.itv_lohi = m->lohi;
+    p.nkt = m->nkt;
+    p.nqb = m->nqb;
+    // split query blocks until there are about four thread blocks per SM
+    const int64_t qblocks = (int64_t)p.B * p.H * p.nqb;
+    p.itv_slices = 1;
+    while (p.itv_slices < 16 && qblocks * p.itv_slices < 4LL * num_sms) p.itv_slices *= 2;
+    bool ready = false;
+    int r = read_counters(m, false, &ready);
+    if (r) return r;
+    const bool tc = m->min_nnz > 0 && dtype == 0 && !(ready && m->n_tiles == 0);
+    if (!tc) {
+        const cudaError_t e = launch_fwd_itv(p, dtype, d, s);
+        if (e != cudaSuccess) return cuda_fail(e, "interval gather kernel launch");
+        return SPATTN_OK;
+    }
+    const int64_t nblocks = (int64_t)m->num_masks * m->nqb;
+    const bool gather = ready ? (m->res_nnz > 0 || m->n_tc_blocks < nblocks) : !m->host_no_residual;
+    float* ws = nullptr;
+    if (gather) {
+        const int64_t rows_all = (int64_t)p.B * p.H * p.n;
+        CUDA_TRY(pool_alloc(&ws, rows_all * (d + 2), pool, s), "partial-state workspace");
+        p.ws_ml = ws;
+        p.ws_acc = ws + rows_all * 2;
+        p.tmap = m->tmap;
+        p.qb_tile_off = m->block_tile_off;
+        p.blk_res = m->blk_res;
+        const cudaError_t e = launch_fwd_itv(p, dtype, d, s);
+        if (e != cudaSuccess) {
+            cudaFreeAsync(ws, s);
+            return cuda_fail(e, "interval gather kernel launch");
+        }
+    }
+    r = launch_tc(p, d, m, dev, gather ? m->blk_res : nullptr, s);
+    if (ws) cudaFreeAsync(ws, s);
+    return r;
+}
+
 }  // namespace
 
 extern "C" {
@@ -292,7 +700,7 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
     if (sp.kind == SPATTN_MASK_BLOCK_STRIDED_GLOBAL &&
         (sp.block < 0 || sp.stride < 0 || sp.n_global < 0))
         return fail(SPATTN_ERR_INVALID_ARG, "block, stride and n_global must be >= 0");
-    if (sp.reserved != 0) return fail(SPATTN_ERR_INVALID_ARG, "spec.reserved must be 0");
+    if (sp.flags & ~(uint32_t)SPATTN_MASK_ASYNC) return fail(SPATTN_ERR_INVALID_ARG, "unknown spec.flags bits");
     if (sp.kind == SPATTN_MASK_CSR || sp.kind == SPATTN_MASK_COO) {
         if (!sp.in_row_ptr) return fail(SPATTN_ERR_INVALID_ARG, "in_row_ptr is NULL");
         if (sp.in_nnz < 0 || sp.in_nnz > 0x7fffffff)
@@ -304,6 +712,10 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
     CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
     cudaMemPool_t pool;
     CUDA_TRY(device_state(dev, &pool, nullptr), "memory pool");
+
+    const int nqb_i = (sp.n + kTileM - 1) / kTileM;
+    if (implicit_kind(sp.kind) && nqb_i <= kItvMaxKeyTiles && (int64_t)sp.num_masks * nqb_i <= kItvMaxBlocks)
+        return create_implicit(sp, s, dev, pool, out);
 
     BuildSpec bs;
     bs.kind = sp.kind;
@@ -445,7 +857,9 @@ int spattn_mask_copy_plan(spattn_mask m, int32_t* block_tile_off, int32_t* tile_
                           void* stream_v) {
     g_msg[0] = 0;
     if (!m) return fail(SPATTN_ERR_INVALID_ARG, "mask is NULL");
-    if (!m->has_plan) return fail(SPATTN_ERR_INVALID_ARG, "the mask has no tile plan");
+    int r = write_plan(m);
+    if (r) return r;
+    if (!m->has_plan || m->n_tiles == 0) return fail(SPATTN_ERR_INVALID_ARG, "the mask has no tile plan");
     cudaStream_t s = (cudaStream_t)stream_v;
     const int64_t rows = (int64_t)m->n * m->num_masks;
     const int64_t nblocks = (int64_t)m->num_masks * m->nqb;
@@ -470,6 +884,9 @@ int spattn_mask_plan_info(spattn_mask m, int64_t* n_tiles, int64_t* residual_nnz
                           int64_t* n_mixed_rows) {
     g_msg[0] = 0;
     if (!m) return fail(SPATTN_ERR_INVALID_ARG, "mask is NULL");
+    int r = read_counters(m, true);
+    if (r == SPATTN_OK && n_mixed_rows) r = write_plan(m);
+    if (r) return r;
     if (n_tiles) *n_tiles = m->has_plan ? m->n_tiles : 0;
     if (residual_nnz) *residual_nnz = m->has_plan ? m->res_nnz : m->nnz;
     if (n_mixed_rows) *n_mixed_rows = m->has_plan ? m->n_mixed : 0;
@@ -480,6 +897,10 @@ int spattn_mask_info(spattn_mask m, int32_t* n, int32_t* num_masks, int64_t* nnz
                      const int32_t** row_ptr, const int32_t** col_idx, int64_t* n_long) {
     g_msg[0] = 0;
     if (!m) return fail(SPATTN_ERR_INVALID_ARG, "mask is NULL");
+    int r = SPATTN_OK;
+    if (nnz || n_long) r = read_counters(m, true);
+    if (r == SPATTN_OK && (row_ptr || col_idx)) r = write_csr(m);
+    if (r) return r;
     if (n) *n = m->n;
     if (num_masks) *num_masks = m->num_masks;
     if (nnz) *nnz = m->nnz;
@@ -493,6 +914,10 @@ int spattn_mask_copy_csr(spattn_mask m, int32_t* row_ptr_dst, int32_t* col_idx_d
                          void* stream_v) {
     g_msg[0] = 0;
     if (!m) return fail(SPATTN_ERR_INVALID_ARG, "mask is NULL");
+    if (row_ptr_dst || col_idx_dst) {
+        const int r = write_csr(m);
+        if (r) return r;
+    }
     cudaStream_t s = (cudaStream_t)stream_v;
     const int64_t rows = (int64_t)m->n * m->num_masks;
     if (row_ptr_dst)
@@ -516,6 +941,14 @@ int spattn_destroy_mask(spattn_mask m) {
     if (m->block_csr && (e2 = cudaFreeAsync(m->block_csr, m->stream)) != cudaSuccess) e = e2;
     if (m->block_col && (e2 = cudaFreeAsync(m->block_col, m->stream)) != cudaSuccess) e = e2;
     free_plan(m);
+    if (m->block_itv && (e2 = cudaFreeAsync(m->block_itv, m->stream)) != cudaSuccess) e = e2;
+    if (m->cnt_host) {
+        HostSlot sl;
+        sl.host = m->cnt_host;
+        sl.dev = m->cnt_dev;
+        sl.ev = m->built;
+        put_slot(m->device, sl);
+    }
     if (prev >= 0 && prev != m->device) cudaSetDevice(prev);
     delete m;
     if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync");
@@ -586,6 +1019,7 @@ int spattn_fwd_mask(const spattn_tensor* q, const spattn_tensor* k, const spattn
     CUDA_TRY(device_state(dev, &pool, &sms), "memory pool");
     p.num_masks = mask->num_masks;
     p.long_count_dev = nullptr;
+    if (mask->implicit) return fwd_interval(p, dtype, d, mask, s, pool, dev, sms);
     if (!(mask->has_plan && dtype == 0)) {  // every entry on the gather kernel
         p.row_ptr = mask->row_ptr;
         p.col_idx = mask->col_idx;
@@ -617,40 +1051,9 @@ int spattn_fwd_mask(const spattn_tensor* q, const spattn_tensor* k, const spattn
             return r;
         }
     }
-    if (!g_err_ptr[dev]) {
-        unsigned* ep = nullptr;
-        CUDA_TRY(error_flag_address(&ep), "error flag address");
-        g_err_ptr[dev] = ep;
-    }
-    TcParams tp;
-    memset(&tp, 0, sizeof tp);
-    tp.B = p.B;
-    tp.H = p.H;
-    tp.n = p.n;
-    tp.num_masks = mask->num_masks;
-    tp.nqb = mask->nqb;
-    tp.block_tile_off = mask->block_tile_off;
-    tp.tile_info = mask->tile_info;
-    tp.tile_bits = mask->tile_bits;
-    tp.res_row_ptr = mask->res_row_ptr;
-    tp.ws_ml = p.ws_ml;
-    tp.ws_acc = p.ws_acc;
-    tp.out = p.out;
-    tp.o_sb = p.o_sb;
-    tp.o_sh = p.o_sh;
-    tp.o_sn = p.o_sn;
-    tp.lse = p.lse;
-    tp.mask = p.mask;
-    tp.bias = p.bias;
-    tp.has_extra = p.has_extra;
-    tp.qk_scale_log2 = p.qk_scale_log2;
-    tp.err = g_err_ptr[dev];
-    const TcOperand oq{p.q, p.q_sn, p.q_sh, p.q_sb}, ok{p.k, p.k_sn, p.k_sh, p.k_sb},
-        ov{p.v, p.v_sn, p.v_sh, p.v_sb};
-    cudaError_t e = launch_fwd_tc(oq, ok, ov, d, tp, s);
+    r = launch_tc(p, d, mask, dev, nullptr, s);
     if (ws) cudaFreeAsync(ws, s);
-    if (e != cudaSuccess) return cuda_fail(e, "tensor-core kernel launch");
-    return SPATTN_OK;
+    return r;
 }
 
 // ---- allocation-free forward: its scratch is this fixed array, part of the

@@ -63,6 +63,16 @@ struct FwdParams {
     int nqb;
     float* ws_ml;   // [B*H*n*2]
     float* ws_acc;  // [B*H*n*d]
+    // Interval masks (k_fwd_itv): row m*n + i is the run [lo, hi) of itv_lohi.
+    // With a tile plan (tmap != nullptr) only the parts in unselected key tiles
+    // (tmap[blk * nkt + kt] < 0) are gathered; the rows of a query block with
+    // tiles hand their partial state to the tensor-core kernel, and only blocks
+    // flagged in blk_res have any.
+    const int2* itv_lohi;
+    const int32_t* tmap;
+    const int32_t* blk_res;
+    int nkt;
+    int itv_slices;  // 1, 2, 4, 8 or 16 thread blocks per 128-row query block
 };
 
 // Tensor-core kernel (fwd_tc.cu).
@@ -76,6 +86,10 @@ struct TcParams {
     const int32_t* tile_info;       // key tile | kTileDenseBit
     const uint32_t* tile_bits;      // [tiles][128 rows][4 words]
     const int32_t* res_row_ptr;     // residual CSR (a row with entries has a partial)
+    // Interval masks: masks come from the row runs instead of tile_bits, and the
+    // rows of blocks flagged in blk_res have a partial (used when its l > 0).
+    const int2* itv_lohi;
+    const int32_t* blk_res;
     const float* ws_ml;             // partials from the gather kernel, or nullptr
     const float* ws_acc;
     void* out;
@@ -124,6 +138,44 @@ cudaError_t build_plan(const int32_t* row_ptr, const int32_t* col_idx, int n, in
                        int64_t nnz, int min_nnz, bool intervals, bool zeroed, bool precounted,
                        const PlanBuffers& b, PlanCounters* counters, cudaStream_t s);
 
+// Implicit interval masks (plan.cu). SLIDING, VARWIN and DENSE rows are single
+// runs [lo, hi); such a mask keeps the runs (int2 per row) and its tile plan,
+// and writes a CSR only when one is asked for.
+struct ItvSpec {
+    int kind, n, num_masks, window;
+    const int32_t* half_widths;  // VARWIN
+    int nqb, nkt;
+    unsigned* err_flags;  // nullable: negative half-widths also raise kErrBadColumn here
+};
+// Results of the build, written by one thread at the end of the select kernel.
+struct ItvCounters {
+    int64_t nnz;
+    int64_t n_tiles;
+    int64_t res_nnz;      // entries outside tensor-core tiles
+    int32_t n_long;       // rows with more than kLongRowThreshold entries
+    int32_t n_tc_blocks;  // query blocks with at least one tile
+    unsigned err;         // kBuildNegativeWidth
+    int32_t pad;
+};
+constexpr int kItvMaxKeyTiles = 8192;   // per-block tile counts live in shared memory
+constexpr int64_t kItvMaxBlocks = 1 << 16;  // the select kernel is one thread block
+// Rows, per-tile counts and selection: two launches, no host synchronisation.
+// cnt: int32 [nblocks * nkt] (becomes the tile map: tile id or -1); bstat: int2
+// [nblocks] scratch; tile_info: int32 [nblocks * nkt]; min_nnz <= 0: select none.
+cudaError_t itv_build(const ItvSpec& s, int2* lohi, int32_t* cnt, int2* bstat, int32_t* block_tile_off,
+                      int32_t* tile_info, int32_t* blk_res, int min_nnz, ItvCounters* counters,
+                      cudaStream_t stream);
+// CSR of an interval mask: counts (scratch int32 [rows]) -> row_ptr [rows + 1]
+// -> col_idx [nnz]. scan_tmp: int64 [scan_tmp_elems(rows)], total/err: device scalars.
+cudaError_t itv_write_csr(const int2* lohi, int64_t rows, int32_t* counts, int32_t* row_ptr,
+                          int32_t* col_idx, int64_t* scan_tmp, int64_t* total, unsigned* err,
+                          cudaStream_t stream);
+// The explicit plan of an interval mask (tile_bits, residual CSR, mixed-row
+// count) from its runs and tile map, as build_plan writes it for CSR masks.
+// b.cnt_map is the tile map; counters->res_n_long, n_mixed must start at 0.
+cudaError_t itv_write_plan(const int2* lohi, int n, int num_masks, const PlanBuffers& b,
+                           PlanCounters* counters, cudaStream_t stream);
+
 // ---------------------------------------------------------------- launchers
 // All launchers enqueue on `stream` and return the cudaGetLastError() result.
 
@@ -136,6 +188,8 @@ cudaError_t launch_fwd_long_rows(const FwdParams& p, int dtype, int d, int num_s
 cudaError_t launch_classify_long_rows(const int32_t* row_ptr, int64_t rows, int64_t nnz,
                                       int32_t* list, int32_t* count, cudaStream_t stream);
 cudaError_t read_and_clear_device_error(unsigned* flags, cudaStream_t stream);
+// Interval-mask gather (fields itv_lohi / tmap / blk_res / nkt of p).
+cudaError_t launch_fwd_itv(const FwdParams& p, int dtype, int d, cudaStream_t stream);
 
 // Mask builder (mask_build.cu).
 struct BuildSpec {

@@ -32,12 +32,13 @@ def device_inputs(wl: workloads.Workload, device="cuda"):
     return q, k, v, m, b
 
 
-def build_mask(mp: workloads.MaskParams, stream=None):
+def build_mask(mp: workloads.MaskParams, stream=None, tile_min_nnz=0, asynchronous=False):
     """The CUDA mask builder, from the same parameters the oracle builds from."""
     import torch
     import sparse_mask_scaled_b200 as sp
     kw = dict(window=mp.window, block=mp.block, stride=mp.stride, n_global=mp.n_global,
-              add_diagonal=mp.add_diagonal, stream=stream)
+              add_diagonal=mp.add_diagonal, stream=stream, tile_min_nnz=tile_min_nnz,
+              asynchronous=asynchronous)
     if mp.kind == "varwin":
         kw["half_widths"] = torch.from_numpy(np.ascontiguousarray(mp.half_widths, np.int32).ravel()).cuda()
     if mp.kind == "coo":

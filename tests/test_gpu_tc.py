@@ -287,15 +287,14 @@ def _check_interval_plan(mask, rp, ci, n, nm, thr):
     assert np.all(np.diff(rci)[same] > 0)
 
 
-@pytest.mark.parametrize("n,thr", [(32000, 9000), (33000, 9000), (33000, 0)])
-def test_interval_plan_both_build_paths(n, thr):
-    """Two masks of n rows each: up to 65,536 rows the mask build runs as one
-    launch that also clears the plan's counts, and the column fill counts the
-    tiles; above it the plan clears and counts by itself. Both must give the
-    same plan and forward."""
+@pytest.mark.parametrize("n,thr,asynchronous", [(32000, 9000, False), (33000, 9000, True), (33000, 0, True)])
+def test_interval_plan_at_scale(n, thr, asynchronous):
+    """Two variable-window masks of n = 32,000 or 33,000 rows each (500 or 516 query blocks):
+    the tile selection, every tile bit and the residual CSR that the interval
+    mask writes on request, and the forward on sampled rows."""
     wl = workloads.make(1, B=2, H=1, n=n)
     rp, ci = oracle.mask_from_params(wl.mask)
-    with _mask_with_thr(wl.mask, thr) as m:
+    with build_mask(wl.mask, tile_min_nnz=thr, asynchronous=asynchronous) as m:
         grp, gci = m.csr()
         assert np.array_equal(grp.cpu().numpy(), rp) and np.array_equal(gci.cpu().numpy(), ci)
         _check_interval_plan(m, rp, ci, n, wl.mask.num_masks, 512 if thr == 0 else thr)
