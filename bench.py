@@ -399,6 +399,8 @@ def bench_ours(args, rank, world, torch, sp):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "step": "device mask build (pattern -> CSR -> row schedule + tile plan) + fused forward",
                    "plan_per_mask_set": plan},
+        "step_ms": {"min": round(min(step_ms), 4), "median": round(statistics.median(step_ms), 4),
+                    "max": round(max(step_ms), 4)},
         "fwd": {"ms": round(t_fwd, 4), "tflops": round(flops / (t_fwd * 1e-3) / 1e12, 3),
                 "effective_gbs": round(eff_gbs, 1)},
         "roofline": roofline,
