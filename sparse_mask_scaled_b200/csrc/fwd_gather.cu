@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(256, 2) k_fwd_itv(const FwdParams P) {
     bool partial = false;
     if (P.tmap) {
         tm = P.tmap + blk * P.nkt;
-        if (P.qb_tile_off[blk + 1] > P.qb_tile_off[blk]) {
+        if (P.qb_ntiles[blk] > 0) {
             if (!P.blk_res[blk]) return;  // the tensor-core kernel does every row alone
             partial = true;
         }

@@ -390,17 +390,28 @@ __global__ void k_plan_zero(int32_t* __restrict__ cnt, int64_t n_cnt, PlanCounte
 }
 
 // ------------------------------------------------- implicit interval masks
-// Step 1, one CTA of 128 threads per query block (128 rows of one mask): each
-// row's run [lo, hi) from the pattern, the block's entry count per key tile
-// (all nkt of them, zeros included, so nothing needs clearing first) and, per
-// block, the rows above kLongRowThreshold entries and the rows with a negative
-// half-width (which are left empty).
+// One CTA of 128 threads per query block (128 rows of one mask): each row's run
+// [lo, hi) from the pattern (a negative half-width leaves the row empty), the
+// block's entry count per key tile accumulated in shared memory (a warp
+// reduction and one shared atomic per tile and warp), the tile selection -- the
+// tiles with at least min_nnz entries, listed in key order at tiles[blk * nkt ..]
+// (bit 31: all 128 x 128 entries present), the map tmap[blk * nkt + kt] = local
+// tile number or -1, whether entries stay outside the selected tiles -- and the
+// block's statistics. The last CTA to finish (a self-resetting counter) adds the
+// statistics up into the mask's totals.
 __global__ void __launch_bounds__(kTileM)
-    k_itv_rows(ItvSpec s, int2* __restrict__ lohi, int32_t* __restrict__ cnt, int2* __restrict__ bstat) {
+    k_itv_build(ItvSpec s, int min_nnz, int2* __restrict__ lohi, int32_t* __restrict__ tmap,
+                int32_t* __restrict__ tiles, int32_t* __restrict__ ntiles, int32_t* __restrict__ blk_res,
+                ItvBlockStat* bstat, unsigned* done, ItvCounters* out) {
     extern __shared__ int32_t cs[];  // [nkt]
+    __shared__ int32_t wsel[4];
+    __shared__ long long wsum[2][4];
+    __shared__ bool last_s;
+    const int64_t nblocks = (int64_t)gridDim.x;
     const int64_t blk = blockIdx.x;
     const int64_t m = blk / s.nqb;
     const int qb = (int)(blk - m * s.nqb);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int kt = threadIdx.x; kt < s.nkt; kt += kTileM) cs[kt] = 0;
     __syncthreads();
     const int i = qb * kTileM + threadIdx.x;
@@ -421,152 +432,126 @@ __global__ void __launch_bounds__(kTileM)
         }
         lohi[r] = make_int2(lo, hi);
     }
-    const int lane = threadIdx.x & 31;
-    const bool any = hi > lo;
-    int k0 = any ? lo >> 7 : 0x7fffffff, k1 = any ? (hi - 1) >> 7 : -1;
+    {
+        const bool any = hi > lo;
+        int k0 = any ? lo >> 7 : 0x7fffffff, k1 = any ? (hi - 1) >> 7 : -1;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        k0 = min(k0, __shfl_xor_sync(0xffffffffu, k0, off));
-        k1 = max(k1, __shfl_xor_sync(0xffffffffu, k1, off));
-    }
-    for (int kt = k0; kt <= k1; ++kt) {  // one shared atomic per tile and warp
-        int c = overlap(lo, hi, kt * kTileN, kt * kTileN + kTileN);
+        for (int off = 16; off > 0; off >>= 1) {
+            k0 = min(k0, __shfl_xor_sync(0xffffffffu, k0, off));
+            k1 = max(k1, __shfl_xor_sync(0xffffffffu, k1, off));
+        }
+        for (int kt = k0; kt <= k1; ++kt) {
+            int c = overlap(lo, hi, kt * kTileN, kt * kTileN + kTileN);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
-        if (lane == 0 && c) atomicAdd(&cs[kt], c);
+            for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+            if (lane == 0 && c) atomicAdd(&cs[kt], c);
+        }
     }
     const int n_long = __syncthreads_count(hi - lo > kLongRowThreshold);
     const int n_bad = __syncthreads_count(bad);
-    for (int kt = threadIdx.x; kt < s.nkt; kt += kTileM) cnt[blk * s.nkt + kt] = cs[kt];
-    if (threadIdx.x == 0) bstat[blk] = make_int2(n_long, n_bad);
-    if (bad && s.err_flags) atomicOr(s.err_flags, kErrBadColumn);
-}
-
-// Step 2, one thread block: the selection of k_tile_select_fused (tiles with at
-// least min_nnz entries, numbered block-major; the count array becomes the
-// tile map), plus, per query block, whether it keeps entries outside its
-// selected tiles (blk_res), and the mask's totals -- written, not accumulated.
-__global__ void __launch_bounds__(1024)
-    k_itv_select(int32_t* __restrict__ cnt_map, int nblocks, int nkt, int min_nnz,
-                 const int2* __restrict__ bstat, int32_t* __restrict__ block_tile_off,
-                 int32_t* __restrict__ tile_info, int32_t* __restrict__ blk_res, ItvCounters* out) {
-    __shared__ int32_t wsum[32];
-    __shared__ int32_t carry_s;
-    __shared__ unsigned long long s_nnz, s_res;
-    __shared__ int s_long, s_bad, s_tcb;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (threadIdx.x == 0) {
-        carry_s = 0;
-        s_nnz = s_res = 0ull;
-        s_long = s_bad = s_tcb = 0;
-    }
-    __syncthreads();
-    unsigned long long nnz = 0, res = 0;
-    int nlong = 0, nbad = 0, tcb = 0;
-    for (int x0 = 0; x0 < nblocks; x0 += 1024) {
-        const int x = x0 + threadIdx.x;
-        int c = 0;
-        if (x < nblocks) {
-            const int32_t* row = cnt_map + (int64_t)x * nkt;
-            int64_t bn = 0, br = 0;
-            int kt = 0;
-            for (; kt + 8 <= nkt; kt += 8) {  // eight independent loads in flight
-                int32_t v[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) v[u] = row[kt + u];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const bool sel = min_nnz > 0 && v[u] >= min_nnz;
-                    c += sel;
-                    bn += v[u];
-                    br += sel ? 0 : v[u];
-                }
-            }
-            for (; kt < nkt; ++kt) {
-                const int32_t v = row[kt];
-                const bool sel = min_nnz > 0 && v >= min_nnz;
-                c += sel;
-                bn += v;
-                br += sel ? 0 : v;
-            }
-            blk_res[x] = br > 0;
-            nnz += bn;
-            res += br;
-            tcb += c > 0;
-            const int2 st = bstat[x];
-            nlong += st.x;
-            nbad += st.y;
-        }
-        int inc = c;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, inc, off);
-            if (lane >= off) inc += y;
-        }
-        if (lane == 31) wsum[warp] = inc;
+    // selection, 128 key tiles at a time, numbered in key order
+    long long nnz = 0, res = 0;
+    int base = 0;
+    for (int c0 = 0; c0 < s.nkt; c0 += kTileM) {
+        const int kt = c0 + threadIdx.x;
+        const int v = kt < s.nkt ? cs[kt] : 0;
+        const bool sel = min_nnz > 0 && v >= min_nnz;
+        const unsigned bal = __ballot_sync(0xffffffffu, sel);
+        if (lane == 0) wsel[warp] = __popc(bal);
         __syncthreads();
-        if (warp == 0) {
-            const int w = wsum[lane];
-            int wi = w;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, wi, off);
-                if (lane >= off) wi += y;
-            }
-            wsum[lane] = wi - w;
+        int off = base;
+        for (int w = 0; w < warp; ++w) off += wsel[w];
+        const int rank = off + __popc(bal & ((1u << lane) - 1u));
+        if (kt < s.nkt) {
+            tmap[blk * s.nkt + kt] = sel ? rank : -1;
+            if (sel) tiles[blk * s.nkt + rank] = kt | (v == kTileM * kTileN ? (int)kTileDenseBit : 0);
         }
-        __syncthreads();
-        const int carry = carry_s;
-        if (x < nblocks) block_tile_off[x] = carry + wsum[warp] + inc - c;
-        __syncthreads();
-        if (threadIdx.x == 1023) carry_s = carry + wsum[warp] + inc;
+        nnz += v;
+        res += sel ? 0 : v;
+        base += wsel[0] + wsel[1] + wsel[2] + wsel[3];
         __syncthreads();
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        nnz += __shfl_xor_sync(0xffffffffu, nnz, off);
-        res += __shfl_xor_sync(0xffffffffu, res, off);
-        nlong += __shfl_xor_sync(0xffffffffu, nlong, off);
-        nbad += __shfl_xor_sync(0xffffffffu, nbad, off);
-        tcb += __shfl_xor_sync(0xffffffffu, tcb, off);
+    for (int o = 16; o > 0; o >>= 1) {
+        nnz += __shfl_xor_sync(0xffffffffu, nnz, o);
+        res += __shfl_xor_sync(0xffffffffu, res, o);
     }
     if (lane == 0) {
-        atomicAdd(&s_nnz, nnz);
-        atomicAdd(&s_res, res);
-        atomicAdd(&s_long, nlong);
-        atomicAdd(&s_bad, nbad);
-        atomicAdd(&s_tcb, tcb);
-    }
-    // one warp per query block numbers its selected tiles
-    for (int x = warp; x < nblocks; x += 32) {
-        int idx = block_tile_off[x];
-        for (int k0 = 0; k0 < nkt; k0 += 32) {
-            const int kt = k0 + lane;
-            const int c = kt < nkt ? cnt_map[(int64_t)x * nkt + kt] : 0;
-            const bool sel = kt < nkt && min_nnz > 0 && c >= min_nnz;
-            const unsigned bal = __ballot_sync(0xffffffffu, sel);
-            if (kt < nkt) {
-                if (sel) {
-                    const int id = idx + __popc(bal & ((1u << lane) - 1u));
-                    tile_info[id] = kt | (c == kTileM * kTileN ? (int)kTileDenseBit : 0);
-                    cnt_map[(int64_t)x * nkt + kt] = id;
-                } else {
-                    cnt_map[(int64_t)x * nkt + kt] = -1;
-                }
-            }
-            idx += __popc(bal);
-        }
+        wsum[0][warp] = nnz;
+        wsum[1][warp] = res;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-        block_tile_off[nblocks] = carry_s;
-        out->nnz = (int64_t)s_nnz;
-        out->n_tiles = carry_s;
-        out->res_nnz = (int64_t)s_res;
-        out->n_long = s_long;
-        out->n_tc_blocks = s_tcb;
-        out->err = s_bad ? (unsigned)kBuildNegativeWidth : 0u;
+        ItvBlockStat st;
+        st.nnz = wsum[0][0] + wsum[0][1] + wsum[0][2] + wsum[0][3];
+        st.res = wsum[1][0] + wsum[1][1] + wsum[1][2] + wsum[1][3];
+        st.n_long = n_long;
+        st.n_bad = n_bad;
+        st.n_tiles = base;
+        st.pad = 0;
+        bstat[blk] = st;
+        ntiles[blk] = base;
+        blk_res[blk] = st.res > 0;
+        __threadfence();
+        last_s = atomicInc(done, (unsigned)(nblocks - 1)) == (unsigned)(nblocks - 1);
+    }
+    if (bad && s.err_flags) atomicOr(s.err_flags, kErrBadColumn);
+    __syncthreads();
+    if (!last_s) return;
+    // the last block: every other block's statistics are written
+    __threadfence();
+    long long t_nnz = 0, t_res = 0, t_tiles = 0;
+    int t_long = 0, t_bad = 0, t_tcb = 0;
+    const volatile ItvBlockStat* vs = bstat;
+    for (int64_t x = threadIdx.x; x < nblocks; x += kTileM) {
+        t_nnz += vs[x].nnz;
+        t_res += vs[x].res;
+        t_tiles += vs[x].n_tiles;
+        t_long += vs[x].n_long;
+        t_bad += vs[x].n_bad;
+        t_tcb += vs[x].n_tiles > 0;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        t_nnz += __shfl_xor_sync(0xffffffffu, t_nnz, o);
+        t_res += __shfl_xor_sync(0xffffffffu, t_res, o);
+        t_tiles += __shfl_xor_sync(0xffffffffu, t_tiles, o);
+        t_long += __shfl_xor_sync(0xffffffffu, t_long, o);
+        t_bad += __shfl_xor_sync(0xffffffffu, t_bad, o);
+        t_tcb += __shfl_xor_sync(0xffffffffu, t_tcb, o);
+    }
+    __shared__ long long fin[6][4];
+    if (lane == 0) {
+        fin[0][warp] = t_nnz;
+        fin[1][warp] = t_res;
+        fin[2][warp] = t_tiles;
+        fin[3][warp] = t_long;
+        fin[4][warp] = t_bad;
+        fin[5][warp] = t_tcb;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        long long f[6];
+        for (int q = 0; q < 6; ++q) f[q] = fin[q][0] + fin[q][1] + fin[q][2] + fin[q][3];
+        out->nnz = f[0];
+        out->res_nnz = f[1];
+        out->n_tiles = f[2];
+        out->n_long = (int32_t)f[3];
+        out->err = f[4] ? (unsigned)kBuildNegativeWidth : 0u;
+        out->n_tc_blocks = (int32_t)f[5];
         out->pad = 0;
+    }
+}
+
+// The per-block tile lists compacted in block order (one warp per query block).
+__global__ void k_compact_tiles(const int32_t* __restrict__ tiles, const int32_t* __restrict__ ntiles,
+                                const int32_t* __restrict__ block_tile_off, int64_t nblocks, int nkt,
+                                int32_t* __restrict__ tile_info) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t x = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5); x < nblocks; x += warps) {
+        const int64_t o = block_tile_off[x];
+        for (int r = lane; r < ntiles[x]; r += 32) tile_info[o + r] = tiles[x * nkt + r];
     }
 }
 
@@ -664,16 +649,13 @@ cudaError_t build_plan(const int32_t* row_ptr, const int32_t* col_idx, int n, in
 }
 
 
-cudaError_t itv_build(const ItvSpec& s, int2* lohi, int32_t* cnt, int2* bstat, int32_t* block_tile_off,
-                      int32_t* tile_info, int32_t* blk_res, int min_nnz, ItvCounters* counters,
-                      cudaStream_t stream) {
+cudaError_t itv_build(const ItvSpec& s, int2* lohi, int32_t* tmap, int32_t* tiles, int32_t* ntiles,
+                      int32_t* blk_res, ItvBlockStat* bstat, int min_nnz, unsigned* done,
+                      ItvCounters* counters, cudaStream_t stream) {
     const int64_t nblocks = (int64_t)s.num_masks * s.nqb;
-    if (s.nkt > kItvMaxKeyTiles || nblocks > kItvMaxBlocks) return cudaErrorInvalidValue;
-    k_itv_rows<<<(unsigned)nblocks, kTileM, (size_t)s.nkt * 4, counted(stream)>>>(s, lohi, cnt, bstat);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    k_itv_select<<<1, 1024, 0, counted(stream)>>>(cnt, (int)nblocks, s.nkt, min_nnz, bstat, block_tile_off,
-                                                  tile_info, blk_res, counters);
+    if (s.nkt > kItvMaxKeyTiles || nblocks > kItvMaxBlocks || nblocks < 1) return cudaErrorInvalidValue;
+    k_itv_build<<<(unsigned)nblocks, kTileM, (size_t)s.nkt * 4, counted(stream)>>>(
+        s, min_nnz, lohi, tmap, tiles, ntiles, blk_res, bstat, done, counters);
     return cudaGetLastError();
 }
 
@@ -691,16 +673,22 @@ cudaError_t itv_write_csr(const int2* lohi, int64_t rows, int32_t* counts, int32
     return e;
 }
 
-cudaError_t itv_write_plan(const int2* lohi, int n, int num_masks, const PlanBuffers& b,
-                           PlanCounters* counters, cudaStream_t s) {
+cudaError_t itv_write_plan(const int2* lohi, int n, int num_masks, const int32_t* tiles,
+                           const int32_t* ntiles, const PlanBuffers& b, PlanCounters* counters,
+                           cudaStream_t s) {
     const int64_t rows = (int64_t)num_masks * n;
     const int nqb = (n + kTileM - 1) / kTileM, nkt = (n + kTileN - 1) / kTileN;
     const int64_t nblocks = (int64_t)num_masks * nqb;
+    cudaError_t e = scan_counts(ntiles, nblocks, b.block_tile_off, b.scan_tmp, &counters->n_tiles,
+                                &counters->err, s);
+    if (e != cudaSuccess) return e;
+    k_compact_tiles<<<grid_for(nblocks, 8), 256, 0, counted(s)>>>(tiles, ntiles, b.block_tile_off, nblocks, nkt,
+                                                                  b.tile_info);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k_itv_bits<<<grid_for(nblocks * kTileM, 256), 256, 0, counted(s)>>>(
         nullptr, nullptr, lohi, n, nblocks, nqb, b.block_tile_off, b.tile_info, b.tile_bits, b.res_cnt,
         b.res_long, &counters->res_n_long);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     e = scan_counts(b.res_cnt, rows, b.res_row_ptr, b.scan_tmp, &counters->res_nnz, &counters->err, s);
     if (e != cudaSuccess) return e;
     k_itv_residual<<<grid_for(rows, 256), 256, 0, counted(s)>>>(nullptr, nullptr, lohi, n, rows, nqb, nkt,

@@ -62,11 +62,14 @@ struct spattn_mask_s {
     int min_nnz;         // selection threshold, 0 = no tile plan
     int32_t nkt;
     int2* lohi;          // [rows]
-    int32_t* tmap;       // [nblocks * nkt]: tile id or -1
+    int32_t* tmap;       // [nblocks * nkt]: the block's tile number, or -1
+    int32_t* itv_tiles;  // [nblocks * nkt]: block x's tiles at x * nkt ..
+    int32_t* itv_ntiles; // [nblocks]
     int32_t* blk_res;    // [nblocks]
-    void* block_itv;     // lohi, tmap, block_tile_off, tile_info, blk_res
+    void* block_itv;     // lohi, tmap, itv_tiles, itv_ntiles, blk_res, block statistics
     ItvCounters* cnt_host;  // mapped host memory the build writes its totals to
     ItvCounters* cnt_dev;   // the same memory as the device addresses it
+    unsigned* done_dev;     // the slot's block counter
     cudaEvent_t built;      // recorded after the build
     bool counters_valid;    // cnt_host has been read into the fields above
     bool plan_written;      // the explicit plan arrays exist
@@ -143,6 +146,7 @@ cudaError_t pool_alloc(T** ptr, int64_t elems, cudaMemPool_t pool, cudaStream_t 
 struct HostSlot {
     ItvCounters* host;
     ItvCounters* dev;
+    unsigned* done;  // device counter of the build's finished blocks (left at 0)
     cudaEvent_t ev;
 };
 std::mutex g_slot_mu;
@@ -170,10 +174,14 @@ cudaError_t get_slot(int dev, HostSlot* out) {
         if (e != cudaSuccess) return e;
         void* d = nullptr;
         if ((e = cudaHostGetDevicePointer(&d, h, 0)) != cudaSuccess) return e;
+        unsigned* dn = nullptr;
+        if ((e = cudaMalloc(&dn, sizeof(unsigned) * kSlotChunk)) != cudaSuccess) return e;
+        if ((e = cudaMemset(dn, 0, sizeof(unsigned) * kSlotChunk)) != cudaSuccess) return e;
         for (int x = 0; x < kSlotChunk; ++x) {
             HostSlot sl;
             sl.host = static_cast<ItvCounters*>(h) + x;
             sl.dev = static_cast<ItvCounters*>(d) + x;
+            sl.done = dn + x;
             if ((e = cudaEventCreateWithFlags(&sl.ev, cudaEventDisableTiming)) != cudaSuccess) return e;
             fr.push_back(sl);
         }
@@ -422,8 +430,8 @@ int create_implicit(const spattn_mask_spec& sp, cudaStream_t s, int dev, cudaMem
         if (r) return r;
     }
     Carve c;
-    const int k_lh = c.add(rows * 8), k_tm = c.add(nblocks * nkt * 4), k_bs = c.add(nblocks * 8),
-              k_bto = c.add((nblocks + 1) * 4), k_ti = c.add(nblocks * nkt * 4), k_br = c.add(nblocks * 4);
+    const int k_lh = c.add(rows * 8), k_tm = c.add(nblocks * nkt * 4), k_ti = c.add(nblocks * nkt * 4),
+              k_nt = c.add(nblocks * 4), k_br = c.add(nblocks * 4), k_bs = c.add(nblocks * sizeof(ItvBlockStat));
     void* blk = nullptr;
     CUDA_TRY(cudaMallocFromPoolAsync(&blk, c.total, pool, s), "mask allocation");
     HostSlot sl;
@@ -441,9 +449,9 @@ int create_implicit(const spattn_mask_spec& sp, cudaStream_t s, int dev, cudaMem
     is.nqb = nqb;
     is.nkt = nkt;
     is.err_flags = ef;
-    e = itv_build(is, c.at<int2>(blk, k_lh), c.at<int32_t>(blk, k_tm), c.at<int2>(blk, k_bs),
-                  c.at<int32_t>(blk, k_bto), c.at<int32_t>(blk, k_ti), c.at<int32_t>(blk, k_br), min_nnz,
-                  sl.dev, s);
+    e = itv_build(is, c.at<int2>(blk, k_lh), c.at<int32_t>(blk, k_tm), c.at<int32_t>(blk, k_ti),
+                  c.at<int32_t>(blk, k_nt), c.at<int32_t>(blk, k_br), c.at<ItvBlockStat>(blk, k_bs), min_nnz,
+                  sl.done, sl.dev, s);
     if (e == cudaSuccess) e = cudaEventRecord(sl.ev, s);
     if (e != cudaSuccess) {
         cudaFreeAsync(blk, s);
@@ -464,12 +472,13 @@ int create_implicit(const spattn_mask_spec& sp, cudaStream_t s, int dev, cudaMem
     m->nkt = nkt;
     m->lohi = c.at<int2>(blk, k_lh);
     m->tmap = c.at<int32_t>(blk, k_tm);
-    m->block_tile_off = c.at<int32_t>(blk, k_bto);
-    m->tile_info = c.at<int32_t>(blk, k_ti);
+    m->itv_tiles = c.at<int32_t>(blk, k_ti);
+    m->itv_ntiles = c.at<int32_t>(blk, k_nt);
     m->blk_res = c.at<int32_t>(blk, k_br);
     m->block_itv = blk;
     m->cnt_host = sl.host;
     m->cnt_dev = sl.dev;
+    m->done_dev = sl.done;
     m->built = sl.ev;
     m->has_plan = min_nnz > 0;
     m->host_no_residual = interval_all_in_tiles(sp.kind, sp.n, sp.window, min_nnz);
@@ -537,12 +546,15 @@ int write_plan(spattn_mask m) {
     cudaMemPool_t pool;
     CUDA_TRY(device_state(m->device, &pool, nullptr), "memory pool");
     cudaStream_t s = m->stream;
+    const int64_t nblocks = (int64_t)m->num_masks * m->nqb;
     Carve cp;
-    const int k_tb = cp.add(m->n_tiles * kTileM * 16), k_rrp = cp.add((rows + 1) * 4),
+    const int k_bto = cp.add((nblocks + 1) * 4), k_ti = cp.add(m->n_tiles * 4),
+              k_tb = cp.add(m->n_tiles * kTileM * 16), k_rrp = cp.add((rows + 1) * 4),
               k_rci = cp.add(m->res_nnz * 4), k_rl = cp.add(rows * 4);
     Carve ct;
+    const int64_t scan_rows = rows > nblocks ? rows : nblocks;
     const int k_pc = ct.add(sizeof(PlanCounters)), k_rc = ct.add(rows * 4),
-              k_st = ct.add(scan_tmp_elems(rows) * 8);
+              k_st = ct.add(scan_tmp_elems(scan_rows) * 8);
     void *a = nullptr, *t = nullptr;
     PlanCounters hpc;
     cudaError_t e = cudaMallocFromPoolAsync(&a, cp.total, pool, s);
@@ -552,8 +564,8 @@ int write_plan(spattn_mask m) {
         PlanBuffers pb;
         memset(&pb, 0, sizeof pb);
         pb.cnt_map = m->tmap;
-        pb.block_tile_off = m->block_tile_off;
-        pb.tile_info = m->tile_info;
+        pb.block_tile_off = cp.at<int32_t>(a, k_bto);
+        pb.tile_info = cp.at<int32_t>(a, k_ti);
         pb.tile_cap = m->n_tiles;
         pb.tile_bits = cp.at<uint32_t>(a, k_tb);
         pb.res_row_ptr = cp.at<int32_t>(a, k_rrp);
@@ -561,7 +573,8 @@ int write_plan(spattn_mask m) {
         pb.res_long = cp.at<int32_t>(a, k_rl);
         pb.res_cnt = ct.at<int32_t>(t, k_rc);
         pb.scan_tmp = ct.at<int64_t>(t, k_st);
-        e = itv_write_plan(m->lohi, m->n, m->num_masks, pb, ct.at<PlanCounters>(t, k_pc), s);
+        e = itv_write_plan(m->lohi, m->n, m->num_masks, m->itv_tiles, m->itv_ntiles, pb,
+                           ct.at<PlanCounters>(t, k_pc), s);
     }
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(&hpc, ct.at<PlanCounters>(t, k_pc), sizeof hpc, cudaMemcpyDeviceToHost, s);
@@ -572,6 +585,8 @@ int write_plan(spattn_mask m) {
         return cuda_fail(e, "writing the mask's tile plan");
     }
     m->block_plan = a;
+    m->block_tile_off = cp.at<int32_t>(a, k_bto);
+    m->tile_info = cp.at<int32_t>(a, k_ti);
     m->tile_bits = cp.at<uint32_t>(a, k_tb);
     m->res_row_ptr = cp.at<int32_t>(a, k_rrp);
     m->res_col_idx = cp.at<int32_t>(a, k_rci);
@@ -602,6 +617,9 @@ int launch_tc(const FwdParams& p, int d, spattn_mask m, int dev, const int32_t* 
     if (m->implicit) {
         tp.itv_lohi = m->lohi;
         tp.blk_res = blk_res;
+        tp.tile_info = m->itv_tiles;
+        tp.block_ntiles = m->itv_ntiles;
+        tp.tile_stride = m->nkt;
     } else {
         tp.tile_bits = m->tile_bits;
         tp.res_row_ptr = m->res_row_ptr;
@@ -658,7 +676,7 @@ int fwd_interval(FwdParams& p, int dtype, int d, spattn_mask m, cudaStream_t s, 
         p.ws_ml = ws;
         p.ws_acc = ws + rows_all * 2;
         p.tmap = m->tmap;
-        p.qb_tile_off = m->block_tile_off;
+        p.qb_ntiles = m->itv_ntiles;
         p.blk_res = m->blk_res;
         const cudaError_t e = launch_fwd_itv(p, dtype, d, s);
         if (e != cudaSuccess) {
@@ -946,6 +964,7 @@ int spattn_destroy_mask(spattn_mask m) {
         HostSlot sl;
         sl.host = m->cnt_host;
         sl.dev = m->cnt_dev;
+        sl.done = m->done_dev;
         sl.ev = m->built;
         put_slot(m->device, sl);
     }

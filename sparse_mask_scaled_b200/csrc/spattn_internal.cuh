@@ -71,6 +71,7 @@ struct FwdParams {
     const int2* itv_lohi;
     const int32_t* tmap;
     const int32_t* blk_res;
+    const int32_t* qb_ntiles;  // tensor-core tiles per query block
     int nkt;
     int itv_slices;  // 1, 2, 4, 8 or 16 thread blocks per 128-row query block
 };
@@ -84,6 +85,10 @@ struct TcParams {
     int B, H, n, num_masks, nqb;
     const int32_t* block_tile_off;  // [num_masks * nqb + 1]
     const int32_t* tile_info;       // key tile | kTileDenseBit
+    // Instead of block_tile_off: block x's tiles are tile_info[x * tile_stride ..
+    // x * tile_stride + block_ntiles[x] - 1] (interval masks).
+    const int32_t* block_ntiles;
+    int tile_stride;
     const uint32_t* tile_bits;      // [tiles][128 rows][4 words]
     const int32_t* res_row_ptr;     // residual CSR (a row with entries has a partial)
     // Interval masks: masks come from the row runs instead of tile_bits, and the
@@ -147,7 +152,7 @@ struct ItvSpec {
     int nqb, nkt;
     unsigned* err_flags;  // nullable: negative half-widths also raise kErrBadColumn here
 };
-// Results of the build, written by one thread at the end of the select kernel.
+// Results of the build, written by the last thread block of the build kernel.
 struct ItvCounters {
     int64_t nnz;
     int64_t n_tiles;
@@ -157,24 +162,34 @@ struct ItvCounters {
     unsigned err;         // kBuildNegativeWidth
     int32_t pad;
 };
-constexpr int kItvMaxKeyTiles = 8192;   // per-block tile counts live in shared memory
-constexpr int64_t kItvMaxBlocks = 1 << 16;  // the select kernel is one thread block
-// Rows, per-tile counts and selection: two launches, no host synchronisation.
-// cnt: int32 [nblocks * nkt] (becomes the tile map: tile id or -1); bstat: int2
-// [nblocks] scratch; tile_info: int32 [nblocks * nkt]; min_nnz <= 0: select none.
-cudaError_t itv_build(const ItvSpec& s, int2* lohi, int32_t* cnt, int2* bstat, int32_t* block_tile_off,
-                      int32_t* tile_info, int32_t* blk_res, int min_nnz, ItvCounters* counters,
-                      cudaStream_t stream);
+// Per query block, for the totals.
+struct ItvBlockStat {
+    int64_t nnz, res;
+    int32_t n_long, n_bad, n_tiles, pad;
+};
+constexpr int kItvMaxKeyTiles = 8192;       // per-block tile counts live in shared memory
+constexpr int64_t kItvMaxBlocks = 1 << 16;  // query blocks of one build
+// One launch, no host synchronisation: per query block (one thread block each)
+// the rows' runs, the entry counts per key tile, the selected tiles (count >=
+// min_nnz; min_nnz <= 0 selects none) listed at tiles[blk * nkt ..] with their
+// number in ntiles[blk], the tile map tmap[blk * nkt + kt] (local tile number or
+// -1) and blk_res[blk] (entries outside the selected tiles); the last block to
+// finish writes the totals. done: a device counter that is 0 and is left 0.
+cudaError_t itv_build(const ItvSpec& s, int2* lohi, int32_t* tmap, int32_t* tiles, int32_t* ntiles,
+                      int32_t* blk_res, ItvBlockStat* bstat, int min_nnz, unsigned* done,
+                      ItvCounters* counters, cudaStream_t stream);
 // CSR of an interval mask: counts (scratch int32 [rows]) -> row_ptr [rows + 1]
 // -> col_idx [nnz]. scan_tmp: int64 [scan_tmp_elems(rows)], total/err: device scalars.
 cudaError_t itv_write_csr(const int2* lohi, int64_t rows, int32_t* counts, int32_t* row_ptr,
                           int32_t* col_idx, int64_t* scan_tmp, int64_t* total, unsigned* err,
                           cudaStream_t stream);
-// The explicit plan of an interval mask (tile_bits, residual CSR, mixed-row
-// count) from its runs and tile map, as build_plan writes it for CSR masks.
-// b.cnt_map is the tile map; counters->res_n_long, n_mixed must start at 0.
-cudaError_t itv_write_plan(const int2* lohi, int n, int num_masks, const PlanBuffers& b,
-                           PlanCounters* counters, cudaStream_t stream);
+// The explicit plan of an interval mask, as build_plan writes it for CSR masks:
+// b.block_tile_off and b.tile_info (compacted from tiles / ntiles), tile_bits,
+// the residual CSR and the mixed-row count. b.cnt_map is the tile map;
+// counters->res_n_long, n_mixed must start at 0.
+cudaError_t itv_write_plan(const int2* lohi, int n, int num_masks, const int32_t* tiles,
+                           const int32_t* ntiles, const PlanBuffers& b, PlanCounters* counters,
+                           cudaStream_t stream);
 
 // ---------------------------------------------------------------- launchers
 // All launchers enqueue on `stream` and return the cudaGetLastError() result.
