@@ -14,6 +14,9 @@ exactly. Additive mask/bias arrays are 4-D and broadcast to ``[B, H, n, n]``
 (size-1 dimensions get stride 0).
 
 Parity pins: every function here is checked in ``tests/test_oracle_pins.py``
+(the gradients in ``tests/test_oracle_bwd_pins.py``: central finite differences
+of the forward, closed forms for one nonzero per row, zero row sums of the score
+gradient)
 against facts fixed by the pages or by mathematics (dense softmax through
 scipy, one nonzero per row, row sums, the streaming form against the two-pass
 form, -inf mask entries against dropping them, shift invariance, uniform scores,
@@ -60,6 +63,9 @@ def _load():
         lib.oracle_row_weights.restype = I32
         lib.oracle_row_weights.argtypes = [I64, I64, I64, I64, P, P, P, I32, I64, P, P, D,
                                            P, I32, P, P, I32, P, I64, P]
+        lib.oracle_sdpa_bwd.restype = I32
+        lib.oracle_sdpa_bwd.argtypes = [I64, I64, I64, I64, P, P, P, I32, I64, P, P, D,
+                                        P, I32, P, P, I32, P, P, I32, P, P, P, P, P, I64]
         lib.oracle_mask_csr.restype = I64
         lib.oracle_mask_csr.argtypes = [I32, I64, I64, I64, I64, I64, I64, P, P, P, I32, P, P]
         _lib = lib
@@ -153,6 +159,39 @@ def row_weights(q, k, v, row_ptr, col_idx, num_masks, scale, flat_row,
                                _ptr(rp), _ptr(ci), float(scale), _ptr(ma), mt, _ptr(ms),
                                _ptr(ba), bt, _ptr(bs), int(flat_row), _ptr(w))
     return w[: int(rp[r + 1] - rp[r])]
+
+
+def masked_sdpa_bwd(q, k, v, row_ptr, col_idx, num_masks, scale, dout, add_mask=None, bias=None,
+                    want_dbias: bool = False):
+    """Gradients (dq, dk, dv [B, H, n, d] fp64, and dbias with the bias's shape or
+    None) of sum(dout * out) for the attention of ``masked_sdpa``."""
+    B, H, n, d = q.shape
+    qa, t = _elem(q)
+    ka, tk = _elem(k)
+    va, tv = _elem(v)
+    assert t == tk == tv
+    da, dt = _elem(dout)
+    assert da.shape == q.shape
+    rp = np.ascontiguousarray(row_ptr, dtype=np.int64)
+    ci = np.ascontiguousarray(col_idx, dtype=np.int32)
+    ma, mt, ms = _addend(add_mask, B, H, n)
+    ba, bt, bs = _addend(bias, B, H, n)
+    dq = np.zeros((B, H, n, d), np.float64)
+    dk = np.zeros_like(dq)
+    dv = np.zeros_like(dq)
+    dbias, dbs, nb = None, None, 0
+    if want_dbias:
+        assert bias is not None
+        dbias = np.zeros(bias.shape, np.float64)
+        dbs = np.array([0 if dbias.shape[x] == 1 else dbias.strides[x] // 8 for x in range(4)], np.int64)
+        nb = dbias.size
+    rc = _load().oracle_sdpa_bwd(B, H, n, d, _ptr(qa), _ptr(ka), _ptr(va), t, num_masks, _ptr(rp),
+                                 _ptr(ci), float(scale), _ptr(ma), mt, _ptr(ms), _ptr(ba), bt,
+                                 _ptr(bs), _ptr(da), dt, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dbias),
+                                 _ptr(dbs), nb)
+    if rc != 0:
+        raise ValueError("oracle_sdpa_bwd: bad argument")
+    return dq, dk, dv, dbias
 
 
 def mask_csr(kind: str, n: int, num_masks: int = 1, *, window: int = 0, block: int = 0,

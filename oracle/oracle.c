@@ -261,6 +261,83 @@ int oracle_row_weights(int64_t B, int64_t H, int64_t n, int64_t d, const void* q
 }
 
 /*
+ * Gradients of masked attention: the chain rule applied to the plain definition
+ * above (row_two_pass), for an upstream gradient dout = dL/dout. For each
+ * (b, h, i) with weights w_ij = softmax over the row's nonzeros of s_ij and
+ * out_i = sum_j w_ij v_j:
+ *   dv_j  += w_ij dout_i
+ *   dw_ij  = <dout_i, v_j>
+ *   ds_ij  = w_ij (dw_ij - sum_k w_ik dw_ik)         (Jacobian of the softmax)
+ *   dq_i  += scale ds_ij k_j ;  dk_j += scale ds_ij q_i
+ *   dbias[b, h, i, j] += ds_ij, summed over the bias's broadcast dimensions
+ *                        (dbias_stride: element strides of dbias, 0 = broadcast)
+ * A degenerate row (weights all 0) contributes nothing. dq, dk, dv: [B, H, n, d]
+ * fp64, overwritten; dbias (optional) is overwritten. Sequential (the column sums
+ * and the broadcast sums would race). Returns 0, or -1 for a bad argument.
+ */
+int oracle_sdpa_bwd(int64_t B, int64_t H, int64_t n, int64_t d, const void* q, const void* k,
+                    const void* v, int qkv_type, int64_t num_masks, const int64_t* row_ptr,
+                    const int32_t* col_idx, double scale, const void* mask, int mask_type,
+                    const int64_t* mask_stride, const void* bias, int bias_type,
+                    const int64_t* bias_stride, const void* dout, int dout_type, double* dq,
+                    double* dk, double* dv, double* dbias, const int64_t* dbias_stride,
+                    int64_t dbias_elems) {
+    if (B < 0 || H < 0 || n < 0 || d <= 0 || (num_masks != 1 && num_masks != B)) return -1;
+    orc_problem P;
+    P.B = B; P.H = H; P.n = n; P.d = d;
+    P.q = q; P.k = k; P.v = v; P.qkv_type = qkv_type;
+    P.num_masks = num_masks; P.row_ptr = row_ptr; P.col_idx = col_idx; P.scale = scale;
+    fill_addend(&P.mask, mask, mask_type, mask_stride);
+    fill_addend(&P.bias, bias, bias_type, bias_stride);
+    for (int64_t p = 0; p < row_ptr[num_masks * n]; ++p)
+        if (col_idx[p] < 0 || col_idx[p] >= n) return -1;
+    const int64_t total = B * H * n * d;
+    for (int64_t x = 0; x < total; ++x) dq[x] = dk[x] = dv[x] = 0.0;
+    if (dbias)
+        for (int64_t x = 0; x < dbias_elems; ++x) dbias[x] = 0.0;
+    const int64_t mx = max_row_len(&P) + 1;
+    double* s = (double*)malloc(sizeof(double) * (size_t)mx);
+    double* w = (double*)malloc(sizeof(double) * (size_t)mx);
+    double* dw = (double*)malloc(sizeof(double) * (size_t)mx);
+    double* out = (double*)malloc(sizeof(double) * (size_t)d);
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t h = 0; h < H; ++h)
+            for (int64_t i = 0; i < n; ++i) {
+                const int64_t base = (b * H + h) * n;
+                double lse;
+                row_two_pass(&P, b, h, i, s, out, &lse, w);
+                int64_t p0, p1;
+                mask_row_range(&P, b, i, &p0, &p1);
+                double sum_wdw = 0.0;
+                for (int64_t t = 0; t < p1 - p0; ++t) {
+                    const int64_t j = col_idx[p0 + t];
+                    double acc = 0.0;
+                    for (int64_t e = 0; e < d; ++e)
+                        acc += read_elem(dout, dout_type, (base + i) * d + e) * v_at(&P, b, h, j, e);
+                    dw[t] = acc;
+                    sum_wdw += w[t] * acc;
+                }
+                for (int64_t t = 0; t < p1 - p0; ++t) {
+                    const int64_t j = col_idx[p0 + t];
+                    const double ds = w[t] * (dw[t] - sum_wdw);
+                    for (int64_t e = 0; e < d; ++e) {
+                        dv[(base + j) * d + e] += w[t] * read_elem(dout, dout_type, (base + i) * d + e);
+                        dq[(base + i) * d + e] += scale * ds * read_elem(k, qkv_type, (base + j) * d + e);
+                        dk[(base + j) * d + e] += scale * ds * read_elem(q, qkv_type, (base + i) * d + e);
+                    }
+                    if (dbias)
+                        dbias[b * dbias_stride[0] + h * dbias_stride[1] + i * dbias_stride[2] +
+                              j * dbias_stride[3]] += ds;
+                }
+            }
+    free(s);
+    free(w);
+    free(dw);
+    free(out);
+    return 0;
+}
+
+/*
  * Mask patterns, by brute force over every (i, j) of the n x n grid.
  *
  * Patterns ("Sparse Attention" notes page, list of common patterns; the variable
