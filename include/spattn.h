@@ -231,6 +231,33 @@ int spattn_fwd_mask(const spattn_tensor* q, const spattn_tensor* k, const spattn
                     spattn_mask mask, const spattn_tensor* add_mask, const spattn_tensor* bias,
                     float scale, const spattn_tensor* out, float* lse, void* stream);
 
+/* Backward pass over a built mask: the gradients of L = sum(dout * out) with
+ * respect to q, k, v and (optionally) the bias, given the forward's out and lse
+ * (the chain rule of the operation above; the pages discuss bias gradients in
+ * "support attentions in AlphaFold2", flash-attention PR 57, the backward
+ * discussion). With P_ij = exp(s_ij - lse_i) and D_i = <dout_i, out_i>:
+ *   dS_ij = P_ij (<dout_i, v_j> - D_i)
+ *   dq_i = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,
+ *   dv_j = sum_i P_ij dout_i,      dbias[b,h,i,j] = dS_ij summed over the bias's
+ *                                  broadcast dimensions.
+ *   q, k, v, add_mask, bias, scale  as given to the forward.
+ *   out, lse  the forward's outputs (lse required).
+ *   dout      [B, H, n, d], q's dtype.
+ *   dq, dk, dv  [B, H, n, d], q's dtype, written (not accumulated).
+ *   dbias     optional (NULL): f32, contiguous, the bias's shape; cleared and then
+ *             accumulated with atomics (the order of the additions varies).
+ * Every entry runs on CUDA cores: a row pass (one warp per query row: dq and
+ * D_i) and a column pass (one warp per key over the transposed mask: dk, dv).
+ * The first call over a mask writes its CSR (interval masks) and its transpose,
+ * kept until the mask is destroyed, on the mask's stream, and synchronises that
+ * stream when it differs from `stream`. Uses a workspace of B*H*n floats from
+ * the library's pool. Errors as spattn_fwd_mask; UNSUPPORTED for n > 1,572,864. */
+int spattn_bwd_mask(const spattn_tensor* q, const spattn_tensor* k, const spattn_tensor* v,
+                    spattn_mask mask, const spattn_tensor* add_mask, const spattn_tensor* bias,
+                    float scale, const spattn_tensor* out, const float* lse, const spattn_tensor* dout,
+                    const spattn_tensor* dq, const spattn_tensor* dk, const spattn_tensor* dv,
+                    const spattn_tensor* dbias, void* stream);
+
 /* The same operation as spattn_fwd, but the call allocates no device memory.
  * For callers that cannot call cudaMalloc or take memory from a pool at run
  * time: for example a host program or plug-in whose memory manager owns the

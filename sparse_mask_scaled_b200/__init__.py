@@ -91,6 +91,8 @@ SIGNATURES = {
                                           _TP, ctypes.c_float, _TP, _P, _P]),
     "spattn_last_error": (ctypes.c_char_p, []),
     "spattn_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "spattn_bwd_mask": (ctypes.c_int, [_TP, _TP, _TP, _P, _TP, _TP, ctypes.c_float, _TP, _P, _TP, _TP,
+                                       _TP, _TP, _TP, _P]),
     "spattn_version": (ctypes.c_int, []),
     "spattn_launch_count": (ctypes.c_uint64, []),
 }
@@ -344,6 +346,31 @@ def spattn_device_error(stream=None) -> int:
 
 def spattn_last_error() -> str:
     return LIB.spattn_last_error().decode()
+
+
+def spattn_bwd_mask(q, k, v, mask: "Mask", out, lse, dout, add_mask=None, bias=None,
+                    scale: Optional[float] = None, want_dbias: bool = False, dq=None, dk=None, dv=None,
+                    dbias=None, stream=None):
+    """Gradients of sum(dout * out) for the forward over ``mask``: returns
+    (dq, dk, dv, dbias or None); dbias is float32 with the bias's shape."""
+    import torch
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
+    dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
+    dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
+    dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv
+    if want_dbias and dbias is None:
+        dbias = torch.empty(bias.shape, dtype=torch.float32, device=bias.device)
+    ds = [tensor_desc(x) for x in (q, k, v, out, dout, dq, dk, dv)]
+    dm = tensor_desc(add_mask) if add_mask is not None else None
+    db = tensor_desc(bias) if bias is not None else None
+    ddb = tensor_desc(dbias) if dbias is not None else None
+    _check(LIB.spattn_bwd_mask(ctypes.byref(ds[0]), ctypes.byref(ds[1]), ctypes.byref(ds[2]), mask.handle,
+                               ctypes.byref(dm) if dm is not None else None,
+                               ctypes.byref(db) if db is not None else None, float(scale),
+                               ctypes.byref(ds[3]), _ptr(lse), ctypes.byref(ds[4]), ctypes.byref(ds[5]),
+                               ctypes.byref(ds[6]), ctypes.byref(ds[7]),
+                               ctypes.byref(ddb) if ddb is not None else None, _stream(stream)))
+    return dq, dk, dv, dbias
 
 
 def spattn_version() -> int:

@@ -461,6 +461,211 @@ __global__ void __launch_bounds__(256, 2) k_fwd_itv(const FwdParams P) {
     for (int i0 = r0; i0 < r1; i0 += 8) itv_rows8<T, D>(P, b, h, mk, i0, tm, partial);
 }
 
+// ------------------------------------------------------------------ backward
+// Gradients of L = sum(dout * out) (the chain rule of the forward's definition):
+// with P_ij = exp(s_ij - lse_i) and D_i = <dout_i, out_i> = sum_j P_ij <dout_i, v_j>,
+//   dS_ij = P_ij (<dout_i, v_j> - D_i),  dq_i = scale sum_j dS_ij k_j,
+//   dk_j = scale sum_i dS_ij q_i,  dv_j = sum_i P_ij dout_i,  dbias_ij += dS_ij.
+// Scores are recomputed in the base-2 domain as in the forward.
+
+template <typename T, int D>
+__device__ __forceinline__ void load_slice(const T* base, int c, float (&f)[Cfg<T, D>::VEC]) {
+    Elem<T>::unpack(ldg16(base + c * Cfg<T, D>::VEC), f);
+}
+
+// Dot product of a lane's VEC slices, summed over the LPR lanes of its group.
+template <typename T, int D>
+__device__ __forceinline__ float group_dot(const float* a, const float* b) {
+    using C = Cfg<T, D>;
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < C::VEC; ++e) acc = fmaf(a[e], b[e], acc);
+#pragma unroll
+    for (int off = 1; off < C::LPR; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    return acc;
+}
+
+template <typename T, int D>
+__device__ __forceinline__ void store_slice(void* base, int64_t off, const float (&f)[Cfg<T, D>::VEC]) {
+    *reinterpret_cast<uint4*>(reinterpret_cast<T*>(base) + off) = Elem<T>::pack(f);
+}
+
+// Sums a per-group VEC accumulator over the warp's groups (every lane ends with the sum).
+template <int VEC, int LPR>
+__device__ __forceinline__ void sum_groups(float (&acc)[VEC]) {
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1) {
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+    }
+}
+
+// Row pass: one warp per query row i of (b, h): dq_i and D_i (and dbias).
+template <typename T, int D>
+__global__ void __launch_bounds__(256) k_bwd_rows(const BwdParams P) {
+    using C = Cfg<T, D>;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane / C::LPR, c = lane % C::LPR;
+    const int per_bh = (P.n + 7) >> 3;
+    const int bh = blockIdx.x / per_bh;
+    const int i = (blockIdx.x - bh * per_bh) * 8 + warp;
+    if (i >= P.n) return;
+    const int b = bh / P.H, h = bh - b * P.H;
+    const int64_t mrow = (int64_t)(P.num_masks == 1 ? 0 : b) * P.n + i;
+    const int64_t wrow = (int64_t)bh * P.n + i;
+    const T* kb = reinterpret_cast<const T*>(P.k) + b * P.k_sb + h * P.k_sh;
+    const T* vb = reinterpret_cast<const T*>(P.v) + b * P.v_sb + h * P.v_sh;
+    float qf[C::VEC], dof[C::VEC], of[C::VEC];
+    load_slice<T, D>(reinterpret_cast<const T*>(P.q) + b * P.q_sb + h * P.q_sh + i * P.q_sn, c, qf);
+    load_slice<T, D>(reinterpret_cast<const T*>(P.dout) + b * P.do_sb + h * P.do_sh + i * P.do_sn, c, dof);
+    load_slice<T, D>(reinterpret_cast<const T*>(P.out) + b * P.o_sb + h * P.o_sh + i * P.o_sn, c, of);
+    const float Di = group_dot<T, D>(dof, of);
+#pragma unroll
+    for (int e = 0; e < C::VEC; ++e) qf[e] *= P.qk_scale_log2;
+    const float lse2 = P.lse[wrow] * kLog2e;
+    const int64_t mask_base = b * P.mask.s0 + h * P.mask.s1 + i * P.mask.s2;
+    const int64_t bias_base = b * P.bias.s0 + h * P.bias.s1 + i * P.bias.s2;
+    const int64_t db_base = b * P.db_s0 + h * P.db_s1 + i * P.db_s2;
+    float dq[C::VEC];
+#pragma unroll
+    for (int e = 0; e < C::VEC; ++e) dq[e] = 0.f;
+    int64_t p0 = P.row_ptr[mrow], p1 = P.row_ptr[mrow + 1];
+    p0 = p0 < 0 ? 0 : (p0 > P.nnz ? P.nnz : p0);
+    p1 = p1 < p0 ? p0 : (p1 > P.nnz ? P.nnz : p1);
+    if (lse2 == -INFINITY) p1 = p0;  // a degenerate row has no weights
+    for (int64_t pb = p0; pb < p1; pb += C::STEP) {
+        int col = -1;
+        float extra = 0.f;
+        if (lane < C::STEP && pb + lane < p1) {
+            const int j = __ldg(P.col_idx + pb + lane);
+            if ((unsigned)j < (unsigned)P.n) {
+                col = j;
+                if (P.has_extra) {
+                    float ex = 0.f;
+                    if (P.mask.data) ex += load_addend(P.mask, mask_base + j * P.mask.s3);
+                    if (P.bias.data) ex += load_addend(P.bias, bias_base + j * P.bias.s3);
+                    extra = ex * kLog2e;
+                }
+            } else {
+                atomicOr(&g_error_flags, kErrBadColumn);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < C::U; ++u) {
+            const int j = __shfl_sync(0xffffffffu, col, u * C::G + g);
+            const float es = __shfl_sync(0xffffffffu, extra, u * C::G + g);
+            float kf[C::VEC], vf[C::VEC];
+            if (j >= 0) {
+                load_slice<T, D>(kb + (int64_t)j * P.k_sn, c, kf);
+                load_slice<T, D>(vb + (int64_t)j * P.v_sn, c, vf);
+            } else {
+#pragma unroll
+                for (int e = 0; e < C::VEC; ++e) kf[e] = vf[e] = 0.f;
+            }
+            const float sc = group_dot<T, D>(qf, kf);
+            const float dp = group_dot<T, D>(dof, vf);
+            const float pw = j >= 0 ? ex2(sc + es - lse2) : 0.f;
+            const float ds = pw * (dp - Di);
+#pragma unroll
+            for (int e = 0; e < C::VEC; ++e) dq[e] = fmaf(ds, kf[e], dq[e]);
+            if (P.dbias && j >= 0 && c == 0 && ds != 0.f)
+                atomicAdd(P.dbias + db_base + (int64_t)j * P.db_s3, ds);
+        }
+    }
+    sum_groups<C::VEC, C::LPR>(dq);
+    if (lane < C::LPR) {
+#pragma unroll
+        for (int e = 0; e < C::VEC; ++e) dq[e] *= P.scale;
+        store_slice<T, D>(P.dq, b * P.dq_sb + h * P.dq_sh + i * P.dq_sn + lane * C::VEC, dq);
+    }
+    if (lane == 0) P.D[wrow] = lse2 == -INFINITY ? 0.f : Di;
+}
+
+// Column pass: one warp per key j of (b, h), over the rows i with j in S_i.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) k_bwd_cols(const BwdParams P) {
+    using C = Cfg<T, D>;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane / C::LPR, c = lane % C::LPR;
+    const int per_bh = (P.n + 7) >> 3;
+    const int bh = blockIdx.x / per_bh;
+    const int j = (blockIdx.x - bh * per_bh) * 8 + warp;
+    if (j >= P.n) return;
+    const int b = bh / P.H, h = bh - b * P.H;
+    const int64_t mcol = (int64_t)(P.num_masks == 1 ? 0 : b) * P.n + j;
+    const T* qb = reinterpret_cast<const T*>(P.q) + b * P.q_sb + h * P.q_sh;
+    const T* dob = reinterpret_cast<const T*>(P.dout) + b * P.do_sb + h * P.do_sh;
+    float kf[C::VEC], vf[C::VEC];
+    load_slice<T, D>(reinterpret_cast<const T*>(P.k) + b * P.k_sb + h * P.k_sh + j * P.k_sn, c, kf);
+    load_slice<T, D>(reinterpret_cast<const T*>(P.v) + b * P.v_sb + h * P.v_sh + j * P.v_sn, c, vf);
+#pragma unroll
+    for (int e = 0; e < C::VEC; ++e) kf[e] *= P.qk_scale_log2;
+    float dk[C::VEC], dv[C::VEC];
+#pragma unroll
+    for (int e = 0; e < C::VEC; ++e) dk[e] = dv[e] = 0.f;
+    const int64_t p0 = P.t_row_ptr[mcol], p1 = P.t_row_ptr[mcol + 1];
+    for (int64_t pb = p0; pb < p1; pb += C::STEP) {
+        int row = -1;
+        float extra = 0.f, lse2 = -INFINITY, Di = 0.f;
+        if (lane < C::STEP && pb + lane < p1) {
+            const int i = __ldg(P.t_col_idx + pb + lane);
+            row = i;
+            const int64_t wrow = (int64_t)bh * P.n + i;
+            lse2 = P.lse[wrow] * kLog2e;
+            Di = P.D[wrow];
+            if (P.has_extra) {
+                float ex = 0.f;
+                if (P.mask.data) ex += load_addend(P.mask, b * P.mask.s0 + h * P.mask.s1 + i * P.mask.s2 + j * P.mask.s3);
+                if (P.bias.data) ex += load_addend(P.bias, b * P.bias.s0 + h * P.bias.s1 + i * P.bias.s2 + j * P.bias.s3);
+                extra = ex * kLog2e;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < C::U; ++u) {
+            const int i = __shfl_sync(0xffffffffu, row, u * C::G + g);
+            const float es = __shfl_sync(0xffffffffu, extra, u * C::G + g);
+            const float ls = __shfl_sync(0xffffffffu, lse2, u * C::G + g);
+            const float di = __shfl_sync(0xffffffffu, Di, u * C::G + g);
+            float qf[C::VEC], dof[C::VEC];
+            if (i >= 0) {
+                load_slice<T, D>(qb + (int64_t)i * P.q_sn, c, qf);
+                load_slice<T, D>(dob + (int64_t)i * P.do_sn, c, dof);
+            } else {
+#pragma unroll
+                for (int e = 0; e < C::VEC; ++e) qf[e] = dof[e] = 0.f;
+            }
+            const float sc = group_dot<T, D>(qf, kf);
+            const float dp = group_dot<T, D>(dof, vf);
+            const float pw = (i >= 0 && ls != -INFINITY) ? ex2(sc + es - ls) : 0.f;
+            const float ds = pw * (dp - di);
+#pragma unroll
+            for (int e = 0; e < C::VEC; ++e) {
+                dv[e] = fmaf(pw, dof[e], dv[e]);
+                dk[e] = fmaf(ds, qf[e], dk[e]);
+            }
+        }
+    }
+    sum_groups<C::VEC, C::LPR>(dk);
+    sum_groups<C::VEC, C::LPR>(dv);
+    if (lane < C::LPR) {
+#pragma unroll
+        for (int e = 0; e < C::VEC; ++e) dk[e] *= P.scale;
+        store_slice<T, D>(P.dk, b * P.dk_sb + h * P.dk_sh + j * P.dk_sn + lane * C::VEC, dk);
+        store_slice<T, D>(P.dv, b * P.dv_sb + h * P.dv_sh + j * P.dv_sn + lane * C::VEC, dv);
+    }
+}
+
+template <typename T, int D>
+cudaError_t launch_bwd_t(const BwdParams& p, cudaStream_t s) {
+    const int64_t blocks = (int64_t)p.B * p.H * ((p.n + 7) / 8);
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    k_bwd_rows<T, D><<<(unsigned)blocks, 256, 0, counted(s)>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    k_bwd_cols<T, D><<<(unsigned)blocks, 256, 0, counted(s)>>>(p);
+    return cudaGetLastError();
+}
+
 constexpr int kLongWarps = 8;
 
 template <typename T, int D>
@@ -593,6 +798,23 @@ cudaError_t launch_fwd_short_rows(const FwdParams& p, int dtype, int d, cudaStre
         case 32: return launch_short_t<float, 32>(p, s);
         case 64: return launch_short_t<float, 64>(p, s);
         case 128: return launch_short_t<float, 128>(p, s);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_bwd(const BwdParams& p, int dtype, int d, cudaStream_t s) {
+    if (dtype == 0) {
+        switch (d) {
+        case 32: return launch_bwd_t<__nv_bfloat16, 32>(p, s);
+        case 64: return launch_bwd_t<__nv_bfloat16, 64>(p, s);
+        case 128: return launch_bwd_t<__nv_bfloat16, 128>(p, s);
+        }
+    } else {
+        switch (d) {
+        case 32: return launch_bwd_t<float, 32>(p, s);
+        case 64: return launch_bwd_t<float, 64>(p, s);
+        case 128: return launch_bwd_t<float, 128>(p, s);
         }
     }
     return cudaErrorInvalidValue;

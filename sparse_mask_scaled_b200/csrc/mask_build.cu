@@ -16,6 +16,7 @@
 #include "spattn_internal.cuh"
 
 #include <limits.h>
+#include <string.h>
 
 namespace spattn {
 namespace {
@@ -562,6 +563,31 @@ unsigned grid_for(int64_t work, int per_block, int64_t cap = 1 << 16) {
     return (unsigned)g;
 }
 
+// Transpose helpers: per-column counts and the unsorted fill (one warp per row).
+__global__ void k_tcount(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx, int n,
+                         int64_t rows, int32_t* __restrict__ cnt) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t r = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+        const int64_t m = r / n;
+        for (int64_t p = row_ptr[r] + lane; p < row_ptr[r + 1]; p += 32) atomicAdd(&cnt[m * n + col_idx[p]], 1);
+    }
+}
+
+__global__ void k_tfill(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx, int n,
+                        int64_t rows, const int32_t* __restrict__ cand_row_ptr, int32_t* __restrict__ cursor,
+                        int32_t* __restrict__ cand_col) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t r = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+        const int64_t m = r / n, i = r - m * n;
+        for (int64_t p = row_ptr[r] + lane; p < row_ptr[r + 1]; p += 32) {
+            const int64_t t = m * n + col_idx[p];
+            cand_col[cand_row_ptr[t] + atomicAdd(&cursor[t], 1)] = (int32_t)i;
+        }
+    }
+}
+
 }  // namespace
 
 int64_t scan_tmp_elems(int64_t rows) { return rows + 1 + (rows + kScanTile - 1) / kScanTile + 1; }
@@ -680,6 +706,62 @@ cudaError_t build_phase2(const BuildSpec& s, const int32_t* row_ptr, const int32
         e = cudaGetLastError();
     }
     return e;
+}
+
+}  // namespace spattn
+
+namespace spattn {
+
+// Scratch layout (int32 words, each part 64-word aligned): cnt [rows], cursor
+// [rows], cand_row_ptr [rows + 1], cand_col [nnz], counts [rows], long_rows
+// [rows], coo_tmp [nnz + rows], info (BuildInfo), scan_tmp (int64, with the COO
+// queue of long rows).
+namespace {
+int64_t al64(int64_t w) { return (w + 63) & ~int64_t(63); }
+}  // namespace
+
+int64_t transpose_scratch_words(int64_t rows, int64_t nnz) {
+    const int64_t scan64 = scan_tmp_elems(rows) + (rows + 6) / 2 + 1;
+    return 2 * al64(rows) + al64(rows + 1) + al64(nnz) + 2 * al64(rows) + al64(nnz + rows) + 64 +
+           2 * scan64;
+}
+
+cudaError_t build_transpose(const int32_t* row_ptr, const int32_t* col_idx, int n, int num_masks,
+                            int64_t nnz, int32_t* t_row_ptr, int32_t* t_col_idx, int32_t* scratch,
+                            cudaStream_t stream) {
+    const int64_t rows = (int64_t)num_masks * n;
+    int32_t* cnt = scratch;
+    int32_t* cursor = cnt + al64(rows);
+    int32_t* cand_row_ptr = cursor + al64(rows);
+    int32_t* cand_col = cand_row_ptr + al64(rows + 1);
+    int32_t* counts = cand_col + al64(nnz);
+    int32_t* long_rows = counts + al64(rows);
+    int32_t* coo_tmp = long_rows + al64(rows);
+    BuildInfo* info = reinterpret_cast<BuildInfo*>(coo_tmp + al64(nnz + rows));
+    int64_t* scan_tmp = reinterpret_cast<int64_t*>(reinterpret_cast<int32_t*>(info) + 64);
+    cudaError_t e = cudaMemsetAsync(cnt, 0, sizeof(int32_t) * (size_t)(2 * al64(rows)), stream);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(info, 0, sizeof(BuildInfo), stream)) != cudaSuccess) return e;
+    k_tcount<<<grid_for(rows, 8), 256, 0, counted(stream)>>>(row_ptr, col_idx, n, rows, cnt);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = scan_counts(cnt, rows, cand_row_ptr, scan_tmp, &info->nnz, &info->err, stream);
+    if (e != cudaSuccess) return e;
+    k_tfill<<<grid_for(rows, 8), 256, 0, counted(stream)>>>(row_ptr, col_idx, n, rows, cand_row_ptr, cursor,
+                                                            cand_col);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // sort each transposed row: the COO builder's path (no repeats to merge)
+    BuildSpec bs;
+    memset(&bs, 0, sizeof bs);
+    bs.kind = SPATTN_MASK_COO;
+    bs.n = n;
+    bs.num_masks = num_masks;
+    bs.in_row_ptr = cand_row_ptr;
+    bs.in_col_idx = cand_col;
+    bs.in_nnz = nnz;
+    bool zeroed = false;
+    e = build_phase1(bs, t_row_ptr, counts, scan_tmp, coo_tmp, info, long_rows, nullptr, 0, &zeroed, stream);
+    if (e != cudaSuccess) return e;
+    return build_phase2(bs, t_row_ptr, coo_tmp, t_col_idx, nullptr, stream);
 }
 
 }  // namespace spattn

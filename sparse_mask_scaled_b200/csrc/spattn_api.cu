@@ -74,6 +74,10 @@ struct spattn_mask_s {
     bool counters_valid;    // cnt_host has been read into the fields above
     bool plan_written;      // the explicit plan arrays exist
     bool host_no_residual;  // known from the parameters: every entry lies in a selected tile
+    // transpose for the backward column pass (written on the first backward call)
+    int32_t* t_row_ptr;
+    int32_t* t_col_idx;
+    void* block_t;
 };
 
 namespace {
@@ -689,6 +693,38 @@ int fwd_interval(FwdParams& p, int dtype, int d, spattn_mask m, cudaStream_t s, 
     return r;
 }
 
+
+// The transposed mask (rows m*n + j listing the i with j in S_i), written on the
+// first backward call over this mask, on the mask's stream.
+int write_transpose(spattn_mask m) {
+    if (m->t_row_ptr) return SPATTN_OK;
+    int r = write_csr(m);
+    if (r) return r;
+    if (m->n > 1572864) return fail(SPATTN_ERR_UNSUPPORTED, "backward needs n <= 1572864");
+    const int64_t rows = (int64_t)m->n * m->num_masks;
+    cudaMemPool_t pool;
+    CUDA_TRY(device_state(m->device, &pool, nullptr), "memory pool");
+    cudaStream_t s = m->stream;
+    Carve c;
+    const int k_rp = c.add((rows + 1) * 4), k_ci = c.add((m->nnz > 0 ? m->nnz : 1) * 4);
+    void *blk = nullptr, *scratch = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync(&blk, c.total, pool, s);
+    if (e == cudaSuccess)
+        e = cudaMallocFromPoolAsync(&scratch, (size_t)transpose_scratch_words(rows, m->nnz) * 4, pool, s);
+    if (e == cudaSuccess)
+        e = build_transpose(m->row_ptr, m->col_idx, m->n, m->num_masks, m->nnz, c.at<int32_t>(blk, k_rp),
+                            c.at<int32_t>(blk, k_ci), static_cast<int32_t*>(scratch), s);
+    if (scratch) cudaFreeAsync(scratch, s);
+    if (e != cudaSuccess) {
+        if (blk) cudaFreeAsync(blk, s);
+        return cuda_fail(e, "transposing the mask");
+    }
+    m->block_t = blk;
+    m->t_row_ptr = c.at<int32_t>(blk, k_rp);
+    m->t_col_idx = c.at<int32_t>(blk, k_ci);
+    return SPATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -960,6 +996,7 @@ int spattn_destroy_mask(spattn_mask m) {
     if (m->block_col && (e2 = cudaFreeAsync(m->block_col, m->stream)) != cudaSuccess) e = e2;
     free_plan(m);
     if (m->block_itv && (e2 = cudaFreeAsync(m->block_itv, m->stream)) != cudaSuccess) e = e2;
+    if (m->block_t && (e2 = cudaFreeAsync(m->block_t, m->stream)) != cudaSuccess) e = e2;
     if (m->cnt_host) {
         HostSlot sl;
         sl.host = m->cnt_host;
@@ -1073,6 +1110,103 @@ int spattn_fwd_mask(const spattn_tensor* q, const spattn_tensor* k, const spattn
     r = launch_tc(p, d, mask, dev, nullptr, s);
     if (ws) cudaFreeAsync(ws, s);
     return r;
+}
+
+int spattn_bwd_mask(const spattn_tensor* q, const spattn_tensor* k, const spattn_tensor* v,
+                    spattn_mask mask, const spattn_tensor* add_mask, const spattn_tensor* bias,
+                    float scale, const spattn_tensor* out, const float* lse, const spattn_tensor* dout,
+                    const spattn_tensor* dq, const spattn_tensor* dk, const spattn_tensor* dv,
+                    const spattn_tensor* dbias, void* stream_v) {
+    g_msg[0] = 0;
+    FwdParams p;
+    int dtype, d;
+    int r = check_fwd(q, k, v, add_mask, bias, scale, out, nullptr, &p, &dtype, &d);
+    if (r) return r;
+    if (!mask) return fail(SPATTN_ERR_INVALID_ARG, "mask is NULL");
+    if (!lse) return fail(SPATTN_ERR_INVALID_ARG, "lse is NULL");
+    if (((uintptr_t)lse) % 4 != 0) return fail(SPATTN_ERR_INVALID_ARG, "lse not aligned");
+    const int64_t shape[4] = {q->shape[0], q->shape[1], q->shape[2], q->shape[3]};
+    if ((r = check_qkv(dout, "dout", shape, q->dtype))) return r;
+    if ((r = check_qkv(dq, "dq", shape, q->dtype))) return r;
+    if ((r = check_qkv(dk, "dk", shape, q->dtype))) return r;
+    if ((r = check_qkv(dv, "dv", shape, q->dtype))) return r;
+    if (dbias) {
+        if (!bias) return fail(SPATTN_ERR_INVALID_ARG, "dbias needs bias");
+        if (dbias->dtype != SPATTN_F32 || dbias->reserved != 0)
+            return fail(SPATTN_ERR_INVALID_ARG, "dbias must be f32");
+        if (!dbias->data) return fail(SPATTN_ERR_INVALID_ARG, "dbias.data is NULL");
+        int64_t acc = 1;
+        for (int x = 3; x >= 0; --x) {
+            if (dbias->shape[x] != bias->shape[x])
+                return fail(SPATTN_ERR_INVALID_ARG, "dbias shape differs from bias shape");
+            if (dbias->shape[x] > 1 && dbias->stride[x] != acc)
+                return fail(SPATTN_ERR_INVALID_ARG, "dbias must be contiguous");
+            acc *= dbias->shape[x];
+        }
+        if (((uintptr_t)dbias->data) % 4 != 0) return fail(SPATTN_ERR_INVALID_ARG, "dbias not aligned");
+    }
+    if (mask->n != p.n) return fail(SPATTN_ERR_INVALID_ARG, "mask n %d != q n %d", mask->n, p.n);
+    if (mask->num_masks != 1 && mask->num_masks != p.B)
+        return fail(SPATTN_ERR_INVALID_ARG, "mask num_masks must be 1 or B");
+    if ((int64_t)p.B * p.H * p.n == 0) return SPATTN_OK;
+    cudaStream_t s = (cudaStream_t)stream_v;
+    int dev;
+    CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
+    if (dev != mask->device) return fail(SPATTN_ERR_INVALID_ARG, "mask lives on another device");
+    cudaMemPool_t pool;
+    CUDA_TRY(device_state(dev, &pool, nullptr), "memory pool");
+    if ((r = write_transpose(mask))) return r;
+    // the transpose was written on the mask's stream; order this stream after it
+    if (mask->stream != s) CUDA_TRY(cudaStreamSynchronize(mask->stream), "mask stream");
+
+    BwdParams bp;
+    memset(&bp, 0, sizeof bp);
+    auto bs = [](const spattn_tensor* t, int x) { return t->shape[x] == 1 ? 0 : t->stride[x]; };
+    bp.q = q->data;
+    bp.k = k->data;
+    bp.v = v->data;
+    bp.out = out->data;
+    bp.dout = dout->data;
+    bp.dq = dq->data;
+    bp.dk = dk->data;
+    bp.dv = dv->data;
+    bp.lse = lse;
+    bp.q_sb = p.q_sb; bp.q_sh = p.q_sh; bp.q_sn = p.q_sn;
+    bp.k_sb = p.k_sb; bp.k_sh = p.k_sh; bp.k_sn = p.k_sn;
+    bp.v_sb = p.v_sb; bp.v_sh = p.v_sh; bp.v_sn = p.v_sn;
+    bp.o_sb = p.o_sb; bp.o_sh = p.o_sh; bp.o_sn = p.o_sn;
+    bp.do_sb = bs(dout, 0); bp.do_sh = bs(dout, 1); bp.do_sn = bs(dout, 2);
+    bp.dq_sb = bs(dq, 0); bp.dq_sh = bs(dq, 1); bp.dq_sn = bs(dq, 2);
+    bp.dk_sb = bs(dk, 0); bp.dk_sh = bs(dk, 1); bp.dk_sn = bs(dk, 2);
+    bp.dv_sb = bs(dv, 0); bp.dv_sh = bs(dv, 1); bp.dv_sn = bs(dv, 2);
+    bp.B = p.B;
+    bp.H = p.H;
+    bp.n = p.n;
+    bp.num_masks = mask->num_masks;
+    bp.row_ptr = mask->row_ptr;
+    bp.col_idx = mask->col_idx;
+    bp.nnz = mask->nnz;
+    bp.t_row_ptr = mask->t_row_ptr;
+    bp.t_col_idx = mask->t_col_idx;
+    bp.mask = p.mask;
+    bp.bias = p.bias;
+    bp.has_extra = p.has_extra;
+    bp.scale = scale;
+    bp.qk_scale_log2 = p.qk_scale_log2;
+    if (dbias) {
+        bp.dbias = static_cast<float*>(dbias->data);
+        bp.db_s0 = bs(dbias, 0); bp.db_s1 = bs(dbias, 1); bp.db_s2 = bs(dbias, 2); bp.db_s3 = bs(dbias, 3);
+        size_t elems = 1;
+        for (int x = 0; x < 4; ++x) elems *= (size_t)dbias->shape[x];
+        CUDA_TRY(cudaMemsetAsync(dbias->data, 0, elems * 4, s), "clearing dbias");
+    }
+    float* Dbuf = nullptr;
+    CUDA_TRY(pool_alloc(&Dbuf, (int64_t)p.B * p.H * p.n, pool, s), "backward workspace");
+    bp.D = Dbuf;
+    const cudaError_t e = launch_bwd(bp, dtype, d, s);
+    cudaFreeAsync(Dbuf, s);
+    if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");
+    return SPATTN_OK;
 }
 
 // ---- allocation-free forward: its scratch is this fixed array, part of the

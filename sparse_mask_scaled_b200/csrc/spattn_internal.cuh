@@ -76,6 +76,32 @@ struct FwdParams {
     int itv_slices;  // 1, 2, 4, 8 or 16 thread blocks per 128-row query block
 };
 
+// Backward pass (fwd_gather.cu): gradients of sum(dout * out) for the same
+// attention, recomputing each score from q, k and the saved lse. The row pass
+// (one warp per query row) writes dq and D_i = <dout_i, out_i>; the column pass
+// (one warp per key, over the transposed mask) writes dk and dv.
+struct BwdParams {
+    const void *q, *k, *v, *out, *dout;
+    void *dq, *dk, *dv;
+    const float* lse;  // natural log, [B*H*n]
+    float* D;          // [B*H*n], written by the row pass
+    float* dbias;      // nullable: f32, accumulated (atomics), element strides db_s*
+    int64_t db_s0, db_s1, db_s2, db_s3;
+    int64_t q_sb, q_sh, q_sn, k_sb, k_sh, k_sn, v_sb, v_sh, v_sn, o_sb, o_sh, o_sn;
+    int64_t do_sb, do_sh, do_sn, dq_sb, dq_sh, dq_sn, dk_sb, dk_sh, dk_sn, dv_sb, dv_sh, dv_sn;
+    int B, H, n, num_masks;
+    const int32_t* row_ptr;    // the mask
+    const int32_t* col_idx;
+    int64_t nnz;
+    const int32_t* t_row_ptr;  // its transpose: row m*n + j lists the i with j in S_i
+    const int32_t* t_col_idx;
+    AddendView mask, bias;
+    int has_extra;
+    float scale;
+    float qk_scale_log2;
+};
+cudaError_t launch_bwd(const BwdParams& p, int dtype, int d, cudaStream_t stream);
+
 // Tensor-core kernel (fwd_tc.cu).
 struct TcOperand {
     const void* data;  // bf16 [B, H, n, d], stride 1 over d
@@ -259,5 +285,13 @@ cudaError_t scan_counts(const int32_t* counts, int64_t rows, int32_t* out, int64
 // per-tile counts for the tile plan.
 cudaError_t build_phase2(const BuildSpec& s, const int32_t* row_ptr, const int32_t* coo_tmp,
                          int32_t* col_idx, int32_t* tile_cnt, cudaStream_t stream);
+
+// Transpose of a CSR mask set: t_row_ptr [rows + 1] / t_col_idx [nnz], row
+// m*n + j listing, ascending, the i with j in row m*n + i. Scratch sizes in
+// int32 words: transpose_scratch_words(rows, nnz). No host synchronisation.
+int64_t transpose_scratch_words(int64_t rows, int64_t nnz);
+cudaError_t build_transpose(const int32_t* row_ptr, const int32_t* col_idx, int n, int num_masks,
+                            int64_t nnz, int32_t* t_row_ptr, int32_t* t_col_idx, int32_t* scratch,
+                            cudaStream_t stream);
 
 }  // namespace spattn
