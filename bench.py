@@ -105,6 +105,11 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            # let nvidia-smi finish starting up (NVML initialisation) before the
+            # timed region, so that it does not stall the first timed step
+            t0 = time.perf_counter()
+            while not self.lines and time.perf_counter() - t0 < 3.0:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
         return self
@@ -461,6 +466,54 @@ def e2e_measure(args, g, torch, stream, flush, flops):
     return {"ms_per_step": sum(times) / len(times), "h2d": int(h2d), "d2h": int(d2h)}
 
 
+def backward_timing(args, torch, sp):
+    """The backward pass (spattn_bwd_mask) on the benchmark workload: the mask and
+    the forward's out / lse are prepared once, then each timed call computes dq,
+    dk, dv (and dbias when the workload has a bias) with L2 flushed before it.
+    FLOPs are counted as 2.5 x the forward's (10 * nnz * d: the score and
+    dout . v recomputed, and the dq, dk, dv products)."""
+    wl = workloads.make(args.config, seed=replica_seed(args.config, 0))
+    g = GpuWorkload(wl, torch, sp)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    dout = torch.randn(g.q.shape, generator=gen, device="cuda").to(g.q.dtype)
+    with g.create() as m:
+        nnz_total = m.nnz * (wl.B * wl.H if wl.mask.num_masks == 1 else wl.H)
+        out, lse = g.fwd(m)
+        dq, dk, dv = (torch.empty_like(g.q) for _ in range(3))
+        dbias = torch.empty(g.bias.shape, dtype=torch.float32, device="cuda") if g.bias is not None else None
+
+        def one():
+            sp.spattn_bwd_mask(g.q, g.k, g.v, m, out, lse, dout, add_mask=g.am, bias=g.bias, scale=wl.scale,
+                               dq=dq, dk=dk, dv=dv, dbias=dbias)
+        for _ in range(3):
+            one()
+        ts = []
+        for _ in range(10):
+            flush.zero_()
+            s = torch.cuda.Event(enable_timing=True)
+            e = torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            one()
+            e.record(stream)
+            e.synchronize()
+            ts.append(s.elapsed_time(e))
+    t = statistics.median(ts)
+    es = 2 if wl.dtype == workloads.BF16 else 4
+    rows = wl.B * wl.H * wl.n
+    # the method's bytes: per nonzero a K and a V row (row pass) and a Q and a dout
+    # row (column pass) plus the two indices and lse_i, D_i; per row q, dout, out,
+    # dq read/written once and k, v, dk, dv likewise, plus lse and D
+    alg = nnz_total * (4 * wl.d * es + 16) + rows * (8 * wl.d * es + 12)
+    hbm_peak, _, _ = measured_peaks()
+    return {"workload": wl.name, "ms": round(t, 4), "flop": 10.0 * nnz_total * wl.d,
+            "tflops": round(10.0 * nnz_total * wl.d / (t * 1e-3) / 1e12, 3),
+            "effective_gbs": round(alg / (t * 1e-3) / 1e9, 1),
+            "frac_hbm_effective": round(alg / (t * 1e-3) / 1e9 / hbm_peak, 4),
+            "path": "CUDA cores: row pass (dq) + column pass over the transposed mask (dk, dv)"}
+
+
 def other_workloads(torch, sp, skip):
     """Forward-only timings of the other workloads (device-resident inputs, L2 flushed)."""
     res = {}
@@ -568,6 +621,10 @@ def main():
     if rank == 0:
         if not args.no_extra and world == 1:
             result["other_workloads_fwd"] = other_workloads(torch, sp, args.config)
+            try:
+                result["backward"] = backward_timing(args, torch, sp)
+            except Exception as ex:  # keep the headline line
+                result["backward"] = {"error": str(ex)[:200]}
         if not args.no_cpu_baseline and world == 1:
             threads = os.cpu_count() or 1
             rate, cnt, nz, t = cpu_oracle_rate(wl, args.cpu_seconds, threads)

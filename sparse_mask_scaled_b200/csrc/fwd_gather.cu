@@ -500,17 +500,15 @@ __device__ __forceinline__ void sum_groups(float (&acc)[VEC]) {
     }
 }
 
-// Row pass: one warp per query row i of (b, h): dq_i and D_i (and dbias).
+// Row pass for query row i of (b, h), one warp: dq_i, D_i and the score
+// gradients -- added to dbias with atomics, or, with db_row, to that shared-memory
+// row of n floats (indexed by key).
 template <typename T, int D>
-__global__ void __launch_bounds__(256) k_bwd_rows(const BwdParams P) {
+__device__ __forceinline__ void bwd_row(const BwdParams& P, int b, int h, int i, float* db_row) {
     using C = Cfg<T, D>;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31;
     const int g = lane / C::LPR, c = lane % C::LPR;
-    const int per_bh = (P.n + 7) >> 3;
-    const int bh = blockIdx.x / per_bh;
-    const int i = (blockIdx.x - bh * per_bh) * 8 + warp;
-    if (i >= P.n) return;
-    const int b = bh / P.H, h = bh - b * P.H;
+    const int bh = b * P.H + h;
     const int64_t mrow = (int64_t)(P.num_masks == 1 ? 0 : b) * P.n + i;
     const int64_t wrow = (int64_t)bh * P.n + i;
     const T* kb = reinterpret_cast<const T*>(P.k) + b * P.k_sb + h * P.k_sh;
@@ -550,26 +548,41 @@ __global__ void __launch_bounds__(256) k_bwd_rows(const BwdParams P) {
                 atomicOr(&g_error_flags, kErrBadColumn);
             }
         }
+        constexpr int UB = 1;  // (more loads in flight cost registers, and occupancy, than they gain)
 #pragma unroll
-        for (int u = 0; u < C::U; ++u) {
-            const int j = __shfl_sync(0xffffffffu, col, u * C::G + g);
-            const float es = __shfl_sync(0xffffffffu, extra, u * C::G + g);
-            float kf[C::VEC], vf[C::VEC];
-            if (j >= 0) {
-                load_slice<T, D>(kb + (int64_t)j * P.k_sn, c, kf);
-                load_slice<T, D>(vb + (int64_t)j * P.v_sn, c, vf);
-            } else {
+        for (int u0 = 0; u0 < C::U; u0 += UB) {
+            int js[UB];
+            float ess[UB];
+            uint4 kr[UB], vr[UB];
 #pragma unroll
-                for (int e = 0; e < C::VEC; ++e) kf[e] = vf[e] = 0.f;
+            for (int t = 0; t < UB; ++t) {
+                js[t] = __shfl_sync(0xffffffffu, col, (u0 + t) * C::G + g);
+                ess[t] = __shfl_sync(0xffffffffu, extra, (u0 + t) * C::G + g);
+                kr[t] = vr[t] = make_uint4(0u, 0u, 0u, 0u);
+                if (js[t] >= 0) {
+                    kr[t] = ldg16(kb + (int64_t)js[t] * P.k_sn + c * C::VEC);
+                    vr[t] = ldg16(vb + (int64_t)js[t] * P.v_sn + c * C::VEC);
+                }
             }
-            const float sc = group_dot<T, D>(qf, kf);
-            const float dp = group_dot<T, D>(dof, vf);
-            const float pw = j >= 0 ? ex2(sc + es - lse2) : 0.f;
-            const float ds = pw * (dp - Di);
 #pragma unroll
-            for (int e = 0; e < C::VEC; ++e) dq[e] = fmaf(ds, kf[e], dq[e]);
-            if (P.dbias && j >= 0 && c == 0 && ds != 0.f)
-                atomicAdd(P.dbias + db_base + (int64_t)j * P.db_s3, ds);
+            for (int t = 0; t < UB; ++t) {
+                const int j = js[t];
+                float kf[C::VEC], vf[C::VEC];
+                Elem<T>::unpack(kr[t], kf);
+                Elem<T>::unpack(vr[t], vf);
+                const float sc = group_dot<T, D>(qf, kf);
+                const float dp = group_dot<T, D>(dof, vf);
+                const float pw = j >= 0 ? ex2(sc + ess[t] - lse2) : 0.f;
+                const float ds = pw * (dp - Di);
+#pragma unroll
+                for (int e = 0; e < C::VEC; ++e) dq[e] = fmaf(ds, kf[e], dq[e]);
+                if (P.dbias && j >= 0 && c == 0 && ds != 0.f) {
+                    if (db_row)
+                        db_row[j] += ds;  // one row per warp, one lane per key
+                    else
+                        atomicAdd(P.dbias + db_base + (int64_t)j * P.db_s3, ds);
+                }
+            }
         }
     }
     sum_groups<C::VEC, C::LPR>(dq);
@@ -581,9 +594,45 @@ __global__ void __launch_bounds__(256) k_bwd_rows(const BwdParams P) {
     if (lane == 0) P.D[wrow] = lse2 == -INFINITY ? 0.f : Di;
 }
 
+// Row pass: one warp per query row i of (b, h).
+template <typename T, int D>
+__global__ void __launch_bounds__(256) k_bwd_rows(const BwdParams P) {
+    const int warp = threadIdx.x >> 5;
+    const int per_bh = (P.n + 7) >> 3;
+    const int bh = blockIdx.x / per_bh;
+    const int i = (blockIdx.x - bh * per_bh) * 8 + warp;
+    if (i >= P.n) return;
+    bwd_row<T, D>(P, bh / P.H, bh - (bh / P.H) * P.H, i, nullptr);
+}
+
+// Row pass when the bias gradient is broadcast over the batch (a pair bias
+// shared by every b): one warp per (h, i) walks every b and adds the score
+// gradients up in a shared-memory row of n floats, then stores it -- one store
+// per element instead of B contending atomics. kDbRowMax keys at most.
+constexpr int kDbRowMax = 1536;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) k_bwd_rows_dbb(const BwdParams P) {
+    extern __shared__ float db_rows[];  // [8][n]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int per_h = (P.n + 7) >> 3;
+    const int h = blockIdx.x / per_h;
+    const int i = (blockIdx.x - h * per_h) * 8 + warp;
+    float* row = db_rows + warp * P.n;
+    for (int j = lane; j < P.n; j += 32) row[j] = 0.f;
+    __syncwarp();
+    if (i >= P.n) return;
+    for (int b = 0; b < P.B; ++b) {
+        bwd_row<T, D>(P, b, h, i, row);
+        __syncwarp();
+    }
+    float* dst = P.dbias + h * P.db_s1 + (int64_t)i * P.db_s2;
+    for (int j = lane; j < P.n; j += 32) dst[(int64_t)j * P.db_s3] = row[j];
+}
+
 // Column pass: one warp per key j of (b, h), over the rows i with j in S_i.
 template <typename T, int D>
-__global__ void __launch_bounds__(256) k_bwd_cols(const BwdParams P) {
+__global__ void __launch_bounds__(256, 3) k_bwd_cols(const BwdParams P) {
     using C = Cfg<T, D>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane / C::LPR, c = lane % C::LPR;
@@ -659,7 +708,20 @@ template <typename T, int D>
 cudaError_t launch_bwd_t(const BwdParams& p, cudaStream_t s) {
     const int64_t blocks = (int64_t)p.B * p.H * ((p.n + 7) / 8);
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    k_bwd_rows<T, D><<<(unsigned)blocks, 256, 0, counted(s)>>>(p);
+    // every (h, i) must own its dbias row for the batch-walking pass
+    const bool own_rows = (p.db_s1 != 0 || p.H == 1) && (p.db_s2 != 0 || p.n == 1);
+    if (p.dbias && p.db_s0 == 0 && p.B > 1 && own_rows && p.n <= kDbRowMax) {
+        const int64_t hb = (int64_t)p.H * ((p.n + 7) / 8);
+        const size_t smem = (size_t)8 * p.n * sizeof(float);
+        if (smem > 48 * 1024) {
+            cudaError_t a = cudaFuncSetAttribute(k_bwd_rows_dbb<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)smem);
+            if (a != cudaSuccess) return a;
+        }
+        k_bwd_rows_dbb<T, D><<<(unsigned)hb, 256, smem, counted(s)>>>(p);
+    } else {
+        k_bwd_rows<T, D><<<(unsigned)blocks, 256, 0, counted(s)>>>(p);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     k_bwd_cols<T, D><<<(unsigned)blocks, 256, 0, counted(s)>>>(p);

@@ -80,8 +80,10 @@ def test_backward_over_interval_mask_built_asynchronously(asynchronous):
         assert torch.equal(x, y)
 
 
-@pytest.mark.parametrize("dtype", [workloads.F32, workloads.BF16])
-def test_backward_empty_and_masked_rows_and_full_bias(dtype):
+@pytest.mark.parametrize("dtype,bias_shape", [(workloads.F32, "BHnn"), (workloads.BF16, "BHnn"),
+                                              (workloads.BF16, "1Hnn"), (workloads.F32, "11nn"),
+                                              (workloads.BF16, "111n")])
+def test_backward_empty_and_masked_rows_and_bias_shapes(dtype, bias_shape):
     rng = np.random.default_rng(8)
     B, H, n, d = 2, 2, 150, 64
     rows, rp = [], [0]
@@ -97,7 +99,8 @@ def test_backward_empty_and_masked_rows_and_full_bias(dtype):
     mask = np.zeros((B, 1, n, n))
     mask[:, :, 5, :] = -np.inf                 # a row whose scores are all -inf
     am = workloads.make_tensor(mask, dtype)
-    bias = workloads.make_tensor(rng.standard_normal((B, H, n, n)), dtype)
+    shape = tuple({"B": B, "H": H, "n": n, "1": 1}[x] for x in bias_shape)
+    bias = workloads.make_tensor(rng.standard_normal(shape), dtype)
     scale = 1 / math.sqrt(d)
     with sp.spattn_create_csr_mask("csr", n, 1, in_row_ptr=torch.from_numpy(rp.astype(np.int32)).cuda(),
                                    in_col_idx=torch.from_numpy(ci).cuda()) as m:
