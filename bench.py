@@ -358,8 +358,12 @@ def bench_ours(args, rank, world, torch, sp):
     smi_id = _smi_id(torch, dev)
     launches0 = sp.spattn_launch_count()
     with ClockSampler(smi_id) as clk:
-        for _ in range(args.steps):
+        for it in range(args.steps):
             flush.zero_()                      # evict L2 between steps (outside the events)
+            if it == 0:
+                # the GPU starts idle: a second flush gives the host time to queue
+                # the first step, as it is ahead for every later one
+                flush.zero_()
             s = torch.cuda.Event(enable_timing=True)
             e = torch.cuda.Event(enable_timing=True)
             s.record(stream)
@@ -400,7 +404,7 @@ def bench_ours(args, rank, world, torch, sp):
         "config": {"workload": f"{wl.name} B={wl.B} H={wl.H} n={wl.n} d={wl.d}", "B": wl.B, "H": wl.H,
                    "n": wl.n, "d": wl.d, "mask": wl.mask.kind, "num_masks": wl.mask.num_masks,
                    "nnz_total": nnz_total, "flop_per_step": flops,
-                   "l2": "flushed before every timed step (256 MiB write)",
+                   "l2": "flushed before every timed step (256 MiB write; twice before the first)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "step": "device mask build (pattern -> CSR -> row schedule + tile plan) + fused forward",
                    "plan_per_mask_set": plan},
@@ -514,6 +518,43 @@ def backward_timing(args, torch, sp):
             "path": "CUDA cores: row pass (dq) + column pass over the transposed mask (dk, dv)"}
 
 
+def fusion_ablation(args, torch, sp):
+    """The fused gather forward (spattn_fwd) against the proposal's three separate
+    stages (spattn_fwd_unfused) on the benchmark workload's CSR, both on CUDA
+    cores, L2 flushed before each call; the unfused path's score buffer is the
+    nnz-sized memory the fused one never allocates."""
+    wl = workloads.make(args.config, seed=replica_seed(args.config, 0))
+    g = GpuWorkload(wl, torch, sp)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    with g.create() as m:
+        rp, ci = m.csr()
+        nnz_mask = m.nnz
+    nm = wl.mask.num_masks
+    nnz_total = nnz_mask * (wl.B * wl.H if nm == 1 else wl.H)
+    res = {}
+    for name, fn in (("fused_gather", sp.spattn_fwd), ("unfused", sp.spattn_fwd_unfused)):
+        call = lambda: fn(g.q, g.k, g.v, rp, ci, nm, add_mask=g.am, bias=g.bias, scale=wl.scale,
+                          out=g.out, lse=g.lse)
+        for _ in range(3):
+            call()
+        ts = []
+        for _ in range(10):
+            flush.zero_()
+            s = torch.cuda.Event(enable_timing=True)
+            e = torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            call()
+            e.record(stream)
+            e.synchronize()
+            ts.append(s.elapsed_time(e))
+        res[name + "_ms"] = round(statistics.median(ts), 4)
+    res["fusion_speedup"] = round(res["unfused_ms"] / res["fused_gather_ms"], 3)
+    res["unfused_score_buffer_bytes"] = 4 * nnz_total
+    res["fused_state_bytes_per_row"] = 4 * (wl.d + 2)
+    return res
+
+
 def other_workloads(torch, sp, skip):
     """Forward-only timings of the other workloads (device-resident inputs, L2 flushed)."""
     res = {}
@@ -625,6 +666,10 @@ def main():
                 result["backward"] = backward_timing(args, torch, sp)
             except Exception as ex:  # keep the headline line
                 result["backward"] = {"error": str(ex)[:200]}
+            try:
+                result["fusion_ablation"] = fusion_ablation(args, torch, sp)
+            except Exception as ex:
+                result["fusion_ablation"] = {"error": str(ex)[:200]}
         if not args.no_cpu_baseline and world == 1:
             threads = os.cpu_count() or 1
             rate, cnt, nz, t = cpu_oracle_rate(wl, args.cpu_seconds, threads)

@@ -231,6 +231,19 @@ int spattn_fwd_mask(const spattn_tensor* q, const spattn_tensor* k, const spattn
                     spattn_mask mask, const spattn_tensor* add_mask, const spattn_tensor* bias,
                     float scale, const spattn_tensor* out, float* lse, void* stream);
 
+/* The same operation as spattn_fwd computed as the proposal's three separate
+ * stages ("[Proposal] Unified Interface/Implementation for Sparse Attention",
+ * opening post: SDDMM, sparse softmax, SpMM): every score goes to an fp32 buffer
+ * of (num_masks == 1 ? B*H : H) * nnz floats taken from the library's pool, a
+ * second kernel turns the scores into softmax weights in place (and writes
+ * lse), a third multiplies the weights with V. It exists to measure what the
+ * fused pass saves (time, and the nnz-sized buffer) on the same inputs.
+ * Arguments and errors as spattn_fwd; OOM when the buffer cannot be had. */
+int spattn_fwd_unfused(const spattn_tensor* q, const spattn_tensor* k, const spattn_tensor* v,
+                       const int32_t* row_ptr, const int32_t* col_idx, int32_t num_masks, int64_t nnz,
+                       const spattn_tensor* add_mask, const spattn_tensor* bias, float scale,
+                       const spattn_tensor* out, float* lse, void* stream);
+
 /* Backward pass over a built mask: the gradients of L = sum(dout * out) with
  * respect to q, k, v and (optionally) the bias, given the forward's out and lse
  * (the chain rule of the operation above; the pages discuss bias gradients in

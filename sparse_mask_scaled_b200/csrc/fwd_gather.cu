@@ -461,6 +461,142 @@ __global__ void __launch_bounds__(256, 2) k_fwd_itv(const FwdParams P) {
     for (int i0 = r0; i0 < r1; i0 += 8) itv_rows8<T, D>(P, b, h, mk, i0, tm, partial);
 }
 
+// ------------------------------------------------------------------ unfused
+// The proposal's three separate stages, for comparison with the fused kernels:
+// an SDDMM that writes every score to memory, a row softmax over those scores
+// (in place, plus lse), and an SpMM of the weights with V. scores: fp32, one
+// copy of the mask's nnz per (b, h) (per h when every b has its own mask),
+// indexed by the mask's CSR position.
+__device__ __forceinline__ int64_t unf_index(const FwdParams& P, int b, int h, int64_t p) {
+    return (P.num_masks == 1 ? (int64_t)b * P.H + h : (int64_t)h) * P.nnz + p;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) k_unf_sddmm(const FwdParams P, float* __restrict__ scores) {
+    using C = Cfg<T, D>;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane / C::LPR, c = lane % C::LPR;
+    const int per_bh = (P.n + 7) >> 3;
+    const int bh = blockIdx.x / per_bh;
+    const int i = (blockIdx.x - bh * per_bh) * 8 + warp;
+    if (i >= P.n) return;
+    const int b = bh / P.H, h = bh - b * P.H;
+    const int64_t mrow = (int64_t)(P.num_masks == 1 ? 0 : b) * P.n + i;
+    int64_t p0, p1;
+    clamp_row(P, mrow, p0, p1);
+    const T* kb = reinterpret_cast<const T*>(P.k) + b * P.k_sb + h * P.k_sh;
+    float qf[C::VEC];
+    Elem<T>::unpack(ldg16(reinterpret_cast<const T*>(P.q) + b * P.q_sb + h * P.q_sh + i * P.q_sn + c * C::VEC), qf);
+    const int64_t mask_base = b * P.mask.s0 + h * P.mask.s1 + i * P.mask.s2;
+    const int64_t bias_base = b * P.bias.s0 + h * P.bias.s1 + i * P.bias.s2;
+    const float scale = P.qk_scale_log2 / kLog2e;
+    for (int64_t pb = p0; pb < p1; pb += C::G) {  // one nonzero per group, same trip count for all
+        const int64_t p = pb + g;
+        const bool in = p < p1;
+        const int j = in ? __ldg(P.col_idx + p) : 0;
+        const bool ok = in && (unsigned)j < (unsigned)P.n;
+        float kf[C::VEC];
+        if (ok) Elem<T>::unpack(ldg16(kb + (int64_t)j * P.k_sn + c * C::VEC), kf);
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < C::VEC; ++e) a = ok ? fmaf(qf[e], kf[e], a) : 0.f;
+#pragma unroll
+        for (int off = 1; off < C::LPR; off <<= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+        if (in && c == 0) {
+            float sc = -INFINITY;
+            if (ok) {
+                sc = scale * a;
+                if (P.mask.data) sc += load_addend(P.mask, mask_base + j * P.mask.s3);
+                if (P.bias.data) sc += load_addend(P.bias, bias_base + j * P.bias.s3);
+            } else {
+                atomicOr(&g_error_flags, kErrBadColumn);
+            }
+            scores[unf_index(P, b, h, p)] = sc;
+        }
+    }
+}
+
+// One warp per row: max, then exp and sum, then the weights in place; lse.
+__global__ void __launch_bounds__(256) k_unf_softmax(const FwdParams P, float* __restrict__ scores) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int per_bh = (P.n + 7) >> 3;
+    const int bh = blockIdx.x / per_bh;
+    const int i = (blockIdx.x - bh * per_bh) * 8 + warp;
+    if (i >= P.n) return;
+    const int b = bh / P.H, h = bh - b * P.H;
+    const int64_t mrow = (int64_t)(P.num_masks == 1 ? 0 : b) * P.n + i;
+    int64_t p0, p1;
+    clamp_row(P, mrow, p0, p1);
+    float* row = scores + unf_index(P, b, h, 0);
+    float m = -INFINITY;
+    for (int64_t p = p0 + lane; p < p1; p += 32) m = fmaxf(m, row[p]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    const float mu = m == -INFINITY ? 0.f : m;
+    float l = 0.f;
+    for (int64_t p = p0 + lane; p < p1; p += 32) {
+        const float e = ex2((row[p] - mu) * kLog2e);
+        row[p] = e;
+        l += e;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    for (int64_t p = p0 + lane; p < p1; p += 32) row[p] *= inv;
+    if (lane == 0 && P.lse) P.lse[(int64_t)bh * P.n + i] = l > 0.f ? m + lg2(l) * kLn2 : -INFINITY;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) k_unf_spmm(const FwdParams P, const float* __restrict__ weights) {
+    using C = Cfg<T, D>;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane / C::LPR, c = lane % C::LPR;
+    const int per_bh = (P.n + 7) >> 3;
+    const int bh = blockIdx.x / per_bh;
+    const int i = (blockIdx.x - bh * per_bh) * 8 + warp;
+    if (i >= P.n) return;
+    const int b = bh / P.H, h = bh - b * P.H;
+    const int64_t mrow = (int64_t)(P.num_masks == 1 ? 0 : b) * P.n + i;
+    int64_t p0, p1;
+    clamp_row(P, mrow, p0, p1);
+    const T* vb = reinterpret_cast<const T*>(P.v) + b * P.v_sb + h * P.v_sh;
+    const float* w = weights + unf_index(P, b, h, 0);
+    float acc[C::VEC];
+#pragma unroll
+    for (int e = 0; e < C::VEC; ++e) acc[e] = 0.f;
+    for (int64_t p = p0 + g; p < p1; p += C::G) {
+        const int j = __ldg(P.col_idx + p);
+        if ((unsigned)j >= (unsigned)P.n) continue;
+        const float wp = w[p];
+        float vf[C::VEC];
+        Elem<T>::unpack(ldg16(vb + (int64_t)j * P.v_sn + c * C::VEC), vf);
+#pragma unroll
+        for (int e = 0; e < C::VEC; ++e) acc[e] = fmaf(wp, vf[e], acc[e]);
+    }
+#pragma unroll
+    for (int off = C::LPR; off < 32; off <<= 1) {
+#pragma unroll
+        for (int e = 0; e < C::VEC; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+    }
+    if (lane < C::LPR) {
+        T* orow = reinterpret_cast<T*>(P.out) + b * P.o_sb + h * P.o_sh + i * P.o_sn;
+        *reinterpret_cast<uint4*>(orow + lane * C::VEC) = Elem<T>::pack(acc);
+    }
+}
+
+template <typename T, int D>
+cudaError_t launch_unfused_t(const FwdParams& p, float* scores, cudaStream_t s) {
+    const int64_t blocks = (int64_t)p.B * p.H * ((p.n + 7) / 8);
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    k_unf_sddmm<T, D><<<(unsigned)blocks, 256, 0, counted(s)>>>(p, scores);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    k_unf_softmax<<<(unsigned)blocks, 256, 0, counted(s)>>>(p, scores);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_unf_spmm<T, D><<<(unsigned)blocks, 256, 0, counted(s)>>>(p, scores);
+    return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ backward
 // Gradients of L = sum(dout * out) (the chain rule of the forward's definition):
 // with P_ij = exp(s_ij - lse_i) and D_i = <dout_i, out_i> = sum_j P_ij <dout_i, v_j>,
@@ -860,6 +996,23 @@ cudaError_t launch_fwd_short_rows(const FwdParams& p, int dtype, int d, cudaStre
         case 32: return launch_short_t<float, 32>(p, s);
         case 64: return launch_short_t<float, 64>(p, s);
         case 128: return launch_short_t<float, 128>(p, s);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_fwd_unfused(const FwdParams& p, int dtype, int d, float* scores, cudaStream_t s) {
+    if (dtype == 0) {
+        switch (d) {
+        case 32: return launch_unfused_t<__nv_bfloat16, 32>(p, scores, s);
+        case 64: return launch_unfused_t<__nv_bfloat16, 64>(p, scores, s);
+        case 128: return launch_unfused_t<__nv_bfloat16, 128>(p, scores, s);
+        }
+    } else {
+        switch (d) {
+        case 32: return launch_unfused_t<float, 32>(p, scores, s);
+        case 64: return launch_unfused_t<float, 64>(p, scores, s);
+        case 128: return launch_unfused_t<float, 128>(p, scores, s);
         }
     }
     return cudaErrorInvalidValue;

@@ -1112,6 +1112,38 @@ int spattn_fwd_mask(const spattn_tensor* q, const spattn_tensor* k, const spattn
     return r;
 }
 
+int spattn_fwd_unfused(const spattn_tensor* q, const spattn_tensor* k, const spattn_tensor* v,
+                       const int32_t* row_ptr, const int32_t* col_idx, int32_t num_masks, int64_t nnz,
+                       const spattn_tensor* add_mask, const spattn_tensor* bias, float scale,
+                       const spattn_tensor* out, float* lse, void* stream_v) {
+    g_msg[0] = 0;
+    FwdParams p;
+    int dtype, d;
+    int r = check_fwd(q, k, v, add_mask, bias, scale, out, lse, &p, &dtype, &d);
+    if (r) return r;
+    if (num_masks != 1 && num_masks != p.B) return fail(SPATTN_ERR_INVALID_ARG, "num_masks must be 1 or B");
+    if (!row_ptr) return fail(SPATTN_ERR_INVALID_ARG, "row_ptr is NULL");
+    if (nnz < 0) return fail(SPATTN_ERR_INVALID_ARG, "nnz < 0");
+    if (nnz > 0 && !col_idx) return fail(SPATTN_ERR_INVALID_ARG, "col_idx is NULL");
+    if ((int64_t)p.B * p.H * p.n == 0) return SPATTN_OK;
+    cudaStream_t s = (cudaStream_t)stream_v;
+    int dev;
+    CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
+    cudaMemPool_t pool;
+    CUDA_TRY(device_state(dev, &pool, nullptr), "memory pool");
+    p.row_ptr = row_ptr;
+    p.col_idx = col_idx;
+    p.nnz = nnz;
+    p.num_masks = num_masks;
+    float* scores = nullptr;
+    const int64_t copies = num_masks == 1 ? (int64_t)p.B * p.H : (int64_t)p.H;
+    CUDA_TRY(pool_alloc(&scores, copies * (nnz > 0 ? nnz : 1), pool, s), "score buffer");
+    const cudaError_t e = launch_fwd_unfused(p, dtype, d, scores, s);
+    cudaFreeAsync(scores, s);
+    if (e != cudaSuccess) return cuda_fail(e, "unfused kernel launch");
+    return SPATTN_OK;
+}
+
 int spattn_bwd_mask(const spattn_tensor* q, const spattn_tensor* k, const spattn_tensor* v,
                     spattn_mask mask, const spattn_tensor* add_mask, const spattn_tensor* bias,
                     float scale, const spattn_tensor* out, const float* lse, const spattn_tensor* dout,

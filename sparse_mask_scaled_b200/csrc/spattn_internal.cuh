@@ -101,6 +101,9 @@ struct BwdParams {
     float qk_scale_log2;
 };
 cudaError_t launch_bwd(const BwdParams& p, int dtype, int d, cudaStream_t stream);
+// The unfused three-stage forward (SDDMM -> row softmax -> SpMM); scores: fp32
+// [(num_masks == 1 ? B*H : H) * nnz].
+cudaError_t launch_fwd_unfused(const FwdParams& p, int dtype, int d, float* scores, cudaStream_t stream);
 
 // Tensor-core kernel (fwd_tc.cu).
 struct TcOperand {
