@@ -96,6 +96,12 @@ class ClockSampler:
         self.device_id = device_id
         self.proc = None
         self.lines = []
+        self.start = 0
+        self.end = None
+
+    def mark(self):
+        """Only samples taken after this call (and before the sampler stops) count."""
+        self.start = len(self.lines)
 
     def __enter__(self):
         try:
@@ -119,6 +125,7 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def __exit__(self, *exc):
+        self.end = len(self.lines)  # samples after this are of an idle GPU
         if self.proc:
             time.sleep(0.25)
             self.proc.terminate()
@@ -130,7 +137,8 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        window = self.lines[self.start:self.end]
+        for ln in window if window else self.lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -347,17 +355,19 @@ def bench_ours(args, rank, world, torch, sp):
         m.close()
         return ev0, ev1
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
     starts, ends, fwd_evs = [], [], []
     smi_id = _smi_id(torch, dev)
-    launches0 = sp.spattn_launch_count()
     with ClockSampler(smi_id) as clk:
+        clk.mark()       # samples from the warm-up (under the same load) and the timed steps
+        # warm-up right before the timed steps (clocks up, pool and caches warm)
+        for _ in range(args.warmup):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        launches0 = sp.spattn_launch_count()
         for it in range(args.steps):
             flush.zero_()                      # evict L2 between steps (outside the events)
             if it == 0:
@@ -518,6 +528,18 @@ def backward_timing(args, torch, sp):
             "path": "CUDA cores: row pass (dq) + column pass over the transposed mask (dk, dv)"}
 
 
+def key_padding_lengths(wl):
+    """Per-batch key lengths when the workload's additive mask is a key-padding
+    mask [B, 1, 1, n] of 0 then -inf, else None."""
+    if wl.add_mask is None or wl.add_mask.raw.shape[1:3] != (1, 1):
+        return None
+    keep = wl.add_mask.f64()[:, 0, 0, :] == 0
+    lengths = keep.sum(axis=1)
+    if not np.array_equal(keep, np.arange(wl.n)[None, :] < lengths[:, None]):
+        return None
+    return [int(x) for x in lengths]
+
+
 def fusion_ablation(args, torch, sp):
     """The fused gather forward (spattn_fwd) against the proposal's three separate
     stages (spattn_fwd_unfused) on the benchmark workload's CSR, both on CUDA
@@ -582,6 +604,25 @@ def other_workloads(torch, sp, skip):
                     e.synchronize()
                     ts.append(s.elapsed_time(e))
                 t = statistics.median(ts)
+                t_kpad = None
+                lengths = key_padding_lengths(wl)
+                if lengths is not None:   # the same forward with the padding given as lengths
+                    sl = torch.tensor(lengths, dtype=torch.int32, device="cuda")
+                    kp = lambda: sp.spattn_fwd_mask_kpad(g.q, g.k, g.v, m, sl, bias=g.bias, scale=wl.scale,
+                                                         out=g.out, lse=g.lse)
+                    for _ in range(3):
+                        kp()
+                    tk = []
+                    for _ in range(10):
+                        flush.zero_()
+                        s = torch.cuda.Event(enable_timing=True)
+                        e = torch.cuda.Event(enable_timing=True)
+                        s.record(stream)
+                        kp()
+                        e.record(stream)
+                        e.synchronize()
+                        tk.append(s.elapsed_time(e))
+                    t_kpad = statistics.median(tk)
                 tb = time.perf_counter()
                 m2 = g.create()
                 torch.cuda.synchronize()
@@ -593,6 +634,8 @@ def other_workloads(torch, sp, skip):
                             "effective_gbs": round(alg / (t * 1e-3) / 1e9, 1),
                             "frac_hbm": round(alg / (t * 1e-3) / 1e9 / hbm_peak, 4),
                             "nnz_total": nnz_total, "mask_build_wall_ms": round(build_ms, 3)}
+            if t_kpad is not None:
+                res[wl.name]["fwd_ms_seqlen_k"] = round(t_kpad, 4)
             del g
         except Exception as ex:  # keep the headline line even if one extra case fails
             res[f"cfg{cfg}"] = {"error": str(ex)[:200]}

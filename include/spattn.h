@@ -271,6 +271,19 @@ int spattn_bwd_mask(const spattn_tensor* q, const spattn_tensor* k, const spattn
                     const spattn_tensor* dq, const spattn_tensor* dk, const spattn_tensor* dv,
                     const spattn_tensor* dbias, void* stream);
 
+/* spattn_fwd_mask with key padding given as lengths: for batch element b only
+ * keys j < seqlen_k[b] exist (seqlen_k: device int32 [B], clamped to [0, n]),
+ * as if every score with j >= seqlen_k[b] were -inf -- the seqlen_k form of the
+ * key-padding mask in "support attentions in AlphaFold2" (flash-attention PR
+ * 57, the discussion of varlen key padding). One int per batch element is read
+ * instead of a mask row, and tensor-core tiles wholly past the length are
+ * skipped. seqlen_k may be NULL (no padding); add_mask and bias still apply.
+ * Arguments and errors otherwise as spattn_fwd_mask. */
+int spattn_fwd_mask_kpad(const spattn_tensor* q, const spattn_tensor* k, const spattn_tensor* v,
+                         spattn_mask mask, const int32_t* seqlen_k, const spattn_tensor* add_mask,
+                         const spattn_tensor* bias, float scale, const spattn_tensor* out, float* lse,
+                         void* stream);
+
 /* The same operation as spattn_fwd, but the call allocates no device memory.
  * For callers that cannot call cudaMalloc or take memory from a pool at run
  * time: for example a host program or plug-in whose memory manager owns the

@@ -91,6 +91,8 @@ SIGNATURES = {
                                           _TP, ctypes.c_float, _TP, _P, _P]),
     "spattn_last_error": (ctypes.c_char_p, []),
     "spattn_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "spattn_fwd_mask_kpad": (ctypes.c_int, [_TP, _TP, _TP, _P, _P, _TP, _TP, ctypes.c_float, _TP, _P,
+                                            _P]),
     "spattn_fwd_unfused": (ctypes.c_int, [_TP, _TP, _TP, _P, _P, ctypes.c_int32, ctypes.c_int64, _TP,
                                           _TP, ctypes.c_float, _TP, _P, _P]),
     "spattn_bwd_mask": (ctypes.c_int, [_TP, _TP, _TP, _P, _TP, _TP, ctypes.c_float, _TP, _P, _TP, _TP,
@@ -348,6 +350,23 @@ def spattn_device_error(stream=None) -> int:
 
 def spattn_last_error() -> str:
     return LIB.spattn_last_error().decode()
+
+
+def spattn_fwd_mask_kpad(q, k, v, mask: "Mask", seqlen_k, add_mask=None, bias=None,
+                         scale: Optional[float] = None, out=None, lse=None, want_lse: bool = True,
+                         stream=None) -> Tuple[object, object]:
+    """``spattn_fwd_mask`` with key padding as lengths: ``seqlen_k`` is an int32
+    CUDA tensor [B]; keys j >= seqlen_k[b] are left out."""
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
+    out, lse = _outputs(q, out, lse, want_lse)
+    dq, dk, dv, do = tensor_desc(q), tensor_desc(k), tensor_desc(v), tensor_desc(out)
+    dm = tensor_desc(add_mask) if add_mask is not None else None
+    db = tensor_desc(bias) if bias is not None else None
+    _check(LIB.spattn_fwd_mask_kpad(ctypes.byref(dq), ctypes.byref(dk), ctypes.byref(dv), mask.handle,
+                                    _ptr(seqlen_k), ctypes.byref(dm) if dm is not None else None,
+                                    ctypes.byref(db) if db is not None else None, float(scale),
+                                    ctypes.byref(do), _ptr(lse), _stream(stream)))
+    return out, lse
 
 
 def spattn_fwd_unfused(q, k, v, row_ptr, col_idx, num_masks: int = 1, add_mask=None, bias=None,

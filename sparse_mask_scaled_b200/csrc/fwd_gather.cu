@@ -118,10 +118,18 @@ __device__ __forceinline__ void clamp_row(const FwdParams& P, int64_t mrow, int6
     p1 = p1 < p0 ? p0 : (p1 > P.nnz ? P.nnz : p1);
 }
 
+// Keys of batch element b that exist: [0, seqlen_k[b]) with key padding, else [0, n).
+__device__ __forceinline__ int key_limit(const FwdParams& P, int b) {
+    if (!P.seqlen_k) return P.n;
+    const int L = P.seqlen_k[b];
+    return L < 0 ? 0 : (L > P.n ? P.n : L);
+}
+
 template <typename T, int D>
 struct RowCtx {
     const T* kb;   // K of (b, h)
     const T* vb;   // V of (b, h)
+    int klim;      // keys >= klim are padding
     int64_t mask_base, bias_base;  // addend offsets of (b, h, i, 0)
     float qf[Cfg<T, D>::VEC];      // this lane's slice of q_i * scale * log2(e)
 };
@@ -136,6 +144,7 @@ __device__ __forceinline__ void init_row(const FwdParams& P, int b, int h, int i
     rc.vb = reinterpret_cast<const T*>(P.v) + b * P.v_sb + h * P.v_sh;
     rc.mask_base = b * P.mask.s0 + h * P.mask.s1 + i * P.mask.s2;
     rc.bias_base = b * P.bias.s0 + h * P.bias.s1 + i * P.bias.s2;
+    rc.klim = key_limit(P, b);
     Elem<T>::unpack(ldg16(q + c * C::VEC), rc.qf);
 #pragma unroll
     for (int e = 0; e < C::VEC; ++e) rc.qf[e] *= P.qk_scale_log2;
@@ -161,7 +170,9 @@ __device__ __forceinline__ void row_steps(const FwdParams& P, const RowCtx<T, D>
         const int64_t mp = pb + lane;
         if (lane < C::STEP && mp < p1) {
             const int j = kRun ? (int)mp : __ldg(P.col_idx + mp);
-            if ((unsigned)j < (unsigned)P.n) {
+            if ((unsigned)j >= (unsigned)P.n) {
+                atomicOr(&g_error_flags, kErrBadColumn);
+            } else if (j < rc.klim) {  // padded keys are left out
                 col = j;
                 if (P.has_extra) {
                     float e = 0.f;
@@ -169,8 +180,6 @@ __device__ __forceinline__ void row_steps(const FwdParams& P, const RowCtx<T, D>
                     if (P.bias.data) e += load_addend(P.bias, rc.bias_base + j * P.bias.s3);
                     extra = e * kLog2e;
                 }
-            } else {
-                atomicOr(&g_error_flags, kErrBadColumn);
             }
         }
         int js[C::U];
@@ -367,11 +376,12 @@ __device__ __forceinline__ void itv_rows8(const FwdParams& P, int b, int h, int 
     __shared__ float sm_acc[8][D];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int i = i0 + warp;
+    const int klim = key_limit(P, b);
     int lo = 0, hi = 0;
     if (i < P.n) {
         const int2 v = P.itv_lohi[(int64_t)mk * P.n + i];
         lo = v.x;
-        hi = v.y;
+        hi = v.y < klim ? v.y : klim;
     }
     int len = 0;
     for_each_run(tm, lo, hi, lane, [&](int a, int z) { len += z - a; });
@@ -388,7 +398,8 @@ __device__ __forceinline__ void itv_rows8(const FwdParams& P, int b, int h, int 
     }
     for (int rr = 0; rr < 8 && i0 + rr < P.n; ++rr) {
         const int ii = i0 + rr;
-        const int2 v = P.itv_lohi[(int64_t)mk * P.n + ii];
+        int2 v = P.itv_lohi[(int64_t)mk * P.n + ii];
+        v.y = v.y < klim ? v.y : klim;
         RowCtx<T, D> rc;
         State<C::VEC> st;
         init_row<T, D>(P, b, h, ii, lane, rc, st);

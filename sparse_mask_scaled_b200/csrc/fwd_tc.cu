@@ -160,6 +160,20 @@ __device__ __forceinline__ void add_addend_run(const AddendView& a, int64_t rowb
     }
 }
 
+// Key padding: the keys of batch element b are [0, L) (L = n without it). Tiles
+// are listed by ascending key tile, so the ones at or past L are dropped from
+// the end; one is kept so that the epilogue still writes the rows.
+__device__ __forceinline__ int key_limit_tc(const TcParams& P, int b) {
+    if (!P.seqlen_k) return P.n;
+    const int L = P.seqlen_k[b];
+    return L < 0 ? 0 : (L > P.n ? P.n : L);
+}
+__device__ __forceinline__ int trim_tiles(const TcParams& P, int t_begin, int T, int L) {
+    if (P.seqlen_k)
+        while (T > 1 && (P.tile_info[t_begin + T - 1] & 0x7fffffff) * kTileN >= L) --T;
+    return T;
+}
+
 // First tile and number of tiles of query block blk.
 __device__ __forceinline__ void block_tiles(const TcParams& P, int64_t blk, int& t_begin, int& T) {
     if (P.block_ntiles) {
@@ -224,7 +238,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t blk = (int64_t)mk * P.nqb + qb;
     int t_begin, T;
     block_tiles(P, blk, t_begin, T);
-    if (T <= 0) return;  // whole CTA: the gather kernel owns this block
+    if (T <= 0) return;
+    const int klim = key_limit_tc(P, b);
+    T = trim_tiles(P, t_begin, T, klim);  // whole CTA: the gather kernel owns this block
     if (smem_u32(smem) & 1023u) {  // the swizzled layouts need a 1024-byte aligned base
         if (tid == 0) atomicOr(P.err, kErrTimeout);
         return;
@@ -350,7 +366,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool dense = info < 0;  // the same for the whole CTA
         const bool extra = P.has_extra && row_ok;
         const int jj0 = kt * 128;
-        const uint4 wb = P.itv_lohi && row_ok && !dense ? tile_row_bits4(P, 0, info, row, rlo, rhi) : wbits;
+        uint4 wb = P.itv_lohi && row_ok && !dense ? tile_row_bits4(P, 0, info, row, rlo, rhi) : wbits;
+        const int lim = klim - jj0;  // keys of this tile that exist
+        const bool cut = lim < 128;
+        if (cut) {
+            if (dense) wb = make_uint4(~0u, ~0u, ~0u, ~0u);
+            wb.x &= run_word(0, lim, 0);
+            wb.y &= run_word(0, lim, 32);
+            wb.z &= run_word(0, lim, 64);
+            wb.w &= run_word(0, lim, 96);
+        }
         const uint32_t bw[4] = {wb.x, wb.y, wb.z, wb.w};
 
         wait(barS, (uint32_t)(u & 1));
@@ -388,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mul2(xh[32 + 2 * k], xh[33 + 2 * k], r1[2 * k], r1[2 * k + 1], c2);
                 }
             }
-            if (!dense) {
+            if (!dense || cut) {
 #pragma unroll
                 for (int j = 0; j < 64; ++j)
                     xh[j] = ((bw[half * 2 + (j >> 5)] >> (j & 31)) & 1u) ? xh[j] : -INFINITY;
@@ -597,7 +622,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
     const int64_t blk = (int64_t)mk * P.nqb + qb;
     int t_begin, T;
     block_tiles(P, blk, t_begin, T);
-    if (T <= 0) return;
+    if (T <= 0) return;  // (key padding goes to k_fwd_tc_ws)
     if (smem_u32(smem) & 1023u) {
         if (tid == 0) atomicOr(P.err, kErrTimeout);
         return;
@@ -948,7 +973,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
 // Variant for d <= 64 without barriers in the tile loop, launched when a mask
 // or bias is added (its global loads then sit on each tile's path, and
 // independent halves hide them better: 7 % faster on the Evoformer workload,
-// 2-3 % slower than k_fwd_tc_pipe without addends).
+// 2-3 % slower than k_fwd_tc_pipe without addends) or keys are padded.
 // Eight warps, two threads per query row, two CTAs per SM.
 //
 // Thread (half, row), half = warp / 4, owns keys 64*half .. 64*half+63 of
@@ -1011,6 +1036,8 @@ __global__ void __launch_bounds__(kWsThreads, 2)
     int t_begin, T;
     block_tiles(P, blk, t_begin, T);
     if (T <= 0) return;
+    const int klim = key_limit_tc(P, b);
+    T = trim_tiles(P, t_begin, T, klim);
     if (smem_u32(smem) & 1023u) {
         if (tid == 0) atomicOr(P.err, kErrTimeout);
         return;
@@ -1174,8 +1201,14 @@ __global__ void __launch_bounds__(kWsThreads, 2)
             if (P.mask.data) add_addend_run<64>(P.mask, mask_rowbase, c0, ncols, x);
             if (P.bias.data) add_addend_run<64>(P.bias, bias_rowbase, c0, ncols, x);
         }
-        if (!dense) {  // entries the mask does not list
-            const uint2 wb = P.itv_lohi ? tile_row_bits2(P, 0, info, row, half, rlo, rhi) : wbits;
+        const int lim = klim - kt * 128 - half * 64;  // keys of this tile half that exist
+        if (!dense || lim < 64) {  // entries the mask does not list, or padding
+            uint2 wb = dense ? make_uint2(~0u, ~0u)
+                             : (P.itv_lohi ? tile_row_bits2(P, 0, info, row, half, rlo, rhi) : wbits);
+            if (lim < 64) {
+                wb.x &= run_word(0, lim, 0);
+                wb.y &= run_word(0, lim, 32);
+            }
             const uint32_t bw[2] = {wb.x, wb.y};
 #pragma unroll
             for (int j = 0; j < 64; ++j) x[j] = ((bw[j >> 5] >> (j & 31)) & 1u) ? x[j] : -INFINITY;
@@ -1387,6 +1420,9 @@ cudaError_t launch_tc_t(const TcOperand& q, const TcOperand& k, const TcOperand&
             if (attr_err == cudaSuccess)
                 attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_ws<DP, true>,
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+            if (attr_err == cudaSuccess)
+                attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_ws<DP, false>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         } else {
             attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc<D>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -1398,13 +1434,15 @@ cudaError_t launch_tc_t(const TcOperand& q, const TcOperand& k, const TcOperand&
     if ((e = make_map(&mq, q, p.B, p.H, p.n, D, C::CHUNK_ELEMS)) != cudaSuccess) return e;
     if ((e = make_map(&mk, k, p.B, p.H, p.n, D, C::CHUNK_ELEMS)) != cudaSuccess) return e;
     // the kernel for mask/bias addends loads V in halves of 64 rows
-    const bool halves = D <= 64 && p.has_extra;
+    const bool halves = D <= 64 && (p.has_extra || p.seqlen_k);
     if ((e = make_map(&mv, v, p.B, p.H, p.n, D, C::CHUNK_ELEMS, halves ? 64 : 128)) != cudaSuccess) return e;
     const int64_t grid = (int64_t)p.B * p.H * p.nqb;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     constexpr int DP = D <= 64 ? D : 64;
     if (D <= 64 && p.has_extra)
         k_fwd_tc_ws<DP, true><<<(unsigned)grid, kWsThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, p);
+    else if (D <= 64 && p.seqlen_k)
+        k_fwd_tc_ws<DP, false><<<(unsigned)grid, kWsThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, p);
     else if (D <= 64)
         k_fwd_tc_pipe<DP, false><<<(unsigned)grid, kPipeThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, p);
     else

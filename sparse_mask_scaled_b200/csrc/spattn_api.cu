@@ -639,6 +639,7 @@ int launch_tc(const FwdParams& p, int d, spattn_mask m, int dev, const int32_t* 
     tp.bias = p.bias;
     tp.has_extra = p.has_extra;
     tp.qk_scale_log2 = p.qk_scale_log2;
+    tp.seqlen_k = p.seqlen_k;
     tp.err = ef;
     const TcOperand oq{p.q, p.q_sn, p.q_sh, p.q_sb}, ok{p.k, p.k_sn, p.k_sh, p.k_sb},
         ov{p.v, p.v_sn, p.v_sh, p.v_sb};
@@ -1057,11 +1058,20 @@ int spattn_fwd(const spattn_tensor* q, const spattn_tensor* k, const spattn_tens
 int spattn_fwd_mask(const spattn_tensor* q, const spattn_tensor* k, const spattn_tensor* v,
                     spattn_mask mask, const spattn_tensor* add_mask, const spattn_tensor* bias,
                     float scale, const spattn_tensor* out, float* lse, void* stream_v) {
+    return spattn_fwd_mask_kpad(q, k, v, mask, nullptr, add_mask, bias, scale, out, lse, stream_v);
+}
+
+int spattn_fwd_mask_kpad(const spattn_tensor* q, const spattn_tensor* k, const spattn_tensor* v,
+                         spattn_mask mask, const int32_t* seqlen_k, const spattn_tensor* add_mask,
+                         const spattn_tensor* bias, float scale, const spattn_tensor* out, float* lse,
+                         void* stream_v) {
     g_msg[0] = 0;
     FwdParams p;
     int dtype, d;
     int r = check_fwd(q, k, v, add_mask, bias, scale, out, lse, &p, &dtype, &d);
     if (r) return r;
+    if (seqlen_k && ((uintptr_t)seqlen_k) % 4 != 0) return fail(SPATTN_ERR_INVALID_ARG, "seqlen_k not aligned");
+    p.seqlen_k = seqlen_k;
     if (!mask) return fail(SPATTN_ERR_INVALID_ARG, "mask is NULL");
     if (mask->n != p.n) return fail(SPATTN_ERR_INVALID_ARG, "mask n %d != q n %d", mask->n, p.n);
     if (mask->num_masks != 1 && mask->num_masks != p.B)

@@ -73,6 +73,7 @@ struct FwdParams {
     const int32_t* blk_res;
     const int32_t* qb_ntiles;  // tensor-core tiles per query block
     int nkt;
+    const int32_t* seqlen_k;  // nullable, [B]: keys j >= seqlen_k[b] are left out (key padding)
     int itv_slices;  // 1, 2, 4, 8 or 16 thread blocks per 128-row query block
 };
 
@@ -118,6 +119,7 @@ struct TcParams {
     // x * tile_stride + block_ntiles[x] - 1] (interval masks).
     const int32_t* block_ntiles;
     int tile_stride;
+    const int32_t* seqlen_k;  // nullable, [B]: keys j >= seqlen_k[b] are left out
     const uint32_t* tile_bits;      // [tiles][128 rows][4 words]
     const int32_t* res_row_ptr;     // residual CSR (a row with entries has a partial)
     // Interval masks: masks come from the row runs instead of tile_bits, and the
