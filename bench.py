@@ -283,7 +283,10 @@ def forward_roofline(wl, plan, nnz_total, flops, alg_bytes, per_nnz, t_fwd_ms, h
     t = t_fwd_ms * 1e-3
     src_peak = "measured MEASURED_PEAKS.json" if peak_src == "measured" else "fallback"
     if plan["tensor_core_tiles"] > 0 and wl.dtype == workloads.BF16:
-        kname = f"k_fwd_tc_pipe<{wl.d},{int(extra)}>" if wl.d <= 64 else f"k_fwd_tc<{wl.d}>"
+        if wl.d > 64:
+            kname = f"k_fwd_tc<{wl.d}>"
+        else:
+            kname = f"k_fwd_tc_ws<{wl.d},1>" if extra else f"k_fwd_tc_quad<{wl.d}>"
         tiles = plan["tensor_core_tiles"] * rep
         mma_flops = tiles * 2 * (2 * 128 * 128 * wl.d)
         ex2 = tiles * 128 * 128

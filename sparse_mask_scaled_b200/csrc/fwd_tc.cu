@@ -3,22 +3,23 @@
 //
 // One CTA owns one 128-row query block of one (b, h) and walks the block's
 // selected key tiles. Per tile:
-//   S = Q K^T               tcgen05.mma (M = 128, N = 128, K = d), S in TMEM
+//   S = Q K^T               tcgen05.mma (M = 128, N = 128 or two N = 64 halves,
+//                           K = d), S in TMEM
 //   s = scale*S + mask + bias, entries the mask does not list set to -inf
 //   running max / sum       the streaming-dataflow SDPA paper's rescaling rule;
 //                           the max used as reference only moves when a tile's
 //                           max exceeds it by more than 2^8, and then the O
 //                           accumulator in TMEM is rescaled by exp2(m_old - m_new)
-//   O += P V                tcgen05.mma (M = 128, N = d, K = 128), P from smem
+//   O += P V                tcgen05.mma (M = 128, N = d), P from TMEM or smem
 // K/V tiles are double-buffered and loaded by TMA (no multicast) while the
 // previous tile's softmax and P V run. At the end O / l is written (bf16) and
 // lse = m + log(l); rows that also have residual (gathered) entries first merge
 // the gather kernel's partial (m, l, acc) with the same rescaling rule.
 //
-// Three kernels: k_fwd_tc<d> (d = 128, one thread per row), k_fwd_tc_pipe<d>
-// (d <= 64 without addends, two threads per row) and k_fwd_tc_ws<d> (d <= 64
-// with a mask or bias, two threads per row with independent key halves and no
-// barrier in the tile loop).
+// Three kernels: k_fwd_tc<d> (d = 128, one thread per row), k_fwd_tc_quad<d>
+// (d <= 64 without addends: one thread per row, 64-key sub-tiles, P in TMEM,
+// four CTAs per SM) and k_fwd_tc_ws<d> (d <= 64 with a mask or bias, two
+// threads per row with independent key halves and no barrier in the tile loop).
 //
 // Every mbarrier wait is bounded: on expiry the CTA raises the device error
 // flag, drains what it issued (bounded again), frees its TMEM and returns.
@@ -222,6 +223,25 @@ __device__ __forceinline__ bool has_partial(const TcParams& P, int64_t blk, int6
     if (!P.ws_ml) return false;
     if (P.blk_res) return P.blk_res[blk] && P.ws_ml[wrow * 2 + 1] > 0.f;
     return P.res_row_ptr[mrow + 1] > P.res_row_ptr[mrow];
+}
+
+// Counts this warp in; true for lane 0 of the warp whose arrival is number
+// `last` (0-based). Orders the warp's earlier shared-memory, async-proxy and
+// tensor-memory accesses before the count and makes the others' visible to the
+// winner.
+__device__ __forceinline__ bool arrive_last(uint32_t* counter, uint32_t last) {
+    tc_fence_before();
+    __syncwarp();
+    bool win = false;
+    if ((threadIdx.x & 31) == 0) {
+        __threadfence_block();
+        win = atomicAdd(counter, 1u) == last;
+        if (win) {
+            __threadfence_block();
+            tc_fence_after();
+        }
+    }
+    return win;
 }
 
 template <int D>
@@ -591,99 +611,147 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ----------------------------------------------------------------------------
-// Variant for d <= 64 without addends: two threads per query row (8 warps per
-// CTA, two CTAs per SM). Thread (half, row) handles keys 64*half .. 64*half + 63 of each tile
-// and O columns half*d/2 .. of its row. Per tile:
-//   wait S(u) | load its 64 scores into registers (one TMEM round trip) | scale,
-//   add mask/bias, drop unlisted entries, partial max | wait P V(u-1) |
-//   partial max to the partner (through the P buffer) | sync -> issue S(u+1)
-//   (the S columns are free: the scores are in registers) | row max; if it grew
-//   by more than 2^8, rescale O in TMEM | exp2, partial sum, P to smem | sync ->
-//   issue P V(u) accumulating into O in TMEM, and K(u+2)
-// O stays in TMEM (M = 128, N = d accumulator) for the whole block, so no tile
-// needs to read it back.
-constexpr int kPipeThreads = 256;
+// Variant for d <= 64 without addends: four warps, one query row per thread
+// (the row's TMEM lane), 128 TMEM columns, so four CTAs share an SM and their
+// per-tile dependency chains overlap. Each 128-key tile of the plan is walked
+// as two 64-key sub-tiles s = 0, 1, ... TMEM: S(s) (fp32) in columns [0, 64);
+// once every row has read it, P(s) (bf16, two per column) overwrites columns
+// [0, 32); O in [64, 64 + d). Per sub-tile, every warp:
+//   wait S(s) | (thread 0: TMA K(s+2) into K(s)'s buffer and V(s+1) into
+//   V(s-1)'s buffer, both free now) | S(s) to registers, scale, drop the
+//   entries the mask does not list, row max | if the max grew past the
+//   threshold, rescale O in TMEM (P V(s-1) is done: S(s) was issued after it)
+//   | exp2, row sum, P(s) to TMEM | the warp whose arrival completes "P
+//   written" issues O (+)= P(s) V(s) (A operand from TMEM), waits for it (P
+//   must be consumed before S(s+1) overwrites it) and issues S(s+1).
+// No warp waits for another except through the data; the block epilogue
+// reads O, divides by the row sum, merges the gather kernel's partial and
+// writes out and lse.
+constexpr int kQuadThreads = 128;
+constexpr uint32_t kQuadCols = 128;
 
-template <int D, bool EXTRA>
-__global__ void __launch_bounds__(kPipeThreads, 2)
-    k_fwd_tc_pipe(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+template <int D>
+struct QuadCfg {
+    using C = TcCfg<D>;
+    static constexpr int Q_BYTES = C::TILE_BYTES;       // 128 rows x d
+    static constexpr int KV_BYTES = C::TILE_BYTES / 2;  // 64 rows x d
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = Q_BYTES;               // two buffers
+    static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;  // two buffers
+    static constexpr int OFF_BAR = OFF_V + 2 * KV_BYTES;
+    // mbarriers Q_full, K_full[2], V_full[2], S_full, O_done; TMEM slot, abort
+    // flag, "P written" arrivals; issue counts (K, V loads, S, P V commits)
+    static constexpr int BAR_BYTES = 7 * 8 + 3 * 4 + 4 * 4;
+    // at most four CTAs per SM (4 x 128 TMEM columns)
+    static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES > 46 * 1024 ? OFF_BAR + BAR_BYTES : 46 * 1024;
+};
+
+// Bounded wait that also gives up as soon as another warp of the CTA has.
+__device__ __forceinline__ bool pers_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitCycles) {
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kQuadThreads, 4)
+    k_fwd_tc_quad(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const TcParams P) {
     using C = TcCfg<D>;
-    static_assert(D <= 64, "two threads per row split d/2 O columns each");
-    constexpr int DH = D / 2;  // O columns per thread
+    using L = QuadCfg<D>;
+    static_assert(D == 32 || D == 64, "head dim");
     extern __shared__ __align__(1024) uint8_t smem[];
 
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int half = warp >> 2;  // key half of each tile (and O column half)
-    const int row = tid & 127;   // query row in the block == TMEM lane
     const int bh = blockIdx.x / P.nqb, qb = blockIdx.x - bh * P.nqb;
     const int b = bh / P.H, h = bh - b * P.H;
     const int mk = P.num_masks == 1 ? 0 : b;
     const int64_t blk = (int64_t)mk * P.nqb + qb;
     int t_begin, T;
     block_tiles(P, blk, t_begin, T);
-    if (T <= 0) return;  // (key padding goes to k_fwd_tc_ws)
+    if (T <= 0) return;
+    const int klim = key_limit_tc(P, b);
+    T = trim_tiles(P, t_begin, T, klim);
     if (smem_u32(smem) & 1023u) {
         if (tid == 0) atomicOr(P.err, kErrTimeout);
         return;
     }
+    const int NS = 2 * T;  // 64-key sub-tiles
 
-    const uint32_t sQ = smem_u32(smem + C::OFF_Q);
-    const uint32_t sK0 = smem_u32(smem + C::OFF_K), sV0 = smem_u32(smem + C::OFF_V);
-    const uint32_t sP = smem_u32(smem + C::OFF_P);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-    // barriers: Q, K[2], V[2], S, O
+    const uint32_t sQ = smem_u32(smem + L::OFF_Q), sK0 = smem_u32(smem + L::OFF_K),
+                   sV0 = smem_u32(smem + L::OFF_V);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
     const uint32_t barQ = smem_u32(bars + 0), barK0 = smem_u32(bars + 1), barV0 = smem_u32(bars + 3),
                    barS = smem_u32(bars + 5), barO = smem_u32(bars + 6);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    // partner exchange slot: row `row` of P chunk (1 - half), first 16 bytes (swizzled);
-    // only the partner reads it, and the partner overwrites it with its own P later
-    const uint32_t my_slot = sP + (uint32_t)((half ^ 1) * 16384 + row * 128 + ((0 ^ (row & 7)) << 4));
-    const uint32_t partner_slot = sP + (uint32_t)(half * 16384 + row * 128 + ((0 ^ (row & 7)) << 4));
+    uint32_t* pcnt = tmem_slot + 2;    // "P written" arrivals
+    uint32_t* issued = tmem_slot + 3;  // [0] K, [1] V loads, [2] S, [3] P V commits
 
-    if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    // the row's state first: these loads run while the CTA sets up and the
+    // first tiles arrive
+    const int i = qb * 128 + tid;
+    const bool row_ok = i < P.n;
+    int rlo = 0, rhi = 0;  // interval masks: the row's run
+    if (P.itv_lohi && row_ok) {
+        const int2 v = P.itv_lohi[(int64_t)mk * P.n + i];
+        rlo = v.x;
+        rhi = v.y;
+    }
+    int info_next = P.tile_info[t_begin];  // the plan entry of the next 128-key tile
+    int info = info_next;
+
+    // K or V sub-tile s (first key `key`) into buffer s & 1
+    auto load_k = [&](int s, int key) {
+        const uint32_t bar = barK0 + 8u * (s & 1);
+        mbar_expect_tx(bar, (uint32_t)L::KV_BYTES);
+        tma_load_4d(sK0 + (uint32_t)((s & 1) * L::KV_BYTES), &tmK, bar, 0, key, h, b);
+        issued[0] += 1u;
+    };
+    auto load_v = [&](int s, int key) {
+        const uint32_t bar = barV0 + 8u * (s & 1);
+        mbar_expect_tx(bar, (uint32_t)L::KV_BYTES);
+        tma_load_4d(sV0 + (uint32_t)((s & 1) * L::KV_BYTES), &tmV, bar, 0, key, h, b);
+        issued[1] += 1u;
+    };
+
+    if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kQuadCols);
     if (tid == 0) {
         for (int x = 0; x < 7; ++x) mbar_init(smem_u32(bars + x), 1);
         *abort_flag = 0;
+        for (int x = 0; x < 5; ++x) pcnt[x] = 0u;  // and issued[]
         fence_mbar_init();
         prefetch_tensormap(&tmQ);
         prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmV);
+        // Q and both halves of the first tile (every block has at least one)
+        mbar_expect_tx(barQ, (uint32_t)L::Q_BYTES);
+        tma_load_4d(sQ, &tmQ, barQ, 0, qb * 128, h, b);
+        const int key = (info & 0x7fffffff) * kTileN;
+        load_k(0, key);
+        load_k(1, key + 64);
+        load_v(0, key);
+        load_v(1, key + 64);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tO = tmem + 128;
-    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem, tP = tmem, tO = tmem + 64;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
 
-    // thread 0: issued operations per barrier (scalars: no dynamically indexed arrays)
-    int n_k0 = 0, n_k1 = 0, n_v0 = 0, n_v1 = 0, n_s = 0, n_pv = 0;
-
-    auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
-        if (*abort_flag) return false;
-        if (mbar_wait_bounded(bar, parity, kWaitCycles)) return true;
-        *abort_flag = 1;
-        return false;
-    };
-    auto tile_kt = [&](int u) { return P.tile_info[t_begin + u] & 0x7fffffff; };
-    auto issue_k = [&](int u) {
-        const uint32_t bar = barK0 + 8u * (u & 1);
-        mbar_expect_tx(bar, (uint32_t)C::TILE_BYTES);
-        tma_load_4d(sK0 + (uint32_t)((u & 1) * C::TILE_BYTES), &tmK, bar, 0, tile_kt(u) * 128, h, b);
-        if (u & 1) ++n_k1; else ++n_k0;
-    };
-    auto issue_v = [&](int u) {
-        const uint32_t bar = barV0 + 8u * (u & 1);
-        mbar_expect_tx(bar, (uint32_t)C::TILE_BYTES);
-        tma_load_4d(sV0 + (uint32_t)((u & 1) * C::TILE_BYTES), &tmV, bar, 0, tile_kt(u) * 128, h, b);
-        if (u & 1) ++n_v1; else ++n_v0;
-    };
-    const uint32_t idS = idesc_bf16_f32(128, 128, false);
-    const uint32_t idO = idesc_bf16_f32(128, D, true);
-    auto issue_S = [&](int u) {
-        const uint32_t sK = sK0 + (uint32_t)((u & 1) * C::TILE_BYTES);
+    auto issue_s = [&](int s) -> bool {  // S(s) = Q K(s)^T once K(s) is loaded
+        if (!pers_wait(barK0 + 8u * (s & 1), (uint32_t)((s >> 1) & 1), abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t sK = sK0 + (uint32_t)((s & 1) * L::KV_BYTES);
+        const uint32_t idS = idesc_bf16_f32(128, 64, false);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
             const uint64_t da = smem_desc(sQ + ks * 32, 16, C::SBO, C::LAYOUT);
@@ -691,97 +759,88 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
             mma_bf16_ss(tS, da, db, idS, ks > 0 ? 1u : 0u);
         }
         mma_commit(barS);
-        ++n_s;
+        issued[2] += 1u;
+        return true;
     };
-    auto issue_PV = [&](int u) {
-        const uint32_t sV = sV0 + (uint32_t)((u & 1) * C::TILE_BYTES);
+    auto issue_pv = [&](int s) -> bool {  // O (+)= P(s) V(s) once V(s) is loaded
+        if (!pers_wait(barV0 + 8u * (s & 1), (uint32_t)((s >> 1) & 1), abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t sV = sV0 + (uint32_t)((s & 1) * L::KV_BYTES);
+        const uint32_t idO = idesc_bf16_f32(128, D, true);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t da = smem_desc(sP + (uint32_t)((ks >> 2) * 16384 + (ks & 3) * 32), 16, 1024,
-                                          cute::UMMA::LayoutType::SWIZZLE_128B);
-            const uint64_t db = smem_desc(sV + (uint32_t)(ks * 16 * C::ROW_BYTES), C::CHUNK_BYTES, C::SBO,
-                                          C::LAYOUT);
-            mma_bf16_ss(tO, da, db, idO, (u > 0 || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t db =
+                smem_desc(sV + (uint32_t)(ks * 16 * C::ROW_BYTES), C::CHUNK_BYTES, C::SBO, C::LAYOUT);
+            mma_bf16_ts(tO, tP + (uint32_t)(ks * 8), db, idO, (s > 0 || ks > 0) ? 1u : 0u);
         }
         mma_commit(barO);
-        ++n_pv;
+        issued[3] += 1u;
+        return true;
     };
 
-    if (tid == 0) {
-        mbar_expect_tx(barQ, (uint32_t)C::TILE_BYTES);
-        tma_load_4d(sQ, &tmQ, barQ, 0, qb * 128, h, b);
-        issue_k(0);
-        issue_v(0);
-        if (T > 1) {
-            issue_k(1);
-            issue_v(1);
-        }
-        if (wait(barQ, 0) && wait(barK0, 0)) {
-            tc_fence_after();
-            issue_S(0);
-        }
-    }
+    if (tid == 0 && pers_wait(barQ, 0u, abort_flag)) issue_s(0);
+    __syncwarp();
 
-    const int i = qb * 128 + row;
-    const bool row_ok = i < P.n;
-    const int64_t mask_rowbase = (int64_t)b * P.mask.s0 + (int64_t)h * P.mask.s1 + (int64_t)i * P.mask.s2;
-    const int64_t bias_rowbase = (int64_t)b * P.bias.s0 + (int64_t)h * P.bias.s1 + (int64_t)i * P.bias.s2;
-    float m_ref = -INFINITY, l = 0.f;  // l: this thread's half of the row sum
-    int rlo = 0, rhi = 0;  // interval masks: the row's run
-    if (P.itv_lohi && row_ok) {
-        const int2 v = P.itv_lohi[(int64_t)mk * P.n + i];
-        rlo = v.x;
-        rhi = v.y;
-    }
-
-    int next_info = P.tile_info[t_begin];
-    uint2 next_bits = make_uint2(0u, 0u);  // stored bits, loaded one tile ahead
-    if (next_info >= 0 && row_ok && !P.itv_lohi)
-        next_bits = tile_row_bits2(P, t_begin, next_info, row, half, rlo, rhi);
     const uint64_t c2 = pack2(P.qk_scale_log2, P.qk_scale_log2);
-
-    for (int u = 0; u < T; ++u) {
-        const int info = next_info;
-        const uint2 wbits = next_bits;
-        if (u + 1 < T) {
-            next_info = P.tile_info[t_begin + u + 1];
-            if (next_info >= 0 && row_ok && !P.itv_lohi)
-                next_bits = tile_row_bits2(P, t_begin + u + 1, next_info, row, half, rlo, rhi);
+    float m_ref = -INFINITY, l = 0.f;
+    for (int s = 0; s < NS; ++s) {
+        if ((s & 1) == 0) {  // a new 128-key tile; fetch the next one's entry early
+            info = info_next;
+            if ((s >> 1) + 1 < T) info_next = P.tile_info[t_begin + (s >> 1) + 1];
         }
-        const int kt = info & 0x7fffffff;
-        const bool dense = info < 0;
-        const bool extra = EXTRA && row_ok;
+        const int c0 = (info & 0x7fffffff) * kTileN + 64 * (s & 1);
+        bool dense = info < 0;
+        uint32_t wb0 = 0u, wb1 = 0u;
+        if (!dense && row_ok) {
+            if (P.itv_lohi) {
+                wb0 = run_word(rlo, rhi, c0);
+                wb1 = run_word(rlo, rhi, c0 + 32);
+            } else {
+                const uint2 v = __ldg(reinterpret_cast<const uint2*>(P.tile_bits) +
+                                      ((int64_t)(t_begin + (s >> 1)) * 128 + tid) * 2 + (s & 1));
+                wb0 = v.x;
+                wb1 = v.y;
+            }
+        }
+        const int kcut = klim - c0;  // keys of this sub-tile inside the key length
+        if (kcut < 64) {
+            if (dense) {
+                dense = false;
+                wb0 = wb1 = 0xffffffffu;
+            }
+            wb0 &= run_word(0, kcut, 0);
+            wb1 &= run_word(0, kcut, 32);
+        }
 
-        float x[64];
-
-        wait(barS, (uint32_t)(u & 1));
+        const bool ok = pers_wait(barS, (uint32_t)(s & 1), abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
-        if (tid == 0 && u + 2 < T && !*abort_flag) issue_k(u + 2);  // S(u) consumed K(u)
-        __syncwarp();
+        if (tid == 0) {  // S(s) done: K(s)'s buffer is free; P V(s-1) done: so is V(s-1)'s
+            // sub-tile s + 2 is the next tile's half s & 1; s + 1 is this tile's
+            // second half (s even) or the next tile's first (s odd)
+            if (s + 2 < NS) load_k(s + 2, (info_next & 0x7fffffff) * kTileN + 64 * (s & 1));
+            if (s >= 1 && s + 1 < NS)
+                load_v(s + 1, (((s & 1) ? info_next : info) & 0x7fffffff) * kTileN + 64 * ((s + 1) & 1));
+        }
+        float x[64];
         {
             uint32_t r0[32], r1[32];
-            tmem_ld32(tS + lane_base + half * 64, r0);
-            tmem_ld32(tS + lane_base + half * 64 + 32, r1);
+            tmem_ld32(tS + lane_base, r0);
+            tmem_ld32(tS + lane_base + 32, r1);
             tmem_wait_ld_dep(r0);
             tmem_wait_ld_dep(r1);
-            // x = scale*log2(e)*S, two lanes per instruction
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 mul2(x[2 * k], x[2 * k + 1], r0[2 * k], r0[2 * k + 1], c2);
                 mul2(x[32 + 2 * k], x[33 + 2 * k], r1[2 * k], r1[2 * k + 1], c2);
             }
         }
-        if (extra) {  // + log2(e) * (mask + bias)
-            const int c0 = kt * 128 + half * 64;
-            const int ncols = P.n - c0 < 64 ? P.n - c0 : 64;
-            if (P.mask.data) add_addend_run<64>(P.mask, mask_rowbase, c0, ncols, x);
-            if (P.bias.data) add_addend_run<64>(P.bias, bias_rowbase, c0, ncols, x);
-        }
-        if (!dense) {  // entries the CSR does not list
-            const uint2 wb = P.itv_lohi ? tile_row_bits2(P, 0, info, row, half, rlo, rhi) : wbits;
-            const uint32_t bw[2] = {wb.x, wb.y};
+        if (!dense) {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) x[j] = ((bw[j >> 5] >> (j & 31)) & 1u) ? x[j] : -INFINITY;
+            for (int jj = 0; jj < 32; ++jj) {
+                x[jj] = ((wb0 >> jj) & 1u) ? x[jj] : -INFINITY;
+                x[32 + jj] = ((wb1 >> jj) & 1u) ? x[32 + jj] : -INFINITY;
+            }
         }
         float ma = -INFINITY, mb = -INFINITY, mc = -INFINITY, md = -INFINITY;
 #pragma unroll
@@ -791,29 +850,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
             mc = fmax3(mc, x[8 * k + 4], x[8 * k + 5]);
             md = fmax3(md, x[8 * k + 6], x[8 * k + 7]);
         }
-        const float my_max = fmax3(ma, mb, fmaxf(mc, md));
-
-        if (u > 0) {  // P V(u-1) must be done: it reads sP and accumulates into O
-            wait(barO, (uint32_t)((u - 1) & 1));
-            tc_fence_after();
-            if (tid == 0 && u + 1 < T && !*abort_flag) issue_v(u + 1);  // V(u-1)'s buffer is free
-            __syncwarp();
-        }
-        asm volatile("st.shared.f32 [%0], %1;" ::"r"(my_slot), "f"(my_max) : "memory");
-        // the S columns are free (scores are in registers): S(u+1) runs during exp2
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0 && u + 1 < T && !*abort_flag) {
-            tc_fence_after();
-            if (wait(barK0 + 8u * ((u + 1) & 1), (uint32_t)(((u + 1) >> 1) & 1))) {
-                tc_fence_after();
-                issue_S(u + 1);
-            }
-        }
-        __syncwarp();
-        float other_max;
-        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(other_max) : "r"(partner_slot) : "memory");
-        const float mx = fmaxf(my_max, other_max);
+        const float mx = fmax3(ma, mb, fmaxf(mc, md));
         const bool need = mx > m_ref + kRescaleThreshold;
         float alpha = 1.f;
         if (need) {
@@ -821,51 +858,33 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
             m_ref = mx;
             l *= alpha;
         }
-        if (u > 0 && __any_sync(0xffffffffu, need)) {  // O holds P V(0..u-1): bring it to the new max
-            const uint32_t src = tO + lane_base + half * DH;
-            if constexpr (DH == 32) {
-                uint32_t ro[32];
-                tmem_ld32(src, ro);
-                tmem_wait_ld_dep(ro);
+        if (s > 0 && __any_sync(0xffffffffu, need)) {  // bring O (= P V(..s-1), complete) to the new max
 #pragma unroll
-                for (int j = 0; j < 32; ++j) ro[j] = __float_as_uint(__uint_as_float(ro[j]) * alpha);
-                tmem_st32(src, ro);
-            } else {
+            for (int c = 0; c < D / 16; ++c) {
                 uint32_t ro[16];
-                tmem_ld16(src, ro);
+                tmem_ld16(tO + lane_base + 16 * c, ro);
                 tmem_wait_ld_dep16(ro);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) ro[j] = __float_as_uint(__uint_as_float(ro[j]) * alpha);
-                tmem_st16(src, ro);
+                for (int jj = 0; jj < 16; ++jj) ro[jj] = __float_as_uint(__uint_as_float(ro[jj]) * alpha);
+                tmem_st16(tO + lane_base + 16 * c, ro);
             }
-            tmem_wait_st();
         }
         const float mu = m_ref == -INFINITY ? 0.f : m_ref;
-        // p = exp2(x - mu), partial sum, P (bf16) into chunk `half` of the K-major,
-        // 128-byte-swizzled A operand layout
         const uint64_t nmu2 = pack2(-mu, -mu);
         uint64_t sa = pack2(0.f, 0.f), sb = sa;
+        uint32_t pk[32];  // P row, two bf16 per word
 #pragma unroll
-        for (int piece = 0; piece < 8; ++piece) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const int k = piece * 4 + t;
-                float p0, p1;
-                unpack2(add2(pack2(x[2 * k], x[2 * k + 1]), nmu2), p0, p1);
-                p0 = ex2(p0);
-                p1 = ex2(p1);
-                if (k & 1)
-                    sb = add2(sb, pack2(p0, p1));
-                else
-                    sa = add2(sa, pack2(p0, p1));
-                __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
-                pk[t] = *reinterpret_cast<uint32_t*>(&hv);
-            }
-            const uint32_t addr = sP + (uint32_t)(half * 16384 + row * 128 + ((piece ^ (row & 7)) << 4));
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[0]), "r"(pk[1]),
-                         "r"(pk[2]), "r"(pk[3])
-                         : "memory");
+        for (int k = 0; k < 32; ++k) {
+            float p0, p1;
+            unpack2(add2(pack2(x[2 * k], x[2 * k + 1]), nmu2), p0, p1);
+            p0 = ex2(p0);
+            p1 = ex2(p1);
+            if (k & 1)
+                sb = add2(sb, pack2(p0, p1));
+            else
+                sa = add2(sa, pack2(p0, p1));
+            __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
+            pk[k] = *reinterpret_cast<uint32_t*>(&hv);
         }
         {
             float s0, s1, s2, s3;
@@ -873,108 +892,97 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
             unpack2(sb, s2, s3);
             l += (s0 + s1) + (s2 + s3);
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0 && !*abort_flag) {
-            tc_fence_after();
-            if (wait(barV0 + 8u * (u & 1), (uint32_t)((u >> 1) & 1))) {
-                tc_fence_after();
-                issue_PV(u);
-            }
+        tmem_st32(tP + lane_base, pk);
+        tmem_wait_st();
+        if (arrive_last(pcnt, 4u * (uint32_t)(s + 1) - 1u) && !*abort_flag) {
+            // every row has written P(s) (and rescaled O): P V(s), then S(s+1) once
+            // P V(s) has consumed P (S(s+1) overwrites it)
+            if (issue_pv(s) && s + 1 < NS && pers_wait(barO, (uint32_t)(s & 1), abort_flag)) issue_s(s + 1);
         }
+        __syncwarp();
     }
 
     // ------------------------------------------------------------ epilogue
-    wait(barO, (uint32_t)((T - 1) & 1));
-    tc_fence_after();
-    __syncwarp();
-    float o[DH];
-    {
-        const uint32_t src = tO + lane_base + half * DH;
-        if constexpr (DH == 32) {
+    const bool ok = pers_wait(barO, (uint32_t)((NS - 1) & 1), abort_flag);
+    if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after();
+        float o[D];
+        {
             uint32_t ro[32];
-            tmem_ld32(src, ro);
-            tmem_wait_ld_dep(ro);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __uint_as_float(ro[j]);
-        } else {
-            uint32_t ro[16];
-            tmem_ld16(src, ro);
-            tmem_wait_ld_dep16(ro);
+            for (int c = 0; c < D / 32; ++c) {
+                tmem_ld32(tO + lane_base + 32 * c, ro);
+                tmem_wait_ld_dep(ro);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) o[j] = __uint_as_float(ro[j]);
-        }
-    }
-    // combine the two halves of the row sum (sP is free: the last P V is done)
-    asm volatile("st.shared.f32 [%0], %1;" ::"r"(my_slot), "f"(l) : "memory");
-    __syncthreads();
-    float l_other;
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(l_other) : "r"(partner_slot) : "memory");
-    const float l_row = l + l_other;
-    if (row_ok && !*abort_flag) {
-        float M = m_ref, L = l_row, fa = 1.f;
-        const int64_t mrow = (int64_t)mk * P.n + i;
-        const int64_t wrow = (int64_t)bh * P.n + i;
-        const bool mixed = has_partial(P, blk, mrow, wrow);
-        float fg = 0.f;
-        if (mixed) {
-            const float mg = P.ws_ml[wrow * 2], lg = P.ws_ml[wrow * 2 + 1];
-            M = fmaxf(m_ref, mg);
-            const float Mu = M == -INFINITY ? 0.f : M;
-            fa = ex2(m_ref - Mu);
-            fg = ex2(mg - Mu);
-            L = l_row * fa + lg * fg;
-        }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(P.out) + (int64_t)b * P.o_sb +
-                              (int64_t)h * P.o_sh + (int64_t)i * P.o_sn + half * DH;
-        const float* acc = mixed ? P.ws_acc + wrow * D + half * DH : nullptr;
-#pragma unroll
-        for (int e8 = 0; e8 < DH / 8; ++e8) {
-            float v[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                float val = o[e8 * 8 + t] * fa;
-                if (mixed) val = fmaf(acc[e8 * 8 + t], fg, val);
-                v[t] = val * inv;
+                for (int jj = 0; jj < 32; ++jj) o[32 * c + jj] = __uint_as_float(ro[jj]);
             }
-            uint32_t w[4];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                __nv_bfloat162 hv = __floats2bfloat162_rn(v[2 * t], v[2 * t + 1]);
-                w[t] = *reinterpret_cast<uint32_t*>(&hv);
-            }
-            *reinterpret_cast<uint4*>(orow + e8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        if (P.lse && half == 0) P.lse[wrow] = L > 0.f ? (M + lg2(L)) * kLn2 : -INFINITY;
+        if (row_ok && !*abort_flag) {
+            const int64_t mrow = (int64_t)mk * P.n + i, wrow = (int64_t)bh * P.n + i;
+            float M = m_ref, Ls = l, fa = 1.f, fg = 0.f;
+            const bool mixed = has_partial(P, blk, mrow, wrow);
+            if (mixed) {
+                const float mg = P.ws_ml[wrow * 2], lg = P.ws_ml[wrow * 2 + 1];
+                M = fmaxf(m_ref, mg);
+                const float Mu = M == -INFINITY ? 0.f : M;
+                fa = ex2(m_ref - Mu);
+                fg = ex2(mg - Mu);
+                Ls = l * fa + lg * fg;
+            }
+            const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(P.out) + (int64_t)b * P.o_sb +
+                                  (int64_t)h * P.o_sh + (int64_t)i * P.o_sn;
+            const float* acc = mixed ? P.ws_acc + wrow * D : nullptr;
+#pragma unroll
+            for (int e8 = 0; e8 < D / 8; ++e8) {
+                float v[8];
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    float val = o[e8 * 8 + t] * fa;
+                    if (mixed) val = fmaf(acc[e8 * 8 + t], fg, val);
+                    v[t] = val * inv;
+                }
+                uint32_t w[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    __nv_bfloat162 hv = __floats2bfloat162_rn(v[2 * t], v[2 * t + 1]);
+                    w[t] = *reinterpret_cast<uint32_t*>(&hv);
+                }
+                *reinterpret_cast<uint4*>(orow + e8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            if (P.lse) P.lse[wrow] = Ls > 0.f ? (M + lg2(Ls)) * kLn2 : -INFINITY;
+        }
     }
 
     // ------------------------------------------------------------ teardown
-    if (tid == 0 && *abort_flag) {
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && *abort_flag) {  // drain what was issued (bounded), then report
         const long long lim = kWaitCycles / 16;
-        const int cnt[4] = {n_k0, n_k1, n_v0, n_v1};
-        const uint32_t bar4[4] = {barK0, barK0 + 8u, barV0, barV0 + 8u};
-        for (int x = 0; x < 4; ++x)
-            if (cnt[x]) mbar_wait_bounded(bar4[x], (uint32_t)((cnt[x] - 1) & 1), lim);
-        if (n_s) mbar_wait_bounded(barS, (uint32_t)((n_s - 1) & 1), lim);
-        if (n_pv) mbar_wait_bounded(barO, (uint32_t)((n_pv - 1) & 1), lim);
+        mbar_wait_bounded(barQ, 0u, lim);
+        for (int x = 0; x < 2; ++x)
+            for (int bnum = 0; bnum < 2; ++bnum) {
+                const int uses = ((int)issued[x] - bnum + 1) / 2;  // loads into buffer bnum
+                if (uses > 0)
+                    mbar_wait_bounded(smem_u32(bars + 1 + 2 * x + bnum), (uint32_t)((uses - 1) & 1), lim);
+            }
+        if (issued[2]) mbar_wait_bounded(barS, (issued[2] - 1u) & 1u, lim);
+        if (issued[3]) mbar_wait_bounded(barO, (issued[3] - 1u) & 1u, lim);
         atomicOr(P.err, kErrTimeout);
     }
-    tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, kQuadCols);
     }
 }
 
 // ----------------------------------------------------------------------------
 // Variant for d <= 64 without barriers in the tile loop, launched when a mask
-// or bias is added (its global loads then sit on each tile's path, and
-// independent halves hide them better: 7 % faster on the Evoformer workload,
-// 2-3 % slower than k_fwd_tc_pipe without addends) or keys are padded.
-// Eight warps, two threads per query row, two CTAs per SM.
+// or bias is added (its global loads then sit on each tile's path; on the
+// Evoformer workload independent halves hide them 7 % better than two
+// threads per row that share one running max). Eight warps, two threads per
+// query row, two CTAs per SM.
 //
 // Thread (half, row), half = warp / 4, owns keys 64*half .. 64*half+63 of
 // every tile with its own running max m_half and sum l_half -- the two halves
@@ -997,24 +1005,6 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
 // TMEM: S columns [0, 128), O_0 [128, 128 + d), O_1 [128 + d, 128 + 2d).
 constexpr int kWsThreads = 256;
 
-// Counts this warp in; true for lane 0 of the warp whose arrival is number
-// `last` (0-based). Orders the warp's earlier shared-memory, async-proxy and
-// tensor-memory accesses before the count and makes the others' visible to the
-// winner.
-__device__ __forceinline__ bool arrive_last(uint32_t* counter, uint32_t last) {
-    tc_fence_before();
-    __syncwarp();
-    bool win = false;
-    if ((threadIdx.x & 31) == 0) {
-        __threadfence_block();
-        win = atomicAdd(counter, 1u) == last;
-        if (win) {
-            __threadfence_block();
-            tc_fence_after();
-        }
-    }
-    return win;
-}
 
 template <int D, bool EXTRA>
 __global__ void __launch_bounds__(kWsThreads, 2)
@@ -1415,14 +1405,12 @@ cudaError_t launch_tc_t(const TcOperand& q, const TcOperand& k, const TcOperand&
     std::call_once(once, []() {
         constexpr int DP = D <= 64 ? D : 64;
         if (D <= 64) {
-            attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_pipe<DP, false>,
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-            if (attr_err == cudaSuccess)
-                attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_ws<DP, true>,
+            attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_ws<DP, true>,
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
             if (attr_err == cudaSuccess)
-                attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_ws<DP, false>,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+                attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_quad<DP>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                QuadCfg<DP>::SMEM_BYTES);
         } else {
             attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc<D>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -1432,20 +1420,19 @@ cudaError_t launch_tc_t(const TcOperand& q, const TcOperand& k, const TcOperand&
     CUtensorMap mq, mk, mv;
     cudaError_t e;
     if ((e = make_map(&mq, q, p.B, p.H, p.n, D, C::CHUNK_ELEMS)) != cudaSuccess) return e;
-    if ((e = make_map(&mk, k, p.B, p.H, p.n, D, C::CHUNK_ELEMS)) != cudaSuccess) return e;
-    // the kernel for mask/bias addends loads V in halves of 64 rows
-    const bool halves = D <= 64 && (p.has_extra || p.seqlen_k);
-    if ((e = make_map(&mv, v, p.B, p.H, p.n, D, C::CHUNK_ELEMS, halves ? 64 : 128)) != cudaSuccess) return e;
+    // d <= 64: k_fwd_tc_quad loads K and V in 64-row sub-tiles, the kernel for
+    // mask/bias addends V in halves of 64 rows
+    const bool quad = D <= 64 && !p.has_extra;
+    if ((e = make_map(&mk, k, p.B, p.H, p.n, D, C::CHUNK_ELEMS, quad ? 64 : 128)) != cudaSuccess) return e;
+    if ((e = make_map(&mv, v, p.B, p.H, p.n, D, C::CHUNK_ELEMS, D <= 64 ? 64 : 128)) != cudaSuccess) return e;
     const int64_t grid = (int64_t)p.B * p.H * p.nqb;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     constexpr int DP = D <= 64 ? D : 64;
-    if (D <= 64 && p.has_extra)
+    if (D <= 64 && p.has_extra) {
         k_fwd_tc_ws<DP, true><<<(unsigned)grid, kWsThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, p);
-    else if (D <= 64 && p.seqlen_k)
-        k_fwd_tc_ws<DP, false><<<(unsigned)grid, kWsThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, p);
-    else if (D <= 64)
-        k_fwd_tc_pipe<DP, false><<<(unsigned)grid, kPipeThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, p);
-    else
+    } else if (D <= 64) {
+        k_fwd_tc_quad<DP><<<(unsigned)grid, kQuadThreads, QuadCfg<DP>::SMEM_BYTES, counted(s)>>>(mq, mk, mv, p);
+    } else
         k_fwd_tc<D><<<(unsigned)grid, kThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }
