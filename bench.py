@@ -286,7 +286,7 @@ def forward_roofline(wl, plan, nnz_total, flops, alg_bytes, per_nnz, t_fwd_ms, h
         if wl.d > 64:
             kname = f"k_fwd_tc<{wl.d}>"
         else:
-            kname = f"k_fwd_tc_ws<{wl.d},1>" if extra else f"k_fwd_tc_quad<{wl.d}>"
+            kname = f"k_fwd_tc_quad<{wl.d},{int(extra)}>"
         tiles = plan["tensor_core_tiles"] * rep
         mma_flops = tiles * 2 * (2 * 128 * 128 * wl.d)
         ex2 = tiles * 128 * 128

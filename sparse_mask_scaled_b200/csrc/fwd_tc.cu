@@ -16,10 +16,9 @@
 // lse = m + log(l); rows that also have residual (gathered) entries first merge
 // the gather kernel's partial (m, l, acc) with the same rescaling rule.
 //
-// Three kernels: k_fwd_tc<d> (d = 128, one thread per row), k_fwd_tc_quad<d>
-// (d <= 64 without addends: one thread per row, 64-key sub-tiles, P in TMEM,
-// four CTAs per SM) and k_fwd_tc_ws<d> (d <= 64 with a mask or bias, two
-// threads per row with independent key halves and no barrier in the tile loop).
+// Two kernels: k_fwd_tc<d> (d = 128, one thread per row) and
+// k_fwd_tc_quad<d, EXTRA> (d <= 64: one thread per row, 64-key sub-tiles, P in
+// TMEM, four CTAs per SM, three with an additive mask or bias).
 //
 // Every mbarrier wait is bounded: on expiry the CTA raises the device error
 // flag, drains what it issued (bounded again), frees its TMEM and returns.
@@ -205,16 +204,6 @@ __device__ __forceinline__ uint4 tile_row_bits4(const TcParams& P, int t, int in
                           run_word(lo, hi, c0 + 96));
     }
     return __ldg(reinterpret_cast<const uint4*>(P.tile_bits) + ((int64_t)t * 128 + row));
-}
-
-// The same for key half `half` (64 columns).
-__device__ __forceinline__ uint2 tile_row_bits2(const TcParams& P, int t, int info, int row, int half, int lo,
-                                                int hi) {
-    if (P.itv_lohi) {
-        const int c0 = (info & 0x7fffffff) * kTileN + half * 64;
-        return make_uint2(run_word(lo, hi, c0), run_word(lo, hi, c0 + 32));
-    }
-    return __ldg(reinterpret_cast<const uint2*>(P.tile_bits) + ((int64_t)t * 128 + row) * 2 + half);
 }
 
 // Whether row (mrow of the mask, wrow of the output) has a partial state from
@@ -611,19 +600,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ----------------------------------------------------------------------------
-// Variant for d <= 64 without addends: four warps, one query row per thread
-// (the row's TMEM lane), 128 TMEM columns, so four CTAs share an SM and their
-// per-tile dependency chains overlap. Each 128-key tile of the plan is walked
-// as two 64-key sub-tiles s = 0, 1, ... TMEM: S(s) (fp32) in columns [0, 64);
-// once every row has read it, P(s) (bf16, two per column) overwrites columns
+// Kernel for d <= 64: four warps, one query row per thread (the row's TMEM
+// lane), 128 TMEM columns, so four CTAs share an SM (three when an additive
+// mask or bias is added, EXTRA: its values take registers) and their per-tile
+// dependency chains overlap. Each 128-key tile of the plan is walked as two
+// 64-key sub-tiles s = 0, 1, ... TMEM: S(s) (fp32) in columns [0, 64); once
+// every row has read it, P(s) (bf16, two per column) overwrites columns
 // [0, 32); O in [64, 64 + d). Per sub-tile, every warp:
 //   wait S(s) | (thread 0: TMA K(s+2) into K(s)'s buffer and V(s+1) into
-//   V(s-1)'s buffer, both free now) | S(s) to registers, scale, drop the
-//   entries the mask does not list, row max | if the max grew past the
-//   threshold, rescale O in TMEM (P V(s-1) is done: S(s) was issued after it)
-//   | exp2, row sum, P(s) to TMEM | the warp whose arrival completes "P
-//   written" issues O (+)= P(s) V(s) (A operand from TMEM), waits for it (P
-//   must be consumed before S(s+1) overwrites it) and issues S(s+1).
+//   V(s-1)'s buffer, both free now) | S(s) to registers, scale, add the
+//   additive terms, drop the entries the mask does not list, row max | if the
+//   max grew past the threshold, rescale O in TMEM (P V(s-1) is done: S(s)
+//   was issued after it) | exp2, row sum, P(s) to TMEM | the warp whose
+//   arrival completes "P written" issues O (+)= P(s) V(s) (A operand from
+//   TMEM), waits for it (P must be consumed before S(s+1) overwrites it) and
+//   issues S(s+1).
 // No warp waits for another except through the data; the block epilogue
 // reads O, divides by the row sum, merges the gather kernel's partial and
 // writes out and lse.
@@ -660,8 +651,8 @@ __device__ __forceinline__ bool pers_wait(uint32_t bar, uint32_t parity, volatil
     }
 }
 
-template <int D>
-__global__ void __launch_bounds__(kQuadThreads, 4)
+template <int D, bool EXTRA>
+__global__ void __launch_bounds__(kQuadThreads, EXTRA ? 3 : 4)
     k_fwd_tc_quad(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const TcParams P) {
     using C = TcCfg<D>;
@@ -707,6 +698,31 @@ __global__ void __launch_bounds__(kQuadThreads, 4)
     }
     int info_next = P.tile_info[t_begin];  // the plan entry of the next 128-key tile
     int info = info_next;
+
+    // Additive mask and bias (EXTRA). One term that varies by row (the bias,
+    // else the mask), when it is bf16 with unit column stride and 16-byte
+    // aligned rows, has the 64 values of the row's next sub-tile fetched as raw
+    // words one sub-tile ahead (after P is stored), so their latency overlaps
+    // P V and the next S. The other term -- typically a key-padding mask shared
+    // by every row, served from L1 -- and every other layout are loaded when used.
+    const int64_t mrb = EXTRA ? (int64_t)b * P.mask.s0 + (int64_t)h * P.mask.s1 + (int64_t)i * P.mask.s2 : 0;
+    const int64_t brb = EXTRA ? (int64_t)b * P.bias.s0 + (int64_t)h * P.bias.s1 + (int64_t)i * P.bias.s2 : 0;
+    // the prefetched term: 2 = bias, 1 = mask, 0 = none
+    const int pre = !EXTRA ? 0 : (P.bias.data && P.bias.s2 != 0) ? 2 : (P.mask.data && P.mask.s2 != 0) ? 1 : 0;
+    const AddendView& pview = pre == 2 ? P.bias : P.mask;
+    const int64_t prb = pre == 2 ? brb : mrb;
+    uint4 praw[EXTRA ? 8 : 1];
+    bool raw = false;  // praw holds the prefetched term's values for the current sub-tile
+    auto fetch = [&](int c0) {
+        raw = false;
+        if (!EXTRA || pre == 0 || !row_ok || c0 + 64 > P.n || pview.dtype != 0 || pview.s3 != 1) return;
+        const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(pview.data) + prb + c0;
+        if (reinterpret_cast<uintptr_t>(src) & 15u) return;
+#pragma unroll
+        for (int k = 0; k < (EXTRA ? 8 : 1); ++k) praw[k] = __ldg(reinterpret_cast<const uint4*>(src) + k);
+        raw = true;
+    };
+    if (EXTRA) fetch((info & 0x7fffffff) * kTileN);
 
     // K or V sub-tile s (first key `key`) into buffer s & 1
     auto load_k = [&](int s, int key) {
@@ -829,10 +845,30 @@ __global__ void __launch_bounds__(kQuadThreads, 4)
             tmem_ld32(tS + lane_base + 32, r1);
             tmem_wait_ld_dep(r0);
             tmem_wait_ld_dep(r1);
+            if (EXTRA && raw) {  // x = scale*log2(e)*S + log2(e)*(prefetched term)
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                mul2(x[2 * k], x[2 * k + 1], r0[2 * k], r0[2 * k + 1], c2);
-                mul2(x[32 + 2 * k], x[33 + 2 * k], r1[2 * k], r1[2 * k + 1], c2);
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t w[4] = {praw[k].x, praw[k].y, praw[k].z, praw[k].w};
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const int j = 8 * k + 2 * t;
+                        const uint32_t s0 = j < 32 ? r0[j] : r1[j - 32], s1 = j < 32 ? r0[j + 1] : r1[j - 31];
+                        x[j] = fmaf(__uint_as_float(s0), P.qk_scale_log2, kLog2e * __uint_as_float(w[t] << 16));
+                        x[j + 1] = fmaf(__uint_as_float(s1), P.qk_scale_log2,
+                                        kLog2e * __uint_as_float(w[t] & 0xffff0000u));
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    mul2(x[2 * k], x[2 * k + 1], r0[2 * k], r0[2 * k + 1], c2);
+                    mul2(x[32 + 2 * k], x[33 + 2 * k], r1[2 * k], r1[2 * k + 1], c2);
+                }
+            }
+            if (EXTRA && row_ok) {  // + log2(e) * (the terms not prefetched), loaded now
+                const int ncols = P.n - c0 < 64 ? P.n - c0 : 64;
+                if (P.mask.data && !(raw && pre == 1)) add_addend_run<64>(P.mask, mrb, c0, ncols, x);
+                if (P.bias.data && !(raw && pre == 2)) add_addend_run<64>(P.bias, brb, c0, ncols, x);
             }
         }
         if (!dense) {
@@ -894,6 +930,8 @@ __global__ void __launch_bounds__(kQuadThreads, 4)
         }
         tmem_st32(tP + lane_base, pk);
         tmem_wait_st();
+        if (EXTRA && s + 1 < NS)  // the next sub-tile: this tile's second half or the next tile's first
+            fetch((((s & 1) ? info_next : info) & 0x7fffffff) * kTileN + 64 * ((s + 1) & 1));
         if (arrive_last(pcnt, 4u * (uint32_t)(s + 1) - 1u) && !*abort_flag) {
             // every row has written P(s) (and rescaled O): P V(s), then S(s+1) once
             // P V(s) has consumed P (S(s+1) overwrites it)
@@ -977,387 +1015,6 @@ __global__ void __launch_bounds__(kQuadThreads, 4)
     }
 }
 
-// ----------------------------------------------------------------------------
-// Variant for d <= 64 without barriers in the tile loop, launched when a mask
-// or bias is added (its global loads then sit on each tile's path; on the
-// Evoformer workload independent halves hide them 7 % better than two
-// threads per row that share one running max). Eight warps, two threads per
-// query row, two CTAs per SM.
-//
-// Thread (half, row), half = warp / 4, owns keys 64*half .. 64*half+63 of
-// every tile with its own running max m_half and sum l_half -- the two halves
-// of a row are two independent streams of the streaming-softmax rule -- and its
-// own accumulator O_half = sum P[:, half keys] V[half keys, :] in TMEM; the
-// halves are merged once, in the epilogue, with the same rule. V is loaded per
-// half (the 64 rows that half's P V reads). Per tile u:
-//   wait S_full | load its 64 scores (one TMEM round trip) | count in to
-//   "S read" | scale, mask/bias, drop unlisted entries, max | wait O_done_half
-//   (u-1) (its P chunk, V_half buffer and O_half are then free) | if the max
-//   grew by more than 2^8, rescale O_half in TMEM | exp2, sum, P chunk to smem
-//   | count in to "P_half written"
-// No thread waits for the others: the warp whose arrival completes "S read"
-// issues S(u+1) = Q K(u+1)^T (the S columns are free, the scores are in
-// registers) and the TMA of K(u+2) into K(u)'s buffer; the warp completing
-// "P_half written" issues O_half += P V_half and the TMA of V_half(u+1) into
-// V_half(u-1)'s buffer. Arrival counters only grow (tile u completes at 8(u+1)
-// or 4(u+1)).
-//
-// TMEM: S columns [0, 128), O_0 [128, 128 + d), O_1 [128 + d, 128 + 2d).
-constexpr int kWsThreads = 256;
-
-
-template <int D, bool EXTRA>
-__global__ void __launch_bounds__(kWsThreads, 2)
-    k_fwd_tc_ws(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const TcParams P) {
-    // tmV: boxes of 64 rows (one half of a key tile)
-    using C = TcCfg<D>;
-    static_assert(D <= 64, "S plus two O halves must fit 256 TMEM columns");
-    constexpr int DH = D / 2;  // output columns per thread in the epilogue
-    extern __shared__ __align__(1024) uint8_t smem[];
-
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int half = warp >> 2;  // key half of each tile
-    const int row = tid & 127;   // query row in the block == TMEM lane
-    const int bh = blockIdx.x / P.nqb, qb = blockIdx.x - bh * P.nqb;
-    const int b = bh / P.H, h = bh - b * P.H;
-    const int mk = P.num_masks == 1 ? 0 : b;
-    const int64_t blk = (int64_t)mk * P.nqb + qb;
-    int t_begin, T;
-    block_tiles(P, blk, t_begin, T);
-    if (T <= 0) return;
-    const int klim = key_limit_tc(P, b);
-    T = trim_tiles(P, t_begin, T, klim);
-    if (smem_u32(smem) & 1023u) {
-        if (tid == 0) atomicOr(P.err, kErrTimeout);
-        return;
-    }
-
-    const uint32_t sQ = smem_u32(smem + C::OFF_Q);
-    const uint32_t sK0 = smem_u32(smem + C::OFF_K), sV0 = smem_u32(smem + C::OFF_V);
-    const uint32_t sP = smem_u32(smem + C::OFF_P);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-    // barriers: Q, K[2], V[buffer][half], S_full, O_done[half]
-    const uint32_t barQ = smem_u32(bars + 0), barK0 = smem_u32(bars + 1), barV0 = smem_u32(bars + 3),
-                   barSf = smem_u32(bars + 7), barO0 = smem_u32(bars + 8);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    // arrival counters: S read, P_0 written, P_1 written; issue counts per
-    // barrier 1 .. 9 (K[2], V[4], S_full, O_done[2])
-    uint32_t* cnt = tmem_slot + 2;
-    int* issued = reinterpret_cast<int*>(tmem_slot + 5);  // (issuers may differ: atomics)
-    // (m, l) of both halves of every row, [2 halves][2][128]; in the P buffer,
-    // which is free once the last P V is done
-    float* xch = reinterpret_cast<float*>(smem + C::OFF_P);
-
-    if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-    if (tid == 0) {
-        for (int x = 0; x < 10; ++x) mbar_init(smem_u32(bars + x), 1);
-        for (int x = 0; x < 3; ++x) cnt[x] = 0u;
-        for (int x = 0; x < 9; ++x) issued[x] = 0;
-        *abort_flag = 0;
-        fence_mbar_init();
-        prefetch_tensormap(&tmQ);
-        prefetch_tensormap(&tmK);
-        prefetch_tensormap(&tmV);
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tO = tmem + 128;
-    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-
-    auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
-        if (*abort_flag) return false;
-        if (mbar_wait_bounded(bar, parity, kWaitCycles)) return true;
-        *abort_flag = 1;
-        return false;
-    };
-    auto tile_kt = [&](int u) { return P.tile_info[t_begin + u] & 0x7fffffff; };
-    auto issue_k = [&](int u) {
-        const uint32_t bar = barK0 + 8u * (u & 1);
-        mbar_expect_tx(bar, (uint32_t)C::TILE_BYTES);
-        tma_load_4d(sK0 + (uint32_t)((u & 1) * C::TILE_BYTES), &tmK, bar, 0, tile_kt(u) * 128, h, b);
-        atomicAdd(&issued[u & 1], 1);
-    };
-    auto issue_v = [&](int u, int hf) {  // rows 64 hf .. 64 hf + 63 of V tile u
-        const uint32_t bar = barV0 + 8u * ((u & 1) * 2 + hf);
-        mbar_expect_tx(bar, (uint32_t)(C::TILE_BYTES / 2));
-        tma_load_4d(sV0 + (uint32_t)((u & 1) * C::TILE_BYTES + hf * 64 * C::ROW_BYTES), &tmV, bar, 0,
-                    tile_kt(u) * 128 + hf * 64, h, b);
-        atomicAdd(&issued[2 + (u & 1) * 2 + hf], 1);
-    };
-    auto issue_S = [&](int u) {
-        const uint32_t idS = idesc_bf16_f32(128, 128, false);
-        const uint32_t sK = sK0 + (uint32_t)((u & 1) * C::TILE_BYTES);
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-            const uint64_t da = smem_desc(sQ + ks * 32, 16, C::SBO, C::LAYOUT);
-            const uint64_t db = smem_desc(sK + ks * 32, 16, C::SBO, C::LAYOUT);
-            mma_bf16_ss(tS, da, db, idS, ks > 0 ? 1u : 0u);
-        }
-        mma_commit(barSf);
-        atomicAdd(&issued[6], 1);
-    };
-    auto issue_PV = [&](int u, int hf) {  // O_hf (+)= P[:, 64 hf ..] V[64 hf .., :]
-        const uint32_t idO = idesc_bf16_f32(128, D, true);
-        const uint32_t sV = sV0 + (uint32_t)((u & 1) * C::TILE_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t da = smem_desc(sP + (uint32_t)(hf * 16384 + kk * 32), 16, 1024,
-                                          cute::UMMA::LayoutType::SWIZZLE_128B);
-            const uint64_t db = smem_desc(sV + (uint32_t)((hf * 4 + kk) * 16 * C::ROW_BYTES), C::CHUNK_BYTES,
-                                          C::SBO, C::LAYOUT);
-            mma_bf16_ss(tO + (uint32_t)(hf * D), da, db, idO, (u > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(barO0 + 8u * hf);
-        atomicAdd(&issued[7 + hf], 1);
-    };
-
-    if (tid == 0) {
-        mbar_expect_tx(barQ, (uint32_t)C::TILE_BYTES);
-        tma_load_4d(sQ, &tmQ, barQ, 0, qb * 128, h, b);
-        issue_k(0);
-        issue_v(0, 0);
-        issue_v(0, 1);
-        if (T > 1) {
-            issue_k(1);
-            issue_v(1, 0);
-            issue_v(1, 1);
-        }
-        if (wait(barQ, 0) && wait(barK0, 0)) {
-            tc_fence_after();
-            issue_S(0);
-        }
-    }
-
-    const int i = qb * 128 + row;
-    const bool row_ok = i < P.n;
-    const int64_t mask_rowbase = (int64_t)b * P.mask.s0 + (int64_t)h * P.mask.s1 + (int64_t)i * P.mask.s2;
-    const int64_t bias_rowbase = (int64_t)b * P.bias.s0 + (int64_t)h * P.bias.s1 + (int64_t)i * P.bias.s2;
-    float m_ref = -INFINITY, l = 0.f;  // this half's running max (reference) and sum
-    int rlo = 0, rhi = 0;               // interval masks: the row's run
-    if (P.itv_lohi && row_ok) {
-        const int2 v = P.itv_lohi[(int64_t)mk * P.n + i];
-        rlo = v.x;
-        rhi = v.y;
-    }
-    int next_info = P.tile_info[t_begin];
-    uint2 next_bits = make_uint2(0u, 0u);  // stored bits, loaded one tile ahead
-    if (next_info >= 0 && row_ok && !P.itv_lohi)
-        next_bits = tile_row_bits2(P, t_begin, next_info, row, half, rlo, rhi);
-    const uint64_t c2 = pack2(P.qk_scale_log2, P.qk_scale_log2);
-    const uint32_t tOh = tO + lane_base + (uint32_t)(half * D);
-
-    for (int u = 0; u < T; ++u) {
-        const int info = next_info;
-        const uint2 wbits = next_bits;
-        if (u + 1 < T) {
-            next_info = P.tile_info[t_begin + u + 1];
-            if (next_info >= 0 && row_ok && !P.itv_lohi)
-                next_bits = tile_row_bits2(P, t_begin + u + 1, next_info, row, half, rlo, rhi);
-        }
-        const int kt = info & 0x7fffffff;
-        const bool dense = info < 0;
-
-        float x[64];
-        wait(barSf, (uint32_t)(u & 1));
-        tc_fence_after();
-        __syncwarp();
-        {
-            uint32_t r0[32], r1[32];
-            tmem_ld32(tS + lane_base + half * 64, r0);
-            tmem_ld32(tS + lane_base + half * 64 + 32, r1);
-            tmem_wait_ld_dep(r0);
-            tmem_wait_ld_dep(r1);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                mul2(x[2 * k], x[2 * k + 1], r0[2 * k], r0[2 * k + 1], c2);
-                mul2(x[32 + 2 * k], x[33 + 2 * k], r1[2 * k], r1[2 * k + 1], c2);
-            }
-        }
-        if (arrive_last(cnt + 0, 8u * (u + 1) - 1u) && !*abort_flag) {
-            // every row has read S(u): S(u+1) may overwrite it; K(u)'s buffer is free
-            if (u + 1 < T && wait(barK0 + 8u * ((u + 1) & 1), (uint32_t)(((u + 1) >> 1) & 1))) {
-                tc_fence_after();
-                issue_S(u + 1);
-            }
-            if (u + 2 < T) issue_k(u + 2);
-        }
-        if (EXTRA && row_ok) {  // + log2(e) * (mask + bias)
-            const int c0 = kt * 128 + half * 64;
-            const int ncols = P.n - c0 < 64 ? P.n - c0 : 64;
-            if (P.mask.data) add_addend_run<64>(P.mask, mask_rowbase, c0, ncols, x);
-            if (P.bias.data) add_addend_run<64>(P.bias, bias_rowbase, c0, ncols, x);
-        }
-        const int lim = klim - kt * 128 - half * 64;  // keys of this tile half that exist
-        if (!dense || lim < 64) {  // entries the mask does not list, or padding
-            uint2 wb = dense ? make_uint2(~0u, ~0u)
-                             : (P.itv_lohi ? tile_row_bits2(P, 0, info, row, half, rlo, rhi) : wbits);
-            if (lim < 64) {
-                wb.x &= run_word(0, lim, 0);
-                wb.y &= run_word(0, lim, 32);
-            }
-            const uint32_t bw[2] = {wb.x, wb.y};
-#pragma unroll
-            for (int j = 0; j < 64; ++j) x[j] = ((bw[j >> 5] >> (j & 31)) & 1u) ? x[j] : -INFINITY;
-        }
-        float ma = -INFINITY, mb = -INFINITY, mc = -INFINITY, md = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            ma = fmax3(ma, x[8 * k + 0], x[8 * k + 1]);
-            mb = fmax3(mb, x[8 * k + 2], x[8 * k + 3]);
-            mc = fmax3(mc, x[8 * k + 4], x[8 * k + 5]);
-            md = fmax3(md, x[8 * k + 6], x[8 * k + 7]);
-        }
-        const float mx = fmax3(ma, mb, fmaxf(mc, md));
-        const bool need = mx > m_ref + kRescaleThreshold;
-        float alpha = 1.f;
-        if (need) {
-            alpha = ex2(m_ref - mx);
-            m_ref = mx;
-            l *= alpha;
-        }
-        if (u > 0) {  // P V(u-1) of this half is done: its P chunk and O_half are free
-            wait(barO0 + 8u * half, (uint32_t)((u - 1) & 1));
-            tc_fence_after();
-            __syncwarp();
-            if (__any_sync(0xffffffffu, need)) {  // bring O_half to the new reference
-#pragma unroll
-                for (int c = 0; c < D; c += 16) {
-                    uint32_t ro[16];
-                    tmem_ld16(tOh + c, ro);
-                    tmem_wait_ld_dep16(ro);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) ro[j] = __float_as_uint(__uint_as_float(ro[j]) * alpha);
-                    tmem_st16(tOh + c, ro);
-                }
-                tmem_wait_st();
-            }
-        }
-        const float mu = m_ref == -INFINITY ? 0.f : m_ref;
-        const uint64_t nmu2 = pack2(-mu, -mu);
-        uint64_t sa = pack2(0.f, 0.f), sb = sa;
-#pragma unroll
-        for (int piece = 0; piece < 8; ++piece) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const int k = piece * 4 + t;
-                float p0, p1;
-                unpack2(add2(pack2(x[2 * k], x[2 * k + 1]), nmu2), p0, p1);
-                p0 = ex2(p0);
-                p1 = ex2(p1);
-                if (k & 1)
-                    sb = add2(sb, pack2(p0, p1));
-                else
-                    sa = add2(sa, pack2(p0, p1));
-                __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
-                pk[t] = *reinterpret_cast<uint32_t*>(&hv);
-            }
-            const uint32_t addr = sP + (uint32_t)(half * 16384 + row * 128 + ((piece ^ (row & 7)) << 4));
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[0]), "r"(pk[1]),
-                         "r"(pk[2]), "r"(pk[3])
-                         : "memory");
-        }
-        {
-            float s0, s1, s2, s3;
-            unpack2(sa, s0, s1);
-            unpack2(sb, s2, s3);
-            l += (s0 + s1) + (s2 + s3);
-        }
-        fence_proxy_async_smem();
-        if (arrive_last(cnt + 1 + half, 4u * (u + 1) - 1u) && !*abort_flag) {
-            // this half's P(u) is complete, and (every warp of the half waited for
-            // it) so is its P V(u-1): V_half(u-1)'s buffer is free
-            if (wait(barV0 + 8u * ((u & 1) * 2 + half), (uint32_t)((u >> 1) & 1))) {
-                tc_fence_after();
-                issue_PV(u, half);
-            }
-            if (u >= 1 && u + 1 < T) issue_v(u + 1, half);
-        }
-    }
-
-    // ------------------------------------------------------------ epilogue
-    // this half's last P V is done (then P is no longer read); after the barrier
-    // so is the other half's. Exchange (m, l) with the partner thread.
-    wait(barO0 + 8u * half, (uint32_t)((T - 1) & 1));
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    xch[(half * 2 + 0) * 128 + row] = m_ref;
-    xch[(half * 2 + 1) * 128 + row] = l;
-    __syncthreads();
-    const float m_o = xch[((half ^ 1) * 2 + 0) * 128 + row];
-    const float l_o = xch[((half ^ 1) * 2 + 1) * 128 + row];
-    const float m0 = half == 0 ? m_ref : m_o, l0 = half == 0 ? l : l_o;
-    const float m1 = half == 0 ? m_o : m_ref, l1 = half == 0 ? l_o : l;
-    const int64_t mrow = (int64_t)mk * P.n + i;
-    const int64_t wrow = (int64_t)bh * P.n + i;
-    const bool mixed = row_ok && has_partial(P, blk, mrow, wrow);
-    const float mg = mixed ? P.ws_ml[wrow * 2] : -INFINITY;
-    const float lg = mixed ? P.ws_ml[wrow * 2 + 1] : 0.f;
-    const float M = fmaxf(fmaxf(m0, m1), mg);
-    const float Mu = M == -INFINITY ? 0.f : M;
-    const float f0 = ex2(m0 - Mu), f1 = ex2(m1 - Mu), fg = mixed ? ex2(mg - Mu) : 0.f;
-    const float L = l0 * f0 + l1 * f1 + lg * fg;
-    // this thread writes output columns half*DH .. half*DH + DH - 1 of its row:
-    // o = O_0 f0 + O_1 f1, 16 columns per TMEM load
-    float o[DH];
-#pragma unroll
-    for (int c = 0; c < DH; c += 16) {
-        uint32_t ro[16];
-        tmem_ld16(tO + lane_base + (uint32_t)(half * DH + c), ro);
-        tmem_wait_ld_dep16(ro);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) o[c + j] = __uint_as_float(ro[j]) * f0;
-        tmem_ld16(tO + lane_base + (uint32_t)(D + half * DH + c), ro);
-        tmem_wait_ld_dep16(ro);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) o[c + j] = fmaf(__uint_as_float(ro[j]), f1, o[c + j]);
-    }
-    if (row_ok && !*abort_flag) {
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(P.out) + (int64_t)b * P.o_sb +
-                              (int64_t)h * P.o_sh + (int64_t)i * P.o_sn + half * DH;
-        const float* acc = mixed ? P.ws_acc + wrow * D + half * DH : nullptr;
-#pragma unroll
-        for (int e8 = 0; e8 < DH / 8; ++e8) {
-            float v[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                float val = o[e8 * 8 + t];
-                if (mixed) val = fmaf(acc[e8 * 8 + t], fg, val);
-                v[t] = val * inv;
-            }
-            uint32_t w[4];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                __nv_bfloat162 hv = __floats2bfloat162_rn(v[2 * t], v[2 * t + 1]);
-                w[t] = *reinterpret_cast<uint32_t*>(&hv);
-            }
-            *reinterpret_cast<uint4*>(orow + e8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        if (P.lse && half == 0) P.lse[wrow] = L > 0.f ? (M + lg2(L)) * kLn2 : -INFINITY;
-    }
-
-    // ------------------------------------------------------------ teardown
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0 && *abort_flag) {  // drain what was issued (bounded), then report
-        const long long lim = kWaitCycles / 16;
-        for (int x = 0; x < 9; ++x)  // barrier x + 1: K[2], V[4], S_full, O_done[2]
-            if (issued[x]) mbar_wait_bounded(smem_u32(bars + 1 + x), (uint32_t)((issued[x] - 1) & 1), lim);
-        atomicOr(P.err, kErrTimeout);
-    }
-    __syncthreads();
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
-    }
-}
-
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
@@ -1405,10 +1062,10 @@ cudaError_t launch_tc_t(const TcOperand& q, const TcOperand& k, const TcOperand&
     std::call_once(once, []() {
         constexpr int DP = D <= 64 ? D : 64;
         if (D <= 64) {
-            attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_ws<DP, true>,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+            attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_quad<DP, true>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, QuadCfg<DP>::SMEM_BYTES);
             if (attr_err == cudaSuccess)
-                attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_quad<DP>,
+                attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_quad<DP, false>,
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 QuadCfg<DP>::SMEM_BYTES);
         } else {
@@ -1420,18 +1077,19 @@ cudaError_t launch_tc_t(const TcOperand& q, const TcOperand& k, const TcOperand&
     CUtensorMap mq, mk, mv;
     cudaError_t e;
     if ((e = make_map(&mq, q, p.B, p.H, p.n, D, C::CHUNK_ELEMS)) != cudaSuccess) return e;
-    // d <= 64: k_fwd_tc_quad loads K and V in 64-row sub-tiles, the kernel for
-    // mask/bias addends V in halves of 64 rows
-    const bool quad = D <= 64 && !p.has_extra;
-    if ((e = make_map(&mk, k, p.B, p.H, p.n, D, C::CHUNK_ELEMS, quad ? 64 : 128)) != cudaSuccess) return e;
-    if ((e = make_map(&mv, v, p.B, p.H, p.n, D, C::CHUNK_ELEMS, D <= 64 ? 64 : 128)) != cudaSuccess) return e;
+    // d <= 64: k_fwd_tc_quad loads K and V in 64-row sub-tiles
+    const int kv_rows = D <= 64 ? 64 : 128;
+    if ((e = make_map(&mk, k, p.B, p.H, p.n, D, C::CHUNK_ELEMS, kv_rows)) != cudaSuccess) return e;
+    if ((e = make_map(&mv, v, p.B, p.H, p.n, D, C::CHUNK_ELEMS, kv_rows)) != cudaSuccess) return e;
     const int64_t grid = (int64_t)p.B * p.H * p.nqb;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     constexpr int DP = D <= 64 ? D : 64;
     if (D <= 64 && p.has_extra) {
-        k_fwd_tc_ws<DP, true><<<(unsigned)grid, kWsThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, p);
+        k_fwd_tc_quad<DP, true><<<(unsigned)grid, kQuadThreads, QuadCfg<DP>::SMEM_BYTES, counted(s)>>>(mq, mk, mv,
+                                                                                                     p);
     } else if (D <= 64) {
-        k_fwd_tc_quad<DP><<<(unsigned)grid, kQuadThreads, QuadCfg<DP>::SMEM_BYTES, counted(s)>>>(mq, mk, mv, p);
+        k_fwd_tc_quad<DP, false><<<(unsigned)grid, kQuadThreads, QuadCfg<DP>::SMEM_BYTES, counted(s)>>>(mq, mk, mv,
+                                                                                                      p);
     } else
         k_fwd_tc<D><<<(unsigned)grid, kThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, p);
     return cudaGetLastError();

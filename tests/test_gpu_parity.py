@@ -143,6 +143,27 @@ def test_odd_lengths_with_mask_and_bias(dtype, d, n):
     _check_raw(B, H, n, d, dtype, rp, ci, B, mask, bias, seed=n + d, what=f"n={n} d={d}")
 
 
+@pytest.mark.parametrize("d", [32, 64])
+@pytest.mark.parametrize("layout", ["row_mask", "bias_only", "pad_mask_and_bias", "row_mask_and_bias",
+                                    "f32_bias"])
+def test_tile_addend_layouts(d, layout):
+    """The tensor-core kernel takes one addend that varies by row from registers
+    fetched a tile ahead (bf16, unit column stride, aligned rows) and loads the
+    other when it is used; every combination must give the same result."""
+    rng = np.random.default_rng(7 + d)
+    B, H, n = 2, 3, 256
+    rp, ci = _rand_csr(rng, n, 1, 0.6)
+    row_mask = workloads.make_tensor(np.where(rng.random((B, 1, n, n)) < 0.1, -np.inf,
+                                              rng.standard_normal((B, 1, n, n))), workloads.BF16)
+    pad_mask = workloads.make_tensor(np.where(rng.random((B, 1, 1, n)) < 0.2, -np.inf, 0.0), workloads.BF16)
+    bias = workloads.make_tensor(rng.standard_normal((1, H, n, n)), workloads.BF16)
+    bias32 = workloads.make_tensor(rng.standard_normal((1, H, n, n)), workloads.F32)
+    mask, b = {"row_mask": (row_mask, None), "bias_only": (None, bias),
+               "pad_mask_and_bias": (pad_mask, bias), "row_mask_and_bias": (row_mask, bias),
+               "f32_bias": (pad_mask, bias32)}[layout]
+    _check_raw(B, H, n, d, workloads.BF16, rp, ci, 1, mask, b, seed=d, what=f"{layout} d={d}")
+
+
 def test_empty_and_fully_masked_rows():
     rng = np.random.default_rng(1)
     B, H, n, d = 2, 2, 96, 64
