@@ -233,6 +233,92 @@ __device__ __forceinline__ bool arrive_last(uint32_t* counter, uint32_t last) {
     return win;
 }
 
+// Writes row i of the output from its state (m, l, o) (log2 units, O not yet
+// divided by l), first merging the gather kernel's partial when the row has
+// one; lse = (m + log2 l) ln 2.
+template <int D>
+__device__ __forceinline__ void tc_write_row(const TcParams& P, int b, int h, int64_t bh, int mk, int64_t blk,
+                                             int i, float m, float l, const float (&o)[D]) {
+    if (i >= P.n) return;
+    float M = m, L = l, fa = 1.f, fg = 0.f;
+    const int64_t mrow = (int64_t)mk * P.n + i;
+    const int64_t wrow = bh * P.n + i;
+    const bool mixed = has_partial(P, blk, mrow, wrow);
+    if (mixed) {
+        const float mg = P.ws_ml[wrow * 2], lg = P.ws_ml[wrow * 2 + 1];
+        M = fmaxf(m, mg);
+        const float Mu = M == -INFINITY ? 0.f : M;
+        fa = ex2(m - Mu);
+        fg = ex2(mg - Mu);
+        L = l * fa + lg * fg;
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(P.out) + (int64_t)b * P.o_sb + (int64_t)h * P.o_sh +
+                          (int64_t)i * P.o_sn;
+    const float* acc = mixed ? P.ws_acc + wrow * D : nullptr;
+#pragma unroll
+    for (int e8 = 0; e8 < D / 8; ++e8) {
+        float v[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            float val = o[e8 * 8 + t] * fa;
+            if (mixed) val = fmaf(acc[e8 * 8 + t], fg, val);
+            v[t] = val * inv;
+        }
+        uint32_t w[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            __nv_bfloat162 hv = __floats2bfloat162_rn(v[2 * t], v[2 * t + 1]);
+            w[t] = *reinterpret_cast<uint32_t*>(&hv);
+        }
+        *reinterpret_cast<uint4*>(orow + e8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    if (P.lse) P.lse[wrow] = L > 0.f ? (M + lg2(L)) * kLn2 : -INFINITY;
+}
+
+// A query block whose tile list is split into chunks (one thread block each):
+// the chunk's partial state (m, l, O) of every row goes to its slot in
+// P.cws ([slot][d + 2][128 rows], so each warp's stores are coalesced); the
+// thread block whose arrival completes the block's count merges all chunks
+// with the running max / sum rule and returns true with the merged state in
+// (m, l, o); the others return false. flag: one int of shared memory.
+template <int D>
+__device__ bool chunk_merge(const TcParams& P, int64_t bh, int64_t blk, int chunk, int nch, int row, float& m,
+                            float& l, float (&o)[D], volatile int* flag) {
+    const int64_t slot0 = (bh * P.n_slots + P.blk_slot[blk]) * (int64_t)(D + 2);
+    float* mine = P.cws + (slot0 + (int64_t)chunk * (D + 2)) * 128 + row;
+    mine[0] = m;
+    mine[128] = l;
+#pragma unroll
+    for (int j = 0; j < D; ++j) mine[(int64_t)(2 + j) * 128] = o[j];
+    __threadfence();
+    __syncthreads();
+    if (row == 0) {
+        const int64_t nblk = (int64_t)P.num_masks * P.nqb;
+        *flag = atomicAdd(P.ccnt + bh * nblk + blk, 1u) == (unsigned)(nch - 1);
+    }
+    __syncthreads();
+    if (!*flag) return false;
+    __threadfence();
+    float M = -INFINITY, L = 0.f;
+#pragma unroll
+    for (int j = 0; j < D; ++j) o[j] = 0.f;
+    for (int c = 0; c < nch; ++c) {
+        const float* pp = P.cws + (slot0 + (int64_t)c * (D + 2)) * 128 + row;
+        const float mc = __ldcg(pp), lc = __ldcg(pp + 128);
+        if (!(lc > 0.f)) continue;
+        const float Mn = fmaxf(M, mc);
+        const float fa = ex2(M - Mn), fb = ex2(mc - Mn);
+#pragma unroll
+        for (int j = 0; j < D; ++j) o[j] = fmaf(__ldcg(pp + (int64_t)(2 + j) * 128), fb, o[j] * fa);
+        L = L * fa + lc * fb;
+        M = Mn;
+    }
+    m = M;
+    l = L;
+    return true;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     k_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -241,7 +327,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ __align__(1024) uint8_t smem[];
 
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int bh = blockIdx.x / P.nqb, qb = blockIdx.x - bh * P.nqb;
+    // thread blocks [0, B*H*nqb) take query block (bh, qb) -- its first chunk
+    // when it is split --; the rest take the further chunks P.chunk_extra lists
+    const int64_t nbase = (int64_t)P.B * P.H * P.nqb;
+    int bh, qb, chunk = 0;
+    if ((int64_t)blockIdx.x < nbase) {
+        bh = (int)(blockIdx.x / P.nqb);
+        qb = (int)(blockIdx.x - (int64_t)bh * P.nqb);
+    } else {
+        const int64_t e = (int64_t)blockIdx.x - nbase;
+        bh = (int)(e / P.n_extra);
+        const int2 x = P.chunk_extra[e - (int64_t)bh * P.n_extra];
+        if (P.num_masks > 1 && x.x / P.nqb != bh / P.H) return;  // a chunk of another batch element's mask
+        qb = x.x % P.nqb;
+        chunk = x.y;
+    }
     const int b = bh / P.H, h = bh - b * P.H;
     const int mk = P.num_masks == 1 ? 0 : b;
     const int64_t blk = (int64_t)mk * P.nqb + qb;
@@ -250,6 +350,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (T <= 0) return;
     const int klim = key_limit_tc(P, b);
     T = trim_tiles(P, t_begin, T, klim);  // whole CTA: the gather kernel owns this block
+    const int nch = P.blk_nch ? P.blk_nch[blk] : 1;
+    if (nch > 1) {  // this chunk's tiles (none when the key length cut them all)
+        t_begin += chunk * P.chunk_tiles;
+        T -= chunk * P.chunk_tiles;
+        T = T < P.chunk_tiles ? T : P.chunk_tiles;
+    }
     if (smem_u32(smem) & 1023u) {  // the swizzled layouts need a 1024-byte aligned base
         if (tid == 0) atomicOr(P.err, kErrTimeout);
         return;
@@ -263,6 +369,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                    barO = smem_u32(bars + 4);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* chunk_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+    float o[D];
+    if (T <= 0) {  // an empty chunk still counts in, with an empty partial
+        float m0 = -INFINITY, l0 = 0.f;
+#pragma unroll
+        for (int j = 0; j < D; ++j) o[j] = 0.f;
+        if (chunk_merge<D>(P, bh, blk, chunk, nch, tid, m0, l0, o, chunk_flag))
+            tc_write_row<D>(P, b, h, bh, mk, blk, qb * 128 + tid, m0, l0, o);
+        return;
+    }
 
     if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     if (tid == 0) {
@@ -531,7 +648,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     wait(barO, (uint32_t)((T - 1) & 1));
     tc_fence_after();
     __syncwarp();
-    float o[D];
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
         uint32_t ro[32];
@@ -540,43 +656,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 32; ++j) o[c * 32 + j] = __uint_as_float(ro[j]);
     }
-    if (row_ok && !*abort_flag) {
-        float M = m_ref, L = l, fa = 1.f;
-        const int64_t mrow = (int64_t)mk * P.n + i;
-        const int64_t wrow = (int64_t)bh * P.n + i;
-        const bool mixed = has_partial(P, blk, mrow, wrow);
-        float mg = -INFINITY, lg = 0.f, fg = 0.f;
-        if (mixed) {
-            mg = P.ws_ml[wrow * 2];
-            lg = P.ws_ml[wrow * 2 + 1];
-            M = fmaxf(m_ref, mg);
-            const float Mu = M == -INFINITY ? 0.f : M;
-            fa = ex2(m_ref - Mu);
-            fg = ex2(mg - Mu);
-            L = l * fa + lg * fg;
-        }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(P.out) + (int64_t)b * P.o_sb +
-                              (int64_t)h * P.o_sh + (int64_t)i * P.o_sn;
-        const float* acc = mixed ? P.ws_acc + wrow * D : nullptr;
-#pragma unroll
-        for (int e8 = 0; e8 < D / 8; ++e8) {
-            float v[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                float val = o[e8 * 8 + t] * fa;
-                if (mixed) val = fmaf(acc[e8 * 8 + t], fg, val);
-                v[t] = val * inv;
-            }
-            uint32_t w[4];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                __nv_bfloat162 hv = __floats2bfloat162_rn(v[2 * t], v[2 * t + 1]);
-                w[t] = *reinterpret_cast<uint32_t*>(&hv);
-            }
-            *reinterpret_cast<uint4*>(orow + e8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        if (P.lse) P.lse[wrow] = L > 0.f ? (M + lg2(L)) * kLn2 : -INFINITY;
+    {
+        float M = m_ref, L = l;
+        __syncthreads();  // every wait is behind us: the abort flag is final and the same for all
+        bool write = !*abort_flag;
+        if (nch > 1 && write) write = chunk_merge<D>(P, bh, blk, chunk, nch, tid, M, L, o, chunk_flag);
+        if (write) tc_write_row<D>(P, b, h, bh, mk, blk, i, M, L, o);
     }
 
     // ------------------------------------------------------------ teardown
@@ -1090,8 +1175,12 @@ cudaError_t launch_tc_t(const TcOperand& q, const TcOperand& k, const TcOperand&
     } else if (D <= 64) {
         k_fwd_tc_quad<DP, false><<<(unsigned)grid, kQuadThreads, QuadCfg<DP>::SMEM_BYTES, counted(s)>>>(mq, mk, mv,
                                                                                                       p);
-    } else
-        k_fwd_tc<D><<<(unsigned)grid, kThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, p);
+    } else {
+        // one thread block per query block, plus one per further chunk of split blocks
+        const int64_t grid2 = grid + (p.blk_nch ? (int64_t)p.B * p.H * p.n_extra : 0);
+        if (grid2 > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+        k_fwd_tc<D><<<(unsigned)grid2, kThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, p);
+    }
     return cudaGetLastError();
 }
 

@@ -53,6 +53,13 @@ struct spattn_mask_s {
     void* block_csr;   // row_ptr, long_rows
     void* block_col;   // col_idx
     void* block_plan;  // block_tile_off, tile_info, tile_bits, res_row_ptr, res_col_idx, res_long
+    // query blocks with more than kChunkTiles tiles, split into chunks for the
+    // d = 128 tile kernel (see TcParams); block_chunk holds the three arrays
+    void* block_chunk;
+    int32_t* blk_nch;
+    int32_t* blk_slot;
+    int2* chunk_extra;
+    int32_t n_extra, n_slots;
     // Implicit interval masks (SLIDING, VARWIN, DENSE): per-row runs and the
     // tile map are what the forward pass reads; row_ptr / col_idx and the
     // explicit plan arrays above are written only when asked for.
@@ -308,7 +315,11 @@ int launch_fwd(FwdParams& p, int dtype, int d, int num_sms, cudaStream_t s) {
 
 void free_plan(spattn_mask m) {
     if (m->block_plan) cudaFreeAsync(m->block_plan, m->stream);
-    m->block_plan = nullptr;
+    if (m->block_chunk) cudaFreeAsync(m->block_chunk, m->stream);
+    m->block_plan = m->block_chunk = nullptr;
+    m->blk_nch = m->blk_slot = nullptr;
+    m->chunk_extra = nullptr;
+    m->n_extra = m->n_slots = 0;
     m->block_tile_off = m->tile_info = m->res_row_ptr = m->res_col_idx = m->res_long = nullptr;
     m->tile_bits = nullptr;
     m->has_plan = false;
@@ -602,6 +613,56 @@ int write_plan(spattn_mask m) {
 }
 
 
+// Splits the query blocks of a CSR mask's tile plan that have more than
+// kChunkTiles tiles into chunks of that many, so that one long block (rows
+// that attend to every key, say) does not serialise the d = 128 tile kernel:
+// per block its chunk count and first partial-state slot, and the list of
+// (block, chunk >= 1) the extra thread blocks take. Synchronises the mask's
+// stream (it runs right after the plan is built, which already does).
+int write_chunks(spattn_mask m, cudaMemPool_t pool) {
+    const int64_t nblocks = (int64_t)m->num_masks * m->nqb;
+    std::vector<int32_t> off((size_t)nblocks + 1);
+    cudaStream_t s = m->stream;
+    CUDA_TRY(cudaMemcpyAsync(off.data(), m->block_tile_off, off.size() * 4, cudaMemcpyDeviceToHost, s),
+             "plan read-back");
+    CUDA_TRY(cudaStreamSynchronize(s), "plan read-back");
+    std::vector<int32_t> nch((size_t)nblocks, 1), slot((size_t)nblocks, -1), extra;
+    int64_t n_slots = 0;
+    for (int64_t x = 0; x < nblocks; ++x) {
+        const int64_t T = off[x + 1] - off[x];
+        if (T <= kChunkTiles) continue;
+        nch[x] = (int32_t)((T + kChunkTiles - 1) / kChunkTiles);
+        slot[x] = (int32_t)n_slots;
+        n_slots += nch[x];
+        for (int32_t c = 1; c < nch[x]; ++c) {
+            extra.push_back((int32_t)x);
+            extra.push_back(c);
+        }
+    }
+    if (n_slots == 0) return SPATTN_OK;
+    Carve cp;
+    const int k_n = cp.add(nblocks * 4), k_s = cp.add(nblocks * 4), k_e = cp.add(extra.size() * 4);
+    void* a = nullptr;
+    CUDA_TRY(cudaMallocFromPoolAsync(&a, cp.total, pool, s), "chunk plan allocation");
+    cudaError_t e = cudaMemcpyAsync(cp.at<int32_t>(a, k_n), nch.data(), nblocks * 4, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(cp.at<int32_t>(a, k_s), slot.data(), nblocks * 4, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(cp.at<int32_t>(a, k_e), extra.data(), extra.size() * 4, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);  // the host vectors go out of scope
+    if (e != cudaSuccess) {
+        cudaFreeAsync(a, s);
+        return cuda_fail(e, "chunk plan upload");
+    }
+    m->block_chunk = a;
+    m->blk_nch = cp.at<int32_t>(a, k_n);
+    m->blk_slot = cp.at<int32_t>(a, k_s);
+    m->chunk_extra = cp.at<int2>(a, k_e);
+    m->n_extra = (int32_t)(extra.size() / 2);
+    m->n_slots = (int32_t)n_slots;
+    return SPATTN_OK;
+}
+
 // The tensor-core kernel over the mask's tiles; blk_res: interval masks whose
 // gather kernel ran (its partial states are in p.ws_ml / p.ws_acc).
 int launch_tc(const FwdParams& p, int d, spattn_mask m, int dev, const int32_t* blk_res,
@@ -641,9 +702,32 @@ int launch_tc(const FwdParams& p, int d, spattn_mask m, int dev, const int32_t* 
     tp.qk_scale_log2 = p.qk_scale_log2;
     tp.seqlen_k = p.seqlen_k;
     tp.err = ef;
+    void* cws = nullptr;  // partial states and arrival counts of split query blocks
+    if (d == 128 && !m->implicit && m->blk_nch) {
+        cudaMemPool_t pool;
+        CUDA_TRY(device_state(dev, &pool, nullptr), "memory pool");
+        const int64_t bh = (int64_t)p.B * p.H, nblocks = (int64_t)m->num_masks * m->nqb;
+        Carve cp;
+        const int k_w = cp.add((size_t)bh * m->n_slots * (d + 2) * kTileM * 4), k_c = cp.add(bh * nblocks * 4);
+        CUDA_TRY(cudaMallocFromPoolAsync(&cws, cp.total, pool, s), "chunk workspace");
+        cudaError_t e = cudaMemsetAsync(cp.at<unsigned>(cws, k_c), 0, bh * nblocks * 4, s);
+        if (e != cudaSuccess) {
+            cudaFreeAsync(cws, s);
+            return cuda_fail(e, "chunk workspace");
+        }
+        tp.blk_nch = m->blk_nch;
+        tp.blk_slot = m->blk_slot;
+        tp.chunk_extra = m->chunk_extra;
+        tp.n_extra = m->n_extra;
+        tp.n_slots = m->n_slots;
+        tp.chunk_tiles = kChunkTiles;
+        tp.cws = cp.at<float>(cws, k_w);
+        tp.ccnt = cp.at<unsigned>(cws, k_c);
+    }
     const TcOperand oq{p.q, p.q_sn, p.q_sh, p.q_sb}, ok{p.k, p.k_sn, p.k_sh, p.k_sb},
         ov{p.v, p.v_sn, p.v_sh, p.v_sb};
     const cudaError_t e = launch_fwd_tc(oq, ok, ov, d, tp, s);
+    if (cws) cudaFreeAsync(cws, s);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core kernel launch");
     return SPATTN_OK;
 }
@@ -902,6 +986,11 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
         m->res_n_long = hpc.res_n_long;
         m->has_plan = hpc.n_tiles > 0;
         if (!m->has_plan) free_plan(m);
+        int r = m->has_plan ? write_chunks(m, pool) : SPATTN_OK;
+        if (r) {
+            spattn_destroy_mask(m);
+            return r;
+        }
     }
     *out = m;
     return SPATTN_OK;

@@ -19,6 +19,9 @@ constexpr int kTileM = 128;
 constexpr int kTileN = 128;
 constexpr unsigned kTileDenseBit = 0x80000000u;  // tile_info flag: all 128 x 128 entries present
 constexpr int kTileMinNnzDefault = 512;
+// The d = 128 tile kernel splits a query block with more tiles than this into
+// chunks of this many, one thread block each.
+constexpr int kChunkTiles = 8;
 // Tile planning is skipped when num_masks * (n/128)^2 exceeds this (count array size).
 constexpr int64_t kPlanZeroInline = 1 << 18;  // words the single-launch build clears
 constexpr int64_t kPlanMaxTileGrid = int64_t(1) << 26;
@@ -128,6 +131,18 @@ struct TcParams {
     const int32_t* blk_res;
     const float* ws_ml;             // partials from the gather kernel, or nullptr
     const float* ws_acc;
+    // Query blocks whose tile lists are split into chunks of chunk_tiles tiles
+    // (d = 128; nullptr blk_nch: none): block x has blk_nch[x] chunks, whose
+    // partial states take slots blk_slot[x] + c of the n_slots of each (b, h)
+    // in cws; chunks c >= 1 run on extra thread blocks, one per entry of
+    // chunk_extra ((block, c); n_extra per (b, h)); ccnt[bh * blocks + x]
+    // counts the chunks done (zero before the launch).
+    const int32_t* blk_nch;
+    const int32_t* blk_slot;
+    const int2* chunk_extra;
+    int n_extra, n_slots, chunk_tiles;
+    float* cws;
+    unsigned* ccnt;
     void* out;
     int64_t o_sb, o_sh, o_sn;
     float* lse;

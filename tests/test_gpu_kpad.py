@@ -62,6 +62,17 @@ def test_evoformer_with_lengths_and_bias():
         _check(wl.q, wl.k, wl.v, rp, ci, 1, wl.n, wl.d, wl.dtype, lengths, m, bias=wl.bias, what="evoformer")
 
 
+def test_split_query_block_with_lengths():
+    """d = 128, block + strided + global: query block 0's tile list is split into
+    chunks; with 500 keys the second chunk has no tile left and only hands an
+    empty partial state to the merge."""
+    wl = workloads.make(3, B=2, H=2, n=2048)
+    rp, ci = oracle.mask_from_params(wl.mask)
+    with build_mask(wl.mask) as m:
+        _check(wl.q, wl.k, wl.v, rp, ci, wl.mask.num_masks, wl.n, wl.d, wl.dtype, [500, 1900], m,
+               what="bsg d=128")
+
+
 @pytest.mark.parametrize("thr", [0, 9000])
 def test_variable_window_with_lengths(thr):
     wl = workloads.make(1, B=3, H=2, n=900)

@@ -87,6 +87,24 @@ def test_fused_forward_matches_oracle(cfg):
     assert sp.spattn_device_error() == 0
 
 
+@pytest.mark.parametrize("n", [1100, 2048])
+def test_split_query_block_d128(n):
+    """Query block 0 of the block + strided + global mask lists every key tile
+    (its global rows attend to all keys); the d = 128 tile kernel splits such a
+    block into chunks of eight tiles, one thread block each, and merges their
+    partial states (n = 1100: chunks of 8 and 1 tiles)."""
+    wl = workloads.make(3, B=1, H=2, n=n)
+    q, k, v, am, bias = device_inputs(wl)
+    rp_ref, ci_ref = _oracle_csr(wl.mask)
+    out_ref, lse_ref = _run_oracle(wl, rp_ref, ci_ref)
+    with build_mask(wl.mask) as m:
+        out, lse = sp.spattn_fwd_mask(q, k, v, m, scale=wl.scale)
+        torch.cuda.synchronize()
+    assert_close(to_f64(out).reshape(-1, wl.d), to_f64(lse), out_ref.reshape(-1, wl.d),
+                 lse_ref.reshape(-1), wl.dtype, f"split block n={n}")
+    assert sp.spattn_device_error() == 0
+
+
 # ------------------------------------------------------------------ edge cases
 def _rand_csr(rng, n, num_masks, p, empty=(), dup=False):
     rows, rp = [], [0]
