@@ -182,6 +182,18 @@ def test_tile_addend_layouts(d, layout):
     _check_raw(B, H, n, d, workloads.BF16, rp, ci, 1, mask, b, seed=d, what=f"{layout} d={d}")
 
 
+@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("scale", [-0.2, 0.0, 0.3])
+def test_tile_scale_sign(d, scale):
+    """The tensor-core kernels keep raw scores until the exponent when the scale
+    is positive; a negative or zero scale takes the scaled-scores path. Both must
+    follow the definition (a zero scale gives every listed entry the same weight)."""
+    rng = np.random.default_rng(11 + d)
+    B, H, n = 1, 2, 256
+    rp, ci = _rand_csr(rng, n, 1, 0.5)
+    _check_raw(B, H, n, d, workloads.BF16, rp, ci, 1, scale=scale, seed=d, what=f"scale={scale} d={d}")
+
+
 def test_empty_and_fully_masked_rows():
     rng = np.random.default_rng(1)
     B, H, n, d = 2, 2, 96, 64
