@@ -60,6 +60,11 @@ struct spattn_mask_s {
     int32_t* blk_slot;
     int2* chunk_extra;
     int32_t n_extra, n_slots;
+    // block + strided + global masks with strided entries outside the plan's
+    // tiles: those entries as a mask of their own in residue-permuted order
+    // (str_mask), the rest as a regular mask (reg_mask); see strided.cu
+    spattn_mask str_mask, reg_mask;
+    int32_t str_stride;
     // Implicit interval masks (SLIDING, VARWIN, DENSE): per-row runs and the
     // tile map are what the forward pass reads; row_ptr / col_idx and the
     // explicit plan arrays above are written only when asked for.
@@ -663,6 +668,127 @@ int write_chunks(spattn_mask m, cudaMemPool_t pool) {
     return SPATTN_OK;
 }
 
+// Moves the strided entries (j = i mod S) that a block + strided + global
+// mask's tile plan leaves to the gather kernel into a mask of their own in
+// residue-permuted order, whose plan covers them with dense tiles, and keeps
+// the rest as a regular mask (both built like user CSR masks, with the same
+// tile threshold). Synchronises the mask's stream.
+int write_strided(spattn_mask m, int S, int32_t tile_min_nnz, cudaMemPool_t pool) {
+    cudaStream_t s = m->stream;
+    const int n = m->n;
+    const int64_t rows = (int64_t)m->num_masks * n;
+    const int nkt = (n + kTileN - 1) / kTileN;
+    const int64_t nblocks = (int64_t)m->num_masks * m->nqb;
+    Carve ct;
+    const int k_cp = ct.add(rows * 4), k_cr = ct.add(rows * 4), k_cg = ct.add(rows * 4),
+              k_sp = ct.add((rows + 1) * 4), k_gp = ct.add((rows + 1) * 4), k_sel = ct.add(nblocks * nkt),
+              k_st = ct.add(scan_tmp_elems(rows) * 8), k_tot = ct.add(2 * 8), k_err = ct.add(4);
+    void* t = nullptr;
+    CUDA_TRY(cudaMallocFromPoolAsync(&t, ct.total, pool, s), "strided split scratch");
+    int32_t *cnt_perm = ct.at<int32_t>(t, k_cp), *cnt_row = ct.at<int32_t>(t, k_cr),
+            *cnt_reg = ct.at<int32_t>(t, k_cg), *srp = ct.at<int32_t>(t, k_sp), *grp = ct.at<int32_t>(t, k_gp);
+    int64_t* tot = ct.at<int64_t>(t, k_tot);
+    unsigned* err = ct.at<unsigned>(t, k_err);
+    int64_t htot[2] = {0, 0};
+    int32_t *sci = nullptr, *gci = nullptr;
+    cudaError_t e = cudaMemsetAsync(err, 0, 4, s);
+    if (e == cudaSuccess)
+        e = strided_split_count(m->res_row_ptr, m->res_col_idx, rows, n, S, cnt_perm, cnt_row, s);
+    if (e == cudaSuccess) e = scan_counts(cnt_perm, rows, srp, ct.at<int64_t>(t, k_st), tot, err, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&htot[0], tot, 8, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess && htot[0] > 0) {
+        e = cudaMallocFromPoolAsync(&sci, (size_t)htot[0] * 4, pool, s);
+        if (e == cudaSuccess)
+            e = strided_split_fill(m->res_row_ptr, m->res_col_idx, m->row_ptr, m->col_idx, m->block_tile_off,
+                                   m->tile_info, rows, n, S, m->nqb, nkt, nblocks, cnt_row, cnt_reg,
+                                   ct.at<uint8_t>(t, k_sel), srp, sci, s);
+        if (e == cudaSuccess) e = scan_counts(cnt_reg, rows, grp, ct.at<int64_t>(t, k_st), tot + 1, err, s);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(&htot[1], tot + 1, 8, cudaMemcpyDeviceToHost, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&gci, (size_t)(htot[1] > 0 ? htot[1] : 1) * 4, pool, s);
+        if (e == cudaSuccess)
+            e = strided_reg_fill(m->row_ptr, m->col_idx, rows, n, S, m->nqb, nkt, ct.at<uint8_t>(t, k_sel), grp,
+                                 gci, s);
+    }
+    int r = SPATTN_OK;
+    if (e != cudaSuccess) {
+        r = cuda_fail(e, "strided split");
+    } else if (htot[0] > 0) {
+        spattn_mask_spec sp;
+        memset(&sp, 0, sizeof sp);
+        sp.kind = SPATTN_MASK_CSR;
+        sp.n = n;
+        sp.num_masks = m->num_masks;
+        sp.tile_min_nnz = tile_min_nnz;
+        sp.in_row_ptr = srp;
+        sp.in_col_idx = sci;
+        sp.in_nnz = htot[0];
+        r = spattn_create_csr_mask(&sp, s, &m->str_mask);
+        if (!r) {
+            sp.in_row_ptr = grp;
+            sp.in_col_idx = gci;
+            sp.in_nnz = htot[1];
+            r = spattn_create_csr_mask(&sp, s, &m->reg_mask);
+        }
+        if (!r && !(m->str_mask->has_plan && m->reg_mask->has_plan)) {  // nothing to gain: keep the mask as is
+            spattn_destroy_mask(m->str_mask);
+            spattn_destroy_mask(m->reg_mask);
+            m->str_mask = m->reg_mask = nullptr;
+        }
+        if (!r && m->str_mask) m->str_stride = S;
+    }
+    if (sci) cudaFreeAsync(sci, s);
+    if (gci) cudaFreeAsync(gci, s);
+    cudaFreeAsync(t, s);
+    return r;
+}
+
+// Forward over a mask split by write_strided: the permuted part over Q, K, V
+// with rows permuted, the regular part over them as they are, then each row
+// merged through the two log-sum-exps.
+int fwd_strided(const spattn_tensor* q, const spattn_tensor* k, const spattn_tensor* v, spattn_mask m,
+                float scale, const spattn_tensor* out, float* lse, cudaStream_t s, const FwdParams& p, int d,
+                cudaMemPool_t pool) {
+    const int B = p.B, H = p.H, n = p.n, S = m->str_stride;
+    const int64_t rows = (int64_t)B * H * n, elems = rows * d;
+    Carve c;
+    const int k_q = c.add(elems * 2), k_k = c.add(elems * 2), k_v = c.add(elems * 2), k_o = c.add(elems * 2),
+              k_l2 = c.add(rows * 4), k_l1 = c.add(rows * 4);
+    void* t = nullptr;
+    CUDA_TRY(cudaMallocFromPoolAsync(&t, c.total, pool, s), "strided forward scratch");
+    auto tensor = [&](int key) {  // contiguous [B, H, n, d] bf16 scratch
+        spattn_tensor x;
+        memset(&x, 0, sizeof x);
+        x.data = c.at<uint8_t>(t, key);
+        x.dtype = SPATTN_BF16;
+        x.shape[0] = B;
+        x.shape[1] = H;
+        x.shape[2] = n;
+        x.shape[3] = d;
+        x.stride[0] = (int64_t)H * n * d;
+        x.stride[1] = (int64_t)n * d;
+        x.stride[2] = d;
+        x.stride[3] = 1;
+        return x;
+    };
+    const spattn_tensor tq = tensor(k_q), tk = tensor(k_k), tv = tensor(k_v), to = tensor(k_o);
+    float* l2 = c.at<float>(t, k_l2);
+    float* l1 = lse ? lse : c.at<float>(t, k_l1);
+    cudaError_t e = strided_permute_rows(p.q, p.q_sb, p.q_sh, p.q_sn, tq.data, B, H, n, d, S, s);
+    if (e == cudaSuccess) e = strided_permute_rows(p.k, p.k_sb, p.k_sh, p.k_sn, tk.data, B, H, n, d, S, s);
+    if (e == cudaSuccess) e = strided_permute_rows(p.v, p.v_sb, p.v_sh, p.v_sn, tv.data, B, H, n, d, S, s);
+    int r = e == cudaSuccess ? SPATTN_OK : cuda_fail(e, "strided forward (permute)");
+    if (!r) r = spattn_fwd_mask(&tq, &tk, &tv, m->str_mask, nullptr, nullptr, scale, &to, l2, s);
+    if (!r) r = spattn_fwd_mask(q, k, v, m->reg_mask, nullptr, nullptr, scale, out, l1, s);
+    if (!r) {
+        e = strided_merge(p.out, p.o_sb, p.o_sh, p.o_sn, l1, to.data, l2, lse, B, H, n, d, S, s);
+        if (e != cudaSuccess) r = cuda_fail(e, "strided forward (merge)");
+    }
+    cudaFreeAsync(t, s);
+    return r;
+}
+
 // The tensor-core kernel over the mask's tiles; blk_res: interval masks whose
 // gather kernel ran (its partial states are in p.ws_ml / p.ws_acc).
 int launch_tc(const FwdParams& p, int d, spattn_mask m, int dev, const int32_t* blk_res,
@@ -987,6 +1113,9 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
         m->has_plan = hpc.n_tiles > 0;
         if (!m->has_plan) free_plan(m);
         int r = m->has_plan ? write_chunks(m, pool) : SPATTN_OK;
+        if (!r && m->has_plan && m->res_nnz > 0 && sp.kind == SPATTN_MASK_BLOCK_STRIDED_GLOBAL &&
+            sp.stride >= 2 && sp.n % sp.stride == 0)
+            r = write_strided(m, sp.stride, sp.tile_min_nnz, pool);
         if (r) {
             spattn_destroy_mask(m);
             return r;
@@ -1085,6 +1214,8 @@ int spattn_destroy_mask(spattn_mask m) {
     if (m->block_csr && (e2 = cudaFreeAsync(m->block_csr, m->stream)) != cudaSuccess) e = e2;
     if (m->block_col && (e2 = cudaFreeAsync(m->block_col, m->stream)) != cudaSuccess) e = e2;
     free_plan(m);
+    if (m->str_mask) spattn_destroy_mask(m->str_mask);
+    if (m->reg_mask) spattn_destroy_mask(m->reg_mask);
     if (m->block_itv && (e2 = cudaFreeAsync(m->block_itv, m->stream)) != cudaSuccess) e = e2;
     if (m->block_t && (e2 = cudaFreeAsync(m->block_t, m->stream)) != cudaSuccess) e = e2;
     if (m->cnt_host) {
@@ -1175,6 +1306,8 @@ int spattn_fwd_mask_kpad(const spattn_tensor* q, const spattn_tensor* k, const s
     p.num_masks = mask->num_masks;
     p.long_count_dev = nullptr;
     if (mask->implicit) return fwd_interval(p, dtype, d, mask, s, pool, dev, sms);
+    if (mask->str_mask && dtype == 0 && !seqlen_k && !p.has_extra)
+        return fwd_strided(q, k, v, mask, scale, out, lse, s, p, d, pool);
     if (!(mask->has_plan && dtype == 0)) {  // every entry on the gather kernel
         p.row_ptr = mask->row_ptr;
         p.col_idx = mask->col_idx;

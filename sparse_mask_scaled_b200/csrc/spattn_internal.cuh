@@ -314,4 +314,30 @@ cudaError_t build_transpose(const int32_t* row_ptr, const int32_t* col_idx, int 
                             int64_t nnz, int32_t* t_row_ptr, int32_t* t_col_idx, int32_t* scratch,
                             cudaStream_t stream);
 
+// Strided entries of a block + strided + global mask (strided.cu). perm(i) =
+// (i mod S) n/S + i div S; n is a multiple of S.
+// Per residual row, its entries j = i (mod S): counted at the row's permuted
+// position (cnt_perm, [rows]) and at its own (cnt_row).
+cudaError_t strided_split_count(const int32_t* res_row_ptr, const int32_t* res_col_idx, int64_t rows, int n,
+                                int S, int32_t* cnt_perm, int32_t* cnt_row, cudaStream_t s);
+// Writes those entries in permuted order (columns perm(j)) at str_row_ptr, and
+// the regular part's row lengths (the mask's rows minus them) to cnt_reg; sel:
+// [nblocks * nkt] bytes of scratch (the plan's tiles).
+cudaError_t strided_split_fill(const int32_t* res_row_ptr, const int32_t* res_col_idx, const int32_t* row_ptr,
+                               const int32_t* col_idx, const int32_t* block_tile_off, const int32_t* tile_info,
+                               int64_t rows, int n, int S, int nqb, int nkt, int64_t nblocks,
+                               const int32_t* cnt_row, int32_t* cnt_reg, uint8_t* sel,
+                               const int32_t* str_row_ptr, int32_t* str_col_idx, cudaStream_t s);
+// The regular part: every entry of the mask but those moved to the permuted one.
+cudaError_t strided_reg_fill(const int32_t* row_ptr, const int32_t* col_idx, int64_t rows, int n, int S, int nqb,
+                             int nkt, const uint8_t* sel, const int32_t* reg_row_ptr, int32_t* reg_col_idx,
+                             cudaStream_t s);
+// dst (contiguous [B, H, n, d] bf16) row perm(i) = src (strides in elements) row i.
+cudaError_t strided_permute_rows(const void* src, int64_t s_b, int64_t s_h, int64_t s_n, void* dst, int B, int H,
+                                 int n, int d, int S, cudaStream_t s);
+// out / lse (nullable) of each row from the regular part's (out, lse1) and the
+// permuted part's (o2, lse2) at the row's permuted position.
+cudaError_t strided_merge(void* out, int64_t o_sb, int64_t o_sh, int64_t o_sn, const float* lse1, const void* o2,
+                          const float* lse2, float* lse, int B, int H, int n, int d, int S, cudaStream_t s);
+
 }  // namespace spattn
