@@ -146,6 +146,14 @@ typedef struct spattn_mask_s* spattn_mask;
  * bit 0 is raised (see spattn_device_error) -- and the size queries below wait
  * for the build. Memory comes from the library's stream-ordered pool and is
  * released by spattn_destroy_mask.
+ * A BLOCK_STRIDED_GLOBAL mask whose n is a multiple of `stride` also keeps the
+ * strided entries that fall outside its tensor-core tiles as a second mask in
+ * residue-permuted order (token i at (i mod stride) n/stride + i div stride),
+ * where they form dense tiles, plus the remaining entries as a third. That is
+ * two more CSR builds (and syncs) and about the CSR's size again in memory.
+ * spattn_fwd_mask uses them for bf16 inputs without additive terms; the results
+ * are the same within rounding (each part's output is rounded to bf16 once
+ * before the two are merged).
  * Errors: INVALID_ARG (bad kind, parameters or flags), BAD_CSR (CSR not
  * sorted/unique, a column outside [0, n), row_ptr not a valid prefix sum, or a
  * negative half-width), UNSUPPORTED (more than 2^31 - 1 nonzeros, or a COO row
