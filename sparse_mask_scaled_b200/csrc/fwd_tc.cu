@@ -414,8 +414,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_expect_tx(bar, 2u * C::TILE_BYTES);
 #pragma unroll
         for (int c = 0; c < C::NCHUNK; ++c) {
-            tma_load_4d(dK + c * C::CHUNK_BYTES, &tmK, bar, c * C::CHUNK_ELEMS, kt * 128, h, b);
-            tma_load_4d(dV + c * C::CHUNK_BYTES, &tmV, bar, c * C::CHUNK_ELEMS, kt * 128, h, b);
+            if (P.perm_G) {  // keys kt*128 .. in permuted order: residue r, positions k0 .. k0 + 127
+                const int r = kt * 128 / P.perm_G, k0 = kt * 128 - r * P.perm_G;
+                tma_load_5d(dK + c * C::CHUNK_BYTES, &tmK, bar, c * C::CHUNK_ELEMS, r, k0, h, b);
+                tma_load_5d(dV + c * C::CHUNK_BYTES, &tmV, bar, c * C::CHUNK_ELEMS, r, k0, h, b);
+            } else {
+                tma_load_4d(dK + c * C::CHUNK_BYTES, &tmK, bar, c * C::CHUNK_ELEMS, kt * 128, h, b);
+                tma_load_4d(dV + c * C::CHUNK_BYTES, &tmV, bar, c * C::CHUNK_ELEMS, kt * 128, h, b);
+            }
         }
         ++n_kv_issued;
     };
@@ -452,7 +458,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_expect_tx(barQ, (uint32_t)C::TILE_BYTES);
 #pragma unroll
         for (int c = 0; c < C::NCHUNK; ++c)
-            tma_load_4d(sQ + c * C::CHUNK_BYTES, &tmQ, barQ, c * C::CHUNK_ELEMS, qb * 128, h, b);
+            if (P.perm_G) {
+                const int r = qb * 128 / P.perm_G, k0 = qb * 128 - r * P.perm_G;
+                tma_load_5d(sQ + c * C::CHUNK_BYTES, &tmQ, barQ, c * C::CHUNK_ELEMS, r, k0, h, b);
+            } else {
+                tma_load_4d(sQ + c * C::CHUNK_BYTES, &tmQ, barQ, c * C::CHUNK_ELEMS, qb * 128, h, b);
+            }
         issue_kv(0);
         if (T > 1) issue_kv(1);
         if (wait(barQ, 0) && wait(barKV0, 0)) {
@@ -1138,6 +1149,28 @@ cudaError_t make_map(CUtensorMap* map, const TcOperand& t, int B, int H, int n, 
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// 5-D map over a [B, H, n, d] bf16 tensor read in residue-permuted order:
+// dims {d, S, G, H, B} (row i = k S + r at (r, k)), box {chunk, 1, 128, 1, 1}:
+// one load brings rows r, r + S, ..., r + 127 S.
+cudaError_t make_perm_map(CUtensorMap* map, const TcOperand& t, int B, int H, int n, int d, int chunk, int G) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const int S = n / G;
+    const uint64_t sn = (uint64_t)t.s_n * 2;
+    const uint64_t sh = H > 1 ? (uint64_t)t.s_h * 2 : sn * (uint64_t)n;
+    const uint64_t sb = B > 1 ? (uint64_t)t.s_b * 2 : sh * (uint64_t)H;
+    cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)S, (cuuint64_t)G, (cuuint64_t)H, (cuuint64_t)B};
+    cuuint64_t strides[4] = {sn, sn * (uint64_t)S, sh, sb};
+    cuuint32_t box[5] = {(cuuint32_t)chunk, 1, 128, 1, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    const CUtensorMapSwizzle sw =
+        chunk * 2 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(t.data), dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int D>
 cudaError_t launch_tc_t(const TcOperand& q, const TcOperand& k, const TcOperand& v, const TcParams& p,
                         cudaStream_t s) {
@@ -1161,6 +1194,16 @@ cudaError_t launch_tc_t(const TcOperand& q, const TcOperand& k, const TcOperand&
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap mq, mk, mv;
     cudaError_t e;
+    if (p.perm_G) {  // d = 128 only (k_fwd_tc), every load a permuted 128-row box
+        if (D != 128 || p.perm_G % 128 != 0 || p.n % p.perm_G != 0) return cudaErrorInvalidValue;
+        if ((e = make_perm_map(&mq, q, p.B, p.H, p.n, D, C::CHUNK_ELEMS, p.perm_G)) != cudaSuccess) return e;
+        if ((e = make_perm_map(&mk, k, p.B, p.H, p.n, D, C::CHUNK_ELEMS, p.perm_G)) != cudaSuccess) return e;
+        if ((e = make_perm_map(&mv, v, p.B, p.H, p.n, D, C::CHUNK_ELEMS, p.perm_G)) != cudaSuccess) return e;
+        const int64_t grid = (int64_t)p.B * p.H * p.nqb + (p.blk_nch ? (int64_t)p.B * p.H * p.n_extra : 0);
+        if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+        k_fwd_tc<D><<<(unsigned)grid, kThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, p);
+        return cudaGetLastError();
+    }
     if ((e = make_map(&mq, q, p.B, p.H, p.n, D, C::CHUNK_ELEMS)) != cudaSuccess) return e;
     // d <= 64: k_fwd_tc_quad loads K and V in 64-row sub-tiles
     const int kv_rows = D <= 64 ? 64 : 128;

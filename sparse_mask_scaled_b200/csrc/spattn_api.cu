@@ -744,17 +744,27 @@ int write_strided(spattn_mask m, int S, int32_t tile_min_nnz, cudaMemPool_t pool
     return r;
 }
 
-// Forward over a mask split by write_strided: the permuted part over Q, K, V
-// with rows permuted, the regular part over them as they are, then each row
-// merged through the two log-sum-exps.
+// The tensor-core kernel over a mask's tiles (below); perm_G: see TcParams.
+int launch_tc(const FwdParams& p, int d, spattn_mask m, int dev, const int32_t* blk_res, cudaStream_t s,
+              int perm_G = 0);
+
+// Forward over a mask split by write_strided: the permuted part, then the
+// regular part over Q, K, V as they are, then each row merged through the two
+// log-sum-exps. For d = 128 with n/S a multiple of 128 and every permuted entry
+// in a tile, the tile kernel reads the permuted rows of Q, K and V in place
+// (five-dimensional maps, stride S); otherwise they are copied in permuted
+// order first.
 int fwd_strided(const spattn_tensor* q, const spattn_tensor* k, const spattn_tensor* v, spattn_mask m,
                 float scale, const spattn_tensor* out, float* lse, cudaStream_t s, const FwdParams& p, int d,
-                cudaMemPool_t pool) {
-    const int B = p.B, H = p.H, n = p.n, S = m->str_stride;
+                cudaMemPool_t pool, int dev) {
+    const int B = p.B, H = p.H, n = p.n, S = m->str_stride, G = n / S;
     const int64_t rows = (int64_t)B * H * n, elems = rows * d;
+    const spattn_mask sm = m->str_mask;
+    const bool in_place = d == 128 && G % kTileM == 0 && sm->has_plan && sm->res_nnz == 0 && sm->n_tiles > 0;
     Carve c;
-    const int k_q = c.add(elems * 2), k_k = c.add(elems * 2), k_v = c.add(elems * 2), k_o = c.add(elems * 2),
-              k_l2 = c.add(rows * 4), k_l1 = c.add(rows * 4);
+    const int k_o = c.add(elems * 2), k_l2 = c.add(rows * 4), k_l1 = c.add(rows * 4),
+              k_q = c.add(in_place ? 0 : elems * 2), k_k = c.add(in_place ? 0 : elems * 2),
+              k_v = c.add(in_place ? 0 : elems * 2);
     void* t = nullptr;
     CUDA_TRY(cudaMallocFromPoolAsync(&t, c.total, pool, s), "strided forward scratch");
     auto tensor = [&](int key) {  // contiguous [B, H, n, d] bf16 scratch
@@ -772,17 +782,30 @@ int fwd_strided(const spattn_tensor* q, const spattn_tensor* k, const spattn_ten
         x.stride[3] = 1;
         return x;
     };
-    const spattn_tensor tq = tensor(k_q), tk = tensor(k_k), tv = tensor(k_v), to = tensor(k_o);
+    const spattn_tensor to = tensor(k_o);
     float* l2 = c.at<float>(t, k_l2);
     float* l1 = lse ? lse : c.at<float>(t, k_l1);
-    cudaError_t e = strided_permute_rows(p.q, p.q_sb, p.q_sh, p.q_sn, tq.data, B, H, n, d, S, s);
-    if (e == cudaSuccess) e = strided_permute_rows(p.k, p.k_sb, p.k_sh, p.k_sn, tk.data, B, H, n, d, S, s);
-    if (e == cudaSuccess) e = strided_permute_rows(p.v, p.v_sb, p.v_sh, p.v_sn, tv.data, B, H, n, d, S, s);
-    int r = e == cudaSuccess ? SPATTN_OK : cuda_fail(e, "strided forward (permute)");
-    if (!r) r = spattn_fwd_mask(&tq, &tk, &tv, m->str_mask, nullptr, nullptr, scale, &to, l2, s);
+    int r = SPATTN_OK;
+    if (in_place) {
+        FwdParams p2 = p;
+        p2.out = to.data;
+        p2.o_sb = to.stride[0];
+        p2.o_sh = to.stride[1];
+        p2.o_sn = to.stride[2];
+        p2.lse = l2;
+        p2.ws_ml = p2.ws_acc = nullptr;
+        r = launch_tc(p2, d, sm, dev, nullptr, s, G);
+    } else {
+        const spattn_tensor tq = tensor(k_q), tk = tensor(k_k), tv = tensor(k_v);
+        cudaError_t e = strided_permute_rows(p.q, p.q_sb, p.q_sh, p.q_sn, tq.data, B, H, n, d, S, s);
+        if (e == cudaSuccess) e = strided_permute_rows(p.k, p.k_sb, p.k_sh, p.k_sn, tk.data, B, H, n, d, S, s);
+        if (e == cudaSuccess) e = strided_permute_rows(p.v, p.v_sb, p.v_sh, p.v_sn, tv.data, B, H, n, d, S, s);
+        r = e == cudaSuccess ? SPATTN_OK : cuda_fail(e, "strided forward (permute)");
+        if (!r) r = spattn_fwd_mask(&tq, &tk, &tv, sm, nullptr, nullptr, scale, &to, l2, s);
+    }
     if (!r) r = spattn_fwd_mask(q, k, v, m->reg_mask, nullptr, nullptr, scale, out, l1, s);
     if (!r) {
-        e = strided_merge(p.out, p.o_sb, p.o_sh, p.o_sn, l1, to.data, l2, lse, B, H, n, d, S, s);
+        const cudaError_t e = strided_merge(p.out, p.o_sb, p.o_sh, p.o_sn, l1, to.data, l2, lse, B, H, n, d, S, s);
         if (e != cudaSuccess) r = cuda_fail(e, "strided forward (merge)");
     }
     cudaFreeAsync(t, s);
@@ -792,7 +815,7 @@ int fwd_strided(const spattn_tensor* q, const spattn_tensor* k, const spattn_ten
 // The tensor-core kernel over the mask's tiles; blk_res: interval masks whose
 // gather kernel ran (its partial states are in p.ws_ml / p.ws_acc).
 int launch_tc(const FwdParams& p, int d, spattn_mask m, int dev, const int32_t* blk_res,
-              cudaStream_t s) {
+              cudaStream_t s, int perm_G) {
     unsigned* ef = nullptr;
     int r = err_flags_ptr(dev, &ef);
     if (r) return r;
@@ -828,6 +851,7 @@ int launch_tc(const FwdParams& p, int d, spattn_mask m, int dev, const int32_t* 
     tp.qk_scale_log2 = p.qk_scale_log2;
     tp.seqlen_k = p.seqlen_k;
     tp.err = ef;
+    tp.perm_G = perm_G;
     void* cws = nullptr;  // partial states and arrival counts of split query blocks
     if (d == 128 && !m->implicit && m->blk_nch) {
         cudaMemPool_t pool;
@@ -1307,7 +1331,7 @@ int spattn_fwd_mask_kpad(const spattn_tensor* q, const spattn_tensor* k, const s
     p.long_count_dev = nullptr;
     if (mask->implicit) return fwd_interval(p, dtype, d, mask, s, pool, dev, sms);
     if (mask->str_mask && dtype == 0 && !seqlen_k && !p.has_extra)
-        return fwd_strided(q, k, v, mask, scale, out, lse, s, p, d, pool);
+        return fwd_strided(q, k, v, mask, scale, out, lse, s, p, d, pool, dev);
     if (!(mask->has_plan && dtype == 0)) {  // every entry on the gather kernel
         p.row_ptr = mask->row_ptr;
         p.col_idx = mask->col_idx;

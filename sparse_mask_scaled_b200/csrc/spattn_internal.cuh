@@ -143,6 +143,11 @@ struct TcParams {
     int n_extra, n_slots, chunk_tiles;
     float* cws;
     unsigned* ccnt;
+    // d = 128 only: rows and keys are numbered in residue-permuted order --
+    // position p = (i mod S) perm_G + i div S holds row / key i of the Q, K, V
+    // tensors (S = n / perm_G, perm_G a multiple of 128) -- and the tile loads
+    // fetch their 128 rows with stride S (five-dimensional maps); 0 = off.
+    int perm_G;
     void* out;
     int64_t o_sb, o_sh, o_sn;
     float* lse;

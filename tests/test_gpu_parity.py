@@ -105,6 +105,27 @@ def test_split_query_block_d128(n):
     assert sp.spattn_device_error() == 0
 
 
+@pytest.mark.parametrize("stride,n", [(64, 8192), (128, 2048)])
+def test_strided_entries_as_permuted_tiles(stride, n):
+    """Block + strided + global masks keep their strided entries as a residue-
+    permuted mask of dense tiles, run as a second tile pass and merged by
+    log-sum-exp. With n / stride a multiple of 128 (stride 64, n = 8192) the
+    d = 128 tile kernel reads the permuted rows in place through five-dimensional
+    maps; otherwise (stride 128, n = 2048) they are copied in permuted order."""
+    import dataclasses
+    wl = workloads.make(3, B=1, H=2, n=n)
+    wl = dataclasses.replace(wl, mask=workloads.MaskParams("bsg", n, 1, block=64, stride=stride, n_global=32))
+    q, k, v, am, bias = device_inputs(wl)
+    rp_ref, ci_ref = _oracle_csr(wl.mask)
+    out_ref, lse_ref = _run_oracle(wl, rp_ref, ci_ref)
+    with build_mask(wl.mask) as m:
+        out, lse = sp.spattn_fwd_mask(q, k, v, m, scale=wl.scale)
+        torch.cuda.synchronize()
+    assert_close(to_f64(out).reshape(-1, wl.d), to_f64(lse), out_ref.reshape(-1, wl.d),
+                 lse_ref.reshape(-1), wl.dtype, f"strided tiles S={stride} n={n}")
+    assert sp.spattn_device_error() == 0
+
+
 # ------------------------------------------------------------------ edge cases
 def _rand_csr(rng, n, num_masks, p, empty=(), dup=False):
     rows, rp = [], [0]
