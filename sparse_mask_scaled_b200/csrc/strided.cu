@@ -88,29 +88,30 @@ __global__ void k_reg_fill(const int32_t* rp, const int32_t* ci, int64_t rows, i
 }
 
 // dst[b, h, perm(i), :] = src[b, h, i, :] (bf16; dst contiguous [B, H, n, d]),
-// one warp per row, 16 bytes per lane and step.
+// one thread per 16-byte chunk (d / 8 consecutive threads per row).
 __global__ void k_perm_rows(const uint4* src, int64_t s_b, int64_t s_h, int64_t s_n, uint4* dst, int H, int n,
                             int d, int S, int G, int64_t rows) {
-    const int64_t w = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
+    const int vec = d / 8;  // 16-byte chunks per row
+    const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    const int64_t w = t / vec;
+    const int c = (int)(t - w * vec);
     if (w >= rows) return;
     const int64_t bh = w / n;
     const int i = (int)(w - bh * n);
     const int64_t b = bh / H, h = bh - b * H;
-    const int vec = d / 8;  // 16-byte chunks per row
-    const uint4* s = src + (b * s_b + h * s_h + (int64_t)i * s_n) / 8;
-    uint4* t = dst + (bh * n + perm_of(i, S, G)) * vec;
-    for (int c = lane; c < vec; c += 32) t[c] = s[c];
+    dst[(bh * n + perm_of(i, S, G)) * vec + c] = src[(b * s_b + h * s_h + (int64_t)i * s_n) / 8 + c];
 }
 
 // out[b, h, i, :] and lse[b, h, i] from the regular part's (out, lse1) and the
 // permuted part's (o2, lse2) at row perm(i): weights exp(lse - L), L their
-// log-sum-exp. One warp per row, 8 elements per lane and step.
+// log-sum-exp. One thread per 8 elements (d / 8 consecutive threads per row).
 __global__ void k_merge_perm(uint4* out, int64_t o_sb, int64_t o_sh, int64_t o_sn, const float* lse1,
                              const uint4* o2, const float* lse2, float* lse, int H, int n, int d, int S, int G,
                              int64_t rows) {
-    const int64_t w = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
+    const int vec = d / 8;
+    const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    const int64_t w = t / vec;
+    const int c = (int)(t - w * vec);
     if (w >= rows) return;
     const int64_t bh = w / n;
     const int i = (int)(w - bh * n);
@@ -126,23 +127,19 @@ __global__ void k_merge_perm(uint4* out, int64_t o_sb, int64_t o_sh, int64_t o_s
         w1 /= tot;
         w2 /= tot;
     }
-    const int vec = d / 8;
-    uint4* orow = out + (b * o_sb + h * o_sh + (int64_t)i * o_sn) / 8;
-    const uint4* prow = o2 + pr * vec;
-    for (int c = lane; c < vec; c += 32) {
-        const uint4 a = orow[c], q = prow[c];
-        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, qw[4] = {q.x, q.y, q.z, q.w};
-        uint32_t rw[4];
+    uint4* op = out + (b * o_sb + h * o_sh + (int64_t)i * o_sn) / 8 + c;
+    const uint4 a = *op, q = o2[pr * vec + c];
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, qw[4] = {q.x, q.y, q.z, q.w};
+    uint32_t rw[4];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            const float lo = __uint_as_float(aw[t] << 16) * w1 + __uint_as_float(qw[t] << 16) * w2;
-            const float hi = __uint_as_float(aw[t] & 0xffff0000u) * w1 + __uint_as_float(qw[t] & 0xffff0000u) * w2;
-            __nv_bfloat162 hv = __floats2bfloat162_rn(lo, hi);
-            rw[t] = *reinterpret_cast<uint32_t*>(&hv);
-        }
-        orow[c] = make_uint4(rw[0], rw[1], rw[2], rw[3]);
+    for (int k = 0; k < 4; ++k) {
+        const float lo = __uint_as_float(aw[k] << 16) * w1 + __uint_as_float(qw[k] << 16) * w2;
+        const float hi = __uint_as_float(aw[k] & 0xffff0000u) * w1 + __uint_as_float(qw[k] & 0xffff0000u) * w2;
+        __nv_bfloat162 hv = __floats2bfloat162_rn(lo, hi);
+        rw[k] = *reinterpret_cast<uint32_t*>(&hv);
     }
-    if (lse && lane == 0) lse[w] = L == -INFINITY ? -INFINITY : L + logf(tot);
+    *op = make_uint4(rw[0], rw[1], rw[2], rw[3]);
+    if (lse && c == 0) lse[w] = L == -INFINITY ? -INFINITY : L + logf(tot);
 }
 
 unsigned blocks_for(int64_t threads, int per) { return (unsigned)((threads + per - 1) / per); }
@@ -180,7 +177,7 @@ cudaError_t strided_permute_rows(const void* src, int64_t s_b, int64_t s_h, int6
                                  int n, int d, int S, cudaStream_t s) {
     const int64_t rows = (int64_t)B * H * n;
     if (rows == 0) return cudaSuccess;
-    k_perm_rows<<<blocks_for(rows * 32, 256), 256, 0, counted(s)>>>(
+    k_perm_rows<<<blocks_for(rows * (d / 8), 256), 256, 0, counted(s)>>>(
         static_cast<const uint4*>(src), s_b, s_h, s_n, static_cast<uint4*>(dst), H, n, d, S, n / S, rows);
     return cudaGetLastError();
 }
@@ -189,7 +186,7 @@ cudaError_t strided_merge(void* out, int64_t o_sb, int64_t o_sh, int64_t o_sn, c
                           const float* lse2, float* lse, int B, int H, int n, int d, int S, cudaStream_t s) {
     const int64_t rows = (int64_t)B * H * n;
     if (rows == 0) return cudaSuccess;
-    k_merge_perm<<<blocks_for(rows * 32, 256), 256, 0, counted(s)>>>(
+    k_merge_perm<<<blocks_for(rows * (d / 8), 256), 256, 0, counted(s)>>>(
         static_cast<uint4*>(out), o_sb, o_sh, o_sn, lse1, static_cast<const uint4*>(o2), lse2, lse, H, n, d, S,
         n / S, rows);
     return cudaGetLastError();
