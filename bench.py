@@ -1,14 +1,15 @@
 #!/usr/bin/env python3
 """Benchmark of sparse-mask scaled dot-product attention on B200.
 
-One step = the whole hot path over one batch of synthetic input: build the CSR
-mask on the device from its pattern parameters (and its row schedule), then the
-fused forward (scores on the mask's nonzeros + additive mask/bias, running
-max/sum softmax, weighted sum of V, normalisation, out + lse).
+One step = the whole hot path over one batch of synthetic input: build the mask
+on the device from its pattern parameters (with its row schedule and tile
+plan), then the fused forward (scores on the mask's nonzeros + additive
+mask/bias, running max/sum softmax, weighted sum of V, normalisation, out +
+lse).
 
-Default workload: variable-window local attention, B=4, H=12, n=4096, d=64,
-bf16 Q/K/V ~ N(0,1), per-token half-width w_i ~ U{32..256} (seeded), one mask
-per batch element shared across heads.
+Default workload: block-local + strided + global tokens, B=1, H=16, n=16384,
+d=128, bf16 Q/K/V ~ N(0, 0.5^2); mask = same 64-token block, j = i (mod 128),
+and the first 32 tokens global (the largest of the five workloads).
 
 Metric: masked-attention TFLOP/s = 4 * nnz * d / step time, nnz summed over
 (b, h). ``--impl reference`` times the fp64 CPU oracle on the host cores instead.
@@ -44,10 +45,12 @@ L2_FLUSH_BYTES = 256 << 20
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, default=1, help="workload index 0..4 (default 1)")
+    ap.add_argument("--config", type=int, default=3, help="workload index 0..4 (default 3)")
+    ap.add_argument("--settle-seconds", type=float, default=1.0,
+                    help="untimed load before the warm-up, so the clock sampler sees the GPU under load")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' forward timings")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
@@ -55,12 +58,18 @@ def parse():
 
 
 def measured_peaks():
+    """(HBM GB/s, dense bf16 TFLOP/s burst, source): the measured copy
+    bandwidth and cuBLAS bf16 GEMM of this machine's B200s, else the fallback."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
         return float(d["hbm_gbs"]), float(d.get("bf16_tflops", 1590.0)), "measured"
     return 6650.0, 1590.0, "fallback"
+
+
+SMS = 148
+MUFU_EX2_PER_CLK_PER_SM = 16   # B200 special-function unit: 4 per SM sub-partition
 
 
 def mask_nnz_total(wl, nnz_per_mask):
@@ -70,10 +79,12 @@ def mask_nnz_total(wl, nnz_per_mask):
     return int(sum(nnz_per_mask)) * wl.H
 
 
-def algorithmic_bytes(wl, nnz_total):
-    """Bytes the method moves per forward: per nonzero a K row and a V row plus
-    the column index (plus one mask and one bias element when present); per
-    query row q_i, out_i, lse_i and its row pointer."""
+def effective_bytes(wl, nnz_total):
+    """The per-nonzero operand bytes of the method (what a gather of every
+    nonzero's rows moves): per nonzero a K row and a V row plus the column
+    index (plus one mask and one bias element when present); per query row q_i,
+    out_i, lse_i and its row pointer. Kernels that reuse rows from L1/L2, or
+    compute whole tiles, move far fewer DRAM bytes than this."""
     es = 2 if wl.dtype == workloads.BF16 else 4
     per_nnz = 2 * wl.d * es + 4
     if wl.add_mask is not None:
@@ -82,6 +93,74 @@ def algorithmic_bytes(wl, nnz_total):
         per_nnz += 2 if wl.bias.dtype == workloads.BF16 else 4
     rows = wl.B * wl.H * wl.n
     return nnz_total * per_nnz + rows * (2 * wl.d * es + 4 + 4), per_nnz
+
+
+def compulsory_bytes(wl, nnz_masks):
+    """Bytes a forward cannot avoid moving through HBM: Q, K, V read and out
+    written once, lse written, the additive mask and bias read once as stored,
+    and the mask as the path stores it (a CSR: row pointers + column indices;
+    an interval mask: one [lo, hi) pair per row; a closed-form pattern:
+    nothing)."""
+    es = 2 if wl.dtype == workloads.BF16 else 4
+    rows = wl.B * wl.H * wl.n
+    b = 4 * rows * wl.d * es + 4 * rows
+    for t in (wl.add_mask, wl.bias):
+        if t is not None:
+            b += t.raw.nbytes
+    mrows = wl.mask.num_masks * wl.n
+    if wl.mask.kind in ("sliding", "varwin", "dense"):
+        b += 8 * mrows
+    elif wl.mask.kind in ("coo", "csr"):
+        b += 4 * (mrows + 1) + 4 * nnz_masks
+    return b
+
+
+def roofline_entry(wl, t_ms, nnz_total, tiles_total, hbm_peak, tc_peak, peak_src, clk_mhz, kernel,
+                   traffic=None, t_warm_ms=None):
+    """Roofline of one forward launch: its algorithmic work (4*nnz*d FLOPs,
+    the compulsory bytes) over the measured time against the measured peaks.
+    ``bound`` follows the arithmetic intensity of that work: below the ridge
+    (peak FLOP/s over peak bytes/s) the forward is bound by HBM, above it by
+    the tensor cores. Beside it, the fractions of each unit the kernels drive:
+    the MMA work executed (whole 128 x 128 tiles, two MMAs each), the exp count
+    on the special-function unit (an upper bound: every element of every tile;
+    the kernels skip 32-key chunks that hold no entry) and, for gathered
+    entries, the per-nonzero effective bytes (served mostly by L2)."""
+    t = t_ms * 1e-3
+    flops = 4.0 * nnz_total * wl.d
+    comp = compulsory_bytes(wl, nnz_total // (wl.B * wl.H if wl.mask.num_masks == 1 else wl.H))
+    eff, per_nnz = effective_bytes(wl, nnz_total)
+    mma = tiles_total * 4.0 * 128 * 128 * wl.d
+    ex2_ub = tiles_total * 128.0 * 128
+    clk = (clk_mhz or 1965.0) * 1e6
+    intensity = flops / comp
+    ridge = tc_peak * 1e12 / (hbm_peak * 1e9)
+    bound = "tensor" if intensity > ridge else "hbm"
+    src = "measured MEASURED_PEAKS.json" if peak_src == "measured" else "fallback"
+    if bound == "tensor":
+        achieved, peak, unit = flops / t / 1e12, tc_peak, "TFLOP/s"
+        psrc = f"bf16_tflops ({src}, burst: the kernel runs for well under a second)"
+    else:
+        achieved, peak, unit = comp / t / 1e9, hbm_peak, "GB/s"
+        psrc = f"hbm_gbs ({src})"
+    e = {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+         "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": kernel,
+         "algorithmic_flop_per_launch": flops, "compulsory_bytes_per_launch": int(comp),
+         "arithmetic_intensity_flop_per_byte": round(intensity, 1), "ridge_flop_per_byte": round(ridge, 1),
+         "fwd_ms": round(t_ms, 4), "peak_source": psrc,
+         "fractions": {
+             "useful_flop_of_bf16_peak": round(flops / t / 1e12 / tc_peak, 4),
+             "executed_mma_of_bf16_peak": round(mma / t / 1e12 / tc_peak, 4),
+             "compulsory_bytes_of_hbm_peak": round(comp / t / 1e9 / hbm_peak, 4),
+             "ex2_upper_bound_of_mufu_peak": round(ex2_ub / t / (SMS * MUFU_EX2_PER_CLK_PER_SM * clk), 4),
+         },
+         "tc_tiles_per_launch": int(tiles_total), "mma_flop_executed_per_launch": mma}
+    if t_warm_ms is not None:
+        e["fwd_ms_warm_l2"] = round(t_warm_ms, 4)
+    if tiles_total == 0:   # every entry gathered: the per-nonzero operand bytes, L2-served
+        e["effective_gbs_l2_served"] = round(eff / t / 1e9, 1)
+        e["effective_bytes_per_nnz"] = per_nnz
+    return e
 
 
 # ---------------------------------------------------------------- clocks
@@ -157,13 +236,20 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- traffic
-def committed_traffic(kernel_src: str, prefix: str, workload: str):
+KERNEL_SOURCES = {"k_fwd_pp": "fwd_pp.cu", "k_fwd_tc": "fwd_tc.cu", "k_fwd_tc_quad": "fwd_tc.cu",
+                  "k_fwd_short": "fwd_gather.cu"}
+
+
+def committed_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary of this kernel and
-    workload, or None when the kernel source changed since the capture."""
-    path = os.path.join(ROOT, "profiles", f"{prefix}_{workload}.md")
-    if not os.path.exists(path):
+    workload (profiles/<kernel base name>_<workload>.md), or None when there is
+    none or the kernel's source changed since the capture."""
+    base = kernel.split("<")[0]
+    path = os.path.join(ROOT, "profiles", f"{base}_{workload}.md")
+    src = KERNEL_SOURCES.get(base)
+    if not src or not os.path.exists(path):
         return None
-    kernel_file = os.path.join(ROOT, "sparse_mask_scaled_b200", "csrc", kernel_src)
+    kernel_file = os.path.join(ROOT, "sparse_mask_scaled_b200", "csrc", src)
     want = hashlib.sha256(open(kernel_file, "rb").read()).hexdigest()[:16]
     vals = {}
     for ln in open(path):
@@ -181,7 +267,7 @@ def committed_traffic(kernel_src: str, prefix: str, workload: str):
 # ---------------------------------------------------------------- CPU side
 def cpu_oracle_rate(wl, seconds: float, threads: int):
     """Time the oracle (as it stands) on a bounded random sample of the
-    workload's rows; returns (TFLOP/s, rows, nnz, elapsed, threads)."""
+    workload's rows; returns (TFLOP/s, rows, nnz, elapsed)."""
     import oracle
     rp, ci = oracle.mask_from_params(wl.mask)
     lens = np.diff(rp)
@@ -265,51 +351,6 @@ class GpuWorkload:
                                        lse=self.lse if lse is None else lse)
 
 
-MUFU_EX2_PER_CLK_PER_SM = 16   # B200 special-function unit: 4 per SM sub-partition
-
-
-def forward_roofline(wl, plan, nnz_total, flops, alg_bytes, per_nnz, t_fwd_ms, hbm_peak, tc_peak, peak_src):
-    """Roofline of the forward's dominant kernel. With a tensor-core plan that
-    kernel is the tcgen05 tile kernel: bound 'tensor', achieved = the metric's
-    algorithmic FLOPs (4 * nnz * d) over the forward time against the measured
-    dense bf16 peak; the MMA FLOPs actually executed (whole 128 x 128 tiles) and
-    the exp2 rate against the special-function-unit peak are reported beside it.
-    Without tiles the gather kernel dominates: bound 'hbm', achieved = the
-    method's bytes (K and V row + column index per nonzero, q/out/lse/row pointer
-    per row) over the forward time against the measured copy bandwidth."""
-    rep = wl.B * wl.H if wl.mask.num_masks == 1 else wl.H
-    dt = "bf16" if wl.dtype == workloads.BF16 else "f32"
-    extra = wl.add_mask is not None or wl.bias is not None
-    t = t_fwd_ms * 1e-3
-    src_peak = "measured MEASURED_PEAKS.json" if peak_src == "measured" else "fallback"
-    if plan["tensor_core_tiles"] > 0 and wl.dtype == workloads.BF16:
-        if wl.d > 64:
-            kname = f"k_fwd_tc<{wl.d}>"
-        else:
-            kname = f"k_fwd_tc_quad<{wl.d},{int(extra)}>"
-        tiles = plan["tensor_core_tiles"] * rep
-        mma_flops = tiles * 2 * (2 * 128 * 128 * wl.d)
-        ex2 = tiles * 128 * 128
-        sms, clk = 148, 1.965e9
-        achieved = flops / t / 1e12
-        return {"bound": "tensor", "achieved": round(achieved, 2), "peak": tc_peak, "unit": "TFLOP/s",
-                "frac": round(achieved / tc_peak, 4),
-                "traffic": committed_traffic("fwd_tc.cu", "tc_fwd", wl.name),
-                "kernel": kname, "algorithmic_flop_per_launch": flops,
-                "mma_flop_executed_per_launch": mma_flops,
-                "mma_tflops_executed": round(mma_flops / t / 1e12, 2),
-                "ex2_per_launch": ex2,
-                "ex2_frac_of_sfu_peak": round(ex2 / t / (sms * MUFU_EX2_PER_CLK_PER_SM * clk), 4),
-                "effective_gbs": round(alg_bytes / t / 1e9, 1),
-                "peak_source": f"bf16_tflops ({src_peak}, burst: the kernel runs for well under a second)"}
-    achieved = alg_bytes / t / 1e9
-    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-            "frac": round(achieved / hbm_peak, 4),
-            "traffic": committed_traffic("fwd_gather.cu", "gather_fwd", wl.name),
-            "kernel": f"k_fwd_short<{dt},{wl.d}>", "algorithmic_bytes_per_launch": alg_bytes,
-            "bytes_per_nnz": per_nnz, "peak_source": f"hbm_gbs ({src_peak})"}
-
-
 def replica_seed(config: int, rank: int) -> int:
     """Each rank runs its own replica of the workload (rank 0: the standard seed)."""
     return 1000 + config + 7919 * rank
@@ -329,6 +370,42 @@ def job_value(world: int, flop_per_step: float, ms_per_step: float) -> float:
     return world * flop_per_step / (ms_per_step * 1e-3) / 1e12
 
 
+def kernel_name(wl, m_tiles):
+    """The forward's dominant kernel for the workload (see the library's source)."""
+    if m_tiles == 0 or wl.dtype != workloads.BF16:
+        return f"k_fwd_short<{'bf16' if wl.dtype == workloads.BF16 else 'f32'},{wl.d}>"
+    extra = wl.add_mask is not None or wl.bias is not None
+    if wl.d in (64, 128) and not extra and wl.mask.kind in ("bsg", "dense", "sliding", "varwin"):
+        return f"k_fwd_pp<{wl.d}>"
+    if wl.d <= 64:
+        return f"k_fwd_tc_quad<{wl.d},{int(extra)}>"
+    return f"k_fwd_tc<{wl.d}>"
+
+
+def time_forward(g, m, torch, flush, reps=20, warm=3):
+    """Median forward time (ms) with L2 flushed before each call, and with L2
+    warm (the same call repeated back to back)."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warm):
+        g.fwd(m)
+
+    def once(do_flush):
+        if do_flush:
+            flush.zero_()
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        g.fwd(m)
+        e.record(stream)
+        return s, e
+
+    cold = [once(True) for _ in range(reps)]
+    hot = [once(False) for _ in range(reps)]
+    torch.cuda.synchronize()
+    return (statistics.median(a.elapsed_time(b) for a, b in cold),
+            statistics.median(a.elapsed_time(b) for a, b in hot))
+
+
 def bench_ours(args, rank, world, torch, sp):
     dev = torch.cuda.current_device()
     wl = workloads.make(args.config, seed=replica_seed(args.config, rank))
@@ -339,13 +416,11 @@ def bench_ours(args, rank, world, torch, sp):
     # mask statistics (same for every step)
     with g.create() as m0:
         nnz_masks = m0.nnz
-        plan = {"tensor_core_tiles": m0.n_tiles, "residual_nnz": m0.residual_nnz,
-                "mixed_rows": m0.n_mixed_rows}
-    # nnz summed over (b, h): every head shares its batch element's mask
-    if wl.mask.num_masks == 1:
-        nnz_total = nnz_masks * wl.B * wl.H
-    else:
-        nnz_total = nnz_masks * wl.H
+        tiles_masks = m0.tc_tiles
+        plan = {"tensor_core_tiles": tiles_masks}
+    rep = wl.B * wl.H if wl.mask.num_masks == 1 else wl.H   # every head shares its batch element's mask
+    nnz_total = nnz_masks * rep
+    tiles_total = tiles_masks * rep
     flops = 4.0 * nnz_total * wl.d
 
     def step():
@@ -361,8 +436,14 @@ def bench_ours(args, rank, world, torch, sp):
     starts, ends, fwd_evs = [], [], []
     smi_id = _smi_id(torch, dev)
     with ClockSampler(smi_id) as clk:
-        clk.mark()       # samples from the warm-up (under the same load) and the timed steps
-        # warm-up right before the timed steps (clocks up, pool and caches warm)
+        clk.mark()
+        # untimed load first, long enough for the sampler to see the clocks
+        # under this work, then the warm-up right before the timed steps
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < args.settle_seconds:
+            for _ in range(20):
+                step()
+            torch.cuda.synchronize()
         for _ in range(args.warmup):
             flush.zero_()
             step()
@@ -393,6 +474,8 @@ def bench_ours(args, rank, world, torch, sp):
     fwd_ms = [a.elapsed_time(b) for a, b in fwd_evs]
     t_total = sum(step_ms)
     t_fwd = sum(fwd_ms) / len(fwd_ms)
+    with g.create() as mw:
+        _, t_warm = time_forward(g, mw, torch, flush)
 
     # ---- end to end: pinned host inputs -> device -> step -> host result
     e2e = e2e_measure(args, g, torch, stream, flush, flops)
@@ -402,29 +485,31 @@ def bench_ours(args, rank, world, torch, sp):
     value = job_value(world, flops, ms_per_step)
     e2e_value = job_value(world, flops, e2e["ms_per_step"])
 
-    alg_bytes, per_nnz = algorithmic_bytes(wl, nnz_total)
     hbm_peak, tc_peak, peak_src = measured_peaks()
-    eff_gbs = alg_bytes / (t_fwd * 1e-3) / 1e9
     clocks = clk.summary()
-    roofline = forward_roofline(wl, plan, nnz_total, flops, alg_bytes, per_nnz, t_fwd, hbm_peak, tc_peak,
-                                peak_src)
+    kname = kernel_name(wl, tiles_total)
+    roofline = roofline_entry(wl, t_fwd, nnz_total, tiles_total, hbm_peak, tc_peak, peak_src,
+                              clocks.get("sm_mhz"), kname, traffic=committed_traffic(kname, wl.name),
+                              t_warm_ms=t_warm)
 
     result = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.dtype == workloads.BF16 else "f32",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if wl.dtype == workloads.BF16 else "f32",
         "data": "synthetic (seeded numpy PCG64; no dataset)",
         "config": {"workload": f"{wl.name} B={wl.B} H={wl.H} n={wl.n} d={wl.d}", "B": wl.B, "H": wl.H,
                    "n": wl.n, "d": wl.d, "mask": wl.mask.kind, "num_masks": wl.mask.num_masks,
                    "nnz_total": nnz_total, "flop_per_step": flops,
                    "l2": "flushed before every timed step (256 MiB write; twice before the first)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "step": "device mask build (pattern -> CSR -> row schedule + tile plan) + fused forward",
+                   "step": "device mask build (pattern -> mask with row schedule and tile plan) + fused forward",
+                   "clocks_window": f"{args.settle_seconds:.1f} s of untimed steps, the warm-up and the timed steps",
                    "plan_per_mask_set": plan},
         "step_ms": {"min": round(min(step_ms), 4), "median": round(statistics.median(step_ms), 4),
                     "max": round(max(step_ms), 4)},
-        "fwd": {"ms": round(t_fwd, 4), "tflops": round(flops / (t_fwd * 1e-3) / 1e12, 3),
-                "effective_gbs": round(eff_gbs, 1)},
+        "fwd": {"ms": round(t_fwd, 4), "ms_warm_l2": round(t_warm, 4),
+                "tflops": round(flops / (t_fwd * 1e-3) / 1e12, 3)},
         "roofline": roofline,
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": round(e2e["ms_per_step"], 4)},
@@ -580,65 +665,50 @@ def fusion_ablation(args, torch, sp):
     return res
 
 
-def other_workloads(torch, sp, skip):
-    """Forward-only timings of the other workloads (device-resident inputs, L2 flushed)."""
+def other_workloads(torch, sp, skip, clk_mhz):
+    """Forward-only timings of the other workloads and the extra dense d = 128
+    case (device-resident inputs; L2 flushed, and warm), each with its roofline."""
     res = {}
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    stream = torch.cuda.current_stream()
-    hbm_peak, _, _ = measured_peaks()
-    for cfg in range(5):
+    hbm_peak, tc_peak, peak_src = measured_peaks()
+    for cfg in range(6):
         if cfg == skip:
             continue
         try:
             wl = workloads.make(cfg)
             g = GpuWorkload(wl, torch, sp)
+            rep = wl.B * wl.H if wl.mask.num_masks == 1 else wl.H
             with g.create() as m:
-                nnz_total = m.nnz * (wl.B * wl.H if wl.mask.num_masks == 1 else wl.H)
-                for _ in range(3):
-                    g.fwd(m)
-                ts = []
-                for _ in range(10):
-                    flush.zero_()
-                    s = torch.cuda.Event(enable_timing=True)
-                    e = torch.cuda.Event(enable_timing=True)
-                    s.record(stream)
-                    g.fwd(m)
-                    e.record(stream)
-                    e.synchronize()
-                    ts.append(s.elapsed_time(e))
-                t = statistics.median(ts)
+                nnz_total = m.nnz * rep
+                tiles_total = m.tc_tiles * rep if wl.dtype == workloads.BF16 else 0
+                t, t_warm = time_forward(g, m, torch, flush)
                 t_kpad = None
                 lengths = key_padding_lengths(wl)
                 if lengths is not None:   # the same forward with the padding given as lengths
                     sl = torch.tensor(lengths, dtype=torch.int32, device="cuda")
-                    kp = lambda: sp.spattn_fwd_mask_kpad(g.q, g.k, g.v, m, sl, bias=g.bias, scale=wl.scale,
-                                                         out=g.out, lse=g.lse)
-                    for _ in range(3):
-                        kp()
-                    tk = []
-                    for _ in range(10):
-                        flush.zero_()
-                        s = torch.cuda.Event(enable_timing=True)
-                        e = torch.cuda.Event(enable_timing=True)
-                        s.record(stream)
-                        kp()
-                        e.record(stream)
-                        e.synchronize()
-                        tk.append(s.elapsed_time(e))
-                    t_kpad = statistics.median(tk)
-                tb = time.perf_counter()
-                m2 = g.create()
-                torch.cuda.synchronize()
-                build_ms = (time.perf_counter() - tb) * 1e3
-                m2.close()
-                plan = {"tiles": m.n_tiles, "residual_nnz": m.residual_nnz, "mixed_rows": m.n_mixed_rows}
-            alg, _ = algorithmic_bytes(wl, nnz_total)
-            res[wl.name] = {"plan": plan, "fwd_ms": round(t, 4), "tflops": round(4.0 * nnz_total * wl.d / (t * 1e-3) / 1e12, 3),
-                            "effective_gbs": round(alg / (t * 1e-3) / 1e9, 1),
-                            "frac_hbm": round(alg / (t * 1e-3) / 1e9 / hbm_peak, 4),
-                            "nnz_total": nnz_total, "mask_build_wall_ms": round(build_ms, 3)}
+
+                    class K:
+                        def fwd(self_, mm):
+                            sp.spattn_fwd_mask_kpad(g.q, g.k, g.v, mm, sl, bias=g.bias, scale=wl.scale,
+                                                    out=g.out, lse=g.lse)
+                    t_kpad, _ = time_forward(K(), m, torch, flush)
+            tb = time.perf_counter()
+            m2 = g.create()
+            torch.cuda.synchronize()
+            build_ms = (time.perf_counter() - tb) * 1e3
+            m2.close()
+            kname = kernel_name(wl, tiles_total)
+            entry = roofline_entry(wl, t, nnz_total, tiles_total, hbm_peak, tc_peak, peak_src, clk_mhz, kname,
+                                   traffic=committed_traffic(kname, wl.name), t_warm_ms=t_warm)
+            entry.update({"nnz_total": nnz_total,
+                          "tflops": round(4.0 * nnz_total * wl.d / (t * 1e-3) / 1e12, 3),
+                          "mask_build_wall_ms": round(build_ms, 3),
+                          "shape": f"B={wl.B} H={wl.H} n={wl.n} d={wl.d} {wl.dtype}"})
             if t_kpad is not None:
-                res[wl.name]["fwd_ms_seqlen_k"] = round(t_kpad, 4)
+                entry["fwd_ms_seqlen_k"] = round(t_kpad, 4)
+            if cfg == 5:
+                entry["note"] = "extra to the five workloads: all-ones mask, d = 128"
+            res[wl.name] = entry
             del g
         except Exception as ex:  # keep the headline line even if one extra case fails
             res[f"cfg{cfg}"] = {"error": str(ex)[:200]}
@@ -707,7 +777,8 @@ def main():
     result, wl = bench_ours(args, rank, world, torch, sp)
     if rank == 0:
         if not args.no_extra and world == 1:
-            result["other_workloads_fwd"] = other_workloads(torch, sp, args.config)
+            result["other_workloads_fwd"] = other_workloads(torch, sp, args.config,
+                                                            result["clocks"].get("sm_mhz"))
             try:
                 result["backward"] = backward_timing(args, torch, sp)
             except Exception as ex:  # keep the headline line
@@ -719,10 +790,14 @@ def main():
         if not args.no_cpu_baseline and world == 1:
             threads = os.cpu_count() or 1
             rate, cnt, nz, t = cpu_oracle_rate(wl, args.cpu_seconds, threads)
+            rate1, cnt1, nz1, t1 = cpu_oracle_rate(wl, max(1.0, args.cpu_seconds / 4), 1)
             result["cpu_baseline"] = {"value": round(rate, 6), "unit": "TFLOP/s", "cores": threads,
                                       "kind": "oracle",
                                       "sample": f"{cnt} random query rows ({nz} nonzeros) of the same "
-                                                f"workload, {t:.1f} s wall, fp64, {cpu_model()}"}
+                                                f"workload, {t:.1f} s wall, fp64, {cpu_model()}",
+                                      "one_thread": {"value": round(rate1, 6), "cores": 1,
+                                                     "sample": f"{cnt1} random query rows ({nz1} nonzeros), "
+                                                               f"{t1:.1f} s wall"}}
         print(json.dumps(result), flush=True)
     if world > 1:
         torch.distributed.barrier()

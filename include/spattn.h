@@ -110,7 +110,9 @@ typedef struct {
     int64_t in_nnz;             /* CSR, COO: in_row_ptr[num_masks * n] */
     int32_t tile_min_nnz;       /* tensor-core tiles: a 128 x 128 tile with at least this many
                                    nonzeros is computed on tensor cores (bf16 inputs);
-                                   0 = default (512), < 0 = never */
+                                   0 = default (512; for BLOCK_STRIDED_GLOBAL it also
+                                   allows the closed form, see spattn_create_csr_mask),
+                                   < 0 = never */
     uint32_t flags;             /* SPATTN_MASK_* flags below, or 0 */
 } spattn_mask_spec;
 
@@ -146,7 +148,19 @@ typedef struct spattn_mask_s* spattn_mask;
  * bit 0 is raised (see spattn_device_error) -- and the size queries below wait
  * for the build. Memory comes from the library's stream-ordered pool and is
  * released by spattn_destroy_mask.
- * A BLOCK_STRIDED_GLOBAL mask whose n is a multiple of `stride` also keeps the
+ * A BLOCK_STRIDED_GLOBAL mask with tile_min_nnz == 0 whose block divides 128,
+ * stride is 0 or 128, n_global <= 128, n is a multiple of 128 and block or
+ * n_global is positive is kept in closed form: the call does no device work
+ * and never synchronises; the forward pass derives every tensor-core tile and
+ * every row's bits from the four parameters, the strided entries outside the
+ * regular tiles running as residue-permuted dense tiles (token i at
+ * (i mod 128) n/128 + i div 128) in the same launch, each row's two partial
+ * states merged with the running max / sum rule in fp32. Its CSR, tile plan,
+ * the backward pass and forward calls the closed form does not take (fp32
+ * inputs, additive terms, key lengths, d = 32) use a CSR-built copy of the
+ * mask made on first need (one build on the mask's stream, with its
+ * synchronisations; kept until the mask is destroyed).
+ * Any other BLOCK_STRIDED_GLOBAL mask whose n is a multiple of `stride` also keeps the
  * strided entries that fall outside its tensor-core tiles as a second mask in
  * residue-permuted order (token i at (i mod stride) n/stride + i div stride),
  * where they form dense tiles, plus the remaining entries as a third. That is
@@ -169,6 +183,20 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream, spattn_ma
 int spattn_mask_info(spattn_mask mask, int32_t* n, int32_t* num_masks, int64_t* nnz,
                      const int32_t** row_ptr, const int32_t** col_idx, int64_t* n_long);
 
+/* The user-visible CSR of a mask: row_ptr int32 [num_masks * n + 1] (global
+ * offsets, row m*n + i of mask m), col_idx int32 [nnz_total], both device
+ * pointers owned by the mask and valid until spattn_destroy_mask, and the
+ * total number of nonzeros over all num_masks masks. Any output pointer may be
+ * NULL. This is the n x n CSR attention mask that "[Proposal] Unified
+ * Interface/Implementation for Sparse Attention" (gluon-nlp issue 1407,
+ * opening post) has the user hand to the operation; the same as
+ * spattn_mask_info with only these outputs (an interval or closed-form mask
+ * writes its CSR first and synchronises the mask's stream once; nnz_total
+ * waits for an asynchronous build). Errors: INVALID_ARG (mask NULL),
+ * UNSUPPORTED (more than 2^31 - 1 nonzeros), OOM, CUDA. */
+int spattn_mask_csr(spattn_mask mask, const int32_t** row_ptr, const int32_t** col_idx,
+                    int64_t* nnz_total);
+
 /* Copy a mask's CSR into caller buffers (device or host memory, any mix):
  * row_ptr_dst int32 [num_masks * n + 1], col_idx_dst int32 [nnz]; either may be
  * NULL to skip it. Stream-ordered on `stream`; host destinations should be
@@ -177,12 +205,29 @@ int spattn_mask_info(spattn_mask mask, int32_t* n, int32_t* num_masks, int64_t* 
 int spattn_mask_copy_csr(spattn_mask mask, int32_t* row_ptr_dst, int32_t* col_idx_dst,
                          void* stream);
 
+/* Copy the mask's list of long rows -- the n_long rows (mask-row ids
+ * m * n + i) with more than 1024 nonzeros, which the gather kernel gives a
+ * whole thread block -- into dst (device or host, int32 [n_long]; the order is
+ * unspecified). Stream-ordered on `stream`; an interval mask lists them from
+ * its CSR on first request, and a closed-form mask from its CSR-built copy
+ * (both synchronise once). Errors: INVALID_ARG (NULL argument), OOM, CUDA. */
+int spattn_mask_copy_long_rows(spattn_mask mask, int32_t* dst, void* stream);
+
 /* The tile plan's sizes: tensor-core tiles, residual nonzeros (the entries the
  * gather kernel processes on bf16 inputs) and rows with entries on both paths.
  * Any output pointer may be NULL. Waits for an asynchronous build; n_mixed_rows
  * of an interval mask writes its explicit plan first (synchronises). */
 int spattn_mask_plan_info(spattn_mask mask, int64_t* n_tiles, int64_t* residual_nnz,
                           int64_t* n_mixed_rows);
+
+/* Diagnostic with no counterpart in the method: the number of 128 x 128
+ * tensor-core tiles one forward pass over this mask computes per (b, h),
+ * summed over the mask's num_masks masks (as nnz is), for bf16 inputs without
+ * additive terms; each tile is two 128 x 128 x d MMAs (S = Q K^T and P V).
+ * For a closed-form block + strided + global mask this counts its regular and
+ * residue-permuted tiles. Waits for an asynchronous build. Errors:
+ * INVALID_ARG (NULL argument). */
+int spattn_mask_tile_count(spattn_mask mask, int64_t* tiles);
 
 /* Copy the tile plan into caller buffers (device or host, any may be NULL):
  * block_tile_off int32 [num_masks * ceil(n/128) + 1] (tiles of query block x are
@@ -330,6 +375,13 @@ const char* spattn_last_error(void);
  * else SPATTN_ERR_BAD_CSR if bit 0 was set. */
 int spattn_device_error(void* stream, uint32_t* flags);
 
+/* spattn_device_error without the flag word: synchronises `stream`, reads and
+ * clears the error flags, and returns SPATTN_ERR_TIMEOUT if a bounded
+ * device-side wait expired, SPATTN_ERR_BAD_CSR if a column outside [0, n) was
+ * skipped (or an asynchronous build met a negative half-width), SPATTN_OK
+ * otherwise (SPATTN_ERR_CUDA if the synchronisation itself fails). */
+int spattn_check_device_error(void* stream);
+
 /* Library version: major * 10000 + minor * 100 + patch. */
 int spattn_version(void);
 
@@ -337,6 +389,12 @@ int spattn_version(void);
  * threads and devices (a diagnostic with no counterpart in the method: it lets
  * a caller count the launches a sequence of calls costs). Never fails. */
 uint64_t spattn_launch_count(void);
+
+/* Number of memory allocations this library has made since it was loaded
+ * (stream-ordered pool blocks, device memory, mapped host memory), over all
+ * threads and devices: a diagnostic with no counterpart in the method, so that
+ * a caller can check that a sequence of calls allocates nothing. Never fails. */
+uint64_t spattn_alloc_count(void);
 
 #ifdef __cplusplus
 }

@@ -79,10 +79,14 @@ SIGNATURES = {
                                         ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(_P),
                                         ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_int64)]),
     "spattn_mask_copy_csr": (ctypes.c_int, [_P, _P, _P, _P]),
+    "spattn_mask_copy_long_rows": (ctypes.c_int, [_P, _P, _P]),
+    "spattn_mask_csr": (ctypes.c_int, [_P, ctypes.POINTER(_P), ctypes.POINTER(_P),
+                                       ctypes.POINTER(ctypes.c_int64)]),
     "spattn_mask_plan_info": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int64),
                                              ctypes.POINTER(ctypes.c_int64),
                                              ctypes.POINTER(ctypes.c_int64)]),
     "spattn_mask_copy_plan": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P]),
+    "spattn_mask_tile_count": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int64)]),
     "spattn_destroy_mask": (ctypes.c_int, [_P]),
     "spattn_fwd": (ctypes.c_int, [_TP, _TP, _TP, _P, _P, ctypes.c_int32, ctypes.c_int64, _TP, _TP,
                                   ctypes.c_float, _TP, _P, _P]),
@@ -91,6 +95,7 @@ SIGNATURES = {
                                           _TP, ctypes.c_float, _TP, _P, _P]),
     "spattn_last_error": (ctypes.c_char_p, []),
     "spattn_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "spattn_check_device_error": (ctypes.c_int, [_P]),
     "spattn_fwd_mask_kpad": (ctypes.c_int, [_TP, _TP, _TP, _P, _P, _TP, _TP, ctypes.c_float, _TP, _P,
                                             _P]),
     "spattn_fwd_unfused": (ctypes.c_int, [_TP, _TP, _TP, _P, _P, ctypes.c_int32, ctypes.c_int64, _TP,
@@ -99,6 +104,7 @@ SIGNATURES = {
                                        _TP, _TP, _TP, _P]),
     "spattn_version": (ctypes.c_int, []),
     "spattn_launch_count": (ctypes.c_uint64, []),
+    "spattn_alloc_count": (ctypes.c_uint64, []),
 }
 
 
@@ -200,6 +206,14 @@ class Mask:
         return self._plan_info()[1]
 
     @property
+    def tc_tiles(self) -> int:
+        """128 x 128 tensor-core tiles one bf16 forward computes per (b, h),
+        summed over the masks (spattn_mask_tile_count)."""
+        t = ctypes.c_int64()
+        _check(LIB.spattn_mask_tile_count(self.handle, ctypes.byref(t)))
+        return t.value
+
+    @property
     def n_mixed_rows(self) -> int:
         if self._mixed is None:
             nm = ctypes.c_int64()
@@ -214,6 +228,14 @@ class Mask:
         ci = torch.empty(max(1, self.nnz), dtype=torch.int32, device="cuda")
         _check(LIB.spattn_mask_copy_csr(self.handle, rp.data_ptr(), ci.data_ptr(), _stream(stream)))
         return rp, ci[: self.nnz]
+
+    def long_rows(self, stream=None):
+        """The rows with more than 1024 nonzeros (mask-row ids m*n + i), sorted,
+        as an int32 CUDA tensor."""
+        import torch
+        out = torch.empty(max(1, self.n_long), dtype=torch.int32, device="cuda")
+        _check(LIB.spattn_mask_copy_long_rows(self.handle, out.data_ptr(), _stream(stream)))
+        return torch.sort(out[: self.n_long]).values
 
     def plan(self, stream=None):
         """Copies of the tile plan (block_tile_off, tile_info, tile_bits,
@@ -348,6 +370,24 @@ def spattn_device_error(stream=None) -> int:
     return flags.value
 
 
+def spattn_check_device_error(stream=None) -> int:
+    """Synchronise the stream, clear the kernels' error flags and return the
+    status they map to (SPATTN_OK, SPATTN_ERR_TIMEOUT or SPATTN_ERR_BAD_CSR);
+    raises only when the synchronisation itself fails."""
+    st = LIB.spattn_check_device_error(_stream(stream))
+    if st not in (SPATTN_OK, SPATTN_ERR_BAD_CSR, SPATTN_ERR_TIMEOUT):
+        _check(st)
+    return st
+
+
+def spattn_mask_csr(mask: "Mask"):
+    """The mask's own CSR through ``spattn_mask_csr``: (row_ptr address,
+    col_idx address, nnz_total); the arrays belong to the mask."""
+    rp, ci, nz = _P(), _P(), ctypes.c_int64()
+    _check(LIB.spattn_mask_csr(mask.handle, ctypes.byref(rp), ctypes.byref(ci), ctypes.byref(nz)))
+    return rp.value, ci.value, nz.value
+
+
 def spattn_last_error() -> str:
     return LIB.spattn_last_error().decode()
 
@@ -419,3 +459,9 @@ def spattn_version() -> int:
 def spattn_launch_count() -> int:
     """Kernels the library has enqueued since it was loaded (all threads, devices)."""
     return int(LIB.spattn_launch_count())
+
+
+def spattn_alloc_count() -> int:
+    """Memory allocations the library has made since it was loaded (pool blocks,
+    device and mapped host memory; all threads, devices)."""
+    return int(LIB.spattn_alloc_count())

@@ -1,0 +1,846 @@
+// Persistent, warp-specialised tensor-core forward for d = 64 and d = 128
+// (tcgen05 MMAs with TMEM accumulators, TMA tile loads without multicast,
+// sm_100a).
+//
+// One CTA per SM walks a list of work items (a 128-row query block and its
+// key tiles). Three warpgroups:
+//   warp 0      TMA producer (one thread): Q tile per item, K and V per tile
+//   warp 1      MMA issuer (one thread):   S = Q K^T, then O (+)= P V
+//   warps 2-3   idle (they complete the first warpgroup, which gives its
+//               registers to the other two: 72 per thread against 216)
+//   warps 4-7   softmax group of slot 0 (one query row per thread)
+//   warps 8-11  softmax group of slot 1
+// The two slots hold one item each, with their own Q, K and V buffers in shared
+// memory and their own S and O in tensor memory (slot s: S in columns
+// [256 s, 256 s + 128), O in [256 s + 128, 256 s + 128 + d); P, in bf16,
+// overwrites the first 64 columns of S). While one slot's softmax group turns
+// S into P, the tensor cores work on the other slot, so the two dependency
+// chains (S -> softmax -> P V -> next S) overlap. Producer and MMA issuer poll
+// both slots and advance whichever is ready; every wait is bounded.
+//
+// Per tile, each thread reads its row of S, scales it, sets the entries the
+// mask does not list to -inf, and keeps a running max and sum: the reference
+// max only moves when a tile's max exceeds it by more than 2^8, and then O is
+// rescaled in TMEM by exp2(m_old - m_new) (the streaming-dataflow SDPA
+// paper's delta rescaling, applied lazily; exact in exact arithmetic). A warp
+// skips the 32-key chunks in which none of its rows has an entry (no TMEM load,
+// no exp; P is zero there).
+//
+// Two sources of work items:
+//   interval masks (sliding, variable window, dense): every (b, h, query
+//     block) with tiles; per-row bits from the row's run; rows that also have
+//     gathered entries merge the gather kernel's partial state;
+//   block + strided + global masks in closed form (bsg_plan.cuh): regular
+//     query blocks (block 0 of a mask with global rows split into chunks,
+//     merged by the warp that completes a per-(b, h, warp) count) and
+//     residue-permuted blocks read through five-dimensional tensor maps; a row
+//     with entries in both meets its partner per row: the first to finish
+//     publishes its fp32 state (m, l, O), the second merges it and writes the
+//     row, and discards the published lines from L2.
+#include "spattn_internal.cuh"
+#include "sm100_ptx.cuh"
+#include "bsg_plan.cuh"
+
+#include <math.h>
+#include <mutex>
+
+namespace spattn {
+namespace {
+
+using namespace sm100;
+
+constexpr int kPpThreads = 384;
+// registers per thread after the split (launched with 168: 384 x 168 = 64,512
+// = 128 x 72 + 256 x 216; per SM sub-partition, warps w, w + 4, w + 8:
+// (72 + 2 x 216) x 32 <= 16,384)
+constexpr int kPpRegsLow = 72;
+constexpr int kPpRegsHigh = 216;
+constexpr uint32_t kPpTmemCols = 512;
+constexpr float kPpRescale = 8.0f;               // log2 units
+constexpr long long kPpDrainCycles = 200000000LL;  // ~0.1 s per drain wait
+
+// mbarriers of slot s: 10 s + one of these; kBarDrain after both slots
+enum : int { kQFull = 0, kQEmpty, kKFull, kKEmpty, kVFull, kVEmpty, kSFull, kPFull, kODone, kOFree, kBarsPerSlot };
+constexpr int kBarDrain = 2 * kBarsPerSlot;
+constexpr int kNumBars = kBarDrain + 1;
+
+template <int D>
+struct PpCfg {
+    static_assert(D == 64 || D == 128, "head dim");
+    static constexpr int ROW_BYTES = 128;                // 64 bf16 per 128-byte swizzled row
+    static constexpr int NCHUNK = D / 64;
+    static constexpr int CHUNK_BYTES = 128 * ROW_BYTES;  // 128 rows of one 64-column chunk
+    static constexpr int TILE_BYTES = NCHUNK * CHUNK_BYTES;
+    static constexpr int SBO = 8 * ROW_BYTES;
+    static constexpr int OFF_Q = 0;                    // [slot]
+    static constexpr int OFF_K = 2 * TILE_BYTES;       // [slot]
+    static constexpr int OFF_V = 4 * TILE_BYTES;       // [slot]
+    static constexpr int OFF_BAR = 6 * TILE_BYTES;
+    static constexpr int OFF_INT = OFF_BAR + kNumBars * 8;  // TMEM base, abort flag
+    // at least 116 KB, so that one CTA (which takes all 512 TMEM columns) runs per SM
+    static constexpr int SMEM_BYTES = OFF_INT + 16 > 116 * 1024 ? OFF_INT + 16 : 116 * 1024;
+};
+
+// A work item as every role sees it.
+struct PpItem {
+    bool valid;
+    int bh, b, h;
+    int perm;           // closed form: permuted block
+    int qb;             // query block (permuted: residue)
+    int pqb;            // permuted: block of positions
+    int chunk;          // closed form: chunk of query block 0
+    int u0;             // closed form: first tile of the chunk
+    int T;              // tiles
+    int64_t blk;        // interval masks: mask block (mask * nqb + qb)
+};
+
+__device__ __forceinline__ PpItem pp_item(const PpParams& P, const bsg::Shape& sh, int64_t x) {
+    PpItem it;
+    it.valid = x < P.n_items;
+    it.perm = 0;
+    it.pqb = 0;
+    it.chunk = 0;
+    it.u0 = 0;
+    it.blk = 0;
+    it.T = 0;
+    if (!it.valid) return it;
+    if (P.mode == 0) {
+        it.bh = (int)(x / P.nqb);
+        it.qb = (int)(x - (int64_t)it.bh * P.nqb);
+        it.b = it.bh / P.H;
+        it.h = it.bh - it.b * P.H;
+        const int mk = P.num_masks == 1 ? 0 : it.b;
+        it.blk = (int64_t)mk * P.nqb + it.qb;
+        it.T = __ldg(P.itv_ntiles + it.blk);
+    } else {
+        const bsg::Item bi = bsg::item(sh, x);
+        it.bh = bi.bh;
+        it.b = bi.bh / P.H;
+        it.h = bi.bh - it.b * P.H;
+        it.perm = bi.perm;
+        it.qb = bi.qb;
+        it.pqb = bi.pqb;
+        it.chunk = bi.chunk;
+        it.u0 = bi.u0;
+        it.T = bi.T;
+    }
+    return it;
+}
+
+// Key tile u of the item: the key tile index, with kTileDenseBit set when
+// every entry of the tile is present (interval masks only).
+__device__ __forceinline__ int pp_tile(const PpParams& P, const bsg::Shape& sh, const PpItem& it, int u) {
+    if (P.mode == 0) return __ldg(P.itv_tiles + it.blk * P.nkt + u);
+    bsg::Item bi;
+    bi.bh = it.bh;
+    bi.perm = it.perm;
+    bi.qb = it.qb;
+    bi.pqb = it.pqb;
+    bi.chunk = it.chunk;
+    bi.u0 = it.u0;
+    bi.T = it.T;
+    return bsg::key_tile(sh, bi, u);
+}
+
+// Bounded wait that also gives up as soon as another thread of the CTA has.
+__device__ __forceinline__ bool pp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, long long limit) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > limit) {
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+template <int R>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <int R>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+
+__device__ __forceinline__ void discard_l2_line(const void* p) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Writes row i of (b, h): out = o / L (bf16, round to nearest even), lse = (M + log2 L) ln 2.
+template <int D>
+__device__ __forceinline__ void pp_write_row(const PpParams& P, int b, int h, int64_t bh, int i, float M, float L,
+                                             const float (&o)[D]) {
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(P.out) + (int64_t)b * P.o_sb + (int64_t)h * P.o_sh +
+                          (int64_t)i * P.o_sn;
+#pragma unroll
+    for (int e8 = 0; e8 < D / 8; ++e8) {
+        uint32_t w[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            __nv_bfloat162 hv = __floats2bfloat162_rn(o[e8 * 8 + 2 * t] * inv, o[e8 * 8 + 2 * t + 1] * inv);
+            w[t] = *reinterpret_cast<uint32_t*>(&hv);
+        }
+        *reinterpret_cast<uint4*>(orow + e8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    if (P.lse) P.lse[bh * P.n + i] = L > 0.f ? (M + lg2(L)) * kLn2 : -INFINITY;
+}
+
+// The end of one item for one warp's rows: state (M, L, o) in base 2, o not
+// yet divided by L. Merges what the row has elsewhere, then writes it (or
+// publishes it for the row's partner).
+template <int D>
+__device__ __forceinline__ void pp_finish(const PpParams& P, const bsg::Shape& sh, const PpItem& it, int quarter, int t, int i,
+                          bool row_ok, float M, float L, float (&o)[D]) {
+    const int lane = threadIdx.x & 31;
+    const int64_t bh = it.bh;
+    if (P.mode == 0) {
+        if (!row_ok) return;
+        const int64_t wrow = bh * P.n + i;
+        if (P.blk_res && __ldg(P.blk_res + it.blk) && P.ws_ml[wrow * 2 + 1] > 0.f) {
+            // the gather kernel's partial state of the row's other entries
+            const float mg = P.ws_ml[wrow * 2], lg = P.ws_ml[wrow * 2 + 1];
+            const float Mn = fmaxf(M, mg);
+            const float Mu = Mn == -INFINITY ? 0.f : Mn;
+            const float fa = ex2(M - Mu), fg = ex2(mg - Mu);
+            const float* acc = P.ws_acc + wrow * D;
+#pragma unroll
+            for (int e = 0; e < D; ++e) o[e] = fmaf(acc[e], fg, o[e] * fa);
+            L = L * fa + lg * fg;
+            M = Mn;
+        }
+        pp_write_row<D>(P, it.b, it.h, bh, i, M, L, o);
+        return;
+    }
+
+    if (!it.perm && sh.nch > 1 && it.qb == 0) {
+        // one chunk of the global-row block: publish, and the warp that
+        // completes this quarter's count merges all chunks (in chunk order)
+        float* mine = P.cws + ((bh * sh.nch + it.chunk) * (int64_t)(D + 2)) * 128 + t;
+        mine[0] = M;
+        mine[128] = L;
+        if (L > 0.f) {
+#pragma unroll
+            for (int e = 0; e < D; ++e) mine[(int64_t)(2 + e) * 128] = o[e];
+        }
+        __threadfence();
+        __syncwarp();
+        unsigned last = 0;
+        if (lane == 0) last = atomicAdd(P.ccnt + bh * 4 + quarter, 1u) == (unsigned)(sh.nch - 1);
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (!last) return;
+        __threadfence();
+        M = -INFINITY;
+        L = 0.f;
+#pragma unroll
+        for (int e = 0; e < D; ++e) o[e] = 0.f;
+        for (int c = 0; c < sh.nch; ++c) {
+            const float* pp = P.cws + ((bh * sh.nch + c) * (int64_t)(D + 2)) * 128 + t;
+            const float mc = __ldcg(pp), lc = __ldcg(pp + 128);
+            if (!(lc > 0.f)) continue;
+            const float Mn = fmaxf(M, mc);
+            const float fa = ex2(M - Mn), fb = ex2(mc - Mn);
+#pragma unroll
+            for (int e = 0; e < D; ++e) o[e] = fmaf(__ldcg(pp + (int64_t)(2 + e) * 128), fb, o[e] * fa);
+            L = L * fa + lc * fb;
+            M = Mn;
+        }
+    }
+    if (!row_ok) return;
+    const bool partner = bsg::has_perm(sh, i);
+    if (it.perm && !partner) return;  // no strided entries of this row here
+    if (partner) {
+        const int64_t prow = bh * P.n + i;
+        unsigned* cnt = P.pcnt + prow;
+        float* pm = P.pml + prow * 2;
+        float* pa = P.pacc + prow * D;
+        const unsigned old = atomicAdd(cnt, 1u);
+        if (old == 0u) {  // first: publish the state for the partner
+            pm[0] = M;
+            pm[1] = L;
+#pragma unroll
+            for (int e = 0; e < D; e += 4)
+                *reinterpret_cast<float4*>(pa + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+            __threadfence();
+            atomicAdd(cnt, 2u);
+            return;
+        }
+        // second: the partner's state is complete once the count reaches 4
+        if (ld_acquire_u32(cnt) != 4u) {
+            const long long t0 = clock64();
+            while (ld_acquire_u32(cnt) != 4u) {
+                if (clock64() - t0 > P.wait_cycles) {
+                    atomicOr(P.err, kErrTimeout);
+                    return;
+                }
+                __nanosleep(64);
+            }
+        }
+        __threadfence();
+        const float Mq = __ldcg(pm), Lq = __ldcg(pm + 1);
+        // regular part first, whichever of the two arrived last
+        const float Mr = it.perm ? Mq : M, Lr = it.perm ? Lq : L;
+        const float Mp = it.perm ? M : Mq, Lp = it.perm ? L : Lq;
+        const float Mn = fmaxf(Mr, Mp);
+        const float Mu = Mn == -INFINITY ? 0.f : Mn;
+        const float fr = ex2(Mr - Mu), fp = ex2(Mp - Mu);
+#pragma unroll
+        for (int e = 0; e < D; e += 4) {
+            const float4 q4 = __ldcg(reinterpret_cast<const float4*>(pa + e));
+            const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+            for (int z = 0; z < 4; ++z) {
+                const float orr = it.perm ? qv[z] : o[e + z], opp = it.perm ? o[e + z] : qv[z];
+                o[e + z] = fmaf(opp, fp, orr * fr);
+            }
+        }
+        L = Lr * fr + Lp * fp;
+        M = Mn;
+        // the published lines are read exactly once: drop them from L2 unwritten
+#pragma unroll
+        for (int z = 0; z < D * 4 / 128; ++z) discard_l2_line(pa + z * 32);
+    }
+    pp_write_row<D>(P, it.b, it.h, bh, i, M, L, o);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPpThreads, 1)
+    k_fwd_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQp,
+             const __grid_constant__ CUtensorMap tmKp, const __grid_constant__ CUtensorMap tmVp,
+             const PpParams P) {
+    using C = PpCfg<D>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (smem_u32(smem) & 1023u) {  // the swizzled layouts need a 1024-byte aligned base
+        if (tid == 0) atomicOr(P.err, kErrTimeout);
+        return;
+    }
+    const bsg::Shape sh = bsg::shape(P.n, P.blk, P.S, P.ng, P.chunk_tiles);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_INT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_INT + 4);
+    auto bar = [&](int s, int which) { return smem_u32(bars + s * kBarsPerSlot + which); };
+    const uint32_t sQ0 = smem_u32(smem + C::OFF_Q), sK0 = smem_u32(smem + C::OFF_K),
+                   sV0 = smem_u32(smem + C::OFF_V);
+    // item j of this CTA (slot j & 1)
+    auto item_x = [&](int s, int m) { return (int64_t)blockIdx.x + (int64_t)(2 * m + s) * gridDim.x; };
+
+    if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kPpTmemCols);
+    if (tid == 0) {
+        for (int s = 0; s < 2; ++s)
+            for (int x = 0; x < kBarsPerSlot; ++x)
+                mbar_init(bar(s, x), (x == kPFull || x == kOFree) ? 4u : 1u);
+        mbar_init(smem_u32(bars + kBarDrain), 1u);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+        if (P.mode == 1 && P.S) {
+            prefetch_tensormap(&tmQp);
+            prefetch_tensormap(&tmKp);
+            prefetch_tensormap(&tmVp);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // the first item with tiles at or after slot s's item m (m past the end: none)
+    auto seek = [&](int s, int& m, int& T) -> bool {
+        while (true) {
+            const PpItem it = pp_item(P, sh, item_x(s, m));
+            if (!it.valid) return false;
+            if (it.T > 0) {
+                T = it.T;
+                return true;
+            }
+            ++m;
+        }
+    };
+
+    if (warp < 4) {
+        regs_dec<kPpRegsLow>();
+    }
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            // per slot three load streams (Q per item; K, V per tile): the
+            // stream's item m, tile u, loads issued, the item's tile count
+            int sm[2][3], su[2][3], sT[2][3];
+            uint32_t cnt[2][3];
+            bool live[2][3];
+#pragma unroll
+            for (int s = 0; s < 2; ++s)
+#pragma unroll
+                for (int k = 0; k < 3; ++k) {
+                    sm[s][k] = su[s][k] = 0;
+                    cnt[s][k] = 0;
+                    sT[s][k] = 0;
+                    live[s][k] = seek(s, sm[s][k], sT[s][k]);
+                }
+            long long t_last = clock64();
+            while (true) {
+                bool any = false, progress = false;
+#pragma unroll
+                for (int s = 0; s < 2; ++s) {
+#pragma unroll
+                    for (int k = 0; k < 3; ++k) {
+                        if (!live[s][k]) continue;
+                        any = true;
+                        const int eb = k == 0 ? kQEmpty : (k == 1 ? kKEmpty : kVEmpty);
+                        if (cnt[s][k] != 0 && !mbar_try_wait(bar(s, eb), (cnt[s][k] - 1) & 1)) continue;
+                        const PpItem it = pp_item(P, sh, item_x(s, sm[s][k]));
+                        const uint32_t fb = bar(s, k == 0 ? kQFull : (k == 1 ? kKFull : kVFull));
+                        const uint32_t dst = (k == 0 ? sQ0 : (k == 1 ? sK0 : sV0)) + s * C::TILE_BYTES;
+                        mbar_expect_tx(fb, C::TILE_BYTES);
+                        if (k == 0) {
+#pragma unroll
+                            for (int c = 0; c < C::NCHUNK; ++c) {
+                                if (it.perm)
+                                    tma_load_5d(dst + c * C::CHUNK_BYTES, &tmQp, fb, c * 64, it.qb, it.pqb * 128, it.h,
+                                                it.b);
+                                else
+                                    tma_load_4d(dst + c * C::CHUNK_BYTES, &tmQ, fb, c * 64, it.qb * 128, it.h, it.b);
+                            }
+                        } else {
+                            const int kt = pp_tile(P, sh, it, su[s][k]) & 0x7fffffff;
+                            const CUtensorMap* map = it.perm ? (k == 1 ? &tmKp : &tmVp) : (k == 1 ? &tmK : &tmV);
+#pragma unroll
+                            for (int c = 0; c < C::NCHUNK; ++c) {
+                                if (it.perm)
+                                    tma_load_5d(dst + c * C::CHUNK_BYTES, map, fb, c * 64, it.qb, kt * 128, it.h, it.b);
+                                else
+                                    tma_load_4d(dst + c * C::CHUNK_BYTES, map, fb, c * 64, kt * 128, it.h, it.b);
+                            }
+                        }
+                        ++cnt[s][k];
+                        if (k == 0 || ++su[s][k] == sT[s][k]) {
+                            su[s][k] = 0;
+                            ++sm[s][k];
+                            live[s][k] = seek(s, sm[s][k], sT[s][k]);
+                        }
+                        progress = true;
+                    }
+                }
+                if (!any) break;
+                if (progress) {
+                    t_last = clock64();
+                } else {
+                    if (*abort_flag) break;
+                    if (clock64() - t_last > P.wait_cycles) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                }
+            }
+            // no load may outlive the CTA: wait (bounded) for the last of each buffer
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+#pragma unroll
+                for (int k = 0; k < 3; ++k) {
+                    const int full = k == 0 ? kQFull : (k == 1 ? kKFull : kVFull);
+                    if (cnt[s][k]) mbar_wait_bounded(bar(s, full), (cnt[s][k] - 1) & 1, kPpDrainCycles);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            struct Slot {
+                int m, u, T, phase;  // phase 0: S(g) next, 1: P V(g) next
+                uint32_t g, items;
+                bool live;
+            };
+            Slot sl[2];
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+                sl[s].m = sl[s].u = sl[s].phase = sl[s].T = 0;
+                sl[s].g = sl[s].items = 0;
+                sl[s].live = seek(s, sl[s].m, sl[s].T);
+            }
+            const uint32_t idS = idesc_bf16_f32(128, 128, false);
+            const uint32_t idO = idesc_bf16_f32(128, D, true);
+            long long t_last = clock64();
+            while (true) {
+                bool all_done = true, progress = false;
+#pragma unroll
+                for (int s = 0; s < 2; ++s) {
+                    Slot& x = sl[s];
+                    if (!x.live) continue;
+                    all_done = false;
+                    const uint32_t tS = tmem + (uint32_t)(s * 256), tO = tS + 128;
+                    if (x.phase == 0) {
+                        // S(g) needs the item's Q, K(g), and P V(g-1) done (P overwrote S)
+                        const bool ready = (x.u != 0 || mbar_try_wait(bar(s, kQFull), x.items & 1)) &&
+                                           mbar_try_wait(bar(s, kKFull), x.g & 1) &&
+                                           (x.g == 0 || mbar_try_wait(bar(s, kODone), (x.g - 1) & 1));
+                        if (ready) {
+                            tc_fence_after();
+                            const uint32_t sQ = sQ0 + s * C::TILE_BYTES, sK = sK0 + s * C::TILE_BYTES;
+#pragma unroll
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const uint32_t off = (uint32_t)((ks / 4) * C::CHUNK_BYTES + (ks % 4) * 32);
+                                mma_bf16_ss(tS, smem_desc(sQ + off, 16, C::SBO, cute::UMMA::LayoutType::SWIZZLE_128B),
+                                            smem_desc(sK + off, 16, C::SBO, cute::UMMA::LayoutType::SWIZZLE_128B),
+                                            idS, ks > 0 ? 1u : 0u);
+                            }
+                            mma_commit(bar(s, kSFull));
+                            mma_commit(bar(s, kKEmpty));
+                            if (x.u == x.T - 1) mma_commit(bar(s, kQEmpty));
+                            x.phase = 1;
+                            progress = true;
+                        }
+                    } else {
+                        // P V(g) needs P(g), V(g), and for an item's first tile the
+                        // previous item's O read out
+                        const bool ready = mbar_try_wait(bar(s, kPFull), x.g & 1) &&
+                                           mbar_try_wait(bar(s, kVFull), x.g & 1) &&
+                                           (x.u != 0 || x.items == 0 || mbar_try_wait(bar(s, kOFree), (x.items - 1) & 1));
+                        if (ready) {
+                            tc_fence_after();
+                            const uint32_t sV = sV0 + s * C::TILE_BYTES;
+#pragma unroll
+                            for (int ks = 0; ks < 8; ++ks) {  // 16 keys per step
+                                const uint64_t db = smem_desc(sV + (uint32_t)(ks * 16 * C::ROW_BYTES), C::CHUNK_BYTES,
+                                                              C::SBO, cute::UMMA::LayoutType::SWIZZLE_128B);
+                                mma_bf16_ts(tO, tS + (uint32_t)(ks * 8), db, idO, (x.u > 0 || ks > 0) ? 1u : 0u);
+                            }
+                            mma_commit(bar(s, kODone));
+                            mma_commit(bar(s, kVEmpty));
+                            ++x.g;
+                            x.phase = 0;
+                            if (++x.u == x.T) {
+                                x.u = 0;
+                                ++x.items;
+                                ++x.m;
+                                x.live = seek(s, x.m, x.T);
+                            }
+                            progress = true;
+                        }
+                    }
+                }
+                if (all_done) break;
+                if (progress) {
+                    t_last = clock64();
+                } else {
+                    if (*abort_flag) break;
+                    if (clock64() - t_last > P.wait_cycles) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                }
+            }
+            // every MMA issued is complete before the CTA releases TMEM
+            mma_commit(smem_u32(bars + kBarDrain));
+            mbar_wait_bounded(smem_u32(bars + kBarDrain), 0u, kPpDrainCycles);
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ softmax groups
+        regs_inc<kPpRegsHigh>();
+        const int s = (warp - 4) >> 2;
+        const int quarter = warp & 3;  // the TMEM lanes this warp may access
+        const int t = quarter * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        const uint32_t tS = tmem + (uint32_t)(s * 256) + lane_base, tO = tS + 128;
+        const uint64_t c2 = pack2(P.qk_scale_log2, P.qk_scale_log2);
+        uint32_t g = 0;
+        bool alive = true;
+        for (int m = 0; alive; ++m) {
+            const PpItem it = pp_item(P, sh, item_x(s, m));
+            if (!it.valid) break;
+            if (it.T <= 0) continue;
+            int i;
+            bool row_ok;
+            int rlo = 0, rhi = 0;
+            if (P.mode == 0) {
+                i = it.qb * 128 + t;
+                row_ok = i < P.n;
+                if (row_ok) {
+                    const int2 v = __ldg(P.itv_lohi + (it.blk / P.nqb) * P.n + i);
+                    rlo = v.x;
+                    rhi = v.y;
+                }
+            } else {
+                bsg::Item bi;
+                bi.bh = it.bh;
+                bi.perm = it.perm;
+                bi.qb = it.qb;
+                bi.pqb = it.pqb;
+                bi.chunk = it.chunk;
+                bi.u0 = it.u0;
+                bi.T = it.T;
+                i = bsg::row_of(sh, bi, t);
+                row_ok = i >= 0;
+            }
+            float m_ref = -INFINITY, l = 0.f;
+            for (int u = 0; u < it.T; ++u, ++g) {
+                const int info = pp_tile(P, sh, it, u);
+                const int kt = info & 0x7fffffff;
+                const bool dense = P.mode == 0 && info < 0;
+                uint32_t w[4] = {0u, 0u, 0u, 0u};
+                if (row_ok && !dense) {
+                    if (P.mode == 0) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) w[q] = bsg::run_word(rlo, rhi, kt * 128 + 32 * q);
+                    } else {
+                        bsg::Item bi;
+                        bi.bh = it.bh;
+                        bi.perm = it.perm;
+                        bi.qb = it.qb;
+                        bi.pqb = it.pqb;
+                        bi.chunk = it.chunk;
+                        bi.u0 = it.u0;
+                        bi.T = it.T;
+                        bsg::row_bits(sh, bi, kt, t, w);
+                    }
+                }
+                uint32_t need = 0;
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (dense || __any_sync(0xffffffffu, w[q] != 0u)) need |= 1u << q;
+
+                const bool ok = pp_wait(bar(s, kSFull), g & 1, abort_flag, P.wait_cycles);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    alive = false;
+                    break;
+                }
+                tc_fence_after();
+                float x[128];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (need & (1u << q)) {
+                        uint32_t r[32];
+                        tmem_ld32(tS + 32 * q, r);
+                        tmem_wait_ld_dep(r);
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) mul2(x[32 * q + 2 * k], x[32 * q + 2 * k + 1], r[2 * k], r[2 * k + 1], c2);
+                        if (!dense) {
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj)
+                                x[32 * q + jj] = ((w[q] >> jj) & 1u) ? x[32 * q + jj] : -INFINITY;
+                        }
+                    } else {
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) x[32 * q + jj] = -INFINITY;
+                    }
+                }
+                float ma = -INFINITY, mb = -INFINITY, mc = -INFINITY, md = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    ma = fmax3(ma, x[8 * k + 0], x[8 * k + 1]);
+                    mb = fmax3(mb, x[8 * k + 2], x[8 * k + 3]);
+                    mc = fmax3(mc, x[8 * k + 4], x[8 * k + 5]);
+                    md = fmax3(md, x[8 * k + 6], x[8 * k + 7]);
+                }
+                const float mx = fmax3(ma, mb, fmaxf(mc, md));
+                const bool grow = mx > m_ref + kPpRescale;
+                float alpha = 1.f;
+                if (grow) {
+                    alpha = ex2(m_ref - mx);
+                    m_ref = mx;
+                    l *= alpha;
+                }
+                if (u > 0 && __any_sync(0xffffffffu, grow)) {
+                    // bring O (P V of the item's tiles so far, complete) to the new max
+                    const bool ok2 = pp_wait(bar(s, kODone), (g - 1) & 1, abort_flag, P.wait_cycles);
+                    if (!__all_sync(0xffffffffu, ok2)) {
+                        alive = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t ro[32];
+                        tmem_ld32(tO + 32 * c, ro);
+                        tmem_wait_ld_dep(ro);
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) ro[jj] = __float_as_uint(__uint_as_float(ro[jj]) * alpha);
+                        tmem_st32(tO + 32 * c, ro);
+                    }
+                }
+                const float mu = m_ref == -INFINITY ? 0.f : m_ref;
+                const uint64_t nmu2 = pack2(-mu, -mu);
+                uint64_t sa = pack2(0.f, 0.f), sb = sa;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t pk[16];
+                    if (need & (1u << q)) {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            float p0, p1;
+                            unpack2(add2(pack2(x[32 * q + 2 * k], x[32 * q + 2 * k + 1]), nmu2), p0, p1);
+                            p0 = ex2(p0);
+                            p1 = ex2(p1);
+                            if (k & 1)
+                                sb = add2(sb, pack2(p0, p1));
+                            else
+                                sa = add2(sa, pack2(p0, p1));
+                            __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
+                            pk[k] = *reinterpret_cast<uint32_t*>(&hv);
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) pk[k] = 0u;
+                    }
+                    tmem_st16(tS + 16 * q, pk);  // P keys 32q .. 32q + 31: columns 16q .. 16q + 15
+                }
+                {
+                    float s0, s1, s2, s3;
+                    unpack2(sa, s0, s1);
+                    unpack2(sb, s2, s3);
+                    l += (s0 + s1) + (s2 + s3);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(s, kPFull));
+            }
+            if (!alive) break;
+            // ---------------------------------------------------------- epilogue
+            const bool ok = pp_wait(bar(s, kODone), (g - 1) & 1, abort_flag, P.wait_cycles);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            float o[D];
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t ro[32];
+                tmem_ld32(tO + 32 * c, ro);
+                tmem_wait_ld_dep(ro);
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) o[32 * c + jj] = __uint_as_float(ro[jj]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(s, kOFree));  // the next item's P V may overwrite O
+            pp_finish<D>(P, sh, it, quarter, t, i, row_ok, m_ref, l, o);
+            __syncwarp();
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && *abort_flag) atomicOr(P.err, kErrTimeout);
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kPpTmemCols);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn pp_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, []() {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [B, H, n, d] bf16 as {d, n, H, B}, box {64, 128, 1, 1}, 128-byte swizzle.
+cudaError_t pp_map4(CUtensorMap* map, const TcOperand& t, int B, int H, int n, int d) {
+    EncodeTiledFn fn = pp_encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const uint64_t sn = (uint64_t)t.s_n * 2;
+    const uint64_t sh = H > 1 ? (uint64_t)t.s_h * 2 : sn * (uint64_t)n;
+    const uint64_t sb = B > 1 ? (uint64_t)t.s_b * 2 : sh * (uint64_t)H;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)H, (cuuint64_t)B};
+    cuuint64_t strides[3] = {sn, sh, sb};
+    cuuint32_t box[4] = {64, 128, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(t.data), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// The same tensor in residue-permuted order: {d, S, G, H, B} (row k S + r at
+// (r, k)), box {64, 1, 128, 1, 1}: one load brings rows r, r + S, ... .
+cudaError_t pp_map5(CUtensorMap* map, const TcOperand& t, int B, int H, int n, int d, int S) {
+    EncodeTiledFn fn = pp_encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const int G = n / S;
+    const uint64_t sn = (uint64_t)t.s_n * 2;
+    const uint64_t sh = H > 1 ? (uint64_t)t.s_h * 2 : sn * (uint64_t)n;
+    const uint64_t sb = B > 1 ? (uint64_t)t.s_b * 2 : sh * (uint64_t)H;
+    cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)S, (cuuint64_t)G, (cuuint64_t)H, (cuuint64_t)B};
+    cuuint64_t strides[4] = {sn, sn * (uint64_t)S, sh, sb};
+    cuuint32_t box[5] = {64, 1, 128, 1, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(t.data), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int D>
+cudaError_t launch_pp_t(const TcOperand& q, const TcOperand& k, const TcOperand& v, const PpParams& p, int num_sms,
+                        cudaStream_t s) {
+    using C = PpCfg<D>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, []() {
+        attr_err = cudaFuncSetAttribute((const void*)k_fwd_pp<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        C::SMEM_BYTES);
+        // setmaxnreg.inc draws on the registers the CTA was launched with: the
+        // split adds up only at exactly 168 per thread (fewer would leave the
+        // softmax warps waiting for registers that never come), so refuse any
+        // other build of the kernel
+        cudaFuncAttributes fa;
+        if (attr_err == cudaSuccess) attr_err = cudaFuncGetAttributes(&fa, (const void*)k_fwd_pp<D>);
+        if (attr_err == cudaSuccess && fa.numRegs * kPpThreads != 128 * kPpRegsLow + 256 * kPpRegsHigh)
+            attr_err = cudaErrorInvalidConfiguration;
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    CUtensorMap mq, mk, mv, mqp, mkp, mvp;
+    cudaError_t e;
+    if ((e = pp_map4(&mq, q, p.B, p.H, p.n, D)) != cudaSuccess) return e;
+    if ((e = pp_map4(&mk, k, p.B, p.H, p.n, D)) != cudaSuccess) return e;
+    if ((e = pp_map4(&mv, v, p.B, p.H, p.n, D)) != cudaSuccess) return e;
+    if (p.mode == 1 && p.S) {
+        if ((e = pp_map5(&mqp, q, p.B, p.H, p.n, D, p.S)) != cudaSuccess) return e;
+        if ((e = pp_map5(&mkp, k, p.B, p.H, p.n, D, p.S)) != cudaSuccess) return e;
+        if ((e = pp_map5(&mvp, v, p.B, p.H, p.n, D, p.S)) != cudaSuccess) return e;
+    } else {
+        mqp = mq;
+        mkp = mk;
+        mvp = mv;
+    }
+    if (p.n_items <= 0) return cudaSuccess;
+    const int64_t grid = p.n_items < num_sms ? p.n_items : num_sms;
+    k_fwd_pp<D><<<(unsigned)grid, kPpThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, mqp, mkp, mvp, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_pp(const TcOperand& q, const TcOperand& k, const TcOperand& v, int d, const PpParams& p,
+                          int num_sms, cudaStream_t s) {
+    switch (d) {
+    case 64: return launch_pp_t<64>(q, k, v, p, num_sms, s);
+    case 128: return launch_pp_t<128>(q, k, v, p, num_sms, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace spattn

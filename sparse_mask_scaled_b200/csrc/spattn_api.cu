@@ -7,9 +7,11 @@
 // device state.
 #include "spattn.h"
 #include "spattn_internal.cuh"
+#include "bsg_plan.cuh"
 
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -22,6 +24,24 @@ using namespace spattn;
 namespace spattn {
 namespace {
 std::atomic<uint64_t> g_launches{0};
+std::atomic<uint64_t> g_allocs{0};
+
+// Every allocation the library makes (stream-ordered pool, device, mapped
+// host) goes through these, which count it for spattn_alloc_count().
+template <typename T>
+cudaError_t lib_malloc_async(T** ptr, size_t bytes, cudaMemPool_t pool, cudaStream_t s) {
+    g_allocs.fetch_add(1, std::memory_order_relaxed);
+    return cudaMallocFromPoolAsync(reinterpret_cast<void**>(ptr), bytes, pool, s);
+}
+template <typename T>
+cudaError_t lib_malloc(T** ptr, size_t bytes) {
+    g_allocs.fetch_add(1, std::memory_order_relaxed);
+    return cudaMalloc(reinterpret_cast<void**>(ptr), bytes);
+}
+cudaError_t lib_host_alloc(void** ptr, size_t bytes, unsigned flags) {
+    g_allocs.fetch_add(1, std::memory_order_relaxed);
+    return cudaHostAlloc(ptr, bytes, flags);
+}
 }  // namespace
 cudaStream_t counted(cudaStream_t s) {
     g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -90,6 +110,16 @@ struct spattn_mask_s {
     int32_t* t_row_ptr;
     int32_t* t_col_idx;
     void* block_t;
+    // interval masks: the long-row list, written when asked for (its count is n_long)
+    void* block_long;
+    // Block + strided + global masks in closed form (bsg_plan.cuh): nothing is
+    // built on the device; the pattern's parameters are the plan. A CSR-built
+    // copy of the same mask (generic) is made on first need: CSR or plan
+    // inspection, the backward pass, fp32 inputs, additive terms, key lengths.
+    bool closed;
+    int32_t bsg_block, bsg_stride, bsg_ng;
+    int64_t closed_tiles;  // tensor-core tiles of one forward per (b, h), over the masks
+    spattn_mask generic;
 };
 
 namespace {
@@ -153,7 +183,7 @@ cudaError_t device_state(int dev, cudaMemPool_t* pool, int* num_sms) {
 template <typename T>
 cudaError_t pool_alloc(T** ptr, int64_t elems, cudaMemPool_t pool, cudaStream_t s) {
     const size_t bytes = (size_t)(elems > 0 ? elems : 1) * sizeof(T);
-    return cudaMallocFromPoolAsync(reinterpret_cast<void**>(ptr), bytes, pool, s);
+    return lib_malloc_async(reinterpret_cast<void**>(ptr), bytes, pool, s);
 }
 
 // Mapped host slots for the totals of an interval-mask build, each with an
@@ -185,13 +215,13 @@ cudaError_t get_slot(int dev, HostSlot* out) {
     (void)cudaGetLastError();  // a not-ready query is not an error of the next call
     if (fr.empty()) {
         void* h = nullptr;
-        cudaError_t e = cudaHostAlloc(&h, sizeof(ItvCounters) * kSlotChunk,
+        cudaError_t e = lib_host_alloc(&h, sizeof(ItvCounters) * kSlotChunk,
                                       cudaHostAllocMapped | cudaHostAllocPortable);
         if (e != cudaSuccess) return e;
         void* d = nullptr;
         if ((e = cudaHostGetDevicePointer(&d, h, 0)) != cudaSuccess) return e;
         unsigned* dn = nullptr;
-        if ((e = cudaMalloc(&dn, sizeof(unsigned) * kSlotChunk)) != cudaSuccess) return e;
+        if ((e = lib_malloc(&dn, sizeof(unsigned) * kSlotChunk)) != cudaSuccess) return e;
         if ((e = cudaMemset(dn, 0, sizeof(unsigned) * kSlotChunk)) != cudaSuccess) return e;
         for (int x = 0; x < kSlotChunk; ++x) {
             HostSlot sl;
@@ -453,7 +483,7 @@ int create_implicit(const spattn_mask_spec& sp, cudaStream_t s, int dev, cudaMem
     const int k_lh = c.add(rows * 8), k_tm = c.add(nblocks * nkt * 4), k_ti = c.add(nblocks * nkt * 4),
               k_nt = c.add(nblocks * 4), k_br = c.add(nblocks * 4), k_bs = c.add(nblocks * sizeof(ItvBlockStat));
     void* blk = nullptr;
-    CUDA_TRY(cudaMallocFromPoolAsync(&blk, c.total, pool, s), "mask allocation");
+    CUDA_TRY(lib_malloc_async(&blk, c.total, pool, s), "mask allocation");
     HostSlot sl;
     cudaError_t e = get_slot(dev, &sl);
     if (e != cudaSuccess) {
@@ -529,9 +559,9 @@ int write_csr(spattn_mask m) {
     Carve ct;
     const int k_cnt = ct.add(rows * 4), k_scan = ct.add(scan_tmp_elems(rows) * 8), k_tot = ct.add(16);
     void *a = nullptr, *t = nullptr, *col = nullptr;
-    cudaError_t e = cudaMallocFromPoolAsync(&a, (size_t)(rows + 1) * 4, pool, s);
-    if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&t, ct.total, pool, s);
-    if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&col, (size_t)(m->nnz > 0 ? m->nnz : 1) * 4, pool, s);
+    cudaError_t e = lib_malloc_async(&a, (size_t)(rows + 1) * 4, pool, s);
+    if (e == cudaSuccess) e = lib_malloc_async(&t, ct.total, pool, s);
+    if (e == cudaSuccess) e = lib_malloc_async(&col, (size_t)(m->nnz > 0 ? m->nnz : 1) * 4, pool, s);
     if (e == cudaSuccess) {
         int64_t* tot = ct.at<int64_t>(t, k_tot);
         e = itv_write_csr(m->lohi, rows, ct.at<int32_t>(t, k_cnt), static_cast<int32_t*>(a),
@@ -577,8 +607,8 @@ int write_plan(spattn_mask m) {
               k_st = ct.add(scan_tmp_elems(scan_rows) * 8);
     void *a = nullptr, *t = nullptr;
     PlanCounters hpc;
-    cudaError_t e = cudaMallocFromPoolAsync(&a, cp.total, pool, s);
-    if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&t, ct.total, pool, s);
+    cudaError_t e = lib_malloc_async(&a, cp.total, pool, s);
+    if (e == cudaSuccess) e = lib_malloc_async(&t, ct.total, pool, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(ct.at<PlanCounters>(t, k_pc), 0, sizeof(PlanCounters), s);
     if (e == cudaSuccess) {
         PlanBuffers pb;
@@ -648,7 +678,7 @@ int write_chunks(spattn_mask m, cudaMemPool_t pool) {
     Carve cp;
     const int k_n = cp.add(nblocks * 4), k_s = cp.add(nblocks * 4), k_e = cp.add(extra.size() * 4);
     void* a = nullptr;
-    CUDA_TRY(cudaMallocFromPoolAsync(&a, cp.total, pool, s), "chunk plan allocation");
+    CUDA_TRY(lib_malloc_async(&a, cp.total, pool, s), "chunk plan allocation");
     cudaError_t e = cudaMemcpyAsync(cp.at<int32_t>(a, k_n), nch.data(), nblocks * 4, cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(cp.at<int32_t>(a, k_s), slot.data(), nblocks * 4, cudaMemcpyHostToDevice, s);
@@ -684,7 +714,7 @@ int write_strided(spattn_mask m, int S, int32_t tile_min_nnz, cudaMemPool_t pool
               k_sp = ct.add((rows + 1) * 4), k_gp = ct.add((rows + 1) * 4), k_sel = ct.add(nblocks * nkt),
               k_st = ct.add(scan_tmp_elems(rows) * 8), k_tot = ct.add(2 * 8), k_err = ct.add(4);
     void* t = nullptr;
-    CUDA_TRY(cudaMallocFromPoolAsync(&t, ct.total, pool, s), "strided split scratch");
+    CUDA_TRY(lib_malloc_async(&t, ct.total, pool, s), "strided split scratch");
     int32_t *cnt_perm = ct.at<int32_t>(t, k_cp), *cnt_row = ct.at<int32_t>(t, k_cr),
             *cnt_reg = ct.at<int32_t>(t, k_cg), *srp = ct.at<int32_t>(t, k_sp), *grp = ct.at<int32_t>(t, k_gp);
     int64_t* tot = ct.at<int64_t>(t, k_tot);
@@ -698,7 +728,7 @@ int write_strided(spattn_mask m, int S, int32_t tile_min_nnz, cudaMemPool_t pool
     if (e == cudaSuccess) e = cudaMemcpyAsync(&htot[0], tot, 8, cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e == cudaSuccess && htot[0] > 0) {
-        e = cudaMallocFromPoolAsync(&sci, (size_t)htot[0] * 4, pool, s);
+        e = lib_malloc_async(&sci, (size_t)htot[0] * 4, pool, s);
         if (e == cudaSuccess)
             e = strided_split_fill(m->res_row_ptr, m->res_col_idx, m->row_ptr, m->col_idx, m->block_tile_off,
                                    m->tile_info, rows, n, S, m->nqb, nkt, nblocks, cnt_row, cnt_reg,
@@ -706,10 +736,10 @@ int write_strided(spattn_mask m, int S, int32_t tile_min_nnz, cudaMemPool_t pool
         if (e == cudaSuccess) e = scan_counts(cnt_reg, rows, grp, ct.at<int64_t>(t, k_st), tot + 1, err, s);
         if (e == cudaSuccess) e = cudaMemcpyAsync(&htot[1], tot + 1, 8, cudaMemcpyDeviceToHost, s);
         if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-        if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&gci, (size_t)(htot[1] > 0 ? htot[1] : 1) * 4, pool, s);
+        if (e == cudaSuccess) e = lib_malloc_async(&gci, (size_t)(htot[1] > 0 ? htot[1] : 1) * 4, pool, s);
         if (e == cudaSuccess)
             e = strided_reg_fill(m->row_ptr, m->col_idx, rows, n, S, m->nqb, nkt, ct.at<uint8_t>(t, k_sel), grp,
-                                 gci, s);
+                                 gci, err, s);
     }
     int r = SPATTN_OK;
     if (e != cudaSuccess) {
@@ -730,6 +760,18 @@ int write_strided(spattn_mask m, int S, int32_t tile_min_nnz, cudaMemPool_t pool
             sp.in_col_idx = gci;
             sp.in_nnz = htot[1];
             r = spattn_create_csr_mask(&sp, s, &m->reg_mask);
+        }
+        if (!r) {  // every row of the regular part must come out at the length its scan allotted
+            unsigned herr = 0;
+            cudaError_t e2 = cudaMemcpyAsync(&herr, err, 4, cudaMemcpyDeviceToHost, s);
+            if (e2 == cudaSuccess) e2 = cudaStreamSynchronize(s);
+            if (e2 != cudaSuccess) r = cuda_fail(e2, "strided split check");
+            else if (herr & kBuildBadRowPtr) r = fail(SPATTN_ERR_BAD_CSR, "strided split: row lengths disagree");
+            if (r) {
+                spattn_destroy_mask(m->str_mask);
+                spattn_destroy_mask(m->reg_mask);
+                m->str_mask = m->reg_mask = nullptr;
+            }
         }
         if (!r && !(m->str_mask->has_plan && m->reg_mask->has_plan)) {  // nothing to gain: keep the mask as is
             spattn_destroy_mask(m->str_mask);
@@ -766,7 +808,7 @@ int fwd_strided(const spattn_tensor* q, const spattn_tensor* k, const spattn_ten
               k_q = c.add(in_place ? 0 : elems * 2), k_k = c.add(in_place ? 0 : elems * 2),
               k_v = c.add(in_place ? 0 : elems * 2);
     void* t = nullptr;
-    CUDA_TRY(cudaMallocFromPoolAsync(&t, c.total, pool, s), "strided forward scratch");
+    CUDA_TRY(lib_malloc_async(&t, c.total, pool, s), "strided forward scratch");
     auto tensor = [&](int key) {  // contiguous [B, H, n, d] bf16 scratch
         spattn_tensor x;
         memset(&x, 0, sizeof x);
@@ -784,7 +826,9 @@ int fwd_strided(const spattn_tensor* q, const spattn_tensor* k, const spattn_ten
     };
     const spattn_tensor to = tensor(k_o);
     float* l2 = c.at<float>(t, k_l2);
-    float* l1 = lse ? lse : c.at<float>(t, k_l1);
+    // the regular part's lse always goes to scratch: the merge reads it and
+    // writes the caller's lse, and the two must not alias
+    float* l1 = c.at<float>(t, k_l1);
     int r = SPATTN_OK;
     if (in_place) {
         FwdParams p2 = p;
@@ -859,7 +903,7 @@ int launch_tc(const FwdParams& p, int d, spattn_mask m, int dev, const int32_t* 
         const int64_t bh = (int64_t)p.B * p.H, nblocks = (int64_t)m->num_masks * m->nqb;
         Carve cp;
         const int k_w = cp.add((size_t)bh * m->n_slots * (d + 2) * kTileM * 4), k_c = cp.add(bh * nblocks * 4);
-        CUDA_TRY(cudaMallocFromPoolAsync(&cws, cp.total, pool, s), "chunk workspace");
+        CUDA_TRY(lib_malloc_async(&cws, cp.total, pool, s), "chunk workspace");
         cudaError_t e = cudaMemsetAsync(cp.at<unsigned>(cws, k_c), 0, bh * nblocks * 4, s);
         if (e != cudaSuccess) {
             cudaFreeAsync(cws, s);
@@ -878,6 +922,103 @@ int launch_tc(const FwdParams& p, int d, spattn_mask m, int dev, const int32_t* 
         ov{p.v, p.v_sn, p.v_sh, p.v_sb};
     const cudaError_t e = launch_fwd_tc(oq, ok, ov, d, tp, s);
     if (cws) cudaFreeAsync(cws, s);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core kernel launch");
+    return SPATTN_OK;
+}
+
+// Limit of every wait in the persistent tile kernel, in SM cycles: about one
+// second, unless SPATTN_DEBUG_WAIT_CYCLES gives another (tests use a tiny one
+// to make the waits expire and check the error path).
+long long pp_wait_cycles() {
+    const char* e = getenv("SPATTN_DEBUG_WAIT_CYCLES");
+    if (e && *e) {
+        const long long v = atoll(e);
+        if (v >= 0) return v;
+    }
+    return 2000000000LL;
+}
+
+void pp_common(PpParams& pp, const FwdParams& p, unsigned* ef) {
+    pp.B = p.B;
+    pp.H = p.H;
+    pp.n = p.n;
+    pp.nqb = (p.n + kTileM - 1) / kTileM;
+    pp.nkt = (p.n + kTileN - 1) / kTileN;
+    pp.out = p.out;
+    pp.o_sb = p.o_sb;
+    pp.o_sh = p.o_sh;
+    pp.o_sn = p.o_sn;
+    pp.lse = p.lse;
+    pp.qk_scale_log2 = p.qk_scale_log2;
+    pp.err = ef;
+    pp.wait_cycles = pp_wait_cycles();
+    pp.chunk_tiles = kChunkTiles;
+}
+
+// Forward over a block + strided + global mask in closed form: one launch of
+// the persistent tile kernel over the regular and the residue-permuted blocks.
+// Per call it takes the partial states of split blocks and of rows met by both
+// kinds of block from the pool, and clears their counts.
+int fwd_closed(const FwdParams& p, int d, spattn_mask m, cudaStream_t s, cudaMemPool_t pool, int dev, int sms) {
+    unsigned* ef = nullptr;
+    int r = err_flags_ptr(dev, &ef);
+    if (r) return r;
+    const bsg::Shape sh = bsg::shape(p.n, m->bsg_block, m->bsg_stride, m->bsg_ng, kChunkTiles);
+    const int64_t bh = (int64_t)p.B * p.H, rows = bh * p.n;
+    const bool chunks = sh.nch > 1, partner = sh.G > 0;
+    Carve c;
+    const int k_cws = c.add(chunks ? (size_t)bh * sh.nch * (d + 2) * kTileM * 4 : 0),
+              k_pml = c.add(partner ? (size_t)rows * 2 * 4 : 0), k_pacc = c.add(partner ? (size_t)rows * d * 4 : 0),
+              k_cnt = c.add((size_t)bh * 4 * 4 + (partner ? (size_t)rows * 4 : 0));
+    void* ws = nullptr;
+    CUDA_TRY(lib_malloc_async(&ws, c.total, pool, s), "tile-kernel workspace");
+    cudaError_t e = cudaMemsetAsync(c.at<uint8_t>(ws, k_cnt), 0, (size_t)bh * 4 * 4 + (partner ? (size_t)rows * 4 : 0), s);
+    if (e == cudaSuccess) {
+        PpParams pp;
+        memset(&pp, 0, sizeof pp);
+        pp_common(pp, p, ef);
+        pp.num_masks = m->num_masks;
+        pp.mode = 1;
+        pp.n_items = bh * sh.items_per_head;
+        pp.blk = m->bsg_block;
+        pp.S = m->bsg_stride;
+        pp.ng = m->bsg_ng;
+        pp.cws = chunks ? c.at<float>(ws, k_cws) : nullptr;
+        pp.ccnt = c.at<unsigned>(ws, k_cnt);
+        pp.pcnt = partner ? c.at<unsigned>(ws, k_cnt) + bh * 4 : nullptr;
+        pp.pml = partner ? c.at<float>(ws, k_pml) : nullptr;
+        pp.pacc = partner ? c.at<float>(ws, k_pacc) : nullptr;
+        const TcOperand oq{p.q, p.q_sn, p.q_sh, p.q_sb}, ok{p.k, p.k_sn, p.k_sh, p.k_sb},
+            ov{p.v, p.v_sn, p.v_sh, p.v_sb};
+        e = launch_fwd_pp(oq, ok, ov, d, pp, sms, s);
+    }
+    cudaFreeAsync(ws, s);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core kernel (closed-form mask)");
+    return SPATTN_OK;
+}
+
+// The persistent tile kernel over an interval mask's tiles (d = 64 or 128,
+// no additive terms, no key lengths); blk_res: the gather kernel ran first and
+// left partial states in p.ws_ml / p.ws_acc for the flagged blocks.
+int launch_pp_interval(const FwdParams& p, int d, spattn_mask m, int dev, int sms, const int32_t* blk_res,
+                       cudaStream_t s) {
+    unsigned* ef = nullptr;
+    int r = err_flags_ptr(dev, &ef);
+    if (r) return r;
+    PpParams pp;
+    memset(&pp, 0, sizeof pp);
+    pp_common(pp, p, ef);
+    pp.num_masks = m->num_masks;
+    pp.mode = 0;
+    pp.n_items = (int64_t)p.B * p.H * m->nqb;
+    pp.itv_lohi = m->lohi;
+    pp.itv_tiles = m->itv_tiles;
+    pp.itv_ntiles = m->itv_ntiles;
+    pp.blk_res = blk_res;
+    pp.ws_ml = p.ws_ml;
+    pp.ws_acc = p.ws_acc;
+    const TcOperand oq{p.q, p.q_sn, p.q_sh, p.q_sb}, ok{p.k, p.k_sn, p.k_sh, p.k_sb}, ov{p.v, p.v_sn, p.v_sh, p.v_sb};
+    const cudaError_t e = launch_fwd_pp(oq, ok, ov, d, pp, sms, s);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core kernel launch");
     return SPATTN_OK;
 }
@@ -923,7 +1064,10 @@ int fwd_interval(FwdParams& p, int dtype, int d, spattn_mask m, cudaStream_t s, 
             return cuda_fail(e, "interval gather kernel launch");
         }
     }
-    r = launch_tc(p, d, m, dev, gather ? m->blk_res : nullptr, s);
+    if ((d == 64 || d == 128) && !p.has_extra && !p.seqlen_k)
+        r = launch_pp_interval(p, d, m, dev, num_sms, gather ? m->blk_res : nullptr, s);
+    else
+        r = launch_tc(p, d, m, dev, gather ? m->blk_res : nullptr, s);
     if (ws) cudaFreeAsync(ws, s);
     return r;
 }
@@ -943,9 +1087,9 @@ int write_transpose(spattn_mask m) {
     Carve c;
     const int k_rp = c.add((rows + 1) * 4), k_ci = c.add((m->nnz > 0 ? m->nnz : 1) * 4);
     void *blk = nullptr, *scratch = nullptr;
-    cudaError_t e = cudaMallocFromPoolAsync(&blk, c.total, pool, s);
+    cudaError_t e = lib_malloc_async(&blk, c.total, pool, s);
     if (e == cudaSuccess)
-        e = cudaMallocFromPoolAsync(&scratch, (size_t)transpose_scratch_words(rows, m->nnz) * 4, pool, s);
+        e = lib_malloc_async(&scratch, (size_t)transpose_scratch_words(rows, m->nnz) * 4, pool, s);
     if (e == cudaSuccess)
         e = build_transpose(m->row_ptr, m->col_idx, m->n, m->num_masks, m->nnz, c.at<int32_t>(blk, k_rp),
                             c.at<int32_t>(blk, k_ci), static_cast<int32_t*>(scratch), s);
@@ -960,17 +1104,78 @@ int write_transpose(spattn_mask m) {
     return SPATTN_OK;
 }
 
-}  // namespace
+// A block + strided + global mask in closed form: no device work at all. Its
+// size is counted here from the pattern (row i of one mask: every key for a
+// global row, else the union of its block, its strided keys and the global
+// keys), and the forward pass derives tiles and bits from the parameters.
+int create_closed(const spattn_mask_spec& sp, cudaStream_t s, int dev, spattn_mask* out) {
+    const bsg::Shape sh = bsg::shape(sp.n, sp.block, sp.stride, sp.n_global, kChunkTiles);
+    const int64_t n = sp.n, ng = sp.n_global;
+    int64_t per = 0, n_long = 0;
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t c;
+        if (i < ng) {
+            c = n;
+        } else {
+            const int64_t blk = sp.block;
+            const int64_t strided = sp.stride ? n / sp.stride : 0;  // keys j = i (mod stride)
+            c = blk + strided + ng;
+            if (blk > 0 && sp.stride) c -= 1;                      // j = i: block and strided
+            if (blk > 0 && ng > 0) {                                // block keys below ng
+                const int64_t b0 = (i / blk) * blk;
+                c -= std::max<int64_t>(0, std::min(b0 + blk, ng) - b0);
+            }
+            if (sp.stride && (i % sp.stride) < ng) c -= 1;         // the strided key below ng
+        }
+        per += c;
+        n_long += c > kLongRowThreshold ? 1 : 0;
+    }
+    // tiles of one forward per (b, h): chunks of block 0, further regular
+    // blocks, permuted blocks (each over every permuted key tile)
+    int64_t tiles = 0;
+    for (int64_t x = 0; x < sh.items_per_head; ++x) tiles += bsg::item(sh, x).T;
+    spattn_mask m = new spattn_mask_s;
+    memset(m, 0, sizeof *m);
+    m->device = dev;
+    m->stream = s;
+    m->n = sp.n;
+    m->num_masks = sp.num_masks;
+    m->kind = sp.kind;
+    m->nnz = per * sp.num_masks;
+    m->n_long = n_long * sp.num_masks;
+    m->nqb = sh.nqb;
+    m->closed = true;
+    m->bsg_block = sp.block;
+    m->bsg_stride = sp.stride;
+    m->bsg_ng = sp.n_global;
+    m->closed_tiles = tiles * sp.num_masks;
+    *out = m;
+    return SPATTN_OK;
+}
 
-extern "C" {
+int create_mask(const spattn_mask_spec* spec, void* stream_v, spattn_mask* out, bool allow_closed);
 
-const char* spattn_last_error(void) { return g_msg; }
+// The CSR-built copy of a closed-form mask, made on first need on the mask's
+// stream (synchronises it, like any CSR build).
+int ensure_generic(spattn_mask m) {
+    if (m->generic) return SPATTN_OK;
+    spattn_mask_spec sp;
+    memset(&sp, 0, sizeof sp);
+    sp.kind = SPATTN_MASK_BLOCK_STRIDED_GLOBAL;
+    sp.n = m->n;
+    sp.num_masks = m->num_masks;
+    sp.block = m->bsg_block;
+    sp.stride = m->bsg_stride;
+    sp.n_global = m->bsg_ng;
+    int prev = -1;
+    cudaGetDevice(&prev);
+    if (prev != m->device) cudaSetDevice(m->device);
+    const int r = create_mask(&sp, m->stream, &m->generic, false);
+    if (prev >= 0 && prev != m->device) cudaSetDevice(prev);
+    return r;
+}
 
-int spattn_version(void) { return 100; /* 0.1.0 */ }
-
-uint64_t spattn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
-
-int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_mask* out) {
+int create_mask(const spattn_mask_spec* spec, void* stream_v, spattn_mask* out, bool allow_closed) {
     g_msg[0] = 0;
     if (!out) return fail(SPATTN_ERR_INVALID_ARG, "out is NULL");
     *out = nullptr;
@@ -1005,6 +1210,9 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
     const int nqb_i = (sp.n + kTileM - 1) / kTileM;
     if (implicit_kind(sp.kind) && nqb_i <= kItvMaxKeyTiles && (int64_t)sp.num_masks * nqb_i <= kItvMaxBlocks)
         return create_implicit(sp, s, dev, pool, out);
+    if (allow_closed && sp.kind == SPATTN_MASK_BLOCK_STRIDED_GLOBAL && sp.tile_min_nnz == 0 &&
+        bsg::supported(sp.n, sp.block, sp.stride, sp.n_global))
+        return create_closed(sp, s, dev, out);
 
     BuildSpec bs;
     bs.kind = sp.kind;
@@ -1044,8 +1252,8 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
               k_st = ct.add(plan_possible ? scan_tmp_elems(scan_rows) * 8 : 0),
               k_rc = ct.add(plan_possible ? rows * 4 : 0);
     void *blk_a = nullptr, *blk_t = nullptr;
-    cudaError_t e = cudaMallocFromPoolAsync(&blk_a, ca.total, pool, s);
-    if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&blk_t, ct.total, pool, s);
+    cudaError_t e = lib_malloc_async(&blk_a, ca.total, pool, s);
+    if (e == cudaSuccess) e = lib_malloc_async(&blk_t, ct.total, pool, s);
     if (e != cudaSuccess) {
         if (blk_a) cudaFreeAsync(blk_a, s);
         return cuda_fail(e, "mask allocation");
@@ -1091,7 +1299,7 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
     memset(&pb, 0, sizeof pb);
     PlanCounters hpc;
     memset(&hpc, 0, sizeof hpc);
-    e = cudaMallocFromPoolAsync(&m->block_col, (size_t)(hinfo.nnz > 0 ? hinfo.nnz : 1) * 4, pool, s);
+    e = lib_malloc_async(&m->block_col, (size_t)(hinfo.nnz > 0 ? hinfo.nnz : 1) * 4, pool, s);
     if (e == cudaSuccess) {
         m->col_idx = static_cast<int32_t*>(m->block_col);
         e = build_phase2(bs, row_ptr, coo_tmp, m->col_idx,
@@ -1104,7 +1312,7 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
         const int k_bto = cp.add((nblocks + 1) * 4), k_ti = cp.add(pb.tile_cap * 4),
                   k_tb = cp.add(pb.tile_cap * kTileM * 16), k_rrp = cp.add((rows + 1) * 4),
                   k_rci = cp.add(hinfo.nnz * 4), k_rl = cp.add(rows * 4);
-        e = cudaMallocFromPoolAsync(&m->block_plan, cp.total, pool, s);
+        e = lib_malloc_async(&m->block_plan, cp.total, pool, s);
         if (e == cudaSuccess) {
             m->block_tile_off = pb.block_tile_off = cp.at<int32_t>(m->block_plan, k_bto);
             m->tile_info = pb.tile_info = cp.at<int32_t>(m->block_plan, k_ti);
@@ -1149,11 +1357,33 @@ int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_
     return SPATTN_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+const char* spattn_last_error(void) { return g_msg; }
+
+int spattn_version(void) { return 100; /* 0.1.0 */ }
+
+uint64_t spattn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+uint64_t spattn_alloc_count(void) { return g_allocs.load(std::memory_order_relaxed); }
+
+int spattn_create_csr_mask(const spattn_mask_spec* spec, void* stream_v, spattn_mask* out) {
+    return create_mask(spec, stream_v, out, true);
+}
+
 int spattn_mask_copy_plan(spattn_mask m, int32_t* block_tile_off, int32_t* tile_info,
                           uint32_t* tile_bits, int32_t* res_row_ptr, int32_t* res_col_idx,
                           void* stream_v) {
     g_msg[0] = 0;
     if (!m) return fail(SPATTN_ERR_INVALID_ARG, "mask is NULL");
+    if (m->closed) {  // the CSR-built copy's plan
+        const int rg = ensure_generic(m);
+        if (rg) return rg;
+        return spattn_mask_copy_plan(m->generic, block_tile_off, tile_info, tile_bits, res_row_ptr, res_col_idx,
+                                     stream_v);
+    }
     int r = write_plan(m);
     if (r) return r;
     if (!m->has_plan || m->n_tiles == 0) return fail(SPATTN_ERR_INVALID_ARG, "the mask has no tile plan");
@@ -1181,6 +1411,11 @@ int spattn_mask_plan_info(spattn_mask m, int64_t* n_tiles, int64_t* residual_nnz
                           int64_t* n_mixed_rows) {
     g_msg[0] = 0;
     if (!m) return fail(SPATTN_ERR_INVALID_ARG, "mask is NULL");
+    if (m->closed) {
+        const int rg = ensure_generic(m);
+        if (rg) return rg;
+        return spattn_mask_plan_info(m->generic, n_tiles, residual_nnz, n_mixed_rows);
+    }
     int r = read_counters(m, true);
     if (r == SPATTN_OK && n_mixed_rows) r = write_plan(m);
     if (r) return r;
@@ -1190,20 +1425,77 @@ int spattn_mask_plan_info(spattn_mask m, int64_t* n_tiles, int64_t* residual_nnz
     return SPATTN_OK;
 }
 
+int spattn_mask_tile_count(spattn_mask m, int64_t* tiles) {
+    g_msg[0] = 0;
+    if (!m || !tiles) return fail(SPATTN_ERR_INVALID_ARG, "mask or tiles is NULL");
+    if (m->closed) {
+        *tiles = m->closed_tiles;
+        return SPATTN_OK;
+    }
+    const int r = read_counters(m, true);
+    if (r) return r;
+    if (m->str_mask)  // the residue-permuted part and the rest, each with its own plan
+        *tiles = m->str_mask->n_tiles + m->reg_mask->n_tiles;
+    else
+        *tiles = m->has_plan ? m->n_tiles : 0;
+    return SPATTN_OK;
+}
+
 int spattn_mask_info(spattn_mask m, int32_t* n, int32_t* num_masks, int64_t* nnz,
                      const int32_t** row_ptr, const int32_t** col_idx, int64_t* n_long) {
     g_msg[0] = 0;
     if (!m) return fail(SPATTN_ERR_INVALID_ARG, "mask is NULL");
     int r = SPATTN_OK;
     if (nnz || n_long) r = read_counters(m, true);
-    if (r == SPATTN_OK && (row_ptr || col_idx)) r = write_csr(m);
+    if (r == SPATTN_OK && (row_ptr || col_idx)) r = m->closed ? ensure_generic(m) : write_csr(m);
     if (r) return r;
+    const spattn_mask c = m->closed ? m->generic : m;  // who holds the CSR
     if (n) *n = m->n;
     if (num_masks) *num_masks = m->num_masks;
     if (nnz) *nnz = m->nnz;
-    if (row_ptr) *row_ptr = m->row_ptr;
-    if (col_idx) *col_idx = m->col_idx;
+    if (row_ptr) *row_ptr = c->row_ptr;
+    if (col_idx) *col_idx = c->col_idx;
     if (n_long) *n_long = m->n_long;
+    return SPATTN_OK;
+}
+
+int spattn_mask_csr(spattn_mask m, const int32_t** row_ptr, const int32_t** col_idx, int64_t* nnz_total) {
+    g_msg[0] = 0;
+    if (!m) return fail(SPATTN_ERR_INVALID_ARG, "mask is NULL");
+    return spattn_mask_info(m, nullptr, nullptr, nnz_total, row_ptr, col_idx, nullptr);
+}
+
+int spattn_mask_copy_long_rows(spattn_mask m, int32_t* dst, void* stream_v) {
+    g_msg[0] = 0;
+    if (!m || !dst) return fail(SPATTN_ERR_INVALID_ARG, "mask or dst is NULL");
+    if (m->closed) {
+        const int rg = ensure_generic(m);
+        if (rg) return rg;
+        return spattn_mask_copy_long_rows(m->generic, dst, stream_v);
+    }
+    int r = read_counters(m, true);
+    if (r) return r;
+    if (m->implicit && !m->long_rows && m->n_long > 0) {  // list them from the CSR, once
+        if ((r = write_csr(m))) return r;
+        cudaMemPool_t pool;
+        CUDA_TRY(device_state(m->device, &pool, nullptr), "memory pool");
+        const int64_t rows = (int64_t)m->n * m->num_masks;
+        int32_t* blk = nullptr;  // [0]: count, [1 ..]: rows
+        CUDA_TRY(lib_malloc_async(&blk, (size_t)(rows + 1) * 4, pool, m->stream), "long-row list");
+        cudaError_t e = cudaMemsetAsync(blk, 0, 4, m->stream);
+        if (e == cudaSuccess) e = launch_classify_long_rows(m->row_ptr, rows, m->nnz, blk + 1, blk, m->stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(m->stream);
+        if (e != cudaSuccess) {
+            cudaFreeAsync(blk, m->stream);
+            return cuda_fail(e, "listing long rows");
+        }
+        m->block_long = blk;
+        m->long_rows = blk + 1;
+    }
+    if (m->n_long > 0)
+        CUDA_TRY(cudaMemcpyAsync(dst, m->long_rows, (size_t)m->n_long * 4, cudaMemcpyDefault,
+                                 (cudaStream_t)stream_v),
+                 "long-row copy");
     return SPATTN_OK;
 }
 
@@ -1211,6 +1503,11 @@ int spattn_mask_copy_csr(spattn_mask m, int32_t* row_ptr_dst, int32_t* col_idx_d
                          void* stream_v) {
     g_msg[0] = 0;
     if (!m) return fail(SPATTN_ERR_INVALID_ARG, "mask is NULL");
+    if (m->closed && (row_ptr_dst || col_idx_dst)) {
+        const int r = ensure_generic(m);
+        if (r) return r;
+        return spattn_mask_copy_csr(m->generic, row_ptr_dst, col_idx_dst, stream_v);
+    }
     if (row_ptr_dst || col_idx_dst) {
         const int r = write_csr(m);
         if (r) return r;
@@ -1240,7 +1537,9 @@ int spattn_destroy_mask(spattn_mask m) {
     free_plan(m);
     if (m->str_mask) spattn_destroy_mask(m->str_mask);
     if (m->reg_mask) spattn_destroy_mask(m->reg_mask);
+    if (m->generic) spattn_destroy_mask(m->generic);
     if (m->block_itv && (e2 = cudaFreeAsync(m->block_itv, m->stream)) != cudaSuccess) e = e2;
+    if (m->block_long && (e2 = cudaFreeAsync(m->block_long, m->stream)) != cudaSuccess) e = e2;
     if (m->block_t && (e2 = cudaFreeAsync(m->block_t, m->stream)) != cudaSuccess) e = e2;
     if (m->cnt_host) {
         HostSlot sl;
@@ -1329,6 +1628,12 @@ int spattn_fwd_mask_kpad(const spattn_tensor* q, const spattn_tensor* k, const s
     CUDA_TRY(device_state(dev, &pool, &sms), "memory pool");
     p.num_masks = mask->num_masks;
     p.long_count_dev = nullptr;
+    if (mask->closed) {
+        if (dtype == 0 && !seqlen_k && !p.has_extra && (d == 64 || d == 128))
+            return fwd_closed(p, d, mask, s, pool, dev, sms);
+        if ((r = ensure_generic(mask))) return r;
+        return spattn_fwd_mask_kpad(q, k, v, mask->generic, seqlen_k, add_mask, bias, scale, out, lse, stream_v);
+    }
     if (mask->implicit) return fwd_interval(p, dtype, d, mask, s, pool, dev, sms);
     if (mask->str_mask && dtype == 0 && !seqlen_k && !p.has_extra)
         return fwd_strided(q, k, v, mask, scale, out, lse, s, p, d, pool, dev);
@@ -1443,6 +1748,11 @@ int spattn_bwd_mask(const spattn_tensor* q, const spattn_tensor* k, const spattn
     if (dev != mask->device) return fail(SPATTN_ERR_INVALID_ARG, "mask lives on another device");
     cudaMemPool_t pool;
     CUDA_TRY(device_state(dev, &pool, nullptr), "memory pool");
+    if (mask->closed) {  // the backward walks the CSR-built copy
+        if ((r = ensure_generic(mask))) return r;
+        return spattn_bwd_mask(q, k, v, mask->generic, add_mask, bias, scale, out, lse, dout, dq, dk, dv, dbias,
+                               stream_v);
+    }
     if ((r = write_transpose(mask))) return r;
     // the transpose was written on the mask's stream; order this stream after it
     if (mask->stream != s) CUDA_TRY(cudaStreamSynchronize(mask->stream), "mask stream");
@@ -1564,6 +1874,8 @@ int spattn_fwd_noalloc(const spattn_tensor* q, const spattn_tensor* k, const spa
     p.long_count_host = -1;
     return launch_fwd(p, dtype, d, sms, s);
 }
+
+int spattn_check_device_error(void* stream_v) { return spattn_device_error(stream_v, nullptr); }
 
 int spattn_device_error(void* stream_v, uint32_t* flags) {
     g_msg[0] = 0;

@@ -158,6 +158,40 @@ struct TcParams {
 };
 cudaError_t launch_fwd_tc(const TcOperand& q, const TcOperand& k, const TcOperand& v, int d,
                           const TcParams& p, cudaStream_t stream);
+
+// Persistent ping-pong tensor-core kernel (fwd_pp.cu), d = 64 or 128, bf16,
+// no additive terms, no key lengths.
+struct PpParams {
+    int B, H, n, num_masks, nqb, nkt;
+    int mode;         // 0: interval-mask tiles; 1: block + strided + global in closed form
+    int64_t n_items;  // work items (mode 0: B*H*nqb; mode 1: B*H*items per head)
+    // mode 0: the interval mask's runs and tile lists, and the gather kernel's
+    // partial states of rows in flagged blocks (blk_res; ws_ml / ws_acc)
+    const int2* itv_lohi;
+    const int32_t* itv_tiles;   // [blocks][nkt]: key tile | kTileDenseBit
+    const int32_t* itv_ntiles;  // [blocks]
+    const int32_t* blk_res;     // nullable
+    const float* ws_ml;
+    const float* ws_acc;
+    // mode 1: pattern parameters (bsg_plan.cuh), chunk partial states
+    // [B*H][nch][d + 2][128] with counts [B*H][4] (zero before the launch),
+    // partner states [B*H*n][2] (m, l) and [B*H*n][d] (O) with counts
+    // [B*H*n] (zero before the launch)
+    int blk, S, ng, chunk_tiles;
+    float* cws;
+    unsigned* ccnt;
+    float* pml;
+    float* pacc;
+    unsigned* pcnt;
+    void* out;
+    int64_t o_sb, o_sh, o_sn;
+    float* lse;  // nullable
+    float qk_scale_log2;
+    unsigned* err;
+    long long wait_cycles;  // limit of every wait (SM cycles)
+};
+cudaError_t launch_fwd_pp(const TcOperand& q, const TcOperand& k, const TcOperand& v, int d, const PpParams& p,
+                          int num_sms, cudaStream_t stream);
 cudaError_t error_flag_address(unsigned** p);
 // Every kernel launch of the library passes its stream through counted(),
 // which adds one to the count spattn_launch_count() reports.
@@ -334,9 +368,11 @@ cudaError_t strided_split_fill(const int32_t* res_row_ptr, const int32_t* res_co
                                const int32_t* cnt_row, int32_t* cnt_reg, uint8_t* sel,
                                const int32_t* str_row_ptr, int32_t* str_col_idx, cudaStream_t s);
 // The regular part: every entry of the mask but those moved to the permuted one.
+// A row whose kept entries do not fill exactly its allotted slots raises
+// kBuildBadRowPtr in *err.
 cudaError_t strided_reg_fill(const int32_t* row_ptr, const int32_t* col_idx, int64_t rows, int n, int S, int nqb,
                              int nkt, const uint8_t* sel, const int32_t* reg_row_ptr, int32_t* reg_col_idx,
-                             cudaStream_t s);
+                             unsigned* err, cudaStream_t s);
 // dst (contiguous [B, H, n, d] bf16) row perm(i) = src (strides in elements) row i.
 cudaError_t strided_permute_rows(const void* src, int64_t s_b, int64_t s_h, int64_t s_n, void* dst, int B, int H,
                                  int n, int d, int S, cudaStream_t s);

@@ -62,7 +62,7 @@ __global__ void k_reg_count(const int32_t* rp, const int32_t* cnt_row, int64_t r
 // tiles. One warp per row, 32 entries at a time, compacted by ballot (rows of
 // global tokens hold every key).
 __global__ void k_reg_fill(const int32_t* rp, const int32_t* ci, int64_t rows, int n, int S, int nqb, int nkt,
-                           const uint8_t* sel, const int32_t* grp, int32_t* gci) {
+                           const uint8_t* sel, const int32_t* grp, int32_t* gci, unsigned* err) {
     const int64_t r = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (r >= rows) return;
@@ -85,6 +85,9 @@ __global__ void k_reg_fill(const int32_t* rp, const int32_t* ci, int64_t rows, i
         if (keep && at < o_end) gci[at] = j;
         o += __popc(bal);
     }
+    // the entries kept must fill exactly the slots the count pass allotted
+    // (k_str_count and this selection agree), else the part is unusable
+    if (lane == 0 && o != o_end) atomicOr(err, (unsigned)kBuildBadRowPtr);
 }
 
 // dst[b, h, perm(i), :] = src[b, h, i, :] (bf16; dst contiguous [B, H, n, d]),
@@ -167,9 +170,10 @@ cudaError_t strided_split_fill(const int32_t* rrp, const int32_t* rci, const int
 }
 
 cudaError_t strided_reg_fill(const int32_t* rp, const int32_t* ci, int64_t rows, int n, int S, int nqb, int nkt,
-                             const uint8_t* sel, const int32_t* grp, int32_t* gci, cudaStream_t s) {
+                             const uint8_t* sel, const int32_t* grp, int32_t* gci, unsigned* err, cudaStream_t s) {
     if (rows == 0) return cudaSuccess;
-    k_reg_fill<<<blocks_for(rows * 32, 256), 256, 0, counted(s)>>>(rp, ci, rows, n, S, nqb, nkt, sel, grp, gci);
+    k_reg_fill<<<blocks_for(rows * 32, 256), 256, 0, counted(s)>>>(rp, ci, rows, n, S, nqb, nkt, sel, grp, gci,
+                                                                   err);
     return cudaGetLastError();
 }
 

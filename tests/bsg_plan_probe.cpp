@@ -1,0 +1,51 @@
+// Test driver for the closed-form block + strided + global tile plan
+// (sparse_mask_scaled_b200/csrc/bsg_plan.cuh), built for the host by
+// tests/test_bsg_plan_cpu.py. For the parameters on the command line it walks
+// every work item of one (b, h), every tile and every row's bits, and writes
+// to stdout, as raw bytes: the n x n count of how many times each entry (i, j)
+// is computed (uint8), the per-row "has entries in a permuted block" flag
+// computed from the bits (uint8 [n]) and the one bsg::has_perm reports (uint8
+// [n]). Exit status 2 when the parameters are outside the closed form.
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <vector>
+
+#include "bsg_plan.cuh"
+
+using namespace spattn::bsg;
+
+int main(int argc, char** argv) {
+    if (argc != 6) return 1;
+    const int n = atoi(argv[1]), block = atoi(argv[2]), S = atoi(argv[3]), ng = atoi(argv[4]),
+              chunk = atoi(argv[5]);
+    if (!supported(n, block, S, ng)) return 2;
+    const Shape s = shape(n, block, S, ng, chunk);
+    std::vector<uint8_t> cnt((size_t)n * n, 0), perm_rows(n, 0), has(n, 0);
+    for (int64_t x = 0; x < s.items_per_head; ++x) {
+        const Item it = item(s, x);
+        if (it.bh != 0) return 3;
+        for (int u = 0; u < it.T; ++u) {
+            const int kt = key_tile(s, it, u);
+            for (int t = 0; t < kTile; ++t) {
+                uint32_t w[4];
+                row_bits(s, it, kt, t, w);
+                const int i = row_of(s, it, t);
+                for (int c = 0; c < kTile; ++c) {
+                    if (!((w[c / 32] >> (c % 32)) & 1u)) continue;
+                    if (i < 0 || i >= n) return 4;  // a bit on a row that does not exist
+                    const int j = it.perm ? (kt * kTile + c) * kTile + it.qb : kt * kTile + c;
+                    if (j < 0 || j >= n) return 5;
+                    if (it.perm) perm_rows[i] = 1;
+                    uint8_t& e = cnt[(size_t)i * n + j];
+                    if (e < 255) ++e;
+                }
+            }
+        }
+    }
+    for (int i = 0; i < n; ++i) has[i] = has_perm(s, i) ? 1 : 0;
+    fwrite(cnt.data(), 1, cnt.size(), stdout);
+    fwrite(perm_rows.data(), 1, n, stdout);
+    fwrite(has.data(), 1, n, stdout);
+    return 0;
+}

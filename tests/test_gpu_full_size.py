@@ -1,8 +1,9 @@
 """The five workloads at full size, in the launch configuration the benchmark
 times (mask built on the device, then the mask-handle forward): the whole CSR is
-compared bit-exactly with the oracle's brute-force mask, and the outputs of a
-sample of rows (random rows plus the first and last rows of every (b, h) and
-the rows of the block-per-row kernel) with the oracle's values for those rows."""
+compared bit-exactly with the oracle's brute-force mask, and the outputs of
+every row of two (b, h) heads (the first and the last), plus a sample of other
+rows (random rows, the first and last rows of every (b, h), the rows of the
+block-per-row kernel), with the oracle's values for those rows."""
 import numpy as np
 import pytest
 
@@ -22,6 +23,8 @@ def _sample_rows(wl, rp, count, seed):
     B, H, n = wl.B, wl.H, wl.n
     total = B * H * n
     rows = set(rng.integers(0, total, size=count).tolist())
+    for bh in (0, B * H - 1):                      # two whole heads
+        rows.update(range(bh * n, (bh + 1) * n))
     for bh in range(0, B * H, max(1, (B * H) // 8)):
         rows.update([bh * n, bh * n + n - 1])
     lens = np.diff(rp)

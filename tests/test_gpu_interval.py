@@ -90,6 +90,7 @@ def test_long_interval_rows(dtype, thr):
         out, lse = sp.spattn_fwd_mask(torch_tensor(q), torch_tensor(k), torch_tensor(v), m,
                                       scale=1 / math.sqrt(d))
         torch.cuda.synchronize()
+        assert np.array_equal(m.long_rows().cpu().numpy(), np.nonzero(np.diff(rp) > 1024)[0])
     assert_close(to_f64(out).reshape(-1, d), to_f64(lse), out_ref.reshape(-1, d), lse_ref.reshape(-1),
                  dtype, f"long rows thr={thr}")
     assert sp.spattn_device_error() == 0

@@ -57,6 +57,8 @@ def test_mask_builder_matches_brute_force(cfg):
         rp, ci = _gpu_csr(m)
         assert m.nnz == rp_ref[-1]
         assert m.n_long == int(np.sum(np.diff(rp_ref) > 1024))
+        # the schedule's long rows are exactly the rows above 1024 nonzeros
+        assert np.array_equal(m.long_rows().cpu().numpy(), np.nonzero(np.diff(rp_ref) > 1024)[0])
     assert np.array_equal(rp, rp_ref)
     assert np.array_equal(ci, ci_ref)
 
@@ -402,6 +404,7 @@ def test_user_csr_both_build_paths(n, nm):
         r2, c2 = m.csr()
         assert m.nnz == int(rp[-1])
         assert m.n_long == int(np.sum(lens > 1024))
+        assert np.array_equal(m.long_rows().cpu().numpy(), np.nonzero(lens > 1024)[0])
         assert torch.equal(r2, drp) and torch.equal(c2, dci)
     bad = rp.copy()
     bad[nm * n // 2] = bad[nm * n // 2 + 1] + 1                 # decreasing row_ptr

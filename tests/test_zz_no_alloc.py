@@ -9,15 +9,19 @@ a fixed array inside the library instead of taking it from the memory pool.
 This file is collected last on purpose. It calls the entry point through the C
 ABI twice in a row, on two different masks, so that the second call would see
 the first call's leftovers if the shared array were not cleared, and compares
-each result with spattn_fwd's under the tolerances of the other tests. It also
-passes when run alone in a fresh process (the first call does the per-device
-set-up).
+each result with the fp64 oracle and with spattn_fwd's under the tolerances of
+the other tests. The library counts every allocation it makes
+(spattn_alloc_count): the count must not move across the two calls, while the
+same work through spattn_fwd does allocate. It also passes when run alone in a
+fresh process (the first call does the per-device set-up).
 """
 import ctypes
+import math
 
 import numpy as np
 import pytest
 
+import oracle
 import workloads
 from helpers import assert_close, to_f64, torch_tensor
 
@@ -52,28 +56,41 @@ def _call_noalloc(q, k, v, rp, ci, nm, mask, out, lse, scale):
     assert st == sp.SPATTN_OK, sp.spattn_last_error()
 
 
-def test_noalloc_matches_spattn_fwd_on_two_calls_in_a_row():
+def test_noalloc_matches_oracle_and_spattn_fwd_on_two_calls_in_a_row():
     rng = np.random.default_rng(2024)
     cases = [
         # (B, H, n, d, dtype, rows made long (> 1024 nonzeros), num_masks)
         (2, 3, 2500, 64, workloads.BF16, set(range(0, 2500, 50)), 2),
         (1, 2, 1800, 128, workloads.F32, {3, 4, 5}, 1),
     ]
+    prepared = []
     for B, H, n, d, dtype, long_rows, nm in cases:
-        q, k, v = (torch_tensor(workloads.make_tensor(rng.standard_normal((B, H, n, d)), dtype))
-                   for _ in range(3))
-        mask = torch_tensor(workloads.make_tensor(
-            np.where(rng.random((B, 1, 1, n)) < 0.05, -np.inf, 0.0), workloads.BF16))
+        tq, tk, tv = (workloads.make_tensor(rng.standard_normal((B, H, n, d)), dtype) for _ in range(3))
+        tm = workloads.make_tensor(np.where(rng.random((B, 1, 1, n)) < 0.05, -np.inf, 0.0), workloads.BF16)
         rp, ci = _csr(rng, n, nm, 0.02, long_rows)
         assert int((rp[1:] - rp[:-1] > 1024).sum()) == len(long_rows) * nm
-        scale = 1.0 / np.sqrt(d)
-        ref_out, ref_lse = sp.spattn_fwd(q, k, v, rp, ci, nm, add_mask=mask, scale=scale)
+        scale = 1.0 / math.sqrt(d)
+        out_ref, lse_ref = oracle.masked_sdpa(tq.raw, tk.raw, tv.raw, rp.cpu().numpy().astype(np.int64),
+                                              ci.cpu().numpy(), nm, scale, add_mask=tm.raw)
+        q, k, v, mask = (torch_tensor(x) for x in (tq, tk, tv, tm))
+        a0 = sp.spattn_alloc_count()
+        fwd_out, fwd_lse = sp.spattn_fwd(q, k, v, rp, ci, nm, add_mask=mask, scale=scale)
+        assert sp.spattn_alloc_count() > a0          # the pool path does allocate (scratch)
         out = torch.empty_like(q)
         lse = torch.empty(B * H * n, dtype=torch.float32, device="cuda")
+        prepared.append((q, k, v, rp, ci, nm, mask, out, lse, scale, d, dtype, out_ref, lse_ref,
+                         fwd_out, fwd_lse))
+    torch.cuda.synchronize()
+    a1 = sp.spattn_alloc_count()
+    for (q, k, v, rp, ci, nm, mask, out, lse, scale, *_rest) in prepared:   # two calls in a row
         _call_noalloc(q, k, v, rp, ci, nm, mask, out, lse, scale)
-        torch.cuda.synchronize()
-        assert_close(to_f64(out).reshape(-1, d), to_f64(lse), to_f64(ref_out).reshape(-1, d),
-                     to_f64(ref_lse), dtype, "noalloc vs spattn_fwd")
+    torch.cuda.synchronize()
+    assert sp.spattn_alloc_count() == a1, "spattn_fwd_noalloc allocated memory"
+    for (q, k, v, rp, ci, nm, mask, out, lse, scale, d, dtype, out_ref, lse_ref, fwd_out, fwd_lse) in prepared:
+        assert_close(to_f64(out).reshape(-1, d), to_f64(lse), out_ref.reshape(-1, d), lse_ref.reshape(-1),
+                     dtype, "noalloc vs oracle")
+        assert_close(to_f64(out).reshape(-1, d), to_f64(lse), to_f64(fwd_out).reshape(-1, d),
+                     to_f64(fwd_lse), dtype, "noalloc vs spattn_fwd")
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():

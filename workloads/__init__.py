@@ -129,13 +129,17 @@ class Workload:
     notes: dict = field(default_factory=dict)
 
 
-# Full sizes of the five workloads.
+# Full sizes of the five workloads, and one extra (index 5): an all-ones mask at
+# d = 128, B*H = 64, n = 4096, the case where the dense-tile path's tensor-core
+# efficiency can show (the Evoformer workload's d = 32 cannot).
 CONFIGS = {
     0: dict(name="tiny-sliding", B=1, H=2, n=128, d=32, dtype=F32, std=1.0),
     1: dict(name="variable-window", B=4, H=12, n=4096, d=64, dtype=BF16, std=1.0),
     2: dict(name="random-csr", B=2, H=16, n=8192, d=64, dtype=BF16, std=1.0),
     3: dict(name="block-strided-global", B=1, H=16, n=16384, d=128, dtype=BF16, std=0.5),
     4: dict(name="evoformer-dense-mask-bias", B=256, H=8, n=256, d=32, dtype=BF16, std=1.0),
+    # extra to the five: an all-ones mask at d = 128, where dense tiles dominate
+    5: dict(name="dense-d128", B=4, H=16, n=4096, d=128, dtype=BF16, std=1.0),
 }
 
 
@@ -168,7 +172,7 @@ def _random_candidates(rng, n: int, mean_extra: float):
 def make(cfg: int, *, B: Optional[int] = None, H: Optional[int] = None,
          n: Optional[int] = None, seed: Optional[int] = None,
          dtype: Optional[str] = None, d: Optional[int] = None) -> Workload:
-    """Workload ``cfg`` (0..4) at full size, or with B/H/n/d/dtype overridden
+    """Workload ``cfg`` (0..4, and 5: the extra dense d = 128 case) at full size, or with B/H/n/d/dtype overridden
     (same recipe, smaller shapes, for parity tests the oracle finishes in seconds)."""
     c = dict(CONFIGS[cfg])
     B = c["B"] if B is None else B
@@ -215,6 +219,8 @@ def make(cfg: int, *, B: Optional[int] = None, H: Optional[int] = None,
         add_mask = make_tensor(m, BF16)
         bias = make_tensor(_normal(mrng, (1, H, n, n), 1.0), BF16)
         notes["key_lengths"] = lengths
+    elif cfg == 5:
+        mask = MaskParams("dense", n, 1)
     else:
         raise ValueError(cfg)
     return Workload(c["name"], B, H, n, d, dtype, float(scale), q, k, v, mask,
