@@ -1,4 +1,4 @@
-// Persistent, warp-specialised tensor-core forward for d = 64 and d = 128
+// Persistent, warp-specialised tensor-core forward for d = 32, 64 and 128
 // (tcgen05 MMAs with TMEM accumulators, TMA tile loads without multicast,
 // sm_100a).
 //
@@ -16,7 +16,8 @@
 // overwrites the first 64 columns of S). While one slot's softmax group turns
 // S into P, the tensor cores work on the other slot, so the two dependency
 // chains (S -> softmax -> P V -> next S) overlap. Producer and MMA issuer poll
-// both slots and advance whichever is ready; every wait is bounded.
+// both slots with non-blocking barrier tests and advance whichever is ready;
+// every wait is bounded.
 //
 // Per tile, each thread reads its row of S, scales it, sets the entries the
 // mask does not list to -inf, and keeps a running max and sum: the reference
@@ -25,6 +26,12 @@
 // paper's delta rescaling, applied lazily; exact in exact arithmetic). A warp
 // skips the 32-key chunks in which none of its rows has an entry (no TMEM load,
 // no exp; P is zero there).
+//
+// With an additive mask or bias (d <= 64, interval masks), the producer also
+// loads each tile's block of the additive terms into the slot's shared memory
+// (by TMA, with the K tile's timing), and the softmax group adds it before the
+// row max; with key lengths, tiles at or past a batch element's length are
+// dropped from the end of each list and the cut tile is masked.
 //
 // Two sources of work items:
 //   interval masks (sliding, variable window, dense): every (b, h, query
@@ -59,23 +66,35 @@ constexpr uint32_t kPpTmemCols = 512;
 constexpr float kPpRescale = 8.0f;               // log2 units
 constexpr long long kPpDrainCycles = 200000000LL;  // ~0.1 s per drain wait
 
-// mbarriers of slot s: 10 s + one of these; kBarDrain after both slots
-enum : int { kQFull = 0, kQEmpty, kKFull, kKEmpty, kVFull, kVEmpty, kSFull, kPFull, kODone, kOFree, kBarsPerSlot };
+// mbarriers of slot s: kBarsPerSlot * s + one of these; kBarDrain after both slots
+enum : int {
+    kQFull = 0, kQEmpty, kKFull, kKEmpty, kVFull, kVEmpty, kSFull, kPFull, kODone, kOFree, kAFull, kAEmpty,
+    kBarsPerSlot
+};
 constexpr int kBarDrain = 2 * kBarsPerSlot;
 constexpr int kNumBars = kBarDrain + 1;
 
-template <int D>
+template <int D, bool EXTRA>
 struct PpCfg {
-    static_assert(D == 64 || D == 128, "head dim");
-    static constexpr int ROW_BYTES = 128;                // 64 bf16 per 128-byte swizzled row
-    static constexpr int NCHUNK = D / 64;
-    static constexpr int CHUNK_BYTES = 128 * ROW_BYTES;  // 128 rows of one 64-column chunk
+    static_assert(D == 32 || D == 64 || D == 128, "head dim");
+    static_assert(!EXTRA || D <= 64, "additive terms: d <= 64");
+    static constexpr int CHUNK_ELEMS = D >= 64 ? 64 : D;  // bf16 per swizzled row
+    static constexpr int ROW_BYTES = CHUNK_ELEMS * 2;     // 128 or 64
+    static constexpr int NCHUNK = D / CHUNK_ELEMS;
+    static constexpr int CHUNK_BYTES = 128 * ROW_BYTES;   // 128 rows of one column chunk
     static constexpr int TILE_BYTES = NCHUNK * CHUNK_BYTES;
     static constexpr int SBO = 8 * ROW_BYTES;
+    static constexpr int KSTEPS_PER_CHUNK = CHUNK_ELEMS / 16;
+    static constexpr cute::UMMA::LayoutType LAYOUT =
+        D >= 64 ? cute::UMMA::LayoutType::SWIZZLE_128B : cute::UMMA::LayoutType::SWIZZLE_64B;
     static constexpr int OFF_Q = 0;                    // [slot]
     static constexpr int OFF_K = 2 * TILE_BYTES;       // [slot]
     static constexpr int OFF_V = 4 * TILE_BYTES;       // [slot]
-    static constexpr int OFF_BAR = 6 * TILE_BYTES;
+    // additive terms: [slot][term] 128 rows x 128 keys bf16 as two 64-key
+    // chunks of 128-byte rows (128-byte swizzle)
+    static constexpr int A_BYTES = 2 * 128 * 128;
+    static constexpr int OFF_A = 6 * TILE_BYTES;
+    static constexpr int OFF_BAR = OFF_A + (EXTRA ? 4 * A_BYTES : 0);
     static constexpr int OFF_INT = OFF_BAR + kNumBars * 8;  // TMEM base, abort flag
     // at least 116 KB, so that one CTA (which takes all 512 TMEM columns) runs per SM
     static constexpr int SMEM_BYTES = OFF_INT + 16 > 116 * 1024 ? OFF_INT + 16 : 116 * 1024;
@@ -93,6 +112,13 @@ struct PpItem {
     int T;              // tiles
     int64_t blk;        // interval masks: mask block (mask * nqb + qb)
 };
+
+// Keys of batch element b: [0, L), L = n without key lengths.
+__device__ __forceinline__ int pp_key_limit(const PpParams& P, int b) {
+    if (!P.seqlen_k) return P.n;
+    const int L = __ldg(P.seqlen_k + b);
+    return L < 0 ? 0 : (L > P.n ? P.n : L);
+}
 
 __device__ __forceinline__ PpItem pp_item(const PpParams& P, const bsg::Shape& sh, int64_t x) {
     PpItem it;
@@ -112,6 +138,10 @@ __device__ __forceinline__ PpItem pp_item(const PpParams& P, const bsg::Shape& s
         const int mk = P.num_masks == 1 ? 0 : it.b;
         it.blk = (int64_t)mk * P.nqb + it.qb;
         it.T = __ldg(P.itv_ntiles + it.blk);
+        if (P.seqlen_k && it.T > 1) {  // tiles past the key length go (ascending key tiles; one stays)
+            const int L = pp_key_limit(P, it.b);
+            while (it.T > 1 && (__ldg(P.itv_tiles + it.blk * P.nkt + it.T - 1) & 0x7fffffff) * 128 >= L) --it.T;
+        }
     } else {
         const bsg::Item bi = bsg::item(sh, x);
         it.bh = bi.bh;
@@ -312,13 +342,15 @@ __device__ __forceinline__ void pp_finish(const PpParams& P, const bsg::Shape& s
     pp_write_row<D>(P, it.b, it.h, bh, i, M, L, o);
 }
 
-template <int D>
+template <int D, bool EXTRA>
 __global__ void __launch_bounds__(kPpThreads, 1)
     k_fwd_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQp,
              const __grid_constant__ CUtensorMap tmKp, const __grid_constant__ CUtensorMap tmVp,
+             const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
              const PpParams P) {
-    using C = PpCfg<D>;
+    using C = PpCfg<D, EXTRA>;
+    constexpr int NSTREAM = EXTRA ? 4 : 3;  // producer streams: Q, K, V (, additive terms)
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (smem_u32(smem) & 1023u) {  // the swizzled layouts need a 1024-byte aligned base
@@ -339,7 +371,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < 2; ++s)
             for (int x = 0; x < kBarsPerSlot; ++x)
-                mbar_init(bar(s, x), (x == kPFull || x == kOFree) ? 4u : 1u);
+                mbar_init(bar(s, x), (x == kPFull || x == kOFree || x == kAEmpty) ? 4u : 1u);
         mbar_init(smem_u32(bars + kBarDrain), 1u);
         *abort_flag = 0;
         fence_mbar_init();
@@ -351,6 +383,8 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             prefetch_tensormap(&tmKp);
             prefetch_tensormap(&tmVp);
         }
+        if (EXTRA && P.extra[0]) prefetch_tensormap(&tmA0);
+        if (EXTRA && P.extra[1]) prefetch_tensormap(&tmA1);
     }
     tc_fence_before();
     __syncthreads();
@@ -376,15 +410,20 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            // per slot three load streams (Q per item; K, V per tile): the
-            // stream's item m, tile u, loads issued, the item's tile count
-            int sm[2][3], su[2][3], sT[2][3];
-            uint32_t cnt[2][3];
-            bool live[2][3];
+            // per slot three load streams (Q per item; K, V per tile; with
+            // additive terms a fourth, their blocks per tile): the stream's
+            // item m, tile u, loads issued, the item's tile count
+            int sm[2][NSTREAM], su[2][NSTREAM], sT[2][NSTREAM];
+            uint32_t cnt[2][NSTREAM];
+            bool live[2][NSTREAM];
+            // bytes of one tile's additive blocks (two 64-key chunks per term)
+            const uint32_t a_bytes = EXTRA ? (uint32_t)((P.extra[0] ? P.a_rows[0] : 0) + (P.extra[1] ? P.a_rows[1] : 0)) *
+                                                 256u
+                                           : 0u;
 #pragma unroll
             for (int s = 0; s < 2; ++s)
 #pragma unroll
-                for (int k = 0; k < 3; ++k) {
+                for (int k = 0; k < NSTREAM; ++k) {
                     sm[s][k] = su[s][k] = 0;
                     cnt[s][k] = 0;
                     sT[s][k] = 0;
@@ -396,33 +435,55 @@ __global__ void __launch_bounds__(kPpThreads, 1)
 #pragma unroll
                 for (int s = 0; s < 2; ++s) {
 #pragma unroll
-                    for (int k = 0; k < 3; ++k) {
+                    for (int k = 0; k < NSTREAM; ++k) {
                         if (!live[s][k]) continue;
                         any = true;
-                        const int eb = k == 0 ? kQEmpty : (k == 1 ? kKEmpty : kVEmpty);
-                        if (cnt[s][k] != 0 && !mbar_try_wait(bar(s, eb), (cnt[s][k] - 1) & 1)) continue;
+                        const int eb = k == 0 ? kQEmpty : (k == 1 ? kKEmpty : (k == 2 ? kVEmpty : kAEmpty));
+                        if (cnt[s][k] != 0 && !mbar_test(bar(s, eb), (cnt[s][k] - 1) & 1)) continue;
                         const PpItem it = pp_item(P, sh, item_x(s, sm[s][k]));
-                        const uint32_t fb = bar(s, k == 0 ? kQFull : (k == 1 ? kKFull : kVFull));
-                        const uint32_t dst = (k == 0 ? sQ0 : (k == 1 ? sK0 : sV0)) + s * C::TILE_BYTES;
-                        mbar_expect_tx(fb, C::TILE_BYTES);
+                        const uint32_t fb = bar(s, k == 0 ? kQFull : (k == 1 ? kKFull : (k == 2 ? kVFull : kAFull)));
                         if (k == 0) {
+                            const uint32_t dst = sQ0 + s * C::TILE_BYTES;
+                            mbar_expect_tx(fb, C::TILE_BYTES);
 #pragma unroll
                             for (int c = 0; c < C::NCHUNK; ++c) {
                                 if (it.perm)
-                                    tma_load_5d(dst + c * C::CHUNK_BYTES, &tmQp, fb, c * 64, it.qb, it.pqb * 128, it.h,
-                                                it.b);
+                                    tma_load_5d(dst + c * C::CHUNK_BYTES, &tmQp, fb, c * C::CHUNK_ELEMS, it.qb,
+                                                it.pqb * 128, it.h, it.b);
                                 else
-                                    tma_load_4d(dst + c * C::CHUNK_BYTES, &tmQ, fb, c * 64, it.qb * 128, it.h, it.b);
+                                    tma_load_4d(dst + c * C::CHUNK_BYTES, &tmQ, fb, c * C::CHUNK_ELEMS, it.qb * 128,
+                                                it.h, it.b);
                             }
-                        } else {
+                        } else if (k < 3) {
+                            const uint32_t dst = (k == 1 ? sK0 : sV0) + s * C::TILE_BYTES;
+                            mbar_expect_tx(fb, C::TILE_BYTES);
                             const int kt = pp_tile(P, sh, it, su[s][k]) & 0x7fffffff;
                             const CUtensorMap* map = it.perm ? (k == 1 ? &tmKp : &tmVp) : (k == 1 ? &tmK : &tmV);
 #pragma unroll
                             for (int c = 0; c < C::NCHUNK; ++c) {
                                 if (it.perm)
-                                    tma_load_5d(dst + c * C::CHUNK_BYTES, map, fb, c * 64, it.qb, kt * 128, it.h, it.b);
+                                    tma_load_5d(dst + c * C::CHUNK_BYTES, map, fb, c * C::CHUNK_ELEMS, it.qb, kt * 128,
+                                                it.h, it.b);
                                 else
-                                    tma_load_4d(dst + c * C::CHUNK_BYTES, map, fb, c * 64, kt * 128, it.h, it.b);
+                                    tma_load_4d(dst + c * C::CHUNK_BYTES, map, fb, c * C::CHUNK_ELEMS, kt * 128, it.h,
+                                                it.b);
+                            }
+                        } else {
+                            // the additive terms' blocks of this tile: term a at
+                            // OFF_A + (2 s + a) A_BYTES, chunk c of a_rows[a] rows at
+                            // c * a_rows[a] * 128 bytes
+                            mbar_expect_tx(fb, a_bytes);
+                            const int kt = pp_tile(P, sh, it, su[s][k]) & 0x7fffffff;
+#pragma unroll
+                            for (int a = 0; a < 2; ++a) {
+                                if (!P.extra[a]) continue;
+                                const uint32_t dst = smem_u32(smem + C::OFF_A + (2 * s + a) * C::A_BYTES);
+                                const int r0 = P.a_rows[a] == 1 ? 0 : it.qb * 128;
+                                const int hh = P.a_h[a] ? it.h : 0, bb = P.a_b[a] ? it.b : 0;
+#pragma unroll
+                                for (int c = 0; c < 2; ++c)
+                                    tma_load_4d(dst + (uint32_t)(c * P.a_rows[a] * 128), a == 0 ? &tmA0 : &tmA1, fb,
+                                                kt * 128 + c * 64, r0, hh, bb);
                             }
                         }
                         ++cnt[s][k];
@@ -449,8 +510,8 @@ __global__ void __launch_bounds__(kPpThreads, 1)
 #pragma unroll
             for (int s = 0; s < 2; ++s) {
 #pragma unroll
-                for (int k = 0; k < 3; ++k) {
-                    const int full = k == 0 ? kQFull : (k == 1 ? kKFull : kVFull);
+                for (int k = 0; k < NSTREAM; ++k) {
+                    const int full = k == 0 ? kQFull : (k == 1 ? kKFull : (k == 2 ? kVFull : kAFull));
                     if (cnt[s][k]) mbar_wait_bounded(bar(s, full), (cnt[s][k] - 1) & 1, kPpDrainCycles);
                 }
             }
@@ -483,18 +544,18 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                     const uint32_t tS = tmem + (uint32_t)(s * 256), tO = tS + 128;
                     if (x.phase == 0) {
                         // S(g) needs the item's Q, K(g), and P V(g-1) done (P overwrote S)
-                        const bool ready = (x.u != 0 || mbar_try_wait(bar(s, kQFull), x.items & 1)) &&
-                                           mbar_try_wait(bar(s, kKFull), x.g & 1) &&
-                                           (x.g == 0 || mbar_try_wait(bar(s, kODone), (x.g - 1) & 1));
+                        const bool ready = (x.u != 0 || mbar_test(bar(s, kQFull), x.items & 1)) &&
+                                           mbar_test(bar(s, kKFull), x.g & 1) &&
+                                           (x.g == 0 || mbar_test(bar(s, kODone), (x.g - 1) & 1));
                         if (ready) {
                             tc_fence_after();
                             const uint32_t sQ = sQ0 + s * C::TILE_BYTES, sK = sK0 + s * C::TILE_BYTES;
 #pragma unroll
                             for (int ks = 0; ks < D / 16; ++ks) {
-                                const uint32_t off = (uint32_t)((ks / 4) * C::CHUNK_BYTES + (ks % 4) * 32);
-                                mma_bf16_ss(tS, smem_desc(sQ + off, 16, C::SBO, cute::UMMA::LayoutType::SWIZZLE_128B),
-                                            smem_desc(sK + off, 16, C::SBO, cute::UMMA::LayoutType::SWIZZLE_128B),
-                                            idS, ks > 0 ? 1u : 0u);
+                                const uint32_t off = (uint32_t)((ks / C::KSTEPS_PER_CHUNK) * C::CHUNK_BYTES +
+                                                                (ks % C::KSTEPS_PER_CHUNK) * 32);
+                                mma_bf16_ss(tS, smem_desc(sQ + off, 16, C::SBO, C::LAYOUT),
+                                            smem_desc(sK + off, 16, C::SBO, C::LAYOUT), idS, ks > 0 ? 1u : 0u);
                             }
                             mma_commit(bar(s, kSFull));
                             mma_commit(bar(s, kKEmpty));
@@ -505,16 +566,16 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                     } else {
                         // P V(g) needs P(g), V(g), and for an item's first tile the
                         // previous item's O read out
-                        const bool ready = mbar_try_wait(bar(s, kPFull), x.g & 1) &&
-                                           mbar_try_wait(bar(s, kVFull), x.g & 1) &&
-                                           (x.u != 0 || x.items == 0 || mbar_try_wait(bar(s, kOFree), (x.items - 1) & 1));
+                        const bool ready = mbar_test(bar(s, kPFull), x.g & 1) &&
+                                           mbar_test(bar(s, kVFull), x.g & 1) &&
+                                           (x.u != 0 || x.items == 0 || mbar_test(bar(s, kOFree), (x.items - 1) & 1));
                         if (ready) {
                             tc_fence_after();
                             const uint32_t sV = sV0 + s * C::TILE_BYTES;
 #pragma unroll
                             for (int ks = 0; ks < 8; ++ks) {  // 16 keys per step
                                 const uint64_t db = smem_desc(sV + (uint32_t)(ks * 16 * C::ROW_BYTES), C::CHUNK_BYTES,
-                                                              C::SBO, cute::UMMA::LayoutType::SWIZZLE_128B);
+                                                              C::SBO, C::LAYOUT);
                                 mma_bf16_ts(tO, tS + (uint32_t)(ks * 8), db, idO, (x.u > 0 || ks > 0) ? 1u : 0u);
                             }
                             mma_commit(bar(s, kODone));
@@ -585,10 +646,11 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                 row_ok = i >= 0;
             }
             float m_ref = -INFINITY, l = 0.f;
+            const int klim = pp_key_limit(P, it.b);
             for (int u = 0; u < it.T; ++u, ++g) {
                 const int info = pp_tile(P, sh, it, u);
                 const int kt = info & 0x7fffffff;
-                const bool dense = P.mode == 0 && info < 0;
+                bool dense = P.mode == 0 && info < 0;
                 uint32_t w[4] = {0u, 0u, 0u, 0u};
                 if (row_ok && !dense) {
                     if (P.mode == 0) {
@@ -606,6 +668,14 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                         bsg::row_bits(sh, bi, kt, t, w);
                     }
                 }
+                if (klim - kt * 128 < 128) {  // the tile the key length cuts
+                    if (dense) {
+                        dense = false;
+                        if (row_ok) w[0] = w[1] = w[2] = w[3] = 0xffffffffu;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) w[q] &= bsg::run_word(0, klim - kt * 128, 32 * q);
+                }
                 uint32_t need = 0;
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
@@ -617,6 +687,13 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                     break;
                 }
                 tc_fence_after();
+                if (EXTRA) {  // this tile's blocks of the additive terms are in shared memory
+                    const bool oka = pp_wait(bar(s, kAFull), g & 1, abort_flag, P.wait_cycles);
+                    if (!__all_sync(0xffffffffu, oka)) {
+                        alive = false;
+                        break;
+                    }
+                }
                 float x[128];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -626,6 +703,30 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                         tmem_wait_ld_dep(r);
 #pragma unroll
                         for (int k = 0; k < 16; ++k) mul2(x[32 * q + 2 * k], x[32 * q + 2 * k + 1], r[2 * k], r[2 * k + 1], c2);
+                        if (EXTRA) {
+                            // + log2(e) * (mask + bias) of keys 32q .. 32q + 31: 16-byte
+                            // units 4 (q & 1) .. + 3 of chunk q / 2 of this row's line
+                            // (128-byte swizzle: unit j of row r at j ^ (r & 7))
+#pragma unroll
+                            for (int a = 0; a < 2; ++a) {
+                                if (!P.extra[a]) continue;
+                                const int rows = P.a_rows[a], r0 = rows == 1 ? 0 : t;
+                                const uint8_t* base =
+                                    smem + C::OFF_A + (2 * s + a) * C::A_BYTES + (q >> 1) * rows * 128 + r0 * 128;
+#pragma unroll
+                                for (int uu = 0; uu < 4; ++uu) {
+                                    const int j = 4 * (q & 1) + uu;
+                                    const int ph = rows == 1 ? j : (j ^ (r0 & 7));
+                                    const uint4 v4 = *reinterpret_cast<const uint4*>(base + ph * 16);
+                                    const uint32_t ws[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) {
+                                        x[32 * q + 8 * uu + 2 * e] += kLog2e * __uint_as_float(ws[e] << 16);
+                                        x[32 * q + 8 * uu + 2 * e + 1] += kLog2e * __uint_as_float(ws[e] & 0xffff0000u);
+                                    }
+                                }
+                            }
+                        }
                         if (!dense) {
 #pragma unroll
                             for (int jj = 0; jj < 32; ++jj)
@@ -635,6 +736,10 @@ __global__ void __launch_bounds__(kPpThreads, 1)
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj) x[32 * q + jj] = -INFINITY;
                     }
+                }
+                if (EXTRA) {  // the additive blocks are read: the producer may refill them
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(s, kAEmpty));
                 }
                 float ma = -INFINITY, mb = -INFINITY, mc = -INFINITY, md = -INFINITY;
 #pragma unroll
@@ -757,20 +862,22 @@ EncodeTiledFn pp_encode_fn() {
     return fn;
 }
 
-// [B, H, n, d] bf16 as {d, n, H, B}, box {64, 128, 1, 1}, 128-byte swizzle.
+// [B, H, n, d] bf16 as {d, n, H, B}, box {min(d, 64), 128, 1, 1}, 128-byte
+// swizzle (64-byte for d = 32).
 cudaError_t pp_map4(CUtensorMap* map, const TcOperand& t, int B, int H, int n, int d) {
     EncodeTiledFn fn = pp_encode_fn();
     if (!fn) return cudaErrorNotSupported;
+    const int chunk = d >= 64 ? 64 : d;
     const uint64_t sn = (uint64_t)t.s_n * 2;
     const uint64_t sh = H > 1 ? (uint64_t)t.s_h * 2 : sn * (uint64_t)n;
     const uint64_t sb = B > 1 ? (uint64_t)t.s_b * 2 : sh * (uint64_t)H;
     cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)H, (cuuint64_t)B};
     cuuint64_t strides[3] = {sn, sh, sb};
-    cuuint32_t box[4] = {64, 128, 1, 1};
+    cuuint32_t box[4] = {(cuuint32_t)chunk, 128, 1, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(t.data), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, chunk == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
@@ -793,26 +900,48 @@ cudaError_t pp_map5(CUtensorMap* map, const TcOperand& t, int B, int H, int n, i
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int D>
-cudaError_t launch_pp_t(const TcOperand& q, const TcOperand& k, const TcOperand& v, const PpParams& p, int num_sms,
-                        cudaStream_t s) {
-    using C = PpCfg<D>;
+// An additive term [B or 1, H or 1, n or 1, n] (bf16, keys contiguous) as
+// {keys, rows, heads, batch}, box {64, rows_box, 1, 1}: 128-byte swizzle for
+// 128-row blocks, none for a term shared by all rows (rows_box 1). Dimensions
+// the term broadcasts over have extent 1.
+cudaError_t pp_map_addend(CUtensorMap* map, const AddendView& a, int B, int H, int n, int rows_box) {
+    EncodeTiledFn fn = pp_encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const uint64_t row_bytes = ((uint64_t)n * 2 + 15) & ~uint64_t(15);  // a valid stride for extent-1 dimensions
+    cuuint64_t dims[4] = {(cuuint64_t)n, (cuuint64_t)(a.s2 ? n : 1), (cuuint64_t)(a.s1 ? H : 1),
+                          (cuuint64_t)(a.s0 ? B : 1)};
+    cuuint64_t strides[3] = {a.s2 ? (uint64_t)a.s2 * 2 : row_bytes, a.s1 ? (uint64_t)a.s1 * 2 : row_bytes,
+                             a.s0 ? (uint64_t)a.s0 * 2 : row_bytes};
+    cuuint32_t box[4] = {64, (cuuint32_t)rows_box, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(a.data), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    rows_box == 1 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int D, bool EXTRA>
+cudaError_t launch_pp_t(const TcOperand& q, const TcOperand& k, const TcOperand& v, const PpParams& p0,
+                        const AddendView& mask, const AddendView& bias, int num_sms, cudaStream_t s) {
+    using C = PpCfg<D, EXTRA>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, []() {
-        attr_err = cudaFuncSetAttribute((const void*)k_fwd_pp<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err = cudaFuncSetAttribute((const void*)k_fwd_pp<D, EXTRA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         C::SMEM_BYTES);
         // setmaxnreg.inc draws on the registers the CTA was launched with: the
         // split adds up only at exactly 168 per thread (fewer would leave the
         // softmax warps waiting for registers that never come), so refuse any
         // other build of the kernel
         cudaFuncAttributes fa;
-        if (attr_err == cudaSuccess) attr_err = cudaFuncGetAttributes(&fa, (const void*)k_fwd_pp<D>);
+        if (attr_err == cudaSuccess) attr_err = cudaFuncGetAttributes(&fa, (const void*)k_fwd_pp<D, EXTRA>);
         if (attr_err == cudaSuccess && fa.numRegs * kPpThreads != 128 * kPpRegsLow + 256 * kPpRegsHigh)
             attr_err = cudaErrorInvalidConfiguration;
     });
     if (attr_err != cudaSuccess) return attr_err;
-    CUtensorMap mq, mk, mv, mqp, mkp, mvp;
+    PpParams p = p0;
+    CUtensorMap mq, mk, mv, mqp, mkp, mvp, ma0, ma1;
     cudaError_t e;
     if ((e = pp_map4(&mq, q, p.B, p.H, p.n, D)) != cudaSuccess) return e;
     if ((e = pp_map4(&mk, k, p.B, p.H, p.n, D)) != cudaSuccess) return e;
@@ -826,21 +955,45 @@ cudaError_t launch_pp_t(const TcOperand& q, const TcOperand& k, const TcOperand&
         mkp = mk;
         mvp = mv;
     }
+    ma0 = ma1 = mq;
+    const AddendView* terms[2] = {&mask, &bias};
+    for (int a = 0; a < 2; ++a) {
+        p.extra[a] = EXTRA && terms[a]->data != nullptr;
+        p.a_rows[a] = terms[a]->s2 ? 128 : 1;
+        p.a_h[a] = terms[a]->s1 != 0;
+        p.a_b[a] = terms[a]->s0 != 0;
+        if (p.extra[a] &&
+            (e = pp_map_addend(a == 0 ? &ma0 : &ma1, *terms[a], p.B, p.H, p.n, p.a_rows[a])) != cudaSuccess)
+            return e;
+    }
     if (p.n_items <= 0) return cudaSuccess;
     const int64_t grid = p.n_items < num_sms ? p.n_items : num_sms;
-    k_fwd_pp<D><<<(unsigned)grid, kPpThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, mqp, mkp, mvp, p);
+    k_fwd_pp<D, EXTRA><<<(unsigned)grid, kPpThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, mqp, mkp, mvp, ma0,
+                                                                                   ma1, p);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_fwd_pp(const TcOperand& q, const TcOperand& k, const TcOperand& v, int d, const PpParams& p,
-                          int num_sms, cudaStream_t s) {
+                          const AddendView& mask, const AddendView& bias, int num_sms, cudaStream_t s) {
+    const bool extra = mask.data || bias.data;
+    if (extra && (p.mode != 0 || d > 64 || !pp_addend_ok(mask) || !pp_addend_ok(bias))) return cudaErrorInvalidValue;
     switch (d) {
-    case 64: return launch_pp_t<64>(q, k, v, p, num_sms, s);
-    case 128: return launch_pp_t<128>(q, k, v, p, num_sms, s);
+    case 32: return extra ? launch_pp_t<32, true>(q, k, v, p, mask, bias, num_sms, s)
+                          : launch_pp_t<32, false>(q, k, v, p, mask, bias, num_sms, s);
+    case 64: return extra ? launch_pp_t<64, true>(q, k, v, p, mask, bias, num_sms, s)
+                          : launch_pp_t<64, false>(q, k, v, p, mask, bias, num_sms, s);
+    case 128: return launch_pp_t<128, false>(q, k, v, p, mask, bias, num_sms, s);
     }
     return cudaErrorInvalidValue;
+}
+
+bool pp_addend_ok(const AddendView& a) {
+    if (!a.data) return true;
+    const uintptr_t base = reinterpret_cast<uintptr_t>(a.data);
+    return a.dtype == 0 && a.s3 == 1 && (base & 15) == 0 && (a.s2 * 2) % 16 == 0 && (a.s1 * 2) % 16 == 0 &&
+           (a.s0 * 2) % 16 == 0;
 }
 
 }  // namespace spattn

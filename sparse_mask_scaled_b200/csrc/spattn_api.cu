@@ -990,16 +990,26 @@ int fwd_closed(const FwdParams& p, int d, spattn_mask m, cudaStream_t s, cudaMem
         pp.pacc = partner ? c.at<float>(ws, k_pacc) : nullptr;
         const TcOperand oq{p.q, p.q_sn, p.q_sh, p.q_sb}, ok{p.k, p.k_sn, p.k_sh, p.k_sb},
             ov{p.v, p.v_sn, p.v_sh, p.v_sb};
-        e = launch_fwd_pp(oq, ok, ov, d, pp, sms, s);
+        AddendView none;
+        memset(&none, 0, sizeof none);
+        e = launch_fwd_pp(oq, ok, ov, d, pp, none, none, sms, s);
     }
     cudaFreeAsync(ws, s);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core kernel (closed-form mask)");
     return SPATTN_OK;
 }
 
-// The persistent tile kernel over an interval mask's tiles (d = 64 or 128,
-// no additive terms, no key lengths); blk_res: the gather kernel ran first and
-// left partial states in p.ws_ml / p.ws_acc for the flagged blocks.
+// Whether the persistent tile kernel takes an interval-mask forward: d = 32,
+// 64 or 128; additive terms only for d <= 64 and when TMA can stage them.
+bool pp_takes_interval(const FwdParams& p, int d) {
+    if (d != 32 && d != 64 && d != 128) return false;
+    if (!p.has_extra) return true;
+    return d <= 64 && pp_addend_ok(p.mask) && pp_addend_ok(p.bias);
+}
+
+// The persistent tile kernel over an interval mask's tiles; blk_res: the
+// gather kernel ran first and left partial states in p.ws_ml / p.ws_acc for
+// the flagged blocks.
 int launch_pp_interval(const FwdParams& p, int d, spattn_mask m, int dev, int sms, const int32_t* blk_res,
                        cudaStream_t s) {
     unsigned* ef = nullptr;
@@ -1017,8 +1027,9 @@ int launch_pp_interval(const FwdParams& p, int d, spattn_mask m, int dev, int sm
     pp.blk_res = blk_res;
     pp.ws_ml = p.ws_ml;
     pp.ws_acc = p.ws_acc;
+    pp.seqlen_k = p.seqlen_k;
     const TcOperand oq{p.q, p.q_sn, p.q_sh, p.q_sb}, ok{p.k, p.k_sn, p.k_sh, p.k_sb}, ov{p.v, p.v_sn, p.v_sh, p.v_sb};
-    const cudaError_t e = launch_fwd_pp(oq, ok, ov, d, pp, sms, s);
+    const cudaError_t e = launch_fwd_pp(oq, ok, ov, d, pp, p.mask, p.bias, sms, s);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core kernel launch");
     return SPATTN_OK;
 }
@@ -1064,7 +1075,7 @@ int fwd_interval(FwdParams& p, int dtype, int d, spattn_mask m, cudaStream_t s, 
             return cuda_fail(e, "interval gather kernel launch");
         }
     }
-    if ((d == 64 || d == 128) && !p.has_extra && !p.seqlen_k)
+    if (pp_takes_interval(p, d))
         r = launch_pp_interval(p, d, m, dev, num_sms, gather ? m->blk_res : nullptr, s);
     else
         r = launch_tc(p, d, m, dev, gather ? m->blk_res : nullptr, s);

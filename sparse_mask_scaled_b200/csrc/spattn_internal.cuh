@@ -159,8 +159,8 @@ struct TcParams {
 cudaError_t launch_fwd_tc(const TcOperand& q, const TcOperand& k, const TcOperand& v, int d,
                           const TcParams& p, cudaStream_t stream);
 
-// Persistent ping-pong tensor-core kernel (fwd_pp.cu), d = 64 or 128, bf16,
-// no additive terms, no key lengths.
+// Persistent ping-pong tensor-core kernel (fwd_pp.cu), d = 32, 64 or 128,
+// bf16; additive terms (d <= 64) and key lengths for interval masks.
 struct PpParams {
     int B, H, n, num_masks, nqb, nkt;
     int mode;         // 0: interval-mask tiles; 1: block + strided + global in closed form
@@ -189,9 +189,17 @@ struct PpParams {
     float qk_scale_log2;
     unsigned* err;
     long long wait_cycles;  // limit of every wait (SM cycles)
+    // mode 0, d <= 64: additive terms (bf16, keys contiguous, 16-byte aligned
+    // rows) staged tile by tile through shared memory by TMA; extra[a] != 0
+    // when term a (0: mask, 1: bias) is present, a_rows[a] = 1 when it is the
+    // same for every query row, else 128; a_h / a_b: it varies with h / b
+    int extra[2], a_rows[2], a_h[2], a_b[2];
+    const int32_t* seqlen_k;  // nullable, [B]: keys j >= seqlen_k[b] are left out
 };
 cudaError_t launch_fwd_pp(const TcOperand& q, const TcOperand& k, const TcOperand& v, int d, const PpParams& p,
-                          int num_sms, cudaStream_t stream);
+                          const AddendView& mask, const AddendView& bias, int num_sms, cudaStream_t stream);
+// Whether an additive term can be staged through shared memory by TMA.
+bool pp_addend_ok(const AddendView& a);
 cudaError_t error_flag_address(unsigned** p);
 // Every kernel launch of the library passes its stream through counted(),
 // which adds one to the count spattn_launch_count() reports.

@@ -1,4 +1,4 @@
-"""The persistent tile kernel against the fp64 oracle (needs a B200).
+"""The persistent tile kernel (k_fwd_pp) against the fp64 oracle (needs a B200).
 
 Block + strided + global masks whose parameters allow it (block dividing 128,
 stride 0 or 128, at most 128 global tokens, n a multiple of 128) are kept in
@@ -9,11 +9,14 @@ row. These tests cover the parameter corners of that plan (no global tokens, no
 block part, no strided part, permuted blocks shorter than a tile, more than one
 permuted tile per residue, one mask per batch element), d = 64 and 128, the
 fallbacks that go through the CSR-built copy of the mask (fp32 inputs, an
-additive term, key lengths), dense interval masks at d = 128 on the same
-kernel, the two section-(b) entry points spattn_mask_csr and
-spattn_check_device_error, and the bounded waits: with a wait limit of zero
-cycles every wait gives up, the call reports SPATTN_ERR_TIMEOUT, and the next
-call is exact again (the kernel released its tensor memory and left no state).
+additive term, key lengths), interval masks (dense, sliding, variable window)
+on the same kernel at d = 32, 64 and 128 -- with additive mask and bias
+layouts staged through shared memory, key lengths, and the layouts that fall
+back to the per-block kernels --, the two section-(b) entry points
+spattn_mask_csr and spattn_check_device_error, and the bounded waits: with a
+wait limit of zero cycles every wait gives up, the call reports
+SPATTN_ERR_TIMEOUT, and the next call is exact again (the kernel released its
+tensor memory and left no state).
 """
 import ctypes
 import math
@@ -160,6 +163,70 @@ def test_dense_interval_mask_d128(n, B, H):
     _check(mp, B, H, 128, seed=n, what=f"dense d=128 n={n}")
 
 
+@pytest.mark.parametrize("d", [32, 64])
+@pytest.mark.parametrize("layout", ["row_mask", "bias_only", "pad_mask_and_bias", "row_mask_and_bias",
+                                    "f32_bias", "head_mask"])
+@pytest.mark.parametrize("kind,n", [("dense", 256), ("sliding", 384), ("dense", 200)])
+def test_interval_mask_with_additive_terms(d, layout, kind, n):
+    """Additive mask and bias on interval masks: bf16 terms with keys
+    contiguous and 16-byte rows are staged through shared memory tile by tile
+    (row-varying, shared by all rows, per head); an fp32 term, or rows that are
+    not 16-byte multiples (n = 200: 400-byte rows are, n odd would not), take
+    the per-block kernel; both must equal the oracle."""
+    rng = np.random.default_rng(7 + d + n)
+    B, H = 2, 3
+    mp = workloads.MaskParams(kind, n, 1, window=40 if kind == "sliding" else 0)
+    q, k, v = _inputs(rng, B, H, n, d, std=1.0)
+    row_mask = workloads.make_tensor(np.where(rng.random((B, 1, n, n)) < 0.1, -np.inf,
+                                              rng.standard_normal((B, 1, n, n))), workloads.BF16)
+    pad_mask = workloads.make_tensor(np.where(rng.random((B, 1, 1, n)) < 0.2, -np.inf, 0.0), workloads.BF16)
+    head_mask = workloads.make_tensor(np.where(rng.random((1, H, 1, n)) < 0.2, -np.inf, 0.0), workloads.BF16)
+    bias = workloads.make_tensor(rng.standard_normal((1, H, n, n)), workloads.BF16)
+    bias32 = workloads.make_tensor(rng.standard_normal((1, H, n, n)), workloads.F32)
+    am, b = {"row_mask": (row_mask, None), "bias_only": (None, bias), "pad_mask_and_bias": (pad_mask, bias),
+             "row_mask_and_bias": (row_mask, bias), "f32_bias": (pad_mask, bias32),
+             "head_mask": (head_mask, bias)}[layout]
+    rp, ci = oracle.mask_from_params(mp)
+    scale = 1 / math.sqrt(d)
+    out_ref, lse_ref = oracle.masked_sdpa(q.raw, k.raw, v.raw, rp, ci, 1, scale,
+                                          add_mask=None if am is None else am.raw,
+                                          bias=None if b is None else b.raw)
+    with build_mask(mp) as m:
+        out, lse = sp.spattn_fwd_mask(torch_tensor(q), torch_tensor(k), torch_tensor(v), m,
+                                      add_mask=None if am is None else torch_tensor(am),
+                                      bias=None if b is None else torch_tensor(b), scale=scale)
+        torch.cuda.synchronize()
+    assert_close(to_f64(out).reshape(-1, d), to_f64(lse), out_ref.reshape(-1, d), lse_ref.reshape(-1),
+                 workloads.BF16, f"{kind} n={n} d={d} {layout}")
+    assert sp.spattn_device_error() == 0
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+def test_key_lengths_with_bias_on_the_persistent_kernel(d):
+    """Key lengths on tile edges with a pair bias (d <= 64 stages the bias; at
+    d = 128 the bias takes the per-block kernel), against the oracle with the
+    equivalent additive key-padding mask."""
+    lengths = [0, 1, 127, 128, 129, 255, 256, 200]
+    B, H, n = len(lengths), 2, 256
+    rng = np.random.default_rng(30 + d)
+    q, k, v = _inputs(rng, B, H, n, d, std=1.0)
+    bias = workloads.make_tensor(rng.standard_normal((1, H, n, n)), workloads.BF16)
+    pad = np.zeros((B, 1, 1, n))
+    for bb, L in enumerate(lengths):
+        pad[bb, 0, 0, L:] = -np.inf
+    rp, ci = oracle.mask_csr("dense", n)
+    scale = 1 / math.sqrt(d)
+    out_ref, lse_ref = oracle.masked_sdpa(q.raw, k.raw, v.raw, rp, ci, 1, scale, add_mask=pad, bias=bias.raw)
+    sl = torch.tensor(lengths, dtype=torch.int32, device="cuda")
+    with sp.spattn_create_csr_mask("dense", n, 1, asynchronous=True) as m:
+        out, lse = sp.spattn_fwd_mask_kpad(torch_tensor(q), torch_tensor(k), torch_tensor(v), m, sl,
+                                           bias=torch_tensor(bias), scale=scale)
+        torch.cuda.synchronize()
+    assert_close(to_f64(out).reshape(-1, d), to_f64(lse), out_ref.reshape(-1, d), lse_ref.reshape(-1),
+                 workloads.BF16, f"lengths + bias d={d}")
+    assert sp.spattn_device_error() == 0
+
+
 def test_variable_window_d128():
     """A variable-window mask at d = 128: tiles on the persistent kernel, the
     window edges outside them gathered first and merged in its epilogue."""
@@ -179,7 +246,7 @@ class _DeviceArray:
     """An int32 device array owned by the library, viewed by torch without a copy."""
 
     def __init__(self, ptr, count):
-        self.__cuda_array_interface__ = {"shape": (count,), "typestr": "<i4", "data": (ptr, True),
+        self.__cuda_array_interface__ = {"shape": (count,), "typestr": "<i4", "data": (ptr, False),
                                          "version": 2}
 
 
