@@ -5,27 +5,29 @@
 // One CTA per SM walks a list of work items (a 128-row query block and its
 // key tiles). Three warpgroups:
 //   warp 0      TMA producer (one thread): Q tile per item, K and V per tile
-//   warp 1      MMA issuer (one thread):   S = Q K^T, then O (+)= P V
-//   warps 2-3   idle (they complete the first warpgroup, which gives its
+//   warps 1-3   idle (they complete the first warpgroup, which gives its
 //               registers to the other two: 72 per thread against 216)
 //   warps 4-7   softmax group of slot 0 (one query row per thread)
 //   warps 8-11  softmax group of slot 1
 // The two slots hold one item each, with their own Q, K and V buffers in shared
 // memory and their own S and O in tensor memory (slot s: S in columns
 // [256 s, 256 s + 128), O in [256 s + 128, 256 s + 128 + d); P, in bf16,
-// overwrites the first 64 columns of S). While one slot's softmax group turns
-// S into P, the tensor cores work on the other slot, so the two dependency
-// chains (S -> softmax -> P V -> next S) overlap. Producer and MMA issuer poll
-// both slots with non-blocking barrier tests and advance whichever is ready;
+// overwrites the first 64 columns of S). Each group's first thread issues its
+// slot's MMAs: once all four warps have written P(g), O (+)= P(g) V(g), then,
+// when that has consumed P, S(g + 1) = Q K(g + 1)^T, which its warps are
+// waiting for. While one slot's group turns S into P, the tensor cores work on
+// the other slot, so the two dependency chains overlap. The producer polls both
+// slots with non-blocking barrier tests and loads whichever buffer is free;
 // every wait is bounded.
 //
-// Per tile, each thread reads its row of S, scales it, sets the entries the
-// mask does not list to -inf, and keeps a running max and sum: the reference
-// max only moves when a tile's max exceeds it by more than 2^8, and then O is
-// rescaled in TMEM by exp2(m_old - m_new) (the streaming-dataflow SDPA
-// paper's delta rescaling, applied lazily; exact in exact arithmetic). A warp
-// skips the 32-key chunks in which none of its rows has an entry (no TMEM load,
-// no exp; P is zero there).
+// Per tile, each thread streams its row of S 32 keys at a time (the next
+// chunk's TMEM load in flight): scale, entries the mask does not list to -inf,
+// p = 2^(x - m_ref) against a running reference max, row sum, bf16 P back to
+// TMEM. The reference only moves when a chunk's max exceeds it by more than
+// 2^8; then the P chunks already written, the sum and O are rescaled by
+// exp2(m_old - m_new) (the streaming-dataflow SDPA paper's delta rescaling,
+// applied lazily; exact in exact arithmetic). A warp skips the 32-key chunks in
+// which none of its rows has an entry (no TMEM load, no exp; P is zero there).
 //
 // With an additive mask or bias (d <= 64, interval masks), the producer also
 // loads each tile's block of the additive terms into the slot's shared memory
@@ -66,13 +68,12 @@ constexpr uint32_t kPpTmemCols = 512;
 constexpr float kPpRescale = 8.0f;               // log2 units
 constexpr long long kPpDrainCycles = 200000000LL;  // ~0.1 s per drain wait
 
-// mbarriers of slot s: kBarsPerSlot * s + one of these; kBarDrain after both slots
+// mbarriers of slot s: kBarsPerSlot * s + one of these
 enum : int {
-    kQFull = 0, kQEmpty, kKFull, kKEmpty, kVFull, kVEmpty, kSFull, kPFull, kODone, kOFree, kAFull, kAEmpty,
+    kQFull = 0, kQEmpty, kKFull, kKEmpty, kVFull, kVEmpty, kSFull, kPFull, kODone, kDrainS, kAFull, kAEmpty,
     kBarsPerSlot
 };
-constexpr int kBarDrain = 2 * kBarsPerSlot;
-constexpr int kNumBars = kBarDrain + 1;
+constexpr int kNumBars = 2 * kBarsPerSlot;
 
 template <int D, bool EXTRA>
 struct PpCfg {
@@ -371,8 +372,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < 2; ++s)
             for (int x = 0; x < kBarsPerSlot; ++x)
-                mbar_init(bar(s, x), (x == kPFull || x == kOFree || x == kAEmpty) ? 4u : 1u);
-        mbar_init(smem_u32(bars + kBarDrain), 1u);
+                mbar_init(bar(s, x), (x == kPFull || x == kAEmpty) ? 4u : 1u);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&tmQ);
@@ -516,97 +516,6 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                 }
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            struct Slot {
-                int m, u, T, phase;  // phase 0: S(g) next, 1: P V(g) next
-                uint32_t g, items;
-                bool live;
-            };
-            Slot sl[2];
-#pragma unroll
-            for (int s = 0; s < 2; ++s) {
-                sl[s].m = sl[s].u = sl[s].phase = sl[s].T = 0;
-                sl[s].g = sl[s].items = 0;
-                sl[s].live = seek(s, sl[s].m, sl[s].T);
-            }
-            const uint32_t idS = idesc_bf16_f32(128, 128, false);
-            const uint32_t idO = idesc_bf16_f32(128, D, true);
-            long long t_last = clock64();
-            while (true) {
-                bool all_done = true, progress = false;
-#pragma unroll
-                for (int s = 0; s < 2; ++s) {
-                    Slot& x = sl[s];
-                    if (!x.live) continue;
-                    all_done = false;
-                    const uint32_t tS = tmem + (uint32_t)(s * 256), tO = tS + 128;
-                    if (x.phase == 0) {
-                        // S(g) needs the item's Q, K(g), and P V(g-1) done (P overwrote S)
-                        const bool ready = (x.u != 0 || mbar_test(bar(s, kQFull), x.items & 1)) &&
-                                           mbar_test(bar(s, kKFull), x.g & 1) &&
-                                           (x.g == 0 || mbar_test(bar(s, kODone), (x.g - 1) & 1));
-                        if (ready) {
-                            tc_fence_after();
-                            const uint32_t sQ = sQ0 + s * C::TILE_BYTES, sK = sK0 + s * C::TILE_BYTES;
-#pragma unroll
-                            for (int ks = 0; ks < D / 16; ++ks) {
-                                const uint32_t off = (uint32_t)((ks / C::KSTEPS_PER_CHUNK) * C::CHUNK_BYTES +
-                                                                (ks % C::KSTEPS_PER_CHUNK) * 32);
-                                mma_bf16_ss(tS, smem_desc(sQ + off, 16, C::SBO, C::LAYOUT),
-                                            smem_desc(sK + off, 16, C::SBO, C::LAYOUT), idS, ks > 0 ? 1u : 0u);
-                            }
-                            mma_commit(bar(s, kSFull));
-                            mma_commit(bar(s, kKEmpty));
-                            if (x.u == x.T - 1) mma_commit(bar(s, kQEmpty));
-                            x.phase = 1;
-                            progress = true;
-                        }
-                    } else {
-                        // P V(g) needs P(g), V(g), and for an item's first tile the
-                        // previous item's O read out
-                        const bool ready = mbar_test(bar(s, kPFull), x.g & 1) &&
-                                           mbar_test(bar(s, kVFull), x.g & 1) &&
-                                           (x.u != 0 || x.items == 0 || mbar_test(bar(s, kOFree), (x.items - 1) & 1));
-                        if (ready) {
-                            tc_fence_after();
-                            const uint32_t sV = sV0 + s * C::TILE_BYTES;
-#pragma unroll
-                            for (int ks = 0; ks < 8; ++ks) {  // 16 keys per step
-                                const uint64_t db = smem_desc(sV + (uint32_t)(ks * 16 * C::ROW_BYTES), C::CHUNK_BYTES,
-                                                              C::SBO, C::LAYOUT);
-                                mma_bf16_ts(tO, tS + (uint32_t)(ks * 8), db, idO, (x.u > 0 || ks > 0) ? 1u : 0u);
-                            }
-                            mma_commit(bar(s, kODone));
-                            mma_commit(bar(s, kVEmpty));
-                            ++x.g;
-                            x.phase = 0;
-                            if (++x.u == x.T) {
-                                x.u = 0;
-                                ++x.items;
-                                ++x.m;
-                                x.live = seek(s, x.m, x.T);
-                            }
-                            progress = true;
-                        }
-                    }
-                }
-                if (all_done) break;
-                if (progress) {
-                    t_last = clock64();
-                } else {
-                    if (*abort_flag) break;
-                    if (clock64() - t_last > P.wait_cycles) {
-                        *abort_flag = 1;
-                        break;
-                    }
-                }
-            }
-            // every MMA issued is complete before the CTA releases TMEM
-            mma_commit(smem_u32(bars + kBarDrain));
-            mbar_wait_bounded(smem_u32(bars + kBarDrain), 0u, kPpDrainCycles);
-        }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ softmax groups
         regs_inc<kPpRegsHigh>();
@@ -616,12 +525,56 @@ __global__ void __launch_bounds__(kPpThreads, 1)
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const uint32_t tS = tmem + (uint32_t)(s * 256) + lane_base, tO = tS + 128;
         const uint64_t c2 = pack2(P.qk_scale_log2, P.qk_scale_log2);
-        uint32_t g = 0;
+        const bool leader = t == 0;  // issues this slot's MMAs
+        // MMAs of this slot (leader only). S(g) = Q K(g)^T into S's columns,
+        // then O (+)= P(g) V(g) with P read from the first 64 of them; since P
+        // overwrites S, S(g + 1) is issued only once P V(g) is complete.
+        const uint32_t tSm = tmem + (uint32_t)(s * 256), tOm = tSm + 128;
+        const uint32_t idS = idesc_bf16_f32(128, 128, false);
+        const uint32_t idO = idesc_bf16_f32(128, D, true);
+        // shared-memory descriptors at the Q buffer of slot 0 (K-major operands)
+        // and at the V buffer of slot 0 (MN-major B); a tile and k-step add
+        // their byte offset / 16 to the start-address field (bits 0-13)
+        const uint64_t dQK0 = smem_desc(sQ0, 16, C::SBO, C::LAYOUT);
+        const uint64_t dV0 = smem_desc(sV0, C::CHUNK_BYTES, C::SBO, C::LAYOUT);
+        // S(gs) once Q (the slot's active item number qi, on its first tile) and K(gs) are in
+        auto issue_s = [&](uint32_t gs, uint32_t qi, bool first, bool last) -> bool {
+            if (first && !pp_wait(bar(s, kQFull), qi & 1, abort_flag, P.wait_cycles)) return false;
+            if (!pp_wait(bar(s, kKFull), gs & 1, abort_flag, P.wait_cycles)) return false;
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const uint64_t off = (uint64_t)(((ks / C::KSTEPS_PER_CHUNK) * C::CHUNK_BYTES +
+                                                 (ks % C::KSTEPS_PER_CHUNK) * 32) >> 4);
+                mma_bf16_ss(tSm, dQK0 + (uint64_t)((C::OFF_Q + s * C::TILE_BYTES) >> 4) + off,
+                            dQK0 + (uint64_t)((C::OFF_K + s * C::TILE_BYTES) >> 4) + off, idS, ks > 0 ? 1u : 0u);
+            }
+            mma_commit(bar(s, kSFull));
+            mma_commit(bar(s, kKEmpty));
+            if (last) mma_commit(bar(s, kQEmpty));
+            return true;
+        };
+        // O (+)= P(gp) V(gp) once V(gp) is in (every row's P is written)
+        auto issue_pv = [&](uint32_t gp, bool first) -> bool {
+            if (!pp_wait(bar(s, kVFull), gp & 1, abort_flag, P.wait_cycles)) return false;
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {  // 16 keys per step
+                const uint64_t db = dV0 + (uint64_t)((s * C::TILE_BYTES + ks * 16 * C::ROW_BYTES) >> 4);
+                mma_bf16_ts(tOm, tSm + (uint32_t)(ks * 8), db, idO, (!first || ks > 0) ? 1u : 0u);
+            }
+            mma_commit(bar(s, kODone));
+            mma_commit(bar(s, kVEmpty));
+            return true;
+        };
+        uint32_t g = 0, qitems = 0;  // tiles and active items of this slot so far
         bool alive = true;
-        for (int m = 0; alive; ++m) {
-            const PpItem it = pp_item(P, sh, item_x(s, m));
-            if (!it.valid) break;
-            if (it.T <= 0) continue;
+        int m = 0, T0 = 0;
+        bool have = seek(s, m, T0);
+        if (leader && have && !issue_s(0, 0, true, T0 == 1)) *abort_flag = 1;
+        __syncwarp();
+        for (; alive && have; ++m) {
+            const PpItem it = pp_item(P, sh, item_x(s, m));  // seek found it: valid, with tiles
             int i;
             bool row_ok;
             int rlo = 0, rhi = 0;
@@ -694,123 +647,169 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                         break;
                     }
                 }
-                float x[128];
+                // Stream the tile 32 keys at a time (the next chunk's TMEM load is
+                // in flight while this one is processed): scale, additive terms,
+                // entries not in the mask to -inf, then p = 2^(x - m_ref) against
+                // the running reference max, row sum, bf16 P into TMEM. When a
+                // chunk's max exceeds the reference by more than 2^8 the
+                // reference moves to it and the P chunks already written (and
+                // the sum) are rescaled in place; O is rescaled after the tile.
+                // P of keys 32q .. 32q + 31 goes to columns 16q .. 16q + 15,
+                // which only hold S chunks already consumed.
+                float alpha_t = 1.f;  // product of this tile's rescales
+                float xa[32], xb[32];
+                if (need & 1u) tmem_ld32f(tS, xa);
+                tmem_wait_ld_depf(xa);
+#pragma unroll 1
+                for (int q = 0; q < 4; q += 2) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    if (need & (1u << q)) {
-                        uint32_t r[32];
-                        tmem_ld32(tS + 32 * q, r);
-                        tmem_wait_ld_dep(r);
+                    for (int hq = 0; hq < 2; ++hq) {
+                        const int qq = q + hq;
+                        float(&xc)[32] = hq == 0 ? xa : xb;
+                        float(&xn)[32] = hq == 0 ? xb : xa;
+                        // next chunk's load first (waited for at the end of this one)
+                        if (qq + 1 < 4 && (need & (2u << qq))) tmem_ld32f(tS + 32 * (qq + 1), xn);
+                        uint32_t pk[16];
+                        if (need & (1u << qq)) {
+                            const uint32_t wq = qq == 0 ? w[0] : (qq == 1 ? w[1] : (qq == 2 ? w[2] : w[3]));
 #pragma unroll
-                        for (int k = 0; k < 16; ++k) mul2(x[32 * q + 2 * k], x[32 * q + 2 * k + 1], r[2 * k], r[2 * k + 1], c2);
-                        if (EXTRA) {
-                            // + log2(e) * (mask + bias) of keys 32q .. 32q + 31: 16-byte
-                            // units 4 (q & 1) .. + 3 of chunk q / 2 of this row's line
-                            // (128-byte swizzle: unit j of row r at j ^ (r & 7))
+                            for (int k = 0; k < 32; ++k) xc[k] *= P.qk_scale_log2;
+                            if (EXTRA) {
+                                // + log2(e) * (mask + bias): 16-byte units 4 (qq & 1) ..
+                                // + 3 of chunk qq / 2 of this row's line (128-byte
+                                // swizzle: unit j of row r at j ^ (r & 7))
 #pragma unroll
-                            for (int a = 0; a < 2; ++a) {
-                                if (!P.extra[a]) continue;
-                                const int rows = P.a_rows[a], r0 = rows == 1 ? 0 : t;
-                                const uint8_t* base =
-                                    smem + C::OFF_A + (2 * s + a) * C::A_BYTES + (q >> 1) * rows * 128 + r0 * 128;
+                                for (int a = 0; a < 2; ++a) {
+                                    if (!P.extra[a]) continue;
+                                    const int rows = P.a_rows[a], r0 = rows == 1 ? 0 : t;
+                                    const uint8_t* base = smem + C::OFF_A + (2 * s + a) * C::A_BYTES +
+                                                          (qq >> 1) * rows * 128 + r0 * 128;
 #pragma unroll
-                                for (int uu = 0; uu < 4; ++uu) {
-                                    const int j = 4 * (q & 1) + uu;
-                                    const int ph = rows == 1 ? j : (j ^ (r0 & 7));
-                                    const uint4 v4 = *reinterpret_cast<const uint4*>(base + ph * 16);
-                                    const uint32_t ws[4] = {v4.x, v4.y, v4.z, v4.w};
+                                    for (int uu = 0; uu < 4; ++uu) {
+                                        const int j = 4 * (qq & 1) + uu;
+                                        const int ph = rows == 1 ? j : (j ^ (r0 & 7));
+                                        const uint4 v4 = *reinterpret_cast<const uint4*>(base + ph * 16);
+                                        const uint32_t ws[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
-                                    for (int e = 0; e < 4; ++e) {
-                                        x[32 * q + 8 * uu + 2 * e] += kLog2e * __uint_as_float(ws[e] << 16);
-                                        x[32 * q + 8 * uu + 2 * e + 1] += kLog2e * __uint_as_float(ws[e] & 0xffff0000u);
+                                        for (int e = 0; e < 4; ++e) {
+                                            xc[8 * uu + 2 * e] += kLog2e * __uint_as_float(ws[e] << 16);
+                                            xc[8 * uu + 2 * e + 1] += kLog2e * __uint_as_float(ws[e] & 0xffff0000u);
+                                        }
                                     }
                                 }
                             }
-                        }
-                        if (!dense) {
+                            if (!dense) {
 #pragma unroll
-                            for (int jj = 0; jj < 32; ++jj)
-                                x[32 * q + jj] = ((w[q] >> jj) & 1u) ? x[32 * q + jj] : -INFINITY;
-                        }
-                    } else {
+                                for (int k = 0; k < 32; ++k) xc[k] = ((wq >> k) & 1u) ? xc[k] : -INFINITY;
+                            }
+                            float ma = -INFINITY, mb = -INFINITY;
 #pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) x[32 * q + jj] = -INFINITY;
+                            for (int k = 0; k < 16; k += 2) {
+                                ma = fmax3(ma, xc[2 * k], xc[2 * k + 1]);
+                                mb = fmax3(mb, xc[2 * k + 2], xc[2 * k + 3]);
+                            }
+                            const float mx = fmaxf(ma, mb);
+                            const bool grow = mx > m_ref + kPpRescale;
+                            if (__any_sync(0xffffffffu, grow)) {
+                                // rare: new reference; P chunks 0 .. qq - 1 of this tile and
+                                // the sum scale by alpha (1 for rows that keep theirs)
+                                float alpha = 1.f;
+                                if (grow) {
+                                    alpha = ex2(m_ref - mx);
+                                    m_ref = mx;
+                                    l *= alpha;
+                                    alpha_t *= alpha;
+                                }
+                                tmem_wait_st();  // the P chunks written so far, before reading them back
+#pragma unroll 1
+                                for (int pq = 0; pq < qq; ++pq) {
+                                    uint32_t pw[16];
+                                    tmem_ld16(tS + 16 * pq, pw);
+                                    tmem_wait_ld_dep16(pw);
+#pragma unroll
+                                    for (int k = 0; k < 16; ++k) {
+                                        __nv_bfloat162 hv = __floats2bfloat162_rn(
+                                            __uint_as_float(pw[k] << 16) * alpha,
+                                            __uint_as_float(pw[k] & 0xffff0000u) * alpha);
+                                        pw[k] = *reinterpret_cast<uint32_t*>(&hv);
+                                    }
+                                    tmem_st16(tS + 16 * pq, pw);
+                                }
+                            }
+                            const float mu = m_ref == -INFINITY ? 0.f : m_ref;
+                            const uint64_t nmu2 = pack2(-mu, -mu);
+                            uint64_t sa = pack2(0.f, 0.f), sb = sa;
+#pragma unroll
+                            for (int k = 0; k < 16; ++k) {
+                                float p0, p1;
+                                unpack2(add2(pack2(xc[2 * k], xc[2 * k + 1]), nmu2), p0, p1);
+                                p0 = ex2(p0);
+                                p1 = ex2(p1);
+                                if (k & 1)
+                                    sb = add2(sb, pack2(p0, p1));
+                                else
+                                    sa = add2(sa, pack2(p0, p1));
+                                __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
+                                pk[k] = *reinterpret_cast<uint32_t*>(&hv);
+                            }
+                            float s0, s1, s2, s3;
+                            unpack2(sa, s0, s1);
+                            unpack2(sb, s2, s3);
+                            l += (s0 + s1) + (s2 + s3);
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < 16; ++k) pk[k] = 0u;
+                        }
+                        tmem_st16(tS + 16 * qq, pk);
+                        tmem_wait_ld_depf(xn);  // the next chunk's S
                     }
                 }
                 if (EXTRA) {  // the additive blocks are read: the producer may refill them
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(s, kAEmpty));
                 }
-                float ma = -INFINITY, mb = -INFINITY, mc = -INFINITY, md = -INFINITY;
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    ma = fmax3(ma, x[8 * k + 0], x[8 * k + 1]);
-                    mb = fmax3(mb, x[8 * k + 2], x[8 * k + 3]);
-                    mc = fmax3(mc, x[8 * k + 4], x[8 * k + 5]);
-                    md = fmax3(md, x[8 * k + 6], x[8 * k + 7]);
-                }
-                const float mx = fmax3(ma, mb, fmaxf(mc, md));
-                const bool grow = mx > m_ref + kPpRescale;
-                float alpha = 1.f;
-                if (grow) {
-                    alpha = ex2(m_ref - mx);
-                    m_ref = mx;
-                    l *= alpha;
-                }
-                if (u > 0 && __any_sync(0xffffffffu, grow)) {
-                    // bring O (P V of the item's tiles so far, complete) to the new max
+                if (u > 0 && __any_sync(0xffffffffu, alpha_t != 1.f)) {
+                    // bring O (P V of the item's tiles so far, complete) to the new reference
                     const bool ok2 = pp_wait(bar(s, kODone), (g - 1) & 1, abort_flag, P.wait_cycles);
                     if (!__all_sync(0xffffffffu, ok2)) {
                         alive = false;
                         break;
                     }
                     tc_fence_after();
-#pragma unroll
+#pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t ro[32];
                         tmem_ld32(tO + 32 * c, ro);
                         tmem_wait_ld_dep(ro);
 #pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) ro[jj] = __float_as_uint(__uint_as_float(ro[jj]) * alpha);
+                        for (int jj = 0; jj < 32; ++jj) ro[jj] = __float_as_uint(__uint_as_float(ro[jj]) * alpha_t);
                         tmem_st32(tO + 32 * c, ro);
                     }
-                }
-                const float mu = m_ref == -INFINITY ? 0.f : m_ref;
-                const uint64_t nmu2 = pack2(-mu, -mu);
-                uint64_t sa = pack2(0.f, 0.f), sb = sa;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t pk[16];
-                    if (need & (1u << q)) {
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) {
-                            float p0, p1;
-                            unpack2(add2(pack2(x[32 * q + 2 * k], x[32 * q + 2 * k + 1]), nmu2), p0, p1);
-                            p0 = ex2(p0);
-                            p1 = ex2(p1);
-                            if (k & 1)
-                                sb = add2(sb, pack2(p0, p1));
-                            else
-                                sa = add2(sa, pack2(p0, p1));
-                            __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
-                            pk[k] = *reinterpret_cast<uint32_t*>(&hv);
-                        }
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) pk[k] = 0u;
-                    }
-                    tmem_st16(tS + 16 * q, pk);  // P keys 32q .. 32q + 31: columns 16q .. 16q + 15
-                }
-                {
-                    float s0, s1, s2, s3;
-                    unpack2(sa, s0, s1);
-                    unpack2(sb, s2, s3);
-                    l += (s0 + s1) + (s2 + s3);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(s, kPFull));
+                if (leader) {
+                    // every row's P(g) is in TMEM: P V(g); then, once it has consumed
+                    // P, the next S -- this item's next tile or the next item's first
+                    bool okl = pp_wait(bar(s, kPFull), g & 1, abort_flag, P.wait_cycles) && issue_pv(g, u == 0);
+                    if (okl) {
+                        int mn = m, Tn = it.T;
+                        bool nxt = u + 1 < it.T, first = false;
+                        if (!nxt) {
+                            mn = m + 1;
+                            nxt = seek(s, mn, Tn);
+                            first = true;
+                        }
+                        const int un = first ? 0 : u + 1;
+                        if (nxt)
+                            okl = pp_wait(bar(s, kODone), g & 1, abort_flag, P.wait_cycles) &&
+                                  issue_s(g + 1, qitems + (first ? 1 : 0), first, un == Tn - 1);
+                    }
+                    if (!okl) *abort_flag = 1;
+                }
+                __syncwarp();
             }
             if (!alive) break;
             // ---------------------------------------------------------- epilogue
@@ -818,19 +817,25 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             float o[D];
+            {  // O loaded in place as fp32, all loads issued before one wait
+                float(&oc)[D / 32][32] = *reinterpret_cast<float(*)[D / 32][32]>(&o);
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t ro[32];
-                tmem_ld32(tO + 32 * c, ro);
-                tmem_wait_ld_dep(ro);
+                for (int c = 0; c < D / 32; ++c) tmem_ld32f(tO + 32 * c, oc[c]);
+                tmem_wait_ld_depf(oc[0]);
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) o[32 * c + jj] = __uint_as_float(ro[jj]);
+                for (int c = 1; c < D / 32; ++c) reg_fence32f(oc[c]);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(s, kOFree));  // the next item's P V may overwrite O
             pp_finish<D>(P, sh, it, quarter, t, i, row_ok, m_ref, l, o);
             __syncwarp();
+            ++qitems;
+            int Tn = 0;
+            ++m;
+            have = seek(s, m, Tn);
+            --m;  // the loop's ++m moves to it
+        }
+        if (leader) {  // every MMA this thread issued is complete before TMEM is released
+            mma_commit(bar(s, kDrainS));
+            mbar_wait_bounded(bar(s, kDrainS), 0u, kPpDrainCycles);
         }
     }
 
