@@ -109,26 +109,31 @@ struct Item {
     int T;      // tiles of this item
 };
 
-// Item x of all B*H*items_per_head: per (b, h) the chunks of query block 0
-// first (most tiles), then regular and permuted blocks alternately (their
-// rows meet in the merge, so they run close together), then the rest.
-BSG_HD Item item(const Shape& s, int64_t x) {
+// Item x of all bh_count * items_per_head: first the chunks of query block 0
+// of every (b, h) (the items with the most tiles, so that they spread over
+// the workers before the short ones), then per (b, h) its regular and
+// permuted blocks alternately (their rows meet in the merge, so they run
+// close together), then the rest.
+BSG_HD Item item(const Shape& s, int64_t x, int bh_count) {
     Item it;
-    it.bh = (int)(x / s.items_per_head);
-    int j = (int)(x - (int64_t)it.bh * s.items_per_head);
     it.perm = 0;
     it.qb = 0;
     it.pqb = 0;
     it.chunk = 0;
     it.u0 = 0;
-    if (j < s.n_lead) {
+    const int64_t leads = (int64_t)bh_count * s.n_lead;
+    if (x < leads) {
+        it.bh = (int)(x / s.n_lead);
+        const int j = (int)(x - (int64_t)it.bh * s.n_lead);
         it.chunk = j;
         it.u0 = j * s.chunk_tiles;
         const int rest = s.nqb - it.u0;
         it.T = rest < s.chunk_tiles ? rest : s.chunk_tiles;
         return it;
     }
-    j -= s.n_lead;
+    const int per = s.items_per_head - s.n_lead;
+    it.bh = (int)((x - leads) / per);
+    int j = (int)((x - leads) - (int64_t)it.bh * per);
     const int both = s.nreg < s.nperm ? s.nreg : s.nperm;
     int reg = -1, perm = -1;
     if (j < 2 * both) {

@@ -17,8 +17,9 @@
 // when that has consumed P, S(g + 1) = Q K(g + 1)^T, which its warps are
 // waiting for. While one slot's group turns S into P, the tensor cores work on
 // the other slot, so the two dependency chains overlap. The producer polls both
-// slots with non-blocking barrier tests and loads whichever buffer is free;
-// every wait is bounded.
+// slots with non-blocking barrier tests, loads whichever buffer is free, and
+// sleeps briefly when nothing is (it shares a sub-partition with two softmax
+// warps); every wait is bounded.
 //
 // Per tile, each thread streams its row of S 32 keys at a time (the next
 // chunk's TMEM load in flight): scale, entries the mask does not list to -inf,
@@ -144,7 +145,7 @@ __device__ __forceinline__ PpItem pp_item(const PpParams& P, const bsg::Shape& s
             while (it.T > 1 && (__ldg(P.itv_tiles + it.blk * P.nkt + it.T - 1) & 0x7fffffff) * 128 >= L) --it.T;
         }
     } else {
-        const bsg::Item bi = bsg::item(sh, x);
+        const bsg::Item bi = bsg::item(sh, x, P.B * P.H);
         it.bh = bi.bh;
         it.b = bi.bh / P.H;
         it.h = bi.bh - it.b * P.H;
@@ -430,6 +431,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                     live[s][k] = seek(s, sm[s][k], sT[s][k]);
                 }
             long long t_last = clock64();
+            unsigned nap = 0;  // back-off when a pass finds nothing to load
             while (true) {
                 bool any = false, progress = false;
 #pragma unroll
@@ -498,7 +500,12 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                 if (!any) break;
                 if (progress) {
                     t_last = clock64();
+                    nap = 0;
                 } else {
+                    // loads run microseconds ahead of their use: sleep rather than
+                    // take issue slots from the softmax warps on this sub-partition
+                    nap = nap ? (nap < 256 ? 2 * nap : 256) : 32;
+                    __nanosleep(nap);
                     if (*abort_flag) break;
                     if (clock64() - t_last > P.wait_cycles) {
                         *abort_flag = 1;

@@ -1144,7 +1144,7 @@ int create_closed(const spattn_mask_spec& sp, cudaStream_t s, int dev, spattn_ma
     // tiles of one forward per (b, h): chunks of block 0, further regular
     // blocks, permuted blocks (each over every permuted key tile)
     int64_t tiles = 0;
-    for (int64_t x = 0; x < sh.items_per_head; ++x) tiles += bsg::item(sh, x).T;
+    for (int64_t x = 0; x < sh.items_per_head; ++x) tiles += bsg::item(sh, x, 1).T;
     spattn_mask m = new spattn_mask_s;
     memset(m, 0, sizeof *m);
     m->device = dev;

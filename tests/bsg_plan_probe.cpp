@@ -1,7 +1,8 @@
 // Test driver for the closed-form block + strided + global tile plan
 // (sparse_mask_scaled_b200/csrc/bsg_plan.cuh), built for the host by
 // tests/test_bsg_plan_cpu.py. For the parameters on the command line it walks
-// every work item of one (b, h), every tile and every row's bits, and writes
+// the work items of three (b, h) heads, keeps those of head 1, and for every
+// tile and every row's bits writes
 // to stdout, as raw bytes: the n x n count of how many times each entry (i, j)
 // is computed (uint8), the per-row "has entries in a permuted block" flag
 // computed from the bits (uint8 [n]) and the one bsg::has_perm reports (uint8
@@ -22,9 +23,12 @@ int main(int argc, char** argv) {
     if (!supported(n, block, S, ng)) return 2;
     const Shape s = shape(n, block, S, ng, chunk);
     std::vector<uint8_t> cnt((size_t)n * n, 0), perm_rows(n, 0), has(n, 0);
-    for (int64_t x = 0; x < s.items_per_head; ++x) {
-        const Item it = item(s, x);
-        if (it.bh != 0) return 3;
+    // every item of three (b, h) heads (the order interleaves heads), keeping head 1's
+    const int heads = 3;
+    for (int64_t x = 0; x < (int64_t)heads * s.items_per_head; ++x) {
+        const Item it = item(s, x, heads);
+        if (it.bh < 0 || it.bh >= heads) return 3;
+        if (it.bh != 1) continue;
         for (int u = 0; u < it.T; ++u) {
             const int kt = key_tile(s, it, u);
             for (int t = 0; t < kTile; ++t) {
