@@ -109,52 +109,61 @@ struct Item {
     int T;      // tiles of this item
 };
 
-// Item x of all bh_count * items_per_head: first the chunks of query block 0
-// of every (b, h) (the items with the most tiles, so that they spread over
-// the workers before the short ones), then per (b, h) its regular and
-// permuted blocks alternately (their rows meet in the merge, so they run
-// close together), then the rest.
+// Item x of all bh_count * items_per_head, in groups: group 0 holds the
+// permuted blocks of (b, h) 0; group g >= 1 the regular blocks of (b, h) g - 1
+// (the chunks of query block 0 first, the items with the most tiles) and then
+// the permuted blocks of (b, h) g. Every regular block of a (b, h) comes after
+// all of its permuted blocks: rows met by both start their regular part from
+// the permuted part's published state, and items taken in this order never
+// wait for a later one.
 BSG_HD Item item(const Shape& s, int64_t x, int bh_count) {
+    (void)bh_count;
     Item it;
     it.perm = 0;
     it.qb = 0;
     it.pqb = 0;
     it.chunk = 0;
     it.u0 = 0;
-    const int64_t leads = (int64_t)bh_count * s.n_lead;
-    if (x < leads) {
-        it.bh = (int)(x / s.n_lead);
-        const int j = (int)(x - (int64_t)it.bh * s.n_lead);
+    const int nregular = s.n_lead + s.nreg;
+    int j;
+    if (x < s.nperm) {
+        it.bh = 0;
+        it.perm = 1;
+        j = (int)x;
+    } else {
+        const int64_t y = x - s.nperm;
+        it.bh = (int)(y / s.items_per_head);
+        j = (int)(y - (int64_t)it.bh * s.items_per_head);
+        if (j >= nregular) {
+            it.perm = 1;
+            j -= nregular;
+            ++it.bh;
+        }
+    }
+    if (it.perm) {
+        it.qb = j / s.npqb;
+        it.pqb = j - it.qb * s.npqb;
+        it.T = s.npqb;
+        return it;
+    }
+    if (j < s.n_lead) {  // a chunk of query block 0 (a mask with global rows)
         it.chunk = j;
         it.u0 = j * s.chunk_tiles;
         const int rest = s.nqb - it.u0;
         it.T = rest < s.chunk_tiles ? rest : s.chunk_tiles;
         return it;
     }
-    const int per = s.items_per_head - s.n_lead;
-    it.bh = (int)((x - leads) / per);
-    int j = (int)((x - leads) - (int64_t)it.bh * per);
-    const int both = s.nreg < s.nperm ? s.nreg : s.nperm;
-    int reg = -1, perm = -1;
-    if (j < 2 * both) {
-        if (j & 1) perm = j >> 1;
-        else reg = j >> 1;
-    } else if (s.nreg > s.nperm) {
-        reg = j - both;
-    } else {
-        perm = j - both;
-    }
-    if (reg >= 0) {
-        it.qb = reg + (s.ng > 0 ? 1 : 0);
-        // tiles 0 (global keys) and qb (block); block 0 here only when ng == 0
-        it.T = (s.ng > 0 ? 1 : 0) + (s.block > 0 ? 1 : 0);
-        return it;
-    }
-    it.perm = 1;
-    it.qb = perm / s.npqb;
-    it.pqb = perm - it.qb * s.npqb;
-    it.T = s.npqb;
+    it.qb = j - s.n_lead + (s.ng > 0 ? 1 : 0);
+    // tiles 0 (global keys) and qb (block); block 0 here only when ng == 0
+    it.T = (s.ng > 0 ? 1 : 0) + (s.block > 0 ? 1 : 0);
     return it;
+}
+
+// Whether a regular item starts from the published state of its rows'
+// permuted parts (the item that holds tile 0 of a query block, when the
+// pattern has permuted blocks).
+BSG_HD bool starts_from_perm(const Shape& s, const Item& it) {
+    return s.G > 0 && !it.perm && it.chunk == 0;
 }
 
 // Key tile of the item's tile u: a key tile for regular items (ascending),

@@ -96,10 +96,16 @@ struct PpCfg {
     // chunks of 128-byte rows (128-byte swizzle)
     static constexpr int A_BYTES = 2 * 128 * 128;
     static constexpr int OFF_A = 6 * TILE_BYTES;
-    static constexpr int OFF_BAR = OFF_A + (EXTRA ? 4 * A_BYTES : 0);
+    // per softmax warp a 4 KB buffer through which the epilogue's global
+    // accesses go as whole lines (when it fits beside the tiles)
+    static constexpr int STG_BYTES = 8 * 4096;
+    static constexpr bool STAGE = OFF_A + (EXTRA ? 4 * A_BYTES : 0) + STG_BYTES + kNumBars * 8 + 16 + 80 <= 227 * 1024;
+    static constexpr int OFF_STG = OFF_A + (EXTRA ? 4 * A_BYTES : 0);
+    static constexpr int OFF_BAR = OFF_STG + (STAGE ? STG_BYTES : 0);
     static constexpr int OFF_INT = OFF_BAR + kNumBars * 8;  // TMEM base, abort flag
+    static constexpr int OFF_RING = OFF_INT + 16;            // [slot][4] items taken (int64), then [slot] counts
     // at least 116 KB, so that one CTA (which takes all 512 TMEM columns) runs per SM
-    static constexpr int SMEM_BYTES = OFF_INT + 16 > 116 * 1024 ? OFF_INT + 16 : 116 * 1024;
+    static constexpr int SMEM_BYTES = OFF_RING + 80 > 116 * 1024 ? OFF_RING + 80 : 116 * 1024;
 };
 
 // A work item as every role sees it.
@@ -207,62 +213,170 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
     return v;
 }
 
-// Writes row i of (b, h): out = o / L (bf16, round to nearest even), lse = (M + log2 L) ln 2.
-template <int D>
-__device__ __forceinline__ void pp_write_row(const PpParams& P, int b, int h, int64_t bh, int i, float M, float L,
-                                             const float (&o)[D]) {
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(P.out) + (int64_t)b * P.o_sb + (int64_t)h * P.o_sh +
-                          (int64_t)i * P.o_sn;
-#pragma unroll
-    for (int e8 = 0; e8 < D / 8; ++e8) {
-        uint32_t w[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            __nv_bfloat162 hv = __floats2bfloat162_rn(o[e8 * 8 + 2 * t] * inv, o[e8 * 8 + 2 * t + 1] * inv);
-            w[t] = *reinterpret_cast<uint32_t*>(&hv);
-        }
-        *reinterpret_cast<uint4*>(orow + e8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-    if (P.lse) P.lse[bh * P.n + i] = L > 0.f ? (M + lg2(L)) * kLn2 : -INFINITY;
+__device__ __forceinline__ void st_shared_v4(uint32_t a, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a) : "memory");
+    return v;
 }
 
-// The end of one item for one warp's rows: state (M, L, o) in base 2, o not
-// yet divided by L. Merges what the row has elsewhere, then writes it (or
-// publishes it for the row's partner).
-template <int D>
+// Rows between registers (lane = row) and global memory through a warp's
+// 4 KB shared-memory buffer, so that each global instruction of the warp
+// covers whole lines (128 / (16 UNITS) rows of 16 UNITS bytes) instead of one
+// 16-byte piece in each of 32 lines. Unit u of row r sits at
+// r * 128 + ((u ^ (r & 7)) << 4), which keeps both the row-per-lane and the
+// line-per-lane-group accesses free of bank conflicts. A row address of 0
+// skips the row. All 32 lanes take part.
+template <int UNITS>
+__device__ __forceinline__ void rows_store(uint32_t stg, int lane, const uint32_t (&w)[4 * UNITS], uint64_t dst) {
+    static_assert(UNITS == 4 || UNITS == 8, "row pieces of 64 or 128 bytes");
+#pragma unroll
+    for (int u = 0; u < UNITS; ++u)
+        st_shared_v4(stg + lane * 128 + ((u ^ (lane & 7)) << 4), make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]));
+    __syncwarp();
+    constexpr int RPI = 32 / UNITS;  // rows per instruction
+    const int u = lane % UNITS;
+#pragma unroll
+    for (int k = 0; k < UNITS; ++k) {
+        const int r = RPI * k + lane / UNITS;
+        const uint64_t p = __shfl_sync(0xffffffffu, dst, r);
+        const uint4 v = ld_shared_v4(stg + r * 128 + ((u ^ (r & 7)) << 4));
+        if (p) *reinterpret_cast<uint4*>(p + u * 16) = v;
+    }
+    __syncwarp();
+}
+
+// 128-byte rows from global memory (read at L2, written by another CTA) into
+// registers, the reverse of rows_store; with DISCARD the lines read are
+// dropped from L2 afterwards, unwritten.
+template <bool DISCARD>
+__device__ __forceinline__ void rows_load(uint32_t stg, int lane, uint32_t (&w)[32], uint64_t src) {
+    const int u = lane & 7;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {  // two batches of four lines in flight
+        uint4 v[4];
+        uint64_t p[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int r = 16 * h + 4 * k + (lane >> 3);
+            p[k] = __shfl_sync(0xffffffffu, src, r);
+            v[k] = p[k] ? __ldcg(reinterpret_cast<const uint4*>(p[k] + u * 16)) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int r = 16 * h + 4 * k + (lane >> 3);
+            st_shared_v4(stg + r * 128 + ((u ^ (r & 7)) << 4), v[k]);
+            if (DISCARD && p[k] && u == 0) discard_l2_line(reinterpret_cast<const void*>(p[k]));
+        }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int uu = 0; uu < 8; ++uu) {
+        const uint4 x = ld_shared_v4(stg + lane * 128 + ((uu ^ (lane & 7)) << 4));
+        w[4 * uu] = x.x;
+        w[4 * uu + 1] = x.y;
+        w[4 * uu + 2] = x.z;
+        w[4 * uu + 3] = x.w;
+    }
+    __syncwarp();
+}
+
+// 32 columns of this warp's rows of O (fp32, not yet divided by L) from TMEM.
+__device__ __forceinline__ void o_chunk(uint32_t tO, int c, float (&x)[32]) {
+    tmem_ld32f(tO + 32 * c, x);
+    tmem_wait_ld_depf(x);
+}
+
+// Output piece p (64 columns, or 32 when D == 32) of the rows whose address
+// orow is not 0: bf16(x * inv), round to nearest even.
+template <int D, bool STAGE>
+__device__ __forceinline__ void put_out_piece(uint64_t orow, int p, float inv, const float (&xa)[32], const float (&xb)[32],
+                                              uint32_t stg, int lane) {
+    constexpr int CW = D >= 64 ? 64 : 32;
+    uint32_t w[CW / 2];
+#pragma unroll
+    for (int k = 0; k < CW / 2; ++k) {
+        const float x0 = k < 16 ? xa[2 * k] : xb[2 * k - 32], x1 = k < 16 ? xa[2 * k + 1] : xb[2 * k - 31];
+        __nv_bfloat162 hv = __floats2bfloat162_rn(x0 * inv, x1 * inv);
+        w[k] = *reinterpret_cast<uint32_t*>(&hv);
+    }
+    const uint64_t dst = orow ? orow + (uint64_t)p * CW * 2 : 0ull;
+    if (STAGE) {
+        rows_store<CW / 8>(stg, lane, w, dst);
+    } else if (dst) {
+#pragma unroll
+        for (int u = 0; u < CW / 8; ++u)
+            *reinterpret_cast<uint4*>(dst + u * 16) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+    }
+}
+
+// The end of one item for one warp's rows: state (M, L) in base 2 in
+// registers, O (not yet divided by L) in TMEM at tO, streamed 32 columns at a
+// time. Interval masks merge the gather kernel's partial state where there is
+// one; chunks of a split block merge through the chunk states; a permuted
+// block publishes its rows' state; the rest writes the rows. All 32 lanes
+// take part; with STAGE the published rows and the output rows move as whole
+// lines through the warp's staging buffer stg.
+template <int D, bool STAGE>
 __device__ __forceinline__ void pp_finish(const PpParams& P, const bsg::Shape& sh, const PpItem& it, int quarter, int t, int i,
-                          bool row_ok, float M, float L, float (&o)[D]) {
+                          bool row_ok, float M, float L, uint32_t tO, uint32_t stg) {
     const int lane = threadIdx.x & 31;
     const int64_t bh = it.bh;
+    const uint64_t orow_any = reinterpret_cast<uint64_t>(reinterpret_cast<__nv_bfloat16*>(P.out) + (int64_t)it.b * P.o_sb +
+                                                         (int64_t)it.h * P.o_sh + (int64_t)(row_ok ? i : 0) * P.o_sn);
     if (P.mode == 0) {
-        if (!row_ok) return;
-        const int64_t wrow = bh * P.n + i;
-        if (P.blk_res && __ldg(P.blk_res + it.blk) && P.ws_ml[wrow * 2 + 1] > 0.f) {
-            // the gather kernel's partial state of the row's other entries
+        const int64_t wrow = bh * P.n + (row_ok ? i : 0);
+        // rows that also have gathered entries: the gather kernel's partial state
+        const bool gm = row_ok && P.blk_res && __ldg(P.blk_res + it.blk) && P.ws_ml[wrow * 2 + 1] > 0.f;
+        float fa = 1.f, fg = 0.f;
+        if (gm) {
             const float mg = P.ws_ml[wrow * 2], lg = P.ws_ml[wrow * 2 + 1];
             const float Mn = fmaxf(M, mg);
             const float Mu = Mn == -INFINITY ? 0.f : Mn;
-            const float fa = ex2(M - Mu), fg = ex2(mg - Mu);
-            const float* acc = P.ws_acc + wrow * D;
-#pragma unroll
-            for (int e = 0; e < D; ++e) o[e] = fmaf(acc[e], fg, o[e] * fa);
+            fa = ex2(M - Mu);
+            fg = ex2(mg - Mu);
             L = L * fa + lg * fg;
             M = Mn;
         }
-        pp_write_row<D>(P, it.b, it.h, bh, i, M, L, o);
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        const float* acc = P.ws_acc + wrow * D;
+#pragma unroll
+        for (int p = 0; p < (D >= 64 ? D / 64 : 1); ++p) {
+            float xa[32], xb[32];
+            o_chunk(tO, (D >= 64 ? 2 : 1) * p, xa);
+            if (D >= 64) o_chunk(tO, 2 * p + 1, xb);
+            if (gm) {
+#pragma unroll
+                for (int z = 0; z < 32; ++z) {
+                    xa[z] = fmaf(acc[(D >= 64 ? 64 : 32) * p + z], fg, xa[z] * fa);
+                    if (D >= 64) xb[z] = fmaf(acc[64 * p + 32 + z], fg, xb[z] * fa);
+                }
+            }
+            put_out_piece<D, STAGE>(row_ok ? orow_any : 0ull, p, inv, xa, xb, stg, lane);
+        }
+        if (row_ok && P.lse) P.lse[bh * P.n + i] = L > 0.f ? (M + lg2(L)) * kLn2 : -INFINITY;
         return;
     }
 
     if (!it.perm && sh.nch > 1 && it.qb == 0) {
-        // one chunk of the global-row block: publish, and the warp that
-        // completes this quarter's count merges all chunks (in chunk order)
+        // one chunk of the global-row block: publish its state, and the warp
+        // that completes this quarter's count merges all chunks' states into
+        // its O (the layout (chunk, value, row) keeps the accesses on whole lines)
         float* mine = P.cws + ((bh * sh.nch + it.chunk) * (int64_t)(D + 2)) * 128 + t;
         mine[0] = M;
         mine[128] = L;
-        if (L > 0.f) {
+        if (__any_sync(0xffffffffu, L > 0.f)) {
 #pragma unroll
-            for (int e = 0; e < D; ++e) mine[(int64_t)(2 + e) * 128] = o[e];
+            for (int c = 0; c < D / 32; ++c) {
+                float x[32];
+                o_chunk(tO, c, x);
+                if (L > 0.f) {
+#pragma unroll
+                    for (int z = 0; z < 32; ++z) mine[(int64_t)(2 + 32 * c + z) * 128] = x[z];
+                }
+            }
         }
         __threadfence();
         __syncwarp();
@@ -271,77 +385,78 @@ __device__ __forceinline__ void pp_finish(const PpParams& P, const bsg::Shape& s
         last = __shfl_sync(0xffffffffu, last, 0);
         if (!last) return;
         __threadfence();
-        M = -INFINITY;
-        L = 0.f;
-#pragma unroll
-        for (int e = 0; e < D; ++e) o[e] = 0.f;
+        const float* base = P.cws + (bh * sh.nch * (int64_t)(D + 2)) * 128 + t;
+        const int64_t rec = (int64_t)(D + 2) * 128;  // floats per chunk record
+        float Mf = -INFINITY;
+        for (int c = 0; c < sh.nch; ++c)
+            if (__ldcg(base + c * rec + 128) > 0.f) Mf = fmaxf(Mf, __ldcg(base + c * rec));
+        float Lf = 0.f;
         for (int c = 0; c < sh.nch; ++c) {
-            const float* pp = P.cws + ((bh * sh.nch + c) * (int64_t)(D + 2)) * 128 + t;
-            const float mc = __ldcg(pp), lc = __ldcg(pp + 128);
-            if (!(lc > 0.f)) continue;
-            const float Mn = fmaxf(M, mc);
-            const float fa = ex2(M - Mn), fb = ex2(mc - Mn);
-#pragma unroll
-            for (int e = 0; e < D; ++e) o[e] = fmaf(__ldcg(pp + (int64_t)(2 + e) * 128), fb, o[e] * fa);
-            L = L * fa + lc * fb;
-            M = Mn;
+            const float lc = __ldcg(base + c * rec + 128);
+            if (lc > 0.f) Lf += lc * ex2(__ldcg(base + c * rec) - Mf);
         }
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+            float acc[32];
+#pragma unroll
+            for (int z = 0; z < 32; ++z) acc[z] = 0.f;
+            for (int c = 0; c < sh.nch; ++c) {
+                const float lc = __ldcg(base + c * rec + 128);
+                if (!(lc > 0.f)) continue;
+                const float wgt = ex2(__ldcg(base + c * rec) - Mf);
+                const float* src = base + c * rec + (int64_t)(2 + 32 * cc) * 128;
+#pragma unroll
+                for (int z = 0; z < 32; ++z) acc[z] = fmaf(__ldcg(src + (int64_t)z * 128), wgt, acc[z]);
+            }
+            uint32_t w[32];
+#pragma unroll
+            for (int z = 0; z < 32; ++z) w[z] = __float_as_uint(acc[z]);
+            tmem_st32(tO + 32 * cc, w);
+        }
+        tmem_wait_st();
+        M = Mf;
+        L = Lf;
     }
-    if (!row_ok) return;
-    const bool partner = bsg::has_perm(sh, i);
-    if (it.perm && !partner) return;  // no strided entries of this row here
-    if (partner) {
-        const int64_t prow = bh * P.n + i;
-        unsigned* cnt = P.pcnt + prow;
-        float* pm = P.pml + prow * 2;
-        float* pa = P.pacc + prow * D;
-        const unsigned old = atomicAdd(cnt, 1u);
-        if (old == 0u) {  // first: publish the state for the partner
-            pm[0] = M;
-            pm[1] = L;
-#pragma unroll
-            for (int e = 0; e < D; e += 4)
-                *reinterpret_cast<float4*>(pa + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
-            __threadfence();
-            atomicAdd(cnt, 2u);
-            return;
+    if (it.perm) {
+        // a permuted block publishes the state of its rows (their regular
+        // block starts from it); the count of its four warps releases it
+        const bool pr = row_ok && bsg::has_perm(sh, i);
+        const int64_t prow = bh * P.n + (pr ? i : 0);
+        if (pr) {
+            P.pml[prow * 2] = M;
+            P.pml[prow * 2 + 1] = L;
         }
-        // second: the partner's state is complete once the count reaches 4
-        if (ld_acquire_u32(cnt) != 4u) {
-            const long long t0 = clock64();
-            while (ld_acquire_u32(cnt) != 4u) {
-                if (clock64() - t0 > P.wait_cycles) {
-                    atomicOr(P.err, kErrTimeout);
-                    return;
-                }
-                __nanosleep(64);
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+            float x[32];
+            o_chunk(tO, c, x);
+            if (STAGE) {
+                uint32_t w[32];
+#pragma unroll
+                for (int z = 0; z < 32; ++z) w[z] = __float_as_uint(x[z]);
+                rows_store<8>(stg, lane, w, pr ? reinterpret_cast<uint64_t>(P.pacc + prow * D + 32 * c) : 0ull);
+            } else if (pr) {
+#pragma unroll
+                for (int z = 0; z < 32; z += 4)
+                    *reinterpret_cast<float4*>(P.pacc + prow * D + 32 * c + z) = make_float4(x[z], x[z + 1], x[z + 2], x[z + 3]);
             }
         }
+        // every lane's stores (lanes write other rows' lines) before the count
         __threadfence();
-        const float Mq = __ldcg(pm), Lq = __ldcg(pm + 1);
-        // regular part first, whichever of the two arrived last
-        const float Mr = it.perm ? Mq : M, Lr = it.perm ? Lq : L;
-        const float Mp = it.perm ? M : Mq, Lp = it.perm ? L : Lq;
-        const float Mn = fmaxf(Mr, Mp);
-        const float Mu = Mn == -INFINITY ? 0.f : Mn;
-        const float fr = ex2(Mr - Mu), fp = ex2(Mp - Mu);
-#pragma unroll
-        for (int e = 0; e < D; e += 4) {
-            const float4 q4 = __ldcg(reinterpret_cast<const float4*>(pa + e));
-            const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
-#pragma unroll
-            for (int z = 0; z < 4; ++z) {
-                const float orr = it.perm ? qv[z] : o[e + z], opp = it.perm ? o[e + z] : qv[z];
-                o[e + z] = fmaf(opp, fp, orr * fr);
-            }
-        }
-        L = Lr * fr + Lp * fp;
-        M = Mn;
-        // the published lines are read exactly once: drop them from L2 unwritten
-#pragma unroll
-        for (int z = 0; z < D * 4 / 128; ++z) discard_l2_line(pa + z * 32);
+        __syncwarp();
+        if (lane == 0) atomicAdd(P.pflag + (bh * sh.npqb + it.pqb) * 128 + it.qb, 1u);
+        return;
     }
-    pp_write_row<D>(P, it.b, it.h, bh, i, M, L, o);
+    // a regular block's rows: the output (their permuted part, if any, is in O already)
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll 1
+    for (int p = 0; p < (D >= 64 ? D / 64 : 1); ++p) {
+        float xa[32], xb[32];
+        o_chunk(tO, (D >= 64 ? 2 : 1) * p, xa);
+        if (D >= 64) o_chunk(tO, 2 * p + 1, xb);
+        put_out_piece<D, STAGE>(row_ok ? orow_any : 0ull, p, inv, xa, xb, stg, lane);
+    }
+    if (row_ok && P.lse) P.lse[bh * P.n + i] = L > 0.f ? (M + lg2(L)) * kLn2 : -INFINITY;
 }
 
 template <int D, bool EXTRA>
@@ -366,8 +481,13 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     auto bar = [&](int s, int which) { return smem_u32(bars + s * kBarsPerSlot + which); };
     const uint32_t sQ0 = smem_u32(smem + C::OFF_Q), sK0 = smem_u32(smem + C::OFF_K),
                    sV0 = smem_u32(smem + C::OFF_V);
-    // item j of this CTA (slot j & 1)
-    auto item_x = [&](int s, int m) { return (int64_t)blockIdx.x + (int64_t)(2 * m + s) * gridDim.x; };
+    // per slot a ring of the items it has taken (the m-th at entry m & 3, -1
+    // after the last), written by the producer before it arms the slot's QFull
+    // barrier for that item and before it raises the slot's count of entries
+    // (the softmax warps go by the count: the producer may be two Q loads
+    // ahead of them, where a barrier's phase parity would not tell)
+    volatile int64_t* ring = reinterpret_cast<volatile int64_t*>(smem + C::OFF_RING);
+    volatile int* ring_n = reinterpret_cast<volatile int*>(smem + C::OFF_RING + 64);
 
     if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kPpTmemCols);
     if (tid == 0) {
@@ -375,6 +495,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             for (int x = 0; x < kBarsPerSlot; ++x)
                 mbar_init(bar(s, x), (x == kPFull || x == kAEmpty) ? 4u : 1u);
         *abort_flag = 0;
+        ring_n[0] = ring_n[1] = 0;
         fence_mbar_init();
         prefetch_tensormap(&tmQ);
         prefetch_tensormap(&tmK);
@@ -392,29 +513,19 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // the first item with tiles at or after slot s's item m (m past the end: none)
-    auto seek = [&](int s, int& m, int& T) -> bool {
-        while (true) {
-            const PpItem it = pp_item(P, sh, item_x(s, m));
-            if (!it.valid) return false;
-            if (it.T > 0) {
-                T = it.T;
-                return true;
-            }
-            ++m;
-        }
-    };
-
     if (warp < 4) {
         regs_dec<kPpRegsLow>();
     }
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            // per slot three load streams (Q per item; K, V per tile; with
-            // additive terms a fourth, their blocks per tile): the stream's
-            // item m, tile u, loads issued, the item's tile count
-            int sm[2][NSTREAM], su[2][NSTREAM], sT[2][NSTREAM];
+            // per slot: items taken (qm), whether the end was reached; load
+            // streams 1.. (K, V per tile; with additive terms their blocks per
+            // tile) each walk the slot's items: item km, tile ku, loads issued
+            int qm[2] = {0, 0};
+            bool qend[2] = {false, false};
+            int64_t scur[2] = {0, 0};  // static order: the slot's next position
+            int km[2][NSTREAM], ku[2][NSTREAM];
             uint32_t cnt[2][NSTREAM];
             bool live[2][NSTREAM];
             // bytes of one tile's additive blocks (two 64-key chunks per term)
@@ -425,41 +536,79 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             for (int s = 0; s < 2; ++s)
 #pragma unroll
                 for (int k = 0; k < NSTREAM; ++k) {
-                    sm[s][k] = su[s][k] = 0;
+                    km[s][k] = ku[s][k] = 0;
                     cnt[s][k] = 0;
-                    sT[s][k] = 0;
-                    live[s][k] = seek(s, sm[s][k], sT[s][k]);
+                    live[s][k] = true;
                 }
+            // the next item with tiles for slot s, or -1: from the claim counter
+            // (items in order over all CTAs), else CTA c's static share
+            auto take = [&](int s) -> int64_t {
+                while (true) {
+                    int64_t x;
+                    if (P.claim) {
+                        x = (int64_t)atomicAdd(P.claim, 1ull);
+                    } else {
+                        x = (int64_t)blockIdx.x + (2 * scur[s] + s) * (int64_t)gridDim.x;
+                        ++scur[s];
+                    }
+                    if (x >= P.n_items) return -1;
+                    if (pp_item(P, sh, x).T > 0) return x;
+                }
+            };
             long long t_last = clock64();
             unsigned nap = 0;  // back-off when a pass finds nothing to load
             while (true) {
                 bool any = false, progress = false;
 #pragma unroll
                 for (int s = 0; s < 2; ++s) {
+                    // Q: take the slot's next item once its Q buffer is free
+                    if (!qend[s]) {
+                        any = true;
+                        if (qm[s] == 0 || mbar_test(bar(s, kQEmpty), (qm[s] - 1) & 1)) {
+                            const int64_t x = take(s);
+                            ring[s * 4 + (qm[s] & 3)] = x;
+                            const uint32_t fb = bar(s, kQFull);
+                            if (x < 0) {
+                                qend[s] = true;
+                                mbar_arrive(fb);  // the phase completes: consumers read the end
+                            } else {
+                                const PpItem it = pp_item(P, sh, x);
+                                const uint32_t dst = sQ0 + s * C::TILE_BYTES;
+                                mbar_expect_tx(fb, C::TILE_BYTES);
 #pragma unroll
-                    for (int k = 0; k < NSTREAM; ++k) {
+                                for (int c = 0; c < C::NCHUNK; ++c) {
+                                    if (it.perm)
+                                        tma_load_5d(dst + c * C::CHUNK_BYTES, &tmQp, fb, c * C::CHUNK_ELEMS, it.qb,
+                                                    it.pqb * 128, it.h, it.b);
+                                    else
+                                        tma_load_4d(dst + c * C::CHUNK_BYTES, &tmQ, fb, c * C::CHUNK_ELEMS, it.qb * 128,
+                                                    it.h, it.b);
+                                }
+                            }
+                            ++qm[s];
+                            __threadfence_block();
+                            ring_n[s] = qm[s];
+                            progress = true;
+                        }
+                    }
+#pragma unroll
+                    for (int k = 1; k < NSTREAM; ++k) {
                         if (!live[s][k]) continue;
                         any = true;
-                        const int eb = k == 0 ? kQEmpty : (k == 1 ? kKEmpty : (k == 2 ? kVEmpty : kAEmpty));
+                        if (km[s][k] >= qm[s]) continue;  // its next item is not taken yet
+                        const int64_t x = ring[s * 4 + (km[s][k] & 3)];
+                        if (x < 0) {
+                            live[s][k] = false;
+                            continue;
+                        }
+                        const int eb = k == 1 ? kKEmpty : (k == 2 ? kVEmpty : kAEmpty);
                         if (cnt[s][k] != 0 && !mbar_test(bar(s, eb), (cnt[s][k] - 1) & 1)) continue;
-                        const PpItem it = pp_item(P, sh, item_x(s, sm[s][k]));
-                        const uint32_t fb = bar(s, k == 0 ? kQFull : (k == 1 ? kKFull : (k == 2 ? kVFull : kAFull)));
-                        if (k == 0) {
-                            const uint32_t dst = sQ0 + s * C::TILE_BYTES;
-                            mbar_expect_tx(fb, C::TILE_BYTES);
-#pragma unroll
-                            for (int c = 0; c < C::NCHUNK; ++c) {
-                                if (it.perm)
-                                    tma_load_5d(dst + c * C::CHUNK_BYTES, &tmQp, fb, c * C::CHUNK_ELEMS, it.qb,
-                                                it.pqb * 128, it.h, it.b);
-                                else
-                                    tma_load_4d(dst + c * C::CHUNK_BYTES, &tmQ, fb, c * C::CHUNK_ELEMS, it.qb * 128,
-                                                it.h, it.b);
-                            }
-                        } else if (k < 3) {
+                        const PpItem it = pp_item(P, sh, x);
+                        const uint32_t fb = bar(s, k == 1 ? kKFull : (k == 2 ? kVFull : kAFull));
+                        const int kt = pp_tile(P, sh, it, ku[s][k]) & 0x7fffffff;
+                        if (k < 3) {
                             const uint32_t dst = (k == 1 ? sK0 : sV0) + s * C::TILE_BYTES;
                             mbar_expect_tx(fb, C::TILE_BYTES);
-                            const int kt = pp_tile(P, sh, it, su[s][k]) & 0x7fffffff;
                             const CUtensorMap* map = it.perm ? (k == 1 ? &tmKp : &tmVp) : (k == 1 ? &tmK : &tmV);
 #pragma unroll
                             for (int c = 0; c < C::NCHUNK; ++c) {
@@ -475,7 +624,6 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                             // OFF_A + (2 s + a) A_BYTES, chunk c of a_rows[a] rows at
                             // c * a_rows[a] * 128 bytes
                             mbar_expect_tx(fb, a_bytes);
-                            const int kt = pp_tile(P, sh, it, su[s][k]) & 0x7fffffff;
 #pragma unroll
                             for (int a = 0; a < 2; ++a) {
                                 if (!P.extra[a]) continue;
@@ -489,10 +637,9 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                             }
                         }
                         ++cnt[s][k];
-                        if (k == 0 || ++su[s][k] == sT[s][k]) {
-                            su[s][k] = 0;
-                            ++sm[s][k];
-                            live[s][k] = seek(s, sm[s][k], sT[s][k]);
+                        if (++ku[s][k] == it.T) {
+                            ku[s][k] = 0;
+                            ++km[s][k];
                         }
                         progress = true;
                     }
@@ -513,12 +660,14 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                     }
                 }
             }
-            // no load may outlive the CTA: wait (bounded) for the last of each buffer
+            // no load may outlive the CTA: wait (bounded) for the last of each
+            // buffer (a slot that reached its end had its last Q consumed)
 #pragma unroll
             for (int s = 0; s < 2; ++s) {
+                if (!qend[s] && qm[s]) mbar_wait_bounded(bar(s, kQFull), (qm[s] - 1) & 1, kPpDrainCycles);
 #pragma unroll
-                for (int k = 0; k < NSTREAM; ++k) {
-                    const int full = k == 0 ? kQFull : (k == 1 ? kKFull : (k == 2 ? kVFull : kAFull));
+                for (int k = 1; k < NSTREAM; ++k) {
+                    const int full = k == 1 ? kKFull : (k == 2 ? kVFull : kAFull);
                     if (cnt[s][k]) mbar_wait_bounded(bar(s, full), (cnt[s][k] - 1) & 1, kPpDrainCycles);
                 }
             }
@@ -531,7 +680,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
         const int t = quarter * 32 + lane;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const uint32_t tS = tmem + (uint32_t)(s * 256) + lane_base, tO = tS + 128;
-        const uint64_t c2 = pack2(P.qk_scale_log2, P.qk_scale_log2);
+        const uint32_t stg = smem_u32(smem + C::OFF_STG) + (uint32_t)(warp - 4) * 4096u;
         const bool leader = t == 0;  // issues this slot's MMAs
         // MMAs of this slot (leader only). S(g) = Q K(g)^T into S's columns,
         // then O (+)= P(g) V(g) with P read from the first 64 of them; since P
@@ -544,7 +693,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
         // their byte offset / 16 to the start-address field (bits 0-13)
         const uint64_t dQK0 = smem_desc(sQ0, 16, C::SBO, C::LAYOUT);
         const uint64_t dV0 = smem_desc(sV0, C::CHUNK_BYTES, C::SBO, C::LAYOUT);
-        // S(gs) once Q (the slot's active item number qi, on its first tile) and K(gs) are in
+        // S(gs) once Q (the slot's item number qi, on its first tile) and K(gs) are in
         auto issue_s = [&](uint32_t gs, uint32_t qi, bool first, bool last) -> bool {
             if (first && !pp_wait(bar(s, kQFull), qi & 1, abort_flag, P.wait_cycles)) return false;
             if (!pp_wait(bar(s, kKFull), gs & 1, abort_flag, P.wait_cycles)) return false;
@@ -561,27 +710,53 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             if (last) mma_commit(bar(s, kQEmpty));
             return true;
         };
-        // O (+)= P(gp) V(gp) once V(gp) is in (every row's P is written)
-        auto issue_pv = [&](uint32_t gp, bool first) -> bool {
+        // O (+)= P(gp) V(gp) once V(gp) is in (every row's P is written); zero
+        // sets O to the product (the item's first tile, O not started from a
+        // published state)
+        auto issue_pv = [&](uint32_t gp, bool zero) -> bool {
             if (!pp_wait(bar(s, kVFull), gp & 1, abort_flag, P.wait_cycles)) return false;
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {  // 16 keys per step
                 const uint64_t db = dV0 + (uint64_t)((s * C::TILE_BYTES + ks * 16 * C::ROW_BYTES) >> 4);
-                mma_bf16_ts(tOm, tSm + (uint32_t)(ks * 8), db, idO, (!first || ks > 0) ? 1u : 0u);
+                mma_bf16_ts(tOm, tSm + (uint32_t)(ks * 8), db, idO, (!zero || ks > 0) ? 1u : 0u);
             }
             mma_commit(bar(s, kODone));
             mma_commit(bar(s, kVEmpty));
             return true;
         };
-        uint32_t g = 0, qitems = 0;  // tiles and active items of this slot so far
-        bool alive = true;
-        int m = 0, T0 = 0;
-        bool have = seek(s, m, T0);
-        if (leader && have && !issue_s(0, 0, true, T0 == 1)) *abort_flag = 1;
-        __syncwarp();
-        for (; alive && have; ++m) {
-            const PpItem it = pp_item(P, sh, item_x(s, m));  // seek found it: valid, with tiles
+        uint32_t g = 0;         // tiles of this slot so far
+        bool s_ready = false;   // leader: S of the current item's first tile is issued
+        for (uint32_t m = 0;; ++m) {
+            // the slot's m-th item, once the producer has taken it
+            bool okq = true;
+            if (ring_n[s] <= (int)m) {
+                const long long t0 = clock64();
+                while (ring_n[s] <= (int)m) {
+                    if (*abort_flag || clock64() - t0 > P.wait_cycles) {
+                        *abort_flag = 1;
+                        okq = false;
+                        break;
+                    }
+                    __nanosleep(32);
+                }
+            }
+            if (!__all_sync(0xffffffffu, okq)) break;
+            __threadfence_block();
+            const int64_t x = ring[s * 4 + (m & 3)];
+            if (x < 0) break;
+            const PpItem it = pp_item(P, sh, x);
+            bsg::Item bi;
+            bi.bh = it.bh;
+            bi.perm = it.perm;
+            bi.qb = it.qb;
+            bi.pqb = it.pqb;
+            bi.chunk = it.chunk;
+            bi.u0 = it.u0;
+            bi.T = it.T;
+            if (leader && !s_ready && !issue_s(g, m, true, it.T == 1)) *abort_flag = 1;
+            s_ready = false;
+            __syncwarp();
             int i;
             bool row_ok;
             int rlo = 0, rhi = 0;
@@ -594,19 +769,50 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                     rhi = v.y;
                 }
             } else {
-                bsg::Item bi;
-                bi.bh = it.bh;
-                bi.perm = it.perm;
-                bi.qb = it.qb;
-                bi.pqb = it.pqb;
-                bi.chunk = it.chunk;
-                bi.u0 = it.u0;
-                bi.T = it.T;
                 i = bsg::row_of(sh, bi, t);
                 row_ok = i >= 0;
             }
             float m_ref = -INFINITY, l = 0.f;
+            // a regular block whose rows also have a permuted part starts from
+            // that part's published state (m, l and O), loaded while S(first
+            // tile) is computed; rows without one start from O = 0
+            const bool init_o = C::STAGE && P.mode == 1 && bsg::starts_from_perm(sh, bi);
+            if (C::STAGE && init_o) {
+                const bool pr = row_ok && bsg::has_perm(sh, i);
+                bool use = pr;
+                const int64_t prow = (int64_t)it.bh * P.n + (pr ? i : 0);
+                if (pr) {
+                    // the permuted block (residue i mod 128, positions block
+                    // (i / 128) / 128) is complete once all four of its warps arrived
+                    const unsigned* f = P.pflag + ((int64_t)it.bh * sh.npqb + ((i >> 7) >> 7)) * 128 + (i & 127);
+                    if (ld_acquire_u32(f) < 4u) {
+                        const long long t0 = clock64();
+                        while (ld_acquire_u32(f) < 4u) {
+                            if (clock64() - t0 > P.wait_cycles || *abort_flag) {
+                                atomicOr(P.err, kErrTimeout);
+                                use = false;
+                                break;
+                            }
+                            __nanosleep(128);
+                        }
+                    }
+                }
+                __syncwarp();
+                if (use) {
+                    m_ref = __ldcg(P.pml + prow * 2);
+                    l = __ldcg(P.pml + prow * 2 + 1);
+                }
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t w[32];
+                    // read exactly once: the lines are dropped from L2 unwritten
+                    rows_load<true>(stg, lane, w, use ? reinterpret_cast<uint64_t>(P.pacc + prow * D + 32 * c) : 0ull);
+                    tmem_st32(tO + 32 * c, w);
+                }
+                tmem_wait_st();
+            }
             const int klim = pp_key_limit(P, it.b);
+            bool alive = true;
             for (int u = 0; u < it.T; ++u, ++g) {
                 const int info = pp_tile(P, sh, it, u);
                 const int kt = info & 0x7fffffff;
@@ -617,14 +823,6 @@ __global__ void __launch_bounds__(kPpThreads, 1)
 #pragma unroll
                         for (int q = 0; q < 4; ++q) w[q] = bsg::run_word(rlo, rhi, kt * 128 + 32 * q);
                     } else {
-                        bsg::Item bi;
-                        bi.bh = it.bh;
-                        bi.perm = it.perm;
-                        bi.qb = it.qb;
-                        bi.pqb = it.pqb;
-                        bi.chunk = it.chunk;
-                        bi.u0 = it.u0;
-                        bi.T = it.T;
                         bsg::row_bits(sh, bi, kt, t, w);
                     }
                 }
@@ -775,14 +973,17 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(s, kAEmpty));
                 }
-                if (u > 0 && __any_sync(0xffffffffu, alpha_t != 1.f)) {
-                    // bring O (P V of the item's tiles so far, complete) to the new reference
-                    const bool ok2 = pp_wait(bar(s, kODone), (g - 1) & 1, abort_flag, P.wait_cycles);
-                    if (!__all_sync(0xffffffffu, ok2)) {
-                        alive = false;
-                        break;
+                if ((u > 0 || init_o) && __any_sync(0xffffffffu, alpha_t != 1.f)) {
+                    // bring O (P V of the item's tiles so far, complete, or the
+                    // published state it started from) to the new reference
+                    if (u > 0) {
+                        const bool ok2 = pp_wait(bar(s, kODone), (g - 1) & 1, abort_flag, P.wait_cycles);
+                        if (!__all_sync(0xffffffffu, ok2)) {
+                            alive = false;
+                            break;
+                        }
+                        tc_fence_after();
                     }
-                    tc_fence_after();
 #pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t ro[32];
@@ -798,21 +999,23 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(s, kPFull));
                 if (leader) {
-                    // every row's P(g) is in TMEM: P V(g); then, once it has consumed
-                    // P, the next S -- this item's next tile or the next item's first
-                    bool okl = pp_wait(bar(s, kPFull), g & 1, abort_flag, P.wait_cycles) && issue_pv(g, u == 0);
+                    // every row's P(g) is in TMEM: P V(g); then, once it has
+                    // consumed P, this item's next S -- or, after its last tile,
+                    // the next item's first S when its Q and K are already in
+                    // (else at that item's start)
+                    bool okl = pp_wait(bar(s, kPFull), g & 1, abort_flag, P.wait_cycles) &&
+                               issue_pv(g, u == 0 && !init_o) &&
+                               pp_wait(bar(s, kODone), g & 1, abort_flag, P.wait_cycles);
                     if (okl) {
-                        int mn = m, Tn = it.T;
-                        bool nxt = u + 1 < it.T, first = false;
-                        if (!nxt) {
-                            mn = m + 1;
-                            nxt = seek(s, mn, Tn);
-                            first = true;
+                        if (u + 1 < it.T) {
+                            okl = issue_s(g + 1, m, false, u + 2 == it.T);
+                        } else if (mbar_test(bar(s, kQFull), (m + 1) & 1)) {
+                            const int64_t xn = ring[s * 4 + ((m + 1) & 3)];
+                            if (xn >= 0 && mbar_test(bar(s, kKFull), (g + 1) & 1)) {
+                                okl = issue_s(g + 1, m + 1, true, pp_item(P, sh, xn).T == 1);
+                                s_ready = true;
+                            }
                         }
-                        const int un = first ? 0 : u + 1;
-                        if (nxt)
-                            okl = pp_wait(bar(s, kODone), g & 1, abort_flag, P.wait_cycles) &&
-                                  issue_s(g + 1, qitems + (first ? 1 : 0), first, un == Tn - 1);
                     }
                     if (!okl) *abort_flag = 1;
                 }
@@ -823,22 +1026,8 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             const bool ok = pp_wait(bar(s, kODone), (g - 1) & 1, abort_flag, P.wait_cycles);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-            float o[D];
-            {  // O loaded in place as fp32, all loads issued before one wait
-                float(&oc)[D / 32][32] = *reinterpret_cast<float(*)[D / 32][32]>(&o);
-#pragma unroll
-                for (int c = 0; c < D / 32; ++c) tmem_ld32f(tO + 32 * c, oc[c]);
-                tmem_wait_ld_depf(oc[0]);
-#pragma unroll
-                for (int c = 1; c < D / 32; ++c) reg_fence32f(oc[c]);
-            }
-            pp_finish<D>(P, sh, it, quarter, t, i, row_ok, m_ref, l, o);
+            pp_finish<D, C::STAGE>(P, sh, it, quarter, t, i, row_ok, m_ref, l, tO, stg);
             __syncwarp();
-            ++qitems;
-            int Tn = 0;
-            ++m;
-            have = seek(s, m, Tn);
-            --m;  // the loop's ++m moves to it
         }
         if (leader) {  // every MMA this thread issued is complete before TMEM is released
             mma_commit(bar(s, kDrainS));

@@ -966,13 +966,17 @@ int fwd_closed(const FwdParams& p, int d, spattn_mask m, cudaStream_t s, cudaMem
     const bsg::Shape sh = bsg::shape(p.n, m->bsg_block, m->bsg_stride, m->bsg_ng, kChunkTiles);
     const int64_t bh = (int64_t)p.B * p.H, rows = bh * p.n;
     const bool chunks = sh.nch > 1, partner = sh.G > 0;
+    // counts: claim counter (8 bytes), chunk counts [bh][4], permuted-block
+    // arrival counts [bh][npqb][128]
+    const size_t n_pflag = partner ? (size_t)bh * sh.npqb * 128 : 0,
+                 cnt_bytes = 8 + (size_t)bh * 4 * 4 + n_pflag * 4;
     Carve c;
     const int k_cws = c.add(chunks ? (size_t)bh * sh.nch * (d + 2) * kTileM * 4 : 0),
               k_pml = c.add(partner ? (size_t)rows * 2 * 4 : 0), k_pacc = c.add(partner ? (size_t)rows * d * 4 : 0),
-              k_cnt = c.add((size_t)bh * 4 * 4 + (partner ? (size_t)rows * 4 : 0));
+              k_cnt = c.add(cnt_bytes);
     void* ws = nullptr;
     CUDA_TRY(lib_malloc_async(&ws, c.total, pool, s), "tile-kernel workspace");
-    cudaError_t e = cudaMemsetAsync(c.at<uint8_t>(ws, k_cnt), 0, (size_t)bh * 4 * 4 + (partner ? (size_t)rows * 4 : 0), s);
+    cudaError_t e = cudaMemsetAsync(c.at<uint8_t>(ws, k_cnt), 0, cnt_bytes, s);
     if (e == cudaSuccess) {
         PpParams pp;
         memset(&pp, 0, sizeof pp);
@@ -983,9 +987,11 @@ int fwd_closed(const FwdParams& p, int d, spattn_mask m, cudaStream_t s, cudaMem
         pp.blk = m->bsg_block;
         pp.S = m->bsg_stride;
         pp.ng = m->bsg_ng;
+        uint8_t* cnt = c.at<uint8_t>(ws, k_cnt);
+        pp.claim = reinterpret_cast<unsigned long long*>(cnt);
+        pp.ccnt = reinterpret_cast<unsigned*>(cnt + 8);
+        pp.pflag = partner ? reinterpret_cast<unsigned*>(cnt + 8) + bh * 4 : nullptr;
         pp.cws = chunks ? c.at<float>(ws, k_cws) : nullptr;
-        pp.ccnt = c.at<unsigned>(ws, k_cnt);
-        pp.pcnt = partner ? c.at<unsigned>(ws, k_cnt) + bh * 4 : nullptr;
         pp.pml = partner ? c.at<float>(ws, k_pml) : nullptr;
         pp.pacc = partner ? c.at<float>(ws, k_pacc) : nullptr;
         const TcOperand oq{p.q, p.q_sn, p.q_sh, p.q_sb}, ok{p.k, p.k_sn, p.k_sh, p.k_sb},

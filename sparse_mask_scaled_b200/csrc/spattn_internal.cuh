@@ -174,15 +174,18 @@ struct PpParams {
     const float* ws_ml;
     const float* ws_acc;
     // mode 1: pattern parameters (bsg_plan.cuh), chunk partial states
-    // [B*H][nch][d + 2][128] with counts [B*H][4] (zero before the launch),
-    // partner states [B*H*n][2] (m, l) and [B*H*n][d] (O) with counts
-    // [B*H*n] (zero before the launch)
+    // [B*H][nch][d + 2][128] with counts [B*H][4], the permuted parts' states
+    // [B*H*n][2] (m, l) and [B*H*n][d] (O) with per permuted block arrival
+    // counts [B*H][npqb][128] (counts zero before the launch)
     int blk, S, ng, chunk_tiles;
     float* cws;
     unsigned* ccnt;
     float* pml;
     float* pacc;
-    unsigned* pcnt;
+    unsigned* pflag;
+    // nullable: items are taken from this counter (zero before the launch) in
+    // order; else CTA c takes items c, c + grid, ... (slots alternating)
+    unsigned long long* claim;
     void* out;
     int64_t o_sb, o_sh, o_sn;
     float* lse;  // nullable

@@ -6,7 +6,8 @@
 // to stdout, as raw bytes: the n x n count of how many times each entry (i, j)
 // is computed (uint8), the per-row "has entries in a permuted block" flag
 // computed from the bits (uint8 [n]) and the one bsg::has_perm reports (uint8
-// [n]). Exit status 2 when the parameters are outside the closed form.
+// [n]). Exit status 2 when the parameters are outside the closed form, 6 when
+// a regular item of a head comes before one of that head's permuted items.
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
@@ -25,9 +26,12 @@ int main(int argc, char** argv) {
     std::vector<uint8_t> cnt((size_t)n * n, 0), perm_rows(n, 0), has(n, 0);
     // every item of three (b, h) heads (the order interleaves heads), keeping head 1's
     const int heads = 3;
+    std::vector<int64_t> last_perm(heads, -1), first_reg(heads, -1);
     for (int64_t x = 0; x < (int64_t)heads * s.items_per_head; ++x) {
         const Item it = item(s, x, heads);
         if (it.bh < 0 || it.bh >= heads) return 3;
+        if (it.perm) last_perm[it.bh] = x;
+        else if (first_reg[it.bh] < 0) first_reg[it.bh] = x;
         if (it.bh != 1) continue;
         for (int u = 0; u < it.T; ++u) {
             const int kt = key_tile(s, it, u);
@@ -47,6 +51,8 @@ int main(int argc, char** argv) {
             }
         }
     }
+    for (int h = 0; h < heads; ++h)
+        if (last_perm[h] >= 0 && first_reg[h] >= 0 && last_perm[h] > first_reg[h]) return 6;
     for (int i = 0; i < n; ++i) has[i] = has_perm(s, i) ? 1 : 0;
     fwrite(cnt.data(), 1, cnt.size(), stdout);
     fwrite(perm_rows.data(), 1, n, stdout);
