@@ -109,15 +109,17 @@ struct Item {
     int T;      // tiles of this item
 };
 
-// Item x of all bh_count * items_per_head, in groups: group 0 holds the
-// permuted blocks of (b, h) 0; group g >= 1 the regular blocks of (b, h) g - 1
-// (the chunks of query block 0 first, the items with the most tiles) and then
-// the permuted blocks of (b, h) g. Every regular block of a (b, h) comes after
-// all of its permuted blocks: rows met by both start their regular part from
-// the permuted part's published state, and items taken in this order never
-// wait for a later one.
+// How many (b, h) heads the permuted blocks run ahead of the regular ones.
+constexpr int kPermLead = 3;
+
+// Item x of all bh_count * items_per_head, in groups g = 0, 1, ...: the
+// permuted blocks of (b, h) g, then the regular blocks of (b, h) g - L (the
+// chunks of query block 0 first, the items with the most tiles), with
+// L = min(kPermLead, bh_count). Every regular block of a (b, h) thus comes L
+// groups after its permuted blocks: rows met by both start their regular part
+// from the permuted part's published state, which is then usually complete,
+// and items taken in this order never wait for a later one.
 BSG_HD Item item(const Shape& s, int64_t x, int bh_count) {
-    (void)bh_count;
     Item it;
     it.perm = 0;
     it.qb = 0;
@@ -125,20 +127,30 @@ BSG_HD Item item(const Shape& s, int64_t x, int bh_count) {
     it.chunk = 0;
     it.u0 = 0;
     const int nregular = s.n_lead + s.nreg;
+    const int L = bh_count < kPermLead ? bh_count : kPermLead;
+    const int64_t lead = (int64_t)L * s.nperm;                               // groups 0 .. L-1
+    const int64_t middle = (int64_t)(bh_count - L) * s.items_per_head;     // groups L .. bh_count-1
     int j;
-    if (x < s.nperm) {
-        it.bh = 0;
+    if (x < lead) {
+        it.bh = (int)(x / s.nperm);
         it.perm = 1;
-        j = (int)x;
-    } else {
-        const int64_t y = x - s.nperm;
-        it.bh = (int)(y / s.items_per_head);
-        j = (int)(y - (int64_t)it.bh * s.items_per_head);
-        if (j >= nregular) {
+        j = (int)(x - (int64_t)it.bh * s.nperm);
+    } else if (x - lead < middle) {
+        const int64_t y = x - lead;
+        const int gi = (int)(y / s.items_per_head);
+        j = (int)(y - (int64_t)gi * s.items_per_head);
+        if (j < s.nperm) {
+            it.bh = L + gi;
             it.perm = 1;
-            j -= nregular;
-            ++it.bh;
+        } else {
+            it.bh = gi;
+            j -= s.nperm;
         }
+    } else {
+        const int64_t z = x - lead - middle;
+        const int hi = (int)(z / nregular);
+        it.bh = bh_count - L + hi;
+        j = (int)(z - (int64_t)hi * nregular);
     }
     if (it.perm) {
         it.qb = j / s.npqb;

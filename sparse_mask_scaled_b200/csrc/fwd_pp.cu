@@ -2,9 +2,10 @@
 // (tcgen05 MMAs with TMEM accumulators, TMA tile loads without multicast,
 // sm_100a).
 //
-// One CTA per SM walks a list of work items (a 128-row query block and its
-// key tiles). Three warpgroups:
-//   warp 0      TMA producer (one thread): Q tile per item, K and V per tile
+// One CTA per SM works through items (a 128-row query block and its key
+// tiles). Three warpgroups:
+//   warp 0      TMA producer (one thread): takes each slot's next item, then
+//               loads its Q tile, and K and V per tile
 //   warps 1-3   idle (they complete the first warpgroup, which gives its
 //               registers to the other two: 72 per thread against 216)
 //   warps 4-7   softmax group of slot 0 (one query row per thread)
@@ -16,10 +17,18 @@
 // slot's MMAs: once all four warps have written P(g), O (+)= P(g) V(g), then,
 // when that has consumed P, S(g + 1) = Q K(g + 1)^T, which its warps are
 // waiting for. While one slot's group turns S into P, the tensor cores work on
-// the other slot, so the two dependency chains overlap. The producer polls both
-// slots with non-blocking barrier tests, loads whichever buffer is free, and
-// sleeps briefly when nothing is (it shares a sub-partition with two softmax
-// warps); every wait is bounded.
+// the other slot, so the two dependency chains overlap. After an item's last
+// tile the first thread issues the next item's first S at once when its Q and
+// K are already in, else at that item's start. The producer polls both slots
+// with non-blocking barrier tests, loads whichever buffer is free, and sleeps
+// briefly when nothing is (it shares a sub-partition with two softmax warps);
+// it hands each slot its items through a small ring in shared memory. Items
+// come either from a counter shared by all CTAs, taken in order as slots free
+// up, or from a fixed share per CTA. Every wait is bounded.
+//
+// The end of an item goes through the warps' staging buffers in shared
+// memory, so that its global writes (and the reads of published states)
+// cover whole 128-byte lines.
 //
 // Per tile, each thread streams its row of S 32 keys at a time (the next
 // chunk's TMEM load in flight): scale, entries the mask does not list to -inf,
@@ -40,13 +49,18 @@
 //   interval masks (sliding, variable window, dense): every (b, h, query
 //     block) with tiles; per-row bits from the row's run; rows that also have
 //     gathered entries merge the gather kernel's partial state;
-//   block + strided + global masks in closed form (bsg_plan.cuh): regular
-//     query blocks (block 0 of a mask with global rows split into chunks,
-//     merged by the warp that completes a per-(b, h, warp) count) and
-//     residue-permuted blocks read through five-dimensional tensor maps; a row
-//     with entries in both meets its partner per row: the first to finish
-//     publishes its fp32 state (m, l, O), the second merges it and writes the
-//     row, and discards the published lines from L2.
+//   block + strided + global masks in closed form (bsg_plan.cuh), taken from
+//     the counter: residue-permuted blocks (read through five-dimensional
+//     tensor maps) publish the fp32 state (m, l, O) of their rows and count
+//     their four warps in; regular query blocks (block 0 of a mask with
+//     global rows split into chunks, merged by the warp that completes a
+//     per-(b, h, warp) count) start each row from the published state of its
+//     permuted part -- O loaded into TMEM, m and l into registers -- so that
+//     the rest of the row accumulates on top of it (the running-max /
+//     running-sum combination of two partial states of the streaming-dataflow
+//     SDPA paper, done inside the accumulator). The order of the items puts a
+//     head's permuted blocks well ahead of its regular ones, and a block only
+//     ever waits for earlier-taken ones.
 #include "spattn_internal.cuh"
 #include "sm100_ptx.cuh"
 #include "bsg_plan.cuh"
@@ -203,10 +217,6 @@ __device__ __forceinline__ void regs_inc() {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
 }
 
-__device__ __forceinline__ void discard_l2_line(const void* p) {
-    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
-}
-
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -248,39 +258,50 @@ __device__ __forceinline__ void rows_store(uint32_t stg, int lane, const uint32_
     __syncwarp();
 }
 
-// 128-byte rows from global memory (read at L2, written by another CTA) into
-// registers, the reverse of rows_store; with DISCARD the lines read are
-// dropped from L2 afterwards, unwritten.
-template <bool DISCARD>
-__device__ __forceinline__ void rows_load(uint32_t stg, int lane, uint32_t (&w)[32], uint64_t src) {
+// The D fp32 values of each of the warp's 32 rows (row address src per lane,
+// 0: zeros) from global memory (read at L2, written by another CTA) into the
+// TMEM columns tO .. tO + D - 1 of the lane's row. The warp's line loads of
+// two 32-column chunks are in flight together (D / 64 round trips to L2);
+// each chunk then reaches its row's lane through the staging buffer. (The
+// lines are read once, but dropping them from L2 unwritten corrupted reads
+// of neighbouring lines still in flight, so they are left to age out.)
+template <int D>
+__device__ __forceinline__ void rows_to_tmem(uint32_t stg, int lane, uint64_t src, uint32_t tO) {
+    constexpr int CB = D >= 64 ? 2 : 1;  // chunks whose loads are in flight together
     const int u = lane & 7;
+    uint64_t p[8];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {  // two batches of four lines in flight
-        uint4 v[4];
-        uint64_t p[4];
+    for (int k = 0; k < 8; ++k) p[k] = __shfl_sync(0xffffffffu, src, 4 * k + (lane >> 3));
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int r = 16 * h + 4 * k + (lane >> 3);
-            p[k] = __shfl_sync(0xffffffffu, src, r);
-            v[k] = p[k] ? __ldcg(reinterpret_cast<const uint4*>(p[k] + u * 16)) : make_uint4(0u, 0u, 0u, 0u);
-        }
+    for (int c0 = 0; c0 < D / 32; c0 += CB) {
+        uint4 v[CB][8];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int r = 16 * h + 4 * k + (lane >> 3);
-            st_shared_v4(stg + r * 128 + ((u ^ (r & 7)) << 4), v[k]);
-            if (DISCARD && p[k] && u == 0) discard_l2_line(reinterpret_cast<const void*>(p[k]));
+        for (int c = 0; c < CB; ++c)
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                v[c][k] = p[k] ? __ldcg(reinterpret_cast<const uint4*>(p[k] + (c0 + c) * 128 + u * 16))
+                               : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int c = 0; c < CB; ++c) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int r = 4 * k + (lane >> 3);
+                st_shared_v4(stg + r * 128 + ((u ^ (r & 7)) << 4), v[c][k]);
+            }
+            __syncwarp();
+            uint32_t w[32];
+#pragma unroll
+            for (int uu = 0; uu < 8; ++uu) {
+                const uint4 x = ld_shared_v4(stg + lane * 128 + ((uu ^ (lane & 7)) << 4));
+                w[4 * uu] = x.x;
+                w[4 * uu + 1] = x.y;
+                w[4 * uu + 2] = x.z;
+                w[4 * uu + 3] = x.w;
+            }
+            __syncwarp();
+            tmem_st32(tO + 32 * (c0 + c), w);
         }
     }
-    __syncwarp();
-#pragma unroll
-    for (int uu = 0; uu < 8; ++uu) {
-        const uint4 x = ld_shared_v4(stg + lane * 128 + ((uu ^ (lane & 7)) << 4));
-        w[4 * uu] = x.x;
-        w[4 * uu + 1] = x.y;
-        w[4 * uu + 2] = x.z;
-        w[4 * uu + 3] = x.w;
-    }
-    __syncwarp();
 }
 
 // 32 columns of this warp's rows of O (fp32, not yet divided by L) from TMEM.
@@ -441,10 +462,14 @@ __device__ __forceinline__ void pp_finish(const PpParams& P, const bsg::Shape& s
                     *reinterpret_cast<float4*>(P.pacc + prow * D + 32 * c + z) = make_float4(x[z], x[z + 1], x[z + 2], x[z + 3]);
             }
         }
-        // every lane's stores (lanes write other rows' lines) before the count
+        // every lane's stores (lanes write other rows' lines) are ordered
+        // before the barrier, and the barrier before lane 0's fence and count
         __threadfence();
         __syncwarp();
-        if (lane == 0) atomicAdd(P.pflag + (bh * sh.npqb + it.pqb) * 128 + it.qb, 1u);
+        if (lane == 0) {
+            __threadfence();
+            atomicAdd(P.pflag + (bh * sh.npqb + it.pqb) * 128 + it.qb, 1u);
+        }
         return;
     }
     // a regular block's rows: the output (their permuted part, if any, is in O already)
@@ -797,18 +822,15 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                         }
                     }
                 }
+                // each row's count is acquired by its own lane; the barrier and
+                // a fence put every lane's loads (lanes load other rows) after them
                 __syncwarp();
+                __threadfence();
                 if (use) {
                     m_ref = __ldcg(P.pml + prow * 2);
                     l = __ldcg(P.pml + prow * 2 + 1);
                 }
-#pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t w[32];
-                    // read exactly once: the lines are dropped from L2 unwritten
-                    rows_load<true>(stg, lane, w, use ? reinterpret_cast<uint64_t>(P.pacc + prow * D + 32 * c) : 0ull);
-                    tmem_st32(tO + 32 * c, w);
-                }
+                rows_to_tmem<D>(stg, lane, use ? reinterpret_cast<uint64_t>(P.pacc + prow * D) : 0ull, tO);
                 tmem_wait_st();
             }
             const int klim = pp_key_limit(P, it.b);

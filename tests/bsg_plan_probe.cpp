@@ -1,7 +1,7 @@
 // Test driver for the closed-form block + strided + global tile plan
 // (sparse_mask_scaled_b200/csrc/bsg_plan.cuh), built for the host by
 // tests/test_bsg_plan_cpu.py. For the parameters on the command line it walks
-// the work items of three (b, h) heads, keeps those of head 1, and for every
+// the work items of five (b, h) heads, keeps those of head 1, and for every
 // tile and every row's bits writes
 // to stdout, as raw bytes: the n x n count of how many times each entry (i, j)
 // is computed (uint8), the per-row "has entries in a permuted block" flag
@@ -24,8 +24,8 @@ int main(int argc, char** argv) {
     if (!supported(n, block, S, ng)) return 2;
     const Shape s = shape(n, block, S, ng, chunk);
     std::vector<uint8_t> cnt((size_t)n * n, 0), perm_rows(n, 0), has(n, 0);
-    // every item of three (b, h) heads (the order interleaves heads), keeping head 1's
-    const int heads = 3;
+    // every item of five (b, h) heads (the order interleaves heads), keeping head 1's
+    const int heads = 5;
     std::vector<int64_t> last_perm(heads, -1), first_reg(heads, -1);
     for (int64_t x = 0; x < (int64_t)heads * s.items_per_head; ++x) {
         const Item it = item(s, x, heads);
