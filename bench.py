@@ -372,14 +372,15 @@ def job_value(world: int, flop_per_step: float, ms_per_step: float) -> float:
 
 def kernel_name(wl, m_tiles):
     """The forward's dominant kernel for the workload (see the library's routing
-    in spattn_fwd_mask_kpad: interval masks and closed-form block + strided +
-    global masks take the persistent kernel, d = 128 with additive terms and
-    CSR masks the per-block tile kernels)."""
+    in spattn_fwd_mask_kpad: closed-form block + strided + global masks and
+    d = 128 interval masks without additive terms take the persistent kernel,
+    d <= 64 the four-CTAs-per-SM tile kernel, d = 128 with additive terms and
+    CSR masks the per-block tile kernel)."""
     if m_tiles == 0 or wl.dtype != workloads.BF16:
         return f"k_fwd_short<{'bf16' if wl.dtype == workloads.BF16 else 'f32'},{wl.d}>"
     extra = wl.add_mask is not None or wl.bias is not None
-    if wl.mask.kind in ("dense", "sliding", "varwin") and (wl.d <= 64 or not extra):
-        return f"k_fwd_pp<{wl.d},{int(extra)}>"
+    if wl.mask.kind in ("dense", "sliding", "varwin") and wl.d == 128 and not extra:
+        return f"k_fwd_pp<{wl.d},0>"
     if wl.mask.kind == "bsg" and not extra and wl.d in (64, 128):
         return f"k_fwd_pp<{wl.d},0>"
     if wl.d <= 64:

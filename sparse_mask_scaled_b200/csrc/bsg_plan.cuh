@@ -110,7 +110,7 @@ struct Item {
 };
 
 // How many (b, h) heads the permuted blocks run ahead of the regular ones.
-constexpr int kPermLead = 3;
+constexpr int kPermLead = 4;
 
 // Item x of all bh_count * items_per_head, in groups g = 0, 1, ...: the
 // permuted blocks of (b, h) g, then the regular blocks of (b, h) g - L (the
@@ -119,7 +119,9 @@ constexpr int kPermLead = 3;
 // groups after its permuted blocks: rows met by both start their regular part
 // from the permuted part's published state, which is then usually complete,
 // and items taken in this order never wait for a later one.
-BSG_HD Item item(const Shape& s, int64_t x, int bh_count) {
+BSG_HD Item item(const Shape& s, int64_t x64, int bh_count) {
+    // 32-bit arithmetic: callers keep bh_count * items_per_head below 2^31
+    const int x = (int)x64;
     Item it;
     it.perm = 0;
     it.qb = 0;
@@ -128,17 +130,17 @@ BSG_HD Item item(const Shape& s, int64_t x, int bh_count) {
     it.u0 = 0;
     const int nregular = s.n_lead + s.nreg;
     const int L = bh_count < kPermLead ? bh_count : kPermLead;
-    const int64_t lead = (int64_t)L * s.nperm;                               // groups 0 .. L-1
-    const int64_t middle = (int64_t)(bh_count - L) * s.items_per_head;     // groups L .. bh_count-1
+    const int lead = L * s.nperm;                               // groups 0 .. L-1
+    const int middle = (bh_count - L) * s.items_per_head;     // groups L .. bh_count-1
     int j;
     if (x < lead) {
-        it.bh = (int)(x / s.nperm);
+        it.bh = x / s.nperm;
         it.perm = 1;
-        j = (int)(x - (int64_t)it.bh * s.nperm);
+        j = x - it.bh * s.nperm;
     } else if (x - lead < middle) {
-        const int64_t y = x - lead;
-        const int gi = (int)(y / s.items_per_head);
-        j = (int)(y - (int64_t)gi * s.items_per_head);
+        const int y = x - lead;
+        const int gi = y / s.items_per_head;
+        j = y - gi * s.items_per_head;
         if (j < s.nperm) {
             it.bh = L + gi;
             it.perm = 1;
@@ -147,10 +149,10 @@ BSG_HD Item item(const Shape& s, int64_t x, int bh_count) {
             j -= s.nperm;
         }
     } else {
-        const int64_t z = x - lead - middle;
-        const int hi = (int)(z / nregular);
+        const int z = x - lead - middle;
+        const int hi = z / nregular;
         it.bh = bh_count - L + hi;
-        j = (int)(z - (int64_t)hi * nregular);
+        j = z - hi * nregular;
     }
     if (it.perm) {
         it.qb = j / s.npqb;

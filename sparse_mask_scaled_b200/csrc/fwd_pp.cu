@@ -4,37 +4,40 @@
 //
 // One CTA per SM works through items (a 128-row query block and its key
 // tiles). Three warpgroups:
-//   warp 0      TMA producer (one thread): takes each slot's next item, then
-//               loads its Q tile, and K and V per tile
-//   warps 1-3   idle (they complete the first warpgroup, which gives its
-//               registers to the other two: 72 per thread against 216)
+//   warp 0      K / V producer (one thread): the slots' K and V tiles by TMA
+//   warp 1      item taker and Q producer (one thread): takes each slot's next
+//               item, hands it over through a small ring in shared memory, and
+//               loads its Q tile
+//   warps 2, 3  MMA issuers of slots 0 and 1 (one thread each)
 //   warps 4-7   softmax group of slot 0 (one query row per thread)
 //   warps 8-11  softmax group of slot 1
-// The two slots hold one item each, with their own Q, K and V buffers in shared
-// memory and their own S and O in tensor memory (slot s: S in columns
-// [256 s, 256 s + 128), O in [256 s + 128, 256 s + 128 + d); P, in bf16,
-// overwrites the first 64 columns of S). Each group's first thread issues its
-// slot's MMAs: once all four warps have written P(g), O (+)= P(g) V(g), then,
-// when that has consumed P, S(g + 1) = Q K(g + 1)^T, which its warps are
-// waiting for. While one slot's group turns S into P, the tensor cores work on
-// the other slot, so the two dependency chains overlap. After an item's last
-// tile the first thread issues the next item's first S at once when its Q and
-// K are already in, else at that item's start. The producer polls both slots
-// with non-blocking barrier tests, loads whichever buffer is free, and sleeps
-// briefly when nothing is (it shares a sub-partition with two softmax warps);
-// it hands each slot its items through a small ring in shared memory. Items
-// come either from a counter shared by all CTAs, taken in order as slots free
-// up, or from a fixed share per CTA. Every wait is bounded.
+// (the first warpgroup gives registers to the other two: 88 per thread
+// against 208). The two slots hold one item each, with their own Q, K and V
+// buffers in shared memory and their own S and O in tensor memory: slot s has
+// S in two 64-key halves at columns [256 s, 256 s + 64) and [256 s + 64,
+// 256 s + 128) and O at [256 s + 128, 256 s + 128 + d); P, in bf16, overwrites
+// the first 32 columns of its half. For tile g the issuer computes S_h(g) =
+// Q K_h(g)^T for both halves; once the softmax group has turned half h into
+// P, O (+)= P_h V_h, and as soon as that product is complete, S_h(g + 1) into
+// the freed half -- so while the softmax group works on one half, the tensor
+// cores compute the other half's S (and the other slot's work): the softmax
+// group waits for S only when the tensor cores or the loads fall behind.
+// After an item's last tile the issuer starts the next item's S at once when
+// its Q and K are in, else at that item's start. The producers poll with
+// non-blocking barrier tests and sleep briefly when nothing is free (they
+// share sub-partitions with softmax warps). Items come either from a counter
+// shared by all CTAs, taken in order as slots free up, or from a fixed share
+// per CTA. Every wait is bounded.
 //
 // The end of an item goes through the warps' staging buffers in shared
 // memory, so that its global writes (and the reads of published states)
 // cover whole 128-byte lines.
 //
-// Per tile, each thread streams its row of S 32 keys at a time (the next
+// Per half, each thread streams its row of S 32 keys at a time (the next
 // chunk's TMEM load in flight): scale, entries the mask does not list to -inf,
 // p = 2^(x - m_ref) against a running reference max, row sum, bf16 P back to
 // TMEM. The reference only moves when a chunk's max exceeds it by more than
-// 2^8; then the P chunks already written, the sum and O are rescaled by
+// 2^8; then the half's P chunk already written, the sum and O are rescaled by
 // exp2(m_old - m_new) (the streaming-dataflow SDPA paper's delta rescaling,
 // applied lazily; exact in exact arithmetic). A warp skips the 32-key chunks in
 // which none of its rows has an entry (no TMEM load, no exp; P is zero there).
@@ -75,18 +78,19 @@ using namespace sm100;
 
 constexpr int kPpThreads = 384;
 // registers per thread after the split (launched with 168: 384 x 168 = 64,512
-// = 128 x 72 + 256 x 216; per SM sub-partition, warps w, w + 4, w + 8:
-// (72 + 2 x 216) x 32 <= 16,384)
-constexpr int kPpRegsLow = 72;
-constexpr int kPpRegsHigh = 216;
+// = 128 x 88 + 256 x 208; per SM sub-partition, warps w, w + 4, w + 8:
+// (88 + 2 x 208) x 32 <= 16,384)
+constexpr int kPpRegsLow = 88;
+constexpr int kPpRegsHigh = 208;
 constexpr uint32_t kPpTmemCols = 512;
 constexpr float kPpRescale = 8.0f;               // log2 units
 constexpr long long kPpDrainCycles = 200000000LL;  // ~0.1 s per drain wait
 
 // mbarriers of slot s: kBarsPerSlot * s + one of these
+// (S, P and their "free" barriers come per 64-key half: half h at + h)
 enum : int {
-    kQFull = 0, kQEmpty, kKFull, kKEmpty, kVFull, kVEmpty, kSFull, kPFull, kODone, kDrainS, kAFull, kAEmpty,
-    kBarsPerSlot
+    kQFull = 0, kQEmpty, kKFull, kKEmpty, kVFull, kVEmpty, kSFull, kSFullB, kPFull, kPFullB, kSFree, kSFreeB,
+    kODone, kDrainS, kAFull, kAEmpty, kBarsPerSlot
 };
 constexpr int kNumBars = 2 * kBarsPerSlot;
 
@@ -113,18 +117,18 @@ struct PpCfg {
     // per softmax warp a 4 KB buffer through which the epilogue's global
     // accesses go as whole lines (when it fits beside the tiles)
     static constexpr int STG_BYTES = 8 * 4096;
-    static constexpr bool STAGE = OFF_A + (EXTRA ? 4 * A_BYTES : 0) + STG_BYTES + kNumBars * 8 + 16 + 80 <= 227 * 1024;
+    static constexpr int RING_BYTES = 2 * 4 * 8 * 4 + 16;  // [slot][4] decoded items (8 words), then [slot] counts
+    static constexpr bool STAGE = OFF_A + (EXTRA ? 4 * A_BYTES : 0) + STG_BYTES + kNumBars * 8 + 16 + RING_BYTES <= 227 * 1024;
     static constexpr int OFF_STG = OFF_A + (EXTRA ? 4 * A_BYTES : 0);
     static constexpr int OFF_BAR = OFF_STG + (STAGE ? STG_BYTES : 0);
     static constexpr int OFF_INT = OFF_BAR + kNumBars * 8;  // TMEM base, abort flag
-    static constexpr int OFF_RING = OFF_INT + 16;            // [slot][4] items taken (int64), then [slot] counts
+    static constexpr int OFF_RING = OFF_INT + 16;
     // at least 116 KB, so that one CTA (which takes all 512 TMEM columns) runs per SM
-    static constexpr int SMEM_BYTES = OFF_RING + 80 > 116 * 1024 ? OFF_RING + 80 : 116 * 1024;
+    static constexpr int SMEM_BYTES = OFF_RING + RING_BYTES > 116 * 1024 ? OFF_RING + RING_BYTES : 116 * 1024;
 };
 
 // A work item as every role sees it.
 struct PpItem {
-    bool valid;
     int bh, b, h;
     int perm;           // closed form: permuted block
     int qb;             // query block (permuted: residue)
@@ -142,19 +146,18 @@ __device__ __forceinline__ int pp_key_limit(const PpParams& P, int b) {
     return L < 0 ? 0 : (L > P.n ? P.n : L);
 }
 
+// Item x (below n_items, which stays below 2^31).
 __device__ __forceinline__ PpItem pp_item(const PpParams& P, const bsg::Shape& sh, int64_t x) {
     PpItem it;
-    it.valid = x < P.n_items;
     it.perm = 0;
     it.pqb = 0;
     it.chunk = 0;
     it.u0 = 0;
     it.blk = 0;
     it.T = 0;
-    if (!it.valid) return it;
     if (P.mode == 0) {
-        it.bh = (int)(x / P.nqb);
-        it.qb = (int)(x - (int64_t)it.bh * P.nqb);
+        it.bh = (int)x / P.nqb;
+        it.qb = (int)x - it.bh * P.nqb;
         it.b = it.bh / P.H;
         it.h = it.bh - it.b * P.H;
         const int mk = P.num_masks == 1 ? 0 : it.b;
@@ -177,6 +180,34 @@ __device__ __forceinline__ PpItem pp_item(const PpParams& P, const bsg::Shape& s
         it.T = bi.T;
     }
     return it;
+}
+
+// Ring entries: the decoded item as eight words (bh, b, h, qb, pqb, chunk,
+// u0, T with the permuted flag in bit 30; word 7 = -1 after the last item).
+__device__ __forceinline__ void ring_put(volatile int* e, const PpItem& it) {
+    e[0] = it.bh;
+    e[1] = it.b;
+    e[2] = it.h;
+    e[3] = it.qb;
+    e[4] = it.pqb;
+    e[5] = it.chunk;
+    e[6] = it.u0;
+    e[7] = it.T | (it.perm << 30);
+}
+__device__ __forceinline__ bool ring_get(const PpParams& P, const volatile int* e, PpItem& it) {
+    const int w7 = e[7];
+    if (w7 < 0) return false;
+    it.bh = e[0];
+    it.b = e[1];
+    it.h = e[2];
+    it.qb = e[3];
+    it.pqb = e[4];
+    it.chunk = e[5];
+    it.u0 = e[6];
+    it.T = w7 & 0x3fffffff;
+    it.perm = (w7 >> 30) & 1;
+    it.blk = (int64_t)(P.num_masks == 1 ? 0 : it.b) * P.nqb + it.qb;
+    return true;
 }
 
 // Key tile u of the item: the key tile index, with kTileDenseBit set when
@@ -216,6 +247,9 @@ template <int R>
 __device__ __forceinline__ void regs_inc() {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
 }
+
+// Release / acquire fence at GPU scope (ordering, not sequential consistency).
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
     unsigned v;
@@ -260,9 +294,9 @@ __device__ __forceinline__ void rows_store(uint32_t stg, int lane, const uint32_
 
 // The D fp32 values of each of the warp's 32 rows (row address src per lane,
 // 0: zeros) from global memory (read at L2, written by another CTA) into the
-// TMEM columns tO .. tO + D - 1 of the lane's row. The warp's line loads of
-// two 32-column chunks are in flight together (D / 64 round trips to L2);
-// each chunk then reaches its row's lane through the staging buffer. (The
+// TMEM columns tO .. tO + D - 1 of the lane's row. All of the warp's line
+// loads are in flight together (one round trip to L2); each 32-column chunk
+// then reaches its row's lane through the staging buffer. (The
 // lines are read once, but dropping them from L2 unwritten corrupted reads
 // of neighbouring lines still in flight, so they are left to age out.)
 template <int D>
@@ -304,6 +338,20 @@ __device__ __forceinline__ void rows_to_tmem(uint32_t stg, int lane, uint64_t sr
     }
 }
 
+// Counts this warp in on a permuted block whose state it published: every
+// lane's stores (lanes wrote other rows' lines) are ordered before the
+// barrier, and the barrier before lane 0's fence and count.
+__device__ __forceinline__ void pp_release(unsigned*& pend) {
+    if (!pend) return;
+    fence_acq_rel_gpu();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) {
+        fence_acq_rel_gpu();
+        atomicAdd(pend, 1u);
+    }
+    pend = nullptr;
+}
+
 // 32 columns of this warp's rows of O (fp32, not yet divided by L) from TMEM.
 __device__ __forceinline__ void o_chunk(uint32_t tO, int c, float (&x)[32]) {
     tmem_ld32f(tO + 32 * c, x);
@@ -342,7 +390,7 @@ __device__ __forceinline__ void put_out_piece(uint64_t orow, int p, float inv, c
 // lines through the warp's staging buffer stg.
 template <int D, bool STAGE>
 __device__ __forceinline__ void pp_finish(const PpParams& P, const bsg::Shape& sh, const PpItem& it, int quarter, int t, int i,
-                          bool row_ok, float M, float L, uint32_t tO, uint32_t stg) {
+                          bool row_ok, float M, float L, uint32_t tO, uint32_t stg, unsigned*& pend) {
     const int lane = threadIdx.x & 31;
     const int64_t bh = it.bh;
     const uint64_t orow_any = reinterpret_cast<uint64_t>(reinterpret_cast<__nv_bfloat16*>(P.out) + (int64_t)it.b * P.o_sb +
@@ -462,14 +510,8 @@ __device__ __forceinline__ void pp_finish(const PpParams& P, const bsg::Shape& s
                     *reinterpret_cast<float4*>(P.pacc + prow * D + 32 * c + z) = make_float4(x[z], x[z + 1], x[z + 2], x[z + 3]);
             }
         }
-        // every lane's stores (lanes write other rows' lines) are ordered
-        // before the barrier, and the barrier before lane 0's fence and count
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) {
-            __threadfence();
-            atomicAdd(P.pflag + (bh * sh.npqb + it.pqb) * 128 + it.qb, 1u);
-        }
+        // counted in later (pp_release), once the stores have long completed
+        pend = P.pflag + (bh * sh.npqb + it.pqb) * 128 + it.qb;
         return;
     }
     // a regular block's rows: the output (their permuted part, if any, is in O already)
@@ -511,14 +553,15 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     // barrier for that item and before it raises the slot's count of entries
     // (the softmax warps go by the count: the producer may be two Q loads
     // ahead of them, where a barrier's phase parity would not tell)
-    volatile int64_t* ring = reinterpret_cast<volatile int64_t*>(smem + C::OFF_RING);
-    volatile int* ring_n = reinterpret_cast<volatile int*>(smem + C::OFF_RING + 64);
+    volatile int* ring = reinterpret_cast<volatile int*>(smem + C::OFF_RING);  // [slot][4][8]
+    volatile int* ring_n = reinterpret_cast<volatile int*>(smem + C::OFF_RING + 2 * 4 * 8 * 4);
+    auto entry = [&](int s, uint32_t m) { return ring + (s * 4 + (int)(m & 3u)) * 8; };
 
     if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kPpTmemCols);
     if (tid == 0) {
         for (int s = 0; s < 2; ++s)
             for (int x = 0; x < kBarsPerSlot; ++x)
-                mbar_init(bar(s, x), (x == kPFull || x == kAEmpty) ? 4u : 1u);
+                mbar_init(bar(s, x), (x == kPFull || x == kPFullB || x == kAEmpty) ? 4u : 1u);
         *abort_flag = 0;
         ring_n[0] = ring_n[1] = 0;
         fence_mbar_init();
@@ -541,15 +584,91 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     if (warp < 4) {
         regs_dec<kPpRegsLow>();
     }
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
+    if (warp == 1) {
+        // ------------------------------------------------------------ Q producer
         if (lane == 0) {
-            // per slot: items taken (qm), whether the end was reached; load
-            // streams 1.. (K, V per tile; with additive terms their blocks per
-            // tile) each walk the slot's items: item km, tile ku, loads issued
+            // per slot: items taken (qm), whether the end was reached
             int qm[2] = {0, 0};
             bool qend[2] = {false, false};
             int64_t scur[2] = {0, 0};  // static order: the slot's next position
+            // the next item with tiles for slot s, or -1: from the claim counter
+            // (items in order over all CTAs), else CTA c's static share
+            auto take = [&](int s, PpItem& it) -> bool {
+                while (true) {
+                    int64_t x;
+                    if (P.claim) {
+                        x = (int64_t)atomicAdd(P.claim, 1ull);
+                    } else {
+                        x = (int64_t)blockIdx.x + (2 * scur[s] + s) * (int64_t)gridDim.x;
+                        ++scur[s];
+                    }
+                    if (x >= P.n_items) return false;
+                    it = pp_item(P, sh, x);
+                    if (it.T > 0) return true;
+                }
+            };
+            long long t_last = clock64();
+            unsigned nap = 0;
+            while (true) {
+                bool any = false, progress = false;
+#pragma unroll
+                for (int s = 0; s < 2; ++s) {
+                    if (qend[s]) continue;
+                    any = true;
+                    // take the slot's next item once its Q buffer is free
+                    if (qm[s] != 0 && !mbar_test(bar(s, kQEmpty), (qm[s] - 1) & 1)) continue;
+                    PpItem it;
+                    const bool got = take(s, it);
+                    volatile int* e = entry(s, qm[s]);
+                    const uint32_t fb = bar(s, kQFull);
+                    if (!got) {
+                        e[7] = -1;
+                        qend[s] = true;
+                        mbar_arrive(fb);  // the phase completes: the end is read
+                    } else {
+                        ring_put(e, it);
+                        const uint32_t dst = sQ0 + s * C::TILE_BYTES;
+                        mbar_expect_tx(fb, C::TILE_BYTES);
+#pragma unroll
+                        for (int c = 0; c < C::NCHUNK; ++c) {
+                            if (it.perm)
+                                tma_load_5d(dst + c * C::CHUNK_BYTES, &tmQp, fb, c * C::CHUNK_ELEMS, it.qb, it.pqb * 128,
+                                            it.h, it.b);
+                            else
+                                tma_load_4d(dst + c * C::CHUNK_BYTES, &tmQ, fb, c * C::CHUNK_ELEMS, it.qb * 128, it.h,
+                                            it.b);
+                        }
+                    }
+                    ++qm[s];
+                    __threadfence_block();
+                    ring_n[s] = qm[s];
+                    progress = true;
+                }
+                if (!any) break;
+                if (progress) {
+                    t_last = clock64();
+                    nap = 0;
+                } else {
+                    nap = nap ? (nap < 256 ? 2 * nap : 256) : 32;
+                    __nanosleep(nap);
+                    if (*abort_flag) break;
+                    if (clock64() - t_last > P.wait_cycles) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                }
+            }
+            // no load may outlive the CTA (a slot that reached its end had its last Q consumed)
+#pragma unroll
+            for (int s = 0; s < 2; ++s)
+                if (!qend[s] && qm[s]) mbar_wait_bounded(bar(s, kQFull), (qm[s] - 1) & 1, kPpDrainCycles);
+        }
+    } else if (warp == 0) {
+        // ------------------------------------------------------------ K / V producer
+        if (lane == 0) {
+            // per slot, load streams 1.. (K, V per tile; with additive terms
+            // their blocks per tile) each walk the slot's items from the ring:
+            // item km, tile ku, loads issued
             int km[2][NSTREAM], ku[2][NSTREAM];
             uint32_t cnt[2][NSTREAM];
             bool live[2][NSTREAM];
@@ -563,72 +682,28 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                 for (int k = 0; k < NSTREAM; ++k) {
                     km[s][k] = ku[s][k] = 0;
                     cnt[s][k] = 0;
-                    live[s][k] = true;
+                    live[s][k] = k > 0;
                 }
-            // the next item with tiles for slot s, or -1: from the claim counter
-            // (items in order over all CTAs), else CTA c's static share
-            auto take = [&](int s) -> int64_t {
-                while (true) {
-                    int64_t x;
-                    if (P.claim) {
-                        x = (int64_t)atomicAdd(P.claim, 1ull);
-                    } else {
-                        x = (int64_t)blockIdx.x + (2 * scur[s] + s) * (int64_t)gridDim.x;
-                        ++scur[s];
-                    }
-                    if (x >= P.n_items) return -1;
-                    if (pp_item(P, sh, x).T > 0) return x;
-                }
-            };
             long long t_last = clock64();
             unsigned nap = 0;  // back-off when a pass finds nothing to load
             while (true) {
                 bool any = false, progress = false;
+                const int rn[2] = {ring_n[0], ring_n[1]};
+                __threadfence_block();  // the entries below the counts are written
 #pragma unroll
                 for (int s = 0; s < 2; ++s) {
-                    // Q: take the slot's next item once its Q buffer is free
-                    if (!qend[s]) {
-                        any = true;
-                        if (qm[s] == 0 || mbar_test(bar(s, kQEmpty), (qm[s] - 1) & 1)) {
-                            const int64_t x = take(s);
-                            ring[s * 4 + (qm[s] & 3)] = x;
-                            const uint32_t fb = bar(s, kQFull);
-                            if (x < 0) {
-                                qend[s] = true;
-                                mbar_arrive(fb);  // the phase completes: consumers read the end
-                            } else {
-                                const PpItem it = pp_item(P, sh, x);
-                                const uint32_t dst = sQ0 + s * C::TILE_BYTES;
-                                mbar_expect_tx(fb, C::TILE_BYTES);
-#pragma unroll
-                                for (int c = 0; c < C::NCHUNK; ++c) {
-                                    if (it.perm)
-                                        tma_load_5d(dst + c * C::CHUNK_BYTES, &tmQp, fb, c * C::CHUNK_ELEMS, it.qb,
-                                                    it.pqb * 128, it.h, it.b);
-                                    else
-                                        tma_load_4d(dst + c * C::CHUNK_BYTES, &tmQ, fb, c * C::CHUNK_ELEMS, it.qb * 128,
-                                                    it.h, it.b);
-                                }
-                            }
-                            ++qm[s];
-                            __threadfence_block();
-                            ring_n[s] = qm[s];
-                            progress = true;
-                        }
-                    }
 #pragma unroll
                     for (int k = 1; k < NSTREAM; ++k) {
                         if (!live[s][k]) continue;
                         any = true;
-                        if (km[s][k] >= qm[s]) continue;  // its next item is not taken yet
-                        const int64_t x = ring[s * 4 + (km[s][k] & 3)];
-                        if (x < 0) {
+                        if (km[s][k] >= rn[s]) continue;  // its next item is not taken yet
+                        PpItem it;
+                        if (!ring_get(P, entry(s, km[s][k]), it)) {
                             live[s][k] = false;
                             continue;
                         }
                         const int eb = k == 1 ? kKEmpty : (k == 2 ? kVEmpty : kAEmpty);
                         if (cnt[s][k] != 0 && !mbar_test(bar(s, eb), (cnt[s][k] - 1) & 1)) continue;
-                        const PpItem it = pp_item(P, sh, x);
                         const uint32_t fb = bar(s, k == 1 ? kKFull : (k == 2 ? kVFull : kAFull));
                         const int kt = pp_tile(P, sh, it, ku[s][k]) & 0x7fffffff;
                         if (k < 3) {
@@ -674,9 +749,10 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                     t_last = clock64();
                     nap = 0;
                 } else {
-                    // loads run microseconds ahead of their use: sleep rather than
-                    // take issue slots from the softmax warps on this sub-partition
-                    nap = nap ? (nap < 256 ? 2 * nap : 256) : 32;
+                    // a short sleep: the next buffer frees within microseconds, and
+                    // spinning would take issue slots from the softmax warps
+                    // sharing this sub-partition
+                    nap = nap ? (nap < 64 ? 2 * nap : 64) : 16;
                     __nanosleep(nap);
                     if (*abort_flag) break;
                     if (clock64() - t_last > P.wait_cycles) {
@@ -685,17 +761,138 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                     }
                 }
             }
-            // no load may outlive the CTA: wait (bounded) for the last of each
-            // buffer (a slot that reached its end had its last Q consumed)
+            // no load may outlive the CTA: wait (bounded) for the last of each buffer
 #pragma unroll
-            for (int s = 0; s < 2; ++s) {
-                if (!qend[s] && qm[s]) mbar_wait_bounded(bar(s, kQFull), (qm[s] - 1) & 1, kPpDrainCycles);
+            for (int s = 0; s < 2; ++s)
 #pragma unroll
                 for (int k = 1; k < NSTREAM; ++k) {
                     const int full = k == 1 ? kKFull : (k == 2 ? kVFull : kAFull);
                     if (cnt[s][k]) mbar_wait_bounded(bar(s, full), (cnt[s][k] - 1) & 1, kPpDrainCycles);
                 }
+        }
+    } else if (warp == 2 || warp == 3) {
+        // ------------------------------------------------------------ MMA issuers
+        // warp 2 issues slot 0's MMAs, warp 3 slot 1's (one thread each). Per
+        // 128-key tile g and 64-key half h: S_h(g) = Q K_h(g)^T into the
+        // half's S columns; once the softmax group has written P_h(g) (bf16, in
+        // the first 32 of them), O (+)= P_h(g) V_h(g). S_h(g + 1) overwrites
+        // P_h(g), so it waits for that product; it is issued right after it,
+        // before the other half's product, so that the softmax group finds the
+        // next half's S ready.
+        if (lane == 0) {
+            const int s = warp - 2;
+            const uint32_t tSm = tmem + (uint32_t)(s * 256), tOm = tSm + 128;
+            const uint32_t idS = idesc_bf16_f32(128, 64, false);
+            const uint32_t idO = idesc_bf16_f32(128, D, true);
+            // shared-memory descriptors at the slot's Q and K buffers (K-major
+            // operands) and V buffer (MN-major B); a k-step, a key half and a
+            // column chunk add their byte offset / 16 to the start-address field
+            const uint64_t dQK0 = smem_desc(sQ0, 16, C::SBO, C::LAYOUT);
+            const uint64_t dQ = dQK0 + (uint64_t)((C::OFF_Q + s * C::TILE_BYTES) >> 4);
+            const uint64_t dK = dQK0 + (uint64_t)((C::OFF_K + s * C::TILE_BYTES) >> 4);
+            const uint64_t dV = smem_desc(sV0, C::CHUNK_BYTES, C::SBO, C::LAYOUT) + (uint64_t)((s * C::TILE_BYTES) >> 4);
+            auto issue_s = [&](int h) {  // S_h of the tile whose K is in
+                tc_fence_after();
+#pragma unroll 1
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint64_t off = (uint64_t)(((ks / C::KSTEPS_PER_CHUNK) * C::CHUNK_BYTES +
+                                                     (ks % C::KSTEPS_PER_CHUNK) * 32) >> 4);
+                    mma_bf16_ss(tSm + (uint32_t)(64 * h), dQ + off, dK + off + (uint64_t)((64 * h * C::ROW_BYTES) >> 4),
+                                idS, ks > 0 ? 1u : 0u);
+                }
+                mma_commit(bar(s, kSFull + h));
+            };
+            auto issue_pv = [&](int h, bool zero) {  // O (+)= P_h V_h (zero: O = the product)
+                tc_fence_after();
+#pragma unroll 1
+                for (int ks = 0; ks < 4; ++ks)  // 16 keys per step
+                    mma_bf16_ts(tOm, tSm + (uint32_t)(64 * h + 8 * ks),
+                                dV + (uint64_t)(((4 * h + ks) * 16 * C::ROW_BYTES) >> 4), idO,
+                                (zero && ks == 0) ? 0u : 1u);
+                mma_commit(bar(s, kSFree + h));
+            };
+            auto W = [&](int which, uint32_t phase) { return pp_wait(bar(s, which), phase & 1, abort_flag, P.wait_cycles); };
+            uint32_t g = 0;        // tiles of this slot so far
+            bool s_ready = false;  // both halves of the current item's first S are issued
+            bool alive = true;
+            for (uint32_t m = 0; alive; ++m) {
+                if (ring_n[s] <= (int)m) {
+                    const long long t0 = clock64();
+                    while (ring_n[s] <= (int)m) {
+                        if (*abort_flag || clock64() - t0 > P.wait_cycles) {
+                            *abort_flag = 1;
+                            alive = false;
+                            break;
+                        }
+                        __nanosleep(32);
+                    }
+                    if (!alive) break;
+                }
+                __threadfence_block();
+                PpItem it;
+                if (!ring_get(P, entry(s, m), it)) break;
+                bsg::Item bi;
+                bi.perm = it.perm;
+                bi.chunk = it.chunk;
+                const bool zero_first = !(C::STAGE && P.mode == 1 && bsg::starts_from_perm(sh, bi));
+                if (!s_ready) {
+                    alive = W(kQFull, m) && W(kKFull, g) && (g == 0 || W(kSFree, g - 1));
+                    if (!alive) break;
+                    issue_s(0);
+                    if (!(alive = g == 0 || W(kSFreeB, g - 1))) break;
+                    issue_s(1);
+                    mma_commit(bar(s, kKEmpty));
+                    if (it.T == 1) mma_commit(bar(s, kQEmpty));
+                }
+                s_ready = false;
+                for (int u = 0; u < it.T; ++u, ++g) {
+                    if (!(alive = W(kPFull, g) && W(kVFull, g))) break;
+                    issue_pv(0, u == 0 && zero_first);
+                    // the next tile: this item's next one, or the next item's
+                    // first when its Q and K are already in (else at its start)
+                    bool nxt = false, nlast = false;
+                    if (u + 1 < it.T) {
+                        nxt = true;
+                        nlast = u + 2 == it.T;
+                    } else if (ring_n[s] > (int)(m + 1) && mbar_test(bar(s, kQFull), (m + 1) & 1) &&
+                               mbar_test(bar(s, kKFull), (g + 1) & 1)) {
+                        PpItem itn;
+                        if (ring_get(P, entry(s, m + 1), itn)) {
+                            nxt = true;
+                            nlast = itn.T == 1;
+                        }
+                    }
+                    // S_a(g + 1) before P_b V_b(g) when its K is already in (the
+                    // softmax group turns to it next), else after
+                    bool a_done = false;
+                    if (nxt) {
+                        if (!(alive = W(kSFree, g))) break;
+                        if (mbar_test(bar(s, kKFull), (g + 1) & 1)) {
+                            issue_s(0);
+                            a_done = true;
+                        }
+                    }
+                    if (!(alive = W(kPFullB, g))) break;
+                    issue_pv(1, false);
+                    mma_commit(bar(s, kVEmpty));
+                    if (u + 1 == it.T) mma_commit(bar(s, kODone));
+                    if (nxt) {
+                        if (!a_done) {
+                            if (!(alive = W(kKFull, g + 1))) break;
+                            issue_s(0);
+                        }
+                        if (!(alive = W(kSFreeB, g))) break;
+                        issue_s(1);
+                        mma_commit(bar(s, kKEmpty));
+                        if (nlast) mma_commit(bar(s, kQEmpty));
+                        if (u + 1 == it.T) s_ready = true;
+                    }
+                }
             }
+            if (!alive) *abort_flag = 1;
+            // every MMA this thread issued is complete before TMEM is released
+            mma_commit(bar(s, kDrainS));
+            mbar_wait_bounded(bar(s, kDrainS), 0u, kPpDrainCycles);
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ softmax groups
@@ -706,52 +903,8 @@ __global__ void __launch_bounds__(kPpThreads, 1)
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const uint32_t tS = tmem + (uint32_t)(s * 256) + lane_base, tO = tS + 128;
         const uint32_t stg = smem_u32(smem + C::OFF_STG) + (uint32_t)(warp - 4) * 4096u;
-        const bool leader = t == 0;  // issues this slot's MMAs
-        // MMAs of this slot (leader only). S(g) = Q K(g)^T into S's columns,
-        // then O (+)= P(g) V(g) with P read from the first 64 of them; since P
-        // overwrites S, S(g + 1) is issued only once P V(g) is complete.
-        const uint32_t tSm = tmem + (uint32_t)(s * 256), tOm = tSm + 128;
-        const uint32_t idS = idesc_bf16_f32(128, 128, false);
-        const uint32_t idO = idesc_bf16_f32(128, D, true);
-        // shared-memory descriptors at the Q buffer of slot 0 (K-major operands)
-        // and at the V buffer of slot 0 (MN-major B); a tile and k-step add
-        // their byte offset / 16 to the start-address field (bits 0-13)
-        const uint64_t dQK0 = smem_desc(sQ0, 16, C::SBO, C::LAYOUT);
-        const uint64_t dV0 = smem_desc(sV0, C::CHUNK_BYTES, C::SBO, C::LAYOUT);
-        // S(gs) once Q (the slot's item number qi, on its first tile) and K(gs) are in
-        auto issue_s = [&](uint32_t gs, uint32_t qi, bool first, bool last) -> bool {
-            if (first && !pp_wait(bar(s, kQFull), qi & 1, abort_flag, P.wait_cycles)) return false;
-            if (!pp_wait(bar(s, kKFull), gs & 1, abort_flag, P.wait_cycles)) return false;
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-                const uint64_t off = (uint64_t)(((ks / C::KSTEPS_PER_CHUNK) * C::CHUNK_BYTES +
-                                                 (ks % C::KSTEPS_PER_CHUNK) * 32) >> 4);
-                mma_bf16_ss(tSm, dQK0 + (uint64_t)((C::OFF_Q + s * C::TILE_BYTES) >> 4) + off,
-                            dQK0 + (uint64_t)((C::OFF_K + s * C::TILE_BYTES) >> 4) + off, idS, ks > 0 ? 1u : 0u);
-            }
-            mma_commit(bar(s, kSFull));
-            mma_commit(bar(s, kKEmpty));
-            if (last) mma_commit(bar(s, kQEmpty));
-            return true;
-        };
-        // O (+)= P(gp) V(gp) once V(gp) is in (every row's P is written); zero
-        // sets O to the product (the item's first tile, O not started from a
-        // published state)
-        auto issue_pv = [&](uint32_t gp, bool zero) -> bool {
-            if (!pp_wait(bar(s, kVFull), gp & 1, abort_flag, P.wait_cycles)) return false;
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {  // 16 keys per step
-                const uint64_t db = dV0 + (uint64_t)((s * C::TILE_BYTES + ks * 16 * C::ROW_BYTES) >> 4);
-                mma_bf16_ts(tOm, tSm + (uint32_t)(ks * 8), db, idO, (!zero || ks > 0) ? 1u : 0u);
-            }
-            mma_commit(bar(s, kODone));
-            mma_commit(bar(s, kVEmpty));
-            return true;
-        };
-        uint32_t g = 0;         // tiles of this slot so far
-        bool s_ready = false;   // leader: S of the current item's first tile is issued
+        uint32_t g = 0;            // tiles of this slot so far
+        unsigned* pend = nullptr;  // a published permuted block this warp has not counted in yet
         for (uint32_t m = 0;; ++m) {
             // the slot's m-th item, once the producer has taken it
             bool okq = true;
@@ -768,9 +921,8 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             }
             if (!__all_sync(0xffffffffu, okq)) break;
             __threadfence_block();
-            const int64_t x = ring[s * 4 + (m & 3)];
-            if (x < 0) break;
-            const PpItem it = pp_item(P, sh, x);
+            PpItem it;
+            if (!ring_get(P, entry(s, m), it)) break;
             bsg::Item bi;
             bi.bh = it.bh;
             bi.perm = it.perm;
@@ -779,9 +931,6 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             bi.chunk = it.chunk;
             bi.u0 = it.u0;
             bi.T = it.T;
-            if (leader && !s_ready && !issue_s(g, m, true, it.T == 1)) *abort_flag = 1;
-            s_ready = false;
-            __syncwarp();
             int i;
             bool row_ok;
             int rlo = 0, rhi = 0;
@@ -799,10 +948,11 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             }
             float m_ref = -INFINITY, l = 0.f;
             // a regular block whose rows also have a permuted part starts from
-            // that part's published state (m, l and O), loaded while S(first
-            // tile) is computed; rows without one start from O = 0
+            // that part's published state (m, l and O), loaded while S of its
+            // first tile is computed; rows without one start from O = 0
             const bool init_o = C::STAGE && P.mode == 1 && bsg::starts_from_perm(sh, bi);
             if (C::STAGE && init_o) {
+                pp_release(pend);  // before waiting on any count
                 const bool pr = row_ok && bsg::has_perm(sh, i);
                 bool use = pr;
                 const int64_t prow = (int64_t)it.bh * P.n + (pr ? i : 0);
@@ -825,7 +975,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                 // each row's count is acquired by its own lane; the barrier and
                 // a fence put every lane's loads (lanes load other rows) after them
                 __syncwarp();
-                __threadfence();
+                fence_acq_rel_gpu();
                 if (use) {
                     m_ref = __ldcg(P.pml + prow * 2);
                     l = __ldcg(P.pml + prow * 2 + 1);
@@ -835,7 +985,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             }
             const int klim = pp_key_limit(P, it.b);
             bool alive = true;
-            for (int u = 0; u < it.T; ++u, ++g) {
+            for (int u = 0; u < it.T && alive; ++u, ++g) {
                 const int info = pp_tile(P, sh, it, u);
                 const int kt = info & 0x7fffffff;
                 bool dense = P.mode == 0 && info < 0;
@@ -860,13 +1010,6 @@ __global__ void __launch_bounds__(kPpThreads, 1)
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
                     if (dense || __any_sync(0xffffffffu, w[q] != 0u)) need |= 1u << q;
-
-                const bool ok = pp_wait(bar(s, kSFull), g & 1, abort_flag, P.wait_cycles);
-                if (!__all_sync(0xffffffffu, ok)) {
-                    alive = false;
-                    break;
-                }
-                tc_fence_after();
                 if (EXTRA) {  // this tile's blocks of the additive terms are in shared memory
                     const bool oka = pp_wait(bar(s, kAFull), g & 1, abort_flag, P.wait_cycles);
                     if (!__all_sync(0xffffffffu, oka)) {
@@ -874,28 +1017,35 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                         break;
                     }
                 }
-                // Stream the tile 32 keys at a time (the next chunk's TMEM load is
-                // in flight while this one is processed): scale, additive terms,
-                // entries not in the mask to -inf, then p = 2^(x - m_ref) against
-                // the running reference max, row sum, bf16 P into TMEM. When a
-                // chunk's max exceeds the reference by more than 2^8 the
-                // reference moves to it and the P chunks already written (and
-                // the sum) are rescaled in place; O is rescaled after the tile.
-                // P of keys 32q .. 32q + 31 goes to columns 16q .. 16q + 15,
-                // which only hold S chunks already consumed.
-                float alpha_t = 1.f;  // product of this tile's rescales
-                float xa[32], xb[32];
-                if (need & 1u) tmem_ld32f(tS, xa);
-                tmem_wait_ld_depf(xa);
 #pragma unroll 1
-                for (int q = 0; q < 4; q += 2) {
+                for (int h = 0; h < 2; ++h) {
+                    const bool ok = pp_wait(bar(s, kSFull + h), g & 1, abort_flag, P.wait_cycles);
+                    if (!__all_sync(0xffffffffu, ok)) {
+                        alive = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t tSh = tS + (uint32_t)(64 * h);
+                    // Stream the half 32 keys at a time (the second chunk's TMEM
+                    // load in flight while the first is processed): scale,
+                    // additive terms, entries not in the mask to -inf, then
+                    // p = 2^(x - m_ref) against the running reference max, row
+                    // sum, bf16 P into TMEM. When a chunk's max exceeds the
+                    // reference by more than 2^8 the reference moves to it and
+                    // the half's P chunk already written (and the sum) are
+                    // rescaled in place; O is rescaled after the half. P of keys
+                    // 64 h + 32 c .. + 31 goes to the half's columns 16 c ..
+                    // 16 c + 15, which only hold S already consumed.
+                    float alpha_h = 1.f;  // product of this half's rescales
+                    float xa[32], xb[32];
+                    if (need & (1u << (2 * h))) tmem_ld32f(tSh, xa);
+                    tmem_wait_ld_depf(xa);
 #pragma unroll
                     for (int hq = 0; hq < 2; ++hq) {
-                        const int qq = q + hq;
+                        const int qq = 2 * h + hq;
                         float(&xc)[32] = hq == 0 ? xa : xb;
-                        float(&xn)[32] = hq == 0 ? xb : xa;
-                        // next chunk's load first (waited for at the end of this one)
-                        if (qq + 1 < 4 && (need & (2u << qq))) tmem_ld32f(tS + 32 * (qq + 1), xn);
+                        // the second chunk's load first (waited for at the end of the first)
+                        if (hq == 0 && (need & (2u << qq))) tmem_ld32f(tSh + 32, xb);
                         uint32_t pk[16];
                         if (need & (1u << qq)) {
                             const uint32_t wq = qq == 0 ? w[0] : (qq == 1 ? w[1] : (qq == 2 ? w[2] : w[3]));
@@ -938,29 +1088,28 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                             const float mx = fmaxf(ma, mb);
                             const bool grow = mx > m_ref + kPpRescale;
                             if (__any_sync(0xffffffffu, grow)) {
-                                // rare: new reference; P chunks 0 .. qq - 1 of this tile and
-                                // the sum scale by alpha (1 for rows that keep theirs)
+                                // rare: new reference; the half's first P chunk (when
+                                // this is its second) and the sum scale by alpha (1
+                                // for rows that keep theirs)
                                 float alpha = 1.f;
                                 if (grow) {
                                     alpha = ex2(m_ref - mx);
                                     m_ref = mx;
                                     l *= alpha;
-                                    alpha_t *= alpha;
+                                    alpha_h *= alpha;
                                 }
-                                tmem_wait_st();  // the P chunks written so far, before reading them back
-#pragma unroll 1
-                                for (int pq = 0; pq < qq; ++pq) {
+                                if (hq == 1) {
+                                    tmem_wait_st();  // the P chunk written, before reading it back
                                     uint32_t pw[16];
-                                    tmem_ld16(tS + 16 * pq, pw);
+                                    tmem_ld16(tSh, pw);
                                     tmem_wait_ld_dep16(pw);
 #pragma unroll
                                     for (int k = 0; k < 16; ++k) {
-                                        __nv_bfloat162 hv = __floats2bfloat162_rn(
-                                            __uint_as_float(pw[k] << 16) * alpha,
-                                            __uint_as_float(pw[k] & 0xffff0000u) * alpha);
+                                        __nv_bfloat162 hv = __floats2bfloat162_rn(__uint_as_float(pw[k] << 16) * alpha,
+                                                                                  __uint_as_float(pw[k] & 0xffff0000u) * alpha);
                                         pw[k] = *reinterpret_cast<uint32_t*>(&hv);
                                     }
-                                    tmem_st16(tS + 16 * pq, pw);
+                                    tmem_st16(tSh, pw);
                                 }
                             }
                             const float mu = m_ref == -INFINITY ? 0.f : m_ref;
@@ -987,74 +1136,55 @@ __global__ void __launch_bounds__(kPpThreads, 1)
 #pragma unroll
                             for (int k = 0; k < 16; ++k) pk[k] = 0u;
                         }
-                        tmem_st16(tS + 16 * qq, pk);
-                        tmem_wait_ld_depf(xn);  // the next chunk's S
+                        tmem_st16(tSh + 16 * hq, pk);
+                        if (hq == 0) tmem_wait_ld_depf(xb);  // the second chunk's S
                     }
+                    if ((u > 0 || h > 0 || init_o) && __any_sync(0xffffffffu, alpha_h != 1.f)) {
+                        // bring O (every product issued before this half's, once
+                        // complete, or the published state it started from) to the
+                        // new reference
+                        if (u > 0 || h > 0) {
+                            const bool ok2 = h > 0 ? pp_wait(bar(s, kSFree), g & 1, abort_flag, P.wait_cycles)
+                                                   : pp_wait(bar(s, kSFreeB), (g - 1) & 1, abort_flag, P.wait_cycles);
+                            if (!__all_sync(0xffffffffu, ok2)) {
+                                alive = false;
+                                break;
+                            }
+                            tc_fence_after();
+                        }
+#pragma unroll 1
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t ro[32];
+                            tmem_ld32(tO + 32 * c, ro);
+                            tmem_wait_ld_dep(ro);
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj) ro[jj] = __float_as_uint(__uint_as_float(ro[jj]) * alpha_h);
+                            tmem_st32(tO + 32 * c, ro);
+                        }
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(s, kPFull + h));
+                    // a permuted block published at the previous item's end: its
+                    // stores have had this half's time to land
+                    if (u == 0 && h == 0) pp_release(pend);
                 }
+                if (!alive) break;
                 if (EXTRA) {  // the additive blocks are read: the producer may refill them
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(s, kAEmpty));
                 }
-                if ((u > 0 || init_o) && __any_sync(0xffffffffu, alpha_t != 1.f)) {
-                    // bring O (P V of the item's tiles so far, complete, or the
-                    // published state it started from) to the new reference
-                    if (u > 0) {
-                        const bool ok2 = pp_wait(bar(s, kODone), (g - 1) & 1, abort_flag, P.wait_cycles);
-                        if (!__all_sync(0xffffffffu, ok2)) {
-                            alive = false;
-                            break;
-                        }
-                        tc_fence_after();
-                    }
-#pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t ro[32];
-                        tmem_ld32(tO + 32 * c, ro);
-                        tmem_wait_ld_dep(ro);
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) ro[jj] = __float_as_uint(__uint_as_float(ro[jj]) * alpha_t);
-                        tmem_st32(tO + 32 * c, ro);
-                    }
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(s, kPFull));
-                if (leader) {
-                    // every row's P(g) is in TMEM: P V(g); then, once it has
-                    // consumed P, this item's next S -- or, after its last tile,
-                    // the next item's first S when its Q and K are already in
-                    // (else at that item's start)
-                    bool okl = pp_wait(bar(s, kPFull), g & 1, abort_flag, P.wait_cycles) &&
-                               issue_pv(g, u == 0 && !init_o) &&
-                               pp_wait(bar(s, kODone), g & 1, abort_flag, P.wait_cycles);
-                    if (okl) {
-                        if (u + 1 < it.T) {
-                            okl = issue_s(g + 1, m, false, u + 2 == it.T);
-                        } else if (mbar_test(bar(s, kQFull), (m + 1) & 1)) {
-                            const int64_t xn = ring[s * 4 + ((m + 1) & 3)];
-                            if (xn >= 0 && mbar_test(bar(s, kKFull), (g + 1) & 1)) {
-                                okl = issue_s(g + 1, m + 1, true, pp_item(P, sh, xn).T == 1);
-                                s_ready = true;
-                            }
-                        }
-                    }
-                    if (!okl) *abort_flag = 1;
-                }
-                __syncwarp();
             }
             if (!alive) break;
             // ---------------------------------------------------------- epilogue
-            const bool ok = pp_wait(bar(s, kODone), (g - 1) & 1, abort_flag, P.wait_cycles);
+            const bool ok = pp_wait(bar(s, kODone), m & 1, abort_flag, P.wait_cycles);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-            pp_finish<D, C::STAGE>(P, sh, it, quarter, t, i, row_ok, m_ref, l, tO, stg);
+            pp_finish<D, C::STAGE>(P, sh, it, quarter, t, i, row_ok, m_ref, l, tO, stg, pend);
             __syncwarp();
         }
-        if (leader) {  // every MMA this thread issued is complete before TMEM is released
-            mma_commit(bar(s, kDrainS));
-            mbar_wait_bounded(bar(s, kDrainS), 0u, kPpDrainCycles);
-        }
+        pp_release(pend);
     }
 
     // ---------------------------------------------------------------- teardown

@@ -1005,12 +1005,19 @@ int fwd_closed(const FwdParams& p, int d, spattn_mask m, cudaStream_t s, cudaMem
     return SPATTN_OK;
 }
 
-// Whether the persistent tile kernel takes an interval-mask forward: d = 32,
-// 64 or 128; additive terms only for d <= 64 and when TMA can stage them.
+// Whether the persistent tile kernel takes an interval-mask forward. By
+// default d = 128 without additive terms: at d <= 64 the four-CTAs-per-SM tile
+// kernel (k_fwd_tc_quad) is faster on the interval workloads (variable window
+// 0.10 against 0.15 ms, the Evoformer shape 0.15 against 0.24 ms, on one
+// B200), so it keeps them. SPATTN_DEBUG_PP_INTERVAL=1 sends d = 32 and 64
+// (additive terms too, when TMA can stage them) to the persistent kernel as
+// well; the tests use it to cover those paths.
 bool pp_takes_interval(const FwdParams& p, int d) {
-    if (d != 32 && d != 64 && d != 128) return false;
-    if (!p.has_extra) return true;
-    return d <= 64 && pp_addend_ok(p.mask) && pp_addend_ok(p.bias);
+    const char* e = getenv("SPATTN_DEBUG_PP_INTERVAL");
+    const bool all = e && e[0] == '1';
+    if (d == 128) return !p.has_extra;
+    if (!all || (d != 32 && d != 64)) return false;
+    return !p.has_extra || (pp_addend_ok(p.mask) && pp_addend_ok(p.bias));
 }
 
 // The persistent tile kernel over an interval mask's tiles; blk_res: the
@@ -1646,7 +1653,10 @@ int spattn_fwd_mask_kpad(const spattn_tensor* q, const spattn_tensor* k, const s
     p.num_masks = mask->num_masks;
     p.long_count_dev = nullptr;
     if (mask->closed) {
-        if (dtype == 0 && !seqlen_k && !p.has_extra && (d == 64 || d == 128))
+        // the kernel numbers its items in 32 bits
+        const bsg::Shape sh = bsg::shape(p.n, mask->bsg_block, mask->bsg_stride, mask->bsg_ng, kChunkTiles);
+        const bool fits = (int64_t)p.B * p.H * sh.items_per_head < ((int64_t)1 << 31);
+        if (dtype == 0 && !seqlen_k && !p.has_extra && (d == 64 || d == 128) && fits)
             return fwd_closed(p, d, mask, s, pool, dev, sms);
         if ((r = ensure_generic(mask))) return r;
         return spattn_fwd_mask_kpad(q, k, v, mask->generic, seqlen_k, add_mask, bias, scale, out, lse, stream_v);

@@ -3,16 +3,17 @@
 Block + strided + global masks whose parameters allow it (block dividing 128,
 stride 0 or 128, at most 128 global tokens, n a multiple of 128) are kept in
 closed form: the forward derives every tile and every row's bits from the
-parameters, runs the regular query blocks and the residue-permuted blocks of
-the strided entries in one launch, and merges the two partial states of each
-row. These tests cover the parameter corners of that plan (no global tokens, no
+parameters and runs the regular query blocks and the residue-permuted blocks
+of the strided entries in one launch, a regular block starting each of its rows
+from the published partial state of the row's permuted part. These tests cover the parameter corners of that plan (no global tokens, no
 block part, no strided part, permuted blocks shorter than a tile, more than one
 permuted tile per residue, one mask per batch element), d = 64 and 128, the
 fallbacks that go through the CSR-built copy of the mask (fp32 inputs, an
 additive term, key lengths), interval masks (dense, sliding, variable window)
-on the same kernel at d = 32, 64 and 128 -- with additive mask and bias
-layouts staged through shared memory, key lengths, and the layouts that fall
-back to the per-block kernels --, the two section-(b) entry points
+on the same kernel at d = 128 (and, with SPATTN_DEBUG_PP_INTERVAL=1, at
+d = 32 and 64, where the default is the four-CTAs-per-SM tile kernel) -- with
+additive mask and bias layouts staged through shared memory, key lengths, and
+the layouts that fall back to the per-block kernels --, the entry points
 spattn_mask_csr and spattn_check_device_error, and the bounded waits: with a
 wait limit of zero cycles every wait gives up, the call reports
 SPATTN_ERR_TIMEOUT, and the next call is exact again (the kernel released its
@@ -163,16 +164,21 @@ def test_dense_interval_mask_d128(n, B, H):
     _check(mp, B, H, 128, seed=n, what=f"dense d=128 n={n}")
 
 
+@pytest.mark.parametrize("route", ["default", "persistent"])
 @pytest.mark.parametrize("d", [32, 64])
 @pytest.mark.parametrize("layout", ["row_mask", "bias_only", "pad_mask_and_bias", "row_mask_and_bias",
                                     "f32_bias", "head_mask"])
 @pytest.mark.parametrize("kind,n", [("dense", 256), ("sliding", 384), ("dense", 200)])
-def test_interval_mask_with_additive_terms(d, layout, kind, n):
-    """Additive mask and bias on interval masks: bf16 terms with keys
-    contiguous and 16-byte rows are staged through shared memory tile by tile
-    (row-varying, shared by all rows, per head); an fp32 term, or rows that are
-    not 16-byte multiples (n = 200: 400-byte rows are, n odd would not), take
-    the per-block kernel; both must equal the oracle."""
+def test_interval_mask_with_additive_terms(d, layout, kind, n, route, monkeypatch):
+    """Additive mask and bias on interval masks at d <= 64: by default on the
+    four-CTAs-per-SM tile kernel; with SPATTN_DEBUG_PP_INTERVAL=1 on the
+    persistent kernel, where bf16 terms with keys contiguous and 16-byte rows
+    are staged through shared memory tile by tile (row-varying, shared by all
+    rows, per head) and an fp32 term, or rows that are not 16-byte multiples
+    (n = 200: 400-byte rows are, n odd would not), take the per-block kernel;
+    every route must equal the oracle."""
+    if route == "persistent":
+        monkeypatch.setenv("SPATTN_DEBUG_PP_INTERVAL", "1")
     rng = np.random.default_rng(7 + d + n)
     B, H = 2, 3
     mp = workloads.MaskParams(kind, n, 1, window=40 if kind == "sliding" else 0)
@@ -201,11 +207,14 @@ def test_interval_mask_with_additive_terms(d, layout, kind, n):
     assert sp.spattn_device_error() == 0
 
 
-@pytest.mark.parametrize("d", [32, 64, 128])
-def test_key_lengths_with_bias_on_the_persistent_kernel(d):
-    """Key lengths on tile edges with a pair bias (d <= 64 stages the bias; at
-    d = 128 the bias takes the per-block kernel), against the oracle with the
-    equivalent additive key-padding mask."""
+@pytest.mark.parametrize("d,route", [(32, "default"), (32, "persistent"), (64, "default"), (64, "persistent"),
+                                     (128, "default")])
+def test_key_lengths_with_bias_on_the_persistent_kernel(d, route, monkeypatch):
+    """Key lengths on tile edges with a pair bias (on the persistent kernel,
+    d <= 64 stages the bias; at d = 128 the bias takes the per-block kernel),
+    against the oracle with the equivalent additive key-padding mask."""
+    if route == "persistent":
+        monkeypatch.setenv("SPATTN_DEBUG_PP_INTERVAL", "1")
     lengths = [0, 1, 127, 128, 129, 255, 256, 200]
     B, H, n = len(lengths), 2, 256
     rng = np.random.default_rng(30 + d)
