@@ -48,7 +48,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, default=3, help="workload index 0..4 (default 3)")
+    ap.add_argument("--config", type=int, default=3, help="workload index 0..5 (default 3)")
     ap.add_argument("--settle-seconds", type=float, default=1.0,
                     help="untimed load before the warm-up, so the clock sampler sees the GPU under load")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' forward timings")
