@@ -117,7 +117,10 @@ struct PpCfg {
     // per softmax warp a 4 KB buffer through which the epilogue's global
     // accesses go as whole lines (when it fits beside the tiles)
     static constexpr int STG_BYTES = 8 * 4096;
-    static constexpr int RING_BYTES = 2 * 4 * 8 * 4 + 16;  // [slot][4] decoded items (8 words), then [slot] counts
+    // [slot][4] decoded items (8 words), [slot] counts; then per softmax warp a
+    // FIFO of published permuted blocks: [8][4] count offsets, [8] pushed,
+    // [8] counted in, one count of warps done
+    static constexpr int RING_BYTES = 2 * 4 * 8 * 4 + 16 + 8 * 4 * 4 + 8 * 4 + 8 * 4 + 16;
     static constexpr bool STAGE = OFF_A + (EXTRA ? 4 * A_BYTES : 0) + STG_BYTES + kNumBars * 8 + 16 + RING_BYTES <= 227 * 1024;
     static constexpr int OFF_STG = OFF_A + (EXTRA ? 4 * A_BYTES : 0);
     static constexpr int OFF_BAR = OFF_STG + (STAGE ? STG_BYTES : 0);
@@ -248,6 +251,15 @@ __device__ __forceinline__ void regs_inc() {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
 }
 
+__device__ __forceinline__ void st_release_cta(volatile int* p, int v) {
+    asm volatile("st.release.cta.shared.b32 [%0], %1;" ::"r"(smem_u32((const void*)p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_cta(volatile int* p) {
+    int v;
+    asm volatile("ld.acquire.cta.shared.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32((const void*)p)) : "memory");
+    return v;
+}
+
 // Release / acquire fence at GPU scope (ordering, not sequential consistency).
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
@@ -338,20 +350,6 @@ __device__ __forceinline__ void rows_to_tmem(uint32_t stg, int lane, uint64_t sr
     }
 }
 
-// Counts this warp in on a permuted block whose state it published: every
-// lane's stores (lanes wrote other rows' lines) are ordered before the
-// barrier, and the barrier before lane 0's fence and count.
-__device__ __forceinline__ void pp_release(unsigned*& pend) {
-    if (!pend) return;
-    fence_acq_rel_gpu();
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) {
-        fence_acq_rel_gpu();
-        atomicAdd(pend, 1u);
-    }
-    pend = nullptr;
-}
-
 // 32 columns of this warp's rows of O (fp32, not yet divided by L) from TMEM.
 __device__ __forceinline__ void o_chunk(uint32_t tO, int c, float (&x)[32]) {
     tmem_ld32f(tO + 32 * c, x);
@@ -390,7 +388,7 @@ __device__ __forceinline__ void put_out_piece(uint64_t orow, int p, float inv, c
 // lines through the warp's staging buffer stg.
 template <int D, bool STAGE>
 __device__ __forceinline__ void pp_finish(const PpParams& P, const bsg::Shape& sh, const PpItem& it, int quarter, int t, int i,
-                          bool row_ok, float M, float L, uint32_t tO, uint32_t stg, unsigned*& pend) {
+                          bool row_ok, float M, float L, uint32_t tO, uint32_t stg, volatile int* pubq) {
     const int lane = threadIdx.x & 31;
     const int64_t bh = it.bh;
     const uint64_t orow_any = reinterpret_cast<uint64_t>(reinterpret_cast<__nv_bfloat16*>(P.out) + (int64_t)it.b * P.o_sb +
@@ -510,8 +508,30 @@ __device__ __forceinline__ void pp_finish(const PpParams& P, const bsg::Shape& s
                     *reinterpret_cast<float4*>(P.pacc + prow * D + 32 * c + z) = make_float4(x[z], x[z + 1], x[z + 2], x[z + 3]);
             }
         }
-        // counted in later (pp_release), once the stores have long completed
-        pend = P.pflag + (bh * sh.npqb + it.pqb) * 128 + it.qb;
+        // queue the block's count for the item-taker thread, which counts this
+        // warp in after a fence at GPU scope (off this warp's path): lane 0
+        // releases the queue entry at CTA scope after the barrier that orders
+        // every lane's stores (lanes wrote other rows' lines) before it
+        __syncwarp();
+        if (lane == 0) {
+            const int w = (threadIdx.x >> 5) - 4;
+            volatile int* pushed = pubq + 32 + w;
+            volatile int* counted = pubq + 40 + w;
+            const int n = *pushed;
+            if (n - *counted >= 4) {  // the queue is full: wait (bounded) for the taker
+                const long long t0 = clock64();
+                while (n - ld_acquire_cta(counted) >= 4) {
+                    if (clock64() - t0 > P.wait_cycles) {
+                        atomicOr(P.err, kErrTimeout);
+                        break;
+                    }
+                    __nanosleep(64);
+                }
+            }
+            pubq[w * 4 + (n & 3)] = (int)((bh * sh.npqb + it.pqb) * 128 + it.qb);
+            st_release_cta(pushed, n + 1);
+        }
+        __syncwarp();
         return;
     }
     // a regular block's rows: the output (their permuted part, if any, is in O already)
@@ -555,6 +575,10 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     // ahead of them, where a barrier's phase parity would not tell)
     volatile int* ring = reinterpret_cast<volatile int*>(smem + C::OFF_RING);  // [slot][4][8]
     volatile int* ring_n = reinterpret_cast<volatile int*>(smem + C::OFF_RING + 2 * 4 * 8 * 4);
+    // per softmax warp w a queue of the permuted blocks it published: entries
+    // pubq[4 w .. 4 w + 3] (count offsets), pushed pubq[32 + w], counted in
+    // pubq[40 + w]; pubq[48]: softmax warps done
+    volatile int* pubq = ring_n + 4;
     auto entry = [&](int s, uint32_t m) { return ring + (s * 4 + (int)(m & 3u)) * 8; };
 
     if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kPpTmemCols);
@@ -564,6 +588,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                 mbar_init(bar(s, x), (x == kPFull || x == kPFullB || x == kAEmpty) ? 4u : 1u);
         *abort_flag = 0;
         ring_n[0] = ring_n[1] = 0;
+        for (int x = 32; x < 49; ++x) pubq[x] = 0;
         fence_mbar_init();
         prefetch_tensormap(&tmQ);
         prefetch_tensormap(&tmK);
@@ -607,10 +632,32 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                     if (it.T > 0) return true;
                 }
             };
+            int counted[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // per softmax warp: blocks counted in
             long long t_last = clock64();
             unsigned nap = 0;
             while (true) {
                 bool any = false, progress = false;
+                // count in the permuted blocks the softmax warps published: one
+                // fence at GPU scope after acquiring their queues, then the counts
+                {
+                    int pushed[8];
+                    bool work = false;
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) {
+                        pushed[w] = ld_acquire_cta(pubq + 32 + w);
+                        work |= pushed[w] != counted[w];
+                    }
+                    if (work) {
+                        fence_acq_rel_gpu();
+#pragma unroll
+                        for (int w = 0; w < 8; ++w) {
+                            for (; counted[w] != pushed[w]; ++counted[w])
+                                atomicAdd(P.pflag + pubq[4 * w + (counted[w] & 3)], 1u);
+                            st_release_cta(pubq + 40 + w, counted[w]);
+                        }
+                        progress = true;
+                    }
+                }
 #pragma unroll
                 for (int s = 0; s < 2; ++s) {
                     if (qend[s]) continue;
@@ -644,7 +691,15 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                     ring_n[s] = qm[s];
                     progress = true;
                 }
-                if (!any) break;
+                // done once every item is handed out and every softmax warp has
+                // finished (its last publication counted in above)
+                if (!any && ld_acquire_cta(pubq + 48) == 8) {
+                    bool drained = true;
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) drained &= ld_acquire_cta(pubq + 32 + w) == counted[w];
+                    if (drained) break;
+                    continue;
+                }
                 if (progress) {
                     t_last = clock64();
                     nap = 0;
@@ -904,7 +959,6 @@ __global__ void __launch_bounds__(kPpThreads, 1)
         const uint32_t tS = tmem + (uint32_t)(s * 256) + lane_base, tO = tS + 128;
         const uint32_t stg = smem_u32(smem + C::OFF_STG) + (uint32_t)(warp - 4) * 4096u;
         uint32_t g = 0;            // tiles of this slot so far
-        unsigned* pend = nullptr;  // a published permuted block this warp has not counted in yet
         for (uint32_t m = 0;; ++m) {
             // the slot's m-th item, once the producer has taken it
             bool okq = true;
@@ -952,7 +1006,6 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             // first tile is computed; rows without one start from O = 0
             const bool init_o = C::STAGE && P.mode == 1 && bsg::starts_from_perm(sh, bi);
             if (C::STAGE && init_o) {
-                pp_release(pend);  // before waiting on any count
                 const bool pr = row_ok && bsg::has_perm(sh, i);
                 bool use = pr;
                 const int64_t prow = (int64_t)it.bh * P.n + (pr ? i : 0);
@@ -1166,9 +1219,6 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(s, kPFull + h));
-                    // a permuted block published at the previous item's end: its
-                    // stores have had this half's time to land
-                    if (u == 0 && h == 0) pp_release(pend);
                 }
                 if (!alive) break;
                 if (EXTRA) {  // the additive blocks are read: the producer may refill them
@@ -1181,10 +1231,12 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             const bool ok = pp_wait(bar(s, kODone), m & 1, abort_flag, P.wait_cycles);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-            pp_finish<D, C::STAGE>(P, sh, it, quarter, t, i, row_ok, m_ref, l, tO, stg, pend);
+            pp_finish<D, C::STAGE>(P, sh, it, quarter, t, i, row_ok, m_ref, l, tO, stg, pubq);
             __syncwarp();
         }
-        pp_release(pend);
+        // this warp publishes nothing more (released after its last queue entry)
+        __syncwarp();
+        if (lane == 0) asm volatile("red.release.cta.shared.add.u32 [%0], 1;" ::"r"(smem_u32((const void*)(pubq + 48))) : "memory");
     }
 
     // ---------------------------------------------------------------- teardown
