@@ -109,36 +109,46 @@ struct Item {
     int T;      // tiles of this item
 };
 
-// Item x of all bh_count * items_per_head: first the permuted blocks of every
-// (b, h), then the regular blocks of every (b, h) (per (b, h) the chunks of
-// query block 0 first, the items with the most tiles). Rows met by both kinds
-// of block start their regular part from the permuted part's published
-// state; with every permuted block ahead of every regular one, a regular
-// block almost never waits for its rows' state, and items taken in this order
-// never wait for a later one. (Interleaving the two kinds head by head keeps
-// the published states in L2 but makes regular blocks wait for late permuted
-// ones, which cost more on one B200: 0.39 against 0.34 ms on the 16-head
-// n = 16384 workload.)
+// Item x of all bh_count * items_per_head, in four phases over every (b, h):
+//   1. the chunks of query block 0 but the first (items with many tiles and
+//      no dependency: they start early, so that they do not end last),
+//   2. the permuted blocks,
+//   3. the first chunk of query block 0 (or query block 0 itself),
+//   4. the remaining regular blocks (the items with the fewest tiles: they
+//      fill the end evenly).
+// Rows met by both kinds of block start their regular part from the permuted
+// part's published state; with every permuted block ahead of every regular
+// one, a regular block almost never waits for its rows' state, and items
+// taken in this order never wait for a later one. (Interleaving the two kinds
+// head by head keeps the published states in L2 but makes regular blocks wait
+// for late permuted ones, which cost more on one B200: 0.39 against 0.34 ms
+// on the 16-head n = 16384 workload.)
 BSG_HD Item item(const Shape& s, int64_t x64, int bh_count) {
     // 32-bit arithmetic: callers keep bh_count * items_per_head below 2^31
-    const int x = (int)x64;
+    int x = (int)x64;
     Item it;
     it.perm = 0;
     it.qb = 0;
     it.pqb = 0;
     it.chunk = 0;
     it.u0 = 0;
-    const int nregular = s.n_lead + s.nreg;
-    const int lead = bh_count * s.nperm;
-    int j;
-    if (x < lead) {
+    const int rest_chunks = s.n_lead > 1 ? s.n_lead - 1 : 0;
+    const int p1 = bh_count * rest_chunks, p2 = bh_count * s.nperm, p3 = s.n_lead > 0 ? bh_count : 0;
+    int j;  // chunk (phases 1 and 3), permuted block (2) or regular block (4) within the (b, h)
+    if (x < p1) {
+        it.bh = x / rest_chunks;
+        j = 1 + (x - it.bh * rest_chunks);
+    } else if ((x -= p1) < p2) {
         it.bh = x / s.nperm;
         it.perm = 1;
         j = x - it.bh * s.nperm;
+    } else if ((x -= p2) < p3) {
+        it.bh = x;
+        j = 0;
     } else {
-        const int z = x - lead;
-        it.bh = z / nregular;
-        j = z - it.bh * nregular;
+        x -= p3;
+        it.bh = x / s.nreg;
+        j = s.n_lead + (x - it.bh * s.nreg);
     }
     if (it.perm) {
         it.qb = j / s.npqb;

@@ -7,7 +7,8 @@
 // is computed (uint8), the per-row "has entries in a permuted block" flag
 // computed from the bits (uint8 [n]) and the one bsg::has_perm reports (uint8
 // [n]). Exit status 2 when the parameters are outside the closed form, 6 when
-// a regular item of a head comes before one of that head's permuted items.
+// a regular item that starts from published states comes before one of its
+// head's permuted items.
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
@@ -31,7 +32,7 @@ int main(int argc, char** argv) {
         const Item it = item(s, x, heads);
         if (it.bh < 0 || it.bh >= heads) return 3;
         if (it.perm) last_perm[it.bh] = x;
-        else if (first_reg[it.bh] < 0) first_reg[it.bh] = x;
+        else if (starts_from_perm(s, it) && first_reg[it.bh] < 0) first_reg[it.bh] = x;
         if (it.bh != 1) continue;
         for (int u = 0; u < it.T; ++u) {
             const int kt = key_tile(s, it, u);
