@@ -236,21 +236,37 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- traffic
-KERNEL_SOURCES = {"k_fwd_pp": "fwd_pp.cu", "k_fwd_tc": "fwd_tc.cu", "k_fwd_tc_quad": "fwd_tc.cu",
-                  "k_fwd_short": "fwd_gather.cu"}
+# source files (under sparse_mask_scaled_b200/csrc) whose contents a kernel's
+# ncu summary was taken on: the kernel's own file and the headers it includes
+KERNEL_SOURCES = {
+    "k_fwd_pp": ["fwd_pp.cu", "bsg_plan.cuh", "sm100_ptx.cuh", "spattn_internal.cuh"],
+    "k_fwd_tc": ["fwd_tc.cu", "sm100_ptx.cuh", "spattn_internal.cuh"],
+    "k_fwd_tc_quad": ["fwd_tc.cu", "sm100_ptx.cuh", "spattn_internal.cuh"],
+    "k_fwd_short": ["fwd_gather.cu", "spattn_internal.cuh"],
+}
+
+
+def kernel_source_hash(base: str):
+    """First 16 hex digits of the SHA-256 over the kernel's source files in
+    order (None for a kernel not listed)."""
+    files = KERNEL_SOURCES.get(base)
+    if not files:
+        return None
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, "sparse_mask_scaled_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
 
 
 def committed_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary of this kernel and
     workload (profiles/<kernel base name>_<workload>.md), or None when there is
-    none or the kernel's source changed since the capture."""
+    none or the kernel's sources changed since the capture."""
     base = kernel.split("<")[0]
     path = os.path.join(ROOT, "profiles", f"{base}_{workload}.md")
-    src = KERNEL_SOURCES.get(base)
-    if not src or not os.path.exists(path):
+    want = kernel_source_hash(base)
+    if not want or not os.path.exists(path):
         return None
-    kernel_file = os.path.join(ROOT, "sparse_mask_scaled_b200", "csrc", src)
-    want = hashlib.sha256(open(kernel_file, "rb").read()).hexdigest()[:16]
     vals = {}
     for ln in open(path):
         if ":" in ln and ln.strip().startswith("- "):
