@@ -154,8 +154,9 @@ typedef struct spattn_mask_s* spattn_mask;
  * and never synchronises; the forward pass derives every tensor-core tile and
  * every row's bits from the four parameters, the strided entries outside the
  * regular tiles running as residue-permuted dense tiles (token i at
- * (i mod 128) n/128 + i div 128) in the same launch, each row's two partial
- * states merged with the running max / sum rule in fp32. Its CSR, tile plan,
+ * (i mod 128) n/128 + i div 128) in the same launch: each row's regular
+ * part starts from the fp32 partial state (m, l, O) its permuted part
+ * published, the running max / sum combination of the two. Its CSR, tile plan,
  * the backward pass and forward calls the closed form does not take (fp32
  * inputs, additive terms, key lengths, d = 32) use a CSR-built copy of the
  * mask made on first need (one build on the mask's stream, with its
