@@ -723,10 +723,11 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                 if (!qend[s] && qm[s]) mbar_wait_bounded(bar(s, kQFull), (qm[s] - 1) & 1, kPpDrainCycles);
         }
     } else if (warp == 0) {
-        // ------------------------------------------------------------ K / V producer
+        // ------------------------------------------------------------ additive-term producer
         if (lane == 0) {
-            // per slot, load streams 1.. (K, V per tile; with additive terms
-            // their blocks per tile) each walk the slot's items from the ring:
+            // per slot, the additive terms' blocks per tile (only with additive
+            // terms; the stream index 3 of a per-slot set whose K and V streams
+            // are left to the MMA issuers) walk the slot's items from the ring:
             // item km, tile ku, loads issued
             int km[2][NSTREAM], ku[2][NSTREAM];
             uint32_t cnt[2][NSTREAM];
@@ -741,7 +742,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                 for (int k = 0; k < NSTREAM; ++k) {
                     km[s][k] = ku[s][k] = 0;
                     cnt[s][k] = 0;
-                    live[s][k] = k > 0;
+                    live[s][k] = k == 3;  // K and V are loaded by the slots' MMA issuers
                 }
             long long t_last = clock64();
             unsigned nap = 0;  // back-off when a pass finds nothing to load
@@ -871,7 +872,25 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                 mma_commit(bar(s, kSFree + h));
             };
             auto W = [&](int which, uint32_t phase) { return pp_wait(bar(s, which), phase & 1, abort_flag, P.wait_cycles); };
+            // K or V tile u of item ti into the slot's buffer (its previous
+            // contents already consumed)
+            auto load = [&](bool isK, const PpItem& ti, int tu) {
+                const uint32_t fb = bar(s, isK ? kKFull : kVFull);
+                const uint32_t dst = (isK ? sK0 : sV0) + s * C::TILE_BYTES;
+                mbar_expect_tx(fb, C::TILE_BYTES);
+                const int kt = pp_tile(P, sh, ti, tu) & 0x7fffffff;
+                const CUtensorMap* map = ti.perm ? (isK ? &tmKp : &tmVp) : (isK ? &tmK : &tmV);
+#pragma unroll
+                for (int c = 0; c < C::NCHUNK; ++c) {
+                    if (ti.perm)
+                        tma_load_5d(dst + c * C::CHUNK_BYTES, map, fb, c * C::CHUNK_ELEMS, ti.qb, kt * 128, ti.h, ti.b);
+                    else
+                        tma_load_4d(dst + c * C::CHUNK_BYTES, map, fb, c * C::CHUNK_ELEMS, kt * 128, ti.h, ti.b);
+                }
+            };
             uint32_t g = 0;        // tiles of this slot so far
+            uint32_t kc = 0, vc = 0;  // K and V tiles loaded so far (this thread issues them: it
+                                      // knows the moment its MMAs free a buffer)
             bool s_ready = false;  // both halves of the current item's first S are issued
             bool alive = true;
             for (uint32_t m = 0; alive; ++m) {
@@ -894,6 +913,17 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                 bi.perm = it.perm;
                 bi.chunk = it.chunk;
                 const bool zero_first = !(C::STAGE && P.mode == 1 && bsg::starts_from_perm(sh, bi));
+                // the first tile's K and V, unless loaded during the previous item
+                if (kc == g) {
+                    if (!(alive = g == 0 || W(kKEmpty, g - 1))) break;
+                    load(true, it, 0);
+                    ++kc;
+                }
+                if (vc == g) {
+                    if (!(alive = g == 0 || W(kVEmpty, g - 1))) break;
+                    load(false, it, 0);
+                    ++vc;
+                }
                 if (!s_ready) {
                     alive = W(kQFull, m) && W(kKFull, g) && (g == 0 || W(kSFree, g - 1));
                     if (!alive) break;
@@ -905,8 +935,33 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                 }
                 s_ready = false;
                 for (int u = 0; u < it.T; ++u, ++g) {
+                    // the next tile: this item's next one, or the next item's first
+                    // once it is taken
+                    PpItem tn;
+                    int un = 0;
+                    auto next_known = [&]() -> bool {
+                        if (u + 1 < it.T) {
+                            tn = it;
+                            un = u + 1;
+                            return true;
+                        }
+                        if (ring_n[s] <= (int)(m + 1)) return false;
+                        __threadfence_block();
+                        un = 0;
+                        return ring_get(P, entry(s, m + 1), tn);
+                    };
+                    // K of the next tile as soon as S of this one is complete
+                    if (kc == g + 1 && next_known()) {
+                        if (!(alive = W(kKEmpty, g))) break;
+                        load(true, tn, un);
+                        ++kc;
+                    }
                     if (!(alive = W(kPFull, g) && W(kVFull, g))) break;
                     issue_pv(0, u == 0 && zero_first);
+                    if (kc == g + 1 && mbar_test(bar(s, kKEmpty), g & 1) && next_known()) {
+                        load(true, tn, un);
+                        ++kc;
+                    }
                     // the next tile: this item's next one, or the next item's
                     // first when its Q and K are already in (else at its start)
                     bool nxt = false, nlast = false;
@@ -935,6 +990,18 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                     issue_pv(1, false);
                     mma_commit(bar(s, kVEmpty));
                     if (u + 1 == it.T) mma_commit(bar(s, kODone));
+                    // V of the next tile as soon as P_b V_b of this one is complete
+                    // (and K, if the next item was not taken earlier)
+                    if (vc == g + 1 && next_known()) {
+                        if (!(alive = W(kVEmpty, g))) break;
+                        load(false, tn, un);
+                        ++vc;
+                        if (kc == g + 1) {
+                            if (!(alive = W(kKEmpty, g))) break;
+                            load(true, tn, un);
+                            ++kc;
+                        }
+                    }
                     if (nxt) {
                         if (!a_done) {
                             if (!(alive = W(kKFull, g + 1))) break;
@@ -949,9 +1016,12 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                 }
             }
             if (!alive) *abort_flag = 1;
-            // every MMA this thread issued is complete before TMEM is released
+            // every MMA this thread issued is complete before TMEM is released,
+            // and no load it issued outlives the CTA
             mma_commit(bar(s, kDrainS));
             mbar_wait_bounded(bar(s, kDrainS), 0u, kPpDrainCycles);
+            if (kc) mbar_wait_bounded(bar(s, kKFull), (kc - 1) & 1, kPpDrainCycles);
+            if (vc) mbar_wait_bounded(bar(s, kVFull), (vc - 1) & 1, kPpDrainCycles);
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ softmax groups
