@@ -271,7 +271,10 @@ def committed_traffic(kernel: str, workload: str):
     for ln in open(path):
         if ":" in ln and ln.strip().startswith("- "):
             k, v = ln.strip()[2:].split(":", 1)
-            vals[k.strip()] = v.strip().strip("`")
+            v = v.strip()
+            if v.startswith("`"):  # `value` (note)
+                v = v[1:].split("`", 1)[0]
+            vals[k.strip()] = v
     if vals.get("source_sha256_16") != want:
         return None
     try:
