@@ -230,37 +230,6 @@ __device__ __forceinline__ int pp_tile(const PpParams& P, const bsg::Shape& sh, 
     return bsg::key_tile(sh, bi, u);
 }
 
-// tcgen05.mma (A in shared or in tensor memory) and tcgen05.commit for a loop
-// that the whole warp runs in convergence (its values warp-uniform): every
-// lane executes the call with the same operands and the lane elect.sync picks
-// issues. A sequence of MMAs goes out markedly faster this way than from one
-// lane alone (about 75 against 100 cycles apiece, measured on one B200).
-__device__ __forceinline__ void mma_bf16_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                                  uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
-}
-__device__ __forceinline__ void mma_bf16_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                                  uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
-}
-__device__ __forceinline__ void mma_commit_elect(uint32_t bar) {
-    asm volatile(
-        "{\n\t.reg .pred e;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
-        : "memory");
-}
-
 // Bounded wait that also gives up as soon as another thread of the CTA has.
 __device__ __forceinline__ bool pp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, long long limit) {
     if (mbar_try_wait(bar, parity)) return true;

@@ -802,10 +802,10 @@ __global__ void __launch_bounds__(kQuadThreads, EXTRA ? 3 : 4)
         for (int ks = 0; ks < D / 16; ++ks) {
             const uint64_t da = smem_desc(sQ + ks * 32, 16, C::SBO, C::LAYOUT);
             const uint64_t db = smem_desc(sK + ks * 32, 16, C::SBO, C::LAYOUT);
-            mma_bf16_ss(tS, da, db, idS, ks > 0 ? 1u : 0u);
+            mma_bf16_ss_elect(tS, da, db, idS, ks > 0 ? 1u : 0u);
         }
-        mma_commit(barS);
-        issued[2] += 1u;
+        mma_commit_elect(barS);
+        if ((tid & 31) == 0) issued[2] += 1u;
         return true;
     };
     auto issue_pv = [&](int s) -> bool {  // O (+)= P(s) V(s) once V(s) is loaded
@@ -817,14 +817,16 @@ __global__ void __launch_bounds__(kQuadThreads, EXTRA ? 3 : 4)
         for (int ks = 0; ks < 4; ++ks) {
             const uint64_t db =
                 smem_desc(sV + (uint32_t)(ks * 16 * C::ROW_BYTES), C::CHUNK_BYTES, C::SBO, C::LAYOUT);
-            mma_bf16_ts(tO, tP + (uint32_t)(ks * 8), db, idO, (s > 0 || ks > 0) ? 1u : 0u);
+            mma_bf16_ts_elect(tO, tP + (uint32_t)(ks * 8), db, idO, (s > 0 || ks > 0) ? 1u : 0u);
         }
-        mma_commit(barO);
-        issued[3] += 1u;
+        mma_commit_elect(barO);
+        if ((tid & 31) == 0) issued[3] += 1u;
         return true;
     };
 
-    if (tid == 0 && pers_wait(barQ, 0u, abort_flag)) issue_s(0);
+    // MMAs are issued by a whole warp (one elected lane): warp 0 here, later
+    // the warp whose arrival completes "P written"
+    if (warp == 0 && pers_wait(barQ, 0u, abort_flag)) issue_s(0);
     __syncwarp();
 
     const uint64_t c2 = pack2(P.qk_scale_log2, P.qk_scale_log2);
@@ -962,7 +964,8 @@ __global__ void __launch_bounds__(kQuadThreads, EXTRA ? 3 : 4)
         tmem_wait_st();
         if (EXTRA && s + 1 < NS)  // the next sub-tile: this tile's second half or the next tile's first
             fetch((((s & 1) ? info_next : info) & 0x7fffffff) * kTileN + 64 * ((s + 1) & 1));
-        if (arrive_last(pcnt, 4u * (uint32_t)(s + 1) - 1u) && !*abort_flag) {
+        const bool last = __shfl_sync(0xffffffffu, arrive_last(pcnt, 4u * (uint32_t)(s + 1) - 1u) ? 1 : 0, 0) != 0;
+        if (last && !*abort_flag) {
             // every row has written P(s) (and rescaled O): P V(s), then S(s+1) once
             // P V(s) has consumed P (S(s+1) overwrites it)
             if (issue_pv(s) && s + 1 < NS && pers_wait(barO, (uint32_t)(s & 1), abort_flag)) issue_s(s + 1);
