@@ -399,9 +399,9 @@ def kernel_name(wl, m_tiles):
         return f"k_fwd_short<{'bf16' if wl.dtype == workloads.BF16 else 'f32'},{wl.d}>"
     extra = wl.add_mask is not None or wl.bias is not None
     if wl.mask.kind in ("dense", "sliding", "varwin") and wl.d == 128 and not extra:
-        return f"k_fwd_pp<{wl.d},0>"
+        return f"k_fwd_pp<{wl.d},0,0>"
     if wl.mask.kind == "bsg" and not extra and wl.d in (64, 128):
-        return f"k_fwd_pp<{wl.d},0>"
+        return f"k_fwd_pp<{wl.d},0,1>"
     if wl.d <= 64:
         return f"k_fwd_tc_quad<{wl.d},{int(extra)}>"
     return f"k_fwd_tc<{wl.d}>"

@@ -552,7 +552,7 @@ __device__ __forceinline__ void pp_finish(const PpParams& P, const bsg::Shape& s
     if (row_ok && P.lse) P.lse[bh * P.n + i] = L > 0.f ? (M + lg2(L)) * kLn2 : -INFINITY;
 }
 
-template <int D, bool EXTRA>
+template <int D, bool EXTRA, bool CF>
 __global__ void __launch_bounds__(kPpThreads, 1)
     k_fwd_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQp,
@@ -560,6 +560,8 @@ __global__ void __launch_bounds__(kPpThreads, 1)
              const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
              const PpParams P) {
     using C = PpCfg<D, EXTRA>;
+    // CF: the build for closed-form masks (no additive terms there)
+    static_assert(!(CF && EXTRA), "closed-form masks carry no additive terms");
     constexpr int NSTREAM = EXTRA ? 4 : 3;  // producer streams: Q, K, V (, additive terms)
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -846,7 +848,14 @@ __global__ void __launch_bounds__(kPpThreads, 1)
         {
             const int s = warp - 2;
             const uint32_t tSm = tmem + (uint32_t)(s * 256), tOm = tSm + 128;
-            const uint32_t idS = idesc_bf16_f32(128, 64, false);
+            // Items of the closed form have one or two tiles (a few have 8):
+            // there S of a tile goes out as one N = 128 product after the
+            // previous tile's P V, which issues fewer MMAs and measured
+            // faster; the long items of interval masks gain more from S per
+            // half, the next tile's first half computed during the softmax of
+            // this tile's second
+            constexpr bool full_s = CF;
+            const uint32_t idS = idesc_bf16_f32(128, full_s ? 128 : 64, false);
             const uint32_t idO = idesc_bf16_f32(128, D, true);
             // shared-memory descriptors at the slot's Q and K buffers (K-major
             // operands) and V buffer (MN-major B); a k-step, a key half and a
@@ -855,7 +864,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             const uint64_t dQ = dQK0 + (uint64_t)((C::OFF_Q + s * C::TILE_BYTES) >> 4);
             const uint64_t dK = dQK0 + (uint64_t)((C::OFF_K + s * C::TILE_BYTES) >> 4);
             const uint64_t dV = smem_desc(sV0, C::CHUNK_BYTES, C::SBO, C::LAYOUT) + (uint64_t)((s * C::TILE_BYTES) >> 4);
-            auto issue_s = [&](int h) {  // S_h of the tile whose K is in
+            auto issue_s = [&](int h) {  // S_h of the tile whose K is in (full_s: both halves, h = 0)
                 tc_fence_after();
 #pragma unroll 1
                 for (int ks = 0; ks < D / 16; ++ks) {
@@ -865,6 +874,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                                       idS, ks > 0 ? 1u : 0u);
                 }
                 mma_commit_elect(bar(s, kSFull + h));
+                if (full_s) mma_commit_elect(bar(s, kSFullB));
             };
             auto issue_pv = [&](int h, bool zero) {  // O (+)= P_h V_h (zero: O = the product)
                 tc_fence_after();
@@ -932,11 +942,13 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                     ++vc;
                 }
                 if (!s_ready) {
-                    alive = W(kQFull, m) && W(kKFull, g) && (g == 0 || W(kSFree, g - 1));
+                    alive = W(kQFull, m) && W(kKFull, g) && (g == 0 || W(full_s ? kSFreeB : kSFree, g - 1));
                     if (!alive) break;
                     issue_s(0);
-                    if (!(alive = g == 0 || W(kSFreeB, g - 1))) break;
-                    issue_s(1);
+                    if (!full_s) {
+                        if (!(alive = g == 0 || W(kSFreeB, g - 1))) break;
+                        issue_s(1);
+                    }
                     mma_commit_elect(bar(s, kKEmpty));
                     if (it.T == 1) mma_commit_elect(bar(s, kQEmpty));
                 }
@@ -986,7 +998,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                     // S_a(g + 1) before P_b V_b(g) when its K is already in (the
                     // softmax group turns to it next), else after
                     bool a_done = false;
-                    if (nxt) {
+                    if (nxt && !full_s) {
                         if (!(alive = W(kSFree, g))) break;
                         if (mbar_test(bar(s, kKFull), (g + 1) & 1)) {
                             issue_s(0);
@@ -997,6 +1009,13 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                     issue_pv(1, false);
                     mma_commit_elect(bar(s, kVEmpty));
                     if (u + 1 == it.T) mma_commit_elect(bar(s, kODone));
+                    if (nxt && full_s) {  // S(g + 1) once P_b V_b(g) has consumed the P it overwrites
+                        if (!(alive = W(kKFull, g + 1) && W(kSFreeB, g))) break;
+                        issue_s(0);
+                        mma_commit_elect(bar(s, kKEmpty));
+                        if (nlast) mma_commit_elect(bar(s, kQEmpty));
+                        if (u + 1 == it.T) s_ready = true;
+                    }
                     // V of the next tile as soon as P_b V_b of this one is complete
                     // (and K, if the next item was not taken earlier)
                     if (vc == g + 1 && next_known()) {
@@ -1009,7 +1028,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                             ++kc;
                         }
                     }
-                    if (nxt) {
+                    if (nxt && !full_s) {
                         if (!a_done) {
                             if (!(alive = W(kKFull, g + 1))) break;
                             issue_s(0);
@@ -1435,14 +1454,14 @@ cudaError_t pp_map_addend(CUtensorMap* map, const AddendView& a, int B, int H, i
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int D, bool EXTRA>
+template <int D, bool EXTRA, bool CF>
 cudaError_t launch_pp_t(const TcOperand& q, const TcOperand& k, const TcOperand& v, const PpParams& p0,
                         const AddendView& mask, const AddendView& bias, int num_sms, cudaStream_t s) {
     using C = PpCfg<D, EXTRA>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, []() {
-        attr_err = cudaFuncSetAttribute((const void*)k_fwd_pp<D, EXTRA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err = cudaFuncSetAttribute((const void*)k_fwd_pp<D, EXTRA, CF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         C::SMEM_BYTES);
         // setmaxnreg.inc draws on the registers the CTA was launched with: the
         // split fits only when the launch holds at least 128 x 96 + 256 x 200
@@ -1450,7 +1469,7 @@ cudaError_t launch_pp_t(const TcOperand& q, const TcOperand& k, const TcOperand&
         // that never come), so refuse any build of the kernel launched with
         // fewer
         cudaFuncAttributes fa;
-        if (attr_err == cudaSuccess) attr_err = cudaFuncGetAttributes(&fa, (const void*)k_fwd_pp<D, EXTRA>);
+        if (attr_err == cudaSuccess) attr_err = cudaFuncGetAttributes(&fa, (const void*)k_fwd_pp<D, EXTRA, CF>);
         if (attr_err == cudaSuccess && fa.numRegs * kPpThreads < 128 * kPpRegsLow + 256 * kPpRegsHigh)
             attr_err = cudaErrorInvalidConfiguration;
     });
@@ -1483,8 +1502,8 @@ cudaError_t launch_pp_t(const TcOperand& q, const TcOperand& k, const TcOperand&
     }
     if (p.n_items <= 0) return cudaSuccess;
     const int64_t grid = p.n_items < num_sms ? p.n_items : num_sms;
-    k_fwd_pp<D, EXTRA><<<(unsigned)grid, kPpThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, mqp, mkp, mvp, ma0,
-                                                                                   ma1, p);
+    k_fwd_pp<D, EXTRA, CF><<<(unsigned)grid, kPpThreads, C::SMEM_BYTES, counted(s)>>>(mq, mk, mv, mqp, mkp, mvp,
+                                                                                       ma0, ma1, p);
     return cudaGetLastError();
 }
 
@@ -1494,12 +1513,17 @@ cudaError_t launch_fwd_pp(const TcOperand& q, const TcOperand& k, const TcOperan
                           const AddendView& mask, const AddendView& bias, int num_sms, cudaStream_t s) {
     const bool extra = mask.data || bias.data;
     if (extra && (p.mode != 0 || d > 64 || !pp_addend_ok(mask) || !pp_addend_ok(bias))) return cudaErrorInvalidValue;
+    // closed-form masks (mode 1) take the build whose S goes out per tile
+    const bool cf = p.mode == 1;
     switch (d) {
-    case 32: return extra ? launch_pp_t<32, true>(q, k, v, p, mask, bias, num_sms, s)
-                          : launch_pp_t<32, false>(q, k, v, p, mask, bias, num_sms, s);
-    case 64: return extra ? launch_pp_t<64, true>(q, k, v, p, mask, bias, num_sms, s)
-                          : launch_pp_t<64, false>(q, k, v, p, mask, bias, num_sms, s);
-    case 128: return launch_pp_t<128, false>(q, k, v, p, mask, bias, num_sms, s);
+    case 32: return extra ? launch_pp_t<32, true, false>(q, k, v, p, mask, bias, num_sms, s)
+                          : cf ? launch_pp_t<32, false, true>(q, k, v, p, mask, bias, num_sms, s)
+                               : launch_pp_t<32, false, false>(q, k, v, p, mask, bias, num_sms, s);
+    case 64: return extra ? launch_pp_t<64, true, false>(q, k, v, p, mask, bias, num_sms, s)
+                          : cf ? launch_pp_t<64, false, true>(q, k, v, p, mask, bias, num_sms, s)
+                               : launch_pp_t<64, false, false>(q, k, v, p, mask, bias, num_sms, s);
+    case 128: return cf ? launch_pp_t<128, false, true>(q, k, v, p, mask, bias, num_sms, s)
+                        : launch_pp_t<128, false, false>(q, k, v, p, mask, bias, num_sms, s);
     }
     return cudaErrorInvalidValue;
 }
