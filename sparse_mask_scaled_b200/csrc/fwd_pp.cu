@@ -262,8 +262,9 @@ __device__ __forceinline__ int ld_acquire_cta(volatile int* p) {
     return v;
 }
 
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+// Bring `bytes` (a multiple of 16, 16-byte aligned) starting at p into L2.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 // Release / acquire fence at GPU scope (ordering, not sequential consistency).
@@ -682,6 +683,15 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                         mbar_arrive(fb);  // the phase completes: the end is read
                     } else {
                         ring_put(e, it);
+                        if (C::STAGE && P.mode == 1 && sh.G > 0 && !it.perm && it.chunk == 0) {
+                            // a regular block that starts from its rows' published
+                            // states (written long before; they may have left L2):
+                            // bring the 128 rows' states, contiguous, into L2 now,
+                            // one item before they are read
+                            const int64_t row0 = (int64_t)it.bh * P.n + (int64_t)it.qb * 128;
+                            prefetch_l2_bulk(P.pacc + row0 * D, 128u * D * 4u);
+                            prefetch_l2_bulk(P.pml + row0 * 2, 128u * 8u);
+                        }
                         const uint32_t dst = sQ0 + s * C::TILE_BYTES;
                         mbar_expect_tx(fb, C::TILE_BYTES);
 #pragma unroll
@@ -1138,35 +1148,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             }
             const int klim = pp_key_limit(P, it.b);
             bool alive = true;
-            bool fetched = !C::STAGE || P.mode != 1 || sh.G == 0;  // the next item's published rows are on their way
             for (int u = 0; u < it.T && alive; ++u, ++g) {
-                if (!fetched && ring_n[s] > (int)(m + 1)) {
-                    // the slot's next item is taken: when it starts from published
-                    // states, bring this warp's rows of them into L2 (they were
-                    // written long before and may have left it)
-                    fetched = true;
-                    __threadfence_block();
-                    PpItem nx;
-                    if (ring_get(P, entry(s, m + 1), nx)) {
-                        bsg::Item nb;
-                        nb.bh = nx.bh;
-                        nb.perm = nx.perm;
-                        nb.qb = nx.qb;
-                        nb.pqb = nx.pqb;
-                        nb.chunk = nx.chunk;
-                        nb.u0 = nx.u0;
-                        nb.T = nx.T;
-                        if (bsg::starts_from_perm(sh, nb)) {
-                            const int ni = bsg::row_of(sh, nb, t);
-                            if (ni >= 0 && bsg::has_perm(sh, ni)) {
-                                const int64_t prow = (int64_t)nx.bh * P.n + ni;
-#pragma unroll
-                                for (int c = 0; c < D / 32; ++c) prefetch_l2(P.pacc + prow * D + 32 * c);
-                                if ((t & 15) == 0) prefetch_l2(P.pml + prow * 2);
-                            }
-                        }
-                    }
-                }
                 const int info = pp_tile(P, sh, it, u);
                 const int kt = info & 0x7fffffff;
                 bool dense = P.mode == 0 && info < 0;
