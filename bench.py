@@ -353,14 +353,15 @@ class GpuWorkload:
         self.out = torch.empty_like(self.q)
         self.lse = torch.empty(wl.B * wl.H * wl.n, dtype=torch.float32, device="cuda")
 
-    def create(self, hw=None, crp=None, ccols=None):
+    def create(self, hw=None, crp=None, ccols=None, tile_min_nnz=0):
         mp = self.wl.mask
         return self.sp.spattn_create_csr_mask(
             mp.kind, mp.n, mp.num_masks, window=mp.window, block=mp.block, stride=mp.stride,
             n_global=mp.n_global, add_diagonal=mp.add_diagonal,
             half_widths=self.hw if hw is None else hw,
             in_row_ptr=self.crp if crp is None else crp,
-            in_col_idx=self.ccols if ccols is None else ccols, asynchronous=True)
+            in_col_idx=self.ccols if ccols is None else ccols, tile_min_nnz=tile_min_nnz,
+            asynchronous=True)
 
     def fwd(self, m, q=None, k=None, v=None, out=None, lse=None):
         return self.sp.spattn_fwd_mask(self.q if q is None else q, self.k if k is None else k,
@@ -690,6 +691,23 @@ def fusion_ablation(args, torch, sp):
     return res
 
 
+def contiguous_runs(torch, sp):
+    """Contiguous column runs two ways, on the variable-window workload (every row
+    one run of up to 513 keys): gathered by the CUDA-core kernel (a mask built
+    with tile_min_nnz < 0: each lane group loads its nonzeros' K and V rows into
+    registers), and as the default 128 x 128 tiles whose K and V tiles TMA stages
+    in shared memory for the tensor cores. Forward only, L2 flushed."""
+    wl = workloads.make(1, seed=replica_seed(1, 0))
+    g = GpuWorkload(wl, torch, sp)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    res = {"workload": wl.name}
+    for name, tmn in (("gathered", -1), ("tma_staged_tiles", 0)):
+        with g.create(tile_min_nnz=tmn) as m:
+            res[name + "_ms"] = round(time_forward(g, m, torch, flush, reps=10)[0], 4)
+    res["tiles_speedup"] = round(res["gathered_ms"] / res["tma_staged_tiles_ms"], 2)
+    return res
+
+
 def other_workloads(torch, sp, skip, clk_mhz):
     """Forward-only timings of the other workloads and the extra dense d = 128
     case (device-resident inputs; L2 flushed, and warm), each with its roofline."""
@@ -812,6 +830,10 @@ def main():
                 result["fusion_ablation"] = fusion_ablation(args, torch, sp)
             except Exception as ex:
                 result["fusion_ablation"] = {"error": str(ex)[:200]}
+            try:
+                result["contiguous_runs"] = contiguous_runs(torch, sp)
+            except Exception as ex:
+                result["contiguous_runs"] = {"error": str(ex)[:200]}
         if not args.no_cpu_baseline and world == 1:
             threads = os.cpu_count() or 1
             rate, cnt, nz, t = cpu_oracle_rate(wl, args.cpu_seconds, threads)
