@@ -651,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr int kQuadThreads = 128;
 constexpr uint32_t kQuadCols = 128;
 
-template <int D>
+template <int D, bool EXTRA>
 struct QuadCfg {
     using C = TcCfg<D>;
     static constexpr int Q_BYTES = C::TILE_BYTES;       // 128 rows x d
@@ -659,10 +659,15 @@ struct QuadCfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = Q_BYTES;               // two buffers
     static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;  // two buffers
-    static constexpr int OFF_BAR = OFF_V + 2 * KV_BYTES;
-    // mbarriers Q_full, K_full[2], V_full[2], S_full, O_done; TMEM slot, abort
-    // flag, "P written" arrivals; issue counts (K, V loads, S, P V commits)
-    static constexpr int BAR_BYTES = 7 * 8 + 3 * 4 + 4 * 4;
+    // with additive terms: the staged term's block of the current sub-tile,
+    // 128 rows x 64 keys bf16 (128-byte rows, 128-byte swizzle)
+    static constexpr int OFF_A = OFF_V + 2 * KV_BYTES;
+    static constexpr int A_BYTES = EXTRA ? 128 * 128 : 0;
+    static constexpr int OFF_BAR = OFF_A + A_BYTES;
+    // mbarriers Q_full, K_full[2], V_full[2], S_full, O_done, A_full; TMEM slot,
+    // abort flag, "P written" arrivals; issue counts (K, V loads, S, P V
+    // commits, staged-term loads)
+    static constexpr int BAR_BYTES = 8 * 8 + 3 * 4 + 5 * 4;
     // at most four CTAs per SM (4 x 128 TMEM columns)
     static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES > 46 * 1024 ? OFF_BAR + BAR_BYTES : 46 * 1024;
 };
@@ -684,9 +689,10 @@ __device__ __forceinline__ bool pers_wait(uint32_t bar, uint32_t parity, volatil
 template <int D, bool EXTRA>
 __global__ void __launch_bounds__(kQuadThreads, EXTRA ? 3 : 4)
     k_fwd_tc_quad(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const TcParams P) {
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmA,
+                  const TcParams P) {
     using C = TcCfg<D>;
-    using L = QuadCfg<D>;
+    using L = QuadCfg<D, EXTRA>;
     static_assert(D == 32 || D == 64, "head dim");
     extern __shared__ __align__(1024) uint8_t smem[];
 
@@ -707,14 +713,14 @@ __global__ void __launch_bounds__(kQuadThreads, EXTRA ? 3 : 4)
     const int NS = 2 * T;  // 64-key sub-tiles
 
     const uint32_t sQ = smem_u32(smem + L::OFF_Q), sK0 = smem_u32(smem + L::OFF_K),
-                   sV0 = smem_u32(smem + L::OFF_V);
+                   sV0 = smem_u32(smem + L::OFF_V), sA = smem_u32(smem + L::OFF_A);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
     const uint32_t barQ = smem_u32(bars + 0), barK0 = smem_u32(bars + 1), barV0 = smem_u32(bars + 3),
-                   barS = smem_u32(bars + 5), barO = smem_u32(bars + 6);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7);
+                   barS = smem_u32(bars + 5), barO = smem_u32(bars + 6), barA = smem_u32(bars + 7);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     uint32_t* pcnt = tmem_slot + 2;    // "P written" arrivals
-    uint32_t* issued = tmem_slot + 3;  // [0] K, [1] V loads, [2] S, [3] P V commits
+    uint32_t* issued = tmem_slot + 3;  // [0] K, [1] V loads, [2] S, [3] P V commits, [4] staged-term loads
 
     // the row's state first: these loads run while the CTA sets up and the
     // first tiles arrive
@@ -730,11 +736,15 @@ __global__ void __launch_bounds__(kQuadThreads, EXTRA ? 3 : 4)
     int info = info_next;
 
     // Additive mask and bias (EXTRA). One term that varies by row (the bias,
-    // else the mask), when it is bf16 with unit column stride and 16-byte
-    // aligned rows, has the 64 values of the row's next sub-tile fetched as raw
-    // words one sub-tile ahead (after P is stored), so their latency overlaps
-    // P V and the next S. The other term -- typically a key-padding mask shared
-    // by every row, served from L1 -- and every other layout are loaded when used.
+    // else the mask) is staged: when TMA can fetch it (P.a_tma), its 128-row x
+    // 64-key block of each sub-tile comes into shared memory in one load, issued
+    // as soon as every warp has used the previous block (by the warp that
+    // completes "P written"), and each thread reads its row from there;
+    // otherwise, when it is bf16 with unit column stride and 16-byte aligned
+    // rows, the 64 values of the row's next sub-tile are fetched as raw words
+    // one sub-tile ahead (after P is stored), so their latency overlaps P V and
+    // the next S. The other term -- typically a key-padding mask shared by every
+    // row, served from L1 -- and every other layout are loaded when used.
     const int64_t mrb = EXTRA ? (int64_t)b * P.mask.s0 + (int64_t)h * P.mask.s1 + (int64_t)i * P.mask.s2 : 0;
     const int64_t brb = EXTRA ? (int64_t)b * P.bias.s0 + (int64_t)h * P.bias.s1 + (int64_t)i * P.bias.s2 : 0;
     // the prefetched term: 2 = bias, 1 = mask, 0 = none
@@ -743,9 +753,16 @@ __global__ void __launch_bounds__(kQuadThreads, EXTRA ? 3 : 4)
     const int64_t prb = pre == 2 ? brb : mrb;
     uint4 praw[EXTRA ? 8 : 1];
     bool raw = false;  // praw holds the prefetched term's values for the current sub-tile
+    const bool staged = EXTRA && P.a_tma && pre != 0;
+    // the staged term's block of sub-tile keys c0 .. c0 + 63 (one thread)
+    auto load_a = [&](int c0) {
+        mbar_expect_tx(barA, (uint32_t)L::A_BYTES);
+        tma_load_4d(sA, &tmA, barA, c0, qb * 128, pview.s1 ? h : 0, pview.s0 ? b : 0);
+        issued[4] += 1u;
+    };
     auto fetch = [&](int c0) {
         raw = false;
-        if (!EXTRA || pre == 0 || !row_ok || c0 + 64 > P.n || pview.dtype != 0 || pview.s3 != 1) return;
+        if (!EXTRA || staged || pre == 0 || !row_ok || c0 + 64 > P.n || pview.dtype != 0 || pview.s3 != 1) return;
         const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(pview.data) + prb + c0;
         if (reinterpret_cast<uintptr_t>(src) & 15u) return;
 #pragma unroll
@@ -770,13 +787,17 @@ __global__ void __launch_bounds__(kQuadThreads, EXTRA ? 3 : 4)
 
     if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kQuadCols);
     if (tid == 0) {
-        for (int x = 0; x < 7; ++x) mbar_init(smem_u32(bars + x), 1);
+        for (int x = 0; x < 8; ++x) mbar_init(smem_u32(bars + x), 1);
         *abort_flag = 0;
-        for (int x = 0; x < 5; ++x) pcnt[x] = 0u;  // and issued[]
+        for (int x = 0; x < 6; ++x) pcnt[x] = 0u;  // and issued[]
         fence_mbar_init();
         prefetch_tensormap(&tmQ);
         prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmV);
+        if (staged) {
+            prefetch_tensormap(&tmA);
+            load_a((info & 0x7fffffff) * kTileN);
+        }
         // Q and both halves of the first tile (every block has at least one)
         mbar_expect_tx(barQ, (uint32_t)L::Q_BYTES);
         tma_load_4d(sQ, &tmQ, barQ, 0, qb * 128, h, b);
@@ -869,6 +890,22 @@ __global__ void __launch_bounds__(kQuadThreads, EXTRA ? 3 : 4)
             if (s + 2 < NS) load_k(s + 2, (info_next & 0x7fffffff) * kTileN + 64 * (s & 1));
             if (s >= 1 && s + 1 < NS)
                 load_v(s + 1, (((s & 1) ? info_next : info) & 0x7fffffff) * kTileN + 64 * ((s + 1) & 1));
+        }
+        if (staged) {  // this sub-tile's block of the staged term, from shared memory
+            const bool oka = pers_wait(barA, (uint32_t)(s & 1), abort_flag);
+            if (!__all_sync(0xffffffffu, oka)) break;
+            // unit u of row r at r * 128 + (u ^ (r & 7)) * 16 (128-byte swizzle)
+            const uint32_t rowa = sA + (uint32_t)tid * 128u;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                uint4 v4;
+                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(v4.x), "=r"(v4.y), "=r"(v4.z), "=r"(v4.w)
+                             : "r"(rowa + (uint32_t)((u ^ (tid & 7)) << 4))
+                             : "memory");
+                praw[u] = v4;
+            }
+            raw = row_ok;
         }
         float x[64];
         {
@@ -966,6 +1003,13 @@ __global__ void __launch_bounds__(kQuadThreads, EXTRA ? 3 : 4)
             fetch((((s & 1) ? info_next : info) & 0x7fffffff) * kTileN + 64 * ((s + 1) & 1));
         const bool last = __shfl_sync(0xffffffffu, arrive_last(pcnt, 4u * (uint32_t)(s + 1) - 1u) ? 1 : 0, 0) != 0;
         if (last && !*abort_flag) {
+            // every warp has used the staged term's block of sub-tile s: bring
+            // in the next one
+            if (staged && s + 1 < NS) {
+                fence_proxy_async_smem();
+                if ((tid & 31) == 0) load_a((((s & 1) ? info_next : info) & 0x7fffffff) * kTileN + 64 * ((s + 1) & 1));
+                __syncwarp();
+            }
             // every row has written P(s) (and rescaled O): P V(s), then S(s+1) once
             // P V(s) has consumed P (S(s+1) overwrites it)
             if (issue_pv(s) && s + 1 < NS && pers_wait(barO, (uint32_t)(s & 1), abort_flag)) issue_s(s + 1);
@@ -1039,6 +1083,7 @@ __global__ void __launch_bounds__(kQuadThreads, EXTRA ? 3 : 4)
             }
         if (issued[2]) mbar_wait_bounded(barS, (issued[2] - 1u) & 1u, lim);
         if (issued[3]) mbar_wait_bounded(barO, (issued[3] - 1u) & 1u, lim);
+        if (issued[4]) mbar_wait_bounded(barA, (issued[4] - 1u) & 1u, lim);
         atomicOr(P.err, kErrTimeout);
     }
     __syncthreads();
@@ -1086,6 +1131,31 @@ cudaError_t make_map(CUtensorMap* map, const TcOperand& t, int B, int H, int n, 
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// Whether TMA can fetch an additive term: bf16 with unit key stride, the base
+// and every stride a multiple of 16 bytes.
+bool addend_tma_ok(const AddendView& a) {
+    const uintptr_t base = reinterpret_cast<uintptr_t>(a.data);
+    return a.dtype == 0 && a.s3 == 1 && (base & 15) == 0 && (a.s2 * 2) % 16 == 0 && (a.s1 * 2) % 16 == 0 &&
+           (a.s0 * 2) % 16 == 0;
+}
+
+// A per-row additive term [B or 1, H or 1, n, n] (bf16, keys contiguous) as
+// {keys, rows, heads, batch}, box {64, 128, 1, 1}, 128-byte swizzle; the
+// dimensions it broadcasts over have extent 1.
+cudaError_t make_addend_map(CUtensorMap* map, const AddendView& a, int B, int H, int n) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const uint64_t row_bytes = ((uint64_t)n * 2 + 15) & ~uint64_t(15);  // a valid stride for extent-1 dimensions
+    cuuint64_t dims[4] = {(cuuint64_t)n, (cuuint64_t)n, (cuuint64_t)(a.s1 ? H : 1), (cuuint64_t)(a.s0 ? B : 1)};
+    cuuint64_t strides[3] = {(uint64_t)a.s2 * 2, a.s1 ? (uint64_t)a.s1 * 2 : row_bytes, a.s0 ? (uint64_t)a.s0 * 2 : row_bytes};
+    cuuint32_t box[4] = {64, 128, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(a.data), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // 5-D map over a [B, H, n, d] bf16 tensor read in residue-permuted order:
 // dims {d, S, G, H, B} (row i = k S + r at (r, k)), box {chunk, 1, 128, 1, 1}:
 // one load brings rows r, r + S, ..., r + 127 S.
@@ -1118,11 +1188,11 @@ cudaError_t launch_tc_t(const TcOperand& q, const TcOperand& k, const TcOperand&
         constexpr int DP = D <= 64 ? D : 64;
         if (D <= 64) {
             attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_quad<DP, true>,
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize, QuadCfg<DP>::SMEM_BYTES);
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, QuadCfg<DP, true>::SMEM_BYTES);
             if (attr_err == cudaSuccess)
                 attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_quad<DP, false>,
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                QuadCfg<DP>::SMEM_BYTES);
+                                                QuadCfg<DP, false>::SMEM_BYTES);
         } else {
             attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc<D>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -1150,10 +1220,16 @@ cudaError_t launch_tc_t(const TcOperand& q, const TcOperand& k, const TcOperand&
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     constexpr int DP = D <= 64 ? D : 64;
     if (D <= 64 && p.has_extra) {
-        k_fwd_tc_quad<DP, true><<<(unsigned)grid, kQuadThreads, QuadCfg<DP>::SMEM_BYTES, counted(s)>>>(mq, mk, mv,
-                                                                                                     p);
+        // the term that varies by row (the bias, else the mask) goes through
+        // shared memory when TMA can fetch it
+        TcParams pe = p;
+        CUtensorMap ma = mq;
+        const AddendView& t = (p.bias.data && p.bias.s2 != 0) ? p.bias : p.mask;
+        pe.a_tma = t.data && t.s2 != 0 && addend_tma_ok(t) && make_addend_map(&ma, t, p.B, p.H, p.n) == cudaSuccess;
+        k_fwd_tc_quad<DP, true><<<(unsigned)grid, kQuadThreads, QuadCfg<DP, true>::SMEM_BYTES, counted(s)>>>(mq, mk, mv, ma,
+                                                                                                           pe);
     } else if (D <= 64) {
-        k_fwd_tc_quad<DP, false><<<(unsigned)grid, kQuadThreads, QuadCfg<DP>::SMEM_BYTES, counted(s)>>>(mq, mk, mv,
+        k_fwd_tc_quad<DP, false><<<(unsigned)grid, kQuadThreads, QuadCfg<DP, false>::SMEM_BYTES, counted(s)>>>(mq, mk, mv, mq,
                                                                                                       p);
     } else {
         // one thread block per query block, plus one per further chunk of split blocks

@@ -153,6 +153,9 @@ struct TcParams {
     float* lse;
     AddendView mask, bias;
     int has_extra;
+    // set by the launcher (d <= 64): the additive term that varies by row is
+    // staged into shared memory by TMA, one 128-row x 64-key block per sub-tile
+    int a_tma;
     float qk_scale_log2;
     unsigned* err;
 };
