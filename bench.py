@@ -404,7 +404,8 @@ def kernel_name(wl, m_tiles):
     if wl.mask.kind == "bsg" and not extra and wl.d in (64, 128):
         return f"k_fwd_pp<{wl.d},0,1>"
     if wl.d <= 64:
-        return f"k_fwd_tc_quad<{wl.d},{int(extra)}>"
+        # with additive terms the bench's (bf16, aligned) per-row term is staged by TMA
+        return f"k_fwd_tc_quad<{wl.d},{int(extra)},{int(extra)}>"
     return f"k_fwd_tc<{wl.d}>"
 
 

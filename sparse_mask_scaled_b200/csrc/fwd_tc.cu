@@ -686,8 +686,8 @@ __device__ __forceinline__ bool pers_wait(uint32_t bar, uint32_t parity, volatil
     }
 }
 
-template <int D, bool EXTRA>
-__global__ void __launch_bounds__(kQuadThreads, EXTRA ? 3 : 4)
+template <int D, bool EXTRA, bool STAGED>
+__global__ void __launch_bounds__(kQuadThreads, EXTRA && !STAGED ? 3 : 4)
     k_fwd_tc_quad(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmA,
                   const TcParams P) {
@@ -753,7 +753,8 @@ __global__ void __launch_bounds__(kQuadThreads, EXTRA ? 3 : 4)
     const int64_t prb = pre == 2 ? brb : mrb;
     uint4 praw[EXTRA ? 8 : 1];
     bool raw = false;  // praw holds the prefetched term's values for the current sub-tile
-    const bool staged = EXTRA && P.a_tma && pre != 0;
+    // STAGED: the build for a term TMA can fetch (the launcher's P.a_tma)
+    constexpr bool staged = EXTRA && STAGED;
     // the staged term's block of sub-tile keys c0 .. c0 + 63 (one thread)
     auto load_a = [&](int c0) {
         mbar_expect_tx(barA, (uint32_t)L::A_BYTES);
@@ -1187,10 +1188,14 @@ cudaError_t launch_tc_t(const TcOperand& q, const TcOperand& k, const TcOperand&
     std::call_once(once, []() {
         constexpr int DP = D <= 64 ? D : 64;
         if (D <= 64) {
-            attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_quad<DP, true>,
+            attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_quad<DP, true, true>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, QuadCfg<DP, true>::SMEM_BYTES);
             if (attr_err == cudaSuccess)
-                attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_quad<DP, false>,
+                attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_quad<DP, true, false>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                QuadCfg<DP, true>::SMEM_BYTES);
+            if (attr_err == cudaSuccess)
+                attr_err = cudaFuncSetAttribute((const void*)k_fwd_tc_quad<DP, false, false>,
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 QuadCfg<DP, false>::SMEM_BYTES);
         } else {
@@ -1226,10 +1231,14 @@ cudaError_t launch_tc_t(const TcOperand& q, const TcOperand& k, const TcOperand&
         CUtensorMap ma = mq;
         const AddendView& t = (p.bias.data && p.bias.s2 != 0) ? p.bias : p.mask;
         pe.a_tma = t.data && t.s2 != 0 && addend_tma_ok(t) && make_addend_map(&ma, t, p.B, p.H, p.n) == cudaSuccess;
-        k_fwd_tc_quad<DP, true><<<(unsigned)grid, kQuadThreads, QuadCfg<DP, true>::SMEM_BYTES, counted(s)>>>(mq, mk, mv, ma,
-                                                                                                           pe);
+        if (pe.a_tma)
+            k_fwd_tc_quad<DP, true, true><<<(unsigned)grid, kQuadThreads, QuadCfg<DP, true>::SMEM_BYTES, counted(s)>>>(
+                mq, mk, mv, ma, pe);
+        else
+            k_fwd_tc_quad<DP, true, false><<<(unsigned)grid, kQuadThreads, QuadCfg<DP, true>::SMEM_BYTES, counted(s)>>>(
+                mq, mk, mv, ma, pe);
     } else if (D <= 64) {
-        k_fwd_tc_quad<DP, false><<<(unsigned)grid, kQuadThreads, QuadCfg<DP, false>::SMEM_BYTES, counted(s)>>>(mq, mk, mv, mq,
+        k_fwd_tc_quad<DP, false, false><<<(unsigned)grid, kQuadThreads, QuadCfg<DP, false>::SMEM_BYTES, counted(s)>>>(mq, mk, mv, mq,
                                                                                                       p);
     } else {
         // one thread block per query block, plus one per further chunk of split blocks
