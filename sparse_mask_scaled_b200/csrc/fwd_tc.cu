@@ -17,8 +17,10 @@
 // the gather kernel's partial (m, l, acc) with the same rescaling rule.
 //
 // Two kernels: k_fwd_tc<d> (d = 128, one thread per row) and
-// k_fwd_tc_quad<d, EXTRA> (d <= 64: one thread per row, 64-key sub-tiles, P in
-// TMEM, four CTAs per SM, three with an additive mask or bias).
+// k_fwd_tc_quad<d, EXTRA, STAGED> (d <= 64: one thread per row, 64-key
+// sub-tiles, P in TMEM, four CTAs per SM; with an additive mask or bias the
+// term that varies by row is staged in shared memory by TMA (STAGED, four CTAs
+// per SM) or, for layouts TMA cannot fetch, prefetched into registers (three)).
 //
 // Every mbarrier wait is bounded: on expiry the CTA raises the device error
 // flag, drains what it issued (bounded again), frees its TMEM and returns.
