@@ -41,6 +41,27 @@ __device__ __forceinline__ uint4 ldg16(const void* p) {
     return __ldg(reinterpret_cast<const uint4*>(p));
 }
 
+// Two fp32 lanes per instruction (fma.rn.f32x2 / mul.rn.f32x2): each lane is
+// the plain fp32 operation, rounded to nearest even.
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void split2(uint64_t r, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 template <typename T>
 struct Elem;
 
@@ -205,10 +226,13 @@ __device__ __forceinline__ void row_steps(const FwdParams& P, const RowCtx<T, D>
         for (int u = 0; u < C::U; ++u) {
             float kf[C::VEC];
             Elem<T>::unpack(kr[u], kf);
-            float a = 0.f;
+            // even and odd elements in the two lanes of one packed FMA
+            uint64_t a2 = f2(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < C::VEC; ++e) a = fmaf(rc.qf[e], kf[e], a);
-            s[u] = a;
+            for (int e = 0; e < C::VEC / 2; ++e) a2 = ffma2(f2(rc.qf[2 * e], rc.qf[2 * e + 1]), f2(kf[2 * e], kf[2 * e + 1]), a2);
+            float ae, ao;
+            split2(a2, ae, ao);
+            s[u] = ae + ao;
         }
 #pragma unroll
         for (int off = 1; off < C::LPR; off <<= 1) {
@@ -224,17 +248,21 @@ __device__ __forceinline__ void row_steps(const FwdParams& P, const RowCtx<T, D>
         const float mu = (mx == -INFINITY) ? 0.f : mx;
         const float alpha = ex2(st.m - mu);
         st.l *= alpha;
+        uint64_t acc2[C::VEC / 2];
 #pragma unroll
-        for (int e = 0; e < C::VEC; ++e) st.acc[e] *= alpha;
+        for (int e = 0; e < C::VEC / 2; ++e) acc2[e] = fmul2(f2(st.acc[2 * e], st.acc[2 * e + 1]), f2(alpha, alpha));
 #pragma unroll
         for (int u = 0; u < C::U; ++u) {
             const float pw = ex2(s[u] - mu);
             st.l += pw;
             float vf[C::VEC];
             Elem<T>::unpack(vr[u], vf);
+            const uint64_t pw2 = f2(pw, pw);
 #pragma unroll
-            for (int e = 0; e < C::VEC; ++e) st.acc[e] = fmaf(pw, vf[e], st.acc[e]);
+            for (int e = 0; e < C::VEC / 2; ++e) acc2[e] = ffma2(pw2, f2(vf[2 * e], vf[2 * e + 1]), acc2[e]);
         }
+#pragma unroll
+        for (int e = 0; e < C::VEC / 2; ++e) split2(acc2[e], st.acc[2 * e], st.acc[2 * e + 1]);
         st.m = mx;
     }
 }
