@@ -25,7 +25,9 @@
 // cores compute the other half's S (and the other slot's work): the softmax
 // group waits for S only when the tensor cores or the loads fall behind.
 // After an item's last tile the issuer starts the next item's S at once when
-// its Q and K are in, else at that item's start. The producers poll with
+// its Q and K are in, else at that item's start. The build for closed-form
+// masks (CF), whose items have one or two tiles, computes S of a tile as one
+// N = 128 product once the previous tile's P_b V_b is complete instead. The producers poll with
 // non-blocking barrier tests and sleep briefly when nothing is free (they
 // share sub-partitions with softmax warps). Items come either from a counter
 // shared by all CTAs, taken in order as slots free up, or from a fixed share
