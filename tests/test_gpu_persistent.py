@@ -171,7 +171,9 @@ def test_dense_interval_mask_d128(n, B, H):
 @pytest.mark.parametrize("kind,n", [("dense", 256), ("sliding", 384), ("dense", 200)])
 def test_interval_mask_with_additive_terms(d, layout, kind, n, route, monkeypatch):
     """Additive mask and bias on interval masks at d <= 64: by default on the
-    four-CTAs-per-SM tile kernel; with SPATTN_DEBUG_PP_INTERVAL=1 on the
+    four-CTAs-per-SM tile kernel (its build that stages the row-varying term by
+    TMA for the bf16 layouts, the one that prefetches it into registers for the
+    fp32 bias); with SPATTN_DEBUG_PP_INTERVAL=1 on the
     persistent kernel, where bf16 terms with keys contiguous and 16-byte rows
     are staged through shared memory tile by tile (row-varying, shared by all
     rows, per head) and an fp32 term, or rows that are not 16-byte multiples
