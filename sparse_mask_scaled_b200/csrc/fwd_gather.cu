@@ -652,12 +652,24 @@ __device__ __forceinline__ void load_slice(const T* base, int c, float (&f)[Cfg<
 template <typename T, int D>
 __device__ __forceinline__ float group_dot(const float* a, const float* b) {
     using C = Cfg<T, D>;
-    float acc = 0.f;
+    // even and odd elements in the two lanes of one packed FMA
+    uint64_t a2 = f2(0.f, 0.f);
 #pragma unroll
-    for (int e = 0; e < C::VEC; ++e) acc = fmaf(a[e], b[e], acc);
+    for (int e = 0; e < C::VEC / 2; ++e) a2 = ffma2(f2(a[2 * e], a[2 * e + 1]), f2(b[2 * e], b[2 * e + 1]), a2);
+    float ae, ao;
+    split2(a2, ae, ao);
+    float acc = ae + ao;
 #pragma unroll
     for (int off = 1; off < C::LPR; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     return acc;
+}
+
+// y += a * x on N floats, two per packed FMA.
+template <int N>
+__device__ __forceinline__ void axpy2(float (&y)[N], float a, const float (&x)[N]) {
+    const uint64_t a2 = f2(a, a);
+#pragma unroll
+    for (int e = 0; e < N / 2; ++e) split2(ffma2(a2, f2(x[2 * e], x[2 * e + 1]), f2(y[2 * e], y[2 * e + 1])), y[2 * e], y[2 * e + 1]);
 }
 
 template <typename T, int D>
@@ -749,8 +761,7 @@ __device__ __forceinline__ void bwd_row(const BwdParams& P, int b, int h, int i,
                 const float dp = group_dot<T, D>(dof, vf);
                 const float pw = j >= 0 ? ex2(sc + ess[t] - lse2) : 0.f;
                 const float ds = pw * (dp - Di);
-#pragma unroll
-                for (int e = 0; e < C::VEC; ++e) dq[e] = fmaf(ds, kf[e], dq[e]);
+                axpy2(dq, ds, kf);
                 if (P.dbias && j >= 0 && c == 0 && ds != 0.f) {
                     if (db_row)
                         db_row[j] += ds;  // one row per warp, one lane per key
@@ -862,11 +873,8 @@ __global__ void __launch_bounds__(256, 3) k_bwd_cols(const BwdParams P) {
             const float dp = group_dot<T, D>(dof, vf);
             const float pw = (i >= 0 && ls != -INFINITY) ? ex2(sc + es - ls) : 0.f;
             const float ds = pw * (dp - di);
-#pragma unroll
-            for (int e = 0; e < C::VEC; ++e) {
-                dv[e] = fmaf(pw, dof[e], dv[e]);
-                dk[e] = fmaf(ds, qf[e], dk[e]);
-            }
+            axpy2(dv, pw, dof);
+            axpy2(dk, ds, qf);
         }
     }
     sum_groups<C::VEC, C::LPR>(dk);
