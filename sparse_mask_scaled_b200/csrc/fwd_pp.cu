@@ -645,7 +645,6 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             };
             int counted[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // per softmax warp: blocks counted in
             long long t_last = clock64();
-            unsigned nap = 0;
             while (true) {
                 bool any = false, progress = false;
                 // count in the permuted blocks the softmax warps published: one
@@ -722,10 +721,9 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                 }
                 if (progress) {
                     t_last = clock64();
-                    nap = 0;
                 } else {
-                    nap = nap ? (nap < 256 ? 2 * nap : 256) : 32;
-                    __nanosleep(nap);
+                    // no back-off: a slot's next item goes out the moment its Q
+                    // buffer frees (sleeping up to 256 ns here measured ~1 % slower)
                     if (*abort_flag) break;
                     if (clock64() - t_last > P.wait_cycles) {
                         *abort_flag = 1;
